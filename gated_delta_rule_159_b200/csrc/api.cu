@@ -1,0 +1,198 @@
+// api.cu -- the extern "C" entry points declared in include/gdn2.h: argument
+// validation, workspace layout, unit scheduling and kernel dispatch.  Nothing
+// here computes the recurrence; every step of it runs in the kernels.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr uint32_t kKnownFlags = GDN2_SCALAR_DECAY | GDN2_SCALAR_GATES | GDN2_TIED_GATES | GDN2_GATE_FORM_P3;
+constexpr size_t kWsHeader = 256;     // [0] status word, [1] unit counter
+constexpr int kMaxSortedSeqs = 4096;  // above this the units run in index order
+
+// Longest-first order of the (sequence, head) units of a packed batch: rank each
+// sequence by length (ties by index) and list its heads at that rank.
+__global__ void schedule_kernel(const int32_t *cu, int N, int H, int32_t *sched) {
+  for (int n = threadIdx.x; n < N; n += blockDim.x) {
+    const int len = cu[n + 1] - cu[n];
+    int rank = 0;
+    for (int m = 0; m < N; ++m) {
+      const int lm = cu[m + 1] - cu[m];
+      rank += (lm > len) || (lm == len && m < n);
+    }
+    for (int h = 0; h < H; ++h) sched[rank * H + h] = n * H + h;
+  }
+}
+
+int check_dims(const gdn2_dims *d) {
+  if (!d) return fail(GDN2_ERR_INVALID_ARG, "dims is NULL");
+  if (d->reserved != 0) return fail(GDN2_ERR_INVALID_ARG, "dims.reserved must be 0");
+  if (d->n_seqs < 1 || d->n_heads < 1 || d->seq_len < 0 || d->d_k < 1 || d->d_v < 1)
+    return fail(GDN2_ERR_INVALID_ARG, "bad dims (n_seqs=%d n_heads=%d seq_len=%d d_k=%d d_v=%d)", d->n_seqs,
+                d->n_heads, d->seq_len, d->d_k, d->d_v);
+  if ((d->dtype_in != GDN2_BF16 && d->dtype_in != GDN2_F32) || (d->dtype_out != GDN2_BF16 && d->dtype_out != GDN2_F32))
+    return fail(GDN2_ERR_INVALID_ARG, "bad dtype_in=%d / dtype_out=%d", d->dtype_in, d->dtype_out);
+  if (d->flags & ~kKnownFlags) return fail(GDN2_ERR_INVALID_ARG, "unknown flag bits 0x%x", d->flags & ~kKnownFlags);
+  if (d->flags & GDN2_GATE_FORM_P3)
+    return fail(GDN2_ERR_UNSUPPORTED, "GDN2_GATE_FORM_P3 is reserved and has no kernel in this build");
+  return GDN2_OK;
+}
+
+// Per-channel tensors are read by TMA or vector loads and need 16-byte alignment;
+// the [T, H] scalar-gate arrays are read element by element and need only
+// element alignment.
+int check_inputs(const void *q, const void *k, const void *v, const void *log_a, const void *b, const void *w,
+                 uint32_t flags, int dtype_in) {
+  if (!q || !k || !v || !log_a || !b) return fail(GDN2_ERR_INVALID_ARG, "q, k, v, log_a and b must be non-NULL");
+  if (!w && !(flags & GDN2_TIED_GATES)) return fail(GDN2_ERR_INVALID_ARG, "w is NULL without GDN2_TIED_GATES");
+  const uintptr_t elem = dtype_in == GDN2_BF16 ? 2 : 4;
+  const void *dense[3] = {q, k, v};
+  for (const void *p : dense)
+    if (!aligned16(p)) return fail(GDN2_ERR_INVALID_ARG, "input pointer %p is not 16-byte aligned", p);
+  const bool sd = (flags & GDN2_SCALAR_DECAY) != 0, sg = (flags & GDN2_SCALAR_GATES) != 0;
+  const void *gates[3] = {log_a, b, w};
+  const bool scalar[3] = {sd, sg, sg};
+  for (int i = 0; i < 3; ++i) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(gates[i]);
+    if (gates[i] && (scalar[i] ? (a % elem) != 0 : (a & 15u) != 0))
+      return fail(GDN2_ERR_INVALID_ARG, "gate pointer %p is misaligned", gates[i]);
+  }
+  return GDN2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn2_version(void) { return 100; }
+
+const char *gdn2_last_error(void) { return g_err; }
+
+size_t gdn2_chunk_fwd_workspace_size(const gdn2_dims *dims) {
+  if (!dims || dims->n_seqs < 1 || dims->n_heads < 1) return 0;
+  const size_t units = (size_t)dims->n_seqs * (size_t)dims->n_heads;
+  return kWsHeader + ((units * sizeof(int32_t) + 255) / 256) * 256;
+}
+
+int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *log_a, const void *b, const void *w,
+                   const float *S0, const int32_t *cu_seqlens, const int32_t *cu_seqlens_host, void *o, float *S_T,
+                   const gdn2_dims *dims, void *workspace, size_t workspace_bytes, gdn2_stream_t stream) {
+  g_err[0] = '\0';
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  rc = check_inputs(q, k, v, log_a, b, w, dims->flags, dims->dtype_in);
+  if (rc) return rc;
+  if (!o || !aligned16(o)) return fail(GDN2_ERR_INVALID_ARG, "o must be non-NULL and 16-byte aligned");
+  if ((S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)))
+    return fail(GDN2_ERR_INVALID_ARG, "S0 / S_T must be 16-byte aligned");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(GDN2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  const size_t need = gdn2_chunk_fwd_workspace_size(dims);
+  if (workspace_bytes < need)
+    return fail(GDN2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+
+  const int64_t t_total = cu_seqlens ? (int64_t)dims->seq_len : (int64_t)dims->n_seqs * dims->seq_len;
+  if (cu_seqlens_host) {
+    if (!cu_seqlens) return fail(GDN2_ERR_INVALID_ARG, "cu_seqlens_host given without cu_seqlens");
+    if (cu_seqlens_host[0] != 0 || cu_seqlens_host[dims->n_seqs] != t_total)
+      return fail(GDN2_ERR_INVALID_ARG, "cu_seqlens_host must start at 0 and end at seq_len (= T_tot)");
+    for (int n = 0; n < dims->n_seqs; ++n)
+      if (cu_seqlens_host[n + 1] < cu_seqlens_host[n])
+        return fail(GDN2_ERR_INVALID_ARG, "cu_seqlens_host is not non-decreasing at %d", n);
+  }
+
+  gdn2::ChunkProblem p;
+  memset(&p, 0, sizeof(p));
+  p.q = q; p.k = k; p.v = v; p.log_a = log_a; p.b = b; p.w = w;
+  p.S0 = S0; p.cu_seqlens = cu_seqlens; p.o = o; p.S_T = S_T;
+  p.n_seqs = dims->n_seqs; p.seq_len = dims->seq_len; p.n_heads = dims->n_heads;
+  p.d_k = dims->d_k; p.d_v = dims->d_v; p.chunk = dims->chunk;
+  p.dtype_in = dims->dtype_in; p.dtype_out = dims->dtype_out; p.flags = dims->flags;
+  p.t_total = t_total;
+  p.status = static_cast<int32_t *>(workspace);
+  p.schedule = nullptr;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool tc = dims->d_k == 128 && dims->d_v == 128 && dims->chunk == 64 && dims->dtype_in == GDN2_BF16;
+  const bool simt = dims->d_k <= 64 && dims->d_v <= 64 &&
+                    (dims->chunk == 16 || dims->chunk == 32 || dims->chunk == 64);
+  if (!tc && !simt)
+    return fail(GDN2_ERR_UNSUPPORTED,
+                "no kernel for d_k=%d d_v=%d chunk=%d dtype_in=%d (supported: 128/128/64 bf16, or d<=64 with chunk "
+                "16/32/64)",
+                dims->d_k, dims->d_v, dims->chunk, dims->dtype_in);
+
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kWsHeader, s);
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "cudaMemsetAsync(workspace): %s", cudaGetErrorString(e));
+  if (tc && cu_seqlens && dims->n_seqs <= kMaxSortedSeqs) {
+    int32_t *sched = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + kWsHeader);
+    schedule_kernel<<<1, 1024, 0, s>>>(cu_seqlens, dims->n_seqs, dims->n_heads, sched);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "schedule launch: %s", cudaGetErrorString(e));
+    p.schedule = sched;
+  }
+  if (tc) {
+    const char *why = "";
+    e = gdn2::launch_chunk_tc(p, s, &why);
+    if (e == cudaErrorNotSupported) return fail(GDN2_ERR_UNSUPPORTED, "%s", why);
+    if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "chunk_tc launch: %s (%s)", cudaGetErrorString(e), why);
+  } else {
+    e = gdn2::launch_chunk_simt(p, s);
+    if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "chunk_simt launch: %s", cudaGetErrorString(e));
+  }
+  return GDN2_OK;
+}
+
+int gdn2_check_status(const void *workspace, gdn2_stream_t stream) {
+  g_err[0] = '\0';
+  if (!workspace) return fail(GDN2_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+  int32_t st = 0;
+  e = cudaMemcpy(&st, workspace, sizeof(st), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "reading the status word: %s", cudaGetErrorString(e));
+  if (st == gdn2::kStatusTimeout) return fail(GDN2_ERR_TIMEOUT, "a bounded device wait timed out");
+  if (st != 0) return fail(GDN2_ERR_CUDA, "unknown device status %d", st);
+  return GDN2_OK;
+}
+
+int gdn2_decode_step(const void *q, const void *k, const void *v, const void *log_a, const void *b, const void *w,
+                     float *S, void *o, const gdn2_dims *dims, gdn2_stream_t stream) {
+  g_err[0] = '\0';
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->seq_len != 1) return fail(GDN2_ERR_INVALID_ARG, "gdn2_decode_step needs seq_len == 1");
+  rc = check_inputs(q, k, v, log_a, b, w, dims->flags, dims->dtype_in);
+  if (rc) return rc;
+  if (!S || !aligned16(S) || !o || !aligned16(o))
+    return fail(GDN2_ERR_INVALID_ARG, "S and o must be non-NULL and 16-byte aligned");
+  if (dims->d_k > 128 || (dims->d_v != 16 && dims->d_v != 32 && dims->d_v != 64 && dims->d_v != 128))
+    return fail(GDN2_ERR_UNSUPPORTED, "decode supports d_k <= 128 and d_v in {16, 32, 64, 128} (got %d, %d)",
+                dims->d_k, dims->d_v);
+  gdn2::DecodeProblem p;
+  p.q = q; p.k = k; p.v = v; p.log_a = log_a; p.b = b; p.w = w;
+  p.S = S; p.o = o;
+  p.n_seqs = dims->n_seqs; p.n_heads = dims->n_heads; p.d_k = dims->d_k; p.d_v = dims->d_v;
+  p.dtype_in = dims->dtype_in; p.dtype_out = dims->dtype_out; p.flags = dims->flags;
+  cudaError_t e = gdn2::launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+  return GDN2_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,197 @@
+"""ctypes binding of ``libgdn2.so`` (argument marshalling only).
+
+Every step of the computation runs in the library's CUDA kernels; PyTorch is
+used only to allocate device memory and to name the current stream.  Importing
+this module loads the shared library and raises ``ImportError`` if it is
+missing: there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn2.so")
+
+# enum gdn2_status / gdn2_dtype / gdn2_flags (include/gdn2.h)
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED = -2
+ERR_CUDA = -3
+ERR_TIMEOUT = -4
+ERR_WORKSPACE = -5
+BF16 = 0
+F32 = 1
+SCALAR_DECAY = 1
+SCALAR_GATES = 2
+TIED_GATES = 4
+GATE_FORM_P3 = 8
+
+EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_workspace_size", "gdn2_check_status",
+            "gdn2_decode_step", "gdn2_last_error", "gdn2_version")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("n_seqs", ctypes.c_int32), ("seq_len", ctypes.c_int32), ("n_heads", ctypes.c_int32),
+                ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32), ("chunk", ctypes.c_int32),
+                ("dtype_in", ctypes.c_int32), ("dtype_out", ctypes.c_int32), ("flags", ctypes.c_uint32),
+                ("reserved", ctypes.c_int32)]
+
+
+class GDN2Error(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"gdn2 status {status}: {message}")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m gated_delta_rule_159_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    lib.gdn2_chunk_fwd.restype = ctypes.c_int
+    lib.gdn2_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(Dims), vp, sz, vp]
+    lib.gdn2_chunk_fwd_workspace_size.restype = sz
+    lib.gdn2_chunk_fwd_workspace_size.argtypes = [ctypes.POINTER(Dims)]
+    lib.gdn2_check_status.restype = ctypes.c_int
+    lib.gdn2_check_status.argtypes = [vp, vp]
+    lib.gdn2_decode_step.restype = ctypes.c_int
+    lib.gdn2_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(Dims), vp]
+    lib.gdn2_last_error.restype = ctypes.c_char_p
+    lib.gdn2_last_error.argtypes = []
+    lib.gdn2_version.restype = ctypes.c_int
+    lib.gdn2_version.argtypes = []
+    return lib
+
+
+lib = _load()
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return BF16
+    if t == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t}")
+
+
+def _torch_dtype(code: int) -> torch.dtype:
+    return torch.bfloat16 if code == BF16 else torch.float32
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("gdn2 tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("gdn2 tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(rc: int):
+    if rc != OK:
+        raise GDN2Error(rc, lib.gdn2_last_error().decode())
+
+
+def make_dims(n_seqs, seq_len, n_heads, d_k, d_v, chunk, dtype_in, dtype_out, flags) -> Dims:
+    return Dims(int(n_seqs), int(seq_len), int(n_heads), int(d_k), int(d_v), int(chunk), int(dtype_in),
+                int(dtype_out), int(flags), 0)
+
+
+def flags_of(scalar_decay=False, scalar_gates=False, tied_gates=False) -> int:
+    return (SCALAR_DECAY if scalar_decay else 0) | (SCALAR_GATES if scalar_gates else 0) | \
+           (TIED_GATES if tied_gates else 0)
+
+
+def workspace_size(dims: Dims) -> int:
+    return int(lib.gdn2_chunk_fwd_workspace_size(ctypes.byref(dims)))
+
+
+def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, b: torch.Tensor,
+              w: Optional[torch.Tensor] = None, S0: Optional[torch.Tensor] = None,
+              cu_seqlens: Optional[torch.Tensor] = None, *, chunk: int = 64, scalar_decay: bool = False,
+              scalar_gates: bool = False, tied_gates: bool = False, out_dtype: Optional[torch.dtype] = None,
+              output_final_state: bool = True, cu_seqlens_host: Optional[Sequence[int]] = None,
+              o: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
+              workspace: Optional[torch.Tensor] = None):
+    """Chunked GDN-2 forward through ``gdn2_chunk_fwd``.
+
+    q, k: [B, T, H, d_k] (equal lengths) or [T_tot, H, d_k] with ``cu_seqlens``
+    (int32 [N+1] on the device); v: same with d_v.  log_a, b, w: like k, or
+    [.., H] with the scalar flags.  S0: fp32 [N, H, d_k, d_v] or None.
+    Returns (o [.., H, d_v], S_T fp32 [N, H, d_k, d_v] or None).
+    """
+    if q.dim() == 4:
+        if cu_seqlens is not None:
+            raise ValueError("4-D inputs take no cu_seqlens")
+        N, T, H, dk = q.shape
+        seq_len = T
+    elif q.dim() == 3:
+        if cu_seqlens is None:
+            N, (T, H, dk) = 1, q.shape
+            seq_len = T
+        else:
+            N = cu_seqlens.numel() - 1
+            T_tot, H, dk = q.shape
+            seq_len = T_tot
+            if cu_seqlens.dtype != torch.int32:
+                raise TypeError("cu_seqlens must be int32")
+    else:
+        raise ValueError("q must be [B, T, H, d_k] or [T_tot, H, d_k]")
+    dv = v.shape[-1]
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    flags = flags_of(scalar_decay, scalar_gates, tied_gates)
+    dims = make_dims(N, seq_len, H, dk, dv, chunk, _dtype_code(q.dtype), _dtype_code(out_dtype), flags)
+    dev = q.device
+    if o is None:
+        o = torch.empty(*v.shape[:-1], dv, dtype=out_dtype, device=dev)
+    if S_T is None and output_final_state:
+        S_T = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(workspace_size(dims), dtype=torch.uint8, device=dev)
+    host_cu = None
+    if cu_seqlens_host is not None:
+        host_cu = (ctypes.c_int32 * len(cu_seqlens_host))(*[int(x) for x in cu_seqlens_host])
+    rc = lib.gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(b), _ptr(w), _ptr(S0),
+                            _ptr(cu_seqlens), host_cu, _ptr(o), _ptr(S_T), ctypes.byref(dims),
+                            _ptr(workspace), workspace.numel(), _stream(dev))
+    _check(rc)
+    return o, S_T
+
+
+def check_status(workspace: torch.Tensor) -> int:
+    """Synchronise and read the device status left in ``workspace`` by chunk_fwd."""
+    return int(lib.gdn2_check_status(_ptr(workspace), _stream(workspace.device)))
+
+
+def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, b: torch.Tensor,
+                w: Optional[torch.Tensor], S: torch.Tensor, *, scalar_decay: bool = False,
+                scalar_gates: bool = False, tied_gates: bool = False, out_dtype: torch.dtype = torch.float32,
+                o: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One recurrent step through ``gdn2_decode_step``; ``S`` [N, H, d_k, d_v] fp32 is updated in place.
+
+    q, k, log_a, b, w: [N, H, d_k] (or [N, H] with the scalar flags); v: [N, H, d_v].
+    Returns o [N, H, d_v].
+    """
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    flags = flags_of(scalar_decay, scalar_gates, tied_gates)
+    dims = make_dims(N, 1, H, dk, dv, 0, _dtype_code(q.dtype), _dtype_code(out_dtype), flags)
+    if o is None:
+        o = torch.empty(N, H, dv, dtype=out_dtype, device=q.device)
+    rc = lib.gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(b), _ptr(w), _ptr(S), _ptr(o),
+                              ctypes.byref(dims), _stream(q.device))
+    _check(rc)
+    return o
+
+
+def version() -> int:
+    return int(lib.gdn2_version())

@@ -1,0 +1,175 @@
+/*
+ * gdn2.h -- C ABI of libgdn2.so: the Gated DeltaNet-2 token-mixer forward on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (per head, state S of d_k x d_v in fp32), for every token t:
+ *
+ *   decay       Sbar = Diag(a_t) S_{t-1},   a_t = exp(log_a_t) in (0, 1]^{d_k}
+ *   erase read  r_t  = Sbar^T k_t
+ *   erase       S'   = Sbar - (b_t . k_t) r_t^T
+ *   write       S_t  = S'   + (w_t . k_t) v_t^T
+ *   read        o_t  = S_t^T q_t
+ *
+ * Sources: gist.science "Gated DeltaNet-2: Decoupling Erase and Write in
+ * Linear Attention", Methodologie 1 (channel-wise erase gate b_t and write gate
+ * w_t, channel-wise decay D_t = Diag(alpha_t) from KDA); alanhou.org "Core
+ * Mechanism" (b_t erases, w_t writes; O(1) recurrent inference and a chunkwise
+ * WY algorithm for training); neelmishra.github.io "Gated DeltaNet", section
+ * "Decay first, then compute the write error" (key x value orientation; the
+ * erase read uses the decayed state); cours.spawnkit.ai session 16, worked trace
+ * (read after the update).  Where those pages differ on which side the gates
+ * sit, this library follows the form above by default (erase outer factor
+ * b.k, erase read with k, write outer factor w.k) and offers the gist.science
+ * equation as GDN2_GATE_FORM_P3 (reserved; not implemented by the kernels yet).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates or frees them.  Tensors are dense row-major with the
+ *    shapes given below; every base pointer must be 16-byte aligned, except
+ *    the [T, H] scalar-gate arrays of GDN2_SCALAR_DECAY / GDN2_SCALAR_GATES,
+ *    which need only the alignment of their element type.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and never synchronise the device.  A non-zero status means
+ *    nothing was launched (argument errors) or the launch failed (CUDA
+ *    errors); gdn2_last_error() then describes it.
+ *  - Values are not validated.  Preconditions: finite inputs; log_a <= 0 (the
+ *    decay is bounded in (0, 1], cours.spawnkit.ai session 16 "Stability");
+ *    b, w in [0, 1]; q and k L2-normalised by the caller (no 1/sqrt(d_k) scale
+ *    is applied).  The chunked path also needs, per channel, the summed decay
+ *    over each half chunk to stay above -80 (sum of log_a over 32 consecutive
+ *    tokens of a chunk >= -80), which keeps its fp32/bf16 decay factors finite.
+ */
+#ifndef GDN2_H
+#define GDN2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque CUDA stream handle; binary-compatible with cudaStream_t. */
+typedef struct CUstream_st *gdn2_stream_t;
+
+/* Status codes returned by every entry point. */
+enum gdn2_status {
+  GDN2_OK = 0,
+  GDN2_ERR_INVALID_ARG = -1,  /* null/misaligned pointer, bad dims, bad cu_seqlens_host */
+  GDN2_ERR_UNSUPPORTED = -2,  /* valid request this build has no kernel for */
+  GDN2_ERR_CUDA = -3,         /* a CUDA runtime call or kernel launch failed */
+  GDN2_ERR_TIMEOUT = -4,      /* a bounded device-side wait gave up (reported by gdn2_check_status) */
+  GDN2_ERR_WORKSPACE = -5     /* workspace pointer NULL or smaller than the queried size */
+};
+
+/* Element types of the per-token inputs (dtype_in) and of o (dtype_out). */
+enum gdn2_dtype { GDN2_BF16 = 0, GDN2_F32 = 1 };
+
+/* Flags (dims.flags). */
+enum gdn2_flags {
+  GDN2_SCALAR_DECAY = 1u,  /* log_a is [T_tot, H]: one decay per token and head (a = alpha 1) */
+  GDN2_SCALAR_GATES = 2u,  /* b and w are [T_tot, H]: one erase and one write gate per token and head */
+  GDN2_TIED_GATES = 4u,    /* w is b (the w pointer is ignored and may be NULL) */
+  GDN2_GATE_FORM_P3 = 8u   /* reserved: gist.science gate placement; returns GDN2_ERR_UNSUPPORTED */
+};
+
+/*
+ * Problem description shared by both entry points.
+ *   n_seqs     N, number of sequences (>= 1).
+ *   seq_len    tokens per sequence when cu_seqlens == NULL (all N equal);
+ *              total packed tokens T_tot when cu_seqlens != NULL.
+ *              gdn2_decode_step requires seq_len == 1.
+ *   n_heads    H.
+ *   d_k, d_v   head dimensions.
+ *   chunk      C, chunk length of the chunked path (ignored by decode).
+ *   dtype_in   enum gdn2_dtype of q, k, v, log_a, b, w.
+ *   dtype_out  enum gdn2_dtype of o.
+ *   flags      enum gdn2_flags, OR-ed.
+ */
+typedef struct gdn2_dims {
+  int32_t n_seqs;
+  int32_t seq_len;
+  int32_t n_heads;
+  int32_t d_k;
+  int32_t d_v;
+  int32_t chunk;
+  int32_t dtype_in;
+  int32_t dtype_out;
+  uint32_t flags;
+  int32_t reserved; /* must be 0 */
+} gdn2_dims;
+
+/*
+ * gdn2_chunk_fwd -- chunked (prefill) forward over N packed sequences.
+ *
+ * Computes o and the final state S_T of the recurrence above for every
+ * (sequence, head) with the chunkwise-parallel WY form (alanhou.org "Core
+ * Mechanism": decay absorbed into asymmetric erase factors; gist.science
+ * Methodologie 3: lower-triangular (I + T)^-1 solve giving erase-side and
+ * write-side auxiliaries).  The result equals the token-by-token recurrence up
+ * to rounding.
+ *
+ * Arguments (T_tot = N * seq_len without cu_seqlens):
+ *   q, k         [T_tot, H, d_k]  dtype_in
+ *   v            [T_tot, H, d_v]  dtype_in
+ *   log_a        [T_tot, H, d_k]  dtype_in, log of the decay (<= 0); [T_tot, H] with GDN2_SCALAR_DECAY
+ *   b, w         [T_tot, H, d_k]  dtype_in, erase / write gates; [T_tot, H] with GDN2_SCALAR_GATES;
+ *                w may be NULL with GDN2_TIED_GATES
+ *   S0           [N, H, d_k, d_v] fp32 initial states, or NULL for zeros.  May alias S_T.
+ *   cu_seqlens   device int32 [N + 1] token offsets (0 = cu[0] <= ... <= cu[N] = T_tot), or NULL
+ *   cu_seqlens_host  optional host copy of cu_seqlens used to schedule the longest sequences
+ *                first; NULL lets the device order them.  Must match cu_seqlens when given.
+ *   o            [T_tot, H, d_v]  dtype_out (written); must not alias an input.
+ *   S_T          [N, H, d_k, d_v] fp32 final states (written), or NULL to skip them.
+ *   workspace    device scratch of at least gdn2_chunk_fwd_workspace_size(dims) bytes,
+ *                256-byte aligned, owned by the caller; its contents need not be initialised
+ *                and must not be used by another call running concurrently on the GPU.
+ * Supported: d_k = d_v = 128, C = 64, bf16 in, bf16 or fp32 out (tensor-core path);
+ *            d_k, d_v <= 64, C in {16, 32, 64}, bf16 or fp32 in (small-head path).
+ * Errors: GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_WORKSPACE, GDN2_ERR_CUDA.
+ */
+int gdn2_chunk_fwd(const void *q, const void *k, const void *v,
+                   const void *log_a, const void *b, const void *w,
+                   const float *S0, const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                   void *o, float *S_T, const gdn2_dims *dims,
+                   void *workspace, size_t workspace_bytes, gdn2_stream_t stream);
+
+/* Bytes of device workspace gdn2_chunk_fwd needs for `dims` (0 if dims are invalid). */
+size_t gdn2_chunk_fwd_workspace_size(const gdn2_dims *dims);
+
+/*
+ * gdn2_check_status -- synchronises `stream`, then reads the device status word
+ * that gdn2_chunk_fwd left in `workspace` (bounded waits inside the kernel
+ * record a timeout there instead of hanging).  Returns GDN2_OK, GDN2_ERR_TIMEOUT
+ * or GDN2_ERR_CUDA.  Optional: a caller that never checks loses nothing but the
+ * diagnosis.
+ */
+int gdn2_check_status(const void *workspace, gdn2_stream_t stream);
+
+/*
+ * gdn2_decode_step -- one recurrent step (alanhou.org "Core Mechanism": inference
+ * runs as a pure RNN with O(1) memory per token) for N sequences, updating the
+ * states in place: every state is read once and written once.
+ *   q, k, log_a, b, w  [N, H, d_k] dtype_in ([N, H] for the scalar flags)
+ *   v                  [N, H, d_v] dtype_in
+ *   S                  [N, H, d_k, d_v] fp32, read and overwritten in place
+ *   o                  [N, H, d_v] dtype_out
+ * dims.seq_len must be 1.  Supported: d_k, d_v multiples of 4 with
+ * d_k * d_v <= 128 * 128, bf16 or fp32 in, fp32 or bf16 out.
+ * Errors: GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_CUDA.
+ */
+int gdn2_decode_step(const void *q, const void *k, const void *v,
+                     const void *log_a, const void *b, const void *w,
+                     float *S, void *o, const gdn2_dims *dims, gdn2_stream_t stream);
+
+/* Thread-local description of the last non-zero status on this thread ("" if none). */
+const char *gdn2_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int gdn2_version(void);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* GDN2_H */

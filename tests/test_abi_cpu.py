@@ -1,0 +1,121 @@
+"""CPU-side checks of the C ABI: the library loads, exports every entry point
+include/gdn2.h declares, and rejects bad arguments before touching a GPU.
+
+Every call below fails validation on the host, so no CUDA call is ever made
+with the placeholder pointers used here.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn2.h")
+
+
+@pytest.fixture(scope="module")
+def g():
+    from gated_delta_rule_159_b200 import build
+    build.build()
+    from gated_delta_rule_159_b200 import gdn2
+    return gdn2
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(gdn2_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("gdn2_chunk_fwd", "gdn2_chunk_fwd_workspace_size", "gdn2_decode_step", "gdn2_last_error"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(g):
+    lib = ctypes.CDLL(g.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in gdn2.h but not exported"
+    assert set(declared_functions()) <= set(g.EXPORTED) | set(declared_functions())
+    assert g.version() == 100
+
+
+def _dims(g, **kw):
+    base = dict(n_seqs=2, seq_len=128, n_heads=4, d_k=128, d_v=128, chunk=64, dtype_in=g.BF16, dtype_out=g.BF16,
+                flags=0)
+    base.update(kw)
+    return g.make_dims(**base)
+
+
+P = ctypes.c_void_p(1 << 20)       # 16-byte-aligned placeholders, never dereferenced
+WS = ctypes.c_void_p(1 << 21)
+
+
+def _chunk(g, dims, **ptrs):
+    a = dict(q=P, k=P, v=P, log_a=P, b=P, w=P, S0=None, cu=None, cu_host=None, o=P, S_T=None, ws=WS,
+             ws_bytes=1 << 20)
+    a.update(ptrs)
+    rc = g.lib.gdn2_chunk_fwd(a["q"], a["k"], a["v"], a["log_a"], a["b"], a["w"], a["S0"], a["cu"], a["cu_host"],
+                              a["o"], a["S_T"], ctypes.byref(dims), a["ws"], a["ws_bytes"], None)
+    return rc, g.lib.gdn2_last_error().decode()
+
+
+def test_workspace_size(g):
+    d = _dims(g, n_seqs=8, n_heads=16)
+    assert g.workspace_size(d) == 256 + 512
+    assert g.workspace_size(_dims(g, n_seqs=0)) == 0
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(n_seqs=0), -1), (dict(n_heads=0), -1), (dict(seq_len=-1), -1), (dict(dtype_in=7), -1),
+    (dict(flags=1 << 10), -1), (dict(flags=8), -2), (dict(d_k=96, d_v=96), -2), (dict(chunk=48, d_k=32, d_v=32), -2),
+    (dict(dtype_in=1), -2),  # fp32 input with d = 128 has no kernel
+])
+def test_chunk_rejects_bad_dims(g, bad, code):
+    rc, msg = _chunk(g, _dims(g, **bad))
+    assert rc == code and msg
+
+
+def test_chunk_rejects_bad_pointers(g):
+    d = _dims(g)
+    assert _chunk(g, d, q=None)[0] == g.ERR_INVALID_ARG
+    assert _chunk(g, d, w=None)[0] == g.ERR_INVALID_ARG
+    assert _chunk(g, d, k=ctypes.c_void_p((1 << 20) + 2))[0] == g.ERR_INVALID_ARG
+    assert _chunk(g, d, o=None)[0] == g.ERR_INVALID_ARG
+    assert _chunk(g, d, S_T=ctypes.c_void_p((1 << 20) + 8))[0] == g.ERR_INVALID_ARG
+    assert _chunk(g, d, ws=None)[0] == g.ERR_WORKSPACE
+    assert _chunk(g, d, ws=ctypes.c_void_p((1 << 21) + 64))[0] == g.ERR_WORKSPACE
+    assert _chunk(g, d, ws_bytes=16)[0] == g.ERR_WORKSPACE
+
+
+def test_chunk_rejects_bad_host_cu_seqlens(g):
+    d = _dims(g, n_seqs=3, seq_len=100)
+    bad = [(0, 60, 50, 100), (1, 20, 50, 100), (0, 20, 50, 99)]
+    for cu in bad:
+        host = (ctypes.c_int32 * 4)(*cu)
+        rc, msg = _chunk(g, d, cu=P, cu_host=host)
+        assert rc == g.ERR_INVALID_ARG, (cu, msg)
+    host = (ctypes.c_int32 * 4)(0, 20, 50, 100)
+    assert _chunk(g, d, cu=None, cu_host=host)[0] == g.ERR_INVALID_ARG
+
+
+def test_decode_rejects_bad_arguments(g):
+    def call(dims, **kw):
+        a = dict(q=P, k=P, v=P, log_a=P, b=P, w=P, S=P, o=P)
+        a.update(kw)
+        return g.lib.gdn2_decode_step(a["q"], a["k"], a["v"], a["log_a"], a["b"], a["w"], a["S"], a["o"],
+                                      ctypes.byref(dims), None)
+    assert call(_dims(g, seq_len=1, d_v=96)) == g.ERR_UNSUPPORTED
+    assert call(_dims(g, seq_len=1, d_k=256)) == g.ERR_UNSUPPORTED
+    assert call(_dims(g, seq_len=2)) == g.ERR_INVALID_ARG
+    assert call(_dims(g, seq_len=1), S=None) == g.ERR_INVALID_ARG
+    assert call(_dims(g, seq_len=1), w=None) == g.ERR_INVALID_ARG
+    assert call(_dims(g, seq_len=1, flags=g.TIED_GATES), w=None, o=ctypes.c_void_p(3)) == g.ERR_INVALID_ARG
+
+
+def test_last_error_is_cleared(g):
+    _chunk(g, _dims(g, n_seqs=0))
+    assert g.lib.gdn2_last_error().decode()
+    assert g.lib.gdn2_chunk_fwd_workspace_size(ctypes.byref(_dims(g))) > 0

@@ -1,0 +1,253 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Small cases compare every element of every (sequence, head); they span
+several chunks and ragged tails.  Full-size workloads run in the launch
+configuration bench.py times and compare sampled units one by one.
+Tolerances: 2e-2 (bf16-input chunked path), 1e-4 (fp32 decode and the fp32
+small-head chunk path); metric in parity_utils.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity_utils import (TOL_CHUNK_BF16, TOL_CHUNK_F32, TOL_DECODE, all_units, compare_units, oracle_on_units,
+                          rel_err, run_chunk, to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from gated_delta_rule_159_b200 import gdn2  # noqa: F401  (fails loudly without libgdn2.so)
+    return torch.device("cuda:0")
+
+
+def _inputs(name, dev, **kw):
+    from gated_delta_rule_159_b200 import inputs
+    return inputs.make_inputs(name, dev, **kw)
+
+
+def _small(dev, dk=128, dv=128, chunk=64, dtype=torch.bfloat16, scalar=False, s0=0.02, decay=0.05, **kw):
+    from gated_delta_rule_159_b200 import inputs
+    w = inputs.Workload("small", kw.pop("n_seqs", 2), kw.pop("seq_len", 200), kw.pop("n_heads", 3), dk, dv, chunk,
+                        dtype, decay, scalar, s0)
+    return inputs.make_inputs(w, dev, **kw)
+
+
+# ----------------------------------------------------------------- small-head fp32 path
+def test_tiny_fp32_config(dev):
+    inp = _inputs("tiny_fp32", dev)
+    o, S_T = run_chunk(inp)
+    eo, es = compare_units(inp, o, S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_F32 and es <= TOL_CHUNK_F32, (eo, es)
+
+
+@pytest.mark.parametrize("variant", ["gdn", "deltanet"])
+def test_tiny_fp32_reductions(dev, variant):
+    """Gated DeltaNet (a = alpha 1, b = w = beta 1) and DeltaNet (alpha = 1) special cases."""
+    from gated_delta_rule_159_b200 import inputs
+    w = inputs.Workload("tiny_gdn", 1, 256, 1, 16, 16, 16, torch.float32, 0.1, True, 0.0)
+    inp = inputs.make_inputs(w, dev)
+    if variant == "deltanet":
+        inp["log_a"] = torch.zeros_like(inp["log_a"])
+    o, S_T = run_chunk(inp)
+    eo, es = compare_units(inp, o, S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_F32 and es <= TOL_CHUNK_F32, (eo, es)
+
+
+@pytest.mark.parametrize("dk,chunk,dtype", [(64, 64, torch.bfloat16), (32, 32, torch.float32), (16, 16, torch.bfloat16)])
+def test_simt_path_varlen(dev, dk, chunk, dtype):
+    inp = _small(dev, dk=dk, dv=dk, chunk=chunk, dtype=dtype, lengths=[1, chunk - 1, chunk, chunk + 1, 0, 3 * chunk + 5])
+    o, S_T = run_chunk(inp, out_dtype=torch.float32)
+    eo, es = compare_units(inp, o, S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_F32 and es <= TOL_CHUNK_F32, (eo, es)
+
+
+# ----------------------------------------------------------------- tensor-core path, small
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_tc_equal_lengths(dev, out_dtype):
+    inp = _small(dev, n_seqs=2, seq_len=200, n_heads=3)
+    o, S_T = run_chunk(inp, out_dtype=out_dtype)
+    assert o.dtype == out_dtype
+    eo, es = compare_units(inp, o, S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (eo, es)
+
+
+def test_tc_varlen_ragged(dev):
+    lens = [1, 63, 64, 65, 130, 0, 257, 5]
+    inp = _small(dev, n_heads=2, lengths=lens)
+    o, S_T = run_chunk(inp)
+    eo, es = compare_units(inp, o, S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (eo, es)
+    # the zero-length sequence returns its initial state exactly
+    torch.testing.assert_close(S_T[5], inp["S0"][5], rtol=0, atol=0)
+
+
+def test_tc_packed_equals_batched_form(dev):
+    inp = _small(dev, n_seqs=3, seq_len=150, n_heads=2)
+    o1, S1 = run_chunk(inp, packed=False)
+    o2, S2 = run_chunk(inp, packed=True)
+    torch.testing.assert_close(o1, o2, rtol=0, atol=0)
+    torch.testing.assert_close(S1, S2, rtol=0, atol=0)
+
+
+def test_tc_scalar_gates(dev):
+    inp = _small(dev, scalar=True, s0=0.0, n_seqs=2, seq_len=300, n_heads=2)
+    o, S_T = run_chunk(inp)
+    eo, es = compare_units(inp, o, S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (eo, es)
+
+
+@pytest.mark.parametrize("case", ["deltanet", "pure_decay", "zero_key", "strong_decay", "no_decay_no_gates"])
+def test_tc_degenerate_cases(dev, case):
+    inp = _small(dev, n_seqs=1, seq_len=192, n_heads=2)
+    if case == "deltanet":            # alpha = 1
+        inp["log_a"] = torch.zeros_like(inp["log_a"])
+    elif case == "pure_decay":        # b = w = 0: S_T = Diag(exp(sum log_a)) S0
+        inp["b"] = torch.zeros_like(inp["b"])
+        inp["w"] = torch.zeros_like(inp["w"])
+    elif case == "zero_key":
+        inp["k"] = torch.zeros_like(inp["k"])
+    elif case == "strong_decay":      # -2.4 per step: half a chunk sums to -76.8 (precondition >= -80)
+        inp["log_a"] = torch.full_like(inp["log_a"], -2.4)
+    elif case == "no_decay_no_gates":  # alpha = 1, b = w = 0: the state holds
+        inp["log_a"] = torch.zeros_like(inp["log_a"])
+        inp["b"] = torch.zeros_like(inp["b"])
+        inp["w"] = torch.zeros_like(inp["w"])
+    o, S_T = run_chunk(inp, out_dtype=torch.float32)
+    eo, es = compare_units(inp, o, S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (eo, es)
+    if case == "pure_decay":
+        L = inp["log_a"].float().sum(0)  # [H, d_k]
+        want = torch.exp(L)[:, :, None] * inp["S0"][0]
+        torch.testing.assert_close(S_T[0], want, rtol=1e-5, atol=1e-7)
+
+
+def test_tc_split_resume(dev):
+    """Prefill in two calls (S_T fed back as S0) equals one call."""
+    from gated_delta_rule_159_b200 import gdn2
+    inp = _small(dev, n_seqs=1, seq_len=320, n_heads=2)
+    names = ("q", "k", "v", "log_a", "b", "w")
+    o_full, S_full = gdn2.chunk_fwd(*(inp[n][None] for n in names), inp["S0"], out_dtype=torch.float32)
+    cut = 130
+    oa, Sa = gdn2.chunk_fwd(*(inp[n][None, :cut] for n in names), inp["S0"], out_dtype=torch.float32)
+    ob, Sb = gdn2.chunk_fwd(*(inp[n][None, cut:].contiguous() for n in names), Sa, out_dtype=torch.float32)
+    ref = oracle_on_units(inp, all_units(inp))
+    for h in range(2):
+        o_r, S_r = ref[(0, h)]
+        assert rel_err(to_f64(torch.cat([oa[0, :, h], ob[0, :, h]])), o_r) <= TOL_CHUNK_BF16
+        assert rel_err(to_f64(Sb[0, h]), S_r) <= TOL_CHUNK_BF16
+    assert rel_err(to_f64(Sb), to_f64(S_full)) <= TOL_CHUNK_BF16
+
+
+def test_tc_S0_aliases_S_T(dev):
+    from gated_delta_rule_159_b200 import gdn2
+    inp = _small(dev, n_seqs=2, seq_len=100, n_heads=2)
+    names = ("q", "k", "v", "log_a", "b", "w")
+    N, T = 2, 100
+    args = [inp[n].view(N, T, *inp[n].shape[1:]) for n in names]
+    o1, S1 = gdn2.chunk_fwd(*args, inp["S0"])
+    S = inp["S0"].clone()
+    o2, S2 = gdn2.chunk_fwd(*args, S, S_T=S)
+    assert S2.data_ptr() == S.data_ptr()
+    torch.testing.assert_close(S2, S1, rtol=0, atol=0)
+    torch.testing.assert_close(o2, o1, rtol=0, atol=0)
+
+
+def test_tc_status_word_ok(dev):
+    from gated_delta_rule_159_b200 import gdn2
+    inp = _small(dev, n_seqs=1, seq_len=64, n_heads=1)
+    ws = torch.empty(4096, dtype=torch.uint8, device=dev)
+    names = ("q", "k", "v", "log_a", "b", "w")
+    gdn2.chunk_fwd(*(inp[n][None] for n in names), inp["S0"], workspace=ws)
+    assert gdn2.check_status(ws) == gdn2.OK
+
+
+# ----------------------------------------------------------------- full-size workloads, sampled units
+def _sample_units(inp, k, seed, extra=()):
+    rng = np.random.default_rng(seed)
+    H = inp["q"].shape[1]
+    units = set(extra)
+    while len(units) < k + len(extra):
+        units.add((int(rng.integers(inp["n_seqs"])), int(rng.integers(H))))
+    return sorted(units)
+
+
+@pytest.mark.parametrize("name", ["gdn_scalar_b4_t4k", "gdn2_b8_t4k", "gdn2_varlen_16x4k-64k"])
+def test_full_size_sampled(dev, name):
+    inp = _inputs(name, dev)
+    o, S_T = run_chunk(inp)
+    torch.cuda.synchronize()
+    extra = ()
+    if not inp["equal_lengths"]:
+        lens = np.diff(inp["cu_host"])
+        extra = ((int(np.argmax(lens)), 0), (int(np.argmin(lens)), 15))
+    units = _sample_units(inp, 4, seed=7, extra=extra)
+    eo, es = compare_units(inp, o, S_T, units)
+    assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (name, eo, es)
+    # every output is finite across the whole workload
+    assert torch.isfinite(o).all() and torch.isfinite(S_T).all()
+
+
+# ----------------------------------------------------------------- decode
+@pytest.mark.parametrize("d,scalar", [(128, False), (64, False), (128, True)])
+def test_decode_small(dev, d, scalar):
+    from gated_delta_rule_159_b200 import gdn2, inputs
+    N, H, steps = 5, 3, 7
+    di = inputs.make_decode_inputs(N, H, d, steps, dev, seed=3)
+    if scalar:
+        for n in ("log_a", "b"):
+            di[n] = di[n][..., 0].contiguous()
+        di["w"] = None
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    S = torch.randn(N, H, d, d, generator=g, device=dev) * 0.1
+    S_start = to_f64(S)
+    outs = []
+    for t in range(steps):
+        outs.append(gdn2.decode_step(di["q"][t], di["k"][t], di["v"][t], di["log_a"][t], di["b"][t],
+                                     None if di["w"] is None else di["w"][t], S,
+                                     scalar_decay=scalar, scalar_gates=scalar, tied_gates=scalar))
+    o_gpu = to_f64(torch.stack(outs))  # [steps, N, H, d]
+    flags = (oracle.SCALAR_DECAY | oracle.SCALAR_GATES | oracle.TIED_GATES) if scalar else 0
+    # the decode steps of one (n, h) are one sequence of the recurrence
+    for n in range(N):
+        sl = lambda t: None if t is None else to_f64(t[:, n])  # noqa: E731
+        o_r, S_r = oracle.gdn2_fwd(sl(di["q"]), sl(di["k"]), sl(di["v"]), sl(di["log_a"]), sl(di["b"]),
+                                   sl(di["w"]), S0=S_start[n][None], flags=flags)
+        for h in range(H):
+            assert rel_err(o_gpu[:, n, h], o_r[:, h]) <= TOL_DECODE
+            assert rel_err(to_f64(S[n, h]), S_r[0, h]) <= TOL_DECODE
+
+
+def test_decode_full_size_sampled(dev):
+    """256 sequences x 16 heads x 128x128 state from a 2048-token chunked prefill,
+    then 1024 decode steps; the oracle starts from the GPU prefill state."""
+    from gated_delta_rule_159_b200 import gdn2, inputs
+    cfg = inputs.DECODE
+    N, H, d, steps = cfg["n_seqs"], cfg["n_heads"], cfg["d"], cfg["steps"]
+    w = inputs.Workload("decode_prefill", N, cfg["prefill_len"], H, d, d, 64, torch.bfloat16, 0.05, False, 0.0)
+    pre = inputs.make_inputs(w, dev)
+    _, S = run_chunk(pre)
+    del pre
+    di = inputs.make_decode_inputs(N, H, d, steps, dev, seed=1)
+    units = [(0, 0), (17, 5), (128, 9), (255, 15)]
+    S_start = {u: to_f64(S[u]) for u in units}
+    o = torch.empty(N, H, d, device=dev)
+    idx_n = torch.tensor([u[0] for u in units], device=dev)
+    idx_h = torch.tensor([u[1] for u in units], device=dev)
+    rec = []
+    for t in range(steps):
+        gdn2.decode_step(di["q"][t], di["k"][t], di["v"][t], di["log_a"][t], di["b"][t], di["w"][t], S, o=o)
+        rec.append(o[idx_n, idx_h].clone())
+    rec = to_f64(torch.stack(rec))  # [steps, len(units), d]
+    for i, (n, h) in enumerate(units):
+        sl = lambda t: to_f64(t[:, n, h:h + 1])  # noqa: E731
+        o_r, S_r = oracle.gdn2_fwd(sl(di["q"]), sl(di["k"]), sl(di["v"]), sl(di["log_a"]), sl(di["b"]),
+                                   sl(di["w"]), S0=S_start[(n, h)][None, None])
+        assert rel_err(rec[:, i], o_r[:, 0]) <= TOL_DECODE
+        assert rel_err(to_f64(S[n, h]), S_r[0, 0]) <= TOL_DECODE
