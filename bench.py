@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Throughput of the Gated DeltaNet-2 forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one chunked GDN-2 forward (every chunk-path row: TMA loads,
+cumulative log-decay, operand build, the A/B/QX/QP GEMM, (I+A)^-1, the W/U
+GEMMs, the state scan and the output epilogue) over the full GDN-2 workload:
+8 sequences x 4096 tokens x 16 heads x 128, bf16 inputs, fp32 state, chunk 64,
+channel-wise decay and decoupled channel-wise gates, S0 ~ N(0, 0.02).  Inputs
+(0.96 GB) are resident in HBM and larger than L2.  `value` is prefill
+tokens/s over all ranks (weak scaling: every rank runs its own batch; the
+units shard with no data-path collective).
+
+The same JSON line carries `decode`: 1024 recurrent decode steps over 256
+sequences x 16 heads with a 268 MB fp32 state built by a 2048-token chunked
+prefill (tokens/s and fraction of HBM bandwidth), the roofline of the chunk
+kernel, the end-to-end number through host buffers, the float64 CPU oracle as
+`cpu_baseline`, and the SM clocks sampled while timing.
+
+`--impl reference` times the float64 CPU oracle on a bounded sample of the
+same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill tokens/s (GDN-2 fwd, 16h×128d, T=4k); decode tok/s, % HBM BW"
+WORKLOAD = "gdn2_b8_t4k"
+FLOP_PER_TOKHEAD = 10 * 64 * 128 + 8 * 64 * 128 + 8 * 128 * 128  # GEMMs the chunk kernel issues (C=64, d=128)
+BYTES_PER_TOKHEAD = 6 * 128 * 2 + 128 * 2                      # six bf16 inputs + bf16 o
+STATE_BYTES = 128 * 128 * 4                                    # one fp32 state
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def kernel_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("chunk_tc.cu", "sm100_ptx.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "gated_delta_rule_159_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_per_launch():
+    """DRAM bytes per chunk-kernel launch from the committed ncu summary, if it
+    was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "chunk_tc_traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        if t.get("kernel_sha") == kernel_sha():
+            return t["bytes_per_launch_full_workload"]
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu_index), "-lms", "200"], stdout=self.file,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        mhz, mx, reasons = [], 0.0, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            try:
+                mhz.append(float(r[1]))
+                mx = max(mx, float(r[2]))
+                for nm, val in zip(names, r[5:9]):
+                    if val.strip().lower() == "active":
+                        reasons.add(nm)
+            except (ValueError, IndexError):
+                continue
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(inp, max_seconds: float, n_units: int = 0):
+    """Time the float64 oracle on whole (sequence, head) units of the workload,
+    as many as fit ~max_seconds of wall time on this host (all cores), or
+    exactly ``n_units`` units when given."""
+    import oracle
+    import torch
+    T = inp["T_tot"] // inp["n_seqs"]
+    H = inp["q"].shape[1]
+    threads = oracle.max_threads()
+    units_all = [(n, h) for n in range(inp["n_seqs"]) for h in range(H)]
+
+    def run(units):
+        sl = lambda t, n, h: t[n * T:(n + 1) * T, h:h + 1].float().cpu().numpy().astype(np.float64)  # noqa: E731
+        cat = {name: np.concatenate([sl(inp[name], n, h) for (n, h) in units])
+               for name in ("q", "k", "v", "log_a", "b", "w")}
+        S0 = np.stack([inp["S0"][n, h:h + 1].cpu().numpy().astype(np.float64) for (n, h) in units])
+        cu = np.arange(len(units) + 1, dtype=np.int64) * T
+        t0 = time.perf_counter()
+        oracle.gdn2_fwd(cat["q"], cat["k"], cat["v"], cat["log_a"], cat["b"], cat["w"], S0=S0, cu_seqlens=cu,
+                        n_threads=threads)
+        return time.perf_counter() - t0
+
+    n0 = min(len(units_all), threads)
+    if n_units:
+        units = units_all[:n_units]
+        dt = run(units)
+    else:
+        # calibrate on one unit per thread, then size the sample
+        dt0 = run(units_all[:n0])
+        per_batch = max(dt0, 1e-3)
+        batches = max(1, min(int(max_seconds / per_batch), math.ceil(len(units_all) / n0)))
+        units = units_all[:min(len(units_all), batches * n0)]
+        dt = run(units) if len(units) > n0 else dt0
+    tokens = len(units) * T / H  # tokens of the metric (a token carries all H heads)
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{len(units)} of {len(units_all)} (sequence, head) units x {T} tokens of {WORKLOAD}, "
+                      f"float64 C recurrence, {threads} OpenMP threads, {dt:.1f} s",
+            "seconds": dt, "n_units": len(units)}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from gated_delta_rule_159_b200 import inputs
+    inp = inputs.make_inputs(WORKLOAD, "cuda" if torch.cuda.is_available() else "cpu", seed=0)
+    per_step = []
+    cb = oracle_sample(inp, max_seconds=args.reference_step_seconds)  # sizes the per-step sample
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample(inp, 0.0, n_units=cb["n_units"])
+        if i >= args.warmup:
+            per_step.append(r)
+        cb = r
+    vals = [r["value"] for r in per_step]
+    secs = [r["seconds"] for r in per_step]
+    value = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.median(secs),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_block(inp, None),
+            "cpu_baseline": {k: cb[k] for k in ("unit", "cores", "kind", "sample")} | {"value": value},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(inp, world):
+    w = inp["workload"]
+    return {"workload": w.name, "batch": inp["n_seqs"], "seq_len": inp["T_tot"] // inp["n_seqs"],
+            "heads": w.n_heads, "d_k": w.d_k, "d_v": w.d_v, "chunk": w.chunk,
+            "gates": "channel-wise decay, decoupled channel-wise erase/write",
+            "tokens_per_step_per_gpu": inp["T_tot"], "l2": "inputs_exceed_l2",
+            "parallelism": f"dp{world}" if world else "cpu"}
+
+
+# ----------------------------------------------------------------------------- our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--reference-step-seconds", type=float, default=6.0)
+    ap.add_argument("--batch", type=int, default=0, help="override the batch size (small profiling cases)")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    from gated_delta_rule_159_b200 import gdn2, inputs
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    hbm_peak, tc_peak, peak_src = peaks()
+
+    # ---------------- prefill (the step)
+    inp = inputs.make_inputs(WORKLOAD, dev, seed=rank, n_seqs=args.batch or None)
+    N, T_tot = inp["n_seqs"], inp["T_tot"]
+    T = T_tot // N
+    names = ("q", "k", "v", "log_a", "b", "w")
+    args4 = [inp[n].view(N, T, *inp[n].shape[1:]) for n in names]
+    o = torch.empty(N, T, 16, 128, dtype=torch.bfloat16, device=dev)
+    ST = torch.empty(N, 16, 128, 128, dtype=torch.float32, device=dev)
+    dims = gdn2.make_dims(N, T, 16, 128, 128, 64, gdn2.BF16, gdn2.BF16, 0)
+    ws = torch.empty(gdn2.workspace_size(dims), dtype=torch.uint8, device=dev)
+
+    def step():
+        gdn2.chunk_fwd(*args4, inp["S0"], None, o=o, S_T=ST, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    sampler.start()
+    stream = torch.cuda.current_stream(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    barrier()
+    clocks = sampler.stop()
+    total_ms = ev[0][0].elapsed_time(ev[-1][1])
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(total_ms)
+    status = gdn2.check_status(ws)
+    if status != gdn2.OK:
+        raise RuntimeError(f"chunk kernel reported device status {status}")
+    tokens_all = T_tot * world * args.steps
+    value = tokens_all / (total_ms / 1e3)
+    ms_per_step = total_ms / args.steps
+
+    avg_launch_s = statistics.mean(launch_ms) / 1e3
+    units = N * 16
+    alg_bytes = BYTES_PER_TOKHEAD * T_tot * 16 + 2 * units * STATE_BYTES
+    alg_flops = FLOP_PER_TOKHEAD * T_tot * 16
+    achieved = alg_bytes / avg_launch_s / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                "traffic": traffic_per_launch(), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
+                "kernel": "chunk_tc_kernel", "alg_bytes_per_launch": alg_bytes,
+                "avg_launch_ms": avg_launch_s * 1e3,
+                "tensor_tflops": alg_flops / avg_launch_s / 1e12,
+                "tensor_frac": alg_flops / avg_launch_s / 1e12 / tc_peak,
+                "tensor_peak": tc_peak, "alg_flops_per_launch": alg_flops}
+
+    # ---------------- end to end through host buffers (pinned), same workload
+    e2e = None
+    if not args.no_e2e:
+        host = {n: args4[i].cpu().pin_memory() for i, n in enumerate(names)}
+        S0_h = inp["S0"].cpu().pin_memory()
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        ST_h = torch.empty(ST.shape, dtype=ST.dtype).pin_memory()
+        dev_in = {n: torch.empty_like(args4[i]) for i, n in enumerate(names)}
+        S0_d = torch.empty_like(inp["S0"])
+
+        def e2e_step():
+            for n in names:
+                dev_in[n].copy_(host[n], non_blocking=True)
+            S0_d.copy_(S0_h, non_blocking=True)
+            gdn2.chunk_fwd(*(dev_in[n] for n in names), S0_d, None, o=o, S_T=ST, workspace=ws)
+            o_h.copy_(o, non_blocking=True)
+            ST_h.copy_(ST, non_blocking=True)
+
+        e2e_step()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+        h2d = sum(t.numel() * t.element_size() for t in host.values()) + S0_h.numel() * 4
+        d2h = o_h.numel() * o_h.element_size() + ST_h.numel() * 4
+        e2e = {"value": T_tot * world * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+               "ms_per_step": e2e_ms / args.e2e_steps,
+               "path": "pinned host -> device copies, gdn2_chunk_fwd via the Python binding, o and S_T back"}
+        del host, dev_in, o_h, ST_h
+
+    # ---------------- CPU baseline (rank 0, one GPU only)
+    cpu = None
+    if not args.no_cpu and world == 1 and rank == 0:
+        cpu = oracle_sample(inp, args.cpu_seconds)
+        cpu.pop("seconds")
+        cpu.pop("n_units")
+
+    cfg = config_block(inp, world)
+    del inp, args4
+    torch.cuda.empty_cache()
+
+    # ---------------- decode
+    decode = None
+    launches = args.steps  # one chunk_tc_kernel launch per timed prefill step
+    if not args.no_decode:
+        dc = inputs.DECODE
+        Nd, Hd, d, steps = dc["n_seqs"], dc["n_heads"], dc["d"], args.decode_steps
+        wpre = inputs.Workload("decode_prefill", Nd, dc["prefill_len"], Hd, d, d, 64, torch.bfloat16, 0.05, False, 0.0)
+        pre = inputs.make_inputs(wpre, dev, seed=100 + rank)
+        _, S = gdn2.chunk_fwd(*(pre[n].view(Nd, dc["prefill_len"], *pre[n].shape[1:]) for n in names), None, None)
+        del pre
+        torch.cuda.empty_cache()
+        di = inputs.make_decode_inputs(Nd, Hd, d, steps, dev, seed=200 + rank)
+        od = torch.empty(Nd, Hd, d, dtype=torch.float32, device=dev)
+        for t in range(3):
+            gdn2.decode_step(*(di[n][t] for n in names), S, o=od)
+        barrier()
+        sd = ClockSampler(dev.index if dev.index is not None else 0)
+        sd.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        e0.record(stream)
+        for t in range(steps):
+            gdn2.decode_step(*(di[n][t] for n in names), S, o=od)
+        e1.record(stream)
+        barrier()
+        dclocks = sd.stop()
+        dms = max_over_ranks(e0.elapsed_time(e1))
+        step_bytes = 2 * Nd * Hd * d * d * 4 + 6 * Nd * Hd * d * 2 + Nd * Hd * d * 4
+        gbs = step_bytes * steps / (dms / 1e3) / 1e9
+        decode = {"value": Nd * world * steps / (dms / 1e3), "unit": "tokens/s", "steps": steps,
+                  "us_per_step": 1e3 * dms / steps, "bytes_per_step": step_bytes, "hbm_gbs": gbs,
+                  "hbm_frac": gbs / hbm_peak, "peak_source": peak_src, "sequences": Nd, "heads": Hd,
+                  "state_bytes": Nd * Hd * d * d * 4, "clocks": dclocks, "kernel": "decode_kernel",
+                  "launch": "one launch per step (plain stream loop)", "gpu_launches": steps}
+        del di, S
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes and distributions of the "
+                                                          "full GDN-2 workload)",
+            "config": cfg, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches, "clocks": clocks, "decode": decode}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
