@@ -77,6 +77,10 @@ int check_inputs(const void *q, const void *k, const void *v, const void *log_a,
 
 }  // namespace
 
+namespace gdn2 {
+int set_last_error(int code, const char *message) { return fail(code, "%s", message); }
+}  // namespace gdn2
+
 extern "C" {
 
 int gdn2_version(void) { return 100; }

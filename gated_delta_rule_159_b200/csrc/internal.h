@@ -38,6 +38,9 @@ struct DecodeProblem {
 // Status word values written by kernels (0 = fine).
 constexpr int32_t kStatusTimeout = 1;
 
+// Record `message` as this thread's gdn2_last_error() text and return `code`.
+int set_last_error(int code, const char *message);
+
 cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream);
 cudaError_t launch_chunk_simt(const ChunkProblem &p, cudaStream_t stream);
 // Tensor-core path (d_k = d_v = 128, C = 64, bf16 in).  Returns cudaErrorNotSupported

@@ -162,6 +162,36 @@ int gdn2_decode_step(const void *q, const void *k, const void *v,
                      const void *log_a, const void *b, const void *w,
                      float *S, void *o, const gdn2_dims *dims, gdn2_stream_t stream);
 
+/*
+ * gdn2_chunk_fwd_noalloc -- gdn2_chunk_fwd for callers that cannot allocate
+ * device memory.  (The paper has no counterpart; this is a deployment aid.)
+ *
+ * Some callers cannot call cudaMalloc: a plugin inside a host framework whose
+ * allocator owns all device memory (e.g. a serving engine that reserves nearly
+ * all of HBM up front), or code on a path where cudaMalloc's implicit device
+ * synchronisation is not allowed.  This entry point takes the same arguments
+ * as gdn2_chunk_fwd minus the workspace, and uses instead a fixed scratch
+ * array of 256 + 4 * GDN2_NOALLOC_MAX_UNITS bytes compiled into the library:
+ * every GPU that loads libgdn2.so holds it until the process exits.  It calls
+ * no cudaMalloc, cudaFree or other allocating routine.  The caller still owns
+ * and passes all inputs and outputs.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents; the
+ *     call clears the parts that must start at zero itself.  Calls whose
+ *     executions overlap on the GPU (different streams, or concurrent host
+ *     threads on one device) race on the array: serialise them.
+ *   - Problems with more than GDN2_NOALLOC_MAX_UNITS (sequence, head) units
+ *     are rejected with GDN2_ERR_UNSUPPORTED and a message naming the limit.
+ * Errors: as gdn2_chunk_fwd, plus GDN2_ERR_UNSUPPORTED for the size limit.
+ */
+#define GDN2_NOALLOC_MAX_UNITS 16384
+int gdn2_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                           const void *log_a, const void *b, const void *w,
+                           const float *S0, const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                           void *o, float *S_T, const gdn2_dims *dims, gdn2_stream_t stream);
+
 /* Thread-local description of the last non-zero status on this thread ("" if none). */
 const char *gdn2_last_error(void);
 
