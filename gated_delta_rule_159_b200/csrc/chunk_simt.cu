@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkProblem p) {
       for (int j = 0; j <= i; ++j) acc += sQP[i * C + j] * sv[j * dv + d] - sQX[i * C + j] * sM[j * dv + d];
       go[((size_t)(bos + c0 + i) * H + h) * dv + d] = from_f32<Tout>(acc);
     }
+    __syncthreads();  // every output has read S before the update below overwrites it
     // 7. state update (each thread reads and writes only its own S elements)
     for (int e = tid; e < dk * dv; e += kThreads) {
       const int c = e / dv, d = e % dv;

@@ -46,9 +46,10 @@ namespace {
 
 constexpr int C = 64;
 constexpr int D = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s
+constexpr float kLog2eF = 1.4426950408889634f;
 
 // Shared-memory map, byte offsets from a 1024-byte-aligned base.  Every operand
 // tile is a stack of 8-row x 128-byte swizzle atoms.
@@ -63,34 +64,37 @@ constexpr uint32_t OFF_QX = 147456;    // QX bf16 [64 x 64]
 constexpr uint32_t OFF_QP = 155648;    // QP bf16 [64 x 64]
 constexpr uint32_t OFF_WT = 163840;    // W_r^T bf16 [128 x 64]; fp32 T during the solve
 constexpr uint32_t OFF_BZ = 180224;    // (B V)^T bf16 [128 x 64]; o staging (with OFF_MT)
-constexpr uint32_t OFF_MT = 196608;    // -M^T bf16 [128 x 64]; solve scratch
+constexpr uint32_t OFF_MT = 196608;    // -M^T bf16 [128 x 64]; per-warp 16x16 scratch in the solve
 constexpr uint32_t OFF_MISC = 212992;
 constexpr uint32_t MISC_GC = 0;        // float[128]  e^{L_C}
 constexpr uint32_t MISC_DL = 512;      // float[128]  e^{L_C - L_ref}
 constexpr uint32_t MISC_SM = 1024;     // float[128]  e^{L_ref}
-constexpr uint32_t MISC_PART = 1536;   // float[4][128] quarter sums of log_a
-constexpr uint32_t MISC_BAR_TMA = 3584;
-constexpr uint32_t MISC_BAR_MMA = 3592;
-constexpr uint32_t MISC_TMEM = 3600;
-constexpr uint32_t MISC_ABORT = 3604;
-constexpr uint32_t MISC_UNIT = 3608;
-constexpr uint32_t MISC_BYTES = 3616;
+constexpr uint32_t MISC_PART = 1536;   // float[16][128] 4-row sums of log_a, then exclusive prefixes
+constexpr uint32_t MISC_REF = 9728;    // float[128]  L_ref
+constexpr uint32_t MISC_BAR = 10240;   // 8 mbarriers
+constexpr uint32_t MISC_TMEM = 10304;
+constexpr uint32_t MISC_ABORT = 10308;
+constexpr uint32_t MISC_UNIT = 10312;
+constexpr uint32_t MISC_BYTES = 10320;
 constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES + 1024;  // + base alignment slack
+// mbarrier slots
+enum { BAR_TMA_A = 0, BAR_TMA_B, BAR_G1, BAR_E1, BAR_E2, BAR_G2, BAR_G3, BAR_G45, kNumBars };
 
 struct TcParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_g, tm_b, tm_w;
+  CUtensorMap tm_o;  // o viewed as (channel, head, token), box 64 (bf16) or 32 (fp32) x 1 x 64, no swizzle
   ChunkProblem p;
   int32_t *counter;
   int n_units;
 };
 
-__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+__device__ __forceinline__ uint2 lds_v2(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
   return v;
 }
-__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
-  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+__device__ __forceinline__ void sts_v2(uint32_t a, uint2 v) {
+  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(v.x), "r"(v.y) : "memory");
 }
 __device__ __forceinline__ void sts_u16(uint32_t a, uint16_t v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(v) : "memory");
@@ -111,7 +115,7 @@ __device__ __forceinline__ uint4 lds_v4(uint32_t a) {
 // fp32 64x64 scratch with a 16-byte-chunk XOR swizzle (conflict-free row writes).
 __device__ __forceinline__ int fidx(int i, int j) { return i * 64 + ((((j >> 2) ^ (i & 7))) << 2) + (j & 3); }
 
-// Byte offset of element pair (row r, 16-byte chunk `chunk`) in a 128B-swizzled tile.
+// Byte offset of (row r, 16-byte chunk `chunk`) in a 128B-swizzled tile.
 __device__ __forceinline__ uint32_t swz(int r, uint32_t chunk) {
   return (uint32_t)r * 128u + (((chunk ^ (uint32_t)(r & 7))) << 4);
 }
@@ -143,6 +147,13 @@ __device__ __forceinline__ uint4 pack8(const float *f, float s) {
   v.w = pack_bf16x2(f[6] * s, f[7] * s);
   return v;
 }
+__device__ __forceinline__ float4 unpack4(uint2 u) {
+  const float2 a = unpack_bf16x2(u.x), b = unpack_bf16x2(u.y);
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ uint2 pack4(float a, float b, float c, float d) {
+  return make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
+}
 
 template <bool kScalarDecay, bool kScalarGates, typename Tout>
 __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_constant__ TcParams P) {
@@ -152,7 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   const uint32_t sb = (raw + 1023u) & ~1023u;
   uint8_t *gb = smem_raw + (sb - raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qd = warp & 3, hf = warp >> 2;
+  const int qd = warp & 3, cg = warp >> 2;   // TMEM lane quadrant, column group
+  const int row = qd * 32 + lane;            // the TMEM lane this thread reads
   const int H = p.n_heads;
   const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
 
@@ -160,14 +172,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   float *sDL = reinterpret_cast<float *>(gb + OFF_MISC + MISC_DL);
   float *sSM = reinterpret_cast<float *>(gb + OFF_MISC + MISC_SM);
   float *part = reinterpret_cast<float *>(gb + OFF_MISC + MISC_PART);
+  float *sRef = reinterpret_cast<float *>(gb + OFF_MISC + MISC_REF);
+  constexpr int kIssuer = 32;  // thread that issues TMA and the early MMAs (warp 1, lane 0)
   volatile int *sAbort = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_ABORT);
   volatile int *sUnit = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_UNIT);
-  const uint32_t barTma = sb + OFF_MISC + MISC_BAR_TMA;
-  const uint32_t barMma = sb + OFF_MISC + MISC_BAR_MMA;
+  auto bar = [&](int i) { return sb + OFF_MISC + MISC_BAR + 8u * (uint32_t)i; };
 
   if (tid == 0) {
-    ptx::mbar_init(barTma, 1);
-    ptx::mbar_init(barMma, 1);
+    for (int i = 0; i < kNumBars; ++i) ptx::mbar_init(bar(i), 1);
     ptx::fence_mbar_init();
     *sAbort = 0;
     ptx::tma_prefetch_desc(&P.tm_q);
@@ -182,17 +194,38 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(gb + OFF_MISC + MISC_TMEM);
-  const uint32_t tmD1 = tmem;        // G1 result, then dS (128 cols)
+  const uint32_t tmD1 = tmem;        // G1 result; then W_r^T | (B V)^T; then M^T (128 cols)
   const uint32_t tmS = tmem + 128;   // fp32 state (128 cols)
-  const uint32_t tmW = tmem + 256;   // W_r^T, then M^T (64 cols)
-  const uint32_t tmBZ = tmem + 320;  // (B V)^T, then O^T (64 cols)
+  const uint32_t tmDS = tmem + 256;  // state increment dS (128 cols)
+  const uint32_t tmO = tmem + 384;   // O^T (64 cols)
   const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
-  const int row = qd * 32 + lane;    // the TMEM lane this thread reads
-  uint32_t tma_phase = 0, mma_phase = 0;
+  uint32_t it = 0;                   // chunks processed by this CTA: parity of every mbarrier
 
   const __nv_bfloat16 *g_la = static_cast<const __nv_bfloat16 *>(p.log_a);
   const __nv_bfloat16 *g_b = static_cast<const __nv_bfloat16 *>(p.b);
   const __nv_bfloat16 *g_w = static_cast<const __nv_bfloat16 *>(tied ? p.b : p.w);
+
+  // TMA issue (thread 0): group A = k, q, v (+ log_a), group B = b, w.
+  auto issue_tma_a = [&](int h, int t0) {
+    uint32_t bytes = 3u * 2u * 8192u + (kScalarDecay ? 0u : 2u * 8192u);
+    ptx::mbar_arrive_expect_tx(bar(BAR_TMA_A), bytes);
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) {
+      ptx::tma_load_3d(sb + OFF_KQ + kb * 16384, &P.tm_k, kb * 64, h, t0, bar(BAR_TMA_A));
+      ptx::tma_load_3d(sb + OFF_KQ + kb * 16384 + 8192, &P.tm_q, kb * 64, h, t0, bar(BAR_TMA_A));
+      ptx::tma_load_3d(sb + OFF_V + kb * 8192, &P.tm_v, kb * 64, h, t0, bar(BAR_TMA_A));
+      if (!kScalarDecay) ptx::tma_load_3d(sb + OFF_G + kb * 8192, &P.tm_g, kb * 64, h, t0, bar(BAR_TMA_A));
+    }
+  };
+  auto issue_tma_b = [&](int h, int t0) {
+    if (kScalarGates) return;
+    ptx::mbar_arrive_expect_tx(bar(BAR_TMA_B), 2u * 2u * 8192u);
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) {
+      ptx::tma_load_3d(sb + OFF_XP + kb * 16384, &P.tm_b, kb * 64, h, t0, bar(BAR_TMA_B));
+      ptx::tma_load_3d(sb + OFF_XP + kb * 16384 + 8192, &P.tm_w, kb * 64, h, t0, bar(BAR_TMA_B));
+    }
+  };
 
   for (;;) {
     if (tid == 0) *sUnit = atomicAdd(P.counter, 1);
@@ -209,12 +242,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       bos = (int64_t)n * p.seq_len;
       len = p.seq_len;
     }
+    const int nchunks = (int)((len + C - 1) / C);
+    if (tid == kIssuer && nchunks > 0 && !*sAbort) {
+      issue_tma_a(h, (int)bos);
+      issue_tma_b(h, (int)bos);
+    }
 
-    // ---- initial state into TMEM (thread: dk row `row`, dv columns [64 hf, 64 hf + 64))
-    for (int h32 = 0; h32 < 2; ++h32) {
+    // ---- initial state into TMEM (thread: dk row `row`, dv columns [32 cg, 32 cg + 32))
+    {
       uint32_t r[32];
       if (p.S0) {
-        const float4 *src = reinterpret_cast<const float4 *>(p.S0 + ((size_t)unit * D + row) * D + hf * 64 + h32 * 32);
+        const float4 *src = reinterpret_cast<const float4 *>(p.S0 + ((size_t)unit * D + row) * D + cg * 32);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const float4 f = src[j];
@@ -227,388 +265,450 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
 #pragma unroll
         for (int j = 0; j < 32; ++j) r[j] = 0u;
       }
-      ptx::tmem_st32(tmS + lane_base + hf * 64 + h32 * 32, r);
+      ptx::tmem_st32(tmS + lane_base + cg * 32, r);
+      ptx::tmem_wait_st();
     }
-    ptx::tmem_wait_st();
 
-    for (int64_t c0 = 0; c0 < len; c0 += C) {
+    for (int ci = 0; ci < nchunks; ++ci, ++it) {
+      const uint32_t par = it & 1u;
+      const int64_t c0 = (int64_t)ci * C;
       const int nvalid = (int)((len - c0) < C ? (len - c0) : C);
       const int t0 = (int)(bos + c0);
+      const bool has_next = ci + 1 < nchunks;
 
-      // ---- a1: TMA loads of the chunk tiles
-      if (tid == 0 && !*sAbort) {
-        uint32_t bytes = 3u * 2u * 8192u;
-        if (!kScalarDecay) bytes += 2u * 8192u;
-        if (!kScalarGates) bytes += 2u * 2u * 8192u;
-        ptx::mbar_arrive_expect_tx(barTma, bytes);
-#pragma unroll
-        for (int kb = 0; kb < 2; ++kb) {
-          ptx::tma_load_3d(sb + OFF_KQ + kb * 16384, &P.tm_k, kb * 64, h, t0, barTma);
-          ptx::tma_load_3d(sb + OFF_KQ + kb * 16384 + 8192, &P.tm_q, kb * 64, h, t0, barTma);
-          ptx::tma_load_3d(sb + OFF_V + kb * 8192, &P.tm_v, kb * 64, h, t0, barTma);
-          if (!kScalarGates) {
-            ptx::tma_load_3d(sb + OFF_XP + kb * 16384, &P.tm_b, kb * 64, h, t0, barTma);
-            ptx::tma_load_3d(sb + OFF_XP + kb * 16384 + 8192, &P.tm_w, kb * 64, h, t0, barTma);
-          }
-          if (!kScalarDecay) ptx::tma_load_3d(sb + OFF_G + kb * 8192, &P.tm_g, kb * 64, h, t0, barTma);
-        }
-      }
-      wait_bar(barTma, tma_phase, sAbort, p.status);
-      tma_phase ^= 1u;
+      wait_bar(bar(BAR_TMA_A), par, sAbort, p.status);
+      if (!kScalarGates) wait_bar(bar(BAR_TMA_B), par, sAbort, p.status);
 
-      // ---- a2/a3: cumulative log-decay and scaled operands, in place
+      // ---- a2/a3: cumulative log-decay and scaled operands, in place.
+      // thread: channels 4 cq .. 4 cq + 3, rows 4 warp .. 4 warp + 3.
       {
-        const int cp = tid & 63, rq = tid >> 6, kb = cp >> 5;
-        const uint32_t ch16 = (uint32_t)((cp & 31) >> 2), cofs = (uint32_t)(cp & 3) * 4u;
-        float L0[16], L1[16];
-        float a0 = 0.f, a1 = 0.f;
+        const int cq = lane, kb = cq >> 4;
+        const uint32_t ch16 = (uint32_t)((cq & 15) >> 1), cofs = (uint32_t)(cq & 1) * 8u;
+        float4 L[4];
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
-          const int r = rq * 16 + rr;
-          float g0 = 0.f, g1 = 0.f;
+        for (int rr = 0; rr < 4; ++rr) {
+          const int r = warp * 4 + rr;
+          float4 g = make_float4(0.f, 0.f, 0.f, 0.f);
           if (r < nvalid) {
             if (kScalarDecay) {
-              g0 = g1 = __bfloat162float(g_la[(size_t)(t0 + r) * H + h]);
+              const float s = __bfloat162float(g_la[(size_t)(t0 + r) * H + h]);
+              g = make_float4(s, s, s, s);
             } else {
-              const float2 f = unpack_bf16x2(lds_u32(sb + OFF_G + kb * 8192 + swz(r, ch16) + cofs));
-              g0 = f.x;
-              g1 = f.y;
+              g = unpack4(lds_v2(sb + OFF_G + kb * 8192 + swz(r, ch16) + cofs));
             }
           }
-          a0 += g0;
-          a1 += g1;
-          L0[rr] = a0;
-          L1[rr] = a1;
+          acc.x += g.x; acc.y += g.y; acc.z += g.z; acc.w += g.w;
+          L[rr] = acc;
         }
-        part[rq * 128 + 2 * cp] = a0;
-        part[rq * 128 + 2 * cp + 1] = a1;
+        *reinterpret_cast<float4 *>(part + warp * 128 + 4 * cq) = acc;
         __syncthreads();
-        float off0 = 0.f, off1 = 0.f;
-        for (int j = 0; j < rq; ++j) {
-          off0 += part[j * 128 + 2 * cp];
-          off1 += part[j * 128 + 2 * cp + 1];
-        }
-        const float ref0 = part[2 * cp] + part[128 + 2 * cp];
-        const float ref1 = part[2 * cp + 1] + part[128 + 2 * cp + 1];
-        const float end0 = ref0 + part[256 + 2 * cp] + part[384 + 2 * cp];
-        const float end1 = ref1 + part[256 + 2 * cp + 1] + part[384 + 2 * cp + 1];
-        if (rq == 0) {
-          sGC[2 * cp] = exp_fast(end0);
-          sGC[2 * cp + 1] = exp_fast(end1);
-          sDL[2 * cp] = exp_fast(end0 - ref0);
-          sDL[2 * cp + 1] = exp_fast(end1 - ref1);
-          sSM[2 * cp] = exp_fast(ref0);
-          sSM[2 * cp + 1] = exp_fast(ref1);
-        }
+        if (tid < D) {  // per channel: exclusive prefix over the 16 row groups, L_ref = L_31, L_C = L_63
+          float run = 0.f, refv = 0.f;
 #pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
-          const int r = rq * 16 + rr;
-          const uint32_t o = kb * 16384 + swz(r, ch16) + cofs;
-          const float l0 = off0 + L0[rr] - ref0, l1 = off1 + L1[rr] - ref1;
-          const float e10 = exp_fast(l0), e11 = exp_fast(l1);
-          const float e20 = exp_fast(-l0), e21 = exp_fast(-l1);
-          float2 kk = unpack_bf16x2(lds_u32(sb + OFF_KQ + o));
-          float2 qq = unpack_bf16x2(lds_u32(sb + OFF_KQ + o + 8192));
-          float2 bb, ww;
+          for (int j = 0; j < 16; ++j) {
+            const float pj = part[j * 128 + tid];
+            part[j * 128 + tid] = run;
+            run += pj;
+            if (j == 7) refv = run;
+          }
+          sRef[tid] = refv;
+          sGC[tid] = ptx::ex2(run * kLog2eF);
+          sDL[tid] = ptx::ex2((run - refv) * kLog2eF);
+          sSM[tid] = ptx::ex2(refv * kLog2eF);
+        }
+        __syncthreads();
+        const float4 off = *reinterpret_cast<const float4 *>(part + warp * 128 + 4 * cq);
+        const float4 ref = *reinterpret_cast<const float4 *>(sRef + 4 * cq);
+        const float4 base = make_float4((off.x - ref.x) * kLog2eF, (off.y - ref.y) * kLog2eF,
+                                        (off.z - ref.z) * kLog2eF, (off.w - ref.w) * kLog2eF);
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          const int r = warp * 4 + rr;
+          const uint32_t o = (uint32_t)kb * 16384u + swz(r, ch16) + cofs;
+          const float l0 = fmaf(L[rr].x, kLog2eF, base.x), l1 = fmaf(L[rr].y, kLog2eF, base.y);
+          const float l2 = fmaf(L[rr].z, kLog2eF, base.z), l3 = fmaf(L[rr].w, kLog2eF, base.w);
+          const float e10 = ptx::ex2(l0), e11 = ptx::ex2(l1), e12 = ptx::ex2(l2), e13 = ptx::ex2(l3);
+          const float e20 = ptx::ex2(-l0), e21 = ptx::ex2(-l1), e22 = ptx::ex2(-l2), e23 = ptx::ex2(-l3);
+          float4 kk = unpack4(lds_v2(sb + OFF_KQ + o));
+          float4 qq = unpack4(lds_v2(sb + OFF_KQ + o + 8192));
+          float4 bb, ww;
           if (kScalarGates) {
-            bb.x = bb.y = 0.f;
+            bb = make_float4(0.f, 0.f, 0.f, 0.f);
             ww = bb;
             if (r < nvalid) {
-              bb.x = bb.y = __bfloat162float(g_b[(size_t)(t0 + r) * H + h]);
-              ww.x = ww.y = __bfloat162float(g_w[(size_t)(t0 + r) * H + h]);
+              const float sbv = __bfloat162float(g_b[(size_t)(t0 + r) * H + h]);
+              const float swv = __bfloat162float(g_w[(size_t)(t0 + r) * H + h]);
+              bb = make_float4(sbv, sbv, sbv, sbv);
+              ww = make_float4(swv, swv, swv, swv);
             }
           } else {
-            bb = unpack_bf16x2(lds_u32(sb + OFF_XP + o));
-            ww = unpack_bf16x2(lds_u32(sb + OFF_XP + o + 8192));
+            bb = unpack4(lds_v2(sb + OFF_XP + o));
+            ww = unpack4(lds_v2(sb + OFF_XP + o + 8192));
           }
           if (r >= nvalid) {
-            kk = make_float2(0.f, 0.f);
+            kk = make_float4(0.f, 0.f, 0.f, 0.f);
             qq = kk;
             bb = kk;
             ww = kk;
-            sts_u32(sb + OFF_V + kb * 8192 + swz(r, ch16) + cofs, 0u);
+            sts_v2(sb + OFF_V + kb * 8192 + swz(r, ch16) + cofs, make_uint2(0u, 0u));
           }
-          sts_u32(sb + OFF_KQ + o, pack_bf16x2(kk.x * e10, kk.y * e11));
-          sts_u32(sb + OFF_KQ + o + 8192, pack_bf16x2(qq.x * e10, qq.y * e11));
-          sts_u32(sb + OFF_XP + o, pack_bf16x2(bb.x * kk.x * e20, bb.y * kk.y * e21));
-          sts_u32(sb + OFF_XP + o + 8192, pack_bf16x2(ww.x * kk.x * e20, ww.y * kk.y * e21));
+          sts_v2(sb + OFF_KQ + o, pack4(kk.x * e10, kk.y * e11, kk.z * e12, kk.w * e13));
+          sts_v2(sb + OFF_KQ + o + 8192, pack4(qq.x * e10, qq.y * e11, qq.z * e12, qq.w * e13));
+          sts_v2(sb + OFF_XP + o, pack4(bb.x * kk.x * e20, bb.y * kk.y * e21, bb.z * kk.z * e22, bb.w * kk.w * e23));
+          sts_v2(sb + OFF_XP + o + 8192,
+                 pack4(ww.x * kk.x * e20, ww.y * kk.y * e21, ww.z * kk.z * e22, ww.w * kk.w * e23));
         }
       }
       __syncthreads();
 
-      // ---- S_r = Diag(e^{L_ref}) S as a bf16 MN-major operand
+      // ---- S_r = Diag(e^{L_ref}) S as a bf16 MN-major operand (dv columns [32 cg, 32 cg + 32))
       {
         const float sm = sSM[row];
-#pragma unroll
-        for (int h32 = 0; h32 < 2; ++h32) {
-          uint32_t r[32];
-          ptx::tmem_ld32(tmS + lane_base + hf * 64 + h32 * 32, r);
-          ptx::tmem_wait_ld();
-          float f[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(r[j]);
-#pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8)
-            sts_v4(sb + OFF_SR + hf * 16384 + swz(row, (uint32_t)(h32 * 4 + q8)), pack8(f + 8 * q8, sm));
-        }
-      }
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      __syncthreads();
-
-      // ---- a4: G1  [A B; QX QP] = [k_r; q_r] [x_r; p_r]^T
-      if (tid == 0) {
-        ptx::tc_fence_after();
-        constexpr uint32_t id = ptx::idesc_bf16(128, 128, false, false);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t ko = (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
-          ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_KQ + ko, 16, 1024),
-                         ptx::sdesc_sw128(sb + OFF_XP + ko, 16, 1024), id, kk > 0);
-        }
-        ptx::umma_commit(barMma);
-      }
-      wait_bar(barMma, mma_phase, sAbort, p.status);
-      mma_phase ^= 1u;
-      ptx::tc_fence_after();
-
-      // masks: A, B strictly lower (fp32 A for the solve, bf16 B); QX, QP lower incl. diagonal
-      {
-        float *Af = reinterpret_cast<float *>(gb + OFF_G);
-#pragma unroll
-        for (int h32 = 0; h32 < 2; ++h32) {
-          uint32_t r[32];
-          ptx::tmem_ld32(tmD1 + lane_base + hf * 64 + h32 * 32, r);
-          ptx::tmem_wait_ld();
-          float f[32];
-          if (qd < 2) {
-            const int i = row;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) f[j] = (h32 * 32 + j < i) ? __uint_as_float(r[j]) : 0.f;
-            if (hf == 0) {
-#pragma unroll
-              for (int j4 = 0; j4 < 8; ++j4)
-                *reinterpret_cast<float4 *>(Af + fidx(i, h32 * 32 + 4 * j4)) =
-                    make_float4(f[4 * j4], f[4 * j4 + 1], f[4 * j4 + 2], f[4 * j4 + 3]);
-            } else {
-#pragma unroll
-              for (int q8 = 0; q8 < 4; ++q8)
-                sts_v4(sb + OFF_BM + swz(i, (uint32_t)(h32 * 4 + q8)), pack8(f + 8 * q8, 1.f));
-            }
-          } else {
-            const int i = row - 64;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) f[j] = (h32 * 32 + j <= i) ? __uint_as_float(r[j]) : 0.f;
-            const uint32_t dst = hf == 0 ? OFF_QX : OFF_QP;
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) sts_v4(sb + dst + swz(i, (uint32_t)(h32 * 4 + q8)), pack8(f + 8 * q8, 1.f));
-          }
-        }
-      }
-      __syncthreads();
-
-      // ---- a5: T = (I + A)^-1 by blocked forward substitution (fp32)
-      {
-        const float *Af = reinterpret_cast<const float *>(gb + OFF_G);
-        float *Tf = reinterpret_cast<float *>(gb + OFF_WT);
-        float *Xs = reinterpret_cast<float *>(gb + OFF_MT);
-        if (tid < 64) {
-          const int I = tid >> 4, m = tid & 15;
-          float t[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float acc = (i == m) ? 1.f : 0.f;
-#pragma unroll
-            for (int j = 0; j < i; ++j) acc -= Af[fidx(16 * I + i, 16 * I + j)] * t[j];
-            t[i] = acc;
-          }
-#pragma unroll
-          for (int i = 0; i < 16; ++i) Tf[fidx(16 * I + i, 16 * I + m)] = t[i];
-        } else {
-          for (int e = tid - 64; e < 6 * 256; e += kThreads - 64) {
-            const int blk = e >> 8, i = (e >> 4) & 15, m = e & 15;
-            const int I = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-            const int J = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-            Tf[fidx(16 * I + i, 16 * J + m)] = 0.f;
-          }
-        }
-        __syncthreads();
-        for (int d = 1; d < 4; ++d) {
-          const int nb = 4 - d;
-          for (int e = tid; e < nb * 256; e += kThreads) {
-            const int J = e >> 8, I = J + d, i = (e >> 4) & 15, m = e & 15;
-            float acc = 0.f;
-            for (int K = J; K < I; ++K) {
-#pragma unroll
-              for (int s = 0; s < 16; ++s) acc += Af[fidx(16 * I + i, 16 * K + s)] * Tf[fidx(16 * K + s, 16 * J + m)];
-            }
-            Xs[e] = acc;
-          }
-          __syncthreads();
-          for (int e = tid; e < nb * 256; e += kThreads) {
-            const int J = e >> 8, I = J + d, i = (e >> 4) & 15, m = e & 15;
-            float acc = 0.f;
-            for (int r2 = 0; r2 <= i; ++r2) acc -= Tf[fidx(16 * I + i, 16 * I + r2)] * Xs[(J << 8) + (r2 << 4) + m];
-            Tf[fidx(16 * I + i, 16 * J + m)] = acc;
-          }
-          __syncthreads();
-        }
-        {
-          const int i = tid >> 2, seg = tid & 3;
-#pragma unroll
-          for (int u2 = 0; u2 < 2; ++u2) {
-            const int j0 = seg * 16 + u2 * 8;
-            float f[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) f[j] = Tf[fidx(i, j0 + j)];
-            sts_v4(sb + OFF_T + swz(i, (uint32_t)(j0 >> 3)), pack8(f, 1.f));
-          }
-        }
-      }
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      __syncthreads();
-
-      // ---- a6: G2  W_r^T = k_r^T T^T,  (B V)^T = V^T B^T
-      if (tid == 0) {
-        ptx::tc_fence_after();
-        constexpr uint32_t id = ptx::idesc_bf16(128, 64, true, false);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmW, ptx::sdesc_sw128(sb + OFF_KQ + kk * 2048, 16384, 1024),
-                         ptx::sdesc_sw128(sb + OFF_T + kk * 32, 16, 1024), id, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmBZ, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
-                         ptx::sdesc_sw128(sb + OFF_BM + kk * 32, 16, 1024), id, kk > 0);
-        ptx::umma_commit(barMma);
-      }
-      wait_bar(barMma, mma_phase, sAbort, p.status);
-      mma_phase ^= 1u;
-      ptx::tc_fence_after();
-      {
-        const uint32_t src = hf == 0 ? tmW : tmBZ;
-        const uint32_t dst = hf == 0 ? OFF_WT : OFF_BZ;
-#pragma unroll
-        for (int h32 = 0; h32 < 2; ++h32) {
-          uint32_t r[32];
-          ptx::tmem_ld32(src + lane_base + h32 * 32, r);
-          ptx::tmem_wait_ld();
-          float f[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(r[j]);
-#pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) sts_v4(sb + dst + swz(row, (uint32_t)(h32 * 4 + q8)), pack8(f + 8 * q8, 1.f));
-        }
-      }
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      __syncthreads();
-
-      // ---- a7 (erase reads): G3  M^T = (B V)^T T^T + S_r^T W_r^T
-      if (tid == 0) {
-        ptx::tc_fence_after();
-        constexpr uint32_t idA = ptx::idesc_bf16(128, 64, false, false);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmW, ptx::sdesc_sw128(sb + OFF_BZ + kk * 32, 16, 1024),
-                         ptx::sdesc_sw128(sb + OFF_T + kk * 32, 16, 1024), idA, kk > 0);
-        constexpr uint32_t idB = ptx::idesc_bf16(128, 64, true, true);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          ptx::umma_bf16(tmW, ptx::sdesc_sw128(sb + OFF_SR + kk * 2048, 16384, 1024),
-                         ptx::sdesc_sw128(sb + OFF_WT + kk * 2048, 16384, 1024), idB, 1);
-        ptx::umma_commit(barMma);
-      }
-      wait_bar(barMma, mma_phase, sAbort, p.status);
-      mma_phase ^= 1u;
-      ptx::tc_fence_after();
-      {
         uint32_t r[32];
-        ptx::tmem_ld32(tmW + lane_base + hf * 32, r);
+        ptx::tmem_ld32(tmS + lane_base + cg * 32, r);
         ptx::tmem_wait_ld();
         float f[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(r[j]);
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) sts_v4(sb + OFF_MT + swz(row, (uint32_t)(hf * 4 + q8)), pack8(f + 8 * q8, -1.f));
+        for (int q8 = 0; q8 < 4; ++q8)
+          sts_v4(sb + OFF_SR + (uint32_t)(cg >> 1) * 16384u + swz(row, (uint32_t)((cg & 1) * 4 + q8)),
+                 pack8(f + 8 * q8, sm));
       }
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncthreads();
 
-      // ---- a7/a8: G4 outputs and G5 state increment
-      if (tid == 0) {
+      // ---- a4: G1 [A B; QX QP] = [k_r; q_r] [x_r; p_r]^T, then the state-independent parts of
+      //      dS (p_r^T V) and O^T (S_r^T q_r^T), which run while the CUDA cores mask and solve.
+      if (tid == 0 && !*sAbort) {
         ptx::tc_fence_after();
-        constexpr uint32_t idO1 = ptx::idesc_bf16(128, 64, true, false);
+        constexpr uint32_t id1 = ptx::idesc_bf16(128, 128, false, false);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t ko = (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
+          ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_KQ + ko, 16, 1024),
+                         ptx::sdesc_sw128(sb + OFF_XP + ko, 16, 1024), id1, kk > 0);
+        }
+        ptx::umma_commit(bar(BAR_G1));
+      }
+      if (tid == kIssuer && !*sAbort) {
+        ptx::tc_fence_after();
+        constexpr uint32_t idS = ptx::idesc_bf16(128, 128, true, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::umma_bf16(tmDS, ptx::sdesc_sw128(sb + OFF_XP + 8192 + kk * 2048, 16384, 1024),
+                         ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024), idS, kk > 0);
+        constexpr uint32_t idO = ptx::idesc_bf16(128, 64, true, false);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          ptx::umma_bf16(tmBZ, ptx::sdesc_sw128(sb + OFF_SR + kk * 2048, 16384, 1024),
-                         ptx::sdesc_sw128(sb + OFF_KQ + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32, 16, 1024), idO1,
+          ptx::umma_bf16(tmO, ptx::sdesc_sw128(sb + OFF_SR + kk * 2048, 16384, 1024),
+                         ptx::sdesc_sw128(sb + OFF_KQ + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32, 16, 1024), idO,
                          kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmBZ, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
-                         ptx::sdesc_sw128(sb + OFF_QP + kk * 32, 16, 1024), idO1, 1);
-        constexpr uint32_t idO2 = ptx::idesc_bf16(128, 64, false, false);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmBZ, ptx::sdesc_sw128(sb + OFF_MT + kk * 32, 16, 1024),
-                         ptx::sdesc_sw128(sb + OFF_QX + kk * 32, 16, 1024), idO2, 1);
-        constexpr uint32_t idS1 = ptx::idesc_bf16(128, 128, true, true);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_XP + 8192 + kk * 2048, 16384, 1024),
-                         ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024), idS1, kk > 0);
-        constexpr uint32_t idS2 = ptx::idesc_bf16(128, 128, true, false);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_XP + kk * 2048, 16384, 1024),
-                         ptx::sdesc_sw128(sb + OFF_MT + kk * 32, 16, 1024), idS2, 1);
-        ptx::umma_commit(barMma);
+        ptx::umma_commit(bar(BAR_E1));
       }
-      wait_bar(barMma, mma_phase, sAbort, p.status);
-      mma_phase ^= 1u;
+      wait_bar(bar(BAR_G1), par, sAbort, p.status);
+      ptx::tc_fence_after();
+
+      // masks: A, B strictly lower (fp32 A for the solve, bf16 B); QX, QP lower incl. diagonal.
+      // warp (qd, cg) reads D1 columns [32 cg, 32 cg + 32).
+      {
+        float *Af = reinterpret_cast<float *>(gb + OFF_G);
+        uint32_t r[32];
+        ptx::tmem_ld32(tmD1 + lane_base + cg * 32, r);
+        ptx::tmem_wait_ld();
+        const int jb = (cg & 1) * 32;  // column offset inside the 64-wide matrix
+        float f[32];
+        if (qd < 2) {
+          const int i = row;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) f[j] = (jb + j < i) ? __uint_as_float(r[j]) : 0.f;
+          if (cg < 2) {
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4)
+              *reinterpret_cast<float4 *>(Af + fidx(i, jb + 4 * j4)) =
+                  make_float4(f[4 * j4], f[4 * j4 + 1], f[4 * j4 + 2], f[4 * j4 + 3]);
+          } else {
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8)
+              sts_v4(sb + OFF_BM + swz(i, (uint32_t)((cg & 1) * 4 + q8)), pack8(f + 8 * q8, 1.f));
+          }
+        } else {
+          const int i = row - 64;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) f[j] = (jb + j <= i) ? __uint_as_float(r[j]) : 0.f;
+          const uint32_t dst = cg < 2 ? OFF_QX : OFF_QP;
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8)
+            sts_v4(sb + dst + swz(i, (uint32_t)((cg & 1) * 4 + q8)), pack8(f + 8 * q8, 1.f));
+        }
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      __syncthreads();
+
+      // O^T += V^T QP^T (state-independent), overlapping the solve
+      if (tid == kIssuer && !*sAbort) {
+        ptx::tc_fence_after();
+        constexpr uint32_t idO = ptx::idesc_bf16(128, 64, true, false);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::umma_bf16(tmO, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
+                         ptx::sdesc_sw128(sb + OFF_QP + kk * 32, 16, 1024), idO, 1);
+        ptx::umma_commit(bar(BAR_E2));
+      }
+
+      if (tid == kIssuer) ptx::bulk_wait_group_read0();  // previous chunk's o store has read its staging
+      // ---- a5: T = (I + A)^-1.  16x16 diagonal blocks by forward substitution (fp32), then the
+      //      off-diagonal blocks level by level, T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ, on tf32 mma.
+      {
+        const float *Af = reinterpret_cast<const float *>(gb + OFF_G);
+        float *Tf = reinterpret_cast<float *>(gb + OFF_WT);
+        float *Xs = reinterpret_cast<float *>(gb + OFF_MT);
+        if (tid < 64) {
+          // column m of (I + A_II)^-1: top 8 rows by forward substitution, then the bottom 8 rows
+          // from rhs = e_m - A[8:16, 0:8] t[0:8] by forward substitution in the bottom 8x8 block
+          const int I = tid >> 4, m = tid & 15, r0 = 16 * I;
+          float t[16];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float acc = (i == m) ? 1.f : 0.f;
+#pragma unroll
+            for (int j = 0; j < i; ++j) acc -= Af[fidx(r0 + i, r0 + j)] * t[j];
+            t[i] = acc;
+          }
+          float rhs[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float acc = (i + 8 == m) ? 1.f : 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc -= Af[fidx(r0 + 8 + i, r0 + j)] * t[j];
+            rhs[i] = acc;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float acc = rhs[i];
+#pragma unroll
+            for (int j = 0; j < i; ++j) acc -= Af[fidx(r0 + 8 + i, r0 + 8 + j)] * t[8 + j];
+            t[8 + i] = acc;
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) Tf[fidx(r0 + i, r0 + m)] = t[i];
+        }
+        __syncthreads();
+        // Block column J depends only on itself: T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ for I = J+1 .. 3,
+        // so warp J (J < 3) walks down its column with no barrier but __syncwarp.
+        if (warp < 3) {
+          const int g = lane >> 2, t4 = lane & 3, J = warp;
+          float *xs = Xs + warp * 256;
+          for (int I = J + 1; I < 4; ++I) {
+            float x[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            for (int K = J; K < I; ++K) {
+#pragma unroll
+              for (int kk = 0; kk < 2; ++kk) {
+                const int kc = 16 * K + 8 * kk + t4;
+                const uint32_t a[4] = {ptx::to_tf32(Af[fidx(16 * I + g, kc)]),
+                                       ptx::to_tf32(Af[fidx(16 * I + g + 8, kc)]),
+                                       ptx::to_tf32(Af[fidx(16 * I + g, kc + 4)]),
+                                       ptx::to_tf32(Af[fidx(16 * I + g + 8, kc + 4)])};
+#pragma unroll
+                for (int nh = 0; nh < 2; ++nh) {
+                  const uint32_t b[2] = {ptx::to_tf32(Tf[fidx(kc, 16 * J + 8 * nh + g)]),
+                                         ptx::to_tf32(Tf[fidx(kc + 4, 16 * J + 8 * nh + g)])};
+                  ptx::mma_tf32_16x8x8(x[nh], a, b);
+                }
+              }
+            }
+#pragma unroll
+            for (int nh = 0; nh < 2; ++nh) {
+              xs[g * 16 + 8 * nh + 2 * t4] = x[nh][0];
+              xs[g * 16 + 8 * nh + 2 * t4 + 1] = x[nh][1];
+              xs[(g + 8) * 16 + 8 * nh + 2 * t4] = x[nh][2];
+              xs[(g + 8) * 16 + 8 * nh + 2 * t4 + 1] = x[nh][3];
+            }
+            __syncwarp();
+            float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              const int kc = 16 * I + 8 * kk + t4;
+              const uint32_t a[4] = {ptx::to_tf32(Tf[fidx(16 * I + g, kc)]), ptx::to_tf32(Tf[fidx(16 * I + g + 8, kc)]),
+                                     ptx::to_tf32(Tf[fidx(16 * I + g, kc + 4)]),
+                                     ptx::to_tf32(Tf[fidx(16 * I + g + 8, kc + 4)])};
+#pragma unroll
+              for (int nh = 0; nh < 2; ++nh) {
+                const uint32_t b[2] = {ptx::to_tf32(xs[(8 * kk + t4) * 16 + 8 * nh + g]),
+                                       ptx::to_tf32(xs[(8 * kk + t4 + 4) * 16 + 8 * nh + g])};
+                ptx::mma_tf32_16x8x8(y[nh], a, b);
+              }
+            }
+#pragma unroll
+            for (int nh = 0; nh < 2; ++nh) {
+              Tf[fidx(16 * I + g, 16 * J + 8 * nh + 2 * t4)] = -y[nh][0];
+              Tf[fidx(16 * I + g, 16 * J + 8 * nh + 2 * t4 + 1)] = -y[nh][1];
+              Tf[fidx(16 * I + g + 8, 16 * J + 8 * nh + 2 * t4)] = -y[nh][2];
+              Tf[fidx(16 * I + g + 8, 16 * J + 8 * nh + 2 * t4 + 1)] = -y[nh][3];
+            }
+            __syncwarp();
+          }
+        }
+        __syncthreads();
+        {
+          const int i = tid >> 3, seg = tid & 7;
+          float f[8];
+          if ((seg >> 1) > (i >> 4)) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) f[j] = 0.f;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) f[j] = Tf[fidx(i, 8 * seg + j)];
+          }
+          sts_v4(sb + OFF_T + swz(i, (uint32_t)seg), pack8(f, 1.f));
+        }
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      __syncthreads();
+
+      // ---- a6: G2  W_r^T = k_r^T T^T (D1 cols 0-63),  (B V)^T = V^T B^T (D1 cols 64-127)
+      if (tid == 0 && !*sAbort) {
+        ptx::tc_fence_after();
+        constexpr uint32_t id = ptx::idesc_bf16(128, 64, true, false);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_KQ + kk * 2048, 16384, 1024),
+                         ptx::sdesc_sw128(sb + OFF_T + kk * 32, 16, 1024), id, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::umma_bf16(tmD1 + 64, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
+                         ptx::sdesc_sw128(sb + OFF_BM + kk * 32, 16, 1024), id, kk > 0);
+        ptx::umma_commit(bar(BAR_G2));
+      }
+      wait_bar(bar(BAR_G2), par, sAbort, p.status);
+      ptx::tc_fence_after();
+      // prefetch the next chunk's k, q, v, log_a: their tiles are no longer read by any MMA
+      if (tid == kIssuer && has_next && !*sAbort) {
+        wait_bar(bar(BAR_E1), par, sAbort, p.status);
+        wait_bar(bar(BAR_E2), par, sAbort, p.status);
+        issue_tma_a(h, t0 + C);
+      }
+      {
+        const uint32_t src = tmD1 + (uint32_t)(cg >> 1) * 64u + (uint32_t)(cg & 1) * 32u;
+        const uint32_t dst = (cg < 2) ? OFF_WT : OFF_BZ;
+        uint32_t r[32];
+        ptx::tmem_ld32(src + lane_base, r);
+        ptx::tmem_wait_ld();
+        float f[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(r[j]);
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8)
+          sts_v4(sb + dst + swz(row, (uint32_t)((cg & 1) * 4 + q8)), pack8(f + 8 * q8, 1.f));
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      __syncthreads();
+
+      // ---- a7 (erase reads): G3  M^T = (B V)^T T^T + S_r^T W_r^T  (D1 cols 0-63)
+      if (tid == 0 && !*sAbort) {
+        ptx::tc_fence_after();
+        constexpr uint32_t idA = ptx::idesc_bf16(128, 64, false, false);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_BZ + kk * 32, 16, 1024),
+                         ptx::sdesc_sw128(sb + OFF_T + kk * 32, 16, 1024), idA, kk > 0);
+        constexpr uint32_t idB = ptx::idesc_bf16(128, 64, true, true);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_SR + kk * 2048, 16384, 1024),
+                         ptx::sdesc_sw128(sb + OFF_WT + kk * 2048, 16384, 1024), idB, 1);
+        ptx::umma_commit(bar(BAR_G3));
+      }
+      wait_bar(bar(BAR_G3), par, sAbort, p.status);
       ptx::tc_fence_after();
       {
-        // o^T lane = dv channel `row`, columns = tokens [32 hf, 32 hf + 32)
-        uint32_t r[32];
-        ptx::tmem_ld32(tmBZ + lane_base + hf * 32, r);
+        uint32_t r[16];
+        ptx::tmem_ld16(tmD1 + lane_base + cg * 16, r);
         ptx::tmem_wait_ld();
+        float f[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int i = hf * 32 + j;
+        for (int j = 0; j < 16; ++j) f[j] = __uint_as_float(r[j]);
+#pragma unroll
+        for (int q8 = 0; q8 < 2; ++q8) sts_v4(sb + OFF_MT + swz(row, (uint32_t)(cg * 2 + q8)), pack8(f + 8 * q8, -1.f));
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      __syncthreads();
+
+      // ---- a7: the state-dependent remainder of O^T and dS
+      if (tid == 0 && !*sAbort) {
+        ptx::tc_fence_after();
+        constexpr uint32_t idO = ptx::idesc_bf16(128, 64, false, false);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::umma_bf16(tmO, ptx::sdesc_sw128(sb + OFF_MT + kk * 32, 16, 1024),
+                         ptx::sdesc_sw128(sb + OFF_QX + kk * 32, 16, 1024), idO, 1);
+        constexpr uint32_t idS = ptx::idesc_bf16(128, 128, true, false);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::umma_bf16(tmDS, ptx::sdesc_sw128(sb + OFF_XP + kk * 2048, 16384, 1024),
+                         ptx::sdesc_sw128(sb + OFF_MT + kk * 32, 16, 1024), idS, 1);
+        ptx::umma_commit(bar(BAR_G45));
+      }
+      wait_bar(bar(BAR_G45), par, sAbort, p.status);
+      ptx::tc_fence_after();
+      if (tid == kIssuer && has_next && !*sAbort) issue_tma_b(h, t0 + C);  // x_r / p_r are dead now
+
+      // ---- a8: outputs and the state update
+      {
+        // o^T: lane = dv channel `row`, columns = tokens [16 cg, 16 cg + 16)
+        uint32_t r[16];
+        ptx::tmem_ld16(tmO + lane_base + cg * 16, r);
+        ptx::tmem_wait_ld();
+        // staging: sub-blocks of [64 tokens][128 B] (64 bf16 or 32 fp32 channels), 8 KB each
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int i = cg * 16 + j;
           const float f = __uint_as_float(r[j]);
           if (sizeof(Tout) == 2) {
             const __nv_bfloat16 hv = __float2bfloat16_rn(f);
-            sts_u16(sb + OFF_BZ + (uint32_t)i * 256u + (uint32_t)row * 2u, *reinterpret_cast<const uint16_t *>(&hv));
+            sts_u16(sb + OFF_BZ + (uint32_t)(row >> 6) * 8192u + (uint32_t)i * 128u + (uint32_t)(row & 63) * 2u,
+                    *reinterpret_cast<const uint16_t *>(&hv));
           } else {
-            sts_f32(sb + OFF_BZ + (uint32_t)i * 512u + (uint32_t)row * 4u, f);
+            sts_f32(sb + OFF_BZ + (uint32_t)(row >> 5) * 8192u + (uint32_t)i * 128u + (uint32_t)(row & 31) * 4u, f);
           }
         }
-        // S <- e^{L_C} S + e^{L_C - L_ref} dS   (thread: dk row `row`)
+        // S <- e^{L_C} S + e^{L_C - L_ref} dS   (thread: dk row `row`, columns [32 cg, +32))
         const float gc = sGC[row], dl = sDL[row];
+        uint32_t s[32], ds[32];
+        ptx::tmem_ld32(tmS + lane_base + cg * 32, s);
+        ptx::tmem_ld32(tmDS + lane_base + cg * 32, ds);
+        ptx::tmem_wait_ld();
 #pragma unroll
-        for (int h32 = 0; h32 < 2; ++h32) {
-          uint32_t s[32], ds[32];
-          ptx::tmem_ld32(tmS + lane_base + hf * 64 + h32 * 32, s);
-          ptx::tmem_ld32(tmD1 + lane_base + hf * 64 + h32 * 32, ds);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            s[j] = __float_as_uint(fmaf(gc, __uint_as_float(s[j]), dl * __uint_as_float(ds[j])));
-          ptx::tmem_st32(tmS + lane_base + hf * 64 + h32 * 32, s);
-        }
+        for (int j = 0; j < 32; ++j) s[j] = __float_as_uint(fmaf(gc, __uint_as_float(s[j]), dl * __uint_as_float(ds[j])));
+        ptx::tmem_st32(tmS + lane_base + cg * 32, s);
         ptx::tmem_wait_st();
       }
+      ptx::fence_proxy_async_smem();  // staging is read by the TMA store below
       __syncthreads();
-      {
+      if (nvalid == C) {
+        // full chunk: asynchronous TMA store; the staging area is not rewritten before the
+        // next chunk's solve, which first waits for these reads (bulk_wait_group_read0)
+        if (tid == kIssuer) {
+          constexpr int kBoxC = sizeof(Tout) == 2 ? 64 : 32;
+#pragma unroll
+          for (int sbk = 0; sbk < D / kBoxC; ++sbk)
+            ptx::tma_store_3d(&P.tm_o, sb + OFF_BZ + (uint32_t)sbk * 8192u, sbk * kBoxC, h, t0);
+          ptx::bulk_commit_group();
+        }
+      } else {
+        // tail chunk: plain stores of the valid rows only
         constexpr int kRowBytes = D * (int)sizeof(Tout);
         constexpr int kU4 = kRowBytes / 16;
         uint8_t *go = static_cast<uint8_t *>(p.o);
         for (int e = tid; e < nvalid * kU4; e += kThreads) {
           const int i = e / kU4, uu = e % kU4;
-          const uint4 val = lds_v4(sb + OFF_BZ + (uint32_t)(i * kRowBytes + uu * 16));
+          const uint4 val = lds_v4(sb + OFF_BZ + (uint32_t)(uu >> 3) * 8192u + (uint32_t)i * 128u + (uint32_t)(uu & 7) * 16u);
           *reinterpret_cast<uint4 *>(go + ((size_t)(t0 + i) * H + h) * kRowBytes + uu * 16) = val;
         }
       }
@@ -619,23 +719,20 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
 
     // ---- a8: final state
     if (p.S_T && !*sAbort) {
-      float *dst = p.S_T + ((size_t)unit * D + row) * D + hf * 64;
+      float *dst = p.S_T + ((size_t)unit * D + row) * D + cg * 32;
+      uint32_t r[32];
+      ptx::tmem_ld32(tmS + lane_base + cg * 32, r);
+      ptx::tmem_wait_ld();
 #pragma unroll
-      for (int h32 = 0; h32 < 2; ++h32) {
-        uint32_t r[32];
-        ptx::tmem_ld32(tmS + lane_base + hf * 64 + h32 * 32, r);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          reinterpret_cast<float4 *>(dst + h32 * 32)[j] =
-              make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]), __uint_as_float(r[4 * j + 2]),
-                          __uint_as_float(r[4 * j + 3]));
-      }
+      for (int j = 0; j < 8; ++j)
+        reinterpret_cast<float4 *>(dst)[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                                          __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
     }
     ptx::tc_fence_before();
     __syncthreads();
   }
 
+  if (tid == kIssuer) ptx::bulk_wait_group0();
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -669,6 +766,22 @@ bool make_map(CUtensorMap *m, const void *base, int64_t t_total, int H) {
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// o: [T_tot][H][128] of bf16 or fp32 viewed as (channel, head, token); box of 128 bytes of
+// channels x 1 head x 64 tokens, unswizzled (matches the kernel's staging sub-blocks).
+bool make_map_o(CUtensorMap *m, void *base, int64_t t_total, int H, bool bf16) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t es = bf16 ? 2 : 4;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)t_total};
+  cuuint64_t strides[2] = {(cuuint64_t)D * es, (cuuint64_t)H * D * es};
+  cuuint32_t box[3] = {bf16 ? 64u : 32u, 1, 64};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -706,6 +819,7 @@ cudaError_t launch_chunk_tc(const ChunkProblem &p, cudaStream_t stream, const ch
             make_map(&P.tm_v, p.v, T, p.n_heads);
   if (ok && !sd) ok = make_map(&P.tm_g, p.log_a, T, p.n_heads);
   if (ok && !sg) ok = make_map(&P.tm_b, p.b, T, p.n_heads) && make_map(&P.tm_w, tied ? p.b : p.w, T, p.n_heads);
+  if (ok) ok = make_map_o(&P.tm_o, p.o, T, p.n_heads, p.dtype_out == GDN2_BF16);
   if (!ok) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad tensor geometry)";
     return cudaErrorInvalidValue;
