@@ -62,9 +62,9 @@ constexpr uint32_t OFF_T = 131072;     // T bf16 [64 x 64]
 constexpr uint32_t OFF_BM = 139264;    // B bf16 [64 x 64]
 constexpr uint32_t OFF_QX = 147456;    // QX bf16 [64 x 64]
 constexpr uint32_t OFF_QP = 155648;    // QP bf16 [64 x 64]
-constexpr uint32_t OFF_WT = 163840;    // W_r^T bf16 [128 x 64]; fp32 T during the solve
-constexpr uint32_t OFF_BZ = 180224;    // (B V)^T bf16 [128 x 64]; o staging (with OFF_MT)
-constexpr uint32_t OFF_MT = 196608;    // -M^T bf16 [128 x 64]; per-warp 16x16 scratch in the solve
+constexpr uint32_t OFF_WT = 163840;    // fp32 T during the solve
+constexpr uint32_t OFF_BZ = 180224;    // R^T bf16 [128 x 64]; o staging (with OFF_MT)
+constexpr uint32_t OFF_MT = 196608;    // -M^T bf16 [128 x 64]; scratch of the solve
 constexpr uint32_t OFF_MISC = 212992;
 constexpr uint32_t MISC_GC = 0;        // float[128]  e^{L_C}
 constexpr uint32_t MISC_DL = 512;      // float[128]  e^{L_C - L_ref}
@@ -78,7 +78,7 @@ constexpr uint32_t MISC_UNIT = 10312;
 constexpr uint32_t MISC_BYTES = 10320;
 constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES + 1024;  // + base alignment slack
 // mbarrier slots
-enum { BAR_TMA_A = 0, BAR_TMA_B, BAR_G1, BAR_E1, BAR_E2, BAR_G2, BAR_G3, BAR_G45, kNumBars };
+enum { BAR_TMA_A = 0, BAR_TMA_B, BAR_G1, BAR_E1, BAR_E2, BAR_GA, BAR_GB, BAR_G45, kNumBars };
 
 struct TcParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_g, tm_b, tm_w;
@@ -88,6 +88,9 @@ struct TcParams {
   int n_units;
 };
 
+__device__ __forceinline__ void named_bar(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 __device__ __forceinline__ uint2 lds_v2(uint32_t a) {
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
@@ -173,7 +176,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   float *sSM = reinterpret_cast<float *>(gb + OFF_MISC + MISC_SM);
   float *part = reinterpret_cast<float *>(gb + OFF_MISC + MISC_PART);
   float *sRef = reinterpret_cast<float *>(gb + OFF_MISC + MISC_REF);
-  constexpr int kIssuer = 32;  // thread that issues TMA and the early MMAs (warp 1, lane 0)
+  constexpr int kIssuer = 32;      // issues the TMA loads and the output stores (warp 1, lane 0)
+  constexpr int kIssueWarp = 15;   // issues the T-independent MMAs during the solve
+  constexpr int kSolveThreads = 480;  // warps 0-14
+  enum { NB_SOLVE = 1 };
   volatile int *sAbort = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_ABORT);
   volatile int *sUnit = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_UNIT);
   auto bar = [&](int i) { return sb + OFF_MISC + MISC_BAR + 8u * (uint32_t)i; };
@@ -380,8 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       ptx::tc_fence_before();
       __syncthreads();
 
-      // ---- a4: G1 [A B; QX QP] = [k_r; q_r] [x_r; p_r]^T, then the state-independent parts of
-      //      dS (p_r^T V) and O^T (S_r^T q_r^T), which run while the CUDA cores mask and solve.
+      // ---- a4: G1 [A B; QX QP] = [k_r; q_r] [x_r; p_r]^T
       if (tid == 0 && !*sAbort) {
         ptx::tc_fence_after();
         constexpr uint32_t id1 = ptx::idesc_bf16(128, 128, false, false);
@@ -392,21 +397,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                          ptx::sdesc_sw128(sb + OFF_XP + ko, 16, 1024), id1, kk > 0);
         }
         ptx::umma_commit(bar(BAR_G1));
-      }
-      if (tid == kIssuer && !*sAbort) {
-        ptx::tc_fence_after();
-        constexpr uint32_t idS = ptx::idesc_bf16(128, 128, true, true);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmDS, ptx::sdesc_sw128(sb + OFF_XP + 8192 + kk * 2048, 16384, 1024),
-                         ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024), idS, kk > 0);
-        constexpr uint32_t idO = ptx::idesc_bf16(128, 64, true, false);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          ptx::umma_bf16(tmO, ptx::sdesc_sw128(sb + OFF_SR + kk * 2048, 16384, 1024),
-                         ptx::sdesc_sw128(sb + OFF_KQ + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32, 16, 1024), idO,
-                         kk > 0);
-        ptx::umma_commit(bar(BAR_E1));
       }
       wait_bar(bar(BAR_G1), par, sAbort, p.status);
       ptx::tc_fence_after();
@@ -448,121 +438,156 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       ptx::tc_fence_before();
       __syncthreads();
 
-      // O^T += V^T QP^T (state-independent), overlapping the solve
-      if (tid == kIssuer && !*sAbort) {
-        ptx::tc_fence_after();
-        constexpr uint32_t idO = ptx::idesc_bf16(128, 64, true, false);
+      // ---- a6 (T-independent MMAs, issued by warp 15 while warps 0-14 solve; one issuing thread
+      //      keeps them in order, and the issue stalls of a full MMA queue delay nobody):
+      //        dS = p_r^T V,  O^T = S_r^T q_r^T                                   (commit E1)
+      //        R^T = V^T B^T + S_r^T k_r^T  (D1 cols 0-63), the right-hand side of M = T R:
+      //          M = (I + A)^-1 (B V + Ytilde S) with Ytilde S = k_r S_r          (commit GA)
+      //        O^T += V^T QP^T                                                     (commit E2)
+      if (warp == kIssueWarp) {
+        if (lane == 0 && !*sAbort) {
+          ptx::tc_fence_after();
+          constexpr uint32_t idS = ptx::idesc_bf16(128, 128, true, true);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmO, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
-                         ptx::sdesc_sw128(sb + OFF_QP + kk * 32, 16, 1024), idO, 1);
-        ptx::umma_commit(bar(BAR_E2));
-      }
-
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::umma_bf16(tmDS, ptx::sdesc_sw128(sb + OFF_XP + 8192 + kk * 2048, 16384, 1024),
+                           ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024), idS, kk > 0);
+          constexpr uint32_t idO = ptx::idesc_bf16(128, 64, true, false);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            ptx::umma_bf16(tmO, ptx::sdesc_sw128(sb + OFF_SR + kk * 2048, 16384, 1024),
+                           ptx::sdesc_sw128(sb + OFF_KQ + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32, 16, 1024), idO,
+                           kk > 0);
+          ptx::umma_commit(bar(BAR_E1));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
+                           ptx::sdesc_sw128(sb + OFF_BM + kk * 32, 16, 1024), idO, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_SR + kk * 2048, 16384, 1024),
+                           ptx::sdesc_sw128(sb + OFF_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), idO, 1);
+          ptx::umma_commit(bar(BAR_GA));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::umma_bf16(tmO, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
+                           ptx::sdesc_sw128(sb + OFF_QP + kk * 32, 16, 1024), idO, 1);
+          ptx::umma_commit(bar(BAR_E2));
+        }
+        __syncwarp();
+      } else {
       if (tid == kIssuer) ptx::bulk_wait_group_read0();  // previous chunk's o store has read its staging
-      // ---- a5: T = (I + A)^-1.  16x16 diagonal blocks by forward substitution (fp32), then the
-      //      off-diagonal blocks level by level, T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ, on tf32 mma.
+
+      // ---- a5: T = (I + A)^-1 (fp32).  8x8 diagonal blocks by forward substitution, then three
+      //      merge levels: for each pair of diagonal blocks of size s (upper U, lower L) of the
+      //      merged 2s block, T_LU = -T_LL (A_LU T_UU).  Blocks above the diagonal are never
+      //      read (loops stop at the triangle), so they are never written either.
       {
         const float *Af = reinterpret_cast<const float *>(gb + OFF_G);
         float *Tf = reinterpret_cast<float *>(gb + OFF_WT);
         float *Xs = reinterpret_cast<float *>(gb + OFF_MT);
         if (tid < 64) {
-          // column m of (I + A_II)^-1: top 8 rows by forward substitution, then the bottom 8 rows
-          // from rhs = e_m - A[8:16, 0:8] t[0:8] by forward substitution in the bottom 8x8 block
-          const int I = tid >> 4, m = tid & 15, r0 = 16 * I;
-          float t[16];
+          const int r0 = 8 * (tid >> 3), m = tid & 7;
+          float a[28];
+          {
+            int n = 0;
+#pragma unroll
+            for (int i = 1; i < 8; ++i)
+#pragma unroll
+              for (int j = 0; j < i; ++j) a[n++] = Af[fidx(r0 + i, r0 + j)];
+          }
+          float t[8];
+          int n = 0;
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             float acc = (i == m) ? 1.f : 0.f;
 #pragma unroll
-            for (int j = 0; j < i; ++j) acc -= Af[fidx(r0 + i, r0 + j)] * t[j];
+            for (int j = 0; j < i; ++j) acc -= a[n++] * t[j];
             t[i] = acc;
           }
-          float rhs[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float acc = (i + 8 == m) ? 1.f : 0.f;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc -= Af[fidx(r0 + 8 + i, r0 + j)] * t[j];
-            rhs[i] = acc;
-          }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float acc = rhs[i];
-#pragma unroll
-            for (int j = 0; j < i; ++j) acc -= Af[fidx(r0 + 8 + i, r0 + 8 + j)] * t[8 + j];
-            t[8 + i] = acc;
-          }
-#pragma unroll
-          for (int i = 0; i < 16; ++i) Tf[fidx(r0 + i, r0 + m)] = t[i];
+          for (int i = 0; i < 8; ++i) Tf[fidx(r0 + i, r0 + m)] = t[i];
         }
-        __syncthreads();
-        // Block column J depends only on itself: T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ for I = J+1 .. 3,
-        // so warp J (J < 3) walks down its column with no barrier but __syncwarp.
-        if (warp < 3) {
-          const int g = lane >> 2, t4 = lane & 3, J = warp;
-          float *xs = Xs + warp * 256;
-          for (int I = J + 1; I < 4; ++I) {
-            float x[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            for (int K = J; K < I; ++K) {
+        named_bar(NB_SOLVE, kSolveThreads);
+        // s = 8: 4 pairs x 64 outputs on CUDA cores
+        if (tid < 256) {
+          const int pr = tid >> 6, r = (tid >> 3) & 7, c = tid & 7, u0 = 16 * pr, l0 = u0 + 8;
+          float acc = 0.f;
 #pragma unroll
-              for (int kk = 0; kk < 2; ++kk) {
-                const int kc = 16 * K + 8 * kk + t4;
-                const uint32_t a[4] = {ptx::to_tf32(Af[fidx(16 * I + g, kc)]),
-                                       ptx::to_tf32(Af[fidx(16 * I + g + 8, kc)]),
-                                       ptx::to_tf32(Af[fidx(16 * I + g, kc + 4)]),
-                                       ptx::to_tf32(Af[fidx(16 * I + g + 8, kc + 4)])};
-#pragma unroll
-                for (int nh = 0; nh < 2; ++nh) {
-                  const uint32_t b[2] = {ptx::to_tf32(Tf[fidx(kc, 16 * J + 8 * nh + g)]),
-                                         ptx::to_tf32(Tf[fidx(kc + 4, 16 * J + 8 * nh + g)])};
-                  ptx::mma_tf32_16x8x8(x[nh], a, b);
-                }
-              }
-            }
-#pragma unroll
-            for (int nh = 0; nh < 2; ++nh) {
-              xs[g * 16 + 8 * nh + 2 * t4] = x[nh][0];
-              xs[g * 16 + 8 * nh + 2 * t4 + 1] = x[nh][1];
-              xs[(g + 8) * 16 + 8 * nh + 2 * t4] = x[nh][2];
-              xs[(g + 8) * 16 + 8 * nh + 2 * t4 + 1] = x[nh][3];
-            }
-            __syncwarp();
-            float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-              const int kc = 16 * I + 8 * kk + t4;
-              const uint32_t a[4] = {ptx::to_tf32(Tf[fidx(16 * I + g, kc)]), ptx::to_tf32(Tf[fidx(16 * I + g + 8, kc)]),
-                                     ptx::to_tf32(Tf[fidx(16 * I + g, kc + 4)]),
-                                     ptx::to_tf32(Tf[fidx(16 * I + g + 8, kc + 4)])};
-#pragma unroll
-              for (int nh = 0; nh < 2; ++nh) {
-                const uint32_t b[2] = {ptx::to_tf32(xs[(8 * kk + t4) * 16 + 8 * nh + g]),
-                                       ptx::to_tf32(xs[(8 * kk + t4 + 4) * 16 + 8 * nh + g])};
-                ptx::mma_tf32_16x8x8(y[nh], a, b);
-              }
-            }
-#pragma unroll
-            for (int nh = 0; nh < 2; ++nh) {
-              Tf[fidx(16 * I + g, 16 * J + 8 * nh + 2 * t4)] = -y[nh][0];
-              Tf[fidx(16 * I + g, 16 * J + 8 * nh + 2 * t4 + 1)] = -y[nh][1];
-              Tf[fidx(16 * I + g + 8, 16 * J + 8 * nh + 2 * t4)] = -y[nh][2];
-              Tf[fidx(16 * I + g + 8, 16 * J + 8 * nh + 2 * t4 + 1)] = -y[nh][3];
-            }
-            __syncwarp();
-          }
+          for (int k = 0; k < 8; ++k) acc += (k >= c ? Af[fidx(l0 + r, u0 + k)] * Tf[fidx(u0 + k, u0 + c)] : 0.f);
+          Xs[tid] = acc;
         }
-        __syncthreads();
+        named_bar(NB_SOLVE, kSolveThreads);
+        if (tid < 256) {
+          const int pr = tid >> 6, r = (tid >> 3) & 7, c = tid & 7, u0 = 16 * pr, l0 = u0 + 8;
+          float acc = 0.f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc -= (k <= r ? Tf[fidx(l0 + r, l0 + k)] * Xs[pr * 64 + k * 8 + c] : 0.f);
+          Tf[fidx(l0 + r, u0 + c)] = acc;
+        }
+        named_bar(NB_SOLVE, kSolveThreads);
+        // s = 16 (2 pairs) and s = 32 (1 pair) on tf32 mma.sync: one warp per 16x8 output tile
+        const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+        for (int lev = 1; lev < 3; ++lev) {
+          const int sz = 8 << lev;                   // 16, 32
+          const int tpp = (sz / 16) * (sz / 8);      // 16x8 tiles per pair: 2, 8
+          const int ntiles = (64 / (2 * sz)) * tpp;  // 4, 8
+          // step a: X = A_LU T_UU (only k >= the tile's first column contributes)
+          if (warp < ntiles) {
+            const int pr = warp / tpp, ti = warp % tpp, mt = ti / (sz / 8), nt = ti % (sz / 8);
+            const int u0 = pr * 2 * sz, l0 = u0 + sz, rr = 16 * mt, cc = 8 * nt;
+            float x[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int kk = cc / 8; kk < sz / 8; ++kk) {
+              const int kc = u0 + 8 * kk + t4;
+              const uint32_t av[4] = {ptx::to_tf32(Af[fidx(l0 + rr + g, kc)]), ptx::to_tf32(Af[fidx(l0 + rr + g + 8, kc)]),
+                                      ptx::to_tf32(Af[fidx(l0 + rr + g, kc + 4)]),
+                                      ptx::to_tf32(Af[fidx(l0 + rr + g + 8, kc + 4)])};
+              const uint32_t bv[2] = {ptx::to_tf32(Tf[fidx(kc, u0 + cc + g)]), ptx::to_tf32(Tf[fidx(kc + 4, u0 + cc + g)])};
+              ptx::mma_tf32_16x8x8(x, av, bv);
+            }
+            float *xs = Xs + pr * sz * sz;
+            xs[(rr + g) * sz + cc + 2 * t4] = x[0];
+            xs[(rr + g) * sz + cc + 2 * t4 + 1] = x[1];
+            xs[(rr + g + 8) * sz + cc + 2 * t4] = x[2];
+            xs[(rr + g + 8) * sz + cc + 2 * t4 + 1] = x[3];
+          }
+          named_bar(NB_SOLVE, kSolveThreads);
+          // step b: T_LU = -T_LL X (only k <= the tile's last row contributes)
+          if (warp < ntiles) {
+            const int pr = warp / tpp, ti = warp % tpp, mt = ti / (sz / 8), nt = ti % (sz / 8);
+            const int u0 = pr * 2 * sz, l0 = u0 + sz, rr = 16 * mt, cc = 8 * nt;
+            const float *xs = Xs + pr * sz * sz;
+            float y[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int kk = 0; kk <= (rr + 15) / 8; ++kk) {
+              // T_LL is lower triangular; its 8x8 blocks above the diagonal were never written
+              const int kc = l0 + 8 * kk + t4, kr = 8 * kk + t4;
+              const uint32_t av[4] = {
+                  ptx::to_tf32(kr <= rr + g ? Tf[fidx(l0 + rr + g, kc)] : 0.f),
+                  ptx::to_tf32(kr <= rr + g + 8 ? Tf[fidx(l0 + rr + g + 8, kc)] : 0.f),
+                  ptx::to_tf32(kr + 4 <= rr + g ? Tf[fidx(l0 + rr + g, kc + 4)] : 0.f),
+                  ptx::to_tf32(kr + 4 <= rr + g + 8 ? Tf[fidx(l0 + rr + g + 8, kc + 4)] : 0.f)};
+              const uint32_t bv[2] = {ptx::to_tf32(xs[(8 * kk + t4) * sz + cc + g]),
+                                      ptx::to_tf32(xs[(8 * kk + t4 + 4) * sz + cc + g])};
+              ptx::mma_tf32_16x8x8(y, av, bv);
+            }
+            Tf[fidx(l0 + rr + g, u0 + cc + 2 * t4)] = -y[0];
+            Tf[fidx(l0 + rr + g, u0 + cc + 2 * t4 + 1)] = -y[1];
+            Tf[fidx(l0 + rr + g + 8, u0 + cc + 2 * t4)] = -y[2];
+            Tf[fidx(l0 + rr + g + 8, u0 + cc + 2 * t4 + 1)] = -y[3];
+          }
+          named_bar(NB_SOLVE, kSolveThreads);
+        }
+        }  // solve scope
+      }  // warps 0-14
+      __syncthreads();
+      {
+        const float *Tf = reinterpret_cast<const float *>(gb + OFF_WT);
         {
           const int i = tid >> 3, seg = tid & 7;
           float f[8];
-          if ((seg >> 1) > (i >> 4)) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) f[j] = 0.f;
-          } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) f[j] = Tf[fidx(i, 8 * seg + j)];
-          }
+          for (int j = 0; j < 8; ++j) f[j] = (8 * seg + j <= i) ? Tf[fidx(i, 8 * seg + j)] : 0.f;
           sts_v4(sb + OFF_T + swz(i, (uint32_t)seg), pack8(f, 1.f));
         }
       }
@@ -570,65 +595,43 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       ptx::tc_fence_before();
       __syncthreads();
 
-      // ---- a6: G2  W_r^T = k_r^T T^T (D1 cols 0-63),  (B V)^T = V^T B^T (D1 cols 64-127)
-      if (tid == 0 && !*sAbort) {
-        ptx::tc_fence_after();
-        constexpr uint32_t id = ptx::idesc_bf16(128, 64, true, false);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_KQ + kk * 2048, 16384, 1024),
-                         ptx::sdesc_sw128(sb + OFF_T + kk * 32, 16, 1024), id, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmD1 + 64, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
-                         ptx::sdesc_sw128(sb + OFF_BM + kk * 32, 16, 1024), id, kk > 0);
-        ptx::umma_commit(bar(BAR_G2));
-      }
-      wait_bar(bar(BAR_G2), par, sAbort, p.status);
+      // ---- round trip of R^T (-> Rt, K-major [dv rows][64 tokens])
+      wait_bar(bar(BAR_GA), par, sAbort, p.status);
       ptx::tc_fence_after();
-      // prefetch the next chunk's k, q, v, log_a: their tiles are no longer read by any MMA
+      // the next chunk's k, q, v, log_a tiles can land once no MMA reads them
       if (tid == kIssuer && has_next && !*sAbort) {
-        wait_bar(bar(BAR_E1), par, sAbort, p.status);
-        wait_bar(bar(BAR_E2), par, sAbort, p.status);
+        wait_bar(bar(BAR_E2), par, sAbort, p.status);  // E1, GA and E2 share one issuing thread
         issue_tma_a(h, t0 + C);
       }
       {
-        const uint32_t src = tmD1 + (uint32_t)(cg >> 1) * 64u + (uint32_t)(cg & 1) * 32u;
-        const uint32_t dst = (cg < 2) ? OFF_WT : OFF_BZ;
-        uint32_t r[32];
-        ptx::tmem_ld32(src + lane_base, r);
+        uint32_t r[16];
+        ptx::tmem_ld16(tmD1 + lane_base + cg * 16, r);
         ptx::tmem_wait_ld();
-        float f[32];
+        float f[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(r[j]);
+        for (int j = 0; j < 16; ++j) f[j] = __uint_as_float(r[j]);
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8)
-          sts_v4(sb + dst + swz(row, (uint32_t)((cg & 1) * 4 + q8)), pack8(f + 8 * q8, 1.f));
+        for (int q8 = 0; q8 < 2; ++q8) sts_v4(sb + OFF_BZ + swz(row, (uint32_t)(cg * 2 + q8)), pack8(f + 8 * q8, 1.f));
       }
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncthreads();
 
-      // ---- a7 (erase reads): G3  M^T = (B V)^T T^T + S_r^T W_r^T  (D1 cols 0-63)
+      // ---- a7 (erase reads): M^T = R^T T^T (D1 cols 64-127); row i of M is r_i = Sbar_i^T k_i
       if (tid == 0 && !*sAbort) {
         ptx::tc_fence_after();
-        constexpr uint32_t idA = ptx::idesc_bf16(128, 64, false, false);
+        constexpr uint32_t idM = ptx::idesc_bf16(128, 64, false, false);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_BZ + kk * 32, 16, 1024),
-                         ptx::sdesc_sw128(sb + OFF_T + kk * 32, 16, 1024), idA, kk > 0);
-        constexpr uint32_t idB = ptx::idesc_bf16(128, 64, true, true);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_SR + kk * 2048, 16384, 1024),
-                         ptx::sdesc_sw128(sb + OFF_WT + kk * 2048, 16384, 1024), idB, 1);
-        ptx::umma_commit(bar(BAR_G3));
+          ptx::umma_bf16(tmD1 + 64, ptx::sdesc_sw128(sb + OFF_BZ + kk * 32, 16, 1024),
+                         ptx::sdesc_sw128(sb + OFF_T + kk * 32, 16, 1024), idM, kk > 0);
+        ptx::umma_commit(bar(BAR_GB));
       }
-      wait_bar(bar(BAR_G3), par, sAbort, p.status);
+      wait_bar(bar(BAR_GB), par, sAbort, p.status);
       ptx::tc_fence_after();
       {
         uint32_t r[16];
-        ptx::tmem_ld16(tmD1 + lane_base + cg * 16, r);
+        ptx::tmem_ld16(tmD1 + 64 + lane_base + cg * 16, r);
         ptx::tmem_wait_ld();
         float f[16];
 #pragma unroll
@@ -642,6 +645,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
 
       // ---- a7: the state-dependent remainder of O^T and dS
       if (tid == 0 && !*sAbort) {
+        // O^T was last accumulated by the other issuing thread: keep the accumulation order fixed
+        wait_bar(bar(BAR_E2), par, sAbort, p.status);
         ptx::tc_fence_after();
         constexpr uint32_t idO = ptx::idesc_bf16(128, 64, false, false);
 #pragma unroll
