@@ -56,29 +56,31 @@ constexpr float kLog2eF = 1.4426950408889634f;
 constexpr uint32_t OFF_KQ = 0;         // 2 K-blocks x [k_r rows 0-63 | q_r rows 0-63], 16 KB each
 constexpr uint32_t OFF_XP = 32768;     // 2 K-blocks x [x_r rows | p_r rows]
 constexpr uint32_t OFF_V = 65536;      // 2 column blocks x [64 rows], 8 KB each
-constexpr uint32_t OFF_G = 81920;      // raw log_a tile; fp32 A during the solve
+constexpr uint32_t OFF_G = 81920;      // raw log_a tile
 constexpr uint32_t OFF_SR = 98304;     // S_r bf16: 2 dv-blocks x [128 dk rows], 16 KB each
 constexpr uint32_t OFF_T = 131072;     // T bf16 [64 x 64]
 constexpr uint32_t OFF_BM = 139264;    // B bf16 [64 x 64]
 constexpr uint32_t OFF_QX = 147456;    // QX bf16 [64 x 64]
 constexpr uint32_t OFF_QP = 155648;    // QP bf16 [64 x 64]
-constexpr uint32_t OFF_WT = 163840;    // fp32 T during the solve
-constexpr uint32_t OFF_BZ = 180224;    // R^T bf16 [128 x 64]; o staging (with OFF_MT)
-constexpr uint32_t OFF_MT = 196608;    // -M^T bf16 [128 x 64]; scratch of the solve
+constexpr uint32_t OFF_AF = 163840;    // fp32 A [64 x 68] (masks -> solve)
+constexpr uint32_t OFF_TF = 181248;    // fp32 T [64 x 68] (solve)
+constexpr uint32_t OFF_XS = 198656;    // fp32 solve scratch, <= 4 KB
+constexpr uint32_t OFF_BZ = 180224;    // R^T bf16 [128 x 64] and o staging (after the solve; overlaps A/T)
+constexpr uint32_t OFF_MT = 196608;    // -M^T bf16 [128 x 64] (after the solve)
 constexpr uint32_t OFF_MISC = 212992;
 constexpr uint32_t MISC_GC = 0;        // float[128]  e^{L_C}
 constexpr uint32_t MISC_DL = 512;      // float[128]  e^{L_C - L_ref}
 constexpr uint32_t MISC_SM = 1024;     // float[128]  e^{L_ref}
 constexpr uint32_t MISC_PART = 1536;   // float[16][128] 4-row sums of log_a, then exclusive prefixes
 constexpr uint32_t MISC_REF = 9728;    // float[128]  L_ref
-constexpr uint32_t MISC_BAR = 10240;   // 8 mbarriers
-constexpr uint32_t MISC_TMEM = 10304;
-constexpr uint32_t MISC_ABORT = 10308;
-constexpr uint32_t MISC_UNIT = 10312;
-constexpr uint32_t MISC_BYTES = 10320;
+constexpr uint32_t MISC_BAR = 10240;   // 9 mbarriers
+constexpr uint32_t MISC_TMEM = 10320;
+constexpr uint32_t MISC_ABORT = 10324;
+constexpr uint32_t MISC_UNIT = 10328;
+constexpr uint32_t MISC_BYTES = 10336;
 constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES + 1024;  // + base alignment slack
 // mbarrier slots
-enum { BAR_TMA_A = 0, BAR_TMA_B, BAR_G1, BAR_E1, BAR_E2, BAR_GA, BAR_GB, BAR_G45, kNumBars };
+enum { BAR_TMA_A = 0, BAR_TMA_W, BAR_TMA_X, BAR_G1, BAR_E1, BAR_E2, BAR_GA, BAR_GB, BAR_G45, kNumBars };
 
 struct TcParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_g, tm_b, tm_w;
@@ -115,8 +117,8 @@ __device__ __forceinline__ uint4 lds_v4(uint32_t a) {
   return v;
 }
 
-// fp32 64x64 scratch with a 16-byte-chunk XOR swizzle (conflict-free row writes).
-__device__ __forceinline__ int fidx(int i, int j) { return i * 64 + ((((j >> 2) ^ (i & 7))) << 2) + (j & 3); }
+// fp32 64x64 scratch, rows padded to 68 floats (272 B): conflict-free float4 row writes.
+__device__ __forceinline__ int fidx(int i, int j) { return i * 68 + j; }
 
 // Byte offset of (row r, 16-byte chunk `chunk`) in a 128B-swizzled tile.
 __device__ __forceinline__ uint32_t swz(int r, uint32_t chunk) {
@@ -223,14 +225,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       if (!kScalarDecay) ptx::tma_load_3d(sb + OFF_G + kb * 8192, &P.tm_g, kb * 64, h, t0, bar(BAR_TMA_A));
     }
   };
-  auto issue_tma_b = [&](int h, int t0) {
+  // w lands in the p_r halves of XP (free once dS = p_r^T V is done), b in the x_r halves
+  // (free once the last GEMM of the chunk is done)
+  auto issue_tma_w = [&](int h, int t0) {
     if (kScalarGates) return;
-    ptx::mbar_arrive_expect_tx(bar(BAR_TMA_B), 2u * 2u * 8192u);
+    ptx::mbar_arrive_expect_tx(bar(BAR_TMA_W), 2u * 8192u);
 #pragma unroll
-    for (int kb = 0; kb < 2; ++kb) {
-      ptx::tma_load_3d(sb + OFF_XP + kb * 16384, &P.tm_b, kb * 64, h, t0, bar(BAR_TMA_B));
-      ptx::tma_load_3d(sb + OFF_XP + kb * 16384 + 8192, &P.tm_w, kb * 64, h, t0, bar(BAR_TMA_B));
-    }
+    for (int kb = 0; kb < 2; ++kb)
+      ptx::tma_load_3d(sb + OFF_XP + kb * 16384 + 8192, &P.tm_w, kb * 64, h, t0, bar(BAR_TMA_W));
+  };
+  auto issue_tma_x = [&](int h, int t0) {
+    if (kScalarGates) return;
+    ptx::mbar_arrive_expect_tx(bar(BAR_TMA_X), 2u * 8192u);
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb)
+      ptx::tma_load_3d(sb + OFF_XP + kb * 16384, &P.tm_b, kb * 64, h, t0, bar(BAR_TMA_X));
   };
 
   for (;;) {
@@ -251,7 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     const int nchunks = (int)((len + C - 1) / C);
     if (tid == kIssuer && nchunks > 0 && !*sAbort) {
       issue_tma_a(h, (int)bos);
-      issue_tma_b(h, (int)bos);
+      issue_tma_w(h, (int)bos);
+      issue_tma_x(h, (int)bos);
     }
 
     // ---- initial state into TMEM (thread: dk row `row`, dv columns [32 cg, 32 cg + 32))
@@ -282,8 +292,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       const int t0 = (int)(bos + c0);
       const bool has_next = ci + 1 < nchunks;
 
+      if (tid == kIssuer) ptx::bulk_wait_group_read0();  // previous chunk's o store has read its staging
       wait_bar(bar(BAR_TMA_A), par, sAbort, p.status);
-      if (!kScalarGates) wait_bar(bar(BAR_TMA_B), par, sAbort, p.status);
+      if (!kScalarGates) wait_bar(bar(BAR_TMA_W), par, sAbort, p.status);
 
       // ---- a2/a3: cumulative log-decay and scaled operands, in place.
       // thread: channels 4 cq .. 4 cq + 3, rows 4 warp .. 4 warp + 3.
@@ -328,6 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         const float4 ref = *reinterpret_cast<const float4 *>(sRef + 4 * cq);
         const float4 base = make_float4((off.x - ref.x) * kLog2eF, (off.y - ref.y) * kLog2eF,
                                         (off.z - ref.z) * kLog2eF, (off.w - ref.w) * kLog2eF);
+        float4 kraw[4], e2v[4];
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr) {
           const int r = warp * 4 + rr;
@@ -335,35 +347,49 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           const float l0 = fmaf(L[rr].x, kLog2eF, base.x), l1 = fmaf(L[rr].y, kLog2eF, base.y);
           const float l2 = fmaf(L[rr].z, kLog2eF, base.z), l3 = fmaf(L[rr].w, kLog2eF, base.w);
           const float e10 = ptx::ex2(l0), e11 = ptx::ex2(l1), e12 = ptx::ex2(l2), e13 = ptx::ex2(l3);
-          const float e20 = ptx::ex2(-l0), e21 = ptx::ex2(-l1), e22 = ptx::ex2(-l2), e23 = ptx::ex2(-l3);
+          e2v[rr] = make_float4(ptx::ex2(-l0), ptx::ex2(-l1), ptx::ex2(-l2), ptx::ex2(-l3));
           float4 kk = unpack4(lds_v2(sb + OFF_KQ + o));
           float4 qq = unpack4(lds_v2(sb + OFF_KQ + o + 8192));
-          float4 bb, ww;
+          float4 ww;
           if (kScalarGates) {
-            bb = make_float4(0.f, 0.f, 0.f, 0.f);
-            ww = bb;
+            ww = make_float4(0.f, 0.f, 0.f, 0.f);
             if (r < nvalid) {
-              const float sbv = __bfloat162float(g_b[(size_t)(t0 + r) * H + h]);
               const float swv = __bfloat162float(g_w[(size_t)(t0 + r) * H + h]);
-              bb = make_float4(sbv, sbv, sbv, sbv);
               ww = make_float4(swv, swv, swv, swv);
             }
           } else {
-            bb = unpack4(lds_v2(sb + OFF_XP + o));
             ww = unpack4(lds_v2(sb + OFF_XP + o + 8192));
           }
           if (r >= nvalid) {
             kk = make_float4(0.f, 0.f, 0.f, 0.f);
             qq = kk;
-            bb = kk;
             ww = kk;
             sts_v2(sb + OFF_V + kb * 8192 + swz(r, ch16) + cofs, make_uint2(0u, 0u));
           }
+          kraw[rr] = kk;
+          const float4 e2 = e2v[rr];
           sts_v2(sb + OFF_KQ + o, pack4(kk.x * e10, kk.y * e11, kk.z * e12, kk.w * e13));
           sts_v2(sb + OFF_KQ + o + 8192, pack4(qq.x * e10, qq.y * e11, qq.z * e12, qq.w * e13));
-          sts_v2(sb + OFF_XP + o, pack4(bb.x * kk.x * e20, bb.y * kk.y * e21, bb.z * kk.z * e22, bb.w * kk.w * e23));
-          sts_v2(sb + OFF_XP + o + 8192,
-                 pack4(ww.x * kk.x * e20, ww.y * kk.y * e21, ww.z * kk.z * e22, ww.w * kk.w * e23));
+          sts_v2(sb + OFF_XP + o + 8192, pack4(ww.x * kk.x * e2.x, ww.y * kk.y * e2.y, ww.z * kk.z * e2.z, ww.w * kk.w * e2.w));
+        }
+        // x_r = b.k e^{L_ref - L}: b lands last
+        if (!kScalarGates) wait_bar(bar(BAR_TMA_X), par, sAbort, p.status);
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          const int r = warp * 4 + rr;
+          const uint32_t o = (uint32_t)kb * 16384u + swz(r, ch16) + cofs;
+          float4 bb;
+          if (kScalarGates) {
+            bb = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r < nvalid) {
+              const float sbv = __bfloat162float(g_b[(size_t)(t0 + r) * H + h]);
+              bb = make_float4(sbv, sbv, sbv, sbv);
+            }
+          } else {
+            bb = unpack4(lds_v2(sb + OFF_XP + o));
+          }
+          const float4 kk = kraw[rr], e2 = e2v[rr];
+          sts_v2(sb + OFF_XP + o, pack4(bb.x * kk.x * e2.x, bb.y * kk.y * e2.y, bb.z * kk.z * e2.z, bb.w * kk.w * e2.w));
         }
       }
       __syncthreads();
@@ -404,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       // masks: A, B strictly lower (fp32 A for the solve, bf16 B); QX, QP lower incl. diagonal.
       // warp (qd, cg) reads D1 columns [32 cg, 32 cg + 32).
       {
-        float *Af = reinterpret_cast<float *>(gb + OFF_G);
+        float *Af = reinterpret_cast<float *>(gb + OFF_AF);
         uint32_t r[32];
         ptx::tmem_ld32(tmD1 + lane_base + cg * 32, r);
         ptx::tmem_wait_ld();
@@ -473,19 +499,22 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             ptx::umma_bf16(tmO, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
                            ptx::sdesc_sw128(sb + OFF_QP + kk * 32, 16, 1024), idO, 1);
           ptx::umma_commit(bar(BAR_E2));
+          if (has_next) {  // p_r is dead once dS = p_r^T V is done: the next chunk's w can land
+            wait_bar(bar(BAR_E1), par, sAbort, p.status);
+            if (!*sAbort) issue_tma_w(h, t0 + C);
+          }
         }
         __syncwarp();
       } else {
-      if (tid == kIssuer) ptx::bulk_wait_group_read0();  // previous chunk's o store has read its staging
 
       // ---- a5: T = (I + A)^-1 (fp32).  8x8 diagonal blocks by forward substitution, then three
       //      merge levels: for each pair of diagonal blocks of size s (upper U, lower L) of the
       //      merged 2s block, T_LU = -T_LL (A_LU T_UU).  Blocks above the diagonal are never
       //      read (loops stop at the triangle), so they are never written either.
       {
-        const float *Af = reinterpret_cast<const float *>(gb + OFF_G);
-        float *Tf = reinterpret_cast<float *>(gb + OFF_WT);
-        float *Xs = reinterpret_cast<float *>(gb + OFF_MT);
+        const float *Af = reinterpret_cast<const float *>(gb + OFF_AF);
+        float *Tf = reinterpret_cast<float *>(gb + OFF_TF);
+        float *Xs = reinterpret_cast<float *>(gb + OFF_XS);
         if (tid < 64) {
           const int r0 = 8 * (tid >> 3), m = tid & 7;
           float a[28];
@@ -578,19 +607,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           }
           named_bar(NB_SOLVE, kSolveThreads);
         }
-        }  // solve scope
-      }  // warps 0-14
-      __syncthreads();
-      {
-        const float *Tf = reinterpret_cast<const float *>(gb + OFF_WT);
-        {
-          const int i = tid >> 3, seg = tid & 7;
+        // T -> bf16 tile (zeros above the diagonal), by the solve warps
+        for (int e = tid; e < 512; e += kSolveThreads) {
+          const int i = e >> 3, seg = e & 7;
           float f[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) f[j] = (8 * seg + j <= i) ? Tf[fidx(i, 8 * seg + j)] : 0.f;
           sts_v4(sb + OFF_T + swz(i, (uint32_t)seg), pack8(f, 1.f));
         }
-      }
+        }  // solve scope
+      }  // warps 0-14
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncthreads();
@@ -662,7 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       }
       wait_bar(bar(BAR_G45), par, sAbort, p.status);
       ptx::tc_fence_after();
-      if (tid == kIssuer && has_next && !*sAbort) issue_tma_b(h, t0 + C);  // x_r / p_r are dead now
+      if (tid == kIssuer && has_next && !*sAbort) issue_tma_x(h, t0 + C);  // x_r is dead now
 
       // ---- a8: outputs and the state update
       {
