@@ -42,7 +42,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "prefill tokens/s (GDN-2 fwd, 16h×128d, T=4k); decode tok/s, % HBM BW"
 WORKLOAD = "gdn2_b8_t4k"
-FLOP_PER_TOKHEAD = 10 * 64 * 128 + 8 * 64 * 128 + 8 * 128 * 128  # GEMMs the chunk kernel issues (C=64, d=128)
+# tcgen05 GEMMs the chunk kernel issues per token-head (C=64, d=128):
+# G1 8*C*dk + R 2*C*dv + 2*dk*dv + M 2*C*dv + O 2*dk*dv + 4*C*dv + dS 4*dk*dv
+FLOP_PER_TOKHEAD = 8 * 64 * 128 + 8 * 64 * 128 + 8 * 128 * 128
 BYTES_PER_TOKHEAD = 6 * 128 * 2 + 128 * 2                      # six bf16 inputs + bf16 o
 STATE_BYTES = 128 * 128 * 4                                    # one fp32 state
 
