@@ -48,8 +48,10 @@ int check_dims(const gdn2_dims *d) {
   if ((d->dtype_in != GDN2_BF16 && d->dtype_in != GDN2_F32) || (d->dtype_out != GDN2_BF16 && d->dtype_out != GDN2_F32))
     return fail(GDN2_ERR_INVALID_ARG, "bad dtype_in=%d / dtype_out=%d", d->dtype_in, d->dtype_out);
   if (d->flags & ~kKnownFlags) return fail(GDN2_ERR_INVALID_ARG, "unknown flag bits 0x%x", d->flags & ~kKnownFlags);
-  if (d->flags & GDN2_GATE_FORM_P3)
-    return fail(GDN2_ERR_UNSUPPORTED, "GDN2_GATE_FORM_P3 is reserved and has no kernel in this build");
+  if ((d->flags & GDN2_GATE_FORM_P3) && (d->flags & GDN2_TIED_GATES) && !(d->flags & GDN2_SCALAR_GATES) &&
+      d->d_k != d->d_v)
+    return fail(GDN2_ERR_INVALID_ARG, "tied per-channel gates in the GDN2_GATE_FORM_P3 form need d_k == d_v "
+                "(b has d_k channels, w has d_v)");
   return GDN2_OK;
 }
 

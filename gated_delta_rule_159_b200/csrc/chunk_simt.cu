@@ -4,12 +4,14 @@
 // Same chunk algebra as the tensor-core path (alanhou.org "Core Mechanism": a
 // chunkwise WY form; gist.science Methodologie 3: a lower-triangular solve
 // gives the erase-side auxiliaries), written for one chunk of rows i, j < n
-// starting from state S, with x = b.k, p = w.k and L = the inclusive cumulative
-// log-decay inside the chunk:
+// starting from state S, with y the erase read vector, x the erase outer
+// factor, p the write outer factor, V the written values (k, b.k, w.k, v by
+// default; b.k, k, k, w.v in the gist.science form) and L the inclusive
+// cumulative log-decay inside the chunk:
 //
-//   A_ij  = sum_c k_ic x_jc e^{L_ic - L_jc}   (j < i)     B_ij  = same with p
+//   A_ij  = sum_c y_ic x_jc e^{L_ic - L_jc}   (j < i)     B_ij  = same with p
 //   QX_ij = sum_c q_ic x_jc e^{L_ic - L_jc}   (j <= i)    QP_ij = same with p
-//   M     = (I + A)^-1 (Ytilde S + B V),      Ytilde_ic = k_ic e^{L_ic}
+//   M     = (I + A)^-1 (Ytilde S + B V),      Ytilde_ic = y_ic e^{L_ic}
 //   O     = Qtilde S + QP V - QX M,           Qtilde_ic = q_ic e^{L_ic}
 //   S'    = Diag(e^{L_C}) S + sum_j Diag(e^{L_C - L_j}) (p_j v_j^T - x_j M_j^T)
 //
@@ -34,6 +36,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkProblem p) {
   const bool scalar_decay = (p.flags & GDN2_SCALAR_DECAY) != 0;
   const bool scalar_gates = (p.flags & GDN2_SCALAR_GATES) != 0;
   const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
+  const bool p3 = (p.flags & GDN2_GATE_FORM_P3) != 0;
 
   int64_t bos, len;
   if (p.cu_seqlens) {
@@ -84,17 +87,26 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkProblem p) {
         kk = to_f32(gk[ik]);
         g = to_f32(scalar_decay ? ga[is] : ga[ik]);
         bb = to_f32(scalar_gates ? gb[is] : gb[ik]);
-        ww = to_f32(scalar_gates ? gw[is] : gw[ik]);
+        if (!p3) ww = to_f32(scalar_gates ? gw[is] : gw[ik]);
       }
+      // sk: erase read vector, sx: erase outer factor, sp: write outer factor.
+      // Default form (k, b.k, w.k); gist.science form (b.k, k, k), whose write
+      // gate scales the values below instead.
       sq[e] = qq;
-      sk[e] = kk;
-      sx[e] = bb * kk;
-      sp[e] = ww * kk;
+      sk[e] = p3 ? bb * kk : kk;
+      sx[e] = p3 ? kk : bb * kk;
+      sp[e] = p3 ? kk : ww * kk;
       sF[e] = g;
     }
     for (int e = tid; e < C * dv; e += kThreads) {
       const int r = e / dv, c = e % dv;
-      sv[e] = r < nr ? to_f32(gv[((size_t)(bos + c0 + r) * H + h) * dv + c]) : 0.f;
+      float vv = 0.f;
+      if (r < nr) {
+        const int64_t tok = bos + c0 + r;
+        vv = to_f32(gv[((size_t)tok * H + h) * dv + c]);
+        if (p3) vv *= to_f32(scalar_gates ? gw[(size_t)tok * H + h] : gw[((size_t)tok * H + h) * dv + c]);
+      }
+      sv[e] = vv;
     }
     __syncthreads();
     // 2. inclusive cumulative log-decay per channel
@@ -126,13 +138,14 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkProblem p) {
       sQP[e] = qp;
     }
     __syncthreads();
-    // decay factors relative to the chunk start (e^{L}) and to its end (e^{L_C - L})
+    // decay factors relative to the chunk end (e^{L_C - L}) and to its start (e^{L});
+    // two passes, since every row reads the last row's L_C before sL is overwritten
     for (int e = tid; e < C * dk; e += kThreads) {
       const int c = e % dk;
-      const float L = sL[e], LC = sL[(C - 1) * dk + c];
-      sF[e] = exp_fast(LC - L);
-      sL[e] = exp_fast(L);
+      sF[e] = exp_fast(sL[(C - 1) * dk + c] - sL[e]);
     }
+    __syncthreads();
+    for (int e = tid; e < C * dk; e += kThreads) sL[e] = exp_fast(sL[e]);
     __syncthreads();
     // 4. right-hand side Ytilde S + B V
     for (int e = tid; e < C * dv; e += kThreads) {

@@ -160,7 +160,11 @@ __device__ __forceinline__ uint2 pack4(float a, float b, float c, float d) {
   return make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
 }
 
-template <bool kScalarDecay, bool kScalarGates, typename Tout>
+// kP3: the gist.science gate placement.  The operands are then k_r = (b.k) e^{L - L_ref}
+// (erase read), x_r = p_r = k e^{L_ref - L} (erase and write outer factors) and the
+// values w.v; the host swaps the gate tensor maps so that the gate needed first (b)
+// arrives with the TMA_W group and w with the TMA_X group.
+template <bool kScalarDecay, bool kScalarGates, bool kP3, typename Tout>
 __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_constant__ TcParams P) {
   extern __shared__ uint8_t smem_raw[];
   const ChunkProblem &p = P.p;
@@ -350,11 +354,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           e2v[rr] = make_float4(ptx::ex2(-l0), ptx::ex2(-l1), ptx::ex2(-l2), ptx::ex2(-l3));
           float4 kk = unpack4(lds_v2(sb + OFF_KQ + o));
           float4 qq = unpack4(lds_v2(sb + OFF_KQ + o + 8192));
-          float4 ww;
+          float4 ww;  // the write gate w (the erase gate b in the gist.science form)
           if (kScalarGates) {
             ww = make_float4(0.f, 0.f, 0.f, 0.f);
             if (r < nvalid) {
-              const float swv = __bfloat162float(g_w[(size_t)(t0 + r) * H + h]);
+              const float swv = __bfloat162float((kP3 ? g_b : g_w)[(size_t)(t0 + r) * H + h]);
               ww = make_float4(swv, swv, swv, swv);
             }
           } else {
@@ -368,9 +372,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           }
           kraw[rr] = kk;
           const float4 e2 = e2v[rr];
-          sts_v2(sb + OFF_KQ + o, pack4(kk.x * e10, kk.y * e11, kk.z * e12, kk.w * e13));
+          if (kP3) {
+            sts_v2(sb + OFF_KQ + o, pack4(ww.x * kk.x * e10, ww.y * kk.y * e11, ww.z * kk.z * e12, ww.w * kk.w * e13));
+            sts_v2(sb + OFF_XP + o + 8192, pack4(kk.x * e2.x, kk.y * e2.y, kk.z * e2.z, kk.w * e2.w));
+          } else {
+            sts_v2(sb + OFF_KQ + o, pack4(kk.x * e10, kk.y * e11, kk.z * e12, kk.w * e13));
+            sts_v2(sb + OFF_XP + o + 8192, pack4(ww.x * kk.x * e2.x, ww.y * kk.y * e2.y, ww.z * kk.z * e2.z, ww.w * kk.w * e2.w));
+          }
           sts_v2(sb + OFF_KQ + o + 8192, pack4(qq.x * e10, qq.y * e11, qq.z * e12, qq.w * e13));
-          sts_v2(sb + OFF_XP + o + 8192, pack4(ww.x * kk.x * e2.x, ww.y * kk.y * e2.y, ww.z * kk.z * e2.z, ww.w * kk.w * e2.w));
         }
         // x_r = b.k e^{L_ref - L}: b lands last
         if (!kScalarGates) wait_bar(bar(BAR_TMA_X), par, sAbort, p.status);
@@ -378,18 +387,27 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         for (int rr = 0; rr < 4; ++rr) {
           const int r = warp * 4 + rr;
           const uint32_t o = (uint32_t)kb * 16384u + swz(r, ch16) + cofs;
-          float4 bb;
+          float4 bb;  // the erase gate b (the value gate w in the gist.science form)
           if (kScalarGates) {
             bb = make_float4(0.f, 0.f, 0.f, 0.f);
             if (r < nvalid) {
-              const float sbv = __bfloat162float(g_b[(size_t)(t0 + r) * H + h]);
+              const float sbv = __bfloat162float((kP3 ? g_w : g_b)[(size_t)(t0 + r) * H + h]);
               bb = make_float4(sbv, sbv, sbv, sbv);
             }
           } else {
             bb = unpack4(lds_v2(sb + OFF_XP + o));
           }
           const float4 kk = kraw[rr], e2 = e2v[rr];
-          sts_v2(sb + OFF_XP + o, pack4(bb.x * kk.x * e2.x, bb.y * kk.y * e2.y, bb.z * kk.z * e2.z, bb.w * kk.w * e2.w));
+          if (kP3) {
+            sts_v2(sb + OFF_XP + o, pack4(kk.x * e2.x, kk.y * e2.y, kk.z * e2.z, kk.w * e2.w));
+            if (r < nvalid) {  // rows past the chunk end were zeroed above
+              const uint32_t ov = sb + OFF_V + (uint32_t)kb * 8192u + swz(r, ch16) + cofs;
+              const float4 vv = unpack4(lds_v2(ov));
+              sts_v2(ov, pack4(vv.x * bb.x, vv.y * bb.y, vv.z * bb.z, vv.w * bb.w));
+            }
+          } else {
+            sts_v2(sb + OFF_XP + o, pack4(bb.x * kk.x * e2.x, bb.y * kk.y * e2.y, bb.z * kk.z * e2.z, bb.w * kk.w * e2.w));
+          }
         }
       }
       __syncthreads();
@@ -816,13 +834,21 @@ bool make_map_o(CUtensorMap *m, void *base, int64_t t_total, int H, bool bf16) {
   return r == CUDA_SUCCESS;
 }
 
-template <bool SD, bool SG, typename Tout>
+template <bool SD, bool SG, bool P3, typename Tout>
 cudaError_t launch_t(const TcParams &P, int grid, cudaStream_t stream) {
-  auto kern = chunk_tc_kernel<SD, SG, Tout>;
+  auto kern = chunk_tc_kernel<SD, SG, P3, Tout>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, kSmemBytes, stream>>>(P);
   return cudaGetLastError();
+}
+
+template <bool P3>
+cudaError_t launch_gates(const TcParams &P, int grid, cudaStream_t stream, bool sd, bool sg, bool obf) {
+  if (sd && sg) return obf ? launch_t<true, true, P3, __nv_bfloat16>(P, grid, stream) : launch_t<true, true, P3, float>(P, grid, stream);
+  if (sd) return obf ? launch_t<true, false, P3, __nv_bfloat16>(P, grid, stream) : launch_t<true, false, P3, float>(P, grid, stream);
+  if (sg) return obf ? launch_t<false, true, P3, __nv_bfloat16>(P, grid, stream) : launch_t<false, true, P3, float>(P, grid, stream);
+  return obf ? launch_t<false, false, P3, __nv_bfloat16>(P, grid, stream) : launch_t<false, false, P3, float>(P, grid, stream);
 }
 
 }  // namespace
@@ -839,6 +865,7 @@ cudaError_t launch_chunk_tc(const ChunkProblem &p, cudaStream_t stream, const ch
   const bool sd = (p.flags & GDN2_SCALAR_DECAY) != 0;
   const bool sg = (p.flags & GDN2_SCALAR_GATES) != 0;
   const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
+  const bool p3 = (p.flags & GDN2_GATE_FORM_P3) != 0;
   TcParams P;
   memset(&P, 0, sizeof(P));
   P.p = p;
@@ -849,7 +876,11 @@ cudaError_t launch_chunk_tc(const ChunkProblem &p, cudaStream_t stream, const ch
   bool ok = make_map(&P.tm_q, p.q, T, p.n_heads) && make_map(&P.tm_k, p.k, T, p.n_heads) &&
             make_map(&P.tm_v, p.v, T, p.n_heads);
   if (ok && !sd) ok = make_map(&P.tm_g, p.log_a, T, p.n_heads);
-  if (ok && !sg) ok = make_map(&P.tm_b, p.b, T, p.n_heads) && make_map(&P.tm_w, tied ? p.b : p.w, T, p.n_heads);
+  // tm_w feeds the first elementwise pass and tm_b the second; the gist.science form
+  // needs its erase gate first and its value gate (w, d_v = d_k channels) second.
+  const void *g_first = p3 ? p.b : (tied ? p.b : p.w);
+  const void *g_second = p3 ? (tied ? p.b : p.w) : p.b;
+  if (ok && !sg) ok = make_map(&P.tm_b, g_second, T, p.n_heads) && make_map(&P.tm_w, g_first, T, p.n_heads);
   if (ok) ok = make_map_o(&P.tm_o, p.o, T, p.n_heads, p.dtype_out == GDN2_BF16);
   if (!ok) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad tensor geometry)";
@@ -860,10 +891,7 @@ cudaError_t launch_chunk_tc(const ChunkProblem &p, cudaStream_t stream, const ch
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = P.n_units < sms ? P.n_units : sms;
   const bool obf = p.dtype_out == GDN2_BF16;
-  if (sd && sg) return obf ? launch_t<true, true, __nv_bfloat16>(P, grid, stream) : launch_t<true, true, float>(P, grid, stream);
-  if (sd) return obf ? launch_t<true, false, __nv_bfloat16>(P, grid, stream) : launch_t<true, false, float>(P, grid, stream);
-  if (sg) return obf ? launch_t<false, true, __nv_bfloat16>(P, grid, stream) : launch_t<false, true, float>(P, grid, stream);
-  return obf ? launch_t<false, false, __nv_bfloat16>(P, grid, stream) : launch_t<false, false, float>(P, grid, stream);
+  return p3 ? launch_gates<true>(P, grid, stream, sd, sg, obf) : launch_gates<false>(P, grid, stream, sd, sg, obf);
 }
 
 }  // namespace gdn2

@@ -106,9 +106,9 @@ def make_dims(n_seqs, seq_len, n_heads, d_k, d_v, chunk, dtype_in, dtype_out, fl
                 int(dtype_out), int(flags), 0)
 
 
-def flags_of(scalar_decay=False, scalar_gates=False, tied_gates=False) -> int:
+def flags_of(scalar_decay=False, scalar_gates=False, tied_gates=False, gate_form_p3=False) -> int:
     return (SCALAR_DECAY if scalar_decay else 0) | (SCALAR_GATES if scalar_gates else 0) | \
-           (TIED_GATES if tied_gates else 0)
+           (TIED_GATES if tied_gates else 0) | (GATE_FORM_P3 if gate_form_p3 else 0)
 
 
 def workspace_size(dims: Dims) -> int:
@@ -118,15 +118,16 @@ def workspace_size(dims: Dims) -> int:
 def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, b: torch.Tensor,
               w: Optional[torch.Tensor] = None, S0: Optional[torch.Tensor] = None,
               cu_seqlens: Optional[torch.Tensor] = None, *, chunk: int = 64, scalar_decay: bool = False,
-              scalar_gates: bool = False, tied_gates: bool = False, out_dtype: Optional[torch.dtype] = None,
-              output_final_state: bool = True, cu_seqlens_host: Optional[Sequence[int]] = None,
+              scalar_gates: bool = False, tied_gates: bool = False, gate_form_p3: bool = False,
+              out_dtype: Optional[torch.dtype] = None, output_final_state: bool = True, cu_seqlens_host: Optional[Sequence[int]] = None,
               o: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
               workspace: Optional[torch.Tensor] = None):
     """Chunked GDN-2 forward through ``gdn2_chunk_fwd``.
 
     q, k: [B, T, H, d_k] (equal lengths) or [T_tot, H, d_k] with ``cu_seqlens``
     (int32 [N+1] on the device); v: same with d_v.  log_a, b, w: like k, or
-    [.., H] with the scalar flags.  S0: fp32 [N, H, d_k, d_v] or None.
+    [.., H] with the scalar flags; with ``gate_form_p3`` (the gist.science gate
+    placement) w has d_v channels.  S0: fp32 [N, H, d_k, d_v] or None.
     Returns (o [.., H, d_v], S_T fp32 [N, H, d_k, d_v] or None).
     """
     if q.dim() == 4:
@@ -148,7 +149,7 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Te
         raise ValueError("q must be [B, T, H, d_k] or [T_tot, H, d_k]")
     dv = v.shape[-1]
     out_dtype = q.dtype if out_dtype is None else out_dtype
-    flags = flags_of(scalar_decay, scalar_gates, tied_gates)
+    flags = flags_of(scalar_decay, scalar_gates, tied_gates, gate_form_p3)
     dims = make_dims(N, seq_len, H, dk, dv, chunk, _dtype_code(q.dtype), _dtype_code(out_dtype), flags)
     dev = q.device
     if o is None:
@@ -174,16 +175,17 @@ def check_status(workspace: torch.Tensor) -> int:
 
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, b: torch.Tensor,
                 w: Optional[torch.Tensor], S: torch.Tensor, *, scalar_decay: bool = False,
-                scalar_gates: bool = False, tied_gates: bool = False, out_dtype: torch.dtype = torch.float32,
-                o: Optional[torch.Tensor] = None) -> torch.Tensor:
+                scalar_gates: bool = False, tied_gates: bool = False, gate_form_p3: bool = False,
+                out_dtype: torch.dtype = torch.float32, o: Optional[torch.Tensor] = None) -> torch.Tensor:
     """One recurrent step through ``gdn2_decode_step``; ``S`` [N, H, d_k, d_v] fp32 is updated in place.
 
-    q, k, log_a, b, w: [N, H, d_k] (or [N, H] with the scalar flags); v: [N, H, d_v].
+    q, k, log_a, b, w: [N, H, d_k] (or [N, H] with the scalar flags; w is [N, H, d_v]
+    with ``gate_form_p3``); v: [N, H, d_v].
     Returns o [N, H, d_v].
     """
     N, H, dk = q.shape
     dv = v.shape[-1]
-    flags = flags_of(scalar_decay, scalar_gates, tied_gates)
+    flags = flags_of(scalar_decay, scalar_gates, tied_gates, gate_form_p3)
     dims = make_dims(N, 1, H, dk, dv, 0, _dtype_code(q.dtype), _dtype_code(out_dtype), flags)
     if o is None:
         o = torch.empty(N, H, dv, dtype=out_dtype, device=q.device)

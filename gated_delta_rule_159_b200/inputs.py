@@ -98,9 +98,11 @@ def _l2n(x: torch.Tensor) -> torch.Tensor:
 
 
 def make_inputs(workload, device="cuda", seed: int = 0, seq_len: Optional[int] = None,
-                n_seqs: Optional[int] = None, lengths: Optional[List[int]] = None) -> dict:
+                n_seqs: Optional[int] = None, lengths: Optional[List[int]] = None,
+                gate_form_p3: bool = False) -> dict:
     """Inputs of a workload (by name or ``Workload``).  ``seq_len``/``n_seqs``/``lengths``
-    override the sizes (smaller parity cases with the same distributions)."""
+    override the sizes (smaller parity cases with the same distributions).  With
+    ``gate_form_p3`` the write gate w has d_v channels (the gist.science placement)."""
     w = WORKLOADS[workload] if isinstance(workload, str) else workload
     device = torch.device(device)
     H, dk, dv = w.n_heads, w.d_k, w.d_v
@@ -122,7 +124,8 @@ def make_inputs(workload, device="cuda", seed: int = 0, seq_len: Optional[int] =
     gshape = (T_tot, H) if w.scalar_gates else (T_tot, H, dk)
     log_a = (-torch.nn.functional.softplus(_randn(gshape, g, device)) * w.decay_scale).to(w.dtype)
     b = torch.sigmoid(_randn(gshape, g, device)).to(w.dtype)
-    wg = None if w.scalar_gates else torch.sigmoid(_randn(gshape, g, device)).to(w.dtype)
+    wshape = (T_tot, H, dv) if gate_form_p3 else gshape
+    wg = None if w.scalar_gates else torch.sigmoid(_randn(wshape, g, device)).to(w.dtype)
     S0 = (_randn((N, H, dk, dv), g, device) * w.s0_std) if w.s0_std > 0 else None
     equal = lengths is None
     return dict(
@@ -130,19 +133,24 @@ def make_inputs(workload, device="cuda", seed: int = 0, seq_len: Optional[int] =
         cu_seqlens=None if equal else torch.tensor(cu, dtype=torch.int32, device=device),
         cu_host=cu.tolist(), n_seqs=N, T_tot=T_tot, equal_lengths=equal,
         scalar_decay=w.scalar_gates, scalar_gates=w.scalar_gates, tied_gates=w.scalar_gates,
+        gate_form_p3=gate_form_p3,
     )
 
 
 def make_decode_inputs(n_seqs: int, n_heads: int, d: int, steps: int, device="cuda", seed: int = 1,
-                       dtype=torch.bfloat16, decay_scale: float = 0.05) -> dict:
-    """Per-step decode inputs [steps, N, H, d] with the full GDN-2 gate distributions."""
+                       dtype=torch.bfloat16, decay_scale: float = 0.05, d_v: Optional[int] = None,
+                       gate_form_p3: bool = False) -> dict:
+    """Per-step decode inputs [steps, N, H, d] (v: d_v, default d) with the full GDN-2
+    gate distributions; w has d_v channels with ``gate_form_p3``."""
     device = torch.device(device)
     g = _gen(device, seed)
+    dv = d if d_v is None else d_v
     shp = (steps, n_seqs, n_heads, d)
+    shv = (steps, n_seqs, n_heads, dv)
     q = _l2n(_randn(shp, g, device)).to(dtype)
     k = _l2n(_randn(shp, g, device)).to(dtype)
-    v = _randn(shp, g, device).to(dtype)
+    v = _randn(shv, g, device).to(dtype)
     log_a = (-torch.nn.functional.softplus(_randn(shp, g, device)) * decay_scale).to(dtype)
     b = torch.sigmoid(_randn(shp, g, device)).to(dtype)
-    w = torch.sigmoid(_randn(shp, g, device)).to(dtype)
+    w = torch.sigmoid(_randn(shv if gate_form_p3 else shp, g, device)).to(dtype)
     return dict(q=q, k=k, v=v, log_a=log_a, b=b, w=w)

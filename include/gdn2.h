@@ -20,7 +20,13 @@
  * (read after the update).  Where those pages differ on which side the gates
  * sit, this library follows the form above by default (erase outer factor
  * b.k, erase read with k, write outer factor w.k) and offers the gist.science
- * equation as GDN2_GATE_FORM_P3 (reserved; not implemented by the kernels yet).
+ * equation as GDN2_GATE_FORM_P3:
+ *
+ *   S_t = (I - k_t (b_t . k_t)^T) Diag(a_t) S_{t-1} + k_t (w_t . v_t)^T,
+ *   o_t = S_t^T q_t,
+ *
+ * where the erase read uses b.k, the erase and write outer factors are k and
+ * the write gate w_t has d_v channels and scales the value.
  *
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
@@ -70,7 +76,8 @@ enum gdn2_flags {
   GDN2_SCALAR_DECAY = 1u,  /* log_a is [T_tot, H]: one decay per token and head (a = alpha 1) */
   GDN2_SCALAR_GATES = 2u,  /* b and w are [T_tot, H]: one erase and one write gate per token and head */
   GDN2_TIED_GATES = 4u,    /* w is b (the w pointer is ignored and may be NULL) */
-  GDN2_GATE_FORM_P3 = 8u   /* reserved: gist.science gate placement; returns GDN2_ERR_UNSUPPORTED */
+  GDN2_GATE_FORM_P3 = 8u   /* gist.science gate placement (above): w is [T_tot, H, d_v]; with
+                              GDN2_TIED_GATES and per-channel gates it needs d_k == d_v */
 };
 
 /*
@@ -114,7 +121,7 @@ typedef struct gdn2_dims {
  *   v            [T_tot, H, d_v]  dtype_in
  *   log_a        [T_tot, H, d_k]  dtype_in, log of the decay (<= 0); [T_tot, H] with GDN2_SCALAR_DECAY
  *   b, w         [T_tot, H, d_k]  dtype_in, erase / write gates; [T_tot, H] with GDN2_SCALAR_GATES;
- *                w may be NULL with GDN2_TIED_GATES
+ *                w may be NULL with GDN2_TIED_GATES; w is [T_tot, H, d_v] with GDN2_GATE_FORM_P3
  *   S0           [N, H, d_k, d_v] fp32 initial states, or NULL for zeros.  May alias S_T.
  *   cu_seqlens   device int32 [N + 1] token offsets (0 = cu[0] <= ... <= cu[N] = T_tot), or NULL
  *   cu_seqlens_host  optional host copy of cu_seqlens used to schedule the longest sequences
@@ -150,12 +157,13 @@ int gdn2_check_status(const void *workspace, gdn2_stream_t stream);
  * gdn2_decode_step -- one recurrent step (alanhou.org "Core Mechanism": inference
  * runs as a pure RNN with O(1) memory per token) for N sequences, updating the
  * states in place: every state is read once and written once.
- *   q, k, log_a, b, w  [N, H, d_k] dtype_in ([N, H] for the scalar flags)
+ *   q, k, log_a, b, w  [N, H, d_k] dtype_in ([N, H] for the scalar flags;
+ *                      w is [N, H, d_v] with GDN2_GATE_FORM_P3)
  *   v                  [N, H, d_v] dtype_in
  *   S                  [N, H, d_k, d_v] fp32, read and overwritten in place
  *   o                  [N, H, d_v] dtype_out
- * dims.seq_len must be 1.  Supported: d_k, d_v multiples of 4 with
- * d_k * d_v <= 128 * 128, bf16 or fp32 in, fp32 or bf16 out.
+ * dims.seq_len must be 1.  Supported: d_k <= 128, d_v in {16, 32, 64, 128},
+ * bf16 or fp32 in, fp32 or bf16 out.
  * Errors: GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_CUDA.
  */
 int gdn2_decode_step(const void *q, const void *k, const void *v,

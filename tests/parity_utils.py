@@ -36,6 +36,8 @@ def oracle_flags(inp) -> int:
         f |= oracle.SCALAR_GATES
     if inp["tied_gates"]:
         f |= oracle.TIED_GATES
+    if inp.get("gate_form_p3", False):
+        f |= oracle.GATE_FORM_P3
     return f
 
 
@@ -101,7 +103,7 @@ def run_chunk(inp, out_dtype=None, S0="inp", packed=None):
     w = inp["workload"]
     S0t = inp["S0"] if S0 == "inp" else S0
     kw = dict(chunk=w.chunk, scalar_decay=inp["scalar_decay"], scalar_gates=inp["scalar_gates"],
-              tied_gates=inp["tied_gates"], out_dtype=out_dtype)
+              tied_gates=inp["tied_gates"], gate_form_p3=inp.get("gate_form_p3", False), out_dtype=out_dtype)
     names = ("q", "k", "v", "log_a", "b", "w")
     if packed is None:
         packed = not inp["equal_lengths"]

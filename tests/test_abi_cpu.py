@@ -70,7 +70,7 @@ def test_workspace_size(g):
 
 @pytest.mark.parametrize("bad,code", [
     (dict(n_seqs=0), -1), (dict(n_heads=0), -1), (dict(seq_len=-1), -1), (dict(dtype_in=7), -1),
-    (dict(flags=1 << 10), -1), (dict(flags=8), -2), (dict(d_k=96, d_v=96), -2), (dict(chunk=48, d_k=32, d_v=32), -2),
+    (dict(flags=1 << 10), -1), (dict(flags=8 | 4, d_k=64, d_v=32), -1), (dict(d_k=96, d_v=96), -2), (dict(chunk=48, d_k=32, d_v=32), -2),
     (dict(dtype_in=1), -2),  # fp32 input with d = 128 has no kernel
 ])
 def test_chunk_rejects_bad_dims(g, bad, code):

@@ -102,6 +102,45 @@ def test_tc_scalar_gates(dev):
     assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (eo, es)
 
 
+# gist.science gate placement: S = (I - k (b.k)^T) D S + k (w.v)^T, w on the d_v axis
+@pytest.mark.parametrize("variant", ["channel", "scalar", "tied"])
+def test_tc_gate_form_p3(dev, variant):
+    lens = [1, 63, 64, 65, 200, 0, 130]
+    inp = _small(dev, n_heads=2, lengths=lens, scalar=(variant == "scalar"), gate_form_p3=True)
+    if variant == "scalar":
+        inp["tied_gates"] = False
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(31)
+        inp["w"] = torch.sigmoid(torch.randn(inp["b"].shape, generator=gen, device=dev)).to(inp["b"].dtype)
+    if variant == "tied":
+        inp["tied_gates"] = True
+        inp["w"] = None
+    o, S_T = run_chunk(inp)
+    eo, es = compare_units(inp, o, S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (eo, es)
+
+
+def test_tc_gate_forms_differ(dev):
+    """With channel-wise b != w the two gate placements give different results: the
+    flag reaches the kernel (each side is checked against its own oracle above)."""
+    inp = _small(dev, n_seqs=1, seq_len=130, n_heads=2, gate_form_p3=True)
+    o3, S3 = run_chunk(inp)
+    inp["gate_form_p3"] = False
+    o0, S0_ = run_chunk(inp)
+    ref = max(float(o3.abs().max()), 1e-30)
+    assert float((o3.float() - o0.float()).abs().max()) / ref > 10 * TOL_CHUNK_BF16
+
+
+@pytest.mark.parametrize("dk,dv,chunk,dtype", [(32, 64, 32, torch.float32), (64, 16, 64, torch.bfloat16)])
+def test_simt_gate_form_p3(dev, dk, dv, chunk, dtype):
+    inp = _small(dev, dk=dk, dv=dv, chunk=chunk, dtype=dtype, n_heads=2,
+                 lengths=[1, chunk - 1, chunk + 1, 0, 3 * chunk + 5], gate_form_p3=True)
+    assert inp["w"].shape[-1] == dv
+    o, S_T = run_chunk(inp, out_dtype=torch.float32)
+    eo, es = compare_units(inp, o, S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_F32 and es <= TOL_CHUNK_F32, (eo, es)
+
+
 @pytest.mark.parametrize("case", ["deltanet", "pure_decay", "zero_key", "strong_decay", "no_decay_no_gates"])
 def test_tc_degenerate_cases(dev, case):
     inp = _small(dev, n_seqs=1, seq_len=192, n_heads=2)
@@ -222,6 +261,58 @@ def test_decode_small(dev, d, scalar):
         for h in range(H):
             assert rel_err(o_gpu[:, n, h], o_r[:, h]) <= TOL_DECODE
             assert rel_err(to_f64(S[n, h]), S_r[0, h]) <= TOL_DECODE
+
+
+@pytest.mark.parametrize("dk,dv,scalar", [(128, 128, False), (64, 32, False), (128, 64, True)])
+def test_decode_gate_form_p3(dev, dk, dv, scalar):
+    from gated_delta_rule_159_b200 import gdn2, inputs
+    N, H, steps = 3, 2, 6
+    di = inputs.make_decode_inputs(N, H, dk, steps, dev, seed=9, d_v=dv, gate_form_p3=True)
+    if scalar:
+        for n in ("log_a", "b", "w"):
+            di[n] = di[n][..., 0].contiguous()
+    g = torch.Generator(device=dev)
+    g.manual_seed(11)
+    S = torch.randn(N, H, dk, dv, generator=g, device=dev) * 0.1
+    S_start = to_f64(S)
+    outs = []
+    for t in range(steps):
+        outs.append(gdn2.decode_step(*(di[n][t] for n in ("q", "k", "v", "log_a", "b", "w")), S,
+                                     scalar_decay=scalar, scalar_gates=scalar, gate_form_p3=True))
+    o_gpu = to_f64(torch.stack(outs))
+    flags = oracle.GATE_FORM_P3 | ((oracle.SCALAR_DECAY | oracle.SCALAR_GATES) if scalar else 0)
+    for n in range(N):
+        sl = lambda t: to_f64(t[:, n])  # noqa: E731
+        o_r, S_r = oracle.gdn2_fwd(*(sl(di[m]) for m in ("q", "k", "v", "log_a", "b", "w")),
+                                   S0=S_start[n][None], flags=flags)
+        for h in range(H):
+            assert rel_err(o_gpu[:, n, h], o_r[:, h]) <= TOL_DECODE
+            assert rel_err(to_f64(S[n, h]), S_r[0, h]) <= TOL_DECODE
+
+
+def test_decode_graph_replay_matches_eager(dev):
+    """Decode steps captured in a CUDA graph and replayed give the eager results bit for bit."""
+    from gated_delta_rule_159_b200 import gdn2, inputs
+    N, H, d, steps = 8, 4, 128, 5
+    names = ("q", "k", "v", "log_a", "b", "w")
+    di = inputs.make_decode_inputs(N, H, d, steps, dev, seed=21)
+    g = torch.Generator(device=dev)
+    g.manual_seed(23)
+    S_init = torch.randn(N, H, d, d, generator=g, device=dev) * 0.1
+    S_eager = S_init.clone()
+    o_eager = [gdn2.decode_step(*(di[n][t] for n in names), S_eager).clone() for t in range(steps)]
+    S_graph = S_init.clone()
+    o_buf = torch.empty(steps, N, H, d, device=dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for t in range(steps):
+            gdn2.decode_step(*(di[n][t] for n in names), S_graph, o=o_buf[t])
+    S_graph.copy_(S_init)  # capture records the launches without running them
+    graph.replay()
+    torch.cuda.synchronize()
+    del graph
+    torch.testing.assert_close(S_graph, S_eager, rtol=0, atol=0)
+    torch.testing.assert_close(o_buf, torch.stack(o_eager), rtol=0, atol=0)
 
 
 def test_decode_full_size_sampled(dev):
