@@ -9,6 +9,8 @@ package.  The CUDA product path never calls it and shares no code with it.
   decay, erase read of the decayed state, erase with b, write with w, read with
   q after the update (see ``gdn2_oracle.c`` for the citations).
 * ``gdn2_decode_step`` -- the same recurrence for one token per sequence.
+* ``gdn2_bwd`` -- reverse-mode gradients of that recurrence in float64 (C),
+  pinned by central finite differences of ``gdn2_fwd``.
 * ``chunked.gdn2_chunked_fwd`` -- the float64 chunkwise (WY) form, used only to
   prove the chunk algebra equal to the recurrence on tiny inputs.
 
@@ -56,6 +58,10 @@ def _load():
         lib.oracle_gdn2_fwd.restype = ctypes.c_int
         lib.oracle_gdn2_fwd.argtypes = [i64, i64, i64, i64, i64, ctypes.POINTER(ctypes.c_int64),
                                         dp, dp, dp, dp, dp, dp, dp, dp, dp, i64]
+        lib.oracle_gdn2_bwd.restype = ctypes.c_int
+        lib.oracle_gdn2_bwd.argtypes = [i64, i64, i64, i64, i64, ctypes.POINTER(ctypes.c_int64),
+                                        dp, dp, dp, dp, dp, dp, dp, dp, dp,
+                                        dp, dp, dp, dp, dp, dp, dp, i64]
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -119,3 +125,38 @@ def gdn2_decode_step(q, k, v, log_a, b, w, S, flags: int = 0, n_threads: int = 0
     N = q.shape[0]
     cu = np.arange(N + 1, dtype=np.int64)
     return gdn2_fwd(q, k, v, log_a, b, w, S0=S, cu_seqlens=cu, flags=flags, n_threads=n_threads)
+
+
+def gdn2_bwd(q, k, v, log_a, b, w, dO, S0=None, dS_T=None, cu_seqlens=None, flags: int = 0,
+             n_threads: int = 0):
+    """Float64 gradients of  sum <dO, o> + <dS_T, S_T>  for ``gdn2_fwd`` with the same
+    arguments.  Returns a dict with dq, dk, dv, dlog_a, db, dw (None with TIED_GATES,
+    whose w gradient is added into db) and dS0, each shaped like its input."""
+    q, k, v, log_a, b = (_f64(t) for t in (q, k, v, log_a, b))
+    w, dO, S0, dS_T = _f64(w), _f64(dO), _f64(S0), _f64(dS_T)
+    T_tot, H, dk = q.shape
+    dv = v.shape[2]
+    cu = np.array([0, T_tot], dtype=np.int64) if cu_seqlens is None else \
+        np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    N = cu.shape[0] - 1
+    if cu[0] != 0 or cu[-1] != T_tot:
+        raise ValueError("cu_seqlens must start at 0 and end at T_tot")
+    tied = bool(flags & TIED_GATES)
+    if w is None and not tied:
+        raise ValueError("w is required unless TIED_GATES")
+    if dO.shape != (T_tot, H, dv):
+        raise ValueError(f"dO shape {dO.shape} != {(T_tot, H, dv)}")
+    for name, t in (("S0", S0), ("dS_T", dS_T)):
+        if t is not None and t.shape != (N, H, dk, dv):
+            raise ValueError(f"{name} shape {t.shape} != {(N, H, dk, dv)}")
+    out = dict(dq=np.zeros_like(q), dk=np.zeros_like(k), dv=np.zeros_like(v), dlog_a=np.zeros_like(log_a),
+               db=np.zeros_like(b), dw=None if tied else np.zeros_like(w),
+               dS0=np.zeros((N, H, dk, dv), dtype=np.float64))
+    rc = _load().oracle_gdn2_bwd(N, H, dk, dv, int(flags), cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                 _ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(b), _ptr(None if tied else w),
+                                 _ptr(S0), _ptr(dO), _ptr(dS_T),
+                                 _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dlog_a"]),
+                                 _ptr(out["db"]), _ptr(out["dw"]), _ptr(out["dS0"]), int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle_gdn2_bwd rejected its arguments")
+    return out
