@@ -11,6 +11,8 @@ package.  The CUDA product path never calls it and shares no code with it.
 * ``gdn2_decode_step`` -- the same recurrence for one token per sequence.
 * ``gdn2_bwd`` -- reverse-mode gradients of that recurrence in float64 (C),
   pinned by central finite differences of ``gdn2_fwd``.
+* ``prologue`` -- the activations (q, k L2-normalised; sigmoid gates) that
+  turn pre-activations into the recurrence inputs, and their gradient.
 * ``chunked.gdn2_chunked_fwd`` -- the float64 chunkwise (WY) form, used only to
   prove the chunk algebra equal to the recurrence on tiny inputs.
 
