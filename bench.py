@@ -18,6 +18,9 @@ prefill (tokens/s and fraction of HBM bandwidth), the roofline of the chunk
 kernel, the end-to-end number through host buffers, the float64 CPU oracle as
 `cpu_baseline`, and the SM clocks sampled while timing.
 
+`bwd` times gdn2_bwd (all gradients of the forward, fp32 reverse mode) on the
+prefill workload with random dO and dS_T.
+
 `--impl reference` times the float64 CPU oracle on a bounded sample of the
 same workload instead (rank 0 only).
 """
@@ -47,6 +50,15 @@ WORKLOAD = "gdn2_b8_t4k"
 FLOP_PER_TOKHEAD = 8 * 64 * 128 + 8 * 64 * 128 + 8 * 128 * 128
 BYTES_PER_TOKHEAD = 6 * 128 * 2 + 128 * 2                      # six bf16 inputs + bf16 o
 STATE_BYTES = 128 * 128 * 4                                    # one fp32 state
+# fp32 operations of the backward per token-head (d_k = d_v = 128): per state
+# element, the forward sweep and the block recompute take 7 each (decay, erase
+# read, erase and write updates) and the reverse step 26.
+BWD_FLOP_PER_TOKHEAD = (7 + 7 + 26) * 128 * 128
+
+
+def fp32_peak_tflops(sm_max_mhz: float) -> float:
+    """CUDA-core fp32 peak: 148 SMs x 128 FMA lanes x 2 flops x the max SM clock."""
+    return 148 * 128 * 2 * sm_max_mhz * 1e6 / 1e12
 
 
 def peaks():
@@ -222,6 +234,8 @@ def main():
     ap.add_argument("--reference-step-seconds", type=float, default=6.0)
     ap.add_argument("--batch", type=int, default=0, help="override the batch size (small profiling cases)")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--bwd-steps", type=int, default=3)
+    ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     args = ap.parse_args()
@@ -381,23 +395,85 @@ def main():
             gdn2.decode_step(*(di[n][t] for n in names), S, o=od)
         e1.record(stream)
         barrier()
+        plain_ms = max_over_ranks(e0.elapsed_time(e1))
+        # The same steps captured once as a CUDA graph and replayed: one graph launch
+        # per decode loop, so the per-step host launch gap leaves the timed region.
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for t in range(steps):
+                gdn2.decode_step(*(di[n][t] for n in names), S, o=od)
+        graph.replay()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        barrier()
         dclocks = sd.stop()
         dms = max_over_ranks(e0.elapsed_time(e1))
+        del graph
+        if gdn2.decode_status() != gdn2.OK:
+            raise RuntimeError("decode kernel reported a timed-out wait")
         step_bytes = 2 * Nd * Hd * d * d * 4 + 6 * Nd * Hd * d * 2 + Nd * Hd * d * 4
         gbs = step_bytes * steps / (dms / 1e3) / 1e9
         decode = {"value": Nd * world * steps / (dms / 1e3), "unit": "tokens/s", "steps": steps,
                   "us_per_step": 1e3 * dms / steps, "bytes_per_step": step_bytes, "hbm_gbs": gbs,
                   "hbm_frac": gbs / hbm_peak, "peak_source": peak_src, "sequences": Nd, "heads": Hd,
-                  "state_bytes": Nd * Hd * d * d * 4, "clocks": dclocks, "kernel": "decode_kernel",
-                  "launch": "one launch per step (plain stream loop)", "gpu_launches": steps}
+                  "state_bytes": Nd * Hd * d * d * 4, "clocks": dclocks, "kernel": "decode_stream_kernel",
+                  "launch": "CUDA graph of all steps, replayed once",
+                  "plain_loop_us_per_step": 1e3 * plain_ms / steps,
+                  "gpu_launches": steps}
         del di, S
+
+    # ---------------- backward (gradients of the prefill step)
+    bwd = None
+    if not args.no_bwd:
+        bi = inputs.make_inputs(WORKLOAD, dev, seed=300 + rank, n_seqs=args.batch or None)
+        Nb, Tb = bi["n_seqs"], bi["T_tot"] // bi["n_seqs"]
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(400 + rank)
+        dO = torch.randn(Nb, Tb, 16, 128, generator=gen, device=dev).to(torch.bfloat16)
+        dS_T = torch.randn(Nb, 16, 128, 128, generator=gen, device=dev) * 0.1
+        bargs = [bi[n].view(Nb, Tb, *bi[n].shape[1:]) for n in names]
+        bdims = gdn2.make_dims(Nb, Tb, 16, 128, 128, 64, gdn2.BF16, gdn2.BF16, 0)
+        bws = torch.empty(int(gdn2.lib.gdn2_bwd_workspace_size(gdn2.ctypes.byref(bdims), 0)), dtype=torch.uint8,
+                          device=dev)
+
+        def bstep():
+            return gdn2.bwd(*bargs, dO, S0=bi["S0"], dS_T=dS_T, workspace=bws)
+
+        bstep()
+        torch.cuda.synchronize()
+        barrier()
+        bs = ClockSampler(dev.index if dev.index is not None else 0)
+        bs.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.bwd_steps):
+            bstep()
+        e1.record(stream)
+        barrier()
+        bclocks = bs.stop()
+        bms = max_over_ranks(e0.elapsed_time(e1)) / args.bwd_steps
+        tokheads = Nb * Tb * 16
+        tflops = BWD_FLOP_PER_TOKHEAD * tokheads / (bms / 1e3) / 1e12
+        peak32 = fp32_peak_tflops(bclocks.get("sm_max_mhz") or 1965.0)
+        bwd = {"value": Nb * Tb * world / (bms / 1e3), "unit": "tokens/s", "ms_per_step": bms,
+               "steps": args.bwd_steps, "dtype": "f32 arithmetic, bf16 inputs and gradients",
+               "roofline": {"bound": "alu", "achieved": tflops, "peak": peak32, "unit": "TFLOP/s",
+                            "frac": tflops / peak32, "traffic": None,
+                            "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x sm_max_mhz",
+                            "alg_flops_per_tokhead": BWD_FLOP_PER_TOKHEAD},
+               "kernels": ["bwd_kernel", "finish_kernel"], "gpu_launches": 2 * args.bwd_steps,
+               "workspace_bytes": bws.numel(), "clocks": bclocks}
+        del bi, dO, dS_T, bargs, bws
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes and distributions of the "
                                                           "full GDN-2 workload)",
             "config": cfg, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches, "clocks": clocks, "decode": decode}
+            "gpu_launches": launches, "clocks": clocks, "decode": decode, "bwd": bwd}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -21,7 +21,8 @@ int fail(int code, const char *fmt, ...) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-constexpr uint32_t kKnownFlags = GDN2_SCALAR_DECAY | GDN2_SCALAR_GATES | GDN2_TIED_GATES | GDN2_GATE_FORM_P3;
+constexpr uint32_t kKnownFlags =
+    GDN2_SCALAR_DECAY | GDN2_SCALAR_GATES | GDN2_TIED_GATES | GDN2_GATE_FORM_P3 | GDN2_FUSED_PROLOGUE;
 constexpr size_t kWsHeader = 256;     // [0] status word, [1] unit counter
 constexpr int kMaxSortedSeqs = 4096;  // above this the units run in index order
 
@@ -164,6 +165,62 @@ int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *log_
   return GDN2_OK;
 }
 
+size_t gdn2_bwd_workspace_size(const gdn2_dims *dims, int32_t packed) {
+  if (!dims || dims->n_seqs < 1 || dims->n_heads < 1 || dims->seq_len < 0 || dims->d_k < 1 || dims->d_v < 1)
+    return 0;
+  if (dims->d_v != 16 && dims->d_v != 32 && dims->d_v != 64 && dims->d_v != 128) return 0;
+  const int64_t t_total = packed ? (int64_t)dims->seq_len : (int64_t)dims->n_seqs * dims->seq_len;
+  return gdn2::bwd_workspace_bytes(dims->n_seqs, t_total, dims->n_heads, dims->d_k, dims->d_v, dims->flags);
+}
+
+int gdn2_bwd(const void *q, const void *k, const void *v, const void *log_a, const void *b, const void *w,
+             const float *S0, const int32_t *cu_seqlens, const void *dO, const float *dS_T, void *dq, void *dk,
+             void *dv, void *dlog_a, void *db, void *dw, float *dS0, const gdn2_dims *dims, void *workspace,
+             size_t workspace_bytes, gdn2_stream_t stream) {
+  g_err[0] = '\0';
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  rc = check_inputs(q, k, v, log_a, b, w, dims->flags, dims->dtype_in);
+  if (rc) return rc;
+  if (dims->d_k > 128 || (dims->d_v != 16 && dims->d_v != 32 && dims->d_v != 64 && dims->d_v != 128))
+    return fail(GDN2_ERR_UNSUPPORTED, "gdn2_bwd supports d_k <= 128 and d_v in {16, 32, 64, 128} (got %d, %d)",
+                dims->d_k, dims->d_v);
+  const bool tied = (dims->flags & GDN2_TIED_GATES) != 0;
+  if (!dO || !dq || !dk || !dv || !dlog_a || !db || (!dw && !tied))
+    return fail(GDN2_ERR_INVALID_ARG, "dO, dq, dk, dv, dlog_a, db (and dw without GDN2_TIED_GATES) must be non-NULL");
+  if ((S0 && !aligned16(S0)) || (dS_T && !aligned16(dS_T)) || (dS0 && !aligned16(dS0)))
+    return fail(GDN2_ERR_INVALID_ARG, "S0, dS_T and dS0 must be 16-byte aligned");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(GDN2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  const int64_t t_total = cu_seqlens ? (int64_t)dims->seq_len : (int64_t)dims->n_seqs * dims->seq_len;
+  const size_t need = gdn2::bwd_workspace_bytes(dims->n_seqs, t_total, dims->n_heads, dims->d_k, dims->d_v,
+                                                dims->flags);
+  if (workspace_bytes < need)
+    return fail(GDN2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+  gdn2::BwdProblem p;
+  memset(&p, 0, sizeof(p));
+  p.q = q; p.k = k; p.v = v; p.log_a = log_a; p.b = b; p.w = w;
+  p.S0 = S0; p.cu_seqlens = cu_seqlens; p.dO = dO; p.dS_T = dS_T;
+  p.dq = dq; p.dk = dk; p.dv = dv; p.dlog_a = dlog_a; p.db = db; p.dw = tied ? nullptr : dw; p.dS0 = dS0;
+  p.n_seqs = dims->n_seqs; p.seq_len = dims->seq_len; p.n_heads = dims->n_heads;
+  p.d_k = dims->d_k; p.d_v = dims->d_v; p.t_total = t_total;
+  p.dtype_in = dims->dtype_in; p.dtype_out = dims->dtype_out; p.flags = dims->flags;
+  gdn2::bwd_carve(p, workspace);
+  cudaError_t e = gdn2::launch_bwd(p, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "bwd launch: %s", cudaGetErrorString(e));
+  return GDN2_OK;
+}
+
+int gdn2_decode_status(gdn2_stream_t stream) {
+  g_err[0] = '\0';
+  int32_t st = 0;
+  const int e = gdn2::read_decode_status(reinterpret_cast<cudaStream_t>(stream), &st);
+  if (e != 0) return fail(GDN2_ERR_CUDA, "reading the decode status: %s", cudaGetErrorString((cudaError_t)e));
+  if (st == gdn2::kStatusTimeout) return fail(GDN2_ERR_TIMEOUT, "a bounded wait of the decode kernel timed out");
+  if (st != 0) return fail(GDN2_ERR_CUDA, "unknown device status %d", st);
+  return GDN2_OK;
+}
+
 int gdn2_check_status(const void *workspace, gdn2_stream_t stream) {
   g_err[0] = '\0';
   if (!workspace) return fail(GDN2_ERR_INVALID_ARG, "workspace is NULL");
@@ -196,6 +253,37 @@ int gdn2_decode_step(const void *q, const void *k, const void *v, const void *lo
   p.S = S; p.o = o;
   p.n_seqs = dims->n_seqs; p.n_heads = dims->n_heads; p.d_k = dims->d_k; p.d_v = dims->d_v;
   p.dtype_in = dims->dtype_in; p.dtype_out = dims->dtype_out; p.flags = dims->flags;
+  p.state_idx = nullptr;
+  p.n_slots = 0;
+  cudaError_t e = gdn2::launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+  return GDN2_OK;
+}
+
+int gdn2_decode_step_indexed(const void *q, const void *k, const void *v, const void *log_a, const void *b,
+                             const void *w, float *S_pool, int32_t n_slots, const int32_t *state_idx, void *o,
+                             const gdn2_dims *dims, gdn2_stream_t stream) {
+  g_err[0] = '\0';
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->seq_len != 1) return fail(GDN2_ERR_INVALID_ARG, "gdn2_decode_step_indexed needs seq_len == 1");
+  rc = check_inputs(q, k, v, log_a, b, w, dims->flags, dims->dtype_in);
+  if (rc) return rc;
+  if (!S_pool || !aligned16(S_pool) || !o || !aligned16(o))
+    return fail(GDN2_ERR_INVALID_ARG, "S_pool and o must be non-NULL and 16-byte aligned");
+  if (!state_idx || reinterpret_cast<uintptr_t>(state_idx) % 4 != 0)
+    return fail(GDN2_ERR_INVALID_ARG, "state_idx must be a non-NULL, 4-byte aligned device int32 array");
+  if (n_slots < 1) return fail(GDN2_ERR_INVALID_ARG, "n_slots must be >= 1 (got %d)", n_slots);
+  if (dims->d_k > 128 || (dims->d_v != 16 && dims->d_v != 32 && dims->d_v != 64 && dims->d_v != 128))
+    return fail(GDN2_ERR_UNSUPPORTED, "decode supports d_k <= 128 and d_v in {16, 32, 64, 128} (got %d, %d)",
+                dims->d_k, dims->d_v);
+  gdn2::DecodeProblem p;
+  p.q = q; p.k = k; p.v = v; p.log_a = log_a; p.b = b; p.w = w;
+  p.S = S_pool; p.o = o;
+  p.n_seqs = dims->n_seqs; p.n_heads = dims->n_heads; p.d_k = dims->d_k; p.d_v = dims->d_v;
+  p.dtype_in = dims->dtype_in; p.dtype_out = dims->dtype_out; p.flags = dims->flags;
+  p.state_idx = state_idx;
+  p.n_slots = n_slots;
   cudaError_t e = gdn2::launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
   return GDN2_OK;

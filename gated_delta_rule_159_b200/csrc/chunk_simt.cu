@@ -37,6 +37,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkProblem p) {
   const bool scalar_gates = (p.flags & GDN2_SCALAR_GATES) != 0;
   const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
   const bool p3 = (p.flags & GDN2_GATE_FORM_P3) != 0;
+  const bool prolog = (p.flags & GDN2_FUSED_PROLOGUE) != 0;
 
   int64_t bos, len;
   if (p.cu_seqlens) {
@@ -88,6 +89,11 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkProblem p) {
         g = to_f32(scalar_decay ? ga[is] : ga[ik]);
         bb = to_f32(scalar_gates ? gb[is] : gb[ik]);
         if (!p3) ww = to_f32(scalar_gates ? gw[is] : gw[ik]);
+        if (prolog) {
+          g = log_sigmoid_f(g);
+          bb = sigmoid_f(bb);
+          ww = sigmoid_f(ww);
+        }
       }
       // sk: erase read vector, sx: erase outer factor, sp: write outer factor.
       // Default form (k, b.k, w.k); gist.science form (b.k, k, k), whose write
@@ -104,11 +110,33 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkProblem p) {
       if (r < nr) {
         const int64_t tok = bos + c0 + r;
         vv = to_f32(gv[((size_t)tok * H + h) * dv + c]);
-        if (p3) vv *= to_f32(scalar_gates ? gw[(size_t)tok * H + h] : gw[((size_t)tok * H + h) * dv + c]);
+        if (p3) {
+          float ww = to_f32(scalar_gates ? gw[(size_t)tok * H + h] : gw[((size_t)tok * H + h) * dv + c]);
+          if (prolog) ww = sigmoid_f(ww);
+          vv *= ww;
+        }
       }
       sv[e] = vv;
     }
     __syncthreads();
+    if (prolog) {  // L2 norms of the q and k rows (one row per thread); sk, sx, sp are all proportional to k
+      const float *kraw = p3 ? sx : sk;
+      if (tid < C) {
+        float qq = 0.f, kk = 0.f;
+        for (int c = 0; c < dk; ++c) {
+          qq += sq[tid * dk + c] * sq[tid * dk + c];
+          kk += kraw[tid * dk + c] * kraw[tid * dk + c];
+        }
+        const float iq = rsqrtf(qq + kNormEps), ik = rsqrtf(kk + kNormEps);
+        for (int c = 0; c < dk; ++c) {
+          sq[tid * dk + c] *= iq;
+          sk[tid * dk + c] *= ik;
+          sx[tid * dk + c] *= ik;
+          sp[tid * dk + c] *= ik;
+        }
+      }
+      __syncthreads();
+    }
     // 2. inclusive cumulative log-decay per channel
     if (tid < dk) {
       float acc = 0.f;

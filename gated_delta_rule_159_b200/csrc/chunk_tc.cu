@@ -164,7 +164,9 @@ __device__ __forceinline__ uint2 pack4(float a, float b, float c, float d) {
 // (erase read), x_r = p_r = k e^{L_ref - L} (erase and write outer factors) and the
 // values w.v; the host swaps the gate tensor maps so that the gate needed first (b)
 // arrives with the TMA_W group and w with the TMA_X group.
-template <bool kScalarDecay, bool kScalarGates, bool kP3, typename Tout>
+// kProlog: the inputs are pre-activations (GDN2_FUSED_PROLOGUE): log_a <- log sigmoid,
+// b, w <- sigmoid, and the q and k rows are L2-normalised here.
+template <bool kScalarDecay, bool kScalarGates, bool kP3, bool kProlog, typename Tout>
 __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_constant__ TcParams P) {
   extern __shared__ uint8_t smem_raw[];
   const ChunkProblem &p = P.p;
@@ -313,10 +315,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           float4 g = make_float4(0.f, 0.f, 0.f, 0.f);
           if (r < nvalid) {
             if (kScalarDecay) {
-              const float s = __bfloat162float(g_la[(size_t)(t0 + r) * H + h]);
+              float s = __bfloat162float(g_la[(size_t)(t0 + r) * H + h]);
+              if (kProlog) s = log_sigmoid_f(s);
               g = make_float4(s, s, s, s);
             } else {
               g = unpack4(lds_v2(sb + OFF_G + kb * 8192 + swz(r, ch16) + cofs));
+              if (kProlog) g = make_float4(log_sigmoid_f(g.x), log_sigmoid_f(g.y), log_sigmoid_f(g.z), log_sigmoid_f(g.w));
             }
           }
           acc.x += g.x; acc.y += g.y; acc.z += g.z; acc.w += g.w;
@@ -358,17 +362,31 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           if (kScalarGates) {
             ww = make_float4(0.f, 0.f, 0.f, 0.f);
             if (r < nvalid) {
-              const float swv = __bfloat162float((kP3 ? g_b : g_w)[(size_t)(t0 + r) * H + h]);
+              float swv = __bfloat162float((kP3 ? g_b : g_w)[(size_t)(t0 + r) * H + h]);
+              if (kProlog) swv = sigmoid_f(swv);
               ww = make_float4(swv, swv, swv, swv);
             }
           } else {
             ww = unpack4(lds_v2(sb + OFF_XP + o + 8192));
+            if (kProlog) ww = make_float4(sigmoid_f(ww.x), sigmoid_f(ww.y), sigmoid_f(ww.z), sigmoid_f(ww.w));
           }
           if (r >= nvalid) {
             kk = make_float4(0.f, 0.f, 0.f, 0.f);
             qq = kk;
             ww = kk;
             sts_v2(sb + OFF_V + kb * 8192 + swz(r, ch16) + cofs, make_uint2(0u, 0u));
+          }
+          if (kProlog) {  // the 32 lanes of this warp hold the row's 128 channels
+            float k2 = kk.x * kk.x + kk.y * kk.y + kk.z * kk.z + kk.w * kk.w;
+            float q2 = qq.x * qq.x + qq.y * qq.y + qq.z * qq.z + qq.w * qq.w;
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) {
+              k2 += __shfl_xor_sync(0xffffffffu, k2, off);
+              q2 += __shfl_xor_sync(0xffffffffu, q2, off);
+            }
+            const float ik = rsqrtf(k2 + kNormEps), iq = rsqrtf(q2 + kNormEps);
+            kk = make_float4(kk.x * ik, kk.y * ik, kk.z * ik, kk.w * ik);
+            qq = make_float4(qq.x * iq, qq.y * iq, qq.z * iq, qq.w * iq);
           }
           kraw[rr] = kk;
           const float4 e2 = e2v[rr];
@@ -391,11 +409,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           if (kScalarGates) {
             bb = make_float4(0.f, 0.f, 0.f, 0.f);
             if (r < nvalid) {
-              const float sbv = __bfloat162float((kP3 ? g_w : g_b)[(size_t)(t0 + r) * H + h]);
+              float sbv = __bfloat162float((kP3 ? g_w : g_b)[(size_t)(t0 + r) * H + h]);
+              if (kProlog) sbv = sigmoid_f(sbv);
               bb = make_float4(sbv, sbv, sbv, sbv);
             }
           } else {
             bb = unpack4(lds_v2(sb + OFF_XP + o));
+            if (kProlog) bb = make_float4(sigmoid_f(bb.x), sigmoid_f(bb.y), sigmoid_f(bb.z), sigmoid_f(bb.w));
           }
           const float4 kk = kraw[rr], e2 = e2v[rr];
           if (kP3) {
@@ -834,21 +854,24 @@ bool make_map_o(CUtensorMap *m, void *base, int64_t t_total, int H, bool bf16) {
   return r == CUDA_SUCCESS;
 }
 
-template <bool SD, bool SG, bool P3, typename Tout>
+template <bool SD, bool SG, bool P3, bool PR, typename Tout>
 cudaError_t launch_t(const TcParams &P, int grid, cudaStream_t stream) {
-  auto kern = chunk_tc_kernel<SD, SG, P3, Tout>;
+  auto kern = chunk_tc_kernel<SD, SG, P3, PR, Tout>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, kSmemBytes, stream>>>(P);
   return cudaGetLastError();
 }
 
-template <bool P3>
+template <bool P3, bool PR>
 cudaError_t launch_gates(const TcParams &P, int grid, cudaStream_t stream, bool sd, bool sg, bool obf) {
-  if (sd && sg) return obf ? launch_t<true, true, P3, __nv_bfloat16>(P, grid, stream) : launch_t<true, true, P3, float>(P, grid, stream);
-  if (sd) return obf ? launch_t<true, false, P3, __nv_bfloat16>(P, grid, stream) : launch_t<true, false, P3, float>(P, grid, stream);
-  if (sg) return obf ? launch_t<false, true, P3, __nv_bfloat16>(P, grid, stream) : launch_t<false, true, P3, float>(P, grid, stream);
-  return obf ? launch_t<false, false, P3, __nv_bfloat16>(P, grid, stream) : launch_t<false, false, P3, float>(P, grid, stream);
+  if (sd && sg)
+    return obf ? launch_t<true, true, P3, PR, __nv_bfloat16>(P, grid, stream) : launch_t<true, true, P3, PR, float>(P, grid, stream);
+  if (sd)
+    return obf ? launch_t<true, false, P3, PR, __nv_bfloat16>(P, grid, stream) : launch_t<true, false, P3, PR, float>(P, grid, stream);
+  if (sg)
+    return obf ? launch_t<false, true, P3, PR, __nv_bfloat16>(P, grid, stream) : launch_t<false, true, P3, PR, float>(P, grid, stream);
+  return obf ? launch_t<false, false, P3, PR, __nv_bfloat16>(P, grid, stream) : launch_t<false, false, P3, PR, float>(P, grid, stream);
 }
 
 }  // namespace
@@ -891,7 +914,9 @@ cudaError_t launch_chunk_tc(const ChunkProblem &p, cudaStream_t stream, const ch
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = P.n_units < sms ? P.n_units : sms;
   const bool obf = p.dtype_out == GDN2_BF16;
-  return p3 ? launch_gates<true>(P, grid, stream, sd, sg, obf) : launch_gates<false>(P, grid, stream, sd, sg, obf);
+  const bool pr = (p.flags & GDN2_FUSED_PROLOGUE) != 0;
+  if (p3) return pr ? launch_gates<true, true>(P, grid, stream, sd, sg, obf) : launch_gates<true, false>(P, grid, stream, sd, sg, obf);
+  return pr ? launch_gates<false, true>(P, grid, stream, sd, sg, obf) : launch_gates<false, false>(P, grid, stream, sd, sg, obf);
 }
 
 }  // namespace gdn2

@@ -14,6 +14,15 @@ constexpr float kLog2e = 1.4426950408889634f;
 // exp(x) via the hardware base-2 exponential: exp(x) = 2^(x * log2(e)).
 __device__ __forceinline__ float exp_fast(float x) { return exp2f(x * kLog2e); }
 
+// Fused prologue (GDN2_FUSED_PROLOGUE): sigmoid gates and the L2 normalisation
+// of q and k, x / sqrt(|x|^2 + kNormEps).
+constexpr float kNormEps = 1e-6f;
+
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.f, 1.f + exp_fast(-x)); }
+
+// log sigmoid(x) = min(x, 0) - log(1 + e^{-|x|}); the argument of the log lies in [1, 2].
+__device__ __forceinline__ float log_sigmoid_f(float x) { return fminf(x, 0.f) - __logf(1.f + exp_fast(-fabsf(x))); }
+
 template <typename T>
 __device__ __forceinline__ float to_f32(T v);
 template <>

@@ -15,31 +15,50 @@
 // which lets the kernel read S only once.
 #include "common.cuh"
 #include "internal.h"
+#include "sm100_ptx.cuh"
 
 namespace gdn2 {
+
+__device__ int g_decode_status = 0;  // kStatusTimeout once a bounded wait of the streaming kernel gave up
+
 namespace {
 
 constexpr int kThreads = 256;
 
-template <int DV, typename Tin, typename Tout>
+// kExt: the gist.science gate placement or the fused prologue may be set (kept out
+// of the default instantiation, whose code they would otherwise slow down).
+template <int DV, bool kIndexed, bool kExt, typename Tin, typename Tout>
 __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeProblem p) {
-  constexpr int G = DV / 4;           // float4 column groups per row
-  constexpr int R = kThreads / G;     // rows covered per pass
+  constexpr int DVT = DV;                 // columns of this CTA (one whole state)
+  constexpr int G = DVT / 4;              // float4 column groups per row
+  constexpr int R = kThreads / G;         // rows covered per pass
   constexpr int MAXIT = (128 + R - 1) / R;
-  const int unit = blockIdx.x;        // n * H + h
+  const int unit = blockIdx.x;            // n * H + h
+  const int c0 = 0;
+  size_t sunit = (size_t)unit;            // state of this (sequence, head)
+  if (kIndexed) {
+    const int n = unit / p.n_heads, slot = p.state_idx[n];
+    if (slot < 0 || slot >= p.n_slots) {  // padding entry: zero output, no state
+      if (threadIdx.x < DV) static_cast<Tout *>(p.o)[(size_t)unit * DV + threadIdx.x] = from_f32<Tout>(0.f);
+      return;
+    }
+    sunit = (size_t)slot * p.n_heads + (size_t)(unit % p.n_heads);
+  }
   const int dk = p.d_k;
   const int t = threadIdx.x, cg = t % G, rg = t / G;
   const bool scalar_decay = (p.flags & GDN2_SCALAR_DECAY) != 0;
   const bool scalar_gates = (p.flags & GDN2_SCALAR_GATES) != 0;
   const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
+  const bool p3 = kExt && (p.flags & GDN2_GATE_FORM_P3) != 0;
+  const bool prolog = kExt && (p.flags & GDN2_FUSED_PROLOGUE) != 0;
 
   __shared__ float s_a[128], s_k[128], s_x[128], s_p[128], s_q[128];
-  __shared__ float s_v[DV];
-  __shared__ __align__(16) float red[2][R][DV];
-  __shared__ __align__(16) float s_r[DV];
-  __shared__ float s_dot[2];
+  __shared__ __align__(16) float s_v[DVT];
+  __shared__ __align__(16) float red[2][R][DVT];
+  __shared__ __align__(16) float s_r[DVT];
+  __shared__ float s_dot[4];  // q.x, q.p, then the 1/|q| and 1/|k| factors of the fused prologue
 
-  float *S = p.S + (size_t)unit * dk * DV;
+  float *S = p.S + sunit * dk * DV + c0;
 
   // Issue the state loads first so their latency overlaps the gate math.
   float4 st[MAXIT];
@@ -51,38 +70,70 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeProblem p) {
 
   const Tin *q = static_cast<const Tin *>(p.q) + (size_t)unit * dk;
   const Tin *k = static_cast<const Tin *>(p.k) + (size_t)unit * dk;
-  const Tin *v = static_cast<const Tin *>(p.v) + (size_t)unit * DV;
+  const Tin *v = static_cast<const Tin *>(p.v) + (size_t)unit * DV + c0;
   const Tin *la = static_cast<const Tin *>(p.log_a);
   const Tin *gb = static_cast<const Tin *>(p.b);
   const Tin *gw = static_cast<const Tin *>(tied ? p.b : p.w);
+  // s_k: erase read vector, s_x: erase outer factor, s_p: write outer factor,
+  // s_v: written value.  Default form (k, b.k, w.k, v); gist.science form
+  // (b.k, k, k, w.v) with w on the d_v axis.  With the fused prologue the gates
+  // are activated here and the L2 norms of q and k enter below as scale factors
+  // (every one of s_k, s_x, s_p is proportional to k).
   if (t < dk) {
     const float kk = to_f32(k[t]);
-    const float g = to_f32(scalar_decay ? la[unit] : la[(size_t)unit * dk + t]);
-    const float bb = to_f32(scalar_gates ? gb[unit] : gb[(size_t)unit * dk + t]);
-    const float ww = to_f32(scalar_gates ? gw[unit] : gw[(size_t)unit * dk + t]);
+    float g = to_f32(scalar_decay ? la[unit] : la[(size_t)unit * dk + t]);
+    float bb = to_f32(scalar_gates ? gb[unit] : gb[(size_t)unit * dk + t]);
+    if (prolog) {
+      g = log_sigmoid_f(g);
+      bb = sigmoid_f(bb);
+    }
     s_a[t] = exp_fast(g);
-    s_k[t] = kk;
-    s_x[t] = bb * kk;
-    s_p[t] = ww * kk;
     s_q[t] = to_f32(q[t]);
+    if (p3) {
+      s_k[t] = bb * kk;
+      s_x[t] = kk;
+      s_p[t] = kk;
+    } else {
+      float ww = to_f32(scalar_gates ? gw[unit] : gw[(size_t)unit * dk + t]);
+      if (prolog) ww = sigmoid_f(ww);
+      s_k[t] = kk;
+      s_x[t] = bb * kk;
+      s_p[t] = ww * kk;
+    }
   }
-  if (t < DV) s_v[t] = to_f32(v[t]);
+  if (t < DVT) {
+    float vv = to_f32(v[t]);
+    if (p3) {
+      float ww = to_f32(scalar_gates ? gw[unit] : gw[(size_t)unit * DV + c0 + t]);
+      if (prolog) ww = sigmoid_f(ww);
+      vv *= ww;
+    }
+    s_v[t] = vv;
+  }
   __syncthreads();
 
-  if (t < 32) {  // q.(b.k) and q.(w.k)
-    float dx = 0.f, dp = 0.f;
+  if (t < 32) {  // q.x and q.p (and |q|^2, |k|^2 for the prologue)
+    float dx = 0.f, dp = 0.f, qq = 0.f, kk = 0.f;
     for (int i = t; i < dk; i += 32) {
       dx += s_q[i] * s_x[i];
       dp += s_q[i] * s_p[i];
+      const float ki = p3 ? s_x[i] : s_k[i];
+      qq += s_q[i] * s_q[i];
+      kk += ki * ki;
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
       dx += __shfl_xor_sync(0xffffffffu, dx, off);
       dp += __shfl_xor_sync(0xffffffffu, dp, off);
+      qq += __shfl_xor_sync(0xffffffffu, qq, off);
+      kk += __shfl_xor_sync(0xffffffffu, kk, off);
     }
     if (t == 0) {
-      s_dot[0] = dx;
-      s_dot[1] = dp;
+      const float iq = prolog ? rsqrtf(qq + kNormEps) : 1.f, ik = prolog ? rsqrtf(kk + kNormEps) : 1.f;
+      s_dot[0] = dx * iq * ik;
+      s_dot[1] = dp * iq * ik;
+      s_dot[2] = iq;
+      s_dot[3] = ik;
     }
   }
 
@@ -104,21 +155,27 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeProblem p) {
   reinterpret_cast<float4 *>(red[1][rg])[cg] = u4;
   __syncthreads();
 
-  if (t < DV) {
+  if (t < DVT) {
     float r = 0.f, u = 0.f;
 #pragma unroll
     for (int g = 0; g < R; ++g) {
       r += red[0][g][t];
       u += red[1][g][t];
     }
+    r *= s_dot[3];
+    u *= s_dot[2];
     s_r[t] = r;
     const float o = u - s_dot[0] * r + s_dot[1] * s_v[t];
-    static_cast<Tout *>(p.o)[(size_t)unit * DV + t] = from_f32<Tout>(o);
+    static_cast<Tout *>(p.o)[(size_t)unit * DV + c0 + t] = from_f32<Tout>(o);
   }
   __syncthreads();
 
-  const float4 rr = reinterpret_cast<const float4 *>(s_r)[cg];
-  const float4 vv = reinterpret_cast<const float4 *>(s_v)[cg];
+  // x and p are proportional to k: the prologue's 1/|k| scales the outer products
+  const float ik = s_dot[3];
+  float4 rr = reinterpret_cast<const float4 *>(s_r)[cg];
+  float4 vv = reinterpret_cast<const float4 *>(s_v)[cg];
+  rr.x *= ik; rr.y *= ik; rr.z *= ik; rr.w *= ik;
+  vv.x *= ik; vv.y *= ik; vv.z *= ik; vv.w *= ik;
 #pragma unroll
   for (int it = 0; it < MAXIT; ++it) {
     const int i = rg + R * it;
@@ -134,21 +191,237 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeProblem p) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Streaming variant for d_k = d_v = 128 with channel-wise gates: one persistent
+// CTA per SM walks its units in order.  The state (64 KiB) and the six input
+// vectors of a unit arrive by bulk copy into one of kStages shared-memory
+// buffers, issued two units ahead; the update runs out of shared memory and the
+// new state leaves by a bulk store, so every SM keeps loads and a store in
+// flight while it computes.  Same arithmetic as decode_kernel.
+constexpr int kStages = 3;
+constexpr int kSThreads = 256;
+constexpr uint64_t kStreamWaitNs = 1000000000ull;  // bounded waits: 1 s
+
+template <typename Tin>
+struct StreamSmem {
+  float S[kStages][128 * 128];
+  Tin vec[kStages][6][128];  // q, k, v, log_a, b, w
+  float s_a[128], s_k[128], s_x[128], s_p[128], s_q[128], s_v[128], s_r[128];
+  float red[2][kSThreads / 32][128];
+  float s_dot[4];
+  unsigned long long full[kStages];
+};
+
+__device__ __forceinline__ bool stream_wait(uint32_t bar, uint32_t parity) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  uint32_t n = 0;
+  while (!ptx::mbar_try_wait(bar, parity)) {
+    if ((++n & 255u) == 0 && global_timer_ns() - t0 > kStreamWaitNs) return false;
+  }
+  return true;
+}
+
+template <bool kExt, typename Tin, typename Tout>
+__global__ void __launch_bounds__(kSThreads, 1) decode_stream_kernel(DecodeProblem p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  StreamSmem<Tin> &sm = *reinterpret_cast<StreamSmem<Tin> *>(smem_raw);
+  constexpr int G = 32, R = kSThreads / G, MAXIT = 128 / R;
+  constexpr uint32_t kVec = 128 * sizeof(Tin), kState = 128 * 128 * sizeof(float);
+  const int t = threadIdx.x, cg = t % G, rg = t / G;
+  const int units = p.n_seqs * p.n_heads;
+  const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
+  const bool p3 = kExt && (p.flags & GDN2_GATE_FORM_P3) != 0;
+  const bool prolog = kExt && (p.flags & GDN2_FUSED_PROLOGUE) != 0;
+  const Tin *src[6] = {static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k), static_cast<const Tin *>(p.v),
+                       static_cast<const Tin *>(p.log_a), static_cast<const Tin *>(p.b),
+                       static_cast<const Tin *>(tied ? p.b : p.w)};
+  auto bar = [&](int st) { return ptx::smem_u32(&sm.full[st]); };
+  auto issue = [&](int unit, int st) {  // thread 0
+    ptx::mbar_arrive_expect_tx(bar(st), kState + 6u * kVec);
+    ptx::bulk_load(ptx::smem_u32(sm.S[st]), p.S + (size_t)unit * 128 * 128, kState, bar(st));
+#pragma unroll
+    for (int j = 0; j < 6; ++j) ptx::bulk_load(ptx::smem_u32(sm.vec[st][j]), src[j] + (size_t)unit * 128, kVec, bar(st));
+  };
+  if (t == 0) {
+#pragma unroll
+    for (int st = 0; st < kStages; ++st) ptx::mbar_init(bar(st), 1);
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  const int first = blockIdx.x, stride = gridDim.x;
+  if (t == 0)
+    for (int j = 0; j < kStages - 1; ++j)
+      if (first + j * stride < units) issue(first + j * stride, j);
+
+  int it = 0;
+  for (int unit = first; unit < units; unit += stride, ++it) {
+    const int st = it % kStages;
+    const bool ok = stream_wait(bar(st), (uint32_t)(it / kStages) & 1u);
+    if (__syncthreads_or(!ok)) {
+      // give up: record it, let the loads already issued land (bounded), then leave
+      if (t == 0) {
+        atomicExch(&g_decode_status, kStatusTimeout);
+        stream_wait(bar(st), (uint32_t)(it / kStages) & 1u);
+        if (unit + stride < units) stream_wait(bar((it + 1) % kStages), (uint32_t)((it + 1) / kStages) & 1u);
+      }
+      break;
+    }
+    const Tin *vq = sm.vec[st][0], *vk = sm.vec[st][1], *vv = sm.vec[st][2];
+    const Tin *vg = sm.vec[st][3], *vb = sm.vec[st][4], *vw = sm.vec[st][5];
+    if (t < 128) {
+      const float kk = to_f32(vk[t]);
+      float g = to_f32(vg[t]), bb = to_f32(vb[t]), ww = to_f32(vw[t]);
+      if (prolog) {
+        g = log_sigmoid_f(g);
+        bb = sigmoid_f(bb);
+        ww = sigmoid_f(ww);
+      }
+      sm.s_a[t] = exp_fast(g);
+      sm.s_q[t] = to_f32(vq[t]);
+      sm.s_k[t] = p3 ? bb * kk : kk;
+      sm.s_x[t] = p3 ? kk : bb * kk;
+      sm.s_p[t] = p3 ? kk : ww * kk;
+      sm.s_v[t] = p3 ? ww * to_f32(vv[t]) : to_f32(vv[t]);
+    }
+    __syncthreads();
+    if (t < 32) {
+      float dx = 0.f, dp = 0.f, qq = 0.f, k2 = 0.f;
+      for (int i = t; i < 128; i += 32) {
+        dx += sm.s_q[i] * sm.s_x[i];
+        dp += sm.s_q[i] * sm.s_p[i];
+        const float ki = p3 ? sm.s_x[i] : sm.s_k[i];
+        qq += sm.s_q[i] * sm.s_q[i];
+        k2 += ki * ki;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        dx += __shfl_xor_sync(0xffffffffu, dx, off);
+        dp += __shfl_xor_sync(0xffffffffu, dp, off);
+        qq += __shfl_xor_sync(0xffffffffu, qq, off);
+        k2 += __shfl_xor_sync(0xffffffffu, k2, off);
+      }
+      if (t == 0) {
+        const float iq = prolog ? rsqrtf(qq + kNormEps) : 1.f, ik = prolog ? rsqrtf(k2 + kNormEps) : 1.f;
+        sm.s_dot[0] = dx * iq * ik;
+        sm.s_dot[1] = dp * iq * ik;
+        sm.s_dot[2] = iq;
+        sm.s_dot[3] = ik;
+      }
+    }
+    float4 *S4 = reinterpret_cast<float4 *>(sm.S[st]);
+    float4 stv[MAXIT];
+    float4 r4 = make_float4(0.f, 0.f, 0.f, 0.f), u4 = r4;
+#pragma unroll
+    for (int j = 0; j < MAXIT; ++j) {
+      const int i = rg + R * j;
+      const float a = sm.s_a[i], kk = sm.s_k[i], qq = sm.s_q[i];
+      float4 v4 = S4[i * G + cg];
+      v4.x *= a; v4.y *= a; v4.z *= a; v4.w *= a;
+      stv[j] = v4;
+      r4.x += v4.x * kk; r4.y += v4.y * kk; r4.z += v4.z * kk; r4.w += v4.w * kk;
+      u4.x += v4.x * qq; u4.y += v4.y * qq; u4.z += v4.z * qq; u4.w += v4.w * qq;
+    }
+    reinterpret_cast<float4 *>(sm.red[0][rg])[cg] = r4;
+    reinterpret_cast<float4 *>(sm.red[1][rg])[cg] = u4;
+    __syncthreads();
+    if (t < 128) {
+      float r = 0.f, u = 0.f;
+#pragma unroll
+      for (int gi = 0; gi < R; ++gi) {
+        r += sm.red[0][gi][t];
+        u += sm.red[1][gi][t];
+      }
+      r *= sm.s_dot[3];
+      u *= sm.s_dot[2];
+      sm.s_r[t] = r;
+      static_cast<Tout *>(p.o)[(size_t)unit * 128 + t] = from_f32<Tout>(u - sm.s_dot[0] * r + sm.s_dot[1] * sm.s_v[t]);
+    }
+    __syncthreads();
+    {
+      const float ik = sm.s_dot[3];
+      float4 rr = reinterpret_cast<const float4 *>(sm.s_r)[cg];
+      float4 vvv = reinterpret_cast<const float4 *>(sm.s_v)[cg];
+      rr.x *= ik; rr.y *= ik; rr.z *= ik; rr.w *= ik;
+      vvv.x *= ik; vvv.y *= ik; vvv.z *= ik; vvv.w *= ik;
+#pragma unroll
+      for (int j = 0; j < MAXIT; ++j) {
+        const int i = rg + R * j;
+        const float x = sm.s_x[i], pp = sm.s_p[i];
+        float4 v4 = stv[j];
+        v4.x += pp * vvv.x - x * rr.x;
+        v4.y += pp * vvv.y - x * rr.y;
+        v4.z += pp * vvv.z - x * rr.z;
+        v4.w += pp * vvv.w - x * rr.w;
+        S4[i * G + cg] = v4;
+      }
+    }
+    ptx::fence_proxy_async_smem();  // the bulk store below reads what the threads just wrote
+    __syncthreads();
+    if (t == 0) {
+      ptx::bulk_store(p.S + (size_t)unit * 128 * 128, ptx::smem_u32(sm.S[st]), kState);
+      ptx::bulk_commit_group();
+      const int nu = unit + (kStages - 1) * stride;
+      if (nu < units) {
+        ptx::bulk_wait_group_read1();  // the store issued one unit ago has left that buffer
+        issue(nu, (it + kStages - 1) % kStages);
+      }
+    }
+  }
+  if (t == 0) ptx::bulk_wait_group0();
+}
+
+template <bool kExt, typename Tin, typename Tout>
+cudaError_t launch_stream_t(const DecodeProblem &p, cudaStream_t stream) {
+  auto kern = decode_stream_kernel<kExt, Tin, Tout>;
+  const int smem = (int)sizeof(StreamSmem<Tin>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int units = p.n_seqs * p.n_heads;
+  kern<<<units < sms ? units : sms, kSThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <int DV, bool kIndexed, bool kExt>
+cudaError_t launch_types(const DecodeProblem &p, unsigned grid, cudaStream_t stream) {
+  const bool in_bf = p.dtype_in == GDN2_BF16, out_bf = p.dtype_out == GDN2_BF16;
+  if (in_bf && out_bf) decode_kernel<DV, kIndexed, kExt, __nv_bfloat16, __nv_bfloat16><<<grid, kThreads, 0, stream>>>(p);
+  else if (in_bf) decode_kernel<DV, kIndexed, kExt, __nv_bfloat16, float><<<grid, kThreads, 0, stream>>>(p);
+  else if (out_bf) decode_kernel<DV, kIndexed, kExt, float, __nv_bfloat16><<<grid, kThreads, 0, stream>>>(p);
+  else decode_kernel<DV, kIndexed, kExt, float, float><<<grid, kThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
 template <int DV>
 cudaError_t launch_dv(const DecodeProblem &p, cudaStream_t stream) {
   const unsigned grid = (unsigned)(p.n_seqs * p.n_heads);
   if (grid == 0) return cudaSuccess;
-  const bool in_bf = p.dtype_in == GDN2_BF16, out_bf = p.dtype_out == GDN2_BF16;
-  if (in_bf && out_bf) decode_kernel<DV, __nv_bfloat16, __nv_bfloat16><<<grid, kThreads, 0, stream>>>(p);
-  else if (in_bf) decode_kernel<DV, __nv_bfloat16, float><<<grid, kThreads, 0, stream>>>(p);
-  else if (out_bf) decode_kernel<DV, float, __nv_bfloat16><<<grid, kThreads, 0, stream>>>(p);
-  else decode_kernel<DV, float, float><<<grid, kThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  const bool ext = (p.flags & (GDN2_GATE_FORM_P3 | GDN2_FUSED_PROLOGUE)) != 0;
+  if (p.state_idx)
+    return ext ? launch_types<DV, true, true>(p, grid, stream) : launch_types<DV, true, false>(p, grid, stream);
+  return ext ? launch_types<DV, false, true>(p, grid, stream) : launch_types<DV, false, false>(p, grid, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream) {
+  const bool channel_gates = (p.flags & (GDN2_SCALAR_DECAY | GDN2_SCALAR_GATES)) == 0;
+  if (p.d_k == 128 && p.d_v == 128 && !p.state_idx && channel_gates && p.n_seqs * p.n_heads > 0) {
+    const bool in_bf = p.dtype_in == GDN2_BF16, out_bf = p.dtype_out == GDN2_BF16;
+    if ((p.flags & (GDN2_GATE_FORM_P3 | GDN2_FUSED_PROLOGUE)) != 0) {
+      if (in_bf && out_bf) return launch_stream_t<true, __nv_bfloat16, __nv_bfloat16>(p, stream);
+      if (in_bf) return launch_stream_t<true, __nv_bfloat16, float>(p, stream);
+      if (out_bf) return launch_stream_t<true, float, __nv_bfloat16>(p, stream);
+      return launch_stream_t<true, float, float>(p, stream);
+    }
+    if (in_bf && out_bf) return launch_stream_t<false, __nv_bfloat16, __nv_bfloat16>(p, stream);
+    if (in_bf) return launch_stream_t<false, __nv_bfloat16, float>(p, stream);
+    if (out_bf) return launch_stream_t<false, float, __nv_bfloat16>(p, stream);
+    return launch_stream_t<false, float, float>(p, stream);
+  }
   switch (p.d_v) {
     case 16: return launch_dv<16>(p, stream);
     case 32: return launch_dv<32>(p, stream);
@@ -158,4 +431,21 @@ cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream) {
   }
 }
 
+}  // namespace gdn2
+
+namespace gdn2 {
+int read_decode_status(cudaStream_t stream, int32_t *out) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return (int)e;
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_decode_status, sizeof(int));
+  if (e != cudaSuccess) return (int)e;
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_decode_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return (int)e;
+  }
+  *out = v;
+  return 0;
+}
 }  // namespace gdn2

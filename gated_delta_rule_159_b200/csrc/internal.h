@@ -33,15 +33,45 @@ struct DecodeProblem {
   int n_seqs, n_heads, d_k, d_v;
   int dtype_in, dtype_out;
   uint32_t flags;
+  const int32_t *state_idx;  // NULL: sequence n owns state n; else slot state_idx[n] of S
+  int n_slots;               // slots in S when state_idx is set
+};
+
+struct BwdProblem {
+  const void *q, *k, *v, *log_a, *b, *w;  // forward inputs (dtype_in)
+  const float *S0;                        // [N, H, d_k, d_v] or NULL
+  const int32_t *cu_seqlens;              // device [N + 1] or NULL
+  const void *dO;                         // [T_tot, H, d_v] (dtype_out)
+  const float *dS_T;                      // [N, H, d_k, d_v] or NULL
+  void *dq, *dk, *dv, *dlog_a, *db, *dw;  // gradients (dtype_out), shaped like the inputs
+  float *dS0;                             // [N, H, d_k, d_v] or NULL
+  float *ckpt, *part, *dz;                // workspace pieces (bwd_carve)
+  float *prolog;                          // workspace for the fused prologue's copies, or NULL
+  const float *inv_norm;                  // [T_tot, H, 2] 1/|q|, 1/|k| when the prologue ran, else NULL
+  int n_seqs, seq_len, n_heads, d_k, d_v;
+  int64_t t_total;
+  int dtype_in, dtype_out;
+  uint32_t flags;
 };
 
 // Status word values written by kernels (0 = fine).
 constexpr int32_t kStatusTimeout = 1;
 
+// Activated fp32 copies of the inputs written by the backward's prologue pass.
+struct PrologueCopies {
+  float *q, *k, *v, *log_a, *b, *w, *inv_norm;
+};
+
+size_t bwd_workspace_bytes(int64_t n_seqs, int64_t t_total, int n_heads, int d_k, int d_v, uint32_t flags);
+void bwd_carve(BwdProblem &p, void *workspace);
+cudaError_t launch_bwd(const BwdProblem &p, cudaStream_t stream);
+
 // Record `message` as this thread's gdn2_last_error() text and return `code`.
 int set_last_error(int code, const char *message);
 
 cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream);
+// Synchronise `stream`, read and clear the decode status word; returns a cudaError_t value.
+int read_decode_status(cudaStream_t stream, int32_t *out);
 cudaError_t launch_chunk_simt(const ChunkProblem &p, cudaStream_t stream);
 // Tensor-core path (d_k = d_v = 128, C = 64, bf16 in).  Returns cudaErrorNotSupported
 // when the problem is outside what it handles.

@@ -76,6 +76,24 @@ __device__ __forceinline__ void bulk_wait_group_read0() {
 }
 // Wait until all committed bulk stores have completed.
 __device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Wait until the shared-memory sources of all but the most recent committed bulk group have been read.
+__device__ __forceinline__ void bulk_wait_group_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+// Untiled bulk copies (no tensor map): both addresses 16-byte aligned, size a multiple of 16.
+// Global -> shared, completion counted on an mbarrier of this CTA.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+// Shared -> global, completion through the bulk-group mechanism.
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
+               "r"(src), "r"(bytes)
+               : "memory");
+}
 
 // ---------------------------------------------------------------- TMEM
 // Allocation / deallocation are warp-wide (.sync.aligned).

@@ -29,9 +29,12 @@ SCALAR_DECAY = 1
 SCALAR_GATES = 2
 TIED_GATES = 4
 GATE_FORM_P3 = 8
+FUSED_PROLOGUE = 16
 
 EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_workspace_size", "gdn2_check_status",
-            "gdn2_decode_step", "gdn2_last_error", "gdn2_version")
+            "gdn2_decode_step", "gdn2_decode_step_indexed", "gdn2_decode_status", "gdn2_bwd",
+            "gdn2_bwd_workspace_size",
+            "gdn2_last_error", "gdn2_version")
 
 
 class Dims(ctypes.Structure):
@@ -60,6 +63,15 @@ def _load():
     lib.gdn2_check_status.argtypes = [vp, vp]
     lib.gdn2_decode_step.restype = ctypes.c_int
     lib.gdn2_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(Dims), vp]
+    lib.gdn2_decode_step_indexed.restype = ctypes.c_int
+    lib.gdn2_decode_step_indexed.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_int32, vp, vp,
+                                             ctypes.POINTER(Dims), vp]
+    lib.gdn2_decode_status.restype = ctypes.c_int
+    lib.gdn2_decode_status.argtypes = [vp]
+    lib.gdn2_bwd.restype = ctypes.c_int
+    lib.gdn2_bwd.argtypes = [vp] * 17 + [ctypes.POINTER(Dims), vp, sz, vp]
+    lib.gdn2_bwd_workspace_size.restype = sz
+    lib.gdn2_bwd_workspace_size.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32]
     lib.gdn2_last_error.restype = ctypes.c_char_p
     lib.gdn2_last_error.argtypes = []
     lib.gdn2_version.restype = ctypes.c_int
@@ -106,9 +118,11 @@ def make_dims(n_seqs, seq_len, n_heads, d_k, d_v, chunk, dtype_in, dtype_out, fl
                 int(dtype_out), int(flags), 0)
 
 
-def flags_of(scalar_decay=False, scalar_gates=False, tied_gates=False, gate_form_p3=False) -> int:
+def flags_of(scalar_decay=False, scalar_gates=False, tied_gates=False, gate_form_p3=False,
+             fused_prologue=False) -> int:
     return (SCALAR_DECAY if scalar_decay else 0) | (SCALAR_GATES if scalar_gates else 0) | \
-           (TIED_GATES if tied_gates else 0) | (GATE_FORM_P3 if gate_form_p3 else 0)
+           (TIED_GATES if tied_gates else 0) | (GATE_FORM_P3 if gate_form_p3 else 0) | \
+           (FUSED_PROLOGUE if fused_prologue else 0)
 
 
 def workspace_size(dims: Dims) -> int:
@@ -119,7 +133,8 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Te
               w: Optional[torch.Tensor] = None, S0: Optional[torch.Tensor] = None,
               cu_seqlens: Optional[torch.Tensor] = None, *, chunk: int = 64, scalar_decay: bool = False,
               scalar_gates: bool = False, tied_gates: bool = False, gate_form_p3: bool = False,
-              out_dtype: Optional[torch.dtype] = None, output_final_state: bool = True, cu_seqlens_host: Optional[Sequence[int]] = None,
+              fused_prologue: bool = False, out_dtype: Optional[torch.dtype] = None,
+              output_final_state: bool = True, cu_seqlens_host: Optional[Sequence[int]] = None,
               o: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
               workspace: Optional[torch.Tensor] = None):
     """Chunked GDN-2 forward through ``gdn2_chunk_fwd``.
@@ -149,7 +164,7 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Te
         raise ValueError("q must be [B, T, H, d_k] or [T_tot, H, d_k]")
     dv = v.shape[-1]
     out_dtype = q.dtype if out_dtype is None else out_dtype
-    flags = flags_of(scalar_decay, scalar_gates, tied_gates, gate_form_p3)
+    flags = flags_of(scalar_decay, scalar_gates, tied_gates, gate_form_p3, fused_prologue)
     dims = make_dims(N, seq_len, H, dk, dv, chunk, _dtype_code(q.dtype), _dtype_code(out_dtype), flags)
     dev = q.device
     if o is None:
@@ -168,6 +183,12 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Te
     return o, S_T
 
 
+def decode_status(device=None) -> int:
+    """Synchronise and read (and clear) the decode kernels' status: OK or ERR_TIMEOUT."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    return int(lib.gdn2_decode_status(_stream(dev)))
+
+
 def check_status(workspace: torch.Tensor) -> int:
     """Synchronise and read the device status left in ``workspace`` by chunk_fwd."""
     return int(lib.gdn2_check_status(_ptr(workspace), _stream(workspace.device)))
@@ -176,6 +197,7 @@ def check_status(workspace: torch.Tensor) -> int:
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, b: torch.Tensor,
                 w: Optional[torch.Tensor], S: torch.Tensor, *, scalar_decay: bool = False,
                 scalar_gates: bool = False, tied_gates: bool = False, gate_form_p3: bool = False,
+              fused_prologue: bool = False,
                 out_dtype: torch.dtype = torch.float32, o: Optional[torch.Tensor] = None) -> torch.Tensor:
     """One recurrent step through ``gdn2_decode_step``; ``S`` [N, H, d_k, d_v] fp32 is updated in place.
 
@@ -185,7 +207,7 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.
     """
     N, H, dk = q.shape
     dv = v.shape[-1]
-    flags = flags_of(scalar_decay, scalar_gates, tied_gates, gate_form_p3)
+    flags = flags_of(scalar_decay, scalar_gates, tied_gates, gate_form_p3, fused_prologue)
     dims = make_dims(N, 1, H, dk, dv, 0, _dtype_code(q.dtype), _dtype_code(out_dtype), flags)
     if o is None:
         o = torch.empty(N, H, dv, dtype=out_dtype, device=q.device)
@@ -193,6 +215,69 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.
                               ctypes.byref(dims), _stream(q.device))
     _check(rc)
     return o
+
+
+def decode_step_indexed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, b: torch.Tensor,
+                        w: Optional[torch.Tensor], S_pool: torch.Tensor, state_idx: torch.Tensor, *,
+                        scalar_decay: bool = False, scalar_gates: bool = False, tied_gates: bool = False,
+                        gate_form_p3: bool = False, fused_prologue: bool = False,
+                        out_dtype: torch.dtype = torch.float32,
+                        o: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One recurrent step through ``gdn2_decode_step_indexed``: row n uses slot
+    ``state_idx[n]`` (int32 on the device) of ``S_pool`` [P, H, d_k, d_v] fp32, updated in
+    place; an index outside [0, P) is a padding row (o row zero, no state touched)."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if state_idx.dtype != torch.int32 or state_idx.numel() != N:
+        raise TypeError("state_idx must be int32 with one entry per row")
+    flags = flags_of(scalar_decay, scalar_gates, tied_gates, gate_form_p3, fused_prologue)
+    dims = make_dims(N, 1, H, dk, dv, 0, _dtype_code(q.dtype), _dtype_code(out_dtype), flags)
+    if o is None:
+        o = torch.empty(N, H, dv, dtype=out_dtype, device=q.device)
+    rc = lib.gdn2_decode_step_indexed(_ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(b), _ptr(w), _ptr(S_pool),
+                                      int(S_pool.shape[0]), _ptr(state_idx), _ptr(o), ctypes.byref(dims),
+                                      _stream(q.device))
+    _check(rc)
+    return o
+
+
+def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, b: torch.Tensor,
+        w: Optional[torch.Tensor], dO: torch.Tensor, S0: Optional[torch.Tensor] = None,
+        dS_T: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None, *,
+        scalar_decay: bool = False, scalar_gates: bool = False, tied_gates: bool = False,
+        gate_form_p3: bool = False, fused_prologue: bool = False, need_dS0: bool = True,
+        workspace: Optional[torch.Tensor] = None) -> dict:
+    """Gradients through ``gdn2_bwd`` of  sum <dO, o> + <dS_T, S_T>  for the forward with the
+    same inputs (layouts as ``chunk_fwd``).  Gradients take dO's dtype.  Returns a dict with
+    dq, dk, dv, dlog_a, db, dw (None with ``tied_gates``: its gradient is added into db) and
+    dS0 (fp32, None unless ``need_dS0``)."""
+    if q.dim() == 4:
+        N, T, H, dk = q.shape
+        seq_len = T
+    elif cu_seqlens is None:
+        N, (T, H, dk) = 1, q.shape
+        seq_len = T
+    else:
+        N = cu_seqlens.numel() - 1
+        seq_len, H, dk = q.shape
+    dv = v.shape[-1]
+    flags = flags_of(scalar_decay, scalar_gates, tied_gates, gate_form_p3, fused_prologue)
+    dims = make_dims(N, seq_len, H, dk, dv, 0, _dtype_code(q.dtype), _dtype_code(dO.dtype), flags)
+    dev = q.device
+    g = dict(dq=torch.empty_like(q, dtype=dO.dtype), dk=torch.empty_like(k, dtype=dO.dtype),
+             dv=torch.empty_like(v, dtype=dO.dtype), dlog_a=torch.empty_like(log_a, dtype=dO.dtype),
+             db=torch.empty_like(b, dtype=dO.dtype),
+             dw=None if tied_gates else torch.empty_like(w, dtype=dO.dtype),
+             dS0=torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev) if need_dS0 else None)
+    if workspace is None:
+        ws = int(lib.gdn2_bwd_workspace_size(ctypes.byref(dims), 1 if cu_seqlens is not None else 0))
+        workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+    rc = lib.gdn2_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(b), _ptr(w), _ptr(S0), _ptr(cu_seqlens),
+                      _ptr(dO), _ptr(dS_T), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_a"]),
+                      _ptr(g["db"]), _ptr(g["dw"]), _ptr(g["dS0"]), ctypes.byref(dims), _ptr(workspace),
+                      workspace.numel(), _stream(dev))
+    _check(rc)
+    return g
 
 
 def version() -> int:

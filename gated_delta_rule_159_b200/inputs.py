@@ -99,10 +99,13 @@ def _l2n(x: torch.Tensor) -> torch.Tensor:
 
 def make_inputs(workload, device="cuda", seed: int = 0, seq_len: Optional[int] = None,
                 n_seqs: Optional[int] = None, lengths: Optional[List[int]] = None,
-                gate_form_p3: bool = False) -> dict:
+                gate_form_p3: bool = False, fused_prologue: bool = False) -> dict:
     """Inputs of a workload (by name or ``Workload``).  ``seq_len``/``n_seqs``/``lengths``
     override the sizes (smaller parity cases with the same distributions).  With
-    ``gate_form_p3`` the write gate w has d_v channels (the gist.science placement)."""
+    ``gate_form_p3`` the write gate w has d_v channels (the gist.science placement).
+    With ``fused_prologue`` q, k, log_a, b, w are pre-activations: q, k ~ 2 N(0, 1)
+    (not normalised), the decay pre-activation ~ N(3, 1) (sigmoid about 0.95) and the
+    gate pre-activations ~ N(0, 1); draws keep the same order."""
     w = WORKLOADS[workload] if isinstance(workload, str) else workload
     device = torch.device(device)
     H, dk, dv = w.n_heads, w.d_k, w.d_v
@@ -118,14 +121,22 @@ def make_inputs(workload, device="cuda", seed: int = 0, seq_len: Optional[int] =
         cu = np.arange(N + 1, dtype=np.int64) * T
         T_tot = N * T
     g = _gen(device, seed)
-    q = _l2n(_randn((T_tot, H, dk), g, device)).to(w.dtype)
-    k = _l2n(_randn((T_tot, H, dk), g, device)).to(w.dtype)
-    v = _randn((T_tot, H, dv), g, device).to(w.dtype)
     gshape = (T_tot, H) if w.scalar_gates else (T_tot, H, dk)
-    log_a = (-torch.nn.functional.softplus(_randn(gshape, g, device)) * w.decay_scale).to(w.dtype)
-    b = torch.sigmoid(_randn(gshape, g, device)).to(w.dtype)
     wshape = (T_tot, H, dv) if gate_form_p3 else gshape
-    wg = None if w.scalar_gates else torch.sigmoid(_randn(wshape, g, device)).to(w.dtype)
+    if fused_prologue:
+        q = (_randn((T_tot, H, dk), g, device) * 2).to(w.dtype)
+        k = (_randn((T_tot, H, dk), g, device) * 2).to(w.dtype)
+        v = _randn((T_tot, H, dv), g, device).to(w.dtype)
+        log_a = (_randn(gshape, g, device) + 3.0).to(w.dtype)
+        b = _randn(gshape, g, device).to(w.dtype)
+        wg = None if w.scalar_gates else _randn(wshape, g, device).to(w.dtype)
+    else:
+        q = _l2n(_randn((T_tot, H, dk), g, device)).to(w.dtype)
+        k = _l2n(_randn((T_tot, H, dk), g, device)).to(w.dtype)
+        v = _randn((T_tot, H, dv), g, device).to(w.dtype)
+        log_a = (-torch.nn.functional.softplus(_randn(gshape, g, device)) * w.decay_scale).to(w.dtype)
+        b = torch.sigmoid(_randn(gshape, g, device)).to(w.dtype)
+        wg = None if w.scalar_gates else torch.sigmoid(_randn(wshape, g, device)).to(w.dtype)
     S0 = (_randn((N, H, dk, dv), g, device) * w.s0_std) if w.s0_std > 0 else None
     equal = lengths is None
     return dict(
@@ -133,7 +144,7 @@ def make_inputs(workload, device="cuda", seed: int = 0, seq_len: Optional[int] =
         cu_seqlens=None if equal else torch.tensor(cu, dtype=torch.int32, device=device),
         cu_host=cu.tolist(), n_seqs=N, T_tot=T_tot, equal_lengths=equal,
         scalar_decay=w.scalar_gates, scalar_gates=w.scalar_gates, tied_gates=w.scalar_gates,
-        gate_form_p3=gate_form_p3,
+        gate_form_p3=gate_form_p3, fused_prologue=fused_prologue,
     )
 
 

@@ -76,8 +76,14 @@ enum gdn2_flags {
   GDN2_SCALAR_DECAY = 1u,  /* log_a is [T_tot, H]: one decay per token and head (a = alpha 1) */
   GDN2_SCALAR_GATES = 2u,  /* b and w are [T_tot, H]: one erase and one write gate per token and head */
   GDN2_TIED_GATES = 4u,    /* w is b (the w pointer is ignored and may be NULL) */
-  GDN2_GATE_FORM_P3 = 8u   /* gist.science gate placement (above): w is [T_tot, H, d_v]; with
+  GDN2_GATE_FORM_P3 = 8u,  /* gist.science gate placement (above): w is [T_tot, H, d_v]; with
                               GDN2_TIED_GATES and per-channel gates it needs d_k == d_v */
+  GDN2_FUSED_PROLOGUE = 16u /* q, k, log_a, b, w carry pre-activations and the kernels apply the
+                              mixer's activations (neelmishra.github.io, "What makes the architecture
+                              more than a recurrence" and "Read the limiting cases"):
+                              q <- q / sqrt(|q|^2 + 1e-6), k likewise (over d_k);
+                              log_a <- log sigmoid(log_a); b <- sigmoid(b); w <- sigmoid(w).
+                              The range precondition on log_a applies to the activated values. */
 };
 
 /*
@@ -169,6 +175,72 @@ int gdn2_check_status(const void *workspace, gdn2_stream_t stream);
 int gdn2_decode_step(const void *q, const void *k, const void *v,
                      const void *log_a, const void *b, const void *w,
                      float *S, void *o, const gdn2_dims *dims, gdn2_stream_t stream);
+
+/*
+ * gdn2_decode_status -- synchronise `stream`, then report whether any decode
+ * step since the last call gave up a bounded device-side wait (the d_k = d_v =
+ * 128 decode streams each state through shared memory with bulk copies and
+ * waits at most 1 s for each).  Returns GDN2_OK or GDN2_ERR_TIMEOUT (and clears
+ * the record), or GDN2_ERR_CUDA.  Optional, like gdn2_check_status.
+ */
+int gdn2_decode_status(gdn2_stream_t stream);
+
+/*
+ * gdn2_decode_step_indexed -- gdn2_decode_step for continuous batching: the N
+ * sequences of this step live in a pool of state slots and sequence n reads and
+ * updates slot state_idx[n].  The per-step operation is the same recurrent
+ * step (alanhou.org "Core Mechanism": O(1) state per sequence at inference);
+ * the pages define no batching scheme, the indirection is this library's.
+ *   q, k, v, log_a, b, w, o   as gdn2_decode_step, N = dims.n_seqs rows
+ *   S_pool      [n_slots, H, d_k, d_v] fp32 device, updated in place (only the
+ *               slots named by state_idx are touched)
+ *   n_slots     number of slots in S_pool (>= 1)
+ *   state_idx   device int32 [N]: slot of sequence n.  An entry outside
+ *               [0, n_slots) marks a padding row: its o row is set to zero and
+ *               no state is read or written.  Two rows naming the same slot in
+ *               one call race on that slot (the result is undefined).
+ * Errors: GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_CUDA.
+ */
+int gdn2_decode_step_indexed(const void *q, const void *k, const void *v,
+                             const void *log_a, const void *b, const void *w,
+                             float *S_pool, int32_t n_slots, const int32_t *state_idx, void *o,
+                             const gdn2_dims *dims, gdn2_stream_t stream);
+
+/*
+ * gdn2_bwd -- gradients of the forward (gdn2_chunk_fwd with the same inputs)
+ * for training.  The method's training path runs a gate-aware backward of its
+ * chunked form (gist.science Methodologie 3; alanhou.org "Core Mechanism"),
+ * whose formula the pages do not print; the gradient is fixed by the forward,
+ * and this call computes it by reverse-mode differentiation of the recurrence
+ * token by token (fp32), recomputing the states from checkpoints kept every 4
+ * tokens in the workspace.  It returns the gradients of
+ *     sum_t <dO_t, o_t> + sum_n <dS_T[n], S_T[n]>.
+ * Arguments (T_tot as for gdn2_chunk_fwd; all device pointers, caller-owned):
+ *   q, k, v, log_a, b, w, S0, cu_seqlens   the forward's inputs, same layouts and flags
+ *                                         (dims.chunk is ignored)
+ *   dO       [T_tot, H, d_v] dtype_out    gradient of o
+ *   dS_T     [N, H, d_k, d_v] fp32 or NULL (zero)
+ *   dq, dk, dlog_a, db, dw, dv            written, dtype_out, each shaped like its input
+ *                                         (scalar-flag gates give [T_tot, H]); with
+ *                                         GDN2_TIED_GATES the w gradient is added into db
+ *                                         and dw may be NULL
+ *   dS0      [N, H, d_k, d_v] fp32 or NULL to skip
+ *   workspace  >= gdn2_bwd_workspace_size(dims) bytes, 256-byte aligned, uninitialised
+ *              is fine; one call at a time per workspace
+ * Supported: d_k <= 128, d_v in {16, 32, 64, 128}, bf16 or fp32 in and out.
+ * Errors: GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_WORKSPACE, GDN2_ERR_CUDA.
+ */
+int gdn2_bwd(const void *q, const void *k, const void *v,
+             const void *log_a, const void *b, const void *w,
+             const float *S0, const int32_t *cu_seqlens,
+             const void *dO, const float *dS_T,
+             void *dq, void *dk, void *dv, void *dlog_a, void *db, void *dw, float *dS0,
+             const gdn2_dims *dims, void *workspace, size_t workspace_bytes, gdn2_stream_t stream);
+
+/* Bytes of device workspace gdn2_bwd needs for `dims` (0 if dims are unsupported).
+ * packed != 0: the call passes cu_seqlens, so dims.seq_len is T_tot; packed == 0:
+ * N equal sequences of dims.seq_len tokens. */
+size_t gdn2_bwd_workspace_size(const gdn2_dims *dims, int32_t packed);
 
 /*
  * gdn2_chunk_fwd_noalloc -- gdn2_chunk_fwd for callers that cannot allocate

@@ -115,7 +115,54 @@ def test_decode_rejects_bad_arguments(g):
     assert call(_dims(g, seq_len=1, flags=g.TIED_GATES), w=None, o=ctypes.c_void_p(3)) == g.ERR_INVALID_ARG
 
 
+def test_decode_indexed_rejects_bad_arguments(g):
+    def call(dims, n_slots=4, **kw):
+        a = dict(q=P, k=P, v=P, log_a=P, b=P, w=P, S=P, idx=P, o=P)
+        a.update(kw)
+        return g.lib.gdn2_decode_step_indexed(a["q"], a["k"], a["v"], a["log_a"], a["b"], a["w"], a["S"], n_slots,
+                                              a["idx"], a["o"], ctypes.byref(dims), None)
+    assert call(_dims(g, seq_len=1), idx=None) == g.ERR_INVALID_ARG
+    assert call(_dims(g, seq_len=1), idx=ctypes.c_void_p((1 << 20) + 2)) == g.ERR_INVALID_ARG
+    assert call(_dims(g, seq_len=1), n_slots=0) == g.ERR_INVALID_ARG
+    assert call(_dims(g, seq_len=1), S=None) == g.ERR_INVALID_ARG
+    assert call(_dims(g, seq_len=3)) == g.ERR_INVALID_ARG
+    assert call(_dims(g, seq_len=1, d_v=96)) == g.ERR_UNSUPPORTED
+
+
 def test_last_error_is_cleared(g):
     _chunk(g, _dims(g, n_seqs=0))
     assert g.lib.gdn2_last_error().decode()
     assert g.lib.gdn2_chunk_fwd_workspace_size(ctypes.byref(_dims(g))) > 0
+
+
+def test_bwd_workspace_size(g):
+    lib = g.lib
+    d = _dims(g, n_seqs=2, seq_len=100, n_heads=3, d_k=128, d_v=128)
+    eq = lib.gdn2_bwd_workspace_size(ctypes.byref(d), 0)          # 2 x 100 tokens
+    d2 = _dims(g, n_seqs=2, seq_len=200, n_heads=3, d_k=128, d_v=128)
+    packed = lib.gdn2_bwd_workspace_size(ctypes.byref(d2), 1)     # 200 tokens packed
+    assert eq == packed > 0
+    ckpt = (200 // 4 + 2) * 3 * 128 * 128 * 4
+    part = 4 * 200 * 3 * 5 * 128 * 4
+    dz = 200 * 3 * 128 * 4
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert eq == up(ckpt) + up(part) + up(dz)
+    assert lib.gdn2_bwd_workspace_size(ctypes.byref(_dims(g, d_v=96)), 0) == 0
+
+
+def test_bwd_rejects_bad_arguments(g):
+    def call(dims, **kw):
+        a = dict(q=P, k=P, v=P, log_a=P, b=P, w=P, S0=None, cu=None, dO=P, dS_T=None, dq=P, dk=P, dv=P, dg=P,
+                 db=P, dw=P, dS0=None, ws=WS, ws_bytes=1 << 20)
+        a.update(kw)
+        return g.lib.gdn2_bwd(a["q"], a["k"], a["v"], a["log_a"], a["b"], a["w"], a["S0"], a["cu"], a["dO"],
+                              a["dS_T"], a["dq"], a["dk"], a["dv"], a["dg"], a["db"], a["dw"], a["dS0"],
+                              ctypes.byref(dims), a["ws"], a["ws_bytes"], None)
+    d = _dims(g, seq_len=16)
+    assert call(d, dO=None) == g.ERR_INVALID_ARG
+    assert call(d, dw=None) == g.ERR_INVALID_ARG
+    assert call(d, dS0=ctypes.c_void_p((1 << 20) + 4)) == g.ERR_INVALID_ARG
+    assert call(d, ws=None) == g.ERR_WORKSPACE
+    assert call(d, ws_bytes=1024) == g.ERR_WORKSPACE
+    assert call(_dims(g, seq_len=16, d_v=48)) == g.ERR_UNSUPPORTED
+    assert call(_dims(g, seq_len=16, d_k=256)) == g.ERR_UNSUPPORTED

@@ -141,6 +141,52 @@ def test_simt_gate_form_p3(dev, dk, dv, chunk, dtype):
     assert eo <= TOL_CHUNK_F32 and es <= TOL_CHUNK_F32, (eo, es)
 
 
+# fused prologue: pre-activations in, q/k L2 norm and sigmoid gates inside the kernels
+@pytest.mark.parametrize("variant", ["channel", "scalar", "p3"])
+def test_tc_fused_prologue(dev, variant):
+    inp = _small(dev, n_heads=2, lengths=[1, 63, 64, 65, 200, 0, 130], scalar=(variant == "scalar"),
+                 gate_form_p3=(variant == "p3"), fused_prologue=True)
+    o, S_T = run_chunk(inp)
+    eo, es = compare_units(inp, o, S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (eo, es)
+
+
+@pytest.mark.parametrize("dk,dv,chunk,dtype,p3", [(32, 64, 32, torch.float32, False), (64, 16, 64, torch.float32, True)])
+def test_simt_fused_prologue(dev, dk, dv, chunk, dtype, p3):
+    inp = _small(dev, dk=dk, dv=dv, chunk=chunk, dtype=dtype, n_heads=2,
+                 lengths=[1, chunk - 1, chunk + 1, 0, 3 * chunk + 5], gate_form_p3=p3, fused_prologue=True)
+    o, S_T = run_chunk(inp, out_dtype=torch.float32)
+    eo, es = compare_units(inp, o, S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_F32 and es <= TOL_CHUNK_F32, (eo, es)
+
+
+@pytest.mark.parametrize("dk,dv,p3", [(128, 128, False), (64, 32, True)])
+def test_decode_fused_prologue(dev, dk, dv, p3):
+    from gated_delta_rule_159_b200 import gdn2
+    from oracle import prologue
+    N, H, steps = 3, 2, 5
+    g = torch.Generator(device=dev)
+    g.manual_seed(41)
+    rn = lambda *s: torch.randn(*s, generator=g, device=dev)  # noqa: E731
+    raw = dict(q=rn(steps, N, H, dk) * 2, k=rn(steps, N, H, dk) * 2, v=rn(steps, N, H, dv), log_a=rn(steps, N, H, dk) + 3,
+               b=rn(steps, N, H, dk), w=rn(steps, N, H, dv if p3 else dk))
+    raw = {n: t.to(torch.bfloat16) for n, t in raw.items()}
+    S = torch.randn(N, H, dk, dv, generator=g, device=dev) * 0.1
+    S_start = to_f64(S)
+    names = ("q", "k", "v", "log_a", "b", "w")
+    outs = [gdn2.decode_step(*(raw[n][t] for n in names), S, gate_form_p3=p3, fused_prologue=True).clone()
+            for t in range(steps)]
+    o_gpu = to_f64(torch.stack(outs))
+    flags = oracle.GATE_FORM_P3 if p3 else 0
+    for n in range(N):
+        r = {m: to_f64(raw[m][:, n]) for m in names}
+        q, k, la, b, w = prologue.apply(r["q"], r["k"], r["log_a"], r["b"], r["w"])
+        o_r, S_r = oracle.gdn2_fwd(q, k, r["v"], la, b, w, S0=S_start[n][None], flags=flags)
+        for h in range(H):
+            assert rel_err(o_gpu[:, n, h], o_r[:, h]) <= TOL_DECODE
+            assert rel_err(to_f64(S[n, h]), S_r[0, h]) <= TOL_DECODE
+
+
 @pytest.mark.parametrize("case", ["deltanet", "pure_decay", "zero_key", "strong_decay", "no_decay_no_gates"])
 def test_tc_degenerate_cases(dev, case):
     inp = _small(dev, n_seqs=1, seq_len=192, n_heads=2)
@@ -252,6 +298,7 @@ def test_decode_small(dev, d, scalar):
                                      None if di["w"] is None else di["w"][t], S,
                                      scalar_decay=scalar, scalar_gates=scalar, tied_gates=scalar))
     o_gpu = to_f64(torch.stack(outs))  # [steps, N, H, d]
+    assert gdn2.decode_status() == gdn2.OK
     flags = (oracle.SCALAR_DECAY | oracle.SCALAR_GATES | oracle.TIED_GATES) if scalar else 0
     # the decode steps of one (n, h) are one sequence of the recurrence
     for n in range(N):
@@ -288,6 +335,33 @@ def test_decode_gate_form_p3(dev, dk, dv, scalar):
         for h in range(H):
             assert rel_err(o_gpu[:, n, h], o_r[:, h]) <= TOL_DECODE
             assert rel_err(to_f64(S[n, h]), S_r[0, h]) <= TOL_DECODE
+
+
+def test_decode_indexed_matches_gathered_states(dev):
+    """Continuous batching: row n updates pool slot state_idx[n]; padding rows (index
+    outside the pool) give zero output; slots no row names stay bit-identical."""
+    from gated_delta_rule_159_b200 import gdn2, inputs
+    P, N, H, d, steps = 7, 5, 3, 128, 3
+    idx = torch.tensor([3, 0, -1, 6, 9], dtype=torch.int32, device=dev)
+    live = [0, 1, 3]
+    di = inputs.make_decode_inputs(N, H, d, steps, dev, seed=13)
+    g = torch.Generator(device=dev)
+    g.manual_seed(17)
+    pool = torch.randn(P, H, d, d, generator=g, device=dev) * 0.1
+    pool_start = pool.clone()
+    names = ("q", "k", "v", "log_a", "b", "w")
+    outs = [gdn2.decode_step_indexed(*(di[n][t] for n in names), pool, idx).clone() for t in range(steps)]
+    o_gpu = to_f64(torch.stack(outs))
+    assert np.all(o_gpu[:, [2, 4]] == 0.0)
+    for s in (1, 2, 4, 5):
+        torch.testing.assert_close(pool[s], pool_start[s], rtol=0, atol=0)
+    for n in live:
+        slot = int(idx[n])
+        sl = lambda t: to_f64(t[:, n])  # noqa: E731
+        o_r, S_r = oracle.gdn2_fwd(*(sl(di[m]) for m in names), S0=to_f64(pool_start[slot])[None])
+        for h in range(H):
+            assert rel_err(o_gpu[:, n, h], o_r[:, h]) <= TOL_DECODE
+            assert rel_err(to_f64(pool[slot, h]), S_r[0, h]) <= TOL_DECODE
 
 
 def test_decode_graph_replay_matches_eager(dev):
@@ -336,6 +410,7 @@ def test_decode_full_size_sampled(dev):
         gdn2.decode_step(di["q"][t], di["k"][t], di["v"][t], di["log_a"][t], di["b"][t], di["w"][t], S, o=o)
         rec.append(o[idx_n, idx_h].clone())
     rec = to_f64(torch.stack(rec))  # [steps, len(units), d]
+    assert gdn2.decode_status() == gdn2.OK
     for i, (n, h) in enumerate(units):
         sl = lambda t: to_f64(t[:, n, h:h + 1])  # noqa: E731
         o_r, S_r = oracle.gdn2_fwd(sl(di["q"]), sl(di["k"]), sl(di["v"]), sl(di["log_a"]), sl(di["b"]),
