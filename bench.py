@@ -236,6 +236,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--bwd-steps", type=int, default=3)
     ap.add_argument("--no-bwd", action="store_true")
+    ap.add_argument("--no-long", action="store_true")
+    ap.add_argument("--split", type=int, default=8, help="segments per sequence of the long-context split forward")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     args = ap.parse_args()
@@ -468,12 +470,46 @@ def main():
                "workspace_bytes": bws.numel(), "clocks": bclocks}
         del bi, dO, dS_T, bargs, bws
 
+    # ---------------- long context: one sequence of 65,536 tokens, 16 heads (16 units on 148
+    # SMs), plain chunked forward against the sequence-parallel split forward
+    long_ctx = None
+    if not args.no_long:
+        wl = inputs.Workload("long_b1_t64k", 1, 65536, 16, 128, 128, 64, torch.bfloat16, 0.05, False, 0.02)
+        li = inputs.make_inputs(wl, dev, seed=500 + rank)
+        largs = [li[n].view(1, 65536, *li[n].shape[1:]) for n in names]
+        ldims = gdn2.make_dims(1, 65536, 16, 128, 128, 64, gdn2.BF16, gdn2.BF16, 0)
+        lws = torch.empty(int(gdn2.lib.gdn2_chunk_fwd_split_workspace_size(gdn2.ctypes.byref(ldims), args.split)),
+                          dtype=torch.uint8, device=dev)
+        pws = torch.empty(gdn2.workspace_size(ldims), dtype=torch.uint8, device=dev)
+
+        def timed(fn, reps=3):
+            fn()
+            torch.cuda.synchronize()
+            barrier()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(reps):
+                fn()
+            a1.record(stream)
+            barrier()
+            return max_over_ranks(a0.elapsed_time(a1)) / reps
+
+        t_plain = timed(lambda: gdn2.chunk_fwd(*largs, li["S0"], None, workspace=pws))
+        t_split = timed(lambda: gdn2.chunk_fwd_split(*largs, li["S0"], n_split=args.split, workspace=lws))
+        if gdn2.check_status(lws) != gdn2.OK or gdn2.check_status(pws) != gdn2.OK:
+            raise RuntimeError("chunk kernel reported a timed-out wait")
+        long_ctx = {"workload": "1 sequence x 65536 tokens x 16 heads x 128, gates as gdn2_b8_t4k",
+                    "plain_ms": t_plain, "split_ms": t_split, "n_split": args.split,
+                    "plain_tokens_per_s": 65536 * world / (t_plain / 1e3),
+                    "split_tokens_per_s": 65536 * world / (t_split / 1e3)}
+        del li, largs, lws, pws
+
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes and distributions of the "
                                                           "full GDN-2 workload)",
             "config": cfg, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches, "clocks": clocks, "decode": decode, "bwd": bwd}
+            "gpu_launches": launches, "clocks": clocks, "decode": decode, "bwd": bwd, "long_context": long_ctx}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

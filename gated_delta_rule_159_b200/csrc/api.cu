@@ -96,9 +96,22 @@ size_t gdn2_chunk_fwd_workspace_size(const gdn2_dims *dims) {
   return kWsHeader + ((units * sizeof(int32_t) + 255) / 256) * 256;
 }
 
+static int chunk_fwd_impl(const void *q, const void *k, const void *v, const void *log_a, const void *b,
+                          const void *w, const float *S0, const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                          void *o, float *S_T, const gdn2_dims *dims, void *workspace, size_t workspace_bytes,
+                          gdn2_stream_t stream, bool reset_status);
+
 int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *log_a, const void *b, const void *w,
                    const float *S0, const int32_t *cu_seqlens, const int32_t *cu_seqlens_host, void *o, float *S_T,
                    const gdn2_dims *dims, void *workspace, size_t workspace_bytes, gdn2_stream_t stream) {
+  return chunk_fwd_impl(q, k, v, log_a, b, w, S0, cu_seqlens, cu_seqlens_host, o, S_T, dims, workspace,
+                        workspace_bytes, stream, true);
+}
+
+static int chunk_fwd_impl(const void *q, const void *k, const void *v, const void *log_a, const void *b,
+                          const void *w, const float *S0, const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                          void *o, float *S_T, const gdn2_dims *dims, void *workspace, size_t workspace_bytes,
+                          gdn2_stream_t stream, bool reset_status) {
   g_err[0] = '\0';
   int rc = check_dims(dims);
   if (rc) return rc;
@@ -144,7 +157,9 @@ int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *log_
                 "16/32/64)",
                 dims->d_k, dims->d_v, dims->chunk, dims->dtype_in);
 
-  cudaError_t e = cudaMemsetAsync(workspace, 0, kWsHeader, s);
+  // header: [0] status word (kept across the passes of one split forward), [1] unit counter
+  cudaError_t e = reset_status ? cudaMemsetAsync(workspace, 0, kWsHeader, s)
+                               : cudaMemsetAsync(static_cast<char *>(workspace) + 4, 0, kWsHeader - 4, s);
   if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "cudaMemsetAsync(workspace): %s", cudaGetErrorString(e));
   if (tc && cu_seqlens && dims->n_seqs <= kMaxSortedSeqs) {
     int32_t *sched = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + kWsHeader);
@@ -218,6 +233,101 @@ int gdn2_decode_status(gdn2_stream_t stream) {
   if (e != 0) return fail(GDN2_ERR_CUDA, "reading the decode status: %s", cudaGetErrorString((cudaError_t)e));
   if (st == gdn2::kStatusTimeout) return fail(GDN2_ERR_TIMEOUT, "a bounded wait of the decode kernel timed out");
   if (st != 0) return fail(GDN2_ERR_CUDA, "unknown device status %d", st);
+  return GDN2_OK;
+}
+
+static gdn2::SplitPlan split_plan_for(const gdn2_dims *dims, int32_t n_split) {
+  const gdn2::SplitPlan p0 = gdn2::split_plan(dims->n_seqs, dims->seq_len, dims->n_heads, n_split, dims->dtype_in,
+                                              dims->dtype_out, 0);
+  gdn2_dims inner = *dims;
+  inner.n_seqs = p0.n_segs;
+  inner.seq_len = dims->n_seqs * dims->seq_len;
+  return gdn2::split_plan(dims->n_seqs, dims->seq_len, dims->n_heads, n_split, dims->dtype_in, dims->dtype_out,
+                          gdn2_chunk_fwd_workspace_size(&inner));
+}
+
+size_t gdn2_chunk_fwd_split_workspace_size(const gdn2_dims *dims, int32_t n_split) {
+  if (!dims || dims->n_seqs < 1 || dims->n_heads < 1 || dims->seq_len < 0 || n_split < 1) return 0;
+  return split_plan_for(dims, n_split).total;
+}
+
+int gdn2_chunk_fwd_split(const void *q, const void *k, const void *v, const void *log_a, const void *b,
+                         const void *w, const float *S0, void *o, float *S_T, const gdn2_dims *dims, int32_t n_split,
+                         void *workspace, size_t workspace_bytes, gdn2_stream_t stream) {
+  g_err[0] = '\0';
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (n_split < 1) return fail(GDN2_ERR_INVALID_ARG, "n_split must be >= 1 (got %d)", n_split);
+  if (dims->d_k != 128 || dims->d_v != 128 || dims->chunk != 64 || dims->dtype_in != GDN2_BF16)
+    return fail(GDN2_ERR_UNSUPPORTED, "gdn2_chunk_fwd_split needs d_k = d_v = 128, chunk 64 and bf16 inputs");
+  if ((int64_t)dims->n_seqs * dims->seq_len >= ((int64_t)1 << 31))
+    return fail(GDN2_ERR_UNSUPPORTED, "gdn2_chunk_fwd_split needs fewer than 2^31 tokens");
+  rc = check_inputs(q, k, v, log_a, b, w, dims->flags, dims->dtype_in);
+  if (rc) return rc;
+  if (!o || !aligned16(o)) return fail(GDN2_ERR_INVALID_ARG, "o must be non-NULL and 16-byte aligned");
+  if ((S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)))
+    return fail(GDN2_ERR_INVALID_ARG, "S0 / S_T must be 16-byte aligned");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(GDN2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  const size_t need = gdn2_chunk_fwd_split_workspace_size(dims, n_split);
+  if (workspace_bytes < need)
+    return fail(GDN2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+  const int N = dims->n_seqs, T = dims->seq_len, H = dims->n_heads;
+  if ((int64_t)N * T == 0) {  // nothing to run: S_T = S0
+    cudaStream_t s0 = reinterpret_cast<cudaStream_t>(stream);
+    if (!S_T) return GDN2_OK;
+    const size_t bytes = (size_t)N * H * 128 * 128 * sizeof(float);
+    const cudaError_t e = S0 ? cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, s0)
+                             : cudaMemsetAsync(S_T, 0, bytes, s0);
+    return e == cudaSuccess ? GDN2_OK : fail(GDN2_ERR_CUDA, "S_T for empty sequences: %s", cudaGetErrorString(e));
+  }
+  char *ws = static_cast<char *>(workspace);
+  gdn2::SplitArgs a;
+  a.plan = split_plan_for(dims, n_split);
+  a.N = N; a.T = T; a.H = H; a.dtype_out = dims->dtype_out;
+  a.cu = reinterpret_cast<int32_t *>(ws + a.plan.off_cu);
+  a.starts = reinterpret_cast<float *>(ws + a.plan.off_start);
+  a.F = reinterpret_cast<float *>(ws + a.plan.off_F);
+  a.G = reinterpret_cast<float *>(ws + a.plan.off_G);
+  a.S_T = S_T;
+  a.S0 = S0;
+  a.o = o;
+  void *zero_v = ws + a.plan.off_zero_v;
+  void *o2 = ws + a.plan.off_o2;
+  a.o2 = o2;
+  void *inner_ws = ws + a.plan.off_inner;
+  const size_t inner_bytes = a.plan.off_cu - a.plan.off_inner;
+  if (a.plan.n_per_seq == 1)  // one segment per sequence: the plain forward
+    return chunk_fwd_impl(q, k, v, log_a, b, w, S0, nullptr, nullptr, o, S_T, dims, inner_ws, inner_bytes, stream,
+                          true);
+  gdn2_dims inner = *dims;
+  inner.n_seqs = a.plan.n_segs;
+  inner.seq_len = N * T;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t vbytes = (size_t)N * T * H * 128 * (dims->dtype_in == GDN2_BF16 ? 2 : 4);
+  cudaError_t e = cudaMemsetAsync(zero_v, 0, vbytes, s);
+  if (e == cudaSuccess) e = gdn2::launch_split_helpers(0, a, s);
+  if (e == cudaSuccess) e = gdn2::launch_split_helpers(1, a, s);
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "split setup: %s", cudaGetErrorString(e));
+  // pass 1: zero starts (S0 in each sequence's first segment): o and the end states G
+  rc = chunk_fwd_impl(q, k, v, log_a, b, w, a.starts, a.cu, nullptr, o, a.G, &inner, inner_ws, inner_bytes, stream,
+                      true);
+  if (rc) return rc;
+  // pass 2: identity starts, v = 0: the transitions F
+  e = gdn2::launch_split_helpers(2, a, s);
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "split identities: %s", cudaGetErrorString(e));
+  rc = chunk_fwd_impl(q, k, zero_v, log_a, b, w, a.starts, a.cu, nullptr, o2, a.F, &inner, inner_ws, inner_bytes,
+                      stream, false);
+  if (rc) return rc;
+  // combine: true start states; S_T
+  e = gdn2::launch_split_helpers(3, a, s);
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "split combine: %s", cudaGetErrorString(e));
+  // pass 3: the outputs' part that comes from the start states, added to o
+  rc = chunk_fwd_impl(q, k, zero_v, log_a, b, w, a.starts, a.cu, nullptr, o2, nullptr, &inner, inner_ws, inner_bytes,
+                      stream, false);
+  if (rc) return rc;
+  e = gdn2::launch_split_helpers(4, a, s);
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "split add: %s", cudaGetErrorString(e));
   return GDN2_OK;
 }
 

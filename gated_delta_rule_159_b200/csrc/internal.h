@@ -66,6 +66,25 @@ size_t bwd_workspace_bytes(int64_t n_seqs, int64_t t_total, int n_heads, int d_k
 void bwd_carve(BwdProblem &p, void *workspace);
 cudaError_t launch_bwd(const BwdProblem &p, cudaStream_t stream);
 
+// Sequence-parallel forward (seqpar.cu): segments of seg_len tokens, workspace offsets.
+struct SplitPlan {
+  int seg_len, n_per_seq, n_segs;
+  size_t off_inner, off_cu, off_start, off_F, off_G, off_zero_v, off_o2, total;
+};
+struct SplitArgs {
+  SplitPlan plan;
+  int N, T, H, dtype_out;
+  int32_t *cu;
+  float *starts, *F, *G, *S_T;
+  const float *S0;
+  void *o;
+  const void *o2;
+};
+// inner_bytes: workspace of the inner chunked forwards over all segments
+SplitPlan split_plan(int N, int T, int H, int n_split, int dtype_in, int dtype_out, size_t inner_bytes);
+// what: 0 segment bounds, 1 pass-1 starts, 2 identity starts, 3 combine, 4 o += o2
+cudaError_t launch_split_helpers(int what, const SplitArgs &a, cudaStream_t stream);
+
 // Record `message` as this thread's gdn2_last_error() text and return `code`.
 int set_last_error(int code, const char *message);
 

@@ -1,0 +1,156 @@
+// seqpar.cu -- sequence-parallel chunked forward: long sequences split into
+// segments that run side by side.
+//
+// The recurrence is affine in its state (neelmishra.github.io, "What makes the
+// architecture more than a recurrence": the affine-composition view of DeltaNet
+// still holds once each transition includes decay).  For a segment with start
+// state S_s the end state is S_e = F S_s + G, and every output splits as
+// o_t = o_t(S_s = 0) + o_t(S_s, v = 0).  With d_k = d_v the transition F is the
+// end state of the segment run from S_s = I with v = 0.  Hence three passes of
+// the chunk kernel over all segments at once, with one serial combine:
+//
+//   1. S_s = 0 (the first segment of a sequence keeps S0): o and G per segment;
+//   2. S_s = I, v = 0: F per segment;
+//   3. combine per (sequence, head): S_s(j+1) = F_j S_s(j) + G_j, S_T = the last;
+//   4. S_s = the combined starts, v = 0, for every segment but the first: the
+//      correction o(S_s, v = 0), added to o.
+//
+// The work is about three forwards, spread over n_split times as many units.
+#include "common.cuh"
+#include "internal.h"
+
+namespace gdn2 {
+namespace {
+
+constexpr int kComb = 512;  // threads of the combine kernel: 4 per row, 32 columns each
+
+// Segment boundaries of N sequences of T tokens cut every L tokens.
+__global__ void seg_bounds_kernel(int32_t *cu, int N, int T, int L, int ns) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i > N * ns) return;
+  const int n = i / ns, j = i % ns;
+  int v;
+  if (i == N * ns) v = N * T;
+  else v = n * T + (j * L < T ? j * L : T);
+  cu[i] = v;
+}
+
+// Start states of pass 1 (S0 in each sequence's first segment, 0 elsewhere) or
+// identities for pass 2.  One CTA per (segment, head), 128 x 128 floats.
+__global__ void seg_states_kernel(float *dst, const float *S0, int ns, int H, bool identity) {
+  const int sh = blockIdx.x;  // seg * H + h
+  const int seg = sh / H, h = sh % H, n = seg / ns, j = seg % ns;
+  float *d = dst + (size_t)sh * 128 * 128;
+  for (int e = threadIdx.x; e < 128 * 128; e += blockDim.x) {
+    float v = 0.f;
+    if (identity) v = (e / 128 == e % 128) ? 1.f : 0.f;
+    else if (j == 0 && S0) v = S0[((size_t)n * H + h) * 128 * 128 + e];
+    d[e] = v;
+  }
+}
+
+// Serial combine per (sequence, head): S <- F_j S + G_j over the segments.
+// starts[(n, j)] receives the start state of segment j (zero for j = 0, whose
+// outputs already include S0); S_T[n] the final state.
+__global__ void __launch_bounds__(kComb) combine_kernel(const float *F, const float *G, float *starts, float *S_T,
+                                                        int ns, int H) {
+  extern __shared__ float Ss[];  // [128][128] current state
+  const int unit = blockIdx.x, n = unit / H, h = unit % H;
+  const int t = threadIdx.x, r = t >> 2, c0 = (t & 3) * 32;
+  auto at = [&](const float *base, int j) { return base + (((size_t)n * ns + j) * H + h) * 128 * 128; };
+  auto start = [&](int j) { return starts + (((size_t)n * ns + j) * H + h) * 128 * 128; };
+  // segment 0 ends in G_0 (its start, S0, is already folded in)
+  for (int e = t; e < 128 * 128; e += kComb) {
+    Ss[e] = at(G, 0)[e];
+    start(0)[e] = 0.f;
+  }
+  __syncthreads();
+  for (int j = 1; j < ns; ++j) {
+    for (int e = t; e < 128 * 128; e += kComb) start(j)[e] = Ss[e];
+    const float *Fr = at(F, j) + (size_t)r * 128;
+    float acc[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) acc[c] = at(G, j)[(size_t)r * 128 + c0 + c];
+    for (int kk = 0; kk < 128; ++kk) {
+      const float f = Fr[kk];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) acc[c] += f * Ss[kk * 128 + c0 + c];
+    }
+    __syncthreads();  // everyone has read the old state
+#pragma unroll
+    for (int c = 0; c < 32; ++c) Ss[r * 128 + c0 + c] = acc[c];
+    __syncthreads();
+  }
+  if (S_T) {
+    float *d = S_T + ((size_t)n * H + h) * 128 * 128;
+    for (int e = t; e < 128 * 128; e += kComb) d[e] = Ss[e];
+  }
+}
+
+template <typename T>
+__global__ void add_kernel(T *o, const T *d, size_t n) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    o[i] = from_f32<T>(to_f32(o[i]) + to_f32(d[i]));
+}
+
+size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+}  // namespace
+
+SplitPlan split_plan(int N, int T, int H, int n_split, int dtype_in, int dtype_out, size_t inner_bytes) {
+  SplitPlan s;
+  const int nc = (T + 63) / 64;
+  const int per = (nc + n_split - 1) / n_split;
+  s.seg_len = per * 64;
+  s.n_per_seq = (T + s.seg_len - 1) / s.seg_len;
+  if (s.n_per_seq < 1) s.n_per_seq = 1;
+  s.n_segs = N * s.n_per_seq;
+  const size_t state = (size_t)s.n_segs * H * 128 * 128 * sizeof(float);
+  const size_t tok = (size_t)N * T * H * 128;
+  const size_t in_e = dtype_in == GDN2_BF16 ? 2 : 4, out_e = dtype_out == GDN2_BF16 ? 2 : 4;
+  // the inner forwards' workspace comes first: its status word is word 0 of the whole workspace
+  s.off_inner = 0;
+  s.off_cu = up256(inner_bytes);
+  s.off_start = s.off_cu + up256((size_t)(s.n_segs + 1) * sizeof(int32_t));
+  s.off_F = s.off_start + up256(state);
+  s.off_G = s.off_F + up256(state);
+  s.off_zero_v = s.off_G + up256(state);
+  s.off_o2 = s.off_zero_v + up256(tok * in_e);
+  s.total = s.off_o2 + up256(tok * out_e);
+  return s;
+}
+
+cudaError_t launch_split_helpers(int what, const SplitArgs &a, cudaStream_t stream) {
+  const int segs = a.plan.n_segs;
+  switch (what) {
+    case 0:  // segment bounds, zero v
+      seg_bounds_kernel<<<(segs + 1 + 255) / 256, 256, 0, stream>>>(a.cu, a.N, a.T, a.plan.seg_len, a.plan.n_per_seq);
+      break;
+    case 1:  // pass 1 starts
+      seg_states_kernel<<<segs * a.H, 256, 0, stream>>>(a.starts, a.S0, a.plan.n_per_seq, a.H, false);
+      break;
+    case 2:  // pass 2 starts: identities
+      seg_states_kernel<<<segs * a.H, 256, 0, stream>>>(a.starts, nullptr, a.plan.n_per_seq, a.H, true);
+      break;
+    case 3: {  // combine
+      const int smem = 128 * 128 * sizeof(float);
+      cudaError_t e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      combine_kernel<<<a.N * a.H, kComb, smem, stream>>>(a.F, a.G, a.starts, a.S_T, a.plan.n_per_seq, a.H);
+      break;
+    }
+    case 4: {  // o += correction
+      const size_t n = (size_t)a.N * a.T * a.H * 128;
+      if (a.dtype_out == GDN2_BF16)
+        add_kernel<__nv_bfloat16><<<592, 256, 0, stream>>>(static_cast<__nv_bfloat16 *>(a.o),
+                                                           static_cast<const __nv_bfloat16 *>(a.o2), n);
+      else
+        add_kernel<float><<<592, 256, 0, stream>>>(static_cast<float *>(a.o), static_cast<const float *>(a.o2), n);
+      break;
+    }
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace gdn2

@@ -33,7 +33,7 @@ FUSED_PROLOGUE = 16
 
 EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_workspace_size", "gdn2_check_status",
             "gdn2_decode_step", "gdn2_decode_step_indexed", "gdn2_decode_status", "gdn2_bwd",
-            "gdn2_bwd_workspace_size",
+            "gdn2_bwd_workspace_size", "gdn2_chunk_fwd_split", "gdn2_chunk_fwd_split_workspace_size",
             "gdn2_last_error", "gdn2_version")
 
 
@@ -66,6 +66,10 @@ def _load():
     lib.gdn2_decode_step_indexed.restype = ctypes.c_int
     lib.gdn2_decode_step_indexed.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_int32, vp, vp,
                                              ctypes.POINTER(Dims), vp]
+    lib.gdn2_chunk_fwd_split.restype = ctypes.c_int
+    lib.gdn2_chunk_fwd_split.argtypes = [vp] * 9 + [ctypes.POINTER(Dims), ctypes.c_int32, vp, sz, vp]
+    lib.gdn2_chunk_fwd_split_workspace_size.restype = sz
+    lib.gdn2_chunk_fwd_split_workspace_size.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32]
     lib.gdn2_decode_status.restype = ctypes.c_int
     lib.gdn2_decode_status.argtypes = [vp]
     lib.gdn2_bwd.restype = ctypes.c_int
@@ -187,6 +191,32 @@ def decode_status(device=None) -> int:
     """Synchronise and read (and clear) the decode kernels' status: OK or ERR_TIMEOUT."""
     dev = torch.device("cuda") if device is None else torch.device(device)
     return int(lib.gdn2_decode_status(_stream(dev)))
+
+
+def chunk_fwd_split(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, b: torch.Tensor,
+                    w: Optional[torch.Tensor] = None, S0: Optional[torch.Tensor] = None, *, n_split: int = 8,
+                    scalar_decay: bool = False, scalar_gates: bool = False, tied_gates: bool = False,
+                    gate_form_p3: bool = False, fused_prologue: bool = False,
+                    out_dtype: Optional[torch.dtype] = None, workspace: Optional[torch.Tensor] = None):
+    """Sequence-parallel chunked forward through ``gdn2_chunk_fwd_split``: inputs
+    [B, T, H, d] (equal lengths), every sequence cut into up to ``n_split`` segments.
+    Returns (o [B, T, H, d_v], S_T fp32 [B, H, d_k, d_v])."""
+    N, T, H, dk = q.shape
+    dv = v.shape[-1]
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    flags = flags_of(scalar_decay, scalar_gates, tied_gates, gate_form_p3, fused_prologue)
+    dims = make_dims(N, T, H, dk, dv, 64, _dtype_code(q.dtype), _dtype_code(out_dtype), flags)
+    dev = q.device
+    o = torch.empty(N, T, H, dv, dtype=out_dtype, device=dev)
+    S_T = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    if workspace is None:
+        ws = int(lib.gdn2_chunk_fwd_split_workspace_size(ctypes.byref(dims), int(n_split)))
+        workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+    rc = lib.gdn2_chunk_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
+                                  _ptr(S_T), ctypes.byref(dims), int(n_split), _ptr(workspace), workspace.numel(),
+                                  _stream(dev))
+    _check(rc)
+    return o, S_T
 
 
 def check_status(workspace: torch.Tensor) -> int:

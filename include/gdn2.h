@@ -177,6 +177,33 @@ int gdn2_decode_step(const void *q, const void *k, const void *v,
                      float *S, void *o, const gdn2_dims *dims, gdn2_stream_t stream);
 
 /*
+ * gdn2_chunk_fwd_split -- gdn2_chunk_fwd for long sequences when the (sequence,
+ * head) units alone would leave SMs idle: every sequence is cut into up to
+ * n_split segments (whole 64-token chunks) that run side by side.  The
+ * recurrence is affine in its state (neelmishra.github.io, "What makes the
+ * architecture more than a recurrence": the affine-composition view holds once
+ * each transition includes decay): a segment maps its start state S_s to
+ * F S_s + G and its outputs split into a part from S_s = 0 and a part from S_s
+ * with v = 0.  Three chunked passes over all segments (start 0; start I with
+ * v = 0, giving F; the combined true starts with v = 0) and a serial combine
+ * per (sequence, head) give the same o and S_T as gdn2_chunk_fwd up to
+ * rounding, for about three times its work.
+ * Arguments as gdn2_chunk_fwd for N = dims.n_seqs equal sequences of
+ * dims.seq_len tokens (no cu_seqlens); n_split >= 1.
+ * Supported: d_k = d_v = 128, chunk 64, bf16 inputs.  workspace: at least
+ * gdn2_chunk_fwd_split_workspace_size(dims, n_split) bytes, 256-byte aligned;
+ * gdn2_check_status(workspace) reports a timed-out wait of any of the passes.
+ * Errors: GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_WORKSPACE, GDN2_ERR_CUDA.
+ */
+int gdn2_chunk_fwd_split(const void *q, const void *k, const void *v,
+                         const void *log_a, const void *b, const void *w,
+                         const float *S0, void *o, float *S_T, const gdn2_dims *dims, int32_t n_split,
+                         void *workspace, size_t workspace_bytes, gdn2_stream_t stream);
+
+/* Bytes of workspace gdn2_chunk_fwd_split needs (0 if the arguments are invalid). */
+size_t gdn2_chunk_fwd_split_workspace_size(const gdn2_dims *dims, int32_t n_split);
+
+/*
  * gdn2_decode_status -- synchronise `stream`, then report whether any decode
  * step since the last call gave up a bounded device-side wait (the d_k = d_v =
  * 128 decode streams each state through shared memory with bulk copies and

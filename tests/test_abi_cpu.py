@@ -166,3 +166,23 @@ def test_bwd_rejects_bad_arguments(g):
     assert call(d, ws_bytes=1024) == g.ERR_WORKSPACE
     assert call(_dims(g, seq_len=16, d_v=48)) == g.ERR_UNSUPPORTED
     assert call(_dims(g, seq_len=16, d_k=256)) == g.ERR_UNSUPPORTED
+
+
+def test_split_forward_rejects_bad_arguments(g):
+    lib = g.lib
+
+    def call(dims, n_split=4, ws_bytes=4096, **kw):  # too small: no call below can reach a launch
+        a = dict(q=P, k=P, v=P, log_a=P, b=P, w=P, S0=None, o=P, S_T=None, ws=WS)
+        a.update(kw)
+        return lib.gdn2_chunk_fwd_split(a["q"], a["k"], a["v"], a["log_a"], a["b"], a["w"], a["S0"], a["o"],
+                                        a["S_T"], ctypes.byref(dims), n_split, a["ws"], ws_bytes, None)
+    d = _dims(g, n_seqs=1, seq_len=4096, n_heads=2)
+    assert lib.gdn2_chunk_fwd_split_workspace_size(ctypes.byref(d), 4) > lib.gdn2_chunk_fwd_split_workspace_size(
+        ctypes.byref(d), 1) > 0
+    assert lib.gdn2_chunk_fwd_split_workspace_size(ctypes.byref(d), 0) == 0
+    assert call(d, n_split=0) == g.ERR_INVALID_ARG
+    assert call(_dims(g, n_seqs=1, seq_len=4096, d_k=64, d_v=64)) == g.ERR_UNSUPPORTED
+    assert call(_dims(g, n_seqs=1, seq_len=4096, dtype_in=1)) == g.ERR_UNSUPPORTED
+    assert call(d, q=None) == g.ERR_INVALID_ARG
+    assert call(d, ws=None) == g.ERR_WORKSPACE
+    assert call(d, ws_bytes=4096) == g.ERR_WORKSPACE

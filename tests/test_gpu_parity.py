@@ -187,6 +187,29 @@ def test_decode_fused_prologue(dev, dk, dv, p3):
             assert rel_err(to_f64(S[n, h]), S_r[0, h]) <= TOL_DECODE
 
 
+# sequence-parallel forward: segments of whole chunks combined through their affine maps
+@pytest.mark.parametrize("n_split,seq_len,variant", [(1, 300, "channel"), (3, 1000, "channel"), (8, 1000, "channel"),
+                                                     (64, 200, "channel"), (4, 700, "scalar"), (5, 640, "p3")])
+def test_tc_split_forward(dev, n_split, seq_len, variant):
+    from gated_delta_rule_159_b200 import gdn2
+    inp = _small(dev, n_seqs=2, seq_len=seq_len, n_heads=2, scalar=(variant == "scalar"),
+                 gate_form_p3=(variant == "p3"))
+    N, T = inp["n_seqs"], inp["T_tot"] // inp["n_seqs"]
+    names = ("q", "k", "v", "log_a", "b", "w")
+    v4 = lambda t: None if t is None else t.view(N, T, *t.shape[1:])  # noqa: E731
+    ws = torch.empty(int(gdn2.lib.gdn2_chunk_fwd_split_workspace_size(
+        gdn2.ctypes.byref(gdn2.make_dims(N, T, 2, 128, 128, 64, gdn2.BF16, gdn2.F32,
+                                         gdn2.flags_of(inp["scalar_decay"], inp["scalar_gates"], inp["tied_gates"],
+                                                       variant == "p3"))), n_split)), dtype=torch.uint8, device=dev)
+    o, S_T = gdn2.chunk_fwd_split(*(v4(inp[n]) for n in names), inp["S0"], n_split=n_split,
+                                  scalar_decay=inp["scalar_decay"], scalar_gates=inp["scalar_gates"],
+                                  tied_gates=inp["tied_gates"], gate_form_p3=(variant == "p3"),
+                                  out_dtype=torch.float32, workspace=ws)
+    assert gdn2.check_status(ws) == gdn2.OK
+    eo, es = compare_units(inp, o.view(inp["T_tot"], 2, 128), S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (eo, es)
+
+
 @pytest.mark.parametrize("case", ["deltanet", "pure_decay", "zero_key", "strong_decay", "no_decay_no_gates"])
 def test_tc_degenerate_cases(dev, case):
     inp = _small(dev, n_seqs=1, seq_len=192, n_heads=2)
