@@ -55,7 +55,17 @@ struct BwdSmem {
   float z[kBlock][W], r[kBlock][W], dout[kBlock][W];
   float red[kThreads / 32][2 * W];              // per-warp column sums
   float col[2 * W];                             // final column sums
+  float ck[kThreads * kStride];                 // next block's checkpoint (cp.async), [row][col]
 };
+
+// 16-byte asynchronous global -> shared copy (each thread copies and later reads its own row).
+__device__ __forceinline__ void cp_async16(float *dst, const float *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // Sum v[0..W) of every thread over the block's rows.  After the warp
 // reduce-scatter lane l holds column l % W; warps then meet in shared memory.
@@ -100,30 +110,29 @@ struct TokenIo {
   const Tin *q, *k, *v, *g, *b, *w;
   bool scalar_decay, scalar_gates, p3;
   int H, dk, dv;
-  // Row values of token `tok` (global index) for row i of head h.
-  __device__ __forceinline__ void row(int64_t tok, int h, int i, float &a, float &y, float &x, float &p,
-                                      float &q_i) const {
+  // Raw inputs of token `tok` (global index) for row i of head h: k, log_a, b, w, q.
+  __device__ __forceinline__ void fetch_row(int64_t tok, int h, int i, float (&r)[5]) const {
     const size_t ik = ((size_t)tok * H + h) * dk + i, is = (size_t)tok * H + h;
-    const float kk = to_f32(k[ik]);
-    const float bb = to_f32(scalar_gates ? b[is] : b[ik]);
-    a = exp_fast(to_f32(scalar_decay ? g[is] : g[ik]));
-    q_i = to_f32(q[ik]);
-    if (p3) {
-      y = bb * kk;
-      x = kk;
-      p = kk;
-    } else {
-      y = kk;
-      x = bb * kk;
-      p = to_f32(scalar_gates ? w[is] : w[ik]) * kk;
-    }
+    r[0] = to_f32(k[ik]);
+    r[1] = to_f32(scalar_decay ? g[is] : g[ik]);
+    r[2] = to_f32(scalar_gates ? b[is] : b[ik]);
+    r[3] = p3 ? 0.f : to_f32(scalar_gates ? w[is] : w[ik]);
+    r[4] = to_f32(q[ik]);
   }
-  // Written value of column c (global column index) of token `tok`.
-  __device__ __forceinline__ float zval(int64_t tok, int h, int c) const {
+  // Row values a, y, x, p, q from the raw inputs.
+  __device__ __forceinline__ void row_values(const float (&r)[5], float (&o)[5]) const {
+    const float kk = r[0], bb = r[2];
+    o[0] = exp_fast(r[1]);
+    o[1] = p3 ? bb * kk : kk;
+    o[2] = p3 ? kk : bb * kk;
+    o[3] = p3 ? kk : r[3] * kk;
+    o[4] = r[4];
+  }
+  // Raw value (and, in the gist.science form, value gate) of column c of token `tok`.
+  __device__ __forceinline__ void fetch_col(int64_t tok, int h, int c, float &vv, float &ww) const {
     const size_t iv = ((size_t)tok * H + h) * dv + c;
-    float z = to_f32(v[iv]);
-    if (p3) z *= to_f32(scalar_gates ? w[(size_t)tok * H + h] : w[iv]);
-    return z;
+    vv = to_f32(v[iv]);
+    ww = p3 ? to_f32(scalar_gates ? w[(size_t)tok * H + h] : w[iv]) : 1.f;
   }
 };
 
@@ -190,45 +199,55 @@ __global__ void __launch_bounds__(kThreads) bwd_kernel(BwdProblem p) {
     for (int j = 0; j < W; ++j) S[j] += pp * zt[j] - x * rout[j];
   };
 
-  // The token values of one block (row values a, y, x, p, q of this thread's row;
-  // z and dO of this slice's columns) go to shared memory with all loads issued
-  // together, so the serial token loop below waits on no global load.
-  auto load_block = [&](int64_t blk, int cnt, bool with_dout) {
-    float rv[kBlock][5], zv[kBlock], dv_[kBlock];
+  // The token values of one block (raw inputs of this thread's row; v, the value
+  // gate and dO of this slice's columns) are fetched into registers one block ahead
+  // and written to shared memory when the block starts, so the serial token loop
+  // waits on no global load.
+  float raw[kBlock][5], rvv[kBlock], rww[kBlock], rdo[kBlock];
+  auto blk_cnt = [&](int64_t blk) { return (int)((len - blk * kBlock) < kBlock ? (len - blk * kBlock) : kBlock); };
+  auto fetch_block = [&](int64_t blk, bool with_dout) {
+    const int cnt = blk_cnt(blk);
 #pragma unroll
     for (int s = 0; s < kBlock; ++s) {
-      rv[s][0] = 1.f; rv[s][1] = rv[s][2] = rv[s][3] = rv[s][4] = 0.f;
-      zv[s] = dv_[s] = 0.f;
+      raw[s][0] = raw[s][1] = raw[s][2] = raw[s][3] = raw[s][4] = 0.f;
+      rvv[s] = rdo[s] = 0.f;
+      rww[s] = 1.f;
       if (s < cnt) {
         const int64_t tok = bos + blk * kBlock + s;
-        if (live) io.row(tok, h, i, rv[s][0], rv[s][1], rv[s][2], rv[s][3], rv[s][4]);
+        if (live) io.fetch_row(tok, h, i, raw[s]);
         if (i < W) {
-          zv[s] = io.zval(tok, h, c0 + i);
-          if (with_dout) dv_[s] = to_f32(dO[((size_t)tok * H + h) * dv + c0 + i]);
+          io.fetch_col(tok, h, c0 + i, rvv[s], rww[s]);
+          if (with_dout) rdo[s] = to_f32(dO[((size_t)tok * H + h) * dv + c0 + i]);
         }
       }
     }
+  };
+  auto commit_block = [&]() {
 #pragma unroll
     for (int s = 0; s < kBlock; ++s) {
+      float o[5];
+      io.row_values(raw[s], o);
 #pragma unroll
-      for (int m = 0; m < 5; ++m) sm.rowv[s][m][i] = rv[s][m];
+      for (int m = 0; m < 5; ++m) sm.rowv[s][m][i] = o[m];
       if (i < W) {
-        sm.z[s][i] = zv[s];
-        sm.dout[s][i] = dv_[s];
+        sm.z[s][i] = rvv[s] * rww[s];
+        sm.dout[s][i] = rdo[s];
       }
     }
   };
 
   // ---- forward sweep: checkpoints before tokens 0, K, 2K, ...
+  if (nblk > 0) fetch_block(0, false);
   for (int64_t blk = 0; blk < nblk; ++blk) {
     if (live) {
       float *cp = ckpt(blk);
 #pragma unroll
       for (int j = 0; j < W; j += 4) store4(cp + j, S + j);
     }
-    const int cnt = (int)((len - blk * kBlock) < kBlock ? (len - blk * kBlock) : kBlock);
-    load_block(blk, cnt, false);
+    const int cnt = blk_cnt(blk);
+    commit_block();
     __syncthreads();
+    if (blk + 1 < nblk) fetch_block(blk + 1, false);
     for (int s = 0; s < cnt; ++s)
       fwd_token(sm.rowv[s][0][i], sm.rowv[s][1][i], sm.rowv[s][2][i], sm.rowv[s][3][i], sm.z[s], sm.col);
     __syncthreads();  // the next block rewrites the token values
@@ -243,16 +262,31 @@ __global__ void __launch_bounds__(kThreads) bwd_kernel(BwdProblem p) {
 #pragma unroll
     for (int j = 0; j < W; ++j) G[j] = 0.f;
   }
-  for (int64_t blk = nblk - 1; blk >= 0; --blk) {
-    const int cnt = (int)((len - blk * kBlock) < kBlock ? (len - blk * kBlock) : kBlock);
+  // the checkpoint of the next block travels by cp.async into sm.ck (own row only)
+  auto fetch_ckpt = [&](int64_t blk) {
     if (live) {
       const float *cp = ckpt(blk);
 #pragma unroll
-      for (int j = 0; j < W; j += 4) load4(S + j, cp + j);
+      for (int j = 0; j < W; j += 4) cp_async16(&sm.ck[i * ST + j], cp + j);
+    }
+    cp_async_commit();
+  };
+  if (nblk > 0) {
+    fetch_block(nblk - 1, true);
+    fetch_ckpt(nblk - 1);
+  }
+  for (int64_t blk = nblk - 1; blk >= 0; --blk) {
+    const int cnt = blk_cnt(blk);
+    cp_async_wait();
+#pragma unroll
+    for (int j = 0; j < W; j += 4) load4(S + j, &sm.ck[i * ST + j]);
+    commit_block();
+    __syncthreads();
+    if (blk > 0) {
+      fetch_block(blk - 1, true);
+      fetch_ckpt(blk - 1);
     }
     // recompute the block, stashing the state before each token (own row only)
-    load_block(blk, cnt, true);
-    __syncthreads();
     for (int s = 0; s < cnt; ++s) {
 #pragma unroll
       for (int j = 0; j < W; j += 4) store4(&sm.stash[s][i * ST + j], S + j);
