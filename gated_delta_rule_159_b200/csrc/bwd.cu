@@ -36,6 +36,11 @@ namespace {
 constexpr int kThreads = 128;  // one thread per row of the state (d_k <= 128)
 constexpr int kBlock = 4;      // tokens per checkpoint block (the stash holds one block: 2 CTAs per SM)
 constexpr int kRows = 5;       // row sums kept per token: dq, dp, dx, dy, dlog_a
+#ifndef GDN2_BWD_SLICE
+#define GDN2_BWD_SLICE 32
+#endif
+constexpr int kSlice = GDN2_BWD_SLICE;  // columns of S per CTA (d_v above it is split into slices)
+__host__ __device__ constexpr int slice_width(int dv) { return dv < kSlice ? dv : kSlice; }
 
 // Four consecutive floats between memory and a register array without taking
 // the array's address (which would move it to local memory).
@@ -370,7 +375,7 @@ __global__ void __launch_bounds__(kThreads) finish_kernel(BwdProblem p) {
   __shared__ float red[5][kThreads / 32];
   const int64_t th = blockIdx.x;  // tok * H + h
   const int i = threadIdx.x;
-  const int H = p.n_heads, dk = p.d_k, dv = p.d_v, NS = dv / (dv < 32 ? dv : 32);
+  const int H = p.n_heads, dk = p.d_k, dv = p.d_v, NS = dv / slice_width(dv);
   const bool sd = (p.flags & GDN2_SCALAR_DECAY) != 0, sg = (p.flags & GDN2_SCALAR_GATES) != 0;
   const bool tied = (p.flags & GDN2_TIED_GATES) != 0, p3 = (p.flags & GDN2_GATE_FORM_P3) != 0;
   const bool prolog = p.inv_norm != nullptr;
@@ -530,10 +535,10 @@ cudaError_t launch_w(const BwdProblem &p, cudaStream_t stream) {
 template <typename Tin, typename Tout>
 cudaError_t launch_types(const BwdProblem &p, cudaStream_t stream) {
   switch (p.d_v) {
-    case 16: return launch_w<16, Tin, Tout>(p, stream);
-    case 32: return launch_w<32, Tin, Tout>(p, stream);
-    case 64: return launch_w<32, Tin, Tout>(p, stream);
-    case 128: return launch_w<32, Tin, Tout>(p, stream);
+    case 16: return launch_w<slice_width(16), Tin, Tout>(p, stream);
+    case 32: return launch_w<slice_width(32), Tin, Tout>(p, stream);
+    case 64: return launch_w<slice_width(64), Tin, Tout>(p, stream);
+    case 128: return launch_w<slice_width(128), Tin, Tout>(p, stream);
     default: return cudaErrorNotSupported;
   }
 }
@@ -561,7 +566,7 @@ PrologueCopies carve_prologue(float *base, int64_t rows, int d_k, int d_v) {
 }  // namespace
 
 size_t bwd_workspace_bytes(int64_t n_seqs, int64_t t_total, int n_heads, int d_k, int d_v, uint32_t flags) {
-  const int W = d_v < 32 ? d_v : 32;
+  const int W = slice_width(d_v);
   const size_t slots = (size_t)(t_total / kBlock + n_seqs);
   const size_t ckpt = slots * n_heads * (size_t)d_k * d_v * sizeof(float);
   const size_t part = (size_t)(d_v / W) * t_total * n_heads * kRows * (size_t)d_k * sizeof(float);
@@ -572,7 +577,7 @@ size_t bwd_workspace_bytes(int64_t n_seqs, int64_t t_total, int n_heads, int d_k
 }
 
 void bwd_carve(BwdProblem &p, void *workspace) {
-  const int W = p.d_v < 32 ? p.d_v : 32;
+  const int W = slice_width(p.d_v);
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t slots = (size_t)(p.t_total / kBlock + p.n_seqs);
   char *base = static_cast<char *>(workspace);

@@ -237,9 +237,17 @@ __global__ void __launch_bounds__(kSThreads, 1) decode_stream_kernel(DecodeProbl
                        static_cast<const Tin *>(p.log_a), static_cast<const Tin *>(p.b),
                        static_cast<const Tin *>(tied ? p.b : p.w)};
   auto bar = [&](int st) { return ptx::smem_u32(&sm.full[st]); };
-  auto issue = [&](int unit, int st) {  // thread 0
-    ptx::mbar_arrive_expect_tx(bar(st), kState + 6u * kVec);
-    ptx::bulk_load(ptx::smem_u32(sm.S[st]), p.S + (size_t)unit * 128 * 128, kState, bar(st));
+  // state of a unit: its own (n * H + h), or slot state_idx[n] of the pool; -1 for a padding row
+  auto state_of = [&](int unit) -> long long {
+    if (!p.state_idx) return unit;
+    const int slot = p.state_idx[unit / p.n_heads];
+    if (slot < 0 || slot >= p.n_slots) return -1;
+    return (long long)slot * p.n_heads + unit % p.n_heads;
+  };
+  auto issue = [&](int unit, int st) {  // thread 0; a padding row loads its input vectors only
+    const long long su = state_of(unit);
+    ptx::mbar_arrive_expect_tx(bar(st), (su >= 0 ? kState : 0u) + 6u * kVec);
+    if (su >= 0) ptx::bulk_load(ptx::smem_u32(sm.S[st]), p.S + (size_t)su * 128 * 128, kState, bar(st));
 #pragma unroll
     for (int j = 0; j < 6; ++j) ptx::bulk_load(ptx::smem_u32(sm.vec[st][j]), src[j] + (size_t)unit * 128, kVec, bar(st));
   };
@@ -266,6 +274,20 @@ __global__ void __launch_bounds__(kSThreads, 1) decode_stream_kernel(DecodeProbl
         if (unit + stride < units) stream_wait(bar((it + 1) % kStages), (uint32_t)((it + 1) / kStages) & 1u);
       }
       break;
+    }
+    const long long su = state_of(unit);
+    if (su < 0) {  // padding row: zero output, no state; an empty store group keeps the accounting
+      if (t < 128) static_cast<Tout *>(p.o)[(size_t)unit * 128 + t] = from_f32<Tout>(0.f);
+      __syncthreads();
+      if (t == 0) {
+        ptx::bulk_commit_group();
+        const int nu = unit + (kStages - 1) * stride;
+        if (nu < units) {
+          ptx::bulk_wait_group_read1();
+          issue(nu, (it + kStages - 1) % kStages);
+        }
+      }
+      continue;
     }
     const Tin *vq = sm.vec[st][0], *vk = sm.vec[st][1], *vv = sm.vec[st][2];
     const Tin *vg = sm.vec[st][3], *vb = sm.vec[st][4], *vw = sm.vec[st][5];
@@ -359,7 +381,7 @@ __global__ void __launch_bounds__(kSThreads, 1) decode_stream_kernel(DecodeProbl
     ptx::fence_proxy_async_smem();  // the bulk store below reads what the threads just wrote
     __syncthreads();
     if (t == 0) {
-      ptx::bulk_store(p.S + (size_t)unit * 128 * 128, ptx::smem_u32(sm.S[st]), kState);
+      ptx::bulk_store(p.S + (size_t)su * 128 * 128, ptx::smem_u32(sm.S[st]), kState);
       ptx::bulk_commit_group();
       const int nu = unit + (kStages - 1) * stride;
       if (nu < units) {
@@ -409,7 +431,7 @@ cudaError_t launch_dv(const DecodeProblem &p, cudaStream_t stream) {
 
 cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream) {
   const bool channel_gates = (p.flags & (GDN2_SCALAR_DECAY | GDN2_SCALAR_GATES)) == 0;
-  if (p.d_k == 128 && p.d_v == 128 && !p.state_idx && channel_gates && p.n_seqs * p.n_heads > 0) {
+  if (p.d_k == 128 && p.d_v == 128 && channel_gates && p.n_seqs * p.n_heads > 0) {
     const bool in_bf = p.dtype_in == GDN2_BF16, out_bf = p.dtype_out == GDN2_BF16;
     if ((p.flags & (GDN2_GATE_FORM_P3 | GDN2_FUSED_PROLOGUE)) != 0) {
       if (in_bf && out_bf) return launch_stream_t<true, __nv_bfloat16, __nv_bfloat16>(p, stream);
