@@ -13,11 +13,13 @@
 //   G += q do^T;  dq = S do;  dp = G z;  dx = -G r;  dz = G^T p;  dr = -G^T x;
 //   Gbar = G + y dr^T;  dy = Sbar dr;  dlog_a_i = sum_j Gbar_ij Sbar_ij;  G = Diag(a) Gbar.
 //
-// Layout of the work: the columns of S evolve independently, so one CTA owns
-// a slice of W columns of one (sequence, head) state and thread i owns row i
-// of the slice (W fp32 registers).  Row sums over the slice (dq, dp, dx, dy,
-// dlog_a) are per-thread; column sums over the rows (r, dz, dr) are warp
-// reduce-scatters plus one cross-warp pass through shared memory.
+// Layout of the work: the columns of S evolve independently, so one CTA of four
+// warps owns a slice of W columns of one (sequence, head) state; warp w owns W/4
+// of those columns and lane l rows 4l .. 4l + 3 of them.  Every column sum of the
+// recurrence (r, dz, dr) is then a sum over the 128 rows held by one warp (warp
+// shuffles only), so the serial token loop has no block-wide barrier.  The row
+// sums (dq, dp, dx, dy, dlog_a) are outputs only: each warp leaves its share in
+// shared memory and they are added up once per block of tokens.
 //
 // bwd_kernel:    a forward sweep writes the state before every K-th token to
 //                the workspace; then, block by block in reverse, the K states
@@ -52,18 +54,7 @@ __device__ __forceinline__ void store4(float *dst, const float *src) {
   *reinterpret_cast<float4 *>(dst) = make_float4(src[0], src[1], src[2], src[3]);
 }
 
-template <int W>
-struct BwdSmem {
-  static constexpr int kStride = W + 4;          // row stride of the stash (float4-aligned, conflict-free)
-  float stash[kBlock][kThreads * kStride];      // state before each token of the block, [row][col]
-  float rowv[kBlock][5][kThreads];              // a, y, x, p, q per token and row
-  float z[kBlock][W], r[kBlock][W], dout[kBlock][W];
-  float red[kThreads / 32][2 * W];              // per-warp column sums
-  float col[2 * W];                             // final column sums
-  float ck[kThreads * kStride];                 // next block's checkpoint (cp.async), [row][col]
-};
-
-// 16-byte asynchronous global -> shared copy (each thread copies and later reads its own row).
+// 16-byte asynchronous global -> shared copy.
 __device__ __forceinline__ void cp_async16(float *dst, const float *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
                "l"(src)
@@ -72,42 +63,38 @@ __device__ __forceinline__ void cp_async16(float *dst, const float *src) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-// Sum v[0..W) of every thread over the block's rows.  After the warp
-// reduce-scatter lane l holds column l % W; warps then meet in shared memory.
-// Results land in out[0..W) (and out[W..2W) for the second vector when TWO).
-template <int W, bool TWO>
-__device__ __forceinline__ void column_sums(float (&v0)[W], float (&v1)[W], BwdSmem<W> &sm, float *out) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// Per-thread block of the state: 4 rows x CW columns, CW = W / 4 (the warp's columns).
+// Shared buffers that hold one such block per thread are float4-interleaved by thread
+// ([vec4][thread][4]): conflict-free, no padding.
+template <int W>
+struct BwdSmem {
+  static constexpr int CW = W / 4, E = 4 * CW, NV = E / 4;
+  static constexpr int NVS = NV > 5 ? NV : 5;  // a slot also holds the 20 row partials of a token
+  float stash[kBlock][NVS][kThreads][4];  // state before each token of the block; then the row partials
+  float ck[NV][kThreads][4];             // next block's checkpoint (cp.async)
+  float rowv[kBlock][5][kThreads];       // a, y, x, p, q per token and row
+  float z[kBlock][W], dout[kBlock][W], r[kBlock][W];
+};
+
+// Sums over the warp's 32 lanes of CW per-lane values; every lane receives all CW sums.
+// Reduce-scatter inside groups of CW lanes, add across the groups, gather back.
+template <int CW>
+__device__ __forceinline__ void warp_colsum(float (&v)[CW], float (&out)[CW]) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int off = W / 2; off >= 1; off >>= 1) {
+  for (int off = CW / 2; off >= 1; off >>= 1) {
     const bool up = (lane & off) != 0;
 #pragma unroll
     for (int j = 0; j < off; ++j) {
-      const float s0 = up ? v0[j] : v0[j + off], k0 = up ? v0[j + off] : v0[j];
-      v0[j] = k0 + __shfl_xor_sync(0xffffffffu, s0, off);
-      if (TWO) {
-        const float s1 = up ? v1[j] : v1[j + off], k1 = up ? v1[j + off] : v1[j];
-        v1[j] = k1 + __shfl_xor_sync(0xffffffffu, s1, off);
-      }
+      const float send = up ? v[j] : v[j + off], keep = up ? v[j + off] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
     }
   }
 #pragma unroll
-  for (int off = W; off < 32; off <<= 1) {
-    v0[0] += __shfl_xor_sync(0xffffffffu, v0[0], off);
-    if (TWO) v1[0] += __shfl_xor_sync(0xffffffffu, v1[0], off);
-  }
-  if (lane < W) {
-    sm.red[warp][lane] = v0[0];
-    if (TWO) sm.red[warp][W + lane] = v1[0];
-  }
-  __syncthreads();
-  if (threadIdx.x < (TWO ? 2 * W : W)) {
-    float s = 0.f;
+  for (int off = CW; off < 32; off <<= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+  // lane l now holds column l % CW
 #pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w) s += sm.red[w][threadIdx.x];
-    out[threadIdx.x] = s;
-  }
-  __syncthreads();
+  for (int c = 0; c < CW; ++c) out[c] = __shfl_sync(0xffffffffu, v[0], c);
 }
 
 template <typename Tin>
@@ -145,13 +132,16 @@ template <int W, typename Tin, typename Tout>
 __global__ void __launch_bounds__(kThreads) bwd_kernel(BwdProblem p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BwdSmem<W> &sm = *reinterpret_cast<BwdSmem<W> *>(smem_raw);
-  constexpr int ST = BwdSmem<W>::kStride;
+  constexpr int CW = BwdSmem<W>::CW, NV = BwdSmem<W>::NV;
   const int NS = p.d_v / W;
   const int unit = blockIdx.x / NS, slice = blockIdx.x % NS;
   const int H = p.n_heads, dk = p.d_k, dv = p.d_v;
   const int n = unit / H, h = unit % H;
-  const int i = threadIdx.x, c0 = slice * W;
-  const bool live = i < dk;
+  const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+  const int c0 = slice * W;                     // first column of the CTA's slice
+  const int cw0 = warp * CW;                    // the warp's columns inside the slice
+  const int r0 = 4 * lane;                      // this thread's rows r0 .. r0 + 3
+  const bool live = i < dk;                     // row i, for the per-row loads
   const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
 
   TokenIo<Tin> io;
@@ -180,34 +170,55 @@ __global__ void __launch_bounds__(kThreads) bwd_kernel(BwdProblem p) {
   const int64_t nblk = (len + kBlock - 1) / kBlock;
   const int64_t slot0 = bos / kBlock + n;  // first checkpoint slot of this sequence
   const size_t D = (size_t)dk * dv;
-  auto ckpt = [&](int64_t j) { return p.ckpt + ((size_t)(slot0 + j) * H + h) * D + (size_t)i * dv + c0; };
+  // element (row r0 + rr, column c0 + cw0 .. + CW) of a [dk][dv] matrix
+  auto at = [&](const float *base, int rr) { return base + (size_t)(r0 + rr) * dv + c0 + cw0; };
+  auto atw = [&](float *base, int rr) { return base + (size_t)(r0 + rr) * dv + c0 + cw0; };
+  auto ckpt = [&](int64_t j) { return p.ckpt + ((size_t)(slot0 + j) * H + h) * D; };
 
-  float S[W], G[W], t0v[W], t1v[W];
-  if (p.S0 && live) {
-    const float *s0 = p.S0 + (size_t)unit * D + (size_t)i * dv + c0;
+  float S[4][CW], G[4][CW];
+  auto load_state = [&](const float *base) {  // zero for rows past d_k or a NULL base
 #pragma unroll
-    for (int j = 0; j < W; j += 4) load4(S + j, s0 + j);
-  } else {
+    for (int rr = 0; rr < 4; ++rr)
 #pragma unroll
-    for (int j = 0; j < W; ++j) S[j] = 0.f;
-  }
+      for (int c = 0; c < CW; c += 4) {
+        if (base && r0 + rr < dk) load4(&S[rr][c], at(base, rr) + c);
+        else S[rr][c] = S[rr][c + 1] = S[rr][c + 2] = S[rr][c + 3] = 0.f;
+      }
+  };
+  load_state(p.S0 ? p.S0 + (size_t)unit * D : nullptr);
 
-  // One forward token on the registers S; r of the token lands in rout (shared).
-  auto fwd_token = [&](float a, float y, float x, float pp, const float *zt, float *rout) {
+  // One forward token on the registers S: Sbar = a S, r = Sbar^T y (warp column sums),
+  // S = Sbar - x r^T + p z^T.  r is returned for the caller to keep.
+  auto fwd_token = [&](int s, float (&rr_out)[CW]) {
+    const float4 a = *reinterpret_cast<const float4 *>(&sm.rowv[s][0][r0]);
+    const float4 y = *reinterpret_cast<const float4 *>(&sm.rowv[s][1][r0]);
+    const float4 x = *reinterpret_cast<const float4 *>(&sm.rowv[s][2][r0]);
+    const float4 pp = *reinterpret_cast<const float4 *>(&sm.rowv[s][3][r0]);
+    const float av[4] = {a.x, a.y, a.z, a.w}, yv[4] = {y.x, y.y, y.z, y.w};
+    const float xv[4] = {x.x, x.y, x.z, x.w}, pv[4] = {pp.x, pp.y, pp.z, pp.w};
+    float part[CW], zc[CW];
 #pragma unroll
-    for (int j = 0; j < W; ++j) {
-      S[j] *= a;
-      t0v[j] = S[j] * y;
+    for (int c = 0; c < CW; ++c) {
+      zc[c] = sm.z[s][cw0 + c];
+      part[c] = 0.f;
     }
-    column_sums<W, false>(t0v, t1v, sm, rout);
 #pragma unroll
-    for (int j = 0; j < W; ++j) S[j] += pp * zt[j] - x * rout[j];
+    for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+      for (int c = 0; c < CW; ++c) {
+        S[rr][c] *= av[rr];
+        part[c] += S[rr][c] * yv[rr];
+      }
+    warp_colsum<CW>(part, rr_out);
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+      for (int c = 0; c < CW; ++c) S[rr][c] += pv[rr] * zc[c] - xv[rr] * rr_out[c];
   };
 
-  // The token values of one block (raw inputs of this thread's row; v, the value
-  // gate and dO of this slice's columns) are fetched into registers one block ahead
-  // and written to shared memory when the block starts, so the serial token loop
-  // waits on no global load.
+  // The token values of one block (raw inputs of row i; v, the value gate and dO of
+  // the slice's columns) are fetched into registers one block ahead and written to
+  // shared memory when the block starts.
   float raw[kBlock][5], rvv[kBlock], rww[kBlock], rdo[kBlock];
   auto blk_cnt = [&](int64_t blk) { return (int)((len - blk * kBlock) < kBlock ? (len - blk * kBlock) : kBlock); };
   auto fetch_block = [&](int64_t blk, bool with_dout) {
@@ -244,36 +255,37 @@ __global__ void __launch_bounds__(kThreads) bwd_kernel(BwdProblem p) {
   // ---- forward sweep: checkpoints before tokens 0, K, 2K, ...
   if (nblk > 0) fetch_block(0, false);
   for (int64_t blk = 0; blk < nblk; ++blk) {
-    if (live) {
-      float *cp = ckpt(blk);
 #pragma unroll
-      for (int j = 0; j < W; j += 4) store4(cp + j, S + j);
-    }
+    for (int rr = 0; rr < 4; ++rr)
+      if (r0 + rr < dk)
+#pragma unroll
+        for (int c = 0; c < CW; c += 4) store4(atw(ckpt(blk), rr) + c, &S[rr][c]);
     const int cnt = blk_cnt(blk);
     commit_block();
     __syncthreads();
     if (blk + 1 < nblk) fetch_block(blk + 1, false);
-    for (int s = 0; s < cnt; ++s)
-      fwd_token(sm.rowv[s][0][i], sm.rowv[s][1][i], sm.rowv[s][2][i], sm.rowv[s][3][i], sm.z[s], sm.col);
+    for (int s = 0; s < cnt; ++s) {
+      float rr_out[CW];
+      fwd_token(s, rr_out);
+    }
     __syncthreads();  // the next block rewrites the token values
   }
 
   // ---- backward, block by block in reverse
-  if (p.dS_T && live) {
-    const float *g0 = p.dS_T + (size_t)unit * D + (size_t)i * dv + c0;
 #pragma unroll
-    for (int j = 0; j < W; j += 4) load4(G + j, g0 + j);
-  } else {
+  for (int rr = 0; rr < 4; ++rr)
 #pragma unroll
-    for (int j = 0; j < W; ++j) G[j] = 0.f;
-  }
-  // the checkpoint of the next block travels by cp.async into sm.ck (own row only)
-  auto fetch_ckpt = [&](int64_t blk) {
-    if (live) {
-      const float *cp = ckpt(blk);
-#pragma unroll
-      for (int j = 0; j < W; j += 4) cp_async16(&sm.ck[i * ST + j], cp + j);
+    for (int c = 0; c < CW; c += 4) {
+      if (p.dS_T && r0 + rr < dk) load4(&G[rr][c], at(p.dS_T + (size_t)unit * D, rr) + c);
+      else G[rr][c] = G[rr][c + 1] = G[rr][c + 2] = G[rr][c + 3] = 0.f;
     }
+  // the checkpoint of the next block travels by cp.async into sm.ck (own elements only)
+  auto fetch_ckpt = [&](int64_t blk) {
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr)
+      if (r0 + rr < dk)
+#pragma unroll
+        for (int c = 0; c < CW; c += 4) cp_async16(sm.ck[(rr * CW + c) / 4][i], atw(ckpt(blk), rr) + c);
     cp_async_commit();
   };
   if (nblk > 0) {
@@ -284,68 +296,127 @@ __global__ void __launch_bounds__(kThreads) bwd_kernel(BwdProblem p) {
     const int cnt = blk_cnt(blk);
     cp_async_wait();
 #pragma unroll
-    for (int j = 0; j < W; j += 4) load4(S + j, &sm.ck[i * ST + j]);
+    for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+      for (int c = 0; c < CW; c += 4) {
+        if (r0 + rr < dk) load4(&S[rr][c], sm.ck[(rr * CW + c) / 4][i]);
+        else S[rr][c] = S[rr][c + 1] = S[rr][c + 2] = S[rr][c + 3] = 0.f;
+      }
     commit_block();
     __syncthreads();
     if (blk > 0) {
       fetch_block(blk - 1, true);
       fetch_ckpt(blk - 1);
     }
-    // recompute the block, stashing the state before each token (own row only)
+    // recompute the block, stashing the state before each token (own elements only);
+    // the warp keeps each token's r for its columns
     for (int s = 0; s < cnt; ++s) {
 #pragma unroll
-      for (int j = 0; j < W; j += 4) store4(&sm.stash[s][i * ST + j], S + j);
-      fwd_token(sm.rowv[s][0][i], sm.rowv[s][1][i], sm.rowv[s][2][i], sm.rowv[s][3][i], sm.z[s], sm.r[s]);
+      for (int v4 = 0; v4 < NV; ++v4) store4(sm.stash[s][v4][i], &S[(4 * v4) / CW][(4 * v4) % CW]);
+      float rr_out[CW];
+      fwd_token(s, rr_out);
+      if (lane == 0)
+#pragma unroll
+        for (int c = 0; c < CW; ++c) sm.r[s][cw0 + c] = rr_out[c];
     }
+    __syncwarp();
     // walk it backward
     for (int s = cnt - 1; s >= 0; --s) {
-      const int64_t tok = bos + blk * kBlock + s;
-      const float a = sm.rowv[s][0][i], y = sm.rowv[s][1][i], x = sm.rowv[s][2][i];
-      const float pp = sm.rowv[s][3][i], qq = sm.rowv[s][4][i];
-      const float *zt = sm.z[s], *rt = sm.r[s], *dt = sm.dout[s];
-      float sbar[W];
-      float dq = 0.f, dp = 0.f, dx = 0.f;
+      const float4 a4 = *reinterpret_cast<const float4 *>(&sm.rowv[s][0][r0]);
+      const float4 y4 = *reinterpret_cast<const float4 *>(&sm.rowv[s][1][r0]);
+      const float4 x4 = *reinterpret_cast<const float4 *>(&sm.rowv[s][2][r0]);
+      const float4 p4 = *reinterpret_cast<const float4 *>(&sm.rowv[s][3][r0]);
+      const float4 q4 = *reinterpret_cast<const float4 *>(&sm.rowv[s][4][r0]);
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w}, yv[4] = {y4.x, y4.y, y4.z, y4.w};
+      const float xv[4] = {x4.x, x4.y, x4.z, x4.w}, pv[4] = {p4.x, p4.y, p4.z, p4.w};
+      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+      float zc[CW], rc[CW], dc[CW];
 #pragma unroll
-      for (int j = 0; j < W; j += 4) load4(sbar + j, &sm.stash[s][i * ST + j]);
+      for (int c = 0; c < CW; ++c) {
+        zc[c] = sm.z[s][cw0 + c];
+        rc[c] = sm.r[s][cw0 + c];
+        dc[c] = sm.dout[s][cw0 + c];
+      }
+      float sb[4][CW];
 #pragma unroll
-      for (int j = 0; j < W; ++j) {
-        sbar[j] *= a;
-        const float st = sbar[j] - x * rt[j] + pp * zt[j];  // S after the token
-        dq += st * dt[j];
-        G[j] += qq * dt[j];
-        dp += G[j] * zt[j];
-        dx -= G[j] * rt[j];
-        t0v[j] = G[j] * pp;   // -> dz
-        t1v[j] = -G[j] * x;   // -> dr
-      }
-      column_sums<W, true>(t0v, t1v, sm, sm.col);
-      float dy = 0.f, dg = 0.f;
+      for (int v4 = 0; v4 < NV; ++v4) load4(&sb[(4 * v4) / CW][(4 * v4) % CW], sm.stash[s][v4][i]);
+      float dq[4], dp[4], dx[4], colA[CW], colB[CW];
 #pragma unroll
-      for (int j = 0; j < W; ++j) {
-        const float dr = sm.col[W + j];
-        const float gb = G[j] + y * dr;
-        dy += sbar[j] * dr;
-        dg += gb * sbar[j];
-        G[j] = a * gb;
+      for (int c = 0; c < CW; ++c) colA[c] = colB[c] = 0.f;
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        dq[rr] = dp[rr] = dx[rr] = 0.f;
+#pragma unroll
+        for (int c = 0; c < CW; ++c) {
+          sb[rr][c] *= av[rr];
+          const float st = sb[rr][c] - xv[rr] * rc[c] + pv[rr] * zc[c];  // S after the token
+          dq[rr] += st * dc[c];
+          G[rr][c] += qv[rr] * dc[c];
+          dp[rr] += G[rr][c] * zc[c];
+          dx[rr] -= G[rr][c] * rc[c];
+          colA[c] += G[rr][c] * pv[rr];  // -> dz
+          colB[c] -= G[rr][c] * xv[rr];  // -> dr
+        }
       }
-      if (live) {
-        float *pr = p.part + (((size_t)slice * p.t_total + tok) * H + h) * kRows * dk + i;
-        pr[0 * dk] = dq;
-        pr[1 * dk] = dp;
-        pr[2 * dk] = dx;
-        pr[3 * dk] = dy;
-        pr[4 * dk] = dg;
+      float dz[CW], dr[CW];
+      warp_colsum<CW>(colA, dz);
+      warp_colsum<CW>(colB, dr);
+      float dy[4], dg[4];
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        dy[rr] = dg[rr] = 0.f;
+#pragma unroll
+        for (int c = 0; c < CW; ++c) {
+          const float gb = G[rr][c] + yv[rr] * dr[c];
+          dy[rr] += sb[rr][c] * dr[c];
+          dg[rr] += gb * sb[rr][c];
+          G[rr][c] = av[rr] * gb;
+        }
       }
-      if (i < W) p.dz[((size_t)tok * H + h) * dv + c0 + i] = sm.col[i];
-      // sm.col is next written after the first barrier of the next column sums
+      // this warp's share of the row sums, into the thread's own (now free) stash slot:
+      // element 5 rr + m of rows r0 + rr, m = dq, dp, dx, dy, dlog_a
+      float rowp[20];
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        rowp[5 * rr + 0] = dq[rr];
+        rowp[5 * rr + 1] = dp[rr];
+        rowp[5 * rr + 2] = dx[rr];
+        rowp[5 * rr + 3] = dy[rr];
+        rowp[5 * rr + 4] = dg[rr];
+      }
+#pragma unroll
+      for (int v4 = 0; v4 < 5; ++v4) store4(sm.stash[s][v4][i], &rowp[4 * v4]);
+      if (lane == 0) {
+        const int64_t tok = bos + blk * kBlock + s;
+        float *dzp = p.dz + ((size_t)tok * H + h) * dv + c0 + cw0;
+#pragma unroll
+        for (int c = 0; c < CW; c += 4) store4(dzp + c, &dz[c]);
+      }
     }
-    __syncthreads();  // the next block's recompute rewrites the stash and row values
-  }
-  if (p.dS0 && live) {
-    float *g0 = p.dS0 + (size_t)unit * D + (size_t)i * dv + c0;
+    __syncthreads();
+    // add the four warps' row sums of each token (thread i: row i)
+    if (live) {
+      const int tr = i >> 2, e0 = 5 * (i & 3);  // lane holding row i in every warp, element base
+      for (int s = 0; s < cnt; ++s) {
+        const int64_t tok = bos + blk * kBlock + s;
+        float *pr = p.part + (((size_t)slice * p.t_total + tok) * H + h) * kRows * dk + i;
 #pragma unroll
-    for (int j = 0; j < W; j += 4) store4(g0 + j, G + j);
+        for (int m = 0; m < kRows; ++m) {
+          const int e = e0 + m;
+          float acc = 0.f;
+#pragma unroll
+          for (int w = 0; w < kThreads / 32; ++w) acc += sm.stash[s][e / 4][w * 32 + tr][e % 4];
+          pr[m * dk] = acc;
+        }
+      }
+    }
+    __syncthreads();  // the next block rewrites the stash and the token values
   }
+#pragma unroll
+  for (int rr = 0; rr < 4; ++rr)
+    if (p.dS0 && r0 + rr < dk)
+#pragma unroll
+      for (int c = 0; c < CW; c += 4) store4(atw(p.dS0 + (size_t)unit * D, rr) + c, &G[rr][c]);
 }
 
 // Sum of v over the block's 128 threads for NV values at once (result in every thread).
