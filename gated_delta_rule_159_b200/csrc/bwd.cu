@@ -102,29 +102,30 @@ struct TokenIo {
   const Tin *q, *k, *v, *g, *b, *w;
   bool scalar_decay, scalar_gates, p3;
   int H, dk, dv;
-  // Raw inputs of token `tok` (global index) for row i of head h: k, log_a, b, w, q.
-  __device__ __forceinline__ void fetch_row(int64_t tok, int h, int i, float (&r)[5]) const {
+  // Raw inputs of token `tok` (global index) for row i of head h: k, log_a, b, w, q,
+  // kept in the input type: converting them here would wait for the loads at once.
+  __device__ __forceinline__ void fetch_row(int64_t tok, int h, int i, Tin (&r)[5]) const {
     const size_t ik = ((size_t)tok * H + h) * dk + i, is = (size_t)tok * H + h;
-    r[0] = to_f32(k[ik]);
-    r[1] = to_f32(scalar_decay ? g[is] : g[ik]);
-    r[2] = to_f32(scalar_gates ? b[is] : b[ik]);
-    r[3] = p3 ? 0.f : to_f32(scalar_gates ? w[is] : w[ik]);
-    r[4] = to_f32(q[ik]);
+    r[0] = k[ik];
+    r[1] = scalar_decay ? g[is] : g[ik];
+    r[2] = scalar_gates ? b[is] : b[ik];
+    r[3] = p3 ? r[0] : (scalar_gates ? w[is] : w[ik]);
+    r[4] = q[ik];
   }
   // Row values a, y, x, p, q from the raw inputs.
-  __device__ __forceinline__ void row_values(const float (&r)[5], float (&o)[5]) const {
-    const float kk = r[0], bb = r[2];
-    o[0] = exp_fast(r[1]);
+  __device__ __forceinline__ void row_values(const Tin (&r)[5], float (&o)[5]) const {
+    const float kk = to_f32(r[0]), bb = to_f32(r[2]);
+    o[0] = exp_fast(to_f32(r[1]));
     o[1] = p3 ? bb * kk : kk;
     o[2] = p3 ? kk : bb * kk;
-    o[3] = p3 ? kk : r[3] * kk;
-    o[4] = r[4];
+    o[3] = p3 ? kk : to_f32(r[3]) * kk;
+    o[4] = to_f32(r[4]);
   }
   // Raw value (and, in the gist.science form, value gate) of column c of token `tok`.
-  __device__ __forceinline__ void fetch_col(int64_t tok, int h, int c, float &vv, float &ww) const {
+  __device__ __forceinline__ void fetch_col(int64_t tok, int h, int c, Tin &vv, Tin &ww) const {
     const size_t iv = ((size_t)tok * H + h) * dv + c;
-    vv = to_f32(v[iv]);
-    ww = p3 ? to_f32(scalar_gates ? w[(size_t)tok * H + h] : w[iv]) : 1.f;
+    vv = v[iv];
+    ww = p3 ? (scalar_gates ? w[(size_t)tok * H + h] : w[iv]) : vv;
   }
 };
 
@@ -219,21 +220,22 @@ __global__ void __launch_bounds__(kThreads) bwd_kernel(BwdProblem p) {
   // The token values of one block (raw inputs of row i; v, the value gate and dO of
   // the slice's columns) are fetched into registers one block ahead and written to
   // shared memory when the block starts.
-  float raw[kBlock][5], rvv[kBlock], rww[kBlock], rdo[kBlock];
+  Tin raw[kBlock][5], rvv[kBlock], rww[kBlock];
+  Tout rdo[kBlock];
   auto blk_cnt = [&](int64_t blk) { return (int)((len - blk * kBlock) < kBlock ? (len - blk * kBlock) : kBlock); };
   auto fetch_block = [&](int64_t blk, bool with_dout) {
     const int cnt = blk_cnt(blk);
 #pragma unroll
     for (int s = 0; s < kBlock; ++s) {
-      raw[s][0] = raw[s][1] = raw[s][2] = raw[s][3] = raw[s][4] = 0.f;
-      rvv[s] = rdo[s] = 0.f;
-      rww[s] = 1.f;
+      raw[s][0] = raw[s][1] = raw[s][2] = raw[s][3] = raw[s][4] = from_f32<Tin>(0.f);
+      rvv[s] = rww[s] = from_f32<Tin>(0.f);
+      rdo[s] = from_f32<Tout>(0.f);
       if (s < cnt) {
         const int64_t tok = bos + blk * kBlock + s;
         if (live) io.fetch_row(tok, h, i, raw[s]);
         if (i < W) {
           io.fetch_col(tok, h, c0 + i, rvv[s], rww[s]);
-          if (with_dout) rdo[s] = to_f32(dO[((size_t)tok * H + h) * dv + c0 + i]);
+          if (with_dout) rdo[s] = dO[((size_t)tok * H + h) * dv + c0 + i];
         }
       }
     }
@@ -246,8 +248,8 @@ __global__ void __launch_bounds__(kThreads) bwd_kernel(BwdProblem p) {
 #pragma unroll
       for (int m = 0; m < 5; ++m) sm.rowv[s][m][i] = o[m];
       if (i < W) {
-        sm.z[s][i] = rvv[s] * rww[s];
-        sm.dout[s][i] = rdo[s];
+        sm.z[s][i] = io.p3 ? to_f32(rvv[s]) * to_f32(rww[s]) : to_f32(rvv[s]);
+        sm.dout[s][i] = to_f32(rdo[s]);
       }
     }
   };
