@@ -438,8 +438,7 @@ def main():
         dS_T = torch.randn(Nb, 16, 128, 128, generator=gen, device=dev) * 0.1
         bargs = [bi[n].view(Nb, Tb, *bi[n].shape[1:]) for n in names]
         bdims = gdn2.make_dims(Nb, Tb, 16, 128, 128, 64, gdn2.BF16, gdn2.BF16, 0)
-        bws = torch.empty(int(gdn2.lib.gdn2_bwd_workspace_size(gdn2.ctypes.byref(bdims), 0)), dtype=torch.uint8,
-                          device=dev)
+        bws = torch.empty(gdn2.bwd_workspace_size(bdims), dtype=torch.uint8, device=dev)
 
         def bstep():
             return gdn2.bwd(*bargs, dO, S0=bi["S0"], dS_T=dS_T, workspace=bws)
@@ -478,8 +477,7 @@ def main():
         li = inputs.make_inputs(wl, dev, seed=500 + rank)
         largs = [li[n].view(1, 65536, *li[n].shape[1:]) for n in names]
         ldims = gdn2.make_dims(1, 65536, 16, 128, 128, 64, gdn2.BF16, gdn2.BF16, 0)
-        lws = torch.empty(int(gdn2.lib.gdn2_chunk_fwd_split_workspace_size(gdn2.ctypes.byref(ldims), args.split)),
-                          dtype=torch.uint8, device=dev)
+        lws = torch.empty(gdn2.split_workspace_size(ldims, args.split), dtype=torch.uint8, device=dev)
         pws = torch.empty(gdn2.workspace_size(ldims), dtype=torch.uint8, device=dev)
 
         def timed(fn, reps=3):

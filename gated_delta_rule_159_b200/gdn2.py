@@ -133,6 +133,16 @@ def workspace_size(dims: Dims) -> int:
     return int(lib.gdn2_chunk_fwd_workspace_size(ctypes.byref(dims)))
 
 
+def split_workspace_size(dims: Dims, n_split: int) -> int:
+    """Workspace bytes of ``gdn2_chunk_fwd_split`` (0 for invalid arguments)."""
+    return int(lib.gdn2_chunk_fwd_split_workspace_size(ctypes.byref(dims), int(n_split)))
+
+
+def bwd_workspace_size(dims: Dims, packed: bool = False) -> int:
+    """Workspace bytes of ``gdn2_bwd``; ``packed``: the call passes cu_seqlens (seq_len = T_tot)."""
+    return int(lib.gdn2_bwd_workspace_size(ctypes.byref(dims), 1 if packed else 0))
+
+
 def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, b: torch.Tensor,
               w: Optional[torch.Tensor] = None, S0: Optional[torch.Tensor] = None,
               cu_seqlens: Optional[torch.Tensor] = None, *, chunk: int = 64, scalar_decay: bool = False,
@@ -210,8 +220,7 @@ def chunk_fwd_split(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: to
     o = torch.empty(N, T, H, dv, dtype=out_dtype, device=dev)
     S_T = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
     if workspace is None:
-        ws = int(lib.gdn2_chunk_fwd_split_workspace_size(ctypes.byref(dims), int(n_split)))
-        workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+        workspace = torch.empty(max(split_workspace_size(dims, n_split), 256), dtype=torch.uint8, device=dev)
     rc = lib.gdn2_chunk_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
                                   _ptr(S_T), ctypes.byref(dims), int(n_split), _ptr(workspace), workspace.numel(),
                                   _stream(dev))
@@ -300,8 +309,7 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, 
              dw=None if tied_gates else torch.empty_like(w, dtype=dO.dtype),
              dS0=torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev) if need_dS0 else None)
     if workspace is None:
-        ws = int(lib.gdn2_bwd_workspace_size(ctypes.byref(dims), 1 if cu_seqlens is not None else 0))
-        workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+        workspace = torch.empty(bwd_workspace_size(dims, cu_seqlens is not None), dtype=torch.uint8, device=dev)
     rc = lib.gdn2_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(b), _ptr(w), _ptr(S0), _ptr(cu_seqlens),
                       _ptr(dO), _ptr(dS_T), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_a"]),
                       _ptr(g["db"]), _ptr(g["dw"]), _ptr(g["dS0"]), ctypes.byref(dims), _ptr(workspace),

@@ -197,10 +197,9 @@ def test_tc_split_forward(dev, n_split, seq_len, variant):
     N, T = inp["n_seqs"], inp["T_tot"] // inp["n_seqs"]
     names = ("q", "k", "v", "log_a", "b", "w")
     v4 = lambda t: None if t is None else t.view(N, T, *t.shape[1:])  # noqa: E731
-    ws = torch.empty(int(gdn2.lib.gdn2_chunk_fwd_split_workspace_size(
-        gdn2.ctypes.byref(gdn2.make_dims(N, T, 2, 128, 128, 64, gdn2.BF16, gdn2.F32,
-                                         gdn2.flags_of(inp["scalar_decay"], inp["scalar_gates"], inp["tied_gates"],
-                                                       variant == "p3"))), n_split)), dtype=torch.uint8, device=dev)
+    dims = gdn2.make_dims(N, T, 2, 128, 128, 64, gdn2.BF16, gdn2.F32,
+                          gdn2.flags_of(inp["scalar_decay"], inp["scalar_gates"], inp["tied_gates"], variant == "p3"))
+    ws = torch.empty(gdn2.split_workspace_size(dims, n_split), dtype=torch.uint8, device=dev)
     o, S_T = gdn2.chunk_fwd_split(*(v4(inp[n]) for n in names), inp["S0"], n_split=n_split,
                                   scalar_decay=inp["scalar_decay"], scalar_gates=inp["scalar_gates"],
                                   tied_gates=inp["tied_gates"], gate_form_p3=(variant == "p3"),
