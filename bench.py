@@ -229,7 +229,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-steps", type=int, default=1024)
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-step-seconds", type=float, default=6.0)
     ap.add_argument("--batch", type=int, default=0, help="override the batch size (small profiling cases)")
@@ -329,27 +329,49 @@ def main():
     # ---------------- end to end through host buffers (pinned), same workload
     e2e = None
     if not args.no_e2e:
+        # Pipelined over two buffer sets: step i+1's inputs go host -> device on one stream
+        # while step i computes and its o and S_T go device -> host on another (the host
+        # link is full duplex); every step still moves its own inputs and results.
         host = {n: args4[i].cpu().pin_memory() for i, n in enumerate(names)}
         S0_h = inp["S0"].cpu().pin_memory()
         o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         ST_h = torch.empty(ST.shape, dtype=ST.dtype).pin_memory()
-        dev_in = {n: torch.empty_like(args4[i]) for i, n in enumerate(names)}
-        S0_d = torch.empty_like(inp["S0"])
+        dev_in = [{n: torch.empty_like(args4[i]) for i, n in enumerate(names)} for _ in range(2)]
+        S0_d = [torch.empty_like(inp["S0"]) for _ in range(2)]
+        o_d = [torch.empty_like(o) for _ in range(2)]
+        ST_d = [torch.empty_like(ST) for _ in range(2)]
+        ws_d = [torch.empty_like(ws) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in", "comp", "out")}
 
-        def e2e_step():
-            for n in names:
-                dev_in[n].copy_(host[n], non_blocking=True)
-            S0_d.copy_(S0_h, non_blocking=True)
-            gdn2.chunk_fwd(*(dev_in[n] for n in names), S0_d, None, o=o, S_T=ST, workspace=ws)
-            o_h.copy_(o, non_blocking=True)
-            ST_h.copy_(ST, non_blocking=True)
+        def e2e_run(steps, start_event=None):
+            if start_event is not None:
+                s_in.wait_event(start_event)
+            for i in range(steps):
+                b = i % 2
+                with torch.cuda.stream(s_in):
+                    s_in.wait_event(ev["comp"][b])  # the forward that read buffer b is done
+                    for n in names:
+                        dev_in[b][n].copy_(host[n], non_blocking=True)
+                    S0_d[b].copy_(S0_h, non_blocking=True)
+                    ev["in"][b].record(s_in)
+                stream.wait_event(ev["in"][b])
+                stream.wait_event(ev["out"][b])  # o_d[b] has been read back
+                gdn2.chunk_fwd(*(dev_in[b][n] for n in names), S0_d[b], None, o=o_d[b], S_T=ST_d[b],
+                               workspace=ws_d[b])
+                ev["comp"][b].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev["comp"][b])
+                    o_h.copy_(o_d[b], non_blocking=True)
+                    ST_h.copy_(ST_d[b], non_blocking=True)
+                    ev["out"][b].record(s_out)
+            stream.wait_stream(s_out)
 
-        e2e_step()
+        e2e_run(2)
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        e2e_run(args.e2e_steps, start_event=e0)
         e1.record(stream)
         barrier()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1))
@@ -358,8 +380,9 @@ def main():
         e2e = {"value": T_tot * world * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                "ms_per_step": e2e_ms / args.e2e_steps,
-               "path": "pinned host -> device copies, gdn2_chunk_fwd via the Python binding, o and S_T back"}
-        del host, dev_in, o_h, ST_h
+               "path": "pinned host -> device copies, gdn2_chunk_fwd via the Python binding, o and S_T back; "
+                       "two buffer sets, copies of the next step overlap this step's compute and read-back"}
+        del host, dev_in, o_h, ST_h, o_d, ST_d, ws_d, S0_d
 
     # ---------------- CPU baseline (rank 0, one GPU only)
     cpu = None
