@@ -13,21 +13,22 @@
 //     x_r = x e^{L_ref - L},  p_r = p e^{L_ref - L},  S_r = Diag(e^{L_ref}) S.
 //   G1  [A B ; QX QP] = [k_r ; q_r] [x_r ; p_r]^T         (M=128 N=128 K=128)
 //       A, B strictly lower; QX, QP lower incl. diagonal.
-//   solve T = (I + A)^-1 (16x16 diagonal blocks by forward substitution, then
-//       the off-diagonal blocks level by level: T_IJ = -T_II sum_K A_IK T_KJ).
-//   G2  W_r^T = k_r^T T^T ,  (B V)^T = V^T B^T              (M=128 N=64 K=64)
-//   G3  M^T = (B V)^T T^T + S_r^T W_r^T                     (M=128 N=64 K=64+128)
-//       row i of M is the erase read r_i = Sbar_i^T k_i of every token.
-//   G4  O^T = S_r^T q_r^T + V^T QP^T - M^T QX^T             (M=128 N=64 K=128+64+64)
-//   G5  dS  = p_r^T V - x_r^T M                             (M=128 N=128 K=64+64)
-//   S  <- Diag(e^{L_C}) S + Diag(e^{L_C - L_ref}) dS.
+//   solve T = (I + A)^-1: 8x8 diagonal blocks by forward substitution, then the
+//       off-diagonal blocks level by level, T_LU = -T_LL (A_LU T_UU).
+//   R^T = V^T B^T + S_r^T k_r^T    (the right-hand side of M = T R)
+//   M^T = R^T T^T                   row i of M is the erase read r_i = Sbar_i^T k_i
+//   O^T = S_r^T q_r^T + V^T QP^T - M^T QX^T
+//   S'  = Diag(e^{L_C - L_ref}) (S_r' + p_r^T V - x_r^T M),  S_r' = Diag(e^{L_ref}) S in fp32.
 // All GEMMs are tcgen05.mma kind::f16 (bf16 operands from shared memory, fp32
-// accumulators in TMEM); the state S is kept in TMEM in fp32 for the whole
-// sequence and only its bf16 image S_r is an MMA operand.  Operand tiles arrive
-// by TMA (128-byte swizzle); transposed operands use MN-major descriptors, so no
-// tile is ever transposed in memory.
+// accumulators in TMEM).  The state lives in TMEM in fp32 for the whole
+// sequence as S = Diag(tau) Sacc: each chunk rewrites Sacc as e^{L_ref} S (whose
+// bf16 image S_r is the MMA operand), the increment GEMMs accumulate onto it,
+// and tau becomes e^{L_C - L_ref}.  Operand tiles arrive by TMA (128-byte
+// swizzle); transposed operands use MN-major descriptors, so no tile is ever
+// transposed in memory.  The T-independent GEMMs run on the tensor core while
+// warps 0-14 solve for T.
 //
-// One CTA (256 threads) per SM, persistent over (sequence, head) units taken
+// One CTA (512 threads) per SM, persistent over (sequence, head) units taken
 // longest-first from an atomic counter in the caller's workspace.  Every
 // mbarrier wait is bounded; a timeout sets the workspace status word and the
 // CTA winds down instead of hanging.
@@ -68,7 +69,7 @@ constexpr uint32_t OFF_XS = 198656;    // fp32 solve scratch, <= 4 KB
 constexpr uint32_t OFF_BZ = 180224;    // R^T bf16 [128 x 64] and o staging (after the solve; overlaps A/T)
 constexpr uint32_t OFF_MT = 196608;    // -M^T bf16 [128 x 64] (after the solve)
 constexpr uint32_t OFF_MISC = 212992;
-constexpr uint32_t MISC_GC = 0;        // float[128]  e^{L_C}
+constexpr uint32_t MISC_GC = 0;        // (unused) float[128]
 constexpr uint32_t MISC_DL = 512;      // float[128]  e^{L_C - L_ref}
 constexpr uint32_t MISC_SM = 1024;     // float[128]  e^{L_ref}
 constexpr uint32_t MISC_PART = 1536;   // float[16][128] 4-row sums of log_a, then exclusive prefixes
@@ -179,7 +180,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   const int H = p.n_heads;
   const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
 
-  float *sGC = reinterpret_cast<float *>(gb + OFF_MISC + MISC_GC);
   float *sDL = reinterpret_cast<float *>(gb + OFF_MISC + MISC_DL);
   float *sSM = reinterpret_cast<float *>(gb + OFF_MISC + MISC_SM);
   float *part = reinterpret_cast<float *>(gb + OFF_MISC + MISC_PART);
@@ -210,7 +210,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(gb + OFF_MISC + MISC_TMEM);
   const uint32_t tmD1 = tmem;        // G1 result; then W_r^T | (B V)^T; then M^T (128 cols)
   const uint32_t tmS = tmem + 128;   // fp32 state (128 cols)
-  const uint32_t tmDS = tmem + 256;  // state increment dS (128 cols)
   const uint32_t tmO = tmem + 384;   // O^T (64 cols)
   const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
   uint32_t it = 0;                   // chunks processed by this CTA: parity of every mbarrier
@@ -290,6 +289,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       ptx::tmem_st32(tmS + lane_base + cg * 32, r);
       ptx::tmem_wait_st();
     }
+    // The state is kept as S = tau * Sacc (tau per dk row, this thread's row): each chunk's
+    // S_r build rewrites Sacc as e^{L_ref} S, the chunk's increment GEMMs accumulate onto
+    // it, and tau becomes e^{L_C - L_ref}: S' = e^{L_C - L_ref} (e^{L_ref} S + dS).
+    float tau = 1.f;
 
     for (int ci = 0; ci < nchunks; ++ci, ++it) {
       const uint32_t par = it & 1u;
@@ -338,7 +341,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             if (j == 7) refv = run;
           }
           sRef[tid] = refv;
-          sGC[tid] = ptx::ex2(run * kLog2eF);
           sDL[tid] = ptx::ex2((run - refv) * kLog2eF);
           sSM[tid] = ptx::ex2(refv * kLog2eF);
         }
@@ -432,19 +434,28 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       }
       __syncthreads();
 
-      // ---- S_r = Diag(e^{L_ref}) S as a bf16 MN-major operand (dv columns [32 cg, 32 cg + 32))
+      // ---- S_r = Diag(e^{L_ref}) S as a bf16 MN-major operand (dv columns [32 cg, 32 cg + 32));
+      //      the fp32 accumulator becomes the same e^{L_ref} S, onto which dS accumulates
       {
+        // two products, in this order: tau * Sacc is the state, O(1); e^{L_ref} tau alone can
+        // underflow (both factors reach e^{-80} under the range precondition)
         const float sm = sSM[row];
         uint32_t r[32];
         ptx::tmem_ld32(tmS + lane_base + cg * 32, r);
         ptx::tmem_wait_ld();
         float f[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(r[j]);
+        for (int j = 0; j < 32; ++j) {
+          f[j] = (__uint_as_float(r[j]) * tau) * sm;
+          r[j] = __float_as_uint(f[j]);
+        }
+        ptx::tmem_st32(tmS + lane_base + cg * 32, r);
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8)
           sts_v4(sb + OFF_SR + (uint32_t)(cg >> 1) * 16384u + swz(row, (uint32_t)((cg & 1) * 4 + q8)),
-                 pack8(f + 8 * q8, sm));
+                 pack8(f + 8 * q8, 1.f));
+        tau = sDL[row];
+        ptx::tmem_wait_st();
       }
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
@@ -514,8 +525,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           constexpr uint32_t idS = ptx::idesc_bf16(128, 128, true, true);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            ptx::umma_bf16(tmDS, ptx::sdesc_sw128(sb + OFF_XP + 8192 + kk * 2048, 16384, 1024),
-                           ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024), idS, kk > 0);
+            ptx::umma_bf16(tmS, ptx::sdesc_sw128(sb + OFF_XP + 8192 + kk * 2048, 16384, 1024),
+                           ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024), idS, 1);
           constexpr uint32_t idO = ptx::idesc_bf16(128, 64, true, false);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
@@ -720,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         constexpr uint32_t idS = ptx::idesc_bf16(128, 128, true, false);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmDS, ptx::sdesc_sw128(sb + OFF_XP + kk * 2048, 16384, 1024),
+          ptx::umma_bf16(tmS, ptx::sdesc_sw128(sb + OFF_XP + kk * 2048, 16384, 1024),
                          ptx::sdesc_sw128(sb + OFF_MT + kk * 32, 16, 1024), idS, 1);
         ptx::umma_commit(bar(BAR_G45));
       }
@@ -728,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       ptx::tc_fence_after();
       if (tid == kIssuer && has_next && !*sAbort) issue_tma_x(h, t0 + C);  // x_r is dead now
 
-      // ---- a8: outputs and the state update
+      // ---- a8: outputs (the state was updated by the increment GEMMs)
       {
         // o^T: lane = dv channel `row`, columns = tokens [16 cg, 16 cg + 16)
         uint32_t r[16];
@@ -747,16 +758,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             sts_f32(sb + OFF_BZ + (uint32_t)(row >> 5) * 8192u + (uint32_t)i * 128u + (uint32_t)(row & 31) * 4u, f);
           }
         }
-        // S <- e^{L_C} S + e^{L_C - L_ref} dS   (thread: dk row `row`, columns [32 cg, +32))
-        const float gc = sGC[row], dl = sDL[row];
-        uint32_t s[32], ds[32];
-        ptx::tmem_ld32(tmS + lane_base + cg * 32, s);
-        ptx::tmem_ld32(tmDS + lane_base + cg * 32, ds);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) s[j] = __float_as_uint(fmaf(gc, __uint_as_float(s[j]), dl * __uint_as_float(ds[j])));
-        ptx::tmem_st32(tmS + lane_base + cg * 32, s);
-        ptx::tmem_wait_st();
       }
       ptx::fence_proxy_async_smem();  // staging is read by the TMA store below
       __syncthreads();
@@ -794,8 +795,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       ptx::tmem_wait_ld();
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        reinterpret_cast<float4 *>(dst)[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                                          __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+        reinterpret_cast<float4 *>(dst)[j] =
+            make_float4(tau * __uint_as_float(r[4 * j]), tau * __uint_as_float(r[4 * j + 1]),
+                        tau * __uint_as_float(r[4 * j + 2]), tau * __uint_as_float(r[4 * j + 3]));
     }
     ptx::tc_fence_before();
     __syncthreads();
