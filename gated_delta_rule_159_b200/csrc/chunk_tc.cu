@@ -69,7 +69,6 @@ constexpr uint32_t OFF_XS = 198656;    // fp32 solve scratch, <= 4 KB
 constexpr uint32_t OFF_BZ = 180224;    // R^T bf16 [128 x 64] and o staging (after the solve; overlaps A/T)
 constexpr uint32_t OFF_MT = 196608;    // -M^T bf16 [128 x 64] (after the solve)
 constexpr uint32_t OFF_MISC = 212992;
-constexpr uint32_t MISC_GC = 0;        // (unused) float[128]
 constexpr uint32_t MISC_DL = 512;      // float[128]  e^{L_C - L_ref}
 constexpr uint32_t MISC_SM = 1024;     // float[128]  e^{L_ref}
 constexpr uint32_t MISC_PART = 1536;   // float[16][128] 4-row sums of log_a, then exclusive prefixes
@@ -167,7 +166,10 @@ __device__ __forceinline__ uint2 pack4(float a, float b, float c, float d) {
 // arrives with the TMA_W group and w with the TMA_X group.
 // kProlog: the inputs are pre-activations (GDN2_FUSED_PROLOGUE): log_a <- log sigmoid,
 // b, w <- sigmoid, and the q and k rows are L2-normalised here.
-template <bool kScalarDecay, bool kScalarGates, bool kP3, bool kProlog, typename Tout>
+// kXP: x_r == p_r (the gist.science form always; the default form with tied gates),
+// so B = A and QP = QX: G1 runs with N = 64 and the masks write B and read QP from the
+// A and QX values.
+template <bool kScalarDecay, bool kScalarGates, bool kP3, bool kProlog, bool kXP, typename Tout>
 __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_constant__ TcParams P) {
   extern __shared__ uint8_t smem_raw[];
   const ChunkProblem &p = P.p;
@@ -464,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       // ---- a4: G1 [A B; QX QP] = [k_r; q_r] [x_r; p_r]^T
       if (tid == 0 && !*sAbort) {
         ptx::tc_fence_after();
-        constexpr uint32_t id1 = ptx::idesc_bf16(128, 128, false, false);
+        constexpr uint32_t id1 = ptx::idesc_bf16(128, kXP ? 64 : 128, false, false);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t ko = (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
@@ -477,8 +479,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       ptx::tc_fence_after();
 
       // masks: A, B strictly lower (fp32 A for the solve, bf16 B); QX, QP lower incl. diagonal.
-      // warp (qd, cg) reads D1 columns [32 cg, 32 cg + 32).
-      {
+      // warp (qd, cg) reads D1 columns [32 cg, 32 cg + 32); with kXP only columns 0-63 exist.
+      if (!kXP || cg < 2) {
         float *Af = reinterpret_cast<float *>(gb + OFF_AF);
         uint32_t r[32];
         ptx::tmem_ld32(tmD1 + lane_base + cg * 32, r);
@@ -494,6 +496,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             for (int j4 = 0; j4 < 8; ++j4)
               *reinterpret_cast<float4 *>(Af + fidx(i, jb + 4 * j4)) =
                   make_float4(f[4 * j4], f[4 * j4 + 1], f[4 * j4 + 2], f[4 * j4 + 3]);
+            if (kXP) {  // B = A
+#pragma unroll
+              for (int q8 = 0; q8 < 4; ++q8)
+                sts_v4(sb + OFF_BM + swz(i, (uint32_t)((cg & 1) * 4 + q8)), pack8(f + 8 * q8, 1.f));
+            }
           } else {
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8)
@@ -546,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             ptx::umma_bf16(tmO, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
-                           ptx::sdesc_sw128(sb + OFF_QP + kk * 32, 16, 1024), idO, 1);
+                           ptx::sdesc_sw128(sb + (kXP ? OFF_QX : OFF_QP) + kk * 32, 16, 1024), idO, 1);
           ptx::umma_commit(bar(BAR_E2));
           if (has_next) {  // p_r is dead once dS = p_r^T V is done: the next chunk's w can land
             wait_bar(bar(BAR_E1), par, sAbort, p.status);
@@ -856,24 +863,28 @@ bool make_map_o(CUtensorMap *m, void *base, int64_t t_total, int H, bool bf16) {
   return r == CUDA_SUCCESS;
 }
 
-template <bool SD, bool SG, bool P3, bool PR, typename Tout>
+template <bool SD, bool SG, bool P3, bool PR, bool XP, typename Tout>
 cudaError_t launch_t(const TcParams &P, int grid, cudaStream_t stream) {
-  auto kern = chunk_tc_kernel<SD, SG, P3, PR, Tout>;
+  auto kern = chunk_tc_kernel<SD, SG, P3, PR, XP, Tout>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, kSmemBytes, stream>>>(P);
   return cudaGetLastError();
 }
 
-template <bool P3, bool PR>
+template <bool P3, bool PR, bool XP>
 cudaError_t launch_gates(const TcParams &P, int grid, cudaStream_t stream, bool sd, bool sg, bool obf) {
   if (sd && sg)
-    return obf ? launch_t<true, true, P3, PR, __nv_bfloat16>(P, grid, stream) : launch_t<true, true, P3, PR, float>(P, grid, stream);
+    return obf ? launch_t<true, true, P3, PR, XP, __nv_bfloat16>(P, grid, stream)
+               : launch_t<true, true, P3, PR, XP, float>(P, grid, stream);
   if (sd)
-    return obf ? launch_t<true, false, P3, PR, __nv_bfloat16>(P, grid, stream) : launch_t<true, false, P3, PR, float>(P, grid, stream);
+    return obf ? launch_t<true, false, P3, PR, XP, __nv_bfloat16>(P, grid, stream)
+               : launch_t<true, false, P3, PR, XP, float>(P, grid, stream);
   if (sg)
-    return obf ? launch_t<false, true, P3, PR, __nv_bfloat16>(P, grid, stream) : launch_t<false, true, P3, PR, float>(P, grid, stream);
-  return obf ? launch_t<false, false, P3, PR, __nv_bfloat16>(P, grid, stream) : launch_t<false, false, P3, PR, float>(P, grid, stream);
+    return obf ? launch_t<false, true, P3, PR, XP, __nv_bfloat16>(P, grid, stream)
+               : launch_t<false, true, P3, PR, XP, float>(P, grid, stream);
+  return obf ? launch_t<false, false, P3, PR, XP, __nv_bfloat16>(P, grid, stream)
+             : launch_t<false, false, P3, PR, XP, float>(P, grid, stream);
 }
 
 }  // namespace
@@ -917,8 +928,15 @@ cudaError_t launch_chunk_tc(const ChunkProblem &p, cudaStream_t stream, const ch
   const int grid = P.n_units < sms ? P.n_units : sms;
   const bool obf = p.dtype_out == GDN2_BF16;
   const bool pr = (p.flags & GDN2_FUSED_PROLOGUE) != 0;
-  if (p3) return pr ? launch_gates<true, true>(P, grid, stream, sd, sg, obf) : launch_gates<true, false>(P, grid, stream, sd, sg, obf);
-  return pr ? launch_gates<false, true>(P, grid, stream, sd, sg, obf) : launch_gates<false, false>(P, grid, stream, sd, sg, obf);
+  // x_r == p_r in the gist.science form, and in the default form when w is b
+  if (p3)
+    return pr ? launch_gates<true, true, true>(P, grid, stream, sd, sg, obf)
+              : launch_gates<true, false, true>(P, grid, stream, sd, sg, obf);
+  if (tied)
+    return pr ? launch_gates<false, true, true>(P, grid, stream, sd, sg, obf)
+              : launch_gates<false, false, true>(P, grid, stream, sd, sg, obf);
+  return pr ? launch_gates<false, true, false>(P, grid, stream, sd, sg, obf)
+            : launch_gates<false, false, false>(P, grid, stream, sd, sg, obf);
 }
 
 }  // namespace gdn2
