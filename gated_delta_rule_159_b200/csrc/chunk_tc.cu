@@ -19,14 +19,15 @@
 //   M^T = R^T T^T                   row i of M is the erase read r_i = Sbar_i^T k_i
 //   O^T = S_r^T q_r^T + V^T QP^T - M^T QX^T
 //   S'  = Diag(e^{L_C - L_ref}) (S_r' + p_r^T V - x_r^T M),  S_r' = Diag(e^{L_ref}) S in fp32.
-// All GEMMs are tcgen05.mma kind::f16 (bf16 operands from shared memory, fp32
-// accumulators in TMEM).  The state lives in TMEM in fp32 for the whole
-// sequence as S = Diag(tau) Sacc: each chunk rewrites Sacc as e^{L_ref} S (whose
-// bf16 image S_r is the MMA operand), the increment GEMMs accumulate onto it,
-// and tau becomes e^{L_C - L_ref}.  Operand tiles arrive by TMA (128-byte
-// swizzle); transposed operands use MN-major descriptors, so no tile is ever
-// transposed in memory.  The T-independent GEMMs run on the tensor core while
-// warps 0-14 solve for T.
+// All GEMMs are tcgen05.mma kind::f16 with fp32 accumulators in TMEM, computed in
+// their transposed forms (M = d_v = 128 rows): O^T, R^T, M^T and S^T.  The state lives
+// in TMEM in fp32 for the whole sequence, transposed, as S = Diag(tau) Sacc: each chunk
+// rewrites Sacc as e^{L_ref} S, the increment GEMMs accumulate onto it, and tau becomes
+// e^{L_C - L_ref}.  The A operands S_r^T, R^T and -M^T are written by the threads into
+// TMEM as bf16 and read from there by the tensor core; the B operands and V^T come
+// from shared memory, where the tiles arrive by TMA (128-byte swizzle) and transposed
+// operands use MN-major descriptors, so no tile is ever transposed in memory.  The
+// T-independent GEMMs run on the tensor core while warps 0-14 solve for T.
 //
 // One CTA (512 threads) per SM, persistent over (sequence, head) units taken
 // longest-first from an atomic counter in the caller's workspace.  Every
@@ -58,7 +59,7 @@ constexpr uint32_t OFF_KQ = 0;         // 2 K-blocks x [k_r rows 0-63 | q_r rows
 constexpr uint32_t OFF_XP = 32768;     // 2 K-blocks x [x_r rows | p_r rows]
 constexpr uint32_t OFF_V = 65536;      // 2 column blocks x [64 rows], 8 KB each
 constexpr uint32_t OFF_G = 81920;      // raw log_a tile
-constexpr uint32_t OFF_SR = 98304;     // S_r bf16: 2 dv-blocks x [128 dk rows], 16 KB each
+                                       // [98304, 131072) unused
 constexpr uint32_t OFF_T = 131072;     // T bf16 [64 x 64]
 constexpr uint32_t OFF_BM = 139264;    // B bf16 [64 x 64]
 constexpr uint32_t OFF_QX = 147456;    // QX bf16 [64 x 64]
@@ -66,10 +67,10 @@ constexpr uint32_t OFF_QP = 155648;    // QP bf16 [64 x 64]
 constexpr uint32_t OFF_AF = 163840;    // fp32 A [64 x 68] (masks -> solve)
 constexpr uint32_t OFF_TF = 181248;    // fp32 T [64 x 68] (solve)
 constexpr uint32_t OFF_XS = 198656;    // fp32 solve scratch, <= 4 KB
-constexpr uint32_t OFF_BZ = 180224;    // R^T bf16 [128 x 64] and o staging (after the solve; overlaps A/T)
-constexpr uint32_t OFF_MT = 196608;    // -M^T bf16 [128 x 64] (after the solve)
+constexpr uint32_t OFF_BZ = 180224;    // o staging (after the solve; overlaps A/T)
 constexpr uint32_t OFF_MISC = 212992;
-constexpr uint32_t MISC_DL = 512;      // float[128]  e^{L_C - L_ref}
+constexpr uint32_t MISC_DL0 = 0;       // float[128]  e^{L_C - L_ref} of the chunks with even parity
+constexpr uint32_t MISC_DL = 512;      // float[128]  e^{L_C - L_ref} of the chunks with odd parity
 constexpr uint32_t MISC_SM = 1024;     // float[128]  e^{L_ref}
 constexpr uint32_t MISC_PART = 1536;   // float[16][128] 4-row sums of log_a, then exclusive prefixes
 constexpr uint32_t MISC_REF = 9728;    // float[128]  L_ref
@@ -182,7 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   const int H = p.n_heads;
   const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
 
-  float *sDL = reinterpret_cast<float *>(gb + OFF_MISC + MISC_DL);
+  // e^{L_C - L_ref} per d_k channel, one buffer per chunk parity: the S_r build of a chunk
+  // reads the previous chunk's factors while the elementwise pass writes this chunk's
+  static_assert(MISC_DL == MISC_DL0 + 512, "the two e^{L_C - L_ref} buffers are adjacent");
+  auto sDLb = [&](uint32_t parity) { return reinterpret_cast<float *>(gb + OFF_MISC + MISC_DL0 + 512u * parity); };
   float *sSM = reinterpret_cast<float *>(gb + OFF_MISC + MISC_SM);
   float *part = reinterpret_cast<float *>(gb + OFF_MISC + MISC_PART);
   float *sRef = reinterpret_cast<float *>(gb + OFF_MISC + MISC_REF);
@@ -210,9 +214,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(gb + OFF_MISC + MISC_TMEM);
-  const uint32_t tmD1 = tmem;        // G1 result; then W_r^T | (B V)^T; then M^T (128 cols)
-  const uint32_t tmS = tmem + 128;   // fp32 state (128 cols)
-  const uint32_t tmO = tmem + 384;   // O^T (64 cols)
+  // The state is held transposed, S^T (lane = d_v channel, column = d_k channel), so that
+  // S_r^T, R^T and -M^T -- the A operands of every state-side GEMM -- are read by the tensor
+  // core straight from TMEM as bf16 (two channels per column) and never visit shared memory.
+  const uint32_t tmD1 = tmem;        // G1 result; then R^T (cols 0-63) and M^T (cols 64-127), fp32
+  const uint32_t tmS = tmem + 128;   // S^T fp32 (128 cols)
+  const uint32_t tmO = tmem + 256;   // O^T fp32 (64 cols)
+  const uint32_t tmSR = tmem + 320;  // S_r^T bf16 A operand (64 cols)
+  const uint32_t tmRb = tmem + 384;  // R^T bf16 A operand (32 cols)
+  const uint32_t tmMb = tmem + 416;  // -M^T bf16 A operand (32 cols)
   const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
   uint32_t it = 0;                   // chunks processed by this CTA: parity of every mbarrier
 
@@ -271,19 +281,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       issue_tma_x(h, (int)bos);
     }
 
-    // ---- initial state into TMEM (thread: dk row `row`, dv columns [32 cg, 32 cg + 32))
+    // ---- initial state into TMEM as S^T (thread: dv channel `row`, dk columns [32 cg, 32 cg + 32));
+    //      each load instruction of a warp reads 32 consecutive dv entries of one dk row
     {
       uint32_t r[32];
       if (p.S0) {
-        const float4 *src = reinterpret_cast<const float4 *>(p.S0 + ((size_t)unit * D + row) * D + cg * 32);
+        const float *src = p.S0 + ((size_t)unit * D + cg * 32) * D + row;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float4 f = src[j];
-          r[4 * j] = __float_as_uint(f.x);
-          r[4 * j + 1] = __float_as_uint(f.y);
-          r[4 * j + 2] = __float_as_uint(f.z);
-          r[4 * j + 3] = __float_as_uint(f.w);
-        }
+        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(src[(size_t)j * D]);
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) r[j] = 0u;
@@ -291,10 +296,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       ptx::tmem_st32(tmS + lane_base + cg * 32, r);
       ptx::tmem_wait_st();
     }
-    // The state is kept as S = tau * Sacc (tau per dk row, this thread's row): each chunk's
-    // S_r build rewrites Sacc as e^{L_ref} S, the chunk's increment GEMMs accumulate onto
-    // it, and tau becomes e^{L_C - L_ref}: S' = e^{L_C - L_ref} (e^{L_ref} S + dS).
-    float tau = 1.f;
+    // The state is kept as S = Diag(tau) Sacc (tau per dk channel): each chunk's S_r build
+    // rewrites Sacc as e^{L_ref} S, the chunk's increment GEMMs accumulate onto it, and tau
+    // becomes that chunk's e^{L_C - L_ref}: S' = e^{L_C - L_ref} (e^{L_ref} S + dS).  tau is
+    // read from the previous chunk's sDLb buffer; it is 1 before the first chunk.
 
     for (int ci = 0; ci < nchunks; ++ci, ++it) {
       const uint32_t par = it & 1u;
@@ -343,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             if (j == 7) refv = run;
           }
           sRef[tid] = refv;
-          sDL[tid] = ptx::ex2((run - refv) * kLog2eF);
+          sDLb(par)[tid] = ptx::ex2((run - refv) * kLog2eF);
           sSM[tid] = ptx::ex2(refv * kLog2eF);
         }
         __syncthreads();
@@ -436,27 +441,34 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       }
       __syncthreads();
 
-      // ---- S_r = Diag(e^{L_ref}) S as a bf16 MN-major operand (dv columns [32 cg, 32 cg + 32));
-      //      the fp32 accumulator becomes the same e^{L_ref} S, onto which dS accumulates
+      // ---- S_r^T = S^T Diag(e^{L_ref}) as the bf16 TMEM A operand (thread: dv channel `row`,
+      //      dk columns [32 cg, 32 cg + 32)); the fp32 accumulator becomes the same, and the
+      //      chunk's increment GEMMs accumulate onto it
       {
         // two products, in this order: tau * Sacc is the state, O(1); e^{L_ref} tau alone can
         // underflow (both factors reach e^{-80} under the range precondition)
-        const float sm = sSM[row];
-        uint32_t r[32];
+        const float *tp = sDLb(par ^ 1u) + cg * 32;
+        const float *smv = sSM + cg * 32;
+        uint32_t r[32], hb[16];
         ptx::tmem_ld32(tmS + lane_base + cg * 32, r);
         ptx::tmem_wait_ld();
-        float f[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          f[j] = (__uint_as_float(r[j]) * tau) * sm;
-          r[j] = __float_as_uint(f[j]);
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 t4 = ci > 0 ? *reinterpret_cast<const float4 *>(tp + 4 * j4) : make_float4(1.f, 1.f, 1.f, 1.f);
+          const float4 s4 = *reinterpret_cast<const float4 *>(smv + 4 * j4);
+          const float f0 = (__uint_as_float(r[4 * j4]) * t4.x) * s4.x;
+          const float f1 = (__uint_as_float(r[4 * j4 + 1]) * t4.y) * s4.y;
+          const float f2 = (__uint_as_float(r[4 * j4 + 2]) * t4.z) * s4.z;
+          const float f3 = (__uint_as_float(r[4 * j4 + 3]) * t4.w) * s4.w;
+          r[4 * j4] = __float_as_uint(f0);
+          r[4 * j4 + 1] = __float_as_uint(f1);
+          r[4 * j4 + 2] = __float_as_uint(f2);
+          r[4 * j4 + 3] = __float_as_uint(f3);
+          hb[2 * j4] = pack_bf16x2(f0, f1);
+          hb[2 * j4 + 1] = pack_bf16x2(f2, f3);
         }
         ptx::tmem_st32(tmS + lane_base + cg * 32, r);
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8)
-          sts_v4(sb + OFF_SR + (uint32_t)(cg >> 1) * 16384u + swz(row, (uint32_t)((cg & 1) * 4 + q8)),
-                 pack8(f + 8 * q8, 1.f));
-        tau = sDL[row];
+        ptx::tmem_st16(tmSR + lane_base + cg * 16, hb);
         ptx::tmem_wait_st();
       }
       ptx::fence_proxy_async_smem();
@@ -529,17 +541,19 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       if (warp == kIssueWarp) {
         if (lane == 0 && !*sAbort) {
           ptx::tc_fence_after();
+          // dS^T = V^T p_r: A = V^T (MN-major), B = p_r as [tokens][dk] (MN-major, N = 128)
           constexpr uint32_t idS = ptx::idesc_bf16(128, 128, true, true);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            ptx::umma_bf16(tmS, ptx::sdesc_sw128(sb + OFF_XP + 8192 + kk * 2048, 16384, 1024),
-                           ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024), idS, 1);
+            ptx::umma_bf16(tmS, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
+                           ptx::sdesc_sw128(sb + OFF_XP + 8192 + kk * 2048, 16384, 1024), idS, 1);
+          constexpr uint32_t idT = ptx::idesc_bf16(128, 64, false, false);  // A from TMEM
           constexpr uint32_t idO = ptx::idesc_bf16(128, 64, true, false);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            ptx::umma_bf16(tmO, ptx::sdesc_sw128(sb + OFF_SR + kk * 2048, 16384, 1024),
-                           ptx::sdesc_sw128(sb + OFF_KQ + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32, 16, 1024), idO,
-                           kk > 0);
+            ptx::umma_bf16_ts(tmO, tmSR + kk * 8,
+                              ptx::sdesc_sw128(sb + OFF_KQ + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32, 16, 1024), idT,
+                              kk > 0);
           ptx::umma_commit(bar(BAR_E1));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
@@ -547,8 +561,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                            ptx::sdesc_sw128(sb + OFF_BM + kk * 32, 16, 1024), idO, kk > 0);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_SR + kk * 2048, 16384, 1024),
-                           ptx::sdesc_sw128(sb + OFF_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), idO, 1);
+            ptx::umma_bf16_ts(tmD1, tmSR + kk * 8,
+                              ptx::sdesc_sw128(sb + OFF_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), idT, 1);
           ptx::umma_commit(bar(BAR_GA));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
@@ -677,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       ptx::tc_fence_before();
       __syncthreads();
 
-      // ---- round trip of R^T (-> Rt, K-major [dv rows][64 tokens])
+      // ---- R^T (fp32, D1 cols 0-63) -> bf16 TMEM A operand
       wait_bar(bar(BAR_GA), par, sAbort, p.status);
       ptx::tc_fence_after();
       // the next chunk's k, q, v, log_a tiles can land once no MMA reads them
@@ -686,16 +700,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         issue_tma_a(h, t0 + C);
       }
       {
-        uint32_t r[16];
+        uint32_t r[16], hb[8];
         ptx::tmem_ld16(tmD1 + lane_base + cg * 16, r);
         ptx::tmem_wait_ld();
-        float f[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) f[j] = __uint_as_float(r[j]);
-#pragma unroll
-        for (int q8 = 0; q8 < 2; ++q8) sts_v4(sb + OFF_BZ + swz(row, (uint32_t)(cg * 2 + q8)), pack8(f + 8 * q8, 1.f));
+        for (int j = 0; j < 8; ++j) hb[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+        ptx::tmem_st8(tmRb + lane_base + cg * 8, hb);
+        ptx::tmem_wait_st();
       }
-      ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncthreads();
 
@@ -705,23 +717,20 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         constexpr uint32_t idM = ptx::idesc_bf16(128, 64, false, false);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmD1 + 64, ptx::sdesc_sw128(sb + OFF_BZ + kk * 32, 16, 1024),
-                         ptx::sdesc_sw128(sb + OFF_T + kk * 32, 16, 1024), idM, kk > 0);
+          ptx::umma_bf16_ts(tmD1 + 64, tmRb + kk * 8, ptx::sdesc_sw128(sb + OFF_T + kk * 32, 16, 1024), idM, kk > 0);
         ptx::umma_commit(bar(BAR_GB));
       }
       wait_bar(bar(BAR_GB), par, sAbort, p.status);
       ptx::tc_fence_after();
-      {
-        uint32_t r[16];
+      {  // -M^T -> bf16 TMEM A operand
+        uint32_t r[16], hb[8];
         ptx::tmem_ld16(tmD1 + 64 + lane_base + cg * 16, r);
         ptx::tmem_wait_ld();
-        float f[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) f[j] = __uint_as_float(r[j]);
-#pragma unroll
-        for (int q8 = 0; q8 < 2; ++q8) sts_v4(sb + OFF_MT + swz(row, (uint32_t)(cg * 2 + q8)), pack8(f + 8 * q8, -1.f));
+        for (int j = 0; j < 8; ++j) hb[j] = pack_bf16x2(-__uint_as_float(r[2 * j]), -__uint_as_float(r[2 * j + 1]));
+        ptx::tmem_st8(tmMb + lane_base + cg * 8, hb);
+        ptx::tmem_wait_st();
       }
-      ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncthreads();
 
@@ -733,13 +742,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         constexpr uint32_t idO = ptx::idesc_bf16(128, 64, false, false);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmO, ptx::sdesc_sw128(sb + OFF_MT + kk * 32, 16, 1024),
-                         ptx::sdesc_sw128(sb + OFF_QX + kk * 32, 16, 1024), idO, 1);
-        constexpr uint32_t idS = ptx::idesc_bf16(128, 128, true, false);
+          ptx::umma_bf16_ts(tmO, tmMb + kk * 8, ptx::sdesc_sw128(sb + OFF_QX + kk * 32, 16, 1024), idO, 1);
+        // dS^T += (-M^T) x_r: B = x_r as [tokens][dk] (MN-major, N = 128)
+        constexpr uint32_t idS = ptx::idesc_bf16(128, 128, false, true);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16(tmS, ptx::sdesc_sw128(sb + OFF_XP + kk * 2048, 16384, 1024),
-                         ptx::sdesc_sw128(sb + OFF_MT + kk * 32, 16, 1024), idS, 1);
+          ptx::umma_bf16_ts(tmS, tmMb + kk * 8, ptx::sdesc_sw128(sb + OFF_XP + kk * 2048, 16384, 1024), idS, 1);
         ptx::umma_commit(bar(BAR_G45));
       }
       wait_bar(bar(BAR_G45), par, sAbort, p.status);
@@ -794,17 +802,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       if (*sAbort) break;
     }
 
-    // ---- a8: final state
+    // ---- a8: final state S = Diag(tau) Sacc, from S^T (thread: dv channel `row`, dk rows
+    //      [32 cg, 32 cg + 32); each store instruction of a warp writes 32 consecutive dv entries)
     if (p.S_T && !*sAbort) {
-      float *dst = p.S_T + ((size_t)unit * D + row) * D + cg * 32;
+      float *dst = p.S_T + ((size_t)unit * D + cg * 32) * D + row;
+      const float *tp = sDLb((it & 1u) ^ 1u) + cg * 32;  // the last chunk's e^{L_C - L_ref}
       uint32_t r[32];
       ptx::tmem_ld32(tmS + lane_base + cg * 32, r);
       ptx::tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        reinterpret_cast<float4 *>(dst)[j] =
-            make_float4(tau * __uint_as_float(r[4 * j]), tau * __uint_as_float(r[4 * j + 1]),
-                        tau * __uint_as_float(r[4 * j + 2]), tau * __uint_as_float(r[4 * j + 3]));
+      for (int j = 0; j < 32; ++j) dst[(size_t)j * D] = (nchunks > 0 ? tp[j] : 1.f) * __uint_as_float(r[j]);
     }
     ptx::tc_fence_before();
     __syncthreads();
