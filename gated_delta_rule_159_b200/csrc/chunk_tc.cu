@@ -59,7 +59,7 @@ constexpr uint32_t OFF_KQ = 0;         // 2 K-blocks x [k_r rows 0-63 | q_r rows
 constexpr uint32_t OFF_XP = 32768;     // 2 K-blocks x [x_r rows | p_r rows]
 constexpr uint32_t OFF_V = 65536;      // 2 column blocks x [64 rows], 8 KB each
 constexpr uint32_t OFF_G = 81920;      // raw log_a tile
-                                       // [98304, 131072) unused
+constexpr uint32_t OFF_OS = 98304;     // o staging: 2 (bf16) or 4 (fp32) sub-blocks of [64 tokens][128 B]
 constexpr uint32_t OFF_T = 131072;     // T bf16 [64 x 64]
 constexpr uint32_t OFF_BM = 139264;    // B bf16 [64 x 64]
 constexpr uint32_t OFF_QX = 147456;    // QX bf16 [64 x 64]
@@ -67,7 +67,6 @@ constexpr uint32_t OFF_QP = 155648;    // QP bf16 [64 x 64]
 constexpr uint32_t OFF_AF = 163840;    // fp32 A [64 x 68] (masks -> solve)
 constexpr uint32_t OFF_TF = 181248;    // fp32 T [64 x 68] (solve)
 constexpr uint32_t OFF_XS = 198656;    // fp32 solve scratch, <= 4 KB
-constexpr uint32_t OFF_BZ = 180224;    // o staging (after the solve; overlaps A/T)
 constexpr uint32_t OFF_MISC = 212992;
 constexpr uint32_t MISC_DL0 = 0;       // float[128]  e^{L_C - L_ref} of the chunks with even parity
 constexpr uint32_t MISC_DL = 512;      // float[128]  e^{L_C - L_ref} of the chunks with odd parity
@@ -104,6 +103,13 @@ __device__ __forceinline__ void sts_v2(uint32_t a, uint2 v) {
 }
 __device__ __forceinline__ void sts_u16(uint32_t a, uint16_t v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(v) : "memory");
+}
+__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint16_t bf16_bits(float v) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  return *reinterpret_cast<const uint16_t *>(&h);
 }
 __device__ __forceinline__ void sts_f32(uint32_t a, float v) {
   asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
@@ -190,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   float *sSM = reinterpret_cast<float *>(gb + OFF_MISC + MISC_SM);
   float *part = reinterpret_cast<float *>(gb + OFF_MISC + MISC_PART);
   float *sRef = reinterpret_cast<float *>(gb + OFF_MISC + MISC_REF);
-  constexpr int kIssuer = 32;      // issues the TMA loads and the output stores (warp 1, lane 0)
+  constexpr int kIssuer = 32;      // issues the first TMA loads of a unit, the b loads and the o stores
   constexpr int kIssueWarp = 15;   // issues the T-independent MMAs during the solve
   constexpr int kSolveThreads = 480;  // warps 0-14
   enum { NB_SOLVE = 1 };
@@ -198,6 +204,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   volatile int *sUnit = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_UNIT);
   auto bar = [&](int i) { return sb + OFF_MISC + MISC_BAR + 8u * (uint32_t)i; };
 
+  // the bf16 T tile's blocks above the diagonal are never written by the solve: zero once
+  sts_v4(sb + OFF_T + 16u * (uint32_t)tid, make_uint4(0u, 0u, 0u, 0u));
+  static_assert(kThreads * 16 == 8192, "one 16-byte store per thread zeroes the 8 KB T tile");
   if (tid == 0) {
     for (int i = 0; i < kNumBars; ++i) ptx::mbar_init(bar(i), 1);
     ptx::fence_mbar_init();
@@ -308,7 +317,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       const int t0 = (int)(bos + c0);
       const bool has_next = ci + 1 < nchunks;
 
-      if (tid == kIssuer) ptx::bulk_wait_group_read0();  // previous chunk's o store has read its staging
       wait_bar(bar(BAR_TMA_A), par, sAbort, p.status);
       if (!kScalarGates) wait_bar(bar(BAR_TMA_W), par, sAbort, p.status);
 
@@ -572,6 +580,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           if (has_next) {  // p_r is dead once dS = p_r^T V is done: the next chunk's w can land
             wait_bar(bar(BAR_E1), par, sAbort, p.status);
             if (!*sAbort) issue_tma_w(h, t0 + C);
+            // k_r, q_r and V are dead once E2 (after GA) is done: the next chunk's k, q, v,
+            // log_a tiles can land (the solve runs meanwhile, so this wait delays nobody)
+            wait_bar(bar(BAR_E2), par, sAbort, p.status);
+            if (!*sAbort) issue_tma_a(h, t0 + C);
           }
         }
         __syncwarp();
@@ -580,7 +592,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       // ---- a5: T = (I + A)^-1 (fp32).  8x8 diagonal blocks by forward substitution, then three
       //      merge levels: for each pair of diagonal blocks of size s (upper U, lower L) of the
       //      merged 2s block, T_LU = -T_LL (A_LU T_UU).  Blocks above the diagonal are never
-      //      read (loops stop at the triangle), so they are never written either.
+      //      read (loops stop at the triangle), so they are never written either.  Each block
+      //      also goes to the bf16 T tile (the MMA operand) as soon as it is final; the tile's
+      //      blocks above the diagonal hold the zeros written at the kernel's start.
       {
         const float *Af = reinterpret_cast<const float *>(gb + OFF_AF);
         float *Tf = reinterpret_cast<float *>(gb + OFF_TF);
@@ -605,7 +619,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             t[i] = acc;
           }
 #pragma unroll
-          for (int i = 0; i < 8; ++i) Tf[fidx(r0 + i, r0 + m)] = t[i];
+          for (int i = 0; i < 8; ++i) {
+            Tf[fidx(r0 + i, r0 + m)] = t[i];
+            sts_u16(sb + OFF_T + swz(r0 + i, (uint32_t)(r0 >> 3)) + (uint32_t)m * 2u, bf16_bits(t[i]));
+          }
         }
         named_bar(NB_SOLVE, kSolveThreads);
         // s = 8: 4 pairs x 64 outputs on CUDA cores
@@ -623,28 +640,40 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
 #pragma unroll
           for (int k = 0; k < 8; ++k) acc -= (k <= r ? Tf[fidx(l0 + r, l0 + k)] * Xs[pr * 64 + k * 8 + c] : 0.f);
           Tf[fidx(l0 + r, u0 + c)] = acc;
+          sts_u16(sb + OFF_T + swz(l0 + r, (uint32_t)(u0 >> 3)) + (uint32_t)c * 2u, bf16_bits(acc));
         }
         named_bar(NB_SOLVE, kSolveThreads);
-        // s = 16 (2 pairs) and s = 32 (1 pair) on tf32 mma.sync: one warp per 16x8 output tile
+        // s = 16 (2 pairs) and s = 32 (1 pair) on tf32 mma.sync: one warp per 16x8 output tile.
+        // Every fragment of a step is loaded before its chain of MMAs starts.
         const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
         for (int lev = 1; lev < 3; ++lev) {
           const int sz = 8 << lev;                   // 16, 32
+          const int nk = sz / 8;                     // 8-wide K steps: 2, 4
           const int tpp = (sz / 16) * (sz / 8);      // 16x8 tiles per pair: 2, 8
           const int ntiles = (64 / (2 * sz)) * tpp;  // 4, 8
-          // step a: X = A_LU T_UU (only k >= the tile's first column contributes)
+          const int pr = warp / tpp, ti = warp % tpp, mt = ti / (sz / 8), nt = ti % (sz / 8);
+          const int u0 = pr * 2 * sz, l0 = u0 + sz, rr = 16 * mt, cc = 8 * nt;
+          // step a: X = A_LU T_UU (only K steps from the tile's first column on contribute;
+          // the blocks of T_UU above its diagonal were never written)
           if (warp < ntiles) {
-            const int pr = warp / tpp, ti = warp % tpp, mt = ti / (sz / 8), nt = ti % (sz / 8);
-            const int u0 = pr * 2 * sz, l0 = u0 + sz, rr = 16 * mt, cc = 8 * nt;
-            float x[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int kk = cc / 8; kk < sz / 8; ++kk) {
-              const int kc = u0 + 8 * kk + t4;
-              const uint32_t av[4] = {ptx::to_tf32(Af[fidx(l0 + rr + g, kc)]), ptx::to_tf32(Af[fidx(l0 + rr + g + 8, kc)]),
-                                      ptx::to_tf32(Af[fidx(l0 + rr + g, kc + 4)]),
-                                      ptx::to_tf32(Af[fidx(l0 + rr + g + 8, kc + 4)])};
-              const uint32_t bv[2] = {ptx::to_tf32(Tf[fidx(kc, u0 + cc + g)]), ptx::to_tf32(Tf[fidx(kc + 4, u0 + cc + g)])};
-              ptx::mma_tf32_16x8x8(x, av, bv);
+            uint32_t av[4][4], bv[4][2];
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              if (kk < nk && kk >= nt) {
+                const int kc = u0 + 8 * kk + t4;
+                av[kk][0] = ptx::to_tf32(Af[fidx(l0 + rr + g, kc)]);
+                av[kk][1] = ptx::to_tf32(Af[fidx(l0 + rr + g + 8, kc)]);
+                av[kk][2] = ptx::to_tf32(Af[fidx(l0 + rr + g, kc + 4)]);
+                av[kk][3] = ptx::to_tf32(Af[fidx(l0 + rr + g + 8, kc + 4)]);
+                bv[kk][0] = ptx::to_tf32(Tf[fidx(kc, u0 + cc + g)]);
+                bv[kk][1] = ptx::to_tf32(Tf[fidx(kc + 4, u0 + cc + g)]);
+              }
             }
+            float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              if (kk < nk && kk >= nt) ptx::mma_tf32_16x8x8(x, av[kk], bv[kk]);
             float *xs = Xs + pr * sz * sz;
             xs[(rr + g) * sz + cc + 2 * t4] = x[0];
             xs[(rr + g) * sz + cc + 2 * t4 + 1] = x[1];
@@ -652,38 +681,38 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             xs[(rr + g + 8) * sz + cc + 2 * t4 + 1] = x[3];
           }
           named_bar(NB_SOLVE, kSolveThreads);
-          // step b: T_LU = -T_LL X (only k <= the tile's last row contributes)
+          // step b: T_LU = -T_LL X (only K steps up to the tile's last row contribute)
           if (warp < ntiles) {
-            const int pr = warp / tpp, ti = warp % tpp, mt = ti / (sz / 8), nt = ti % (sz / 8);
-            const int u0 = pr * 2 * sz, l0 = u0 + sz, rr = 16 * mt, cc = 8 * nt;
             const float *xs = Xs + pr * sz * sz;
-            float y[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int kk = 0; kk <= (rr + 15) / 8; ++kk) {
-              // T_LL is lower triangular; its 8x8 blocks above the diagonal were never written
-              const int kc = l0 + 8 * kk + t4, kr = 8 * kk + t4;
-              const uint32_t av[4] = {
-                  ptx::to_tf32(kr <= rr + g ? Tf[fidx(l0 + rr + g, kc)] : 0.f),
-                  ptx::to_tf32(kr <= rr + g + 8 ? Tf[fidx(l0 + rr + g + 8, kc)] : 0.f),
-                  ptx::to_tf32(kr + 4 <= rr + g ? Tf[fidx(l0 + rr + g, kc + 4)] : 0.f),
-                  ptx::to_tf32(kr + 4 <= rr + g + 8 ? Tf[fidx(l0 + rr + g + 8, kc + 4)] : 0.f)};
-              const uint32_t bv[2] = {ptx::to_tf32(xs[(8 * kk + t4) * sz + cc + g]),
-                                      ptx::to_tf32(xs[(8 * kk + t4 + 4) * sz + cc + g])};
-              ptx::mma_tf32_16x8x8(y, av, bv);
-            }
-            Tf[fidx(l0 + rr + g, u0 + cc + 2 * t4)] = -y[0];
-            Tf[fidx(l0 + rr + g, u0 + cc + 2 * t4 + 1)] = -y[1];
-            Tf[fidx(l0 + rr + g + 8, u0 + cc + 2 * t4)] = -y[2];
-            Tf[fidx(l0 + rr + g + 8, u0 + cc + 2 * t4 + 1)] = -y[3];
-          }
-          named_bar(NB_SOLVE, kSolveThreads);
-        }
-        // T -> bf16 tile (zeros above the diagonal), by the solve warps
-        for (int e = tid; e < 512; e += kSolveThreads) {
-          const int i = e >> 3, seg = e & 7;
-          float f[8];
+            uint32_t av[4][4], bv[4][2];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) f[j] = (8 * seg + j <= i) ? Tf[fidx(i, 8 * seg + j)] : 0.f;
-          sts_v4(sb + OFF_T + swz(i, (uint32_t)seg), pack8(f, 1.f));
+            for (int kk = 0; kk < 4; ++kk) {
+              if (kk < nk && kk <= (rr + 15) / 8) {
+                // T_LL is lower triangular; its 8x8 blocks above the diagonal were never written
+                const int kc = l0 + 8 * kk + t4, kr = 8 * kk + t4;
+                av[kk][0] = ptx::to_tf32(kr <= rr + g ? Tf[fidx(l0 + rr + g, kc)] : 0.f);
+                av[kk][1] = ptx::to_tf32(kr <= rr + g + 8 ? Tf[fidx(l0 + rr + g + 8, kc)] : 0.f);
+                av[kk][2] = ptx::to_tf32(kr + 4 <= rr + g ? Tf[fidx(l0 + rr + g, kc + 4)] : 0.f);
+                av[kk][3] = ptx::to_tf32(kr + 4 <= rr + g + 8 ? Tf[fidx(l0 + rr + g + 8, kc + 4)] : 0.f);
+                bv[kk][0] = ptx::to_tf32(xs[(8 * kk + t4) * sz + cc + g]);
+                bv[kk][1] = ptx::to_tf32(xs[(8 * kk + t4 + 4) * sz + cc + g]);
+              }
+            }
+            float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              if (kk < nk && kk <= (rr + 15) / 8) ptx::mma_tf32_16x8x8(y, av[kk], bv[kk]);
+            const int ri = l0 + rr + g, cj = u0 + cc + 2 * t4;
+            if (lev == 1) {  // the last level's T_LU is read by no later level: bf16 only
+              Tf[fidx(ri, cj)] = -y[0];
+              Tf[fidx(ri, cj + 1)] = -y[1];
+              Tf[fidx(ri + 8, cj)] = -y[2];
+              Tf[fidx(ri + 8, cj + 1)] = -y[3];
+            }
+            sts_u32(sb + OFF_T + swz(ri, (uint32_t)(cj >> 3)) + (uint32_t)(cj & 7) * 2u, pack_bf16x2(-y[0], -y[1]));
+            sts_u32(sb + OFF_T + swz(ri + 8, (uint32_t)(cj >> 3)) + (uint32_t)(cj & 7) * 2u, pack_bf16x2(-y[2], -y[3]));
+          }
+          if (lev == 1) named_bar(NB_SOLVE, kSolveThreads);
         }
         }  // solve scope
       }  // warps 0-14
@@ -694,11 +723,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       // ---- R^T (fp32, D1 cols 0-63) -> bf16 TMEM A operand
       wait_bar(bar(BAR_GA), par, sAbort, p.status);
       ptx::tc_fence_after();
-      // the next chunk's k, q, v, log_a tiles can land once no MMA reads them
-      if (tid == kIssuer && has_next && !*sAbort) {
-        wait_bar(bar(BAR_E2), par, sAbort, p.status);  // E1, GA and E2 share one issuing thread
-        issue_tma_a(h, t0 + C);
-      }
       {
         uint32_t r[16], hb[8];
         ptx::tmem_ld16(tmD1 + lane_base + cg * 16, r);
@@ -731,6 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         ptx::tmem_st8(tmMb + lane_base + cg * 8, hb);
         ptx::tmem_wait_st();
       }
+      if (tid == kIssuer) ptx::bulk_wait_group_read0();  // the previous chunk's o store has read the staging
       ptx::tc_fence_before();
       __syncthreads();
 
@@ -767,23 +792,23 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           const float f = __uint_as_float(r[j]);
           if (sizeof(Tout) == 2) {
             const __nv_bfloat16 hv = __float2bfloat16_rn(f);
-            sts_u16(sb + OFF_BZ + (uint32_t)(row >> 6) * 8192u + (uint32_t)i * 128u + (uint32_t)(row & 63) * 2u,
+            sts_u16(sb + OFF_OS + (uint32_t)(row >> 6) * 8192u + (uint32_t)i * 128u + (uint32_t)(row & 63) * 2u,
                     *reinterpret_cast<const uint16_t *>(&hv));
           } else {
-            sts_f32(sb + OFF_BZ + (uint32_t)(row >> 5) * 8192u + (uint32_t)i * 128u + (uint32_t)(row & 31) * 4u, f);
+            sts_f32(sb + OFF_OS + (uint32_t)(row >> 5) * 8192u + (uint32_t)i * 128u + (uint32_t)(row & 31) * 4u, f);
           }
         }
       }
       ptx::fence_proxy_async_smem();  // staging is read by the TMA store below
       __syncthreads();
       if (nvalid == C) {
-        // full chunk: asynchronous TMA store; the staging area is not rewritten before the
-        // next chunk's solve, which first waits for these reads (bulk_wait_group_read0)
+        // full chunk: asynchronous TMA store; the next chunk's epilogue rewrites the staging
+        // area only after the issuing thread has seen these reads done (bulk_wait_group_read0)
         if (tid == kIssuer) {
           constexpr int kBoxC = sizeof(Tout) == 2 ? 64 : 32;
 #pragma unroll
           for (int sbk = 0; sbk < D / kBoxC; ++sbk)
-            ptx::tma_store_3d(&P.tm_o, sb + OFF_BZ + (uint32_t)sbk * 8192u, sbk * kBoxC, h, t0);
+            ptx::tma_store_3d(&P.tm_o, sb + OFF_OS + (uint32_t)sbk * 8192u, sbk * kBoxC, h, t0);
           ptx::bulk_commit_group();
         }
       } else {
@@ -793,7 +818,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         uint8_t *go = static_cast<uint8_t *>(p.o);
         for (int e = tid; e < nvalid * kU4; e += kThreads) {
           const int i = e / kU4, uu = e % kU4;
-          const uint4 val = lds_v4(sb + OFF_BZ + (uint32_t)(uu >> 3) * 8192u + (uint32_t)i * 128u + (uint32_t)(uu & 7) * 16u);
+          const uint4 val = lds_v4(sb + OFF_OS + (uint32_t)(uu >> 3) * 8192u + (uint32_t)i * 128u + (uint32_t)(uu & 7) * 16u);
           *reinterpret_cast<uint4 *>(go + ((size_t)(t0 + i) * H + h) * kRowBytes + uu * 16) = val;
         }
       }
