@@ -73,14 +73,15 @@ constexpr uint32_t MISC_DL = 512;      // float[128]  e^{L_C - L_ref} of the chu
 constexpr uint32_t MISC_SM = 1024;     // float[128]  e^{L_ref}
 constexpr uint32_t MISC_PART = 1536;   // float[16][128] 4-row sums of log_a, then exclusive prefixes
 constexpr uint32_t MISC_REF = 9728;    // float[128]  L_ref
-constexpr uint32_t MISC_BAR = 10240;   // 9 mbarriers
+constexpr uint32_t MISC_BAR = 10240;   // 10 mbarriers
 constexpr uint32_t MISC_TMEM = 10320;
 constexpr uint32_t MISC_ABORT = 10324;
 constexpr uint32_t MISC_UNIT = 10328;
 constexpr uint32_t MISC_BYTES = 10336;
 constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES + 1024;  // + base alignment slack
 // mbarrier slots
-enum { BAR_TMA_A = 0, BAR_TMA_W, BAR_TMA_X, BAR_G1, BAR_E1, BAR_E2, BAR_GA, BAR_GB, BAR_G45, kNumBars };
+enum { BAR_TMA_A = 0, BAR_TMA_W, BAR_TMA_X, BAR_G1, BAR_E1, BAR_E2, BAR_GA, BAR_GB, BAR_G4, BAR_G5, kNumBars };
+static_assert(MISC_BAR + 8 * kNumBars <= MISC_TMEM, "mbarriers overlap the TMEM address slot");
 
 struct TcParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_g, tm_b, tm_w;
@@ -251,8 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       if (!kScalarDecay) ptx::tma_load_3d(sb + OFF_G + kb * 8192, &P.tm_g, kb * 64, h, t0, bar(BAR_TMA_A));
     }
   };
-  // w lands in the p_r halves of XP (free once dS = p_r^T V is done), b in the x_r halves
-  // (free once the last GEMM of the chunk is done)
+  // w lands in the p_r halves of XP (free once dS = p_r^T V is done), b in the log_a slot
+  // (free once the cumulative decay of its chunk is done)
   auto issue_tma_w = [&](int h, int t0) {
     if (kScalarGates) return;
     ptx::mbar_arrive_expect_tx(bar(BAR_TMA_W), 2u * 8192u);
@@ -265,7 +266,145 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     ptx::mbar_arrive_expect_tx(bar(BAR_TMA_X), 2u * 8192u);
 #pragma unroll
     for (int kb = 0; kb < 2; ++kb)
-      ptx::tma_load_3d(sb + OFF_XP + kb * 16384, &P.tm_b, kb * 64, h, t0, bar(BAR_TMA_X));
+      ptx::tma_load_3d(sb + OFF_G + kb * 8192, &P.tm_b, kb * 64, h, t0, bar(BAR_TMA_X));
+  };
+
+  // ---- a2/a3: cumulative log-decay and scaled operands of one chunk (rows t0n .. t0n + 63 of
+  //      head h, the first nvn of them valid), in place, in three passes that the chunk loop
+  //      runs between the previous chunk's GEMMs.  Thread: channels 4 lane .. 4 lane + 3,
+  //      rows 4 warp .. 4 warp + 3.
+  const int e_kb = lane >> 4;
+  const uint32_t e_ch16 = (uint32_t)((lane & 15) >> 1), e_cofs = (uint32_t)(lane & 1) * 8u;
+  // pass 1 (needs the log_a tile): inclusive cumsum L of this thread's rows, then per channel
+  // the exclusive prefixes over the 16 row groups, L_ref = L_31, e^{L_C - L_ref} into the
+  // parity-pn buffer and e^{L_ref}.  Ends with a CTA barrier, after which the log_a slot is free.
+  auto elem_cumsum = [&](uint32_t pn, int t0n, int nvn, int h, float4 (&L)[4]) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+      const int r = warp * 4 + rr;
+      float4 g = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < nvn) {
+        if (kScalarDecay) {
+          float sv = __bfloat162float(g_la[(size_t)(t0n + r) * H + h]);
+          if (kProlog) sv = log_sigmoid_f(sv);
+          g = make_float4(sv, sv, sv, sv);
+        } else {
+          g = unpack4(lds_v2(sb + OFF_G + e_kb * 8192 + swz(r, e_ch16) + e_cofs));
+          if (kProlog) g = make_float4(log_sigmoid_f(g.x), log_sigmoid_f(g.y), log_sigmoid_f(g.z), log_sigmoid_f(g.w));
+        }
+      }
+      acc.x += g.x; acc.y += g.y; acc.z += g.z; acc.w += g.w;
+      L[rr] = acc;
+    }
+    *reinterpret_cast<float4 *>(part + warp * 128 + 4 * lane) = acc;
+    __syncthreads();
+    if (tid < D) {  // per channel: exclusive prefix over the 16 row groups, L_ref = L_31, L_C = L_63
+      float run = 0.f, refv = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float pj = part[j * 128 + tid];
+        part[j * 128 + tid] = run;
+        run += pj;
+        if (j == 7) refv = run;
+      }
+      sRef[tid] = refv;
+      sDLb(pn)[tid] = ptx::ex2((run - refv) * kLog2eF);
+      sSM[tid] = ptx::ex2(refv * kLog2eF);
+    }
+    __syncthreads();
+  };
+  // pass 2 (needs the k, q, v tiles and the w tile): k_r, q_r and p_r in place; rows past the
+  // chunk end are zeroed (v too).  ke2 keeps k e^{L_ref - L} for pass 3.
+  auto elem_scale = [&](int t0n, int nvn, int h, const float4 (&L)[4], float4 (&ke2)[4]) {
+    const float4 off = *reinterpret_cast<const float4 *>(part + warp * 128 + 4 * lane);
+    const float4 ref = *reinterpret_cast<const float4 *>(sRef + 4 * lane);
+    const float4 base = make_float4((off.x - ref.x) * kLog2eF, (off.y - ref.y) * kLog2eF,
+                                    (off.z - ref.z) * kLog2eF, (off.w - ref.w) * kLog2eF);
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+      const int r = warp * 4 + rr;
+      const uint32_t o = (uint32_t)e_kb * 16384u + swz(r, e_ch16) + e_cofs;
+      const float l0 = fmaf(L[rr].x, kLog2eF, base.x), l1 = fmaf(L[rr].y, kLog2eF, base.y);
+      const float l2 = fmaf(L[rr].z, kLog2eF, base.z), l3 = fmaf(L[rr].w, kLog2eF, base.w);
+      const float e10 = ptx::ex2(l0), e11 = ptx::ex2(l1), e12 = ptx::ex2(l2), e13 = ptx::ex2(l3);
+      const float4 e2 = make_float4(ptx::ex2(-l0), ptx::ex2(-l1), ptx::ex2(-l2), ptx::ex2(-l3));
+      float4 kk = unpack4(lds_v2(sb + OFF_KQ + o));
+      float4 qq = unpack4(lds_v2(sb + OFF_KQ + o + 8192));
+      float4 ww;  // the write gate w (the erase gate b in the gist.science form)
+      if (kScalarGates) {
+        ww = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < nvn) {
+          float swv = __bfloat162float((kP3 ? g_b : g_w)[(size_t)(t0n + r) * H + h]);
+          if (kProlog) swv = sigmoid_f(swv);
+          ww = make_float4(swv, swv, swv, swv);
+        }
+      } else {
+        ww = unpack4(lds_v2(sb + OFF_XP + o + 8192));
+        if (kProlog) ww = make_float4(sigmoid_f(ww.x), sigmoid_f(ww.y), sigmoid_f(ww.z), sigmoid_f(ww.w));
+      }
+      if (r >= nvn) {
+        kk = make_float4(0.f, 0.f, 0.f, 0.f);
+        qq = kk;
+        ww = kk;
+        sts_v2(sb + OFF_V + e_kb * 8192 + swz(r, e_ch16) + e_cofs, make_uint2(0u, 0u));
+      }
+      if (kProlog) {  // the 32 lanes of this warp hold the row's 128 channels
+        float k2 = kk.x * kk.x + kk.y * kk.y + kk.z * kk.z + kk.w * kk.w;
+        float q2 = qq.x * qq.x + qq.y * qq.y + qq.z * qq.z + qq.w * qq.w;
+#pragma unroll
+        for (int sh = 16; sh >= 1; sh >>= 1) {
+          k2 += __shfl_xor_sync(0xffffffffu, k2, sh);
+          q2 += __shfl_xor_sync(0xffffffffu, q2, sh);
+        }
+        const float ik = rsqrtf(k2 + kNormEps), iq = rsqrtf(q2 + kNormEps);
+        kk = make_float4(kk.x * ik, kk.y * ik, kk.z * ik, kk.w * ik);
+        qq = make_float4(qq.x * iq, qq.y * iq, qq.z * iq, qq.w * iq);
+      }
+      ke2[rr] = make_float4(kk.x * e2.x, kk.y * e2.y, kk.z * e2.z, kk.w * e2.w);
+      const float4 ke = ke2[rr];
+      if (kP3) {
+        sts_v2(sb + OFF_KQ + o, pack4(ww.x * kk.x * e10, ww.y * kk.y * e11, ww.z * kk.z * e12, ww.w * kk.w * e13));
+        sts_v2(sb + OFF_XP + o + 8192, pack4(ke.x, ke.y, ke.z, ke.w));
+      } else {
+        sts_v2(sb + OFF_KQ + o, pack4(kk.x * e10, kk.y * e11, kk.z * e12, kk.w * e13));
+        sts_v2(sb + OFF_XP + o + 8192, pack4(ww.x * ke.x, ww.y * ke.y, ww.z * ke.z, ww.w * ke.w));
+      }
+      sts_v2(sb + OFF_KQ + o + 8192, pack4(qq.x * e10, qq.y * e11, qq.z * e12, qq.w * e13));
+    }
+  };
+  // pass 3 (needs the b tile, which lands in the log_a slot, and a free x_r slot): x_r = b.k
+  // e^{L_ref - L}; in the gist.science form x_r = k e^{L_ref - L} and the values are scaled by
+  // the value gate.
+  auto elem_x = [&](int t0n, int nvn, int h, const float4 (&ke2)[4]) {
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+      const int r = warp * 4 + rr;
+      const uint32_t o = (uint32_t)e_kb * 16384u + swz(r, e_ch16) + e_cofs;
+      float4 bb;  // the erase gate b (the value gate w in the gist.science form)
+      if (kScalarGates) {
+        bb = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < nvn) {
+          float sbv = __bfloat162float((kP3 ? g_w : g_b)[(size_t)(t0n + r) * H + h]);
+          if (kProlog) sbv = sigmoid_f(sbv);
+          bb = make_float4(sbv, sbv, sbv, sbv);
+        }
+      } else {
+        bb = unpack4(lds_v2(sb + OFF_G + e_kb * 8192 + swz(r, e_ch16) + e_cofs));
+        if (kProlog) bb = make_float4(sigmoid_f(bb.x), sigmoid_f(bb.y), sigmoid_f(bb.z), sigmoid_f(bb.w));
+      }
+      const float4 ke = ke2[rr];
+      if (kP3) {
+        sts_v2(sb + OFF_XP + o, pack4(ke.x, ke.y, ke.z, ke.w));
+        if (r < nvn) {  // rows past the chunk end were zeroed in pass 2
+          const uint32_t ov = sb + OFF_V + (uint32_t)e_kb * 8192u + swz(r, e_ch16) + e_cofs;
+          const float4 vv = unpack4(lds_v2(ov));
+          sts_v2(ov, pack4(vv.x * bb.x, vv.y * bb.y, vv.z * bb.z, vv.w * bb.w));
+        }
+      } else {
+        sts_v2(sb + OFF_XP + o, pack4(bb.x * ke.x, bb.y * ke.y, bb.z * ke.z, bb.w * ke.w));
+      }
+    }
   };
 
   for (;;) {
@@ -287,7 +426,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     if (tid == kIssuer && nchunks > 0 && !*sAbort) {
       issue_tma_a(h, (int)bos);
       issue_tma_w(h, (int)bos);
-      issue_tma_x(h, (int)bos);
     }
 
     // ---- initial state into TMEM as S^T (thread: dv channel `row`, dk columns [32 cg, 32 cg + 32));
@@ -310,144 +448,44 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     // becomes that chunk's e^{L_C - L_ref}: S' = e^{L_C - L_ref} (e^{L_ref} S + dS).  tau is
     // read from the previous chunk's sDLb buffer; it is 1 before the first chunk.
 
+    // The operands of chunk c + 1 are built while chunk c's GEMMs run; a unit's first chunk
+    // builds them here.
+    float4 L[4], ke2[4];
+    if (nchunks > 0) {
+      const int nv0 = (int)(len < C ? len : C);
+      const uint32_t par0 = it & 1u;
+      wait_bar(bar(BAR_TMA_A), par0, sAbort, p.status);
+      elem_cumsum(par0, (int)bos, nv0, h, L);
+      if (tid == kIssuer && !*sAbort) issue_tma_x(h, (int)bos);
+      if (!kScalarGates) wait_bar(bar(BAR_TMA_W), par0, sAbort, p.status);
+      elem_scale((int)bos, nv0, h, L, ke2);
+      if (!kScalarGates) wait_bar(bar(BAR_TMA_X), par0, sAbort, p.status);
+      elem_x((int)bos, nv0, h, ke2);
+      ptx::fence_proxy_async_smem();
+      __syncthreads();
+    }
+
     for (int ci = 0; ci < nchunks; ++ci, ++it) {
       const uint32_t par = it & 1u;
       const int64_t c0 = (int64_t)ci * C;
       const int nvalid = (int)((len - c0) < C ? (len - c0) : C);
       const int t0 = (int)(bos + c0);
       const bool has_next = ci + 1 < nchunks;
+      const int nvalid_next = has_next ? (int)((len - c0 - C) < C ? (len - c0 - C) : C) : 0;
 
-      wait_bar(bar(BAR_TMA_A), par, sAbort, p.status);
-      if (!kScalarGates) wait_bar(bar(BAR_TMA_W), par, sAbort, p.status);
-
-      // ---- a2/a3: cumulative log-decay and scaled operands, in place.
-      // thread: channels 4 cq .. 4 cq + 3, rows 4 warp .. 4 warp + 3.
-      {
-        const int cq = lane, kb = cq >> 4;
-        const uint32_t ch16 = (uint32_t)((cq & 15) >> 1), cofs = (uint32_t)(cq & 1) * 8u;
-        float4 L[4];
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      // ---- a4: G1 [A B; QX QP] = [k_r; q_r] [x_r; p_r]^T, issued first: it needs only this
+      //      chunk's operands (built during the previous chunk) and runs under the S_r build
+      if (tid == 0 && !*sAbort) {
+        ptx::tc_fence_after();
+        constexpr uint32_t id1 = ptx::idesc_bf16(128, kXP ? 64 : 128, false, false);
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-          const int r = warp * 4 + rr;
-          float4 g = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (r < nvalid) {
-            if (kScalarDecay) {
-              float s = __bfloat162float(g_la[(size_t)(t0 + r) * H + h]);
-              if (kProlog) s = log_sigmoid_f(s);
-              g = make_float4(s, s, s, s);
-            } else {
-              g = unpack4(lds_v2(sb + OFF_G + kb * 8192 + swz(r, ch16) + cofs));
-              if (kProlog) g = make_float4(log_sigmoid_f(g.x), log_sigmoid_f(g.y), log_sigmoid_f(g.z), log_sigmoid_f(g.w));
-            }
-          }
-          acc.x += g.x; acc.y += g.y; acc.z += g.z; acc.w += g.w;
-          L[rr] = acc;
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t ko = (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
+          ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_KQ + ko, 16, 1024),
+                         ptx::sdesc_sw128(sb + OFF_XP + ko, 16, 1024), id1, kk > 0);
         }
-        *reinterpret_cast<float4 *>(part + warp * 128 + 4 * cq) = acc;
-        __syncthreads();
-        if (tid < D) {  // per channel: exclusive prefix over the 16 row groups, L_ref = L_31, L_C = L_63
-          float run = 0.f, refv = 0.f;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float pj = part[j * 128 + tid];
-            part[j * 128 + tid] = run;
-            run += pj;
-            if (j == 7) refv = run;
-          }
-          sRef[tid] = refv;
-          sDLb(par)[tid] = ptx::ex2((run - refv) * kLog2eF);
-          sSM[tid] = ptx::ex2(refv * kLog2eF);
-        }
-        __syncthreads();
-        const float4 off = *reinterpret_cast<const float4 *>(part + warp * 128 + 4 * cq);
-        const float4 ref = *reinterpret_cast<const float4 *>(sRef + 4 * cq);
-        const float4 base = make_float4((off.x - ref.x) * kLog2eF, (off.y - ref.y) * kLog2eF,
-                                        (off.z - ref.z) * kLog2eF, (off.w - ref.w) * kLog2eF);
-        float4 kraw[4], e2v[4];
-#pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-          const int r = warp * 4 + rr;
-          const uint32_t o = (uint32_t)kb * 16384u + swz(r, ch16) + cofs;
-          const float l0 = fmaf(L[rr].x, kLog2eF, base.x), l1 = fmaf(L[rr].y, kLog2eF, base.y);
-          const float l2 = fmaf(L[rr].z, kLog2eF, base.z), l3 = fmaf(L[rr].w, kLog2eF, base.w);
-          const float e10 = ptx::ex2(l0), e11 = ptx::ex2(l1), e12 = ptx::ex2(l2), e13 = ptx::ex2(l3);
-          e2v[rr] = make_float4(ptx::ex2(-l0), ptx::ex2(-l1), ptx::ex2(-l2), ptx::ex2(-l3));
-          float4 kk = unpack4(lds_v2(sb + OFF_KQ + o));
-          float4 qq = unpack4(lds_v2(sb + OFF_KQ + o + 8192));
-          float4 ww;  // the write gate w (the erase gate b in the gist.science form)
-          if (kScalarGates) {
-            ww = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (r < nvalid) {
-              float swv = __bfloat162float((kP3 ? g_b : g_w)[(size_t)(t0 + r) * H + h]);
-              if (kProlog) swv = sigmoid_f(swv);
-              ww = make_float4(swv, swv, swv, swv);
-            }
-          } else {
-            ww = unpack4(lds_v2(sb + OFF_XP + o + 8192));
-            if (kProlog) ww = make_float4(sigmoid_f(ww.x), sigmoid_f(ww.y), sigmoid_f(ww.z), sigmoid_f(ww.w));
-          }
-          if (r >= nvalid) {
-            kk = make_float4(0.f, 0.f, 0.f, 0.f);
-            qq = kk;
-            ww = kk;
-            sts_v2(sb + OFF_V + kb * 8192 + swz(r, ch16) + cofs, make_uint2(0u, 0u));
-          }
-          if (kProlog) {  // the 32 lanes of this warp hold the row's 128 channels
-            float k2 = kk.x * kk.x + kk.y * kk.y + kk.z * kk.z + kk.w * kk.w;
-            float q2 = qq.x * qq.x + qq.y * qq.y + qq.z * qq.z + qq.w * qq.w;
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) {
-              k2 += __shfl_xor_sync(0xffffffffu, k2, off);
-              q2 += __shfl_xor_sync(0xffffffffu, q2, off);
-            }
-            const float ik = rsqrtf(k2 + kNormEps), iq = rsqrtf(q2 + kNormEps);
-            kk = make_float4(kk.x * ik, kk.y * ik, kk.z * ik, kk.w * ik);
-            qq = make_float4(qq.x * iq, qq.y * iq, qq.z * iq, qq.w * iq);
-          }
-          kraw[rr] = kk;
-          const float4 e2 = e2v[rr];
-          if (kP3) {
-            sts_v2(sb + OFF_KQ + o, pack4(ww.x * kk.x * e10, ww.y * kk.y * e11, ww.z * kk.z * e12, ww.w * kk.w * e13));
-            sts_v2(sb + OFF_XP + o + 8192, pack4(kk.x * e2.x, kk.y * e2.y, kk.z * e2.z, kk.w * e2.w));
-          } else {
-            sts_v2(sb + OFF_KQ + o, pack4(kk.x * e10, kk.y * e11, kk.z * e12, kk.w * e13));
-            sts_v2(sb + OFF_XP + o + 8192, pack4(ww.x * kk.x * e2.x, ww.y * kk.y * e2.y, ww.z * kk.z * e2.z, ww.w * kk.w * e2.w));
-          }
-          sts_v2(sb + OFF_KQ + o + 8192, pack4(qq.x * e10, qq.y * e11, qq.z * e12, qq.w * e13));
-        }
-        // x_r = b.k e^{L_ref - L}: b lands last
-        if (!kScalarGates) wait_bar(bar(BAR_TMA_X), par, sAbort, p.status);
-#pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-          const int r = warp * 4 + rr;
-          const uint32_t o = (uint32_t)kb * 16384u + swz(r, ch16) + cofs;
-          float4 bb;  // the erase gate b (the value gate w in the gist.science form)
-          if (kScalarGates) {
-            bb = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (r < nvalid) {
-              float sbv = __bfloat162float((kP3 ? g_w : g_b)[(size_t)(t0 + r) * H + h]);
-              if (kProlog) sbv = sigmoid_f(sbv);
-              bb = make_float4(sbv, sbv, sbv, sbv);
-            }
-          } else {
-            bb = unpack4(lds_v2(sb + OFF_XP + o));
-            if (kProlog) bb = make_float4(sigmoid_f(bb.x), sigmoid_f(bb.y), sigmoid_f(bb.z), sigmoid_f(bb.w));
-          }
-          const float4 kk = kraw[rr], e2 = e2v[rr];
-          if (kP3) {
-            sts_v2(sb + OFF_XP + o, pack4(kk.x * e2.x, kk.y * e2.y, kk.z * e2.z, kk.w * e2.w));
-            if (r < nvalid) {  // rows past the chunk end were zeroed above
-              const uint32_t ov = sb + OFF_V + (uint32_t)kb * 8192u + swz(r, ch16) + cofs;
-              const float4 vv = unpack4(lds_v2(ov));
-              sts_v2(ov, pack4(vv.x * bb.x, vv.y * bb.y, vv.z * bb.z, vv.w * bb.w));
-            }
-          } else {
-            sts_v2(sb + OFF_XP + o, pack4(bb.x * kk.x * e2.x, bb.y * kk.y * e2.y, bb.z * kk.z * e2.z, bb.w * kk.w * e2.w));
-          }
-        }
+        ptx::umma_commit(bar(BAR_G1));
       }
-      __syncthreads();
 
       // ---- S_r^T = S^T Diag(e^{L_ref}) as the bf16 TMEM A operand (thread: dv channel `row`,
       //      dk columns [32 cg, 32 cg + 32)); the fp32 accumulator becomes the same, and the
@@ -458,6 +496,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         const float *tp = sDLb(par ^ 1u) + cg * 32;
         const float *smv = sSM + cg * 32;
         uint32_t r[32], hb[16];
+        if (ci > 0) {  // the previous chunk's increment GEMMs have landed in the state
+          wait_bar(bar(BAR_G5), par ^ 1u, sAbort, p.status);
+          ptx::tc_fence_after();
+        }
         ptx::tmem_ld32(tmS + lane_base + cg * 32, r);
         ptx::tmem_wait_ld();
 #pragma unroll
@@ -479,22 +521,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         ptx::tmem_st16(tmSR + lane_base + cg * 16, hb);
         ptx::tmem_wait_st();
       }
-      ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncthreads();
 
-      // ---- a4: G1 [A B; QX QP] = [k_r; q_r] [x_r; p_r]^T
-      if (tid == 0 && !*sAbort) {
-        ptx::tc_fence_after();
-        constexpr uint32_t id1 = ptx::idesc_bf16(128, kXP ? 64 : 128, false, false);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t ko = (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
-          ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_KQ + ko, 16, 1024),
-                         ptx::sdesc_sw128(sb + OFF_XP + ko, 16, 1024), id1, kk > 0);
-        }
-        ptx::umma_commit(bar(BAR_G1));
-      }
+
       wait_bar(bar(BAR_G1), par, sAbort, p.status);
       ptx::tc_fence_after();
 
@@ -744,6 +774,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           ptx::umma_bf16_ts(tmD1 + 64, tmRb + kk * 8, ptx::sdesc_sw128(sb + OFF_T + kk * 32, 16, 1024), idM, kk > 0);
         ptx::umma_commit(bar(BAR_GB));
       }
+      // ---- while M^T is computed: the next chunk's cumulative decay (its log_a tile landed
+      //      during the solve); then its b tile may take the log_a slot
+      if (has_next) {
+        wait_bar(bar(BAR_TMA_A), par ^ 1u, sAbort, p.status);
+        elem_cumsum(par ^ 1u, t0 + C, nvalid_next, h, L);
+        if (tid == kIssuer && !*sAbort) issue_tma_x(h, t0 + C);
+      }
       wait_bar(bar(BAR_GB), par, sAbort, p.status);
       ptx::tc_fence_after();
       {  // -M^T -> bf16 TMEM A operand
@@ -768,16 +805,22 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           ptx::umma_bf16_ts(tmO, tmMb + kk * 8, ptx::sdesc_sw128(sb + OFF_QX + kk * 32, 16, 1024), idO, 1);
+        ptx::umma_commit(bar(BAR_G4));  // O^T is complete: the epilogue need not wait for dS
         // dS^T += (-M^T) x_r: B = x_r as [tokens][dk] (MN-major, N = 128)
         constexpr uint32_t idS = ptx::idesc_bf16(128, 128, false, true);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           ptx::umma_bf16_ts(tmS, tmMb + kk * 8, ptx::sdesc_sw128(sb + OFF_XP + kk * 2048, 16384, 1024), idS, 1);
-        ptx::umma_commit(bar(BAR_G45));
+        ptx::umma_commit(bar(BAR_G5));  // the state is complete (waited for by the next S_r build)
       }
-      wait_bar(bar(BAR_G45), par, sAbort, p.status);
+      // ---- while O^T and dS are finished: the next chunk's k_r, q_r, p_r (its k, q, v tiles
+      //      landed during the solve, its w tile once dS = p_r^T V was done)
+      if (has_next) {
+        if (!kScalarGates) wait_bar(bar(BAR_TMA_W), par ^ 1u, sAbort, p.status);
+        elem_scale(t0 + C, nvalid_next, h, L, ke2);
+      }
+      wait_bar(bar(BAR_G4), par, sAbort, p.status);
       ptx::tc_fence_after();
-      if (tid == kIssuer && has_next && !*sAbort) issue_tma_x(h, t0 + C);  // x_r is dead now
 
       // ---- a8: outputs (the state was updated by the increment GEMMs)
       {
@@ -811,7 +854,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             ptx::tma_store_3d(&P.tm_o, sb + OFF_OS + (uint32_t)sbk * 8192u, sbk * kBoxC, h, t0);
           ptx::bulk_commit_group();
         }
-      } else {
+      }
+      if (nvalid < C) {
         // tail chunk: plain stores of the valid rows only
         constexpr int kRowBytes = D * (int)sizeof(Tout);
         constexpr int kU4 = kRowBytes / 16;
@@ -822,13 +866,25 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           *reinterpret_cast<uint4 *>(go + ((size_t)(t0 + i) * H + h) * kRowBytes + uu * 16) = val;
         }
       }
+      // ---- the next chunk's x_r, once dS (the last reader of this chunk's x_r) is done
+      if (has_next) {
+        wait_bar(bar(BAR_G5), par, sAbort, p.status);
+        if (!kScalarGates) wait_bar(bar(BAR_TMA_X), par ^ 1u, sAbort, p.status);
+        elem_x(t0 + C, nvalid_next, h, ke2);
+        ptx::fence_proxy_async_smem();
+      }
       ptx::tc_fence_before();
       __syncthreads();
       if (*sAbort) break;
     }
 
     // ---- a8: final state S = Diag(tau) Sacc, from S^T (thread: dv channel `row`, dk rows
-    //      [32 cg, 32 cg + 32); each store instruction of a warp writes 32 consecutive dv entries)
+    //      [32 cg, 32 cg + 32); each store instruction of a warp writes 32 consecutive dv entries).
+    //      The last chunk's increment GEMMs must have landed (also before the next unit's S0).
+    if (nchunks > 0) {
+      wait_bar(bar(BAR_G5), (it & 1u) ^ 1u, sAbort, p.status);
+      ptx::tc_fence_after();
+    }
     if (p.S_T && !*sAbort) {
       float *dst = p.S_T + ((size_t)unit * D + cg * 32) * D + row;
       const float *tp = sDLb((it & 1u) ^ 1u) + cg * 32;  // the last chunk's e^{L_C - L_ref}
