@@ -61,9 +61,9 @@ constexpr uint32_t OFF_V = 65536;      // 2 column blocks x [64 rows], 8 KB each
 constexpr uint32_t OFF_G = 81920;      // raw log_a tile
 constexpr uint32_t OFF_OS = 98304;     // o staging: 2 (bf16) or 4 (fp32) sub-blocks of [64 tokens][128 B]
 constexpr uint32_t OFF_T = 131072;     // T bf16 [64 x 64]
-constexpr uint32_t OFF_BM = 139264;    // B bf16 [64 x 64]
-constexpr uint32_t OFF_QX = 147456;    // QX bf16 [64 x 64]
-constexpr uint32_t OFF_QP = 155648;    // QP bf16 [64 x 64]
+constexpr uint32_t OFF_BM = 139264;    // B bf16 [64 x 64]; with QP right after it, the 128-row B operand [B; QP]
+constexpr uint32_t OFF_QP = 147456;    // QP bf16 [64 x 64] (QX when x_r == p_r)
+constexpr uint32_t OFF_QX = 155648;    // QX bf16 [64 x 64]
 constexpr uint32_t OFF_AF = 163840;    // fp32 A [64 x 68] (masks -> solve)
 constexpr uint32_t OFF_TF = 181248;    // fp32 T [64 x 68] (solve)
 constexpr uint32_t OFF_XS = 198656;    // fp32 solve scratch, <= 4 KB
@@ -73,14 +73,14 @@ constexpr uint32_t MISC_DL = 512;      // float[128]  e^{L_C - L_ref} of the chu
 constexpr uint32_t MISC_SM = 1024;     // float[128]  e^{L_ref}
 constexpr uint32_t MISC_PART = 1536;   // float[16][128] 4-row sums of log_a, then exclusive prefixes
 constexpr uint32_t MISC_REF = 9728;    // float[128]  L_ref
-constexpr uint32_t MISC_BAR = 10240;   // 10 mbarriers
+constexpr uint32_t MISC_BAR = 10240;   // 9 mbarriers
 constexpr uint32_t MISC_TMEM = 10320;
 constexpr uint32_t MISC_ABORT = 10324;
 constexpr uint32_t MISC_UNIT = 10328;
 constexpr uint32_t MISC_BYTES = 10336;
 constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES + 1024;  // + base alignment slack
 // mbarrier slots
-enum { BAR_TMA_A = 0, BAR_TMA_W, BAR_TMA_X, BAR_G1, BAR_E1, BAR_E2, BAR_GA, BAR_GB, BAR_G4, BAR_G5, kNumBars };
+enum { BAR_TMA_A = 0, BAR_TMA_W, BAR_TMA_X, BAR_G1, BAR_E1, BAR_GA, BAR_GB, BAR_G4, BAR_G5, kNumBars };
 static_assert(MISC_BAR + 8 * kNumBars <= MISC_TMEM, "mbarriers overlap the TMEM address slot");
 
 struct TcParams {
@@ -227,9 +227,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   // The state is held transposed, S^T (lane = d_v channel, column = d_k channel), so that
   // S_r^T, R^T and -M^T -- the A operands of every state-side GEMM -- are read by the tensor
   // core straight from TMEM as bf16 (two channels per column) and never visit shared memory.
-  const uint32_t tmD1 = tmem;        // G1 result; then R^T (cols 0-63) and M^T (cols 64-127), fp32
+  const uint32_t tmD1 = tmem;        // G1 result; then [R^T | O^T] (cols 0-63 | 64-127), fp32
   const uint32_t tmS = tmem + 128;   // S^T fp32 (128 cols)
-  const uint32_t tmO = tmem + 256;   // O^T fp32 (64 cols)
+  const uint32_t tmO = tmem + 64;    // O^T fp32 (64 cols), beside R^T: both come from one N = 128 product
+  const uint32_t tmM = tmem + 256;   // M^T fp32 (64 cols)
   const uint32_t tmSR = tmem + 320;  // S_r^T bf16 A operand (64 cols)
   const uint32_t tmRb = tmem + 384;  // R^T bf16 A operand (32 cols)
   const uint32_t tmMb = tmem + 416;  // -M^T bf16 A operand (32 cols)
@@ -560,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           const int i = row - 64;
 #pragma unroll
           for (int j = 0; j < 32; ++j) f[j] = (jb + j <= i) ? __uint_as_float(r[j]) : 0.f;
-          const uint32_t dst = cg < 2 ? OFF_QX : OFF_QP;
+          const uint32_t dst = (cg < 2 && !kXP) ? OFF_QX : OFF_QP;  // with x_r == p_r, QX = QP: one slot
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8)
             sts_v4(sb + dst + swz(i, (uint32_t)((cg & 1) * 4 + q8)), pack8(f + 8 * q8, 1.f));
@@ -571,11 +572,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       __syncthreads();
 
       // ---- a6 (T-independent MMAs, issued by warp 15 while warps 0-14 solve; one issuing thread
-      //      keeps them in order, and the issue stalls of a full MMA queue delay nobody):
-      //        dS = p_r^T V,  O^T = S_r^T q_r^T                                   (commit E1)
-      //        R^T = V^T B^T + S_r^T k_r^T  (D1 cols 0-63), the right-hand side of M = T R:
-      //          M = (I + A)^-1 (B V + Ytilde S) with Ytilde S = k_r S_r          (commit GA)
-      //        O^T += V^T QP^T                                                     (commit E2)
+      //      keeps them in order, and the issue stalls of the MMA queue delay nobody):
+      //        dS = p_r^T V                                                        (commit E1)
+      //        [R^T | O^T] = V^T [B; QP]^T + S_r^T [k_r; q_r]^T, one N = 128 product each:
+      //          R = B V + k_r S_r is the right-hand side of M = T R,
+      //          M = (I + A)^-1 (B V + Ytilde S) with Ytilde S = k_r S_r;
+      //          O^T = S_r^T q_r^T + V^T QP^T before the erase term                (commit GA)
       if (warp == kIssueWarp) {
         if (lane == 0 && !*sAbort) {
           ptx::tc_fence_after();
@@ -585,34 +587,24 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           for (int kk = 0; kk < 4; ++kk)
             ptx::umma_bf16(tmS, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
                            ptx::sdesc_sw128(sb + OFF_XP + 8192 + kk * 2048, 16384, 1024), idS, 1);
-          constexpr uint32_t idT = ptx::idesc_bf16(128, 64, false, false);  // A from TMEM
-          constexpr uint32_t idO = ptx::idesc_bf16(128, 64, true, false);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            ptx::umma_bf16_ts(tmO, tmSR + kk * 8,
-                              ptx::sdesc_sw128(sb + OFF_KQ + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32, 16, 1024), idT,
-                              kk > 0);
           ptx::umma_commit(bar(BAR_E1));
+          constexpr uint32_t idV = ptx::idesc_bf16(128, 128, true, false);   // A = V^T (MN-major)
+          constexpr uint32_t idT = ptx::idesc_bf16(128, 128, false, false);  // A from TMEM
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
-                           ptx::sdesc_sw128(sb + OFF_BM + kk * 32, 16, 1024), idO, kk > 0);
+                           ptx::sdesc_sw128(sb + OFF_BM + kk * 32, 16, 1024), idV, kk > 0);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             ptx::umma_bf16_ts(tmD1, tmSR + kk * 8,
                               ptx::sdesc_sw128(sb + OFF_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), idT, 1);
           ptx::umma_commit(bar(BAR_GA));
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            ptx::umma_bf16(tmO, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
-                           ptx::sdesc_sw128(sb + (kXP ? OFF_QX : OFF_QP) + kk * 32, 16, 1024), idO, 1);
-          ptx::umma_commit(bar(BAR_E2));
           if (has_next) {  // p_r is dead once dS = p_r^T V is done: the next chunk's w can land
             wait_bar(bar(BAR_E1), par, sAbort, p.status);
             if (!*sAbort) issue_tma_w(h, t0 + C);
-            // k_r, q_r and V are dead once E2 (after GA) is done: the next chunk's k, q, v,
-            // log_a tiles can land (the solve runs meanwhile, so this wait delays nobody)
-            wait_bar(bar(BAR_E2), par, sAbort, p.status);
+            // k_r, q_r and V are dead once GA is done: the next chunk's k, q, v, log_a tiles
+            // can land (the solve runs meanwhile, so this wait delays nobody)
+            wait_bar(bar(BAR_GA), par, sAbort, p.status);
             if (!*sAbort) issue_tma_a(h, t0 + C);
           }
         }
@@ -765,13 +757,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       ptx::tc_fence_before();
       __syncthreads();
 
-      // ---- a7 (erase reads): M^T = R^T T^T (D1 cols 64-127); row i of M is r_i = Sbar_i^T k_i
+      // ---- a7 (erase reads): M^T = R^T T^T (own 64 columns); row i of M is r_i = Sbar_i^T k_i
       if (tid == 0 && !*sAbort) {
         ptx::tc_fence_after();
         constexpr uint32_t idM = ptx::idesc_bf16(128, 64, false, false);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16_ts(tmD1 + 64, tmRb + kk * 8, ptx::sdesc_sw128(sb + OFF_T + kk * 32, 16, 1024), idM, kk > 0);
+          ptx::umma_bf16_ts(tmM, tmRb + kk * 8, ptx::sdesc_sw128(sb + OFF_T + kk * 32, 16, 1024), idM, kk > 0);
         ptx::umma_commit(bar(BAR_GB));
       }
       // ---- while M^T is computed: the next chunk's cumulative decay (its log_a tile landed
@@ -785,7 +777,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       ptx::tc_fence_after();
       {  // -M^T -> bf16 TMEM A operand
         uint32_t r[16], hb[8];
-        ptx::tmem_ld16(tmD1 + 64 + lane_base + cg * 16, r);
+        ptx::tmem_ld16(tmM + lane_base + cg * 16, r);
         ptx::tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 8; ++j) hb[j] = pack_bf16x2(-__uint_as_float(r[2 * j]), -__uint_as_float(r[2 * j + 1]));
@@ -798,13 +790,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
 
       // ---- a7: the state-dependent remainder of O^T and dS
       if (tid == 0 && !*sAbort) {
-        // O^T was last accumulated by the other issuing thread: keep the accumulation order fixed
-        wait_bar(bar(BAR_E2), par, sAbort, p.status);
         ptx::tc_fence_after();
         constexpr uint32_t idO = ptx::idesc_bf16(128, 64, false, false);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16_ts(tmO, tmMb + kk * 8, ptx::sdesc_sw128(sb + OFF_QX + kk * 32, 16, 1024), idO, 1);
+          ptx::umma_bf16_ts(tmO, tmMb + kk * 8, ptx::sdesc_sw128(sb + (kXP ? OFF_QP : OFF_QX) + kk * 32, 16, 1024), idO, 1);
         ptx::umma_commit(bar(BAR_G4));  // O^T is complete: the epilogue need not wait for dS
         // dS^T += (-M^T) x_r: B = x_r as [tokens][dk] (MN-major, N = 128)
         constexpr uint32_t idS = ptx::idesc_bf16(128, 128, false, true);
