@@ -567,7 +567,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             sts_v4(sb + dst + swz(i, (uint32_t)((cg & 1) * 4 + q8)), pack8(f + 8 * q8, 1.f));
         }
       }
-      ptx::fence_proxy_async_smem();
+      // a proxy fence costs each thread that runs it far more than a barrier: only the warps
+      // whose stores an MMA reads (B, QX, QP) run it; the fp32 A is read by the solve's threads
+      if (kXP ? (cg < 2) : !(qd < 2 && cg < 2)) ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncthreads();
 
@@ -738,7 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         }
         }  // solve scope
       }  // warps 0-14
-      ptx::fence_proxy_async_smem();
+      if (warp < 8) ptx::fence_proxy_async_smem();  // warps 0-7 wrote the bf16 T tile
       ptx::tc_fence_before();
       __syncthreads();
 
@@ -832,7 +834,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           }
         }
       }
-      ptx::fence_proxy_async_smem();  // staging is read by the TMA store below
+      // ---- the next chunk's x_r, once dS (the last reader of this chunk's x_r) is done
+      if (has_next) {
+        wait_bar(bar(BAR_G5), par, sAbort, p.status);
+        if (!kScalarGates) wait_bar(bar(BAR_TMA_X), par ^ 1u, sAbort, p.status);
+        elem_x(t0 + C, nvalid_next, h, ke2);
+      }
+      // one proxy fence per thread covers the o staging (read by the TMA store below) and the
+      // next chunk's operands (read by its G1)
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
       __syncthreads();
       if (nvalid == C) {
         // full chunk: asynchronous TMA store; the next chunk's epilogue rewrites the staging
@@ -844,8 +855,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             ptx::tma_store_3d(&P.tm_o, sb + OFF_OS + (uint32_t)sbk * 8192u, sbk * kBoxC, h, t0);
           ptx::bulk_commit_group();
         }
-      }
-      if (nvalid < C) {
+      } else {
         // tail chunk: plain stores of the valid rows only
         constexpr int kRowBytes = D * (int)sizeof(Tout);
         constexpr int kU4 = kRowBytes / 16;
@@ -856,15 +866,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           *reinterpret_cast<uint4 *>(go + ((size_t)(t0 + i) * H + h) * kRowBytes + uu * 16) = val;
         }
       }
-      // ---- the next chunk's x_r, once dS (the last reader of this chunk's x_r) is done
-      if (has_next) {
-        wait_bar(bar(BAR_G5), par, sAbort, p.status);
-        if (!kScalarGates) wait_bar(bar(BAR_TMA_X), par ^ 1u, sAbort, p.status);
-        elem_x(t0 + C, nvalid_next, h, ke2);
-        ptx::fence_proxy_async_smem();
-      }
-      ptx::tc_fence_before();
-      __syncthreads();
       if (*sAbort) break;
     }
 
