@@ -73,14 +73,14 @@ constexpr uint32_t MISC_DL = 512;      // float[128]  e^{L_C - L_ref} of the chu
 constexpr uint32_t MISC_SM = 1024;     // float[128]  e^{L_ref}
 constexpr uint32_t MISC_PART = 1536;   // float[16][128] 4-row sums of log_a, then exclusive prefixes
 constexpr uint32_t MISC_REF = 9728;    // float[128]  L_ref
-constexpr uint32_t MISC_BAR = 10240;   // 9 mbarriers
+constexpr uint32_t MISC_BAR = 10240;   // 10 mbarriers
 constexpr uint32_t MISC_TMEM = 10320;
 constexpr uint32_t MISC_ABORT = 10324;
 constexpr uint32_t MISC_UNIT = 10328;
 constexpr uint32_t MISC_BYTES = 10336;
 constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES + 1024;  // + base alignment slack
 // mbarrier slots
-enum { BAR_TMA_A = 0, BAR_TMA_W, BAR_TMA_X, BAR_G1, BAR_E1, BAR_GA, BAR_GB, BAR_G4, BAR_G5, kNumBars };
+enum { BAR_TMA_A = 0, BAR_TMA_L, BAR_TMA_W, BAR_TMA_X, BAR_G1, BAR_E1, BAR_GA, BAR_GB, BAR_G4, BAR_G5, kNumBars };
 static_assert(MISC_BAR + 8 * kNumBars <= MISC_TMEM, "mbarriers overlap the TMEM address slot");
 
 struct TcParams {
@@ -242,16 +242,22 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   const __nv_bfloat16 *g_w = static_cast<const __nv_bfloat16 *>(tied ? p.b : p.w);
 
   // TMA issue (thread 0): group A = k, q, v (+ log_a), group B = b, w.
+  // TMA issue: group A = k, q, v; group L = log_a (into the log_a slot, free from the start of
+  // the previous chunk, so it is requested a whole chunk ahead); group W = w; group X = b.
   auto issue_tma_a = [&](int h, int t0) {
-    uint32_t bytes = 3u * 2u * 8192u + (kScalarDecay ? 0u : 2u * 8192u);
-    ptx::mbar_arrive_expect_tx(bar(BAR_TMA_A), bytes);
+    ptx::mbar_arrive_expect_tx(bar(BAR_TMA_A), 3u * 2u * 8192u);
 #pragma unroll
     for (int kb = 0; kb < 2; ++kb) {
       ptx::tma_load_3d(sb + OFF_KQ + kb * 16384, &P.tm_k, kb * 64, h, t0, bar(BAR_TMA_A));
       ptx::tma_load_3d(sb + OFF_KQ + kb * 16384 + 8192, &P.tm_q, kb * 64, h, t0, bar(BAR_TMA_A));
       ptx::tma_load_3d(sb + OFF_V + kb * 8192, &P.tm_v, kb * 64, h, t0, bar(BAR_TMA_A));
-      if (!kScalarDecay) ptx::tma_load_3d(sb + OFF_G + kb * 8192, &P.tm_g, kb * 64, h, t0, bar(BAR_TMA_A));
     }
+  };
+  auto issue_tma_l = [&](int h, int t0) {
+    if (kScalarDecay) return;
+    ptx::mbar_arrive_expect_tx(bar(BAR_TMA_L), 2u * 8192u);
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) ptx::tma_load_3d(sb + OFF_G + kb * 8192, &P.tm_g, kb * 64, h, t0, bar(BAR_TMA_L));
   };
   // w lands in the p_r halves of XP (free once dS = p_r^T V is done), b in the log_a slot
   // (free once the cumulative decay of its chunk is done)
@@ -425,6 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     }
     const int nchunks = (int)((len + C - 1) / C);
     if (tid == kIssuer && nchunks > 0 && !*sAbort) {
+      issue_tma_l(h, (int)bos);
       issue_tma_a(h, (int)bos);
       issue_tma_w(h, (int)bos);
     }
@@ -455,9 +462,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     if (nchunks > 0) {
       const int nv0 = (int)(len < C ? len : C);
       const uint32_t par0 = it & 1u;
-      wait_bar(bar(BAR_TMA_A), par0, sAbort, p.status);
+      if (!kScalarDecay) wait_bar(bar(BAR_TMA_L), par0, sAbort, p.status);
       elem_cumsum(par0, (int)bos, nv0, h, L);
       if (tid == kIssuer && !*sAbort) issue_tma_x(h, (int)bos);
+      wait_bar(bar(BAR_TMA_A), par0, sAbort, p.status);
       if (!kScalarGates) wait_bar(bar(BAR_TMA_W), par0, sAbort, p.status);
       elem_scale((int)bos, nv0, h, L, ke2);
       if (!kScalarGates) wait_bar(bar(BAR_TMA_X), par0, sAbort, p.status);
@@ -473,6 +481,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       const int t0 = (int)(bos + c0);
       const bool has_next = ci + 1 < nchunks;
       const int nvalid_next = has_next ? (int)((len - c0 - C) < C ? (len - c0 - C) : C) : 0;
+
+      // the log_a slot is free (the b tile it last held was consumed by this chunk's x_r):
+      // the next chunk's log_a can land
+      if (tid == kIssuer && has_next && !*sAbort) issue_tma_l(h, t0 + C);
 
       // ---- a4: G1 [A B; QX QP] = [k_r; q_r] [x_r; p_r]^T, issued first: it needs only this
       //      chunk's operands (built during the previous chunk) and runs under the S_r build
@@ -604,8 +616,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           if (has_next) {  // p_r is dead once dS = p_r^T V is done: the next chunk's w can land
             wait_bar(bar(BAR_E1), par, sAbort, p.status);
             if (!*sAbort) issue_tma_w(h, t0 + C);
-            // k_r, q_r and V are dead once GA is done: the next chunk's k, q, v, log_a tiles
-            // can land (the solve runs meanwhile, so this wait delays nobody)
+            // k_r, q_r and V are dead once GA is done: the next chunk's k, q, v tiles can land
+            // (the solve runs meanwhile, so this wait delays nobody)
             wait_bar(bar(BAR_GA), par, sAbort, p.status);
             if (!*sAbort) issue_tma_a(h, t0 + C);
           }
@@ -771,7 +783,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       // ---- while M^T is computed: the next chunk's cumulative decay (its log_a tile landed
       //      during the solve); then its b tile may take the log_a slot
       if (has_next) {
-        wait_bar(bar(BAR_TMA_A), par ^ 1u, sAbort, p.status);
+        if (!kScalarDecay) wait_bar(bar(BAR_TMA_L), par ^ 1u, sAbort, p.status);
         elem_cumsum(par ^ 1u, t0 + C, nvalid_next, h, L);
         if (tid == kIssuer && !*sAbort) issue_tma_x(h, t0 + C);
       }
@@ -808,6 +820,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       // ---- while O^T and dS are finished: the next chunk's k_r, q_r, p_r (its k, q, v tiles
       //      landed during the solve, its w tile once dS = p_r^T V was done)
       if (has_next) {
+        wait_bar(bar(BAR_TMA_A), par ^ 1u, sAbort, p.status);
         if (!kScalarGates) wait_bar(bar(BAR_TMA_W), par ^ 1u, sAbort, p.status);
         elem_scale(t0 + C, nvalid_next, h, L, ke2);
       }
