@@ -237,7 +237,9 @@ def main():
     ap.add_argument("--bwd-steps", type=int, default=3)
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-long", action="store_true")
-    ap.add_argument("--split", type=int, default=8, help="segments per sequence of the long-context split forward")
+    ap.add_argument("--split", type=int, default=0,
+                    help="segments per sequence of the long-context split forward (0: as many as keep "
+                         "the 16 heads' segments within the SM count)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     args = ap.parse_args()
@@ -500,6 +502,8 @@ def main():
         li = inputs.make_inputs(wl, dev, seed=500 + rank)
         largs = [li[n].view(1, 65536, *li[n].shape[1:]) for n in names]
         ldims = gdn2.make_dims(1, 65536, 16, 128, 128, 64, gdn2.BF16, gdn2.BF16, 0)
+        if args.split <= 0:  # one segment unit per SM at most: 148 SMs / 16 heads -> 9 segments
+            args.split = max(1, torch.cuda.get_device_properties(dev).multi_processor_count // 16)
         lws = torch.empty(gdn2.split_workspace_size(ldims, args.split), dtype=torch.uint8, device=dev)
         pws = torch.empty(gdn2.workspace_size(ldims), dtype=torch.uint8, device=dev)
 
