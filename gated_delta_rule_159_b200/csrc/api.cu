@@ -331,6 +331,123 @@ int gdn2_chunk_fwd_split(const void *q, const void *k, const void *v, const void
   return GDN2_OK;
 }
 
+// ---------------------------------------------------------------- one segment per rank
+// Workspace of gdn2_segment_maps / gdn2_segment_correct: the inner forward's workspace, a zero
+// v, scratch outputs and (maps only) the identity start states.
+struct SegLayout {
+  size_t off_zero_v, off_o2, off_ident, total;
+};
+static size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+static SegLayout seg_layout(const gdn2_dims *d, bool maps) {
+  SegLayout L;
+  const size_t tok = (size_t)d->n_seqs * (size_t)d->seq_len * (size_t)d->n_heads;
+  const size_t in_e = d->dtype_in == GDN2_BF16 ? 2 : 4, out_e = d->dtype_out == GDN2_BF16 ? 2 : 4;
+  L.off_zero_v = up256(gdn2_chunk_fwd_workspace_size(d));
+  L.off_o2 = L.off_zero_v + up256(tok * (size_t)d->d_v * in_e);
+  L.off_ident = L.off_o2 + up256(tok * (size_t)d->d_v * out_e);
+  L.total = L.off_ident + (maps ? up256((size_t)d->n_seqs * d->n_heads * d->d_k * d->d_v * sizeof(float)) : 0);
+  return L;
+}
+
+static int check_segment_call(const gdn2_dims *dims, const void *workspace, size_t workspace_bytes, size_t need) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->d_k != 128 || dims->d_v != 128 || dims->chunk != 64 || dims->dtype_in != GDN2_BF16)
+    return fail(GDN2_ERR_UNSUPPORTED, "the segment calls need d_k = d_v = 128, chunk 64 and bf16 inputs");
+  if ((int64_t)dims->n_seqs * dims->seq_len >= ((int64_t)1 << 31))
+    return fail(GDN2_ERR_UNSUPPORTED, "the segment calls need fewer than 2^31 tokens");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(GDN2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  if (workspace_bytes < need) return fail(GDN2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+  return GDN2_OK;
+}
+
+size_t gdn2_segment_maps_workspace_size(const gdn2_dims *dims) {
+  if (!dims || dims->n_seqs < 1 || dims->n_heads < 1 || dims->seq_len < 0) return 0;
+  return seg_layout(dims, true).total;
+}
+
+size_t gdn2_segment_correct_workspace_size(const gdn2_dims *dims) {
+  if (!dims || dims->n_seqs < 1 || dims->n_heads < 1 || dims->seq_len < 0) return 0;
+  return seg_layout(dims, false).total;
+}
+
+int gdn2_segment_maps(const void *q, const void *k, const void *v, const void *log_a, const void *b, const void *w,
+                      const float *S0, void *o, float *F, float *G, const gdn2_dims *dims, void *workspace,
+                      size_t workspace_bytes, gdn2_stream_t stream) {
+  g_err[0] = '\0';
+  int rc = check_segment_call(dims, workspace, workspace_bytes, gdn2_segment_maps_workspace_size(dims));
+  if (rc) return rc;
+  if (dims->seq_len > 0) {  // every check before the first launch (an empty segment reads no input)
+    rc = check_inputs(q, k, v, log_a, b, w, dims->flags, dims->dtype_in);
+    if (rc) return rc;
+    if (!o || !aligned16(o)) return fail(GDN2_ERR_INVALID_ARG, "o must be non-NULL and 16-byte aligned");
+  }
+  if (S0 && !aligned16(S0)) return fail(GDN2_ERR_INVALID_ARG, "S0 must be 16-byte aligned");
+  if (!F || !G || !aligned16(F) || !aligned16(G)) return fail(GDN2_ERR_INVALID_ARG, "F and G must be non-NULL and 16-byte aligned");
+  const SegLayout L = seg_layout(dims, true);
+  char *ws = static_cast<char *>(workspace);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int units = dims->n_seqs * dims->n_heads;
+  const size_t state_bytes = (size_t)units * 128 * 128 * sizeof(float);
+  float *ident = reinterpret_cast<float *>(ws + L.off_ident);
+  cudaError_t e = gdn2::launch_identities(ident, units, s);
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "identity states: %s", cudaGetErrorString(e));
+  if (dims->seq_len == 0) {  // an empty segment maps S to S: F = I, G = S0 (or 0)
+    e = cudaMemcpyAsync(F, ident, state_bytes, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess)
+      e = S0 ? cudaMemcpyAsync(G, S0, state_bytes, cudaMemcpyDeviceToDevice, s) : cudaMemsetAsync(G, 0, state_bytes, s);
+    return e == cudaSuccess ? GDN2_OK : fail(GDN2_ERR_CUDA, "empty segment: %s", cudaGetErrorString(e));
+  }
+  const size_t inner_bytes = L.off_zero_v;
+  // o and G: the segment from its given start (S0, or 0)
+  rc = chunk_fwd_impl(q, k, v, log_a, b, w, S0, nullptr, nullptr, o, G, dims, ws, inner_bytes, stream, true);
+  if (rc) return rc;
+  // F: the segment from the identity with v = 0
+  const size_t vbytes = (size_t)dims->n_seqs * dims->seq_len * dims->n_heads * 128 * 2;
+  e = cudaMemsetAsync(ws + L.off_zero_v, 0, vbytes, s);
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "zero v: %s", cudaGetErrorString(e));
+  return chunk_fwd_impl(q, k, ws + L.off_zero_v, log_a, b, w, ident, nullptr, nullptr, ws + L.off_o2, F, dims, ws,
+                        inner_bytes, stream, false);
+}
+
+int gdn2_affine_prefix(const float *F_all, const float *G_all, float *start, float *S_T, int32_t n_seqs,
+                       int32_t n_heads, int32_t n_segs, int32_t seg, gdn2_stream_t stream) {
+  g_err[0] = '\0';
+  if (!F_all || !G_all) return fail(GDN2_ERR_INVALID_ARG, "F_all and G_all must be non-NULL");
+  if (n_seqs < 1 || n_heads < 1 || n_segs < 1 || seg < 0 || seg >= n_segs)
+    return fail(GDN2_ERR_INVALID_ARG, "bad sizes (n_seqs=%d n_heads=%d n_segs=%d seg=%d)", n_seqs, n_heads, n_segs, seg);
+  if (!start && !S_T) return GDN2_OK;
+  const size_t per_seg = (size_t)n_seqs * n_heads;
+  const cudaError_t e = gdn2::launch_prefix(F_all, G_all, per_seg, (size_t)n_heads, start, S_T, seg, n_segs, n_seqs,
+                                            n_heads, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GDN2_OK : fail(GDN2_ERR_CUDA, "affine prefix: %s", cudaGetErrorString(e));
+}
+
+int gdn2_segment_correct(const void *q, const void *k, const void *log_a, const void *b, const void *w,
+                         const float *start, void *o, const gdn2_dims *dims, void *workspace, size_t workspace_bytes,
+                         gdn2_stream_t stream) {
+  g_err[0] = '\0';
+  int rc = check_segment_call(dims, workspace, workspace_bytes, gdn2_segment_correct_workspace_size(dims));
+  if (rc) return rc;
+  if (dims->seq_len == 0) return GDN2_OK;  // nothing to correct
+  rc = check_inputs(q, k, q, log_a, b, w, dims->flags, dims->dtype_in);  // (v is not read: q stands in)
+  if (rc) return rc;
+  if (!start || !aligned16(start)) return fail(GDN2_ERR_INVALID_ARG, "start must be non-NULL and 16-byte aligned");
+  if (!o || !aligned16(o)) return fail(GDN2_ERR_INVALID_ARG, "o must be non-NULL and 16-byte aligned");
+  const SegLayout L = seg_layout(dims, false);
+  char *ws = static_cast<char *>(workspace);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t n_out = (size_t)dims->n_seqs * dims->seq_len * dims->n_heads * 128;
+  cudaError_t e = cudaMemsetAsync(ws + L.off_zero_v, 0, n_out * 2, s);
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "zero v: %s", cudaGetErrorString(e));
+  rc = chunk_fwd_impl(q, k, ws + L.off_zero_v, log_a, b, w, start, nullptr, nullptr, ws + L.off_o2, nullptr, dims, ws,
+                      L.off_zero_v, stream, true);
+  if (rc) return rc;
+  e = gdn2::launch_add(o, ws + L.off_o2, n_out, dims->dtype_out, s);
+  return e == cudaSuccess ? GDN2_OK : fail(GDN2_ERR_CUDA, "o += correction: %s", cudaGetErrorString(e));
+}
+
 int gdn2_check_status(const void *workspace, gdn2_stream_t stream) {
   g_err[0] = '\0';
   if (!workspace) return fail(GDN2_ERR_INVALID_ARG, "workspace is NULL");

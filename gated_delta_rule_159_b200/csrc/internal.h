@@ -84,6 +84,12 @@ struct SplitArgs {
 SplitPlan split_plan(int N, int T, int H, int n_split, int dtype_in, int dtype_out, size_t inner_bytes);
 // what: 0 segment bounds, 1 pass-1 starts, 2 identity starts, 3 combine, 4 o += o2
 cudaError_t launch_split_helpers(int what, const SplitArgs &a, cudaStream_t stream);
+// Helpers of the per-rank segment calls: `units` 128 x 128 identities; o += o2 (n elements);
+// the start state of segment `upto` and the end state after n_segs segments (see prefix_kernel).
+cudaError_t launch_identities(float *dst, int units, cudaStream_t stream);
+cudaError_t launch_add(void *o, const void *o2, size_t n, int dtype_out, cudaStream_t stream);
+cudaError_t launch_prefix(const float *F, const float *G, size_t seg_stride, size_t seq_stride, float *start,
+                          float *S_T, int upto, int n_segs, int N, int H, cudaStream_t stream);
 
 // Record `message` as this thread's gdn2_last_error() text and return `code`.
 int set_last_error(int code, const char *message);

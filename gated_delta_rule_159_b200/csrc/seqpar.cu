@@ -87,6 +87,48 @@ __global__ void __launch_bounds__(kComb) combine_kernel(const float *F, const fl
   }
 }
 
+// Start state of segment `upto` and, when S_T is given, the end state after all n_segs
+// segments, for one (sequence, head) per CTA, from per-segment maps laid out with element
+// strides (in 128 x 128 matrices) seg_stride between segments and seq_stride between
+// sequences: S <- F_j S + G_j from S = 0 (segment 0's map already carries the true S0).
+__global__ void __launch_bounds__(kComb) prefix_kernel(const float *F, const float *G, size_t seg_stride,
+                                                       size_t seq_stride, float *start, float *S_T, int upto,
+                                                       int n_segs, int H) {
+  extern __shared__ float Ss[];  // [128][128] current state
+  const int unit = blockIdx.x, n = unit / H, h = unit % H;
+  const int t = threadIdx.x, r = t >> 2, c0 = (t & 3) * 32;
+  auto at = [&](const float *base, int j) { return base + ((size_t)j * seg_stride + (size_t)n * seq_stride + h) * 128 * 128; };
+  for (int e = t; e < 128 * 128; e += kComb) Ss[e] = 0.f;
+  __syncthreads();
+  const int last = S_T ? n_segs : upto;
+  for (int j = 0; j <= last; ++j) {
+    if (j == upto && start) {
+      float *d = start + (size_t)unit * 128 * 128;
+      for (int e = t; e < 128 * 128; e += kComb) d[e] = Ss[e];
+    }
+    if (j == last) break;
+    const float *Fr = at(F, j) + (size_t)r * 128;
+    float acc[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) acc[c] = at(G, j)[(size_t)r * 128 + c0 + c];
+    if (j > 0) {  // S = 0 before segment 0
+      for (int kk = 0; kk < 128; ++kk) {
+        const float f = Fr[kk];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) acc[c] += f * Ss[kk * 128 + c0 + c];
+      }
+    }
+    __syncthreads();  // everyone has read the old state
+#pragma unroll
+    for (int c = 0; c < 32; ++c) Ss[r * 128 + c0 + c] = acc[c];
+    __syncthreads();
+  }
+  if (S_T) {
+    float *d = S_T + (size_t)unit * 128 * 128;
+    for (int e = t; e < 128 * 128; e += kComb) d[e] = Ss[e];
+  }
+}
+
 template <typename T>
 __global__ void add_kernel(T *o, const T *d, size_t n) {
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
@@ -118,6 +160,29 @@ SplitPlan split_plan(int N, int T, int H, int n_split, int dtype_in, int dtype_o
   s.off_o2 = s.off_zero_v + up256(tok * in_e);
   s.total = s.off_o2 + up256(tok * out_e);
   return s;
+}
+
+cudaError_t launch_identities(float *dst, int units, cudaStream_t stream) {
+  seg_states_kernel<<<units, 256, 0, stream>>>(dst, nullptr, 1, 1, true);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_add(void *o, const void *o2, size_t n, int dtype_out, cudaStream_t stream) {
+  if (dtype_out == GDN2_BF16)
+    add_kernel<__nv_bfloat16><<<592, 256, 0, stream>>>(static_cast<__nv_bfloat16 *>(o),
+                                                       static_cast<const __nv_bfloat16 *>(o2), n);
+  else
+    add_kernel<float><<<592, 256, 0, stream>>>(static_cast<float *>(o), static_cast<const float *>(o2), n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefix(const float *F, const float *G, size_t seg_stride, size_t seq_stride, float *start,
+                          float *S_T, int upto, int n_segs, int N, int H, cudaStream_t stream) {
+  const int smem = 128 * 128 * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  prefix_kernel<<<N * H, kComb, smem, stream>>>(F, G, seg_stride, seq_stride, start, S_T, upto, n_segs, H);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_split_helpers(int what, const SplitArgs &a, cudaStream_t stream) {

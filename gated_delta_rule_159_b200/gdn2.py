@@ -34,6 +34,8 @@ FUSED_PROLOGUE = 16
 EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_workspace_size", "gdn2_check_status",
             "gdn2_decode_step", "gdn2_decode_step_indexed", "gdn2_decode_status", "gdn2_bwd",
             "gdn2_bwd_workspace_size", "gdn2_chunk_fwd_split", "gdn2_chunk_fwd_split_workspace_size",
+            "gdn2_segment_maps", "gdn2_segment_maps_workspace_size", "gdn2_affine_prefix",
+            "gdn2_segment_correct", "gdn2_segment_correct_workspace_size",
             "gdn2_last_error", "gdn2_version")
 
 
@@ -70,6 +72,16 @@ def _load():
     lib.gdn2_chunk_fwd_split.argtypes = [vp] * 9 + [ctypes.POINTER(Dims), ctypes.c_int32, vp, sz, vp]
     lib.gdn2_chunk_fwd_split_workspace_size.restype = sz
     lib.gdn2_chunk_fwd_split_workspace_size.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32]
+    lib.gdn2_segment_maps.restype = ctypes.c_int
+    lib.gdn2_segment_maps.argtypes = [vp] * 10 + [ctypes.POINTER(Dims), vp, sz, vp]
+    lib.gdn2_segment_maps_workspace_size.restype = sz
+    lib.gdn2_segment_maps_workspace_size.argtypes = [ctypes.POINTER(Dims)]
+    lib.gdn2_affine_prefix.restype = ctypes.c_int
+    lib.gdn2_affine_prefix.argtypes = [vp, vp, vp, vp] + [ctypes.c_int32] * 4 + [vp]
+    lib.gdn2_segment_correct.restype = ctypes.c_int
+    lib.gdn2_segment_correct.argtypes = [vp] * 7 + [ctypes.POINTER(Dims), vp, sz, vp]
+    lib.gdn2_segment_correct_workspace_size.restype = sz
+    lib.gdn2_segment_correct_workspace_size.argtypes = [ctypes.POINTER(Dims)]
     lib.gdn2_decode_status.restype = ctypes.c_int
     lib.gdn2_decode_status.argtypes = [vp]
     lib.gdn2_bwd.restype = ctypes.c_int
@@ -225,6 +237,95 @@ def chunk_fwd_split(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: to
                                   _ptr(S_T), ctypes.byref(dims), int(n_split), _ptr(workspace), workspace.numel(),
                                   _stream(dev))
     _check(rc)
+    return o, S_T
+
+
+def _segment_dims(q, v, flags, out_dtype):
+    N, L, H, dk = q.shape
+    return make_dims(N, L, H, dk, v.shape[-1], 64, _dtype_code(q.dtype), _dtype_code(out_dtype), flags)
+
+
+def segment_maps(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, b: torch.Tensor,
+                 w: Optional[torch.Tensor] = None, S0: Optional[torch.Tensor] = None, *,
+                 scalar_decay: bool = False, scalar_gates: bool = False, tied_gates: bool = False,
+                 gate_form_p3: bool = False, fused_prologue: bool = False,
+                 out_dtype: Optional[torch.dtype] = None, workspace: Optional[torch.Tensor] = None):
+    """One rank's segment [N, L, H, d] of N sequences through ``gdn2_segment_maps``.
+    Returns (o from the start S0 or 0, F, G): the segment maps a start state S to F S + G
+    (F, G fp32 [N, H, d_k, d_v])."""
+    N, L, H, dk = q.shape
+    dv = v.shape[-1]
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    dims = _segment_dims(q, v, flags_of(scalar_decay, scalar_gates, tied_gates, gate_form_p3, fused_prologue),
+                         out_dtype)
+    dev = q.device
+    o = torch.empty(N, L, H, dv, dtype=out_dtype, device=dev)
+    F = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    G = torch.empty_like(F)
+    if workspace is None:
+        workspace = torch.empty(max(int(lib.gdn2_segment_maps_workspace_size(ctypes.byref(dims))), 256),
+                                dtype=torch.uint8, device=dev)
+    _check(lib.gdn2_segment_maps(_ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(b), _ptr(w), _ptr(S0), _ptr(o), _ptr(F),
+                                 _ptr(G), ctypes.byref(dims), _ptr(workspace), workspace.numel(), _stream(dev)))
+    return o, F, G
+
+
+def affine_prefix(F_all: torch.Tensor, G_all: torch.Tensor, seg: int, *, want_S_T: bool = True):
+    """``gdn2_affine_prefix``: F_all, G_all [R, N, H, d_k, d_v] (segment r = rank r).
+    Returns (the start state of segment ``seg`` [N, H, d_k, d_v], the end state after all R
+    segments or None)."""
+    R, N, H, dk, dv = F_all.shape
+    start = torch.empty(N, H, dk, dv, dtype=torch.float32, device=F_all.device)
+    S_T = torch.empty_like(start) if want_S_T else None
+    _check(lib.gdn2_affine_prefix(_ptr(F_all), _ptr(G_all), _ptr(start), _ptr(S_T), N, H, R, int(seg),
+                                  _stream(F_all.device)))
+    return start, S_T
+
+
+def segment_correct(q: torch.Tensor, k: torch.Tensor, log_a: torch.Tensor, b: torch.Tensor,
+                    w: Optional[torch.Tensor], start: torch.Tensor, o: torch.Tensor, *,
+                    scalar_decay: bool = False, scalar_gates: bool = False, tied_gates: bool = False,
+                    gate_form_p3: bool = False, fused_prologue: bool = False,
+                    workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """``gdn2_segment_correct``: o += the segment's outputs from ``start`` with v = 0 (in place)."""
+    dims = _segment_dims(q, o, flags_of(scalar_decay, scalar_gates, tied_gates, gate_form_p3, fused_prologue),
+                         o.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(int(lib.gdn2_segment_correct_workspace_size(ctypes.byref(dims))), 256),
+                                dtype=torch.uint8, device=q.device)
+    _check(lib.gdn2_segment_correct(_ptr(q), _ptr(k), _ptr(log_a), _ptr(b), _ptr(w), _ptr(start), _ptr(o),
+                                    ctypes.byref(dims), _ptr(workspace), workspace.numel(), _stream(q.device)))
+    return o
+
+
+class SegmentOps:
+    """The three per-rank calls of the sequence-parallel forward (the library's kernels)."""
+    segment_maps = staticmethod(segment_maps)
+    affine_prefix = staticmethod(affine_prefix)
+    segment_correct = staticmethod(segment_correct)
+
+
+def chunk_fwd_seq_ranks(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, b: torch.Tensor,
+                        w: Optional[torch.Tensor] = None, S0: Optional[torch.Tensor] = None, *, group=None,
+                        ops=SegmentOps, **flags):
+    """Sequence-parallel chunked forward across the ranks of ``group`` (one process per
+    GPU): rank r holds tokens [r L, (r + 1) L) of each of the N sequences as [N, L, H, d]
+    tensors (S0 is read on rank 0 only).  Each rank computes its segment's outputs and
+    affine map (F, G), the maps are all-gathered (the one collective: 2 x 64 KiB per
+    (sequence, head) per rank), each rank folds the maps of the ranks before it into its
+    true start state and adds that start state's contribution to its outputs.
+    Returns (o [N, L, H, d_v] of this rank's tokens, S_T [N, H, d_k, d_v] of the whole
+    sequences, on every rank)."""
+    import torch.distributed as dist
+    rank, world = dist.get_rank(group), dist.get_world_size(group)
+    o, F, G = ops.segment_maps(q, k, v, log_a, b, w, S0 if rank == 0 else None, **flags)
+    F_all = torch.empty((world,) + tuple(F.shape), dtype=F.dtype, device=F.device)
+    G_all = torch.empty_like(F_all)
+    dist.all_gather(list(F_all.unbind(0)), F.contiguous(), group=group)
+    dist.all_gather(list(G_all.unbind(0)), G.contiguous(), group=group)
+    start, S_T = ops.affine_prefix(F_all, G_all, rank)
+    if rank > 0:
+        ops.segment_correct(q, k, log_a, b, w, start, o, **flags)
     return o, S_T
 
 

@@ -204,6 +204,58 @@ int gdn2_chunk_fwd_split(const void *q, const void *k, const void *v,
 size_t gdn2_chunk_fwd_split_workspace_size(const gdn2_dims *dims, int32_t n_split);
 
 /*
+ * Sequence parallelism across ranks (one process per GPU): rank r of R holds tokens
+ * [r L, (r + 1) L) of each of N equal sequences (all heads) and runs, on its own GPU,
+ *
+ *   1. gdn2_segment_maps: its outputs o from the start state 0 (rank 0: the true S0),
+ *      and its segment's affine map S_end = F S_start + G (the same affine view as
+ *      gdn2_chunk_fwd_split: F is the end state from S_start = I with v = 0, G the end
+ *      state from the start above);
+ *   2. an all-gather of every rank's F and G (the caller's collective, e.g. NCCL), laid
+ *      out [R][N][H][128][128] fp32;
+ *   3. gdn2_affine_prefix: its true start state S_s(r) = F_{r-1} S_s(r-1) + G_{r-1},
+ *      S_s(0) = 0 (rank 0's outputs and G already include S0), and, when S_T is given,
+ *      the end state of the whole sequences;
+ *   4. gdn2_segment_correct (ranks r > 0): o += the outputs of its segment from S_s(r)
+ *      with v = 0.
+ * Together they give gdn2_chunk_fwd's o (each rank its tokens) and S_T up to rounding.
+ * dims describe the rank's local segment: N = dims.n_seqs sequences of dims.seq_len
+ * tokens, no cu_seqlens.  Supported: d_k = d_v = 128, chunk 64, bf16 inputs.  All
+ * pointers are device pointers owned by the caller; workspaces are 256-byte aligned
+ * and at least the size the matching *_workspace_size call returns.
+ * Errors: GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_WORKSPACE, GDN2_ERR_CUDA.
+ *
+ * gdn2_segment_maps: q, k, v, log_a, b, w, S0 (may be NULL), o as gdn2_chunk_fwd with
+ * 4-D-equivalent layout [N * L, H, d]; F, G: [N][H][128][128] fp32 outputs.  An empty
+ * segment (dims.seq_len = 0) reads no input: F = I, G = S0 (or 0).
+ */
+int gdn2_segment_maps(const void *q, const void *k, const void *v,
+                      const void *log_a, const void *b, const void *w,
+                      const float *S0, void *o, float *F, float *G, const gdn2_dims *dims,
+                      void *workspace, size_t workspace_bytes, gdn2_stream_t stream);
+size_t gdn2_segment_maps_workspace_size(const gdn2_dims *dims);
+
+/*
+ * gdn2_affine_prefix: F_all, G_all [n_segs][n_seqs][n_heads][128][128] fp32 (segment
+ * `seg` = rank `seg`); start (may be NULL): [n_seqs][n_heads][128][128] fp32, receives
+ * S_s(seg) (zeros for seg 0); S_T (may be NULL): receives the state after all n_segs
+ * segments.  One CTA per (sequence, head), serial over the segments.
+ */
+int gdn2_affine_prefix(const float *F_all, const float *G_all, float *start, float *S_T,
+                       int32_t n_seqs, int32_t n_heads, int32_t n_segs, int32_t seg,
+                       gdn2_stream_t stream);
+
+/*
+ * gdn2_segment_correct: o (dims.dtype_out, [N * L, H, 128]) += the outputs of the
+ * segment run from `start` ([N][H][128][128] fp32) with v = 0; q, k, log_a, b, w as
+ * gdn2_chunk_fwd (v is not needed).
+ */
+int gdn2_segment_correct(const void *q, const void *k, const void *log_a, const void *b, const void *w,
+                         const float *start, void *o, const gdn2_dims *dims,
+                         void *workspace, size_t workspace_bytes, gdn2_stream_t stream);
+size_t gdn2_segment_correct_workspace_size(const gdn2_dims *dims);
+
+/*
  * gdn2_decode_status -- synchronise `stream`, then report whether any decode
  * step since the last call gave up a bounded device-side wait (the d_k = d_v =
  * 128 decode streams each state through shared memory with bulk copies and

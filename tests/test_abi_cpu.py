@@ -186,3 +186,38 @@ def test_split_forward_rejects_bad_arguments(g):
     assert call(d, q=None) == g.ERR_INVALID_ARG
     assert call(d, ws=None) == g.ERR_WORKSPACE
     assert call(d, ws_bytes=4096) == g.ERR_WORKSPACE
+
+
+def test_segment_calls_reject_bad_arguments(g):
+    """The per-rank sequence-parallel calls validate everything before their first launch."""
+    lib = g.lib
+    d = _dims(g, n_seqs=2, seq_len=256, n_heads=2)
+    need = lib.gdn2_segment_maps_workspace_size(ctypes.byref(d))
+    assert need > lib.gdn2_segment_correct_workspace_size(ctypes.byref(d)) > 0
+    assert lib.gdn2_segment_maps_workspace_size(None) == 0
+
+    def maps(dims, ws_bytes=None, **kw):
+        a = dict(q=P, k=P, v=P, log_a=P, b=P, w=P, S0=None, o=P, F=P, G=P, ws=WS)
+        a.update(kw)
+        return lib.gdn2_segment_maps(a["q"], a["k"], a["v"], a["log_a"], a["b"], a["w"], a["S0"], a["o"], a["F"],
+                                     a["G"], ctypes.byref(dims), a["ws"], need if ws_bytes is None else ws_bytes, None)
+    assert maps(d, q=None) == g.ERR_INVALID_ARG
+    assert maps(d, F=None) == g.ERR_INVALID_ARG
+    assert maps(d, o=ctypes.c_void_p((1 << 20) + 4)) == g.ERR_INVALID_ARG
+    assert maps(d, ws=None) == g.ERR_WORKSPACE
+    assert maps(d, ws_bytes=need - 1) == g.ERR_WORKSPACE
+    assert maps(_dims(g, n_seqs=2, seq_len=256, d_k=64, d_v=64)) == g.ERR_UNSUPPORTED
+
+    def correct(dims, **kw):
+        a = dict(q=P, k=P, log_a=P, b=P, w=P, start=P, o=P, ws=WS)
+        a.update(kw)
+        return lib.gdn2_segment_correct(a["q"], a["k"], a["log_a"], a["b"], a["w"], a["start"], a["o"],
+                                        ctypes.byref(dims), a["ws"], 1 << 30, None)
+    assert correct(d, start=None) == g.ERR_INVALID_ARG
+    assert correct(d, k=None) == g.ERR_INVALID_ARG
+    assert correct(d, o=None) == g.ERR_INVALID_ARG
+    # affine prefix: the segment index must name one of the n_segs segments
+    assert lib.gdn2_affine_prefix(P, P, P, None, 2, 2, 3, 3, None) == g.ERR_INVALID_ARG
+    assert lib.gdn2_affine_prefix(P, P, P, None, 2, 2, 3, -1, None) == g.ERR_INVALID_ARG
+    assert lib.gdn2_affine_prefix(None, P, P, None, 2, 2, 3, 0, None) == g.ERR_INVALID_ARG
+    assert lib.gdn2_affine_prefix(P, P, None, None, 2, 2, 3, 0, None) == g.OK  # nothing requested: no launch

@@ -209,6 +209,44 @@ def test_tc_split_forward(dev, n_split, seq_len, variant):
     assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (eo, es)
 
 
+# sequence parallelism across ranks: the per-rank calls, with the ranks emulated in one process
+# (the all-gather of the maps becomes a stack); bounds need not fall on chunk boundaries
+@pytest.mark.parametrize("bounds,variant", [((0, 200, 400), "channel"), ((0, 64, 317, 580, 704), "channel"),
+                                            ((0, 333, 333, 700), "channel"), ((0, 256, 640), "scalar"),
+                                            ((0, 150, 512), "p3")])
+def test_segment_calls_emulated_ranks(dev, bounds, variant):
+    from gated_delta_rule_159_b200 import gdn2
+    T = bounds[-1]
+    inp = _small(dev, n_seqs=2, seq_len=T, n_heads=2, scalar=(variant == "scalar"), gate_form_p3=(variant == "p3"))
+    N = inp["n_seqs"]
+    names = ("q", "k", "v", "log_a", "b", "w")
+    v4 = lambda t: None if t is None else t.view(N, T, *t.shape[1:])  # noqa: E731
+    flags = dict(scalar_decay=inp["scalar_decay"], scalar_gates=inp["scalar_gates"], tied_gates=inp["tied_gates"],
+                 gate_form_p3=(variant == "p3"))
+    full = {n: v4(inp[n]) for n in names}
+    R = len(bounds) - 1
+    pieces = []
+    for r in range(R):  # step 1 on every rank
+        lo, hi = bounds[r], bounds[r + 1]
+        loc = {n: None if full[n] is None else full[n][:, lo:hi].contiguous() for n in names}
+        o, F, G = gdn2.segment_maps(*(loc[n] for n in names), inp["S0"] if r == 0 else None, out_dtype=torch.float32,
+                                    **flags)
+        pieces.append((loc, o, F, G))
+    F_all = torch.stack([pc[2] for pc in pieces])  # step 2: the all-gather
+    G_all = torch.stack([pc[3] for pc in pieces])
+    outs, S_T = [], None
+    for r in range(R):  # steps 3 and 4
+        loc, o, _, _ = pieces[r]
+        start, S_T = gdn2.affine_prefix(F_all, G_all, r)
+        if r > 0:
+            gdn2.segment_correct(*(loc[n] for n in ("q", "k", "log_a", "b", "w")), start, o, **flags)
+        outs.append(o)
+    torch.cuda.synchronize()
+    o = torch.cat(outs, dim=1)
+    eo, es = compare_units(inp, o.reshape(inp["T_tot"], 2, 128), S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (eo, es)
+
+
 @pytest.mark.parametrize("case", ["deltanet", "pure_decay", "zero_key", "strong_decay", "no_decay_no_gates"])
 def test_tc_degenerate_cases(dev, case):
     inp = _small(dev, n_seqs=1, seq_len=192, n_heads=2)

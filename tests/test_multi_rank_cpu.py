@@ -11,6 +11,7 @@ import socket
 
 import numpy as np
 import pytest
+import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
@@ -103,3 +104,97 @@ def test_sequence_ranges_balance_tokens():
     assert r[0][0] == 0 and r[-1][1] == 5 and r[0][1] == r[1][0]
     assert shard.sequence_ranges([0, 5], 3) == [(0, 0), (0, 1), (1, 1)]
     assert [shard.head_range(16, r, 3) for r in range(3)] == [(0, 6), (6, 11), (11, 16)]
+
+
+# ----------------------------------------------------------------- sequence parallelism across ranks
+class _OracleSegmentOps:
+    """The three per-rank calls of gdn2.chunk_fwd_seq_ranks computed by the float64 oracle
+    (these tests run without a GPU; the library's own calls are checked on the GPU)."""
+
+    @staticmethod
+    def _run(q, k, v, log_a, b, w, S0):
+        import oracle
+        N, L, H, d = q.shape
+        flat = lambda t: None if t is None else t.reshape((N * L,) + tuple(t.shape[2:])).double().numpy()  # noqa: E731
+        cu = np.arange(N + 1, dtype=np.int64) * L
+        o, S = oracle.gdn2_fwd(flat(q), flat(k), flat(v), flat(log_a), flat(b), flat(w),
+                               S0=None if S0 is None else S0.double().numpy(), cu_seqlens=cu)
+        return torch.from_numpy(o.reshape(N, L, H, -1)), torch.from_numpy(S)
+
+    @staticmethod
+    def segment_maps(q, k, v, log_a, b, w, S0, **flags):
+        N, L, H, d = q.shape
+        o, G = _OracleSegmentOps._run(q, k, v, log_a, b, w, S0)
+        ident = torch.eye(d, dtype=torch.float64).expand(N, H, d, d).contiguous()
+        _, F = _OracleSegmentOps._run(q, k, torch.zeros_like(v), log_a, b, w, ident)
+        return o, F, G
+
+    @staticmethod
+    def affine_prefix(F_all, G_all, seg):
+        S, start = torch.zeros_like(F_all[0]), None
+        for j in range(F_all.shape[0]):
+            if j == seg:
+                start = S.clone()
+            S = F_all[j] @ S + G_all[j]
+        return start, S
+
+    @staticmethod
+    def segment_correct(q, k, log_a, b, w, start, o, **flags):
+        N, L, H, _ = q.shape
+        dv = o.shape[-1]
+        o2, _ = _OracleSegmentOps._run(q, k, torch.zeros(N, L, H, dv, dtype=q.dtype), log_a, b, w, start)
+        o += o2
+        return o
+
+
+def _seq_problem(N=2, T=48, H=2, d=4, seed=3):
+    g = torch.Generator().manual_seed(seed)
+    f = lambda *s: torch.randn(*s, generator=g, dtype=torch.float64)  # noqa: E731
+    q, k, v = f(N, T, H, d), f(N, T, H, d), f(N, T, H, d)
+    log_a = -0.3 * torch.rand(N, T, H, d, generator=g, dtype=torch.float64)
+    b, w = torch.rand(N, T, H, d, generator=g, dtype=torch.float64), torch.rand(N, T, H, d, generator=g,
+                                                                                 dtype=torch.float64)
+    S0 = 0.1 * f(N, H, d, d)
+    return (q, k, v, log_a, b, w), S0
+
+
+def _seq_worker(rank, world, port, out_q):
+    from gated_delta_rule_159_b200 import gdn2
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        xs, S0 = _seq_problem()
+        T = xs[0].shape[1]
+        lo, hi = rank * T // world, (rank + 1) * T // world
+        local = [x[:, lo:hi].contiguous() for x in xs]
+        o, S_T = gdn2.chunk_fwd_seq_ranks(*local, S0, ops=_OracleSegmentOps)
+        gathered = [None] * world
+        dist.all_gather_object(gathered, (lo, hi, o, S_T))
+        if rank == 0:
+            out_q.put(gathered)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sequence_ranks_equal_unsplit(world):
+    """Each rank holds a slice of every sequence; the gathered outputs and every rank's S_T
+    equal the unsplit recurrence (only the (F, G) maps cross ranks)."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_seq_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    gathered = q.get(timeout=180)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    xs, S0 = _seq_problem()
+    o_ref, S_ref = _OracleSegmentOps._run(*xs, S0)
+    o = torch.zeros_like(o_ref)
+    for lo, hi, o_r, S_r in gathered:
+        o[:, lo:hi] = o_r
+        assert torch.allclose(S_r, S_ref, rtol=1e-10, atol=1e-12)
+    assert torch.allclose(o, o_ref, rtol=1e-10, atol=1e-12)
