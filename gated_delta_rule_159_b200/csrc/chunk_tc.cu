@@ -27,7 +27,12 @@
 // TMEM as bf16 and read from there by the tensor core; the B operands and V^T come
 // from shared memory, where the tiles arrive by TMA (128-byte swizzle) and transposed
 // operands use MN-major descriptors, so no tile is ever transposed in memory.  The
-// T-independent GEMMs run on the tensor core while warps 0-14 solve for T.
+// T-independent GEMMs run on the tensor core while warps 0-14 solve for T, and the next
+// chunk's operands (cumulative decay, k_r, q_r, p_r, x_r) are built while this chunk's
+// remaining GEMMs (M = T R, the last terms of O and of the state) run; a chunk's G1 is
+// issued before its S_r build.  A tcgen05.mma holds its issuing thread for roughly
+// its execution time, so products are merged into as few N = 128 instructions as the
+// operand layouts allow.
 //
 // One CTA (512 threads) per SM, persistent over (sequence, head) units taken
 // longest-first from an atomic counter in the caller's workspace.  Every
@@ -58,7 +63,7 @@ constexpr float kLog2eF = 1.4426950408889634f;
 constexpr uint32_t OFF_KQ = 0;         // 2 K-blocks x [k_r rows 0-63 | q_r rows 0-63], 16 KB each
 constexpr uint32_t OFF_XP = 32768;     // 2 K-blocks x [x_r rows | p_r rows]
 constexpr uint32_t OFF_V = 65536;      // 2 column blocks x [64 rows], 8 KB each
-constexpr uint32_t OFF_G = 81920;      // raw log_a tile
+constexpr uint32_t OFF_G = 81920;      // raw log_a tile; after the cumulative decay, the raw b tile
 constexpr uint32_t OFF_OS = 98304;     // o staging: 2 (bf16) or 4 (fp32) sub-blocks of [64 tokens][128 B]
 constexpr uint32_t OFF_T = 131072;     // T bf16 [64 x 64]
 constexpr uint32_t OFF_BM = 139264;    // B bf16 [64 x 64]; with QP right after it, the 128-row B operand [B; QP]
@@ -197,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   float *sSM = reinterpret_cast<float *>(gb + OFF_MISC + MISC_SM);
   float *part = reinterpret_cast<float *>(gb + OFF_MISC + MISC_PART);
   float *sRef = reinterpret_cast<float *>(gb + OFF_MISC + MISC_REF);
-  constexpr int kIssuer = 32;      // issues the first TMA loads of a unit, the b loads and the o stores
+  constexpr int kIssuer = 32;      // issues a unit's first TMA loads, the log_a and b loads and the o stores
   constexpr int kIssueWarp = 15;   // issues the T-independent MMAs during the solve
   constexpr int kSolveThreads = 480;  // warps 0-14
   enum { NB_SOLVE = 1 };
