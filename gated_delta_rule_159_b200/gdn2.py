@@ -307,7 +307,7 @@ class SegmentOps:
 
 def chunk_fwd_seq_ranks(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, b: torch.Tensor,
                         w: Optional[torch.Tensor] = None, S0: Optional[torch.Tensor] = None, *, group=None,
-                        ops=SegmentOps, **flags):
+                        ops=SegmentOps, out_dtype: Optional[torch.dtype] = None, **flags):
     """Sequence-parallel chunked forward across the ranks of ``group`` (one process per
     GPU): rank r holds tokens [r L, (r + 1) L) of each of the N sequences as [N, L, H, d]
     tensors (S0 is read on rank 0 only).  Each rank computes its segment's outputs and
@@ -318,7 +318,8 @@ def chunk_fwd_seq_ranks(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a
     sequences, on every rank)."""
     import torch.distributed as dist
     rank, world = dist.get_rank(group), dist.get_world_size(group)
-    o, F, G = ops.segment_maps(q, k, v, log_a, b, w, S0 if rank == 0 else None, **flags)
+    maps_kw = dict(flags) if out_dtype is None else dict(flags, out_dtype=out_dtype)
+    o, F, G = ops.segment_maps(q, k, v, log_a, b, w, S0 if rank == 0 else None, **maps_kw)
     F_all = torch.empty((world,) + tuple(F.shape), dtype=F.dtype, device=F.device)
     G_all = torch.empty_like(F_all)
     dist.all_gather(list(F_all.unbind(0)), F.contiguous(), group=group)

@@ -247,6 +247,32 @@ def test_segment_calls_emulated_ranks(dev, bounds, variant):
     assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (eo, es)
 
 
+def test_seq_ranks_one_rank_nccl(dev):
+    """gdn2.chunk_fwd_seq_ranks over a one-rank NCCL group: the collective path of the
+    sequence-parallel forward on one GPU (the all-gather has one participant)."""
+    import datetime
+    import socket
+    import torch.distributed as dist
+    from gated_delta_rule_159_b200 import gdn2
+    inp = _small(dev, n_seqs=2, seq_len=300, n_heads=2)
+    N, T = inp["n_seqs"], inp["T_tot"] // inp["n_seqs"]
+    names = ("q", "k", "v", "log_a", "b", "w")
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        o, S_T = gdn2.chunk_fwd_seq_ranks(*(inp[n].view(N, T, *inp[n].shape[1:]) for n in names), inp["S0"],
+                                          out_dtype=torch.float32)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    eo, es = compare_units(inp, o.reshape(inp["T_tot"], 2, 128), S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (eo, es)
+
+
 @pytest.mark.parametrize("case", ["deltanet", "pure_decay", "zero_key", "strong_decay", "no_decay_no_gates"])
 def test_tc_degenerate_cases(dev, case):
     inp = _small(dev, n_seqs=1, seq_len=192, n_heads=2)
