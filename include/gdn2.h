@@ -62,7 +62,7 @@ typedef struct CUstream_st *gdn2_stream_t;
 enum gdn2_status {
   GDN2_OK = 0,
   GDN2_ERR_INVALID_ARG = -1,  /* null/misaligned pointer, bad dims, bad cu_seqlens_host */
-  GDN2_ERR_UNSUPPORTED = -2,  /* valid request this build has no kernel for */
+  GDN2_ERR_UNSUPPORTED = -2,  /* valid request the library has no kernel for */
   GDN2_ERR_CUDA = -3,         /* a CUDA runtime call or kernel launch failed */
   GDN2_ERR_TIMEOUT = -4,      /* a bounded device-side wait gave up (reported by gdn2_check_status) */
   GDN2_ERR_WORKSPACE = -5     /* workspace pointer NULL or smaller than the queried size */

@@ -182,7 +182,7 @@ def test_hold_when_alpha1_beta0():
 # --------------------------------------------------------------------------
 
 def test_erase_gate_placement_closed_form():
-    """k = (e1 + e2)/sqrt2, b = (1, 0), w = 0, no decay.  The benchmark spec form
+    """k = (e1 + e2)/sqrt2, b = (1, 0), w = 0, no decay.  The default gate placement
     erases with the OUTER factor b.k = (1/sqrt2, 0) and reads with k:
         row1 -= (row1 + row2)/2,  row2 unchanged.
     Swapping the sides (read with b.k, erase along k) would instead give
