@@ -461,6 +461,7 @@ __global__ void __launch_bounds__(kThreads) finish_kernel(BwdProblem p) {
 
   float vdq = 0.f, vdp = 0.f, vdx = 0.f, vdy = 0.f, vdg = 0.f;
   if (i < dk) {
+#pragma unroll 4
     for (int s = 0; s < NS; ++s) {
       const float *pr = p.part + ((size_t)s * p.t_total * p.n_heads + th) * kRows * dk + i;
       vdq += pr[0 * dk];
@@ -502,8 +503,10 @@ __global__ void __launch_bounds__(kThreads) finish_kernel(BwdProblem p) {
   // per-channel gate gradient of b (tied gates add the w gradient; P3 tied needs d_k == d_v)
   const float gbt = gb + (tied ? (p3 ? gwv : gw) : 0.f);
   // block sums: channel sums for the scalar flags, q.dq and k.dk for the L2-norm gradient
+  // (the block-wide flag test keeps the barrier inside uniform; without those flags nothing
+  // reads the sums)
   float sums[5] = {vdg, gb, p3 ? gwv : gw, qq * vdq, kk * gdk};
-  block_sums<5>(sums, red);
+  if (sd || sg || prolog) block_sums<5>(sums, red);
 
   // sigmoid' = s (1 - s) from the activated value s; d/dx log sigmoid(x) = 1 - a
   auto dsig = [&](float s) { return prolog ? s * (1.f - s) : 1.f; };
