@@ -527,6 +527,16 @@ def main():
                     "plain_ms": t_plain, "split_ms": t_split, "n_split": args.split,
                     "plain_tokens_per_s": 65536 * world / (t_plain / 1e3),
                     "split_tokens_per_s": 65536 * world / (t_split / 1e3)}
+        if world > 1 and 65536 % world == 0:
+            # one 65,536-token sequence spread over the ranks: rank r holds tokens
+            # [r L, (r + 1) L), L = 65536 / N; each rank's segment maps are all-gathered
+            Lr = 65536 // world
+            rargs = [a[:, rank * Lr:(rank + 1) * Lr].contiguous() for a in largs]
+            t_ranks = timed(lambda: gdn2.chunk_fwd_seq_ranks(*rargs, li["S0"]))
+            long_ctx.update({"ranks_ms": t_ranks, "ranks": world,
+                             "ranks_tokens_per_s": 65536 / (t_ranks / 1e3),
+                             "ranks_path": "gdn2_segment_maps, all-gather of (F, G) over NCCL, "
+                                           "gdn2_affine_prefix, gdn2_segment_correct"})
         del li, largs, lws, pws
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
