@@ -216,14 +216,18 @@ def decode_status(device=None) -> int:
 
 
 def chunk_fwd_split(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, b: torch.Tensor,
-                    w: Optional[torch.Tensor] = None, S0: Optional[torch.Tensor] = None, *, n_split: int = 8,
+                    w: Optional[torch.Tensor] = None, S0: Optional[torch.Tensor] = None, *,
+                    n_split: Optional[int] = None,
                     scalar_decay: bool = False, scalar_gates: bool = False, tied_gates: bool = False,
                     gate_form_p3: bool = False, fused_prologue: bool = False,
                     out_dtype: Optional[torch.dtype] = None, workspace: Optional[torch.Tensor] = None):
     """Sequence-parallel chunked forward through ``gdn2_chunk_fwd_split``: inputs
-    [B, T, H, d] (equal lengths), every sequence cut into up to ``n_split`` segments.
+    [B, T, H, d] (equal lengths), every sequence cut into up to ``n_split`` segments
+    (default: as many as keep the B x H x n_split segment units within the SM count).
     Returns (o [B, T, H, d_v], S_T fp32 [B, H, d_k, d_v])."""
     N, T, H, dk = q.shape
+    if n_split is None:
+        n_split = max(1, torch.cuda.get_device_properties(q.device).multi_processor_count // (N * H))
     dv = v.shape[-1]
     out_dtype = q.dtype if out_dtype is None else out_dtype
     flags = flags_of(scalar_decay, scalar_gates, tied_gates, gate_form_p3, fused_prologue)

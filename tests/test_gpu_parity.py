@@ -209,6 +209,18 @@ def test_tc_split_forward(dev, n_split, seq_len, variant):
     assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (eo, es)
 
 
+def test_tc_split_forward_default_split(dev):
+    """chunk_fwd_split with its default segment count (from the SM count) equals the oracle."""
+    from gated_delta_rule_159_b200 import gdn2
+    inp = _small(dev, n_seqs=1, seq_len=1500, n_heads=2)
+    N, T = inp["n_seqs"], inp["T_tot"] // inp["n_seqs"]
+    names = ("q", "k", "v", "log_a", "b", "w")
+    o, S_T = gdn2.chunk_fwd_split(*(inp[n].view(N, T, *inp[n].shape[1:]) for n in names), inp["S0"],
+                                  out_dtype=torch.float32)
+    eo, es = compare_units(inp, o.view(inp["T_tot"], 2, 128), S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (eo, es)
+
+
 # sequence parallelism across ranks: the per-rank calls, with the ranks emulated in one process
 # (the all-gather of the maps becomes a stack); bounds need not fall on chunk boundaries
 @pytest.mark.parametrize("bounds,variant", [((0, 200, 400), "channel"), ((0, 64, 317, 580, 704), "channel"),
