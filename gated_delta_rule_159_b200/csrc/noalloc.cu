@@ -24,8 +24,12 @@
 
 namespace {
 
-// 256-byte header (status word, unit counter) + one int32 per (sequence, head) unit.
-constexpr size_t kNoAllocScratchBytes = 256 + 4 * (size_t)GDN2_NOALLOC_MAX_UNITS;
+// 256-byte header (status word, unit counter) + one int32 per (sequence, head) unit, the
+// schedule part rounded up to 256 bytes exactly as gdn2_chunk_fwd_workspace_size rounds it,
+// so that a request at the limit always fits.
+constexpr size_t kNoAllocScheduleBytes = ((4 * (size_t)GDN2_NOALLOC_MAX_UNITS + 255) / 256) * 256;
+constexpr size_t kNoAllocScratchBytes = 256 + kNoAllocScheduleBytes;
+static_assert(kNoAllocScratchBytes >= 256 + 4 * (size_t)GDN2_NOALLOC_MAX_UNITS, "scratch too small");
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -34,7 +38,8 @@ std::mutex g_setup_mutex;
 void *g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_noalloc_scratch on the current device (looked up once per device).
-int scratch_for_current_device(void **out) {
+// With lookup == false a device that has never run the entry point reports NULL.
+int scratch_for_current_device(void **out, bool lookup = true) {
   char msg[256];
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -48,7 +53,7 @@ int scratch_for_current_device(void **out) {
     return gdn2::set_last_error(GDN2_ERR_UNSUPPORTED, msg);
   }
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch_ptr[dev] && lookup) {
     void *ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
     if (e != cudaSuccess || ptr == nullptr) {
@@ -82,4 +87,14 @@ extern "C" int gdn2_chunk_fwd_noalloc(const void *q, const void *k, const void *
   if (rc != GDN2_OK) return rc;
   return gdn2_chunk_fwd(q, k, v, log_a, b, w, S0, cu_seqlens, cu_seqlens_host, o, S_T, dims, scratch,
                         kNoAllocScratchBytes, stream);
+}
+
+// Status of the last gdn2_chunk_fwd_noalloc on the current device: its bounded device waits
+// record a timeout in word 0 of the fixed array, which the caller has no pointer to.
+extern "C" int gdn2_chunk_fwd_noalloc_status(gdn2_stream_t stream) {
+  void *scratch = nullptr;
+  int rc = scratch_for_current_device(&scratch, false);
+  if (rc != GDN2_OK) return rc;
+  if (!scratch) return GDN2_OK;  // no call has run on this device
+  return gdn2_check_status(scratch, stream);
 }

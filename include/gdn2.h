@@ -351,6 +351,16 @@ int gdn2_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
                            const float *S0, const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
                            void *o, float *S_T, const gdn2_dims *dims, gdn2_stream_t stream);
 
+/*
+ * gdn2_chunk_fwd_noalloc_status -- gdn2_check_status for gdn2_chunk_fwd_noalloc:
+ * synchronises `stream`, then reads the status word that the last
+ * gdn2_chunk_fwd_noalloc on the current device left in the fixed array (the
+ * caller holds no pointer to it).  Returns GDN2_OK (also when no such call has
+ * run on this device), GDN2_ERR_TIMEOUT or GDN2_ERR_CUDA.  The next
+ * gdn2_chunk_fwd_noalloc clears the word, so read it before that call.
+ */
+int gdn2_chunk_fwd_noalloc_status(gdn2_stream_t stream);
+
 /* Thread-local description of the last non-zero status on this thread ("" if none). */
 const char *gdn2_last_error(void);
 

@@ -41,6 +41,20 @@ FWD = [
     # gist.science form: erase read with k instead of b.k
     ("for (int64_t j = 0; j < dv; ++j) r[j] += S[i * dv + j] * x[i];",
      "for (int64_t j = 0; j < dv; ++j) r[j] += S[i * dv + j] * kt[i];"),
+    # gist.science form: erase sides swapped (read with k, erase along b.k)
+    ("                for (int64_t j = 0; j < dv; ++j) r[j] += S[i * dv + j] * x[i];\n"
+     "            for (int64_t i = 0; i < dk; ++i)\n"
+     "                for (int64_t j = 0; j < dv; ++j) S[i * dv + j] -= kt[i] * r[j];",
+     "                for (int64_t j = 0; j < dv; ++j) r[j] += S[i * dv + j] * kt[i];\n"
+     "            for (int64_t i = 0; i < dk; ++i)\n"
+     "                for (int64_t j = 0; j < dv; ++j) S[i * dv + j] -= x[i] * r[j];"),
+    # gist.science form: write gate on the key axis, (w.k) v^T instead of k (w.v)^T
+    ("            for (int64_t j = 0; j < dv; ++j) p[j] = (scalar_gates ? wt[0] : wt[j]) * vt[j];\n"
+     "            for (int64_t i = 0; i < dk; ++i)\n"
+     "                for (int64_t j = 0; j < dv; ++j) S[i * dv + j] += kt[i] * p[j];",
+     "            for (int64_t i = 0; i < dk; ++i)\n"
+     "                for (int64_t j = 0; j < dv; ++j)\n"
+     "                    S[i * dv + j] += (scalar_gates ? wt[0] : wt[i]) * kt[i] * vt[j];"),
 ]
 BWD = [
     ("const double gb = G[i * dv + j] + y[i] * dr[j];", "const double gb = G[i * dv + j];"),

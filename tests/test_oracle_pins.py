@@ -307,6 +307,119 @@ def test_reduces_to_kda_and_p3_agrees_when_tied():
         np.testing.assert_allclose(S[0, 0], want_S, rtol=1e-11, atol=1e-12)
 
 
+# --------------------------------------------------------------------------
+# The gist.science gate placement (Methodologie 1, the printed update
+# S_t = (I - k_t (b_t . k_t)^T) D_t S_{t-1} + k_t (w_t . v_t)^T) with
+# channel-wise b != w: hand-derived closed forms in which the erase read side,
+# the erase outer side and the write axis each change the answer.
+# --------------------------------------------------------------------------
+
+def _p3_run(S0, log_a, k, v, b, w, q=None):
+    """Tokens through the oracle in the gist.science form: k, log_a, b [T, d_k];
+    v, w [T, d_v]; S0 [d_k, d_v]."""
+    k = np.atleast_2d(np.asarray(k, float))
+    T, dk = k.shape
+    v = np.atleast_2d(np.asarray(v, float))
+    dv = v.shape[1]
+    q = k if q is None else np.atleast_2d(np.asarray(q, float))
+    return oracle.gdn2_fwd(q.reshape(T, 1, dk), k.reshape(T, 1, dk), v.reshape(T, 1, dv),
+                           np.broadcast_to(np.asarray(log_a, float), (T, dk)).reshape(T, 1, dk),
+                           np.atleast_2d(np.asarray(b, float)).reshape(T, 1, dk),
+                           np.atleast_2d(np.asarray(w, float)).reshape(T, 1, dv),
+                           S0=np.asarray(S0, float).reshape(1, 1, dk, dv), flags=oracle.GATE_FORM_P3)
+
+
+def test_p3_erase_side_closed_form():
+    """No decay, w = 0, k = (e1 + e2)/sqrt2, b = (1, 0).  In the gist.science form
+    the erase READS with b.k = (1/sqrt2, 0) and erases ALONG k:
+        (b.k)^T S = row1 / sqrt2,   S' = S - k (row1 / sqrt2)  ->  row1 -= row1/2, row2 -= row1/2.
+    Reading with k and erasing along b.k (the other placement) instead gives
+        row1 -= (row1 + row2)/2, row2 unchanged."""
+    S0 = np.array([[2.0, -1.0, 0.5], [4.0, 3.0, -2.0]])
+    k = np.array([1.0, 1.0]) / math.sqrt(2)
+    _, S = _p3_run(S0, 0.0, k, np.zeros(3), [1.0, 0.0], np.zeros(3))
+    want = S0.copy()
+    want[0] -= S0[0] / 2
+    want[1] -= S0[0] / 2
+    np.testing.assert_allclose(S[0, 0], want, atol=1e-14)
+    other = S0.copy()
+    other[0] -= (S0[0] + S0[1]) / 2
+    assert np.max(np.abs(S[0, 0] - other)) > 0.5
+
+
+def test_p3_erase_with_decay_two_channels():
+    """One token, d_k = d_v = 2, decay a = (0.5, 0.8), k = (0.6, 0.8), b = (0.25, 1), w = 0.
+    By hand: Sbar = Diag(a) S; (b.k) = (0.15, 0.8); e^T Sbar = 0.15 Sbar_1 + 0.8 Sbar_2;
+    S' = Sbar - k (e^T Sbar).  With S = [[4, -2], [1, 3]]: Sbar = [[2, -1], [0.8, 2.4]],
+    e^T Sbar = (0.3 + 0.64, -0.15 + 1.92) = (0.94, 1.77),
+    S' = [[2 - 0.564, -1 - 1.062], [0.8 - 0.752, 2.4 - 1.416]]."""
+    S0 = np.array([[4.0, -2.0], [1.0, 3.0]])
+    _, S = _p3_run(S0, np.log([0.5, 0.8]), [0.6, 0.8], [0.0, 0.0], [0.25, 1.0], [0.0, 0.0])
+    want = np.array([[2 - 0.564, -1 - 1.062], [0.8 - 0.752, 2.4 - 1.416]])
+    np.testing.assert_allclose(S[0, 0], want, atol=1e-13)
+
+
+def test_p3_write_axis_closed_form():
+    """b = 0 in the gist.science form: S_T = Gamma_T S0 + sum_t Diag(gamma_T / gamma_t) k_t (w_t . v_t)^T,
+    with w on the VALUE axis (d_v = 4 channels, d_k = 3): the write gate scales columns, not rows."""
+    rng = np.random.default_rng(31)
+    dk, dv, T = 3, 4, 6
+    S0 = rng.standard_normal((dk, dv))
+    k = rng.standard_normal((T, dk))
+    v = rng.standard_normal((T, dv))
+    w = rng.uniform(0, 1, (T, dv))
+    la = -rng.uniform(0, 0.5, (T, dk))
+    _, S = oracle.gdn2_fwd(rng.standard_normal((T, 1, dk)), k.reshape(T, 1, dk), v.reshape(T, 1, dv),
+                           la.reshape(T, 1, dk), np.zeros((T, 1, dk)), w.reshape(T, 1, dv),
+                           S0=S0.reshape(1, 1, dk, dv), flags=oracle.GATE_FORM_P3)
+    L = np.cumsum(la, axis=0)
+    want = np.exp(L[-1])[:, None] * S0
+    for t in range(T):
+        want += np.outer(np.exp(L[-1] - L[t]) * k[t], w[t] * v[t])
+    np.testing.assert_allclose(S[0, 0], want, rtol=1e-12, atol=1e-13)
+
+
+def test_p3_erase_only_rank_one_projection():
+    """w = 0, no decay, unit key e_j, b = e_j: (I - e_j e_j^T) S removes exactly row j;
+    with b = 0 nothing is erased (the read side carries the gate)."""
+    S0 = np.arange(12, dtype=float).reshape(4, 3) + 1
+    for j in range(4):
+        k = np.zeros(4)
+        k[j] = 1.0
+        _, S = _p3_run(S0, 0.0, k, [5.0, 6.0, 7.0], k, np.zeros(3))
+        want = S0.copy()
+        want[j] = 0
+        np.testing.assert_array_equal(S[0, 0], want)
+        _, S = _p3_run(S0, 0.0, k, [5.0, 6.0, 7.0], np.zeros(4), np.zeros(3))
+        np.testing.assert_array_equal(S[0, 0], S0)
+
+
+def test_p3_printed_update_matrix_form():
+    """Several tokens with channel-wise b != w and d_k != d_v against the update as the
+    gist.science page prints it, applied as whole matrices (I - k (b.k)^T) Diag(a) S + k (w.v)^T,
+    with the read o_t = S_t^T q_t after the update."""
+    rng = np.random.default_rng(33)
+    dk, dv, T = 5, 3, 7
+    S = rng.standard_normal((dk, dv))
+    S0 = S.copy()
+    q = rng.standard_normal((T, dk))
+    k = rng.standard_normal((T, dk))
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    v = rng.standard_normal((T, dv))
+    la = -rng.uniform(0, 0.6, (T, dk))
+    b = rng.uniform(0, 1, (T, dk))
+    w = rng.uniform(0, 1, (T, dv))
+    o_want = []
+    for t in range(T):
+        S = (np.eye(dk) - np.outer(k[t], b[t] * k[t])) @ np.diag(np.exp(la[t])) @ S + np.outer(k[t], w[t] * v[t])
+        o_want.append(S.T @ q[t])
+    o, Sg = oracle.gdn2_fwd(q.reshape(T, 1, dk), k.reshape(T, 1, dk), v.reshape(T, 1, dv), la.reshape(T, 1, dk),
+                            b.reshape(T, 1, dk), w.reshape(T, 1, dv), S0=S0.reshape(1, 1, dk, dv),
+                            flags=oracle.GATE_FORM_P3)
+    np.testing.assert_allclose(Sg[0, 0], S, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(o[:, 0], np.array(o_want), rtol=1e-12, atol=1e-13)
+
+
 def test_p3_form_differs_when_gates_are_channelwise():
     """With channel-wise b != w the two gate placements are different models."""
     rng = np.random.default_rng(13)
