@@ -12,6 +12,15 @@ channel-wise decay and decoupled channel-wise gates, S0 ~ N(0, 0.02).  Inputs
 tokens/s over all ranks (weak scaling: every rank runs its own batch; the
 units shard with no data-path collective).
 
+With --gpus N > 1 the script runs one rank per GPU: launched by torchrun it
+checks that WORLD_SIZE equals N; launched plainly it starts the N ranks itself
+through torch.distributed.run (rendezvous on 127.0.0.1).  Times are CUDA-event
+times on each rank, reported as the maximum over ranks; rank 0 prints.
+
+`configs` times the other prefill workloads on the same line: the tied
+scalar-gate Gated DeltaNet batch (4 x 4096 x 16) and the packed varlen batch
+(16 sequences of 4k-64k tokens, 524,288 in total), each with its roofline.
+
 The same JSON line carries `decode`: 1024 recurrent decode steps over 256
 sequences x 16 heads with a 268 MB fp32 state built by a 2048-token chunked
 prefill (tokens/s and fraction of HBM bandwidth), the roofline of the chunk
@@ -48,7 +57,10 @@ WORKLOAD = "gdn2_b8_t4k"
 # tcgen05 GEMMs the chunk kernel issues per token-head (C=64, d=128):
 # G1 8*C*dk + R 2*C*dv + 2*dk*dv + M 2*C*dv + O 2*dk*dv + 4*C*dv + dS 4*dk*dv
 FLOP_PER_TOKHEAD = 8 * 64 * 128 + 8 * 64 * 128 + 8 * 128 * 128
+# with x_r == p_r (tied gates) the first GEMM runs at N = 64: 4 C dk instead of 8 C dk
+FLOP_PER_TOKHEAD_TIED = FLOP_PER_TOKHEAD - 4 * 64 * 128
 BYTES_PER_TOKHEAD = 6 * 128 * 2 + 128 * 2                      # six bf16 inputs + bf16 o
+BYTES_PER_TOKHEAD_SCALAR = 3 * 128 * 2 + 2 * 2 + 128 * 2       # q, k, v + scalar alpha, beta + o
 STATE_BYTES = 128 * 128 * 4                                    # one fp32 state
 # fp32 operations of the backward per token-head (d_k = d_v = 128): per state
 # element, the forward sweep and the block recompute take 7 each (decay, erase
@@ -143,6 +155,54 @@ class ClockSampler:
                 "samples": len(mhz)}
 
 
+# ----------------------------------------------------------------------------- ranks
+def free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def ensure_ranks(gpus: int, argv, script: str):
+    """One process per GPU.  Under torchrun (WORLD_SIZE set) the world size must equal
+    ``gpus``.  Without it and with ``gpus`` > 1, start ``gpus`` ranks of this same command
+    through torch.distributed.run (rendezvous on 127.0.0.1) and return their exit status;
+    otherwise return None and let the caller run as the only rank."""
+    ws = os.environ.get("WORLD_SIZE")
+    if ws is not None:
+        if int(ws) != gpus:
+            raise SystemExit(f"WORLD_SIZE={ws} but --gpus {gpus}: run one rank per GPU")
+        return None
+    if gpus <= 1:
+        return None
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+           "--master-addr=127.0.0.1", f"--master-port={free_port()}", script, *argv]
+    return subprocess.call(cmd)
+
+
+def rank_env():
+    """(world, rank, local rank) from the torchrun environment (1, 0, 0 without it)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The maximum of ``x`` over all ranks (a device-side time is reported as its max)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def emit(line: dict, rank: int):
+    """Rank 0 prints the one JSON line."""
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_sample(inp, max_seconds: float, n_units: int = 0):
     """Time the float64 oracle on whole (sequence, head) units of the workload,
@@ -187,7 +247,7 @@ def oracle_sample(inp, max_seconds: float, n_units: int = 0):
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args):
     import torch
-    rank = int(os.environ.get("RANK", "0"))
+    _, rank, _ = rank_env()
     if rank != 0:
         return 0
     from gated_delta_rule_159_b200 import inputs
@@ -241,19 +301,22 @@ def main():
                     help="segments per sequence of the long-context split forward (0: as many as keep "
                          "the 16 heads' segments within the SM count)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true")
+    ap.add_argument("--config-steps", type=int, default=5)
     ap.add_argument("--no-cpu", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    rc = ensure_ranks(args.gpus, sys.argv[1:], os.path.abspath(__file__))
+    if rc is not None:
+        return rc
 
     import torch
     import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     if world > 1:
         os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
         torch.cuda.set_device(local)
@@ -268,12 +331,8 @@ def main():
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rmax(x: float) -> float:
+        return max_over_ranks(x, world, dev)
 
     hbm_peak, tc_peak, peak_src = peaks()
 
@@ -307,7 +366,7 @@ def main():
     clocks = sampler.stop()
     total_ms = ev[0][0].elapsed_time(ev[-1][1])
     launch_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = max_over_ranks(total_ms)
+    total_ms = rmax(total_ms)
     status = gdn2.check_status(ws)
     if status != gdn2.OK:
         raise RuntimeError(f"chunk kernel reported device status {status}")
@@ -376,7 +435,7 @@ def main():
         e2e_run(args.e2e_steps, start_event=e0)
         e1.record(stream)
         barrier()
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+        e2e_ms = rmax(e0.elapsed_time(e1))
         h2d = sum(t.numel() * t.element_size() for t in host.values()) + S0_h.numel() * 4
         d2h = o_h.numel() * o_h.element_size() + ST_h.numel() * 4
         e2e = {"value": T_tot * world * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
@@ -396,6 +455,68 @@ def main():
     cfg = config_block(inp, world)
     del inp, args4
     torch.cuda.empty_cache()
+
+    # ---------------- the other prefill workloads: tied scalar-gate Gated DeltaNet (4 x 4096 x 16)
+    # and the packed varlen long-context batch (16 sequences of 4k-64k tokens, 524,288 in total)
+    configs = None
+    if not args.no_configs:
+        configs = {}
+        for wname in ("gdn_scalar_b4_t4k", "gdn2_varlen_16x4k-64k"):
+            ci = inputs.make_inputs(wname, dev, seed=600 + rank)
+            wl = ci["workload"]
+            Nc, Tc = ci["n_seqs"], ci["T_tot"]
+            kw = dict(scalar_decay=ci["scalar_decay"], scalar_gates=ci["scalar_gates"], tied_gates=ci["tied_gates"])
+            if ci["equal_lengths"]:
+                cargs = [None if ci[n] is None else ci[n].view(Nc, Tc // Nc, *ci[n].shape[1:]) for n in names]
+                cu, cu_h = None, None
+            else:
+                cargs = [ci[n] for n in names]
+                cu, cu_h = ci["cu_seqlens"], ci["cu_host"]
+            co = torch.empty(*cargs[2].shape, dtype=torch.bfloat16, device=dev)
+            cS = torch.empty(Nc, 16, 128, 128, dtype=torch.float32, device=dev)
+            cdims = gdn2.make_dims(Nc, Tc if cu is not None else Tc // Nc, 16, 128, 128, 64, gdn2.BF16, gdn2.BF16,
+                                   gdn2.flags_of(**kw))
+            cws = torch.empty(gdn2.workspace_size(cdims), dtype=torch.uint8, device=dev)
+
+            def cstep():
+                gdn2.chunk_fwd(*cargs, ci["S0"], cu, cu_seqlens_host=cu_h, o=co, S_T=cS, workspace=cws, **kw)
+
+            for _ in range(args.warmup):
+                cstep()
+            barrier()
+            reps = args.config_steps
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(reps):
+                cstep()
+            a1.record(stream)
+            barrier()
+            cms = rmax(a0.elapsed_time(a1)) / reps
+            if gdn2.check_status(cws) != gdn2.OK:
+                raise RuntimeError(f"chunk kernel reported a timed-out wait ({wname})")
+            tokheads = Tc * 16
+            units_c = Nc * 16
+            per_tok = BYTES_PER_TOKHEAD_SCALAR if wl.scalar_gates else BYTES_PER_TOKHEAD
+            states = (2 if ci["S0"] is not None else 1) * units_c * STATE_BYTES
+            cbytes = per_tok * tokheads + states
+            cflops = (FLOP_PER_TOKHEAD_TIED if ci["tied_gates"] else FLOP_PER_TOKHEAD) * tokheads
+            gbs = cbytes / (cms / 1e3) / 1e9
+            tfs = cflops / (cms / 1e3) / 1e12
+            bound = "hbm" if cbytes / (hbm_peak * 1e9) >= cflops / (tc_peak * 1e12) else "tensor"
+            configs[wname] = {
+                "ms": cms, "value": Tc * world / (cms / 1e3), "unit": "tokens/s", "steps": reps,
+                "sequences": Nc, "tokens": Tc, "units": units_c,
+                "gates": "tied scalar alpha, beta (b = w = beta 1)" if wl.scalar_gates else
+                         "channel-wise decay, decoupled channel-wise erase/write",
+                "roofline": {"bound": bound, "achieved": gbs if bound == "hbm" else tfs,
+                             "peak": hbm_peak if bound == "hbm" else tc_peak,
+                             "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+                             "frac": gbs / hbm_peak if bound == "hbm" else tfs / tc_peak,
+                             "hbm_frac": gbs / hbm_peak, "tensor_frac": tfs / tc_peak,
+                             "alg_bytes_per_launch": cbytes, "alg_flops_per_launch": cflops,
+                             "traffic": None, "peak_source": peak_src}}
+            del ci, cargs, co, cS, cws
+            torch.cuda.empty_cache()
 
     # ---------------- decode
     decode = None
@@ -422,7 +543,7 @@ def main():
             gdn2.decode_step(*(di[n][t] for n in names), S, o=od)
         e1.record(stream)
         barrier()
-        plain_ms = max_over_ranks(e0.elapsed_time(e1))
+        plain_ms = rmax(e0.elapsed_time(e1))
         # The same steps captured once as a CUDA graph and replayed: one graph launch
         # per decode loop, so the per-step host launch gap leaves the timed region.
         graph = torch.cuda.CUDAGraph()
@@ -437,7 +558,7 @@ def main():
         e1.record(stream)
         barrier()
         dclocks = sd.stop()
-        dms = max_over_ranks(e0.elapsed_time(e1))
+        dms = rmax(e0.elapsed_time(e1))
         del graph
         if gdn2.decode_status() != gdn2.OK:
             raise RuntimeError("decode kernel reported a timed-out wait")
@@ -480,7 +601,7 @@ def main():
         e1.record(stream)
         barrier()
         bclocks = bs.stop()
-        bms = max_over_ranks(e0.elapsed_time(e1)) / args.bwd_steps
+        bms = rmax(e0.elapsed_time(e1)) / args.bwd_steps
         tokheads = Nb * Tb * 16
         tflops = BWD_FLOP_PER_TOKHEAD * tokheads / (bms / 1e3) / 1e12
         peak32 = fp32_peak_tflops(bclocks.get("sm_max_mhz") or 1965.0)
@@ -517,7 +638,7 @@ def main():
                 fn()
             a1.record(stream)
             barrier()
-            return max_over_ranks(a0.elapsed_time(a1)) / reps
+            return rmax(a0.elapsed_time(a1)) / reps
 
         t_plain = timed(lambda: gdn2.chunk_fwd(*largs, li["S0"], None, workspace=pws))
         t_split = timed(lambda: gdn2.chunk_fwd_split(*largs, li["S0"], n_split=args.split, workspace=lws))
@@ -544,9 +665,9 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes and distributions of the "
                                                           "full GDN-2 workload)",
             "config": cfg, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches, "clocks": clocks, "decode": decode, "bwd": bwd, "long_context": long_ctx}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+            "gpu_launches": launches, "clocks": clocks, "configs": configs, "decode": decode, "bwd": bwd,
+            "long_context": long_ctx}
+    emit(line, rank)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
