@@ -1,6 +1,7 @@
 // api.cu -- the extern "C" entry points declared in include/gdn2.h: argument
 // validation, workspace layout, unit scheduling and kernel dispatch.  Nothing
 // here computes the recurrence; every step of it runs in the kernels.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -82,11 +83,36 @@ int check_inputs(const void *q, const void *k, const void *v, const void *log_a,
 
 namespace gdn2 {
 int set_last_error(int code, const char *message) { return fail(code, "%s", message); }
+
+namespace {
+std::atomic<int> g_debug_site{0};
+std::atomic<unsigned long long> g_debug_ns{0};
+}  // namespace
+
+bool take_debug_timeout(int site, uint64_t *wait_ns) {
+  int armed = site;
+  if (g_debug_site.load(std::memory_order_relaxed) != site ||
+      !g_debug_site.compare_exchange_strong(armed, 0))
+    return false;
+  *wait_ns = g_debug_ns.load();
+  return true;
+}
 }  // namespace gdn2
 
 extern "C" {
 
 int gdn2_version(void) { return 100; }
+
+int gdn2_debug_timeout_once(int32_t site, uint64_t wait_ns) {
+  g_err[0] = '\0';
+  if (site != GDN2_DEBUG_CHUNK && site != GDN2_DEBUG_DECODE)
+    return fail(GDN2_ERR_INVALID_ARG, "unknown debug site %d", site);
+  if (wait_ns < 1000ull || wait_ns > 10000000000ull)
+    return fail(GDN2_ERR_INVALID_ARG, "wait_ns must lie in [1000, 1e10] (got %llu)", (unsigned long long)wait_ns);
+  gdn2::g_debug_ns.store(wait_ns);
+  gdn2::g_debug_site.store(site);
+  return GDN2_OK;
+}
 
 const char *gdn2_last_error(void) { return g_err; }
 

@@ -7,10 +7,15 @@
 // of rows i, j in [0, 64) starting from state S (d_k x d_v):
 //
 //   x = b.k (erase outer), y = k (erase read), p = w.k (write outer), z = v,
-//   L_i = sum_{j<=i} log_a_j (per channel), L_ref = L_31, L_C = L_63.
-//   Scaled operands (every factor's exponent is bounded by half a chunk):
+//   L_i = sum_{j<=i} log_a_j (per channel), L_C = L_63,
+//   L_ref = (L_0 + L_63) / 2 per channel, the midpoint of the chunk's decay range.
+//   Scaled operands (every factor's exponent is at most half the chunk's decay range):
 //     k_r = k e^{L - L_ref},  q_r = q e^{L - L_ref},
 //     x_r = x e^{L_ref - L},  p_r = p e^{L_ref - L},  S_r = Diag(e^{L_ref}) S.
+//   A chunk in which some channel decays by more than kFastSpan (128 nats) between its
+//   first and last row would need factors beyond e^{64}; such a chunk runs the
+//   recurrence token by token instead (CUDA cores, the state kept in registers), which
+//   is exact for any finite log_a <= 0.
 //   G1  [A B ; QX QP] = [k_r ; q_r] [x_r ; p_r]^T         (M=128 N=128 K=128)
 //       A, B strictly lower; QX, QP lower incl. diagonal.
 //   solve T = (I + A)^-1: 8x8 diagonal blocks by forward substitution, then the
@@ -57,6 +62,11 @@ constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s
 constexpr float kLog2eF = 1.4426950408889634f;
+// Largest in-chunk decay range L_0 - L_63 (nats, per channel) of the factored form: its
+// operand factors then stay within e^{+-64}, far from the fp32/bf16 limit (e^{88.7}), and
+// a state term that underflows in S_r = e^{L_ref} S can only have been worth e^{64 - 87.3}
+// of the state's size in any output.
+constexpr float kFastSpan = 128.f;
 
 // Shared-memory map, byte offsets from a 1024-byte-aligned base.  Every operand
 // tile is a stack of 8-row x 128-byte swizzle atoms.
@@ -78,15 +88,26 @@ constexpr uint32_t MISC_DL = 512;      // float[128]  e^{L_C - L_ref} of the chu
 constexpr uint32_t MISC_SM = 1024;     // float[128]  e^{L_ref}
 constexpr uint32_t MISC_PART = 1536;   // float[16][128] 4-row sums of log_a, then exclusive prefixes
 constexpr uint32_t MISC_REF = 9728;    // float[128]  L_ref
-constexpr uint32_t MISC_BAR = 10240;   // 10 mbarriers
-constexpr uint32_t MISC_TMEM = 10320;
-constexpr uint32_t MISC_ABORT = 10324;
-constexpr uint32_t MISC_UNIT = 10328;
-constexpr uint32_t MISC_BYTES = 10336;
+constexpr uint32_t MISC_BAR = 10240;   // 12 mbarriers
+constexpr uint32_t MISC_TMEM = 10336;
+constexpr uint32_t MISC_ABORT = 10340;
+constexpr uint32_t MISC_UNIT = 10344;
+constexpr uint32_t MISC_ISS = 10352;   // uint32[4]   phases armed per TMA barrier (A, L, W, X)
+constexpr uint32_t MISC_L0 = 10368;    // float[128]  L_0 (the chunk's first row)
+constexpr uint32_t MISC_BYTES = 10880;
+// Token-serial chunks stage their per-token vectors in [OFF_OS, OFF_MISC) (fp32):
+// a, q, y, x, p as [32 tokens][128], z as [32][128], q.x and q.p [32], and the
+// cross-warp exchange of the column sums [2][4][128] float2.
+constexpr uint32_t SER_A = 0, SER_Q = 4096, SER_Y = 8192, SER_X = 12288, SER_P = 16384, SER_Z = 20480;
+constexpr uint32_t SER_QX = 24576, SER_QP = 24608, SER_XCH = 24640;  // float offsets from OFF_OS
+static_assert(OFF_OS + 4 * SER_XCH + 2 * 4 * 128 * 8 <= OFF_MISC, "token-serial staging overflows");
 constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES + 1024;  // + base alignment slack
 // mbarrier slots
-enum { BAR_TMA_A = 0, BAR_TMA_L, BAR_TMA_W, BAR_TMA_X, BAR_G1, BAR_E1, BAR_GA, BAR_GB, BAR_G4, BAR_G5, kNumBars };
+// (BAR_DRAIN0/1: used once, after a timed-out wait, to let the MMAs of the two issuing threads finish)
+enum { BAR_TMA_A = 0, BAR_TMA_L, BAR_TMA_W, BAR_TMA_X, BAR_G1, BAR_E1, BAR_GA, BAR_GB, BAR_G4, BAR_G5,
+       BAR_DRAIN0, BAR_DRAIN1, kNumBars };
 static_assert(MISC_BAR + 8 * kNumBars <= MISC_TMEM, "mbarriers overlap the TMEM address slot");
+static_assert(MISC_ISS + 16 <= MISC_L0, "issue counters overlap L_0");
 
 struct TcParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_g, tm_b, tm_w;
@@ -94,6 +115,8 @@ struct TcParams {
   ChunkProblem p;
   int32_t *counter;
   int n_units;
+  uint64_t wait_ns;  // limit of every mbarrier wait (kWaitTimeoutNs unless the timeout test hook is armed)
+  int dbg_skip;      // timeout test hook: CTA 0 arms its first k/q/v load group but issues none of its copies
 };
 
 __device__ __forceinline__ void named_bar(int id, int count) {
@@ -139,7 +162,7 @@ __device__ __forceinline__ uint32_t swz(int r, uint32_t chunk) {
 }
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                         int32_t *status) {
+                                         int32_t *status, uint64_t limit_ns) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   if (*abort_flag) return false;
   const uint64_t t0 = global_timer_ns();
@@ -147,7 +170,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   while (!ptx::mbar_try_wait(bar, parity)) {
     if ((++it & 255u) == 0) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         if (status) atomicExch(status, kStatusTimeout);
         return false;
@@ -155,6 +178,15 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     }
   }
   return true;
+}
+
+// Bounded wait that ignores the abort flag: the wind-down after a timed-out wait uses it to let
+// the copies and MMAs this CTA issued land before it frees its memory.
+__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  uint32_t it = 0;
+  while (!ptx::mbar_try_wait(bar, parity))
+    if ((++it & 255u) == 0 && global_timer_ns() - t0 > limit_ns) return;
 }
 
 __device__ __forceinline__ uint4 pack8(const float *f, float s) {
@@ -171,6 +203,174 @@ __device__ __forceinline__ float4 unpack4(uint2 u) {
 }
 __device__ __forceinline__ uint2 pack4(float a, float b, float c, float d) {
   return make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
+}
+
+// A chunk whose decay range is beyond the factored form, token by token (CUDA cores, fp32):
+// per token, Sbar = Diag(a) S; r = Sbar^T y; u = Sbar^T q; o = u - (q.x) r + (q.p) z;
+// S = Sbar - x r^T + p z^T, with (y, x, p, z) = (k, b.k, w.k, v), or (b.k, k, k, w.v) in the
+// gist.science form.  The 512 threads hold the state as the chunk kernel's TMEM layout gives it
+// (thread: dv channel `row`, dk channels [32 cg, 32 cg + 32)); the four warps of a lane
+// quadrant add their column sums through shared memory.  The per-token vectors of 32 tokens at
+// a time are staged in fp32 in [OFF_OS, OFF_MISC).  tmem_s: this thread's 32 state columns;
+// tau: the previous chunk's e^{L_C - L_ref} for them (NULL: 1); the state goes back to TMEM
+// as it is (tau = 1).  Kept out of line so that its registers do not press on the factored path.
+template <bool kScalarDecay, bool kScalarGates, bool kP3, bool kProlog, typename Tout>
+__device__ __noinline__ void serial_chunk(const ChunkProblem &p, uint8_t *gb, uint32_t tmem_s, const float *tau,
+                                          int t0, int nvalid, int h) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, cg = warp >> 2, row = qd * 32 + lane;
+  const int H = p.n_heads;
+  const __nv_bfloat16 *g_la = static_cast<const __nv_bfloat16 *>(p.log_a);
+  const __nv_bfloat16 *g_b = static_cast<const __nv_bfloat16 *>(p.b);
+  const __nv_bfloat16 *g_w = static_cast<const __nv_bfloat16 *>((p.flags & GDN2_TIED_GATES) ? p.b : p.w);
+  float *fs = reinterpret_cast<float *>(gb + OFF_OS);
+  const __nv_bfloat16 *g_q = static_cast<const __nv_bfloat16 *>(p.q);
+  const __nv_bfloat16 *g_k = static_cast<const __nv_bfloat16 *>(p.k);
+  const __nv_bfloat16 *g_v = static_cast<const __nv_bfloat16 *>(p.v);
+  for (int half = 0; half * 32 < nvalid; ++half) {
+    const int nt = nvalid - half * 32 < 32 ? nvalid - half * 32 : 32;
+    // stage the per-token vectors of tokens [32 half, 32 half + nt): one token row per warp
+    // at a time, lane l holding channels 4 l .. 4 l + 3 (both d_k and d_v are 128)
+    for (int tl = warp; tl < nt; tl += 16) {
+      const size_t rt = (size_t)(t0 + half * 32 + tl) * H + h;
+      float4 la, bb, ww;
+      float4 kk = unpack4(*reinterpret_cast<const uint2 *>(g_k + rt * D + 4 * lane));
+      float4 qq = unpack4(*reinterpret_cast<const uint2 *>(g_q + rt * D + 4 * lane));
+      const float4 vv = unpack4(*reinterpret_cast<const uint2 *>(g_v + rt * D + 4 * lane));
+      if (kScalarDecay) {
+        const float x = __bfloat162float(g_la[rt]);
+        la = make_float4(x, x, x, x);
+      } else {
+        la = unpack4(*reinterpret_cast<const uint2 *>(g_la + rt * D + 4 * lane));
+      }
+      if (kScalarGates) {
+        const float xb = __bfloat162float(g_b[rt]), xw = __bfloat162float(g_w[rt]);
+        bb = make_float4(xb, xb, xb, xb);
+        ww = make_float4(xw, xw, xw, xw);
+      } else {
+        bb = unpack4(*reinterpret_cast<const uint2 *>(g_b + rt * D + 4 * lane));
+        ww = unpack4(*reinterpret_cast<const uint2 *>(g_w + rt * D + 4 * lane));
+      }
+      if (kProlog) {
+        la = make_float4(log_sigmoid_f(la.x), log_sigmoid_f(la.y), log_sigmoid_f(la.z), log_sigmoid_f(la.w));
+        bb = make_float4(sigmoid_f(bb.x), sigmoid_f(bb.y), sigmoid_f(bb.z), sigmoid_f(bb.w));
+        ww = make_float4(sigmoid_f(ww.x), sigmoid_f(ww.y), sigmoid_f(ww.z), sigmoid_f(ww.w));
+        float k2 = kk.x * kk.x + kk.y * kk.y + kk.z * kk.z + kk.w * kk.w;
+        float q2 = qq.x * qq.x + qq.y * qq.y + qq.z * qq.z + qq.w * qq.w;
+#pragma unroll
+        for (int sh = 16; sh >= 1; sh >>= 1) {
+          k2 += __shfl_xor_sync(0xffffffffu, k2, sh);
+          q2 += __shfl_xor_sync(0xffffffffu, q2, sh);
+        }
+        const float ik = rsqrtf(k2 + kNormEps), iq = rsqrtf(q2 + kNormEps);
+        kk = make_float4(kk.x * ik, kk.y * ik, kk.z * ik, kk.w * ik);
+        qq = make_float4(qq.x * iq, qq.y * iq, qq.z * iq, qq.w * iq);
+      }
+      const float4 bk = make_float4(bb.x * kk.x, bb.y * kk.y, bb.z * kk.z, bb.w * kk.w);
+      // erase read y, erase outer x, write outer p and written value z (per d_v channel):
+      // (k, b.k, w.k, v) by default, (b.k, k, k, w.v) in the gist.science form
+      const float4 yy = kP3 ? bk : kk;
+      const float4 xx = kP3 ? kk : bk;
+      const float4 pp = kP3 ? kk : make_float4(ww.x * kk.x, ww.y * kk.y, ww.z * kk.z, ww.w * kk.w);
+      const float4 zz = kP3 ? make_float4(ww.x * vv.x, ww.y * vv.y, ww.z * vv.z, ww.w * vv.w) : vv;
+      const float4 aa = make_float4(ptx::ex2(la.x * kLog2eF), ptx::ex2(la.y * kLog2eF), ptx::ex2(la.z * kLog2eF),
+                                    ptx::ex2(la.w * kLog2eF));
+      float qx = qq.x * xx.x + qq.y * xx.y + qq.z * xx.z + qq.w * xx.w;
+      float qp = qq.x * pp.x + qq.y * pp.y + qq.z * pp.z + qq.w * pp.w;
+#pragma unroll
+      for (int sh = 16; sh >= 1; sh >>= 1) {
+        qx += __shfl_xor_sync(0xffffffffu, qx, sh);
+        qp += __shfl_xor_sync(0xffffffffu, qp, sh);
+      }
+      const int e = tl * 128 + 4 * lane;
+      *reinterpret_cast<float4 *>(fs + SER_A + e) = aa;
+      *reinterpret_cast<float4 *>(fs + SER_Q + e) = qq;
+      *reinterpret_cast<float4 *>(fs + SER_Y + e) = yy;
+      *reinterpret_cast<float4 *>(fs + SER_X + e) = xx;
+      *reinterpret_cast<float4 *>(fs + SER_P + e) = pp;
+      *reinterpret_cast<float4 *>(fs + SER_Z + e) = zz;
+      if (lane == 0) {
+        fs[SER_QX + tl] = qx;
+        fs[SER_QP + tl] = qp;
+      }
+    }
+    __syncthreads();
+    // the state into registers (dv channel `row`, dk channels [32 cg, 32 cg + 32)): the first
+    // half takes S = Diag(tau) Sacc, the second the first half's result
+    float sv[32];
+    {
+      uint32_t r[32];
+      ptx::tmem_ld32(tmem_s, r);
+      ptx::tmem_wait_ld();
+      const bool scale = half == 0 && tau != nullptr;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(r[j]) * (scale ? tau[j] : 1.f);
+    }
+    // per token: Sbar = Diag(a) S; r = Sbar^T y and u = Sbar^T q (column sums over d_k, the
+    // four warps of a lane quadrant holding a quarter each); o = u - (q.x) r + (q.p) z;
+    // S = Sbar - x r^T + p z^T
+    float2 *xch = reinterpret_cast<float2 *>(fs + SER_XCH);
+    for (int tl = 0; tl < nt; ++tl) {
+      const float *A = fs + SER_A + tl * 128 + cg * 32;
+      const float *Y = fs + SER_Y + tl * 128 + cg * 32;
+      const float *Qv = fs + SER_Q + tl * 128 + cg * 32;
+      float rp = 0.f, up = 0.f;
+#pragma unroll
+      for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 a4 = *reinterpret_cast<const float4 *>(A + 4 * j4);
+        const float4 y4 = *reinterpret_cast<const float4 *>(Y + 4 * j4);
+        const float4 q4 = *reinterpret_cast<const float4 *>(Qv + 4 * j4);
+        sv[4 * j4] *= a4.x;
+        sv[4 * j4 + 1] *= a4.y;
+        sv[4 * j4 + 2] *= a4.z;
+        sv[4 * j4 + 3] *= a4.w;
+        rp = fmaf(sv[4 * j4], y4.x, rp);
+        rp = fmaf(sv[4 * j4 + 1], y4.y, rp);
+        rp = fmaf(sv[4 * j4 + 2], y4.z, rp);
+        rp = fmaf(sv[4 * j4 + 3], y4.w, rp);
+        up = fmaf(sv[4 * j4], q4.x, up);
+        up = fmaf(sv[4 * j4 + 1], q4.y, up);
+        up = fmaf(sv[4 * j4 + 2], q4.z, up);
+        up = fmaf(sv[4 * j4 + 3], q4.w, up);
+        asm volatile("" ::: "memory");  // keep the loads of one step at a time in registers
+      }
+      xch[((tl & 1) * 4 + cg) * 128 + row] = make_float2(rp, up);
+      named_bar(2 + qd, 128);  // the four warps of this lane quadrant
+      float r = 0.f, u = 0.f;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {  // the same order in all four warps: identical r and u
+        const float2 pr = xch[((tl & 1) * 4 + g) * 128 + row];
+        r += pr.x;
+        u += pr.y;
+      }
+      const float zr = fs[SER_Z + tl * 128 + row];
+      if (cg == 0) {
+        const float ov = u - fs[SER_QX + tl] * r + fs[SER_QP + tl] * zr;
+        Tout *go = static_cast<Tout *>(p.o) + ((size_t)(t0 + half * 32 + tl) * H + h) * D + row;
+        *go = from_f32<Tout>(ov);
+      }
+      const float *X = fs + SER_X + tl * 128 + cg * 32;
+      const float *P = fs + SER_P + tl * 128 + cg * 32;
+#pragma unroll
+      for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 x4 = *reinterpret_cast<const float4 *>(X + 4 * j4);
+        const float4 p4 = *reinterpret_cast<const float4 *>(P + 4 * j4);
+        sv[4 * j4] = fmaf(p4.x, zr, fmaf(-x4.x, r, sv[4 * j4]));
+        sv[4 * j4 + 1] = fmaf(p4.y, zr, fmaf(-x4.y, r, sv[4 * j4 + 1]));
+        sv[4 * j4 + 2] = fmaf(p4.z, zr, fmaf(-x4.z, r, sv[4 * j4 + 2]));
+        sv[4 * j4 + 3] = fmaf(p4.w, zr, fmaf(-x4.w, r, sv[4 * j4 + 3]));
+        asm volatile("" ::: "memory");
+      }
+    }
+    {  // the state back into TMEM (as Sacc with tau = 1)
+      uint32_t r[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(sv[j]);
+      ptx::tmem_st32(tmem_s, r);
+      ptx::tmem_wait_st();
+    }
+    __syncthreads();  // the staging of the next half overwrites what the token loop read
+  }
 }
 
 // kP3: the gist.science gate placement.  The operands are then k_r = (b.k) e^{L - L_ref}
@@ -202,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   float *sSM = reinterpret_cast<float *>(gb + OFF_MISC + MISC_SM);
   float *part = reinterpret_cast<float *>(gb + OFF_MISC + MISC_PART);
   float *sRef = reinterpret_cast<float *>(gb + OFF_MISC + MISC_REF);
+  float *sL0 = reinterpret_cast<float *>(gb + OFF_MISC + MISC_L0);
   constexpr int kIssuer = 32;      // issues a unit's first TMA loads, the log_a and b loads and the o stores
   constexpr int kIssueWarp = 15;   // issues the T-independent MMAs during the solve
   constexpr int kSolveThreads = 480;  // warps 0-14
@@ -209,6 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   volatile int *sAbort = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_ABORT);
   volatile int *sUnit = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_UNIT);
   auto bar = [&](int i) { return sb + OFF_MISC + MISC_BAR + 8u * (uint32_t)i; };
+  auto waitb = [&](uint32_t b, uint32_t parity) { return wait_bar(b, parity, sAbort, p.status, P.wait_ns); };
+  volatile uint32_t *sIss = reinterpret_cast<volatile uint32_t *>(gb + OFF_MISC + MISC_ISS);
 
   // the bf16 T tile's blocks above the diagonal are never written by the solve: zero once
   sts_v4(sb + OFF_T + 16u * (uint32_t)tid, make_uint4(0u, 0u, 0u, 0u));
@@ -217,6 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     for (int i = 0; i < kNumBars; ++i) ptx::mbar_init(bar(i), 1);
     ptx::fence_mbar_init();
     *sAbort = 0;
+    for (int i = 0; i < 4; ++i) sIss[i] = 0u;
     ptx::tma_prefetch_desc(&P.tm_q);
     ptx::tma_prefetch_desc(&P.tm_k);
     ptx::tma_prefetch_desc(&P.tm_v);
@@ -249,8 +453,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   // TMA issue (thread 0): group A = k, q, v (+ log_a), group B = b, w.
   // TMA issue: group A = k, q, v; group L = log_a (into the log_a slot, free from the start of
   // the previous chunk, so it is requested a whole chunk ahead); group W = w; group X = b.
+  bool dbg_armed = P.dbg_skip != 0 && blockIdx.x == 0;  // the timeout test hook (thread kIssuer)
   auto issue_tma_a = [&](int h, int t0) {
     ptx::mbar_arrive_expect_tx(bar(BAR_TMA_A), 3u * 2u * 8192u);
+    sIss[BAR_TMA_A] = sIss[BAR_TMA_A] + 1u;
+    if (dbg_armed) {  // bytes announced, no copy issued: the wait for this group runs out
+      dbg_armed = false;
+      return;
+    }
 #pragma unroll
     for (int kb = 0; kb < 2; ++kb) {
       ptx::tma_load_3d(sb + OFF_KQ + kb * 16384, &P.tm_k, kb * 64, h, t0, bar(BAR_TMA_A));
@@ -261,6 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   auto issue_tma_l = [&](int h, int t0) {
     if (kScalarDecay) return;
     ptx::mbar_arrive_expect_tx(bar(BAR_TMA_L), 2u * 8192u);
+    sIss[BAR_TMA_L] = sIss[BAR_TMA_L] + 1u;
 #pragma unroll
     for (int kb = 0; kb < 2; ++kb) ptx::tma_load_3d(sb + OFF_G + kb * 8192, &P.tm_g, kb * 64, h, t0, bar(BAR_TMA_L));
   };
@@ -269,6 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   auto issue_tma_w = [&](int h, int t0) {
     if (kScalarGates) return;
     ptx::mbar_arrive_expect_tx(bar(BAR_TMA_W), 2u * 8192u);
+    sIss[BAR_TMA_W] = sIss[BAR_TMA_W] + 1u;
 #pragma unroll
     for (int kb = 0; kb < 2; ++kb)
       ptx::tma_load_3d(sb + OFF_XP + kb * 16384 + 8192, &P.tm_w, kb * 64, h, t0, bar(BAR_TMA_W));
@@ -276,6 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   auto issue_tma_x = [&](int h, int t0) {
     if (kScalarGates) return;
     ptx::mbar_arrive_expect_tx(bar(BAR_TMA_X), 2u * 8192u);
+    sIss[BAR_TMA_X] = sIss[BAR_TMA_X] + 1u;
 #pragma unroll
     for (int kb = 0; kb < 2; ++kb)
       ptx::tma_load_3d(sb + OFF_G + kb * 8192, &P.tm_b, kb * 64, h, t0, bar(BAR_TMA_X));
@@ -288,9 +501,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   const int e_kb = lane >> 4;
   const uint32_t e_ch16 = (uint32_t)((lane & 15) >> 1), e_cofs = (uint32_t)(lane & 1) * 8u;
   // pass 1 (needs the log_a tile): inclusive cumsum L of this thread's rows, then per channel
-  // the exclusive prefixes over the 16 row groups, L_ref = L_31, e^{L_C - L_ref} into the
-  // parity-pn buffer and e^{L_ref}.  Ends with a CTA barrier, after which the log_a slot is free.
-  auto elem_cumsum = [&](uint32_t pn, int t0n, int nvn, int h, float4 (&L)[4]) {
+  // the exclusive prefixes over the 16 row groups, L_ref = (L_0 + L_63) / 2, e^{L_C - L_ref}
+  // into the parity-pn buffer and e^{L_ref}.  Ends with a CTA barrier, after which the log_a
+  // slot is free; returns non-zero (in every thread) when some channel's decay range
+  // L_0 - L_63 exceeds kFastSpan, i.e. the chunk must run token by token.
+  auto elem_cumsum = [&](uint32_t pn, int t0n, int nvn, int h, float4 (&L)[4]) -> int {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int rr = 0; rr < 4; ++rr) {
@@ -310,21 +525,25 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       L[rr] = acc;
     }
     *reinterpret_cast<float4 *>(part + warp * 128 + 4 * lane) = acc;
+    if (warp == 0) *reinterpret_cast<float4 *>(sL0 + 4 * lane) = L[0];  // L_0 = log_a of row 0
     __syncthreads();
-    if (tid < D) {  // per channel: exclusive prefix over the 16 row groups, L_ref = L_31, L_C = L_63
-      float run = 0.f, refv = 0.f;
+    int wide = 0;
+    if (tid < D) {  // per channel: exclusive prefix over the 16 row groups, L_C = L_63, the reference
+      float run = 0.f;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const float pj = part[j * 128 + tid];
         part[j * 128 + tid] = run;
         run += pj;
-        if (j == 7) refv = run;
       }
+      const float l0 = sL0[tid];
+      const float refv = 0.5f * (l0 + run);
+      wide = !(l0 - run <= kFastSpan);
       sRef[tid] = refv;
       sDLb(pn)[tid] = ptx::ex2((run - refv) * kLog2eF);
       sSM[tid] = ptx::ex2(refv * kLog2eF);
     }
-    __syncthreads();
+    return __syncthreads_or(wide);
   };
   // pass 2 (needs the k, q, v tiles and the w tile): k_r, q_r and p_r in place; rows past the
   // chunk end are zeroed (v too).  ke2 keeps k e^{L_ref - L} for pass 3.
@@ -464,16 +683,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     // The operands of chunk c + 1 are built while chunk c's GEMMs run; a unit's first chunk
     // builds them here.
     float4 L[4], ke2[4];
+    int wide_next = 0;  // the next chunk to run needs the token-serial form (set by elem_cumsum)
     if (nchunks > 0) {
       const int nv0 = (int)(len < C ? len : C);
       const uint32_t par0 = it & 1u;
-      if (!kScalarDecay) wait_bar(bar(BAR_TMA_L), par0, sAbort, p.status);
-      elem_cumsum(par0, (int)bos, nv0, h, L);
+      if (!kScalarDecay) waitb(bar(BAR_TMA_L), par0);
+      wide_next = elem_cumsum(par0, (int)bos, nv0, h, L);
       if (tid == kIssuer && !*sAbort) issue_tma_x(h, (int)bos);
-      wait_bar(bar(BAR_TMA_A), par0, sAbort, p.status);
-      if (!kScalarGates) wait_bar(bar(BAR_TMA_W), par0, sAbort, p.status);
+      waitb(bar(BAR_TMA_A), par0);
+      if (!kScalarGates) waitb(bar(BAR_TMA_W), par0);
       elem_scale((int)bos, nv0, h, L, ke2);
-      if (!kScalarGates) wait_bar(bar(BAR_TMA_X), par0, sAbort, p.status);
+      if (!kScalarGates) waitb(bar(BAR_TMA_X), par0);
       elem_x((int)bos, nv0, h, ke2);
       ptx::fence_proxy_async_smem();
       __syncthreads();
@@ -490,6 +710,57 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       // the log_a slot is free (the b tile it last held was consumed by this chunk's x_r):
       // the next chunk's log_a can land
       if (tid == kIssuer && has_next && !*sAbort) issue_tma_l(h, t0 + C);
+
+      if (wide_next) {
+        // ---- a decay range beyond the factored form: the recurrence token by token.  The
+        //      chunk's operand tiles are not used; its raw inputs are re-read from global memory.
+        if (ci > 0) {  // the previous chunk's GEMMs (the last of them updates the state) are done
+          waitb(bar(BAR_G5), par ^ 1u);
+          ptx::tc_fence_after();
+        }
+        if (tid == kIssuer) ptx::bulk_wait_group_read0();  // the previous o store has read the staging area
+        __syncthreads();
+        // One arrival per chunk on every MMA barrier keeps their phases in step with the chunk
+        // count (plain arrivals: this chunk issues no MMA, and the previous chunk's are done).
+        // They come after the barrier above: every thread has then seen the previous chunk's G5
+        // phase complete, so no wait can find that barrier two phases ahead.
+        if (tid == 0) {
+          ptx::mbar_arrive(bar(BAR_G1));
+          ptx::mbar_arrive(bar(BAR_E1));
+          ptx::mbar_arrive(bar(BAR_GA));
+          ptx::mbar_arrive(bar(BAR_GB));
+          ptx::mbar_arrive(bar(BAR_G4));
+          ptx::mbar_arrive(bar(BAR_G5));
+        }
+        // the tiles of this chunk are dead: the next chunk's w, k, q, v can land now
+        if (tid == kIssuer && has_next && !*sAbort) {
+          issue_tma_w(h, t0 + C);
+          issue_tma_a(h, t0 + C);
+        }
+        serial_chunk<kScalarDecay, kScalarGates, kP3, kProlog, Tout>(p, gb, tmS + lane_base + cg * 32,
+                                                                   ci > 0 ? sDLb(par ^ 1u) + cg * 32 : nullptr,
+                                                                   t0, nvalid, h);
+        if (tid < D) sDLb(par)[tid] = 1.f;  // the next chunk reads the state with tau = 1
+        // the staging covered the bf16 T tile, whose blocks above the diagonal the solve never
+        // writes: zero it again
+        sts_v4(sb + OFF_T + 16u * (uint32_t)tid, make_uint4(0u, 0u, 0u, 0u));
+        // the next chunk's operands, as the factored path builds them under its GEMMs
+        if (has_next) {
+          if (!kScalarDecay) waitb(bar(BAR_TMA_L), par ^ 1u);
+          wide_next = elem_cumsum(par ^ 1u, t0 + C, nvalid_next, h, L);
+          if (tid == kIssuer && !*sAbort) issue_tma_x(h, t0 + C);
+          waitb(bar(BAR_TMA_A), par ^ 1u);
+          if (!kScalarGates) waitb(bar(BAR_TMA_W), par ^ 1u);
+          elem_scale(t0 + C, nvalid_next, h, L, ke2);
+          if (!kScalarGates) waitb(bar(BAR_TMA_X), par ^ 1u);
+          elem_x(t0 + C, nvalid_next, h, ke2);
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncthreads();
+        if (*sAbort) break;
+        continue;
+      }
 
       // ---- a4: G1 [A B; QX QP] = [k_r; q_r] [x_r; p_r]^T, issued first: it needs only this
       //      chunk's operands (built during the previous chunk) and runs under the S_r build
@@ -515,7 +786,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         const float *smv = sSM + cg * 32;
         uint32_t r[32], hb[16];
         if (ci > 0) {  // the previous chunk's increment GEMMs have landed in the state
-          wait_bar(bar(BAR_G5), par ^ 1u, sAbort, p.status);
+          waitb(bar(BAR_G5), par ^ 1u);
           ptx::tc_fence_after();
         }
         ptx::tmem_ld32(tmS + lane_base + cg * 32, r);
@@ -543,7 +814,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       __syncthreads();
 
 
-      wait_bar(bar(BAR_G1), par, sAbort, p.status);
+      waitb(bar(BAR_G1), par);
       ptx::tc_fence_after();
 
       // masks: A, B strictly lower (fp32 A for the solve, bf16 B); QX, QP lower incl. diagonal.
@@ -619,11 +890,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                               ptx::sdesc_sw128(sb + OFF_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), idT, 1);
           ptx::umma_commit(bar(BAR_GA));
           if (has_next) {  // p_r is dead once dS = p_r^T V is done: the next chunk's w can land
-            wait_bar(bar(BAR_E1), par, sAbort, p.status);
+            waitb(bar(BAR_E1), par);
             if (!*sAbort) issue_tma_w(h, t0 + C);
             // k_r, q_r and V are dead once GA is done: the next chunk's k, q, v tiles can land
             // (the solve runs meanwhile, so this wait delays nobody)
-            wait_bar(bar(BAR_GA), par, sAbort, p.status);
+            waitb(bar(BAR_GA), par);
             if (!*sAbort) issue_tma_a(h, t0 + C);
           }
         }
@@ -762,7 +1033,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       __syncthreads();
 
       // ---- R^T (fp32, D1 cols 0-63) -> bf16 TMEM A operand
-      wait_bar(bar(BAR_GA), par, sAbort, p.status);
+      waitb(bar(BAR_GA), par);
       ptx::tc_fence_after();
       {
         uint32_t r[16], hb[8];
@@ -788,11 +1059,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       // ---- while M^T is computed: the next chunk's cumulative decay (its log_a tile landed
       //      during the solve); then its b tile may take the log_a slot
       if (has_next) {
-        if (!kScalarDecay) wait_bar(bar(BAR_TMA_L), par ^ 1u, sAbort, p.status);
-        elem_cumsum(par ^ 1u, t0 + C, nvalid_next, h, L);
+        if (!kScalarDecay) waitb(bar(BAR_TMA_L), par ^ 1u);
+        wide_next = elem_cumsum(par ^ 1u, t0 + C, nvalid_next, h, L);
         if (tid == kIssuer && !*sAbort) issue_tma_x(h, t0 + C);
       }
-      wait_bar(bar(BAR_GB), par, sAbort, p.status);
+      waitb(bar(BAR_GB), par);
       ptx::tc_fence_after();
       {  // -M^T -> bf16 TMEM A operand
         uint32_t r[16], hb[8];
@@ -825,11 +1096,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       // ---- while O^T and dS are finished: the next chunk's k_r, q_r, p_r (its k, q, v tiles
       //      landed during the solve, its w tile once dS = p_r^T V was done)
       if (has_next) {
-        wait_bar(bar(BAR_TMA_A), par ^ 1u, sAbort, p.status);
-        if (!kScalarGates) wait_bar(bar(BAR_TMA_W), par ^ 1u, sAbort, p.status);
+        waitb(bar(BAR_TMA_A), par ^ 1u);
+        if (!kScalarGates) waitb(bar(BAR_TMA_W), par ^ 1u);
         elem_scale(t0 + C, nvalid_next, h, L, ke2);
       }
-      wait_bar(bar(BAR_G4), par, sAbort, p.status);
+      waitb(bar(BAR_G4), par);
       ptx::tc_fence_after();
 
       // ---- a8: outputs (the state was updated by the increment GEMMs)
@@ -854,8 +1125,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       }
       // ---- the next chunk's x_r, once dS (the last reader of this chunk's x_r) is done
       if (has_next) {
-        wait_bar(bar(BAR_G5), par, sAbort, p.status);
-        if (!kScalarGates) wait_bar(bar(BAR_TMA_X), par ^ 1u, sAbort, p.status);
+        waitb(bar(BAR_G5), par);
+        if (!kScalarGates) waitb(bar(BAR_TMA_X), par ^ 1u);
         elem_x(t0 + C, nvalid_next, h, ke2);
       }
       // one proxy fence per thread covers the o staging (read by the TMA store below) and the
@@ -891,7 +1162,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     //      [32 cg, 32 cg + 32); each store instruction of a warp writes 32 consecutive dv entries).
     //      The last chunk's increment GEMMs must have landed (also before the next unit's S0).
     if (nchunks > 0) {
-      wait_bar(bar(BAR_G5), (it & 1u) ^ 1u, sAbort, p.status);
+      waitb(bar(BAR_G5), (it & 1u) ^ 1u);
       ptx::tc_fence_after();
     }
     if (p.S_T && !*sAbort) {
@@ -908,6 +1179,22 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   }
 
   if (tid == kIssuer) ptx::bulk_wait_group0();
+  if (*sAbort) {
+    // wind-down after a timed-out wait (every wait of the loop then returned at once): let the
+    // MMAs of the two issuing threads and the last armed phase of every TMA barrier finish,
+    // each within the wait limit, before the tensor memory is freed and the CTA leaves
+    if (tid == 0) {
+      ptx::umma_commit(bar(BAR_DRAIN0));
+      drain_bar(bar(BAR_DRAIN0), 0u, P.wait_ns);
+#pragma unroll
+      for (int b = BAR_TMA_A; b <= BAR_TMA_X; ++b)
+        if (sIss[b] > 0u) drain_bar(bar(b), (sIss[b] - 1u) & 1u, P.wait_ns);
+    }
+    if (warp == kIssueWarp && lane == 0) {
+      ptx::umma_commit(bar(BAR_DRAIN1));
+      drain_bar(bar(BAR_DRAIN1), 0u, P.wait_ns);
+    }
+  }
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -1004,6 +1291,7 @@ cudaError_t launch_chunk_tc(const ChunkProblem &p, cudaStream_t stream, const ch
   P.p = p;
   P.n_units = p.n_seqs * p.n_heads;
   P.counter = p.status + 1;
+  P.wait_ns = kWaitTimeoutNs;
   if (P.n_units == 0) return cudaSuccess;
   const int64_t T = p.t_total > 0 ? p.t_total : 1;
   bool ok = make_map(&P.tm_q, p.q, T, p.n_heads) && make_map(&P.tm_k, p.k, T, p.n_heads) &&
@@ -1025,6 +1313,11 @@ cudaError_t launch_chunk_tc(const ChunkProblem &p, cudaStream_t stream, const ch
   const int grid = P.n_units < sms ? P.n_units : sms;
   const bool obf = p.dtype_out == GDN2_BF16;
   const bool pr = (p.flags & GDN2_FUSED_PROLOGUE) != 0;
+  uint64_t hook_ns = 0;
+  if (take_debug_timeout(GDN2_DEBUG_CHUNK, &hook_ns)) {  // the timeout test hook, armed for this launch
+    P.dbg_skip = 1;
+    P.wait_ns = hook_ns;
+  }
   // x_r == p_r in the gist.science form, and in the default form when w is b
   if (p3)
     return pr ? launch_gates<true, true, true>(P, grid, stream, sd, sg, obf)

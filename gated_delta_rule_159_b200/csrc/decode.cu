@@ -192,12 +192,15 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeProblem p) {
 }
 
 // ---------------------------------------------------------------------------
-// Streaming variant for d_k = d_v = 128 with channel-wise gates: one persistent
-// CTA per SM walks its units in order.  The state (64 KiB) and the six input
-// vectors of a unit arrive by bulk copy into one of kStages shared-memory
-// buffers, issued two units ahead; the update runs out of shared memory and the
-// new state leaves by a bulk store, so every SM keeps loads and a store in
-// flight while it computes.  Same arithmetic as decode_kernel.
+// Streaming variant for d_k = d_v = 128: one persistent CTA per SM walks its
+// units in order.  The state (64 KiB) and the per-channel input vectors of a
+// unit arrive by bulk copy into one of kStages shared-memory buffers, issued
+// two units ahead; the update runs out of shared memory and the new state
+// leaves by a bulk store, so every SM keeps loads and a store in flight while
+// it computes.  Scalar decay / scalar gates ([N, H] arrays) are read with plain
+// loads instead of bulk copies.  With a state-slot index (continuous batching)
+// a unit reads and writes its pool slot; a padding row loads no state.  Same
+// arithmetic as decode_kernel.
 constexpr int kStages = 3;
 constexpr int kSThreads = 256;
 constexpr uint64_t kStreamWaitNs = 1000000000ull;  // bounded waits: 1 s
@@ -212,12 +215,12 @@ struct StreamSmem {
   unsigned long long full[kStages];
 };
 
-__device__ __forceinline__ bool stream_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool stream_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   uint32_t n = 0;
   while (!ptx::mbar_try_wait(bar, parity)) {
-    if ((++n & 255u) == 0 && global_timer_ns() - t0 > kStreamWaitNs) return false;
+    if ((++n & 255u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
   }
   return true;
 }
@@ -233,9 +236,13 @@ __global__ void __launch_bounds__(kSThreads, 1) decode_stream_kernel(DecodeProbl
   const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
   const bool p3 = kExt && (p.flags & GDN2_GATE_FORM_P3) != 0;
   const bool prolog = kExt && (p.flags & GDN2_FUSED_PROLOGUE) != 0;
+  const bool sdecay = (p.flags & GDN2_SCALAR_DECAY) != 0;
+  const bool sgates = (p.flags & GDN2_SCALAR_GATES) != 0;
   const Tin *src[6] = {static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k), static_cast<const Tin *>(p.v),
                        static_cast<const Tin *>(p.log_a), static_cast<const Tin *>(p.b),
                        static_cast<const Tin *>(tied ? p.b : p.w)};
+  // vectors that arrive by bulk copy: q, k, v always; log_a, b, w unless they are scalars
+  const uint32_t nvec = 3u + (sdecay ? 0u : 1u) + (sgates ? 0u : 2u);
   auto bar = [&](int st) { return ptx::smem_u32(&sm.full[st]); };
   // state of a unit: its own (n * H + h), or slot state_idx[n] of the pool; -1 for a padding row
   auto state_of = [&](int unit) -> long long {
@@ -244,12 +251,19 @@ __global__ void __launch_bounds__(kSThreads, 1) decode_stream_kernel(DecodeProbl
     if (slot < 0 || slot >= p.n_slots) return -1;
     return (long long)slot * p.n_heads + unit % p.n_heads;
   };
+  bool dbg_armed = p.dbg_skip != 0 && blockIdx.x == 0;  // the timeout test hook
   auto issue = [&](int unit, int st) {  // thread 0; a padding row loads its input vectors only
     const long long su = state_of(unit);
-    ptx::mbar_arrive_expect_tx(bar(st), (su >= 0 ? kState : 0u) + 6u * kVec);
+    ptx::mbar_arrive_expect_tx(bar(st), (su >= 0 ? kState : 0u) + nvec * kVec);
+    if (dbg_armed) {  // bytes announced, no copy issued: the wait for this stage runs out
+      dbg_armed = false;
+      return;
+    }
     if (su >= 0) ptx::bulk_load(ptx::smem_u32(sm.S[st]), p.S + (size_t)su * 128 * 128, kState, bar(st));
 #pragma unroll
-    for (int j = 0; j < 6; ++j) ptx::bulk_load(ptx::smem_u32(sm.vec[st][j]), src[j] + (size_t)unit * 128, kVec, bar(st));
+    for (int j = 0; j < 6; ++j)
+      if (j < 3 || (j == 3 ? !sdecay : !sgates))
+        ptx::bulk_load(ptx::smem_u32(sm.vec[st][j]), src[j] + (size_t)unit * 128, kVec, bar(st));
   };
   if (t == 0) {
 #pragma unroll
@@ -265,13 +279,14 @@ __global__ void __launch_bounds__(kSThreads, 1) decode_stream_kernel(DecodeProbl
   int it = 0;
   for (int unit = first; unit < units; unit += stride, ++it) {
     const int st = it % kStages;
-    const bool ok = stream_wait(bar(st), (uint32_t)(it / kStages) & 1u);
+    const bool ok = stream_wait(bar(st), (uint32_t)(it / kStages) & 1u, p.wait_ns);
     if (__syncthreads_or(!ok)) {
       // give up: record it, let the loads already issued land (bounded), then leave
       if (t == 0) {
         atomicExch(&g_decode_status, kStatusTimeout);
-        stream_wait(bar(st), (uint32_t)(it / kStages) & 1u);
-        if (unit + stride < units) stream_wait(bar((it + 1) % kStages), (uint32_t)((it + 1) / kStages) & 1u);
+        stream_wait(bar(st), (uint32_t)(it / kStages) & 1u, p.wait_ns);
+        if (unit + stride < units)
+          stream_wait(bar((it + 1) % kStages), (uint32_t)((it + 1) / kStages) & 1u, p.wait_ns);
       }
       break;
     }
@@ -293,7 +308,8 @@ __global__ void __launch_bounds__(kSThreads, 1) decode_stream_kernel(DecodeProbl
     const Tin *vg = sm.vec[st][3], *vb = sm.vec[st][4], *vw = sm.vec[st][5];
     if (t < 128) {
       const float kk = to_f32(vk[t]);
-      float g = to_f32(vg[t]), bb = to_f32(vb[t]), ww = to_f32(vw[t]);
+      float g = to_f32(sdecay ? src[3][unit] : vg[t]);
+      float bb = to_f32(sgates ? src[4][unit] : vb[t]), ww = to_f32(sgates ? src[5][unit] : vw[t]);
       if (prolog) {
         g = log_sigmoid_f(g);
         bb = sigmoid_f(bb);
@@ -429,9 +445,16 @@ cudaError_t launch_dv(const DecodeProblem &p, cudaStream_t stream) {
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream) {
-  const bool channel_gates = (p.flags & (GDN2_SCALAR_DECAY | GDN2_SCALAR_GATES)) == 0;
-  if (p.d_k == 128 && p.d_v == 128 && channel_gates && p.n_seqs * p.n_heads > 0) {
+cudaError_t launch_decode(const DecodeProblem &p_in, cudaStream_t stream) {
+  DecodeProblem p = p_in;
+  p.wait_ns = kStreamWaitNs;
+  p.dbg_skip = 0;
+  if (p.d_k == 128 && p.d_v == 128 && p.n_seqs * p.n_heads > 0) {
+    uint64_t hook_ns = 0;
+    if (take_debug_timeout(GDN2_DEBUG_DECODE, &hook_ns)) {  // the timeout test hook, armed for this launch
+      p.dbg_skip = 1;
+      p.wait_ns = hook_ns;
+    }
     const bool in_bf = p.dtype_in == GDN2_BF16, out_bf = p.dtype_out == GDN2_BF16;
     if ((p.flags & (GDN2_GATE_FORM_P3 | GDN2_FUSED_PROLOGUE)) != 0) {
       if (in_bf && out_bf) return launch_stream_t<true, __nv_bfloat16, __nv_bfloat16>(p, stream);

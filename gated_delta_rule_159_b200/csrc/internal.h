@@ -35,6 +35,8 @@ struct DecodeProblem {
   uint32_t flags;
   const int32_t *state_idx;  // NULL: sequence n owns state n; else slot state_idx[n] of S
   int n_slots;               // slots in S when state_idx is set
+  uint64_t wait_ns;          // limit of the streaming kernel's bounded waits (set by launch_decode)
+  int dbg_skip;              // timeout test hook: CTA 0 arms its first load group without issuing it
 };
 
 struct BwdProblem {
@@ -93,6 +95,11 @@ cudaError_t launch_prefix(const float *F, const float *G, size_t seg_stride, siz
 
 // Record `message` as this thread's gdn2_last_error() text and return `code`.
 int set_last_error(int code, const char *message);
+
+// The one-shot timeout test hook (gdn2_debug_timeout_once): true, with the armed wait limit,
+// when the next launch of the kernel at `site` (GDN2_DEBUG_CHUNK / GDN2_DEBUG_DECODE) is to
+// run it; the hook is then disarmed.
+bool take_debug_timeout(int site, uint64_t *wait_ns);
 
 cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream);
 // Synchronise `stream`, read and clear the decode status word; returns a cudaError_t value.

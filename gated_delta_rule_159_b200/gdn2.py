@@ -36,7 +36,10 @@ EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_workspace_size", "gdn2_check_statu
             "gdn2_bwd_workspace_size", "gdn2_chunk_fwd_split", "gdn2_chunk_fwd_split_workspace_size",
             "gdn2_segment_maps", "gdn2_segment_maps_workspace_size", "gdn2_affine_prefix",
             "gdn2_segment_correct", "gdn2_segment_correct_workspace_size",
+            "gdn2_chunk_fwd_noalloc", "gdn2_chunk_fwd_noalloc_status", "gdn2_debug_timeout_once",
             "gdn2_last_error", "gdn2_version")
+DEBUG_CHUNK = 1
+DEBUG_DECODE = 2
 
 
 class Dims(ctypes.Structure):
@@ -84,6 +87,8 @@ def _load():
     lib.gdn2_segment_correct_workspace_size.argtypes = [ctypes.POINTER(Dims)]
     lib.gdn2_decode_status.restype = ctypes.c_int
     lib.gdn2_decode_status.argtypes = [vp]
+    lib.gdn2_debug_timeout_once.restype = ctypes.c_int
+    lib.gdn2_debug_timeout_once.argtypes = [ctypes.c_int32, ctypes.c_uint64]
     lib.gdn2_bwd.restype = ctypes.c_int
     lib.gdn2_bwd.argtypes = [vp] * 17 + [ctypes.POINTER(Dims), vp, sz, vp]
     lib.gdn2_bwd_workspace_size.restype = sz
@@ -207,6 +212,13 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Te
                             _ptr(workspace), workspace.numel(), _stream(dev))
     _check(rc)
     return o, S_T
+
+
+def debug_timeout_once(site: int, wait_ns: int) -> None:
+    """Test hook: the next launch of the kernel at ``site`` (DEBUG_CHUNK / DEBUG_DECODE) runs
+    its bounded waits with a ``wait_ns`` limit and lets one of them run out (see
+    ``gdn2_debug_timeout_once`` in include/gdn2.h).  Not for production use."""
+    _check(lib.gdn2_debug_timeout_once(int(site), int(wait_ns)))
 
 
 def decode_status(device=None) -> int:

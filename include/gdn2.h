@@ -41,9 +41,12 @@
  *  - Values are not validated.  Preconditions: finite inputs; log_a <= 0 (the
  *    decay is bounded in (0, 1], cours.spawnkit.ai session 16 "Stability");
  *    b, w in [0, 1]; q and k L2-normalised by the caller (no 1/sqrt(d_k) scale
- *    is applied).  The chunked path also needs, per channel, the summed decay
- *    over each half chunk to stay above -80 (sum of log_a over 32 consecutive
- *    tokens of a chunk >= -80), which keeps its fp32/bf16 decay factors finite.
+ *    is applied).  Any finite log_a <= 0 is in range: the tensor-core chunked
+ *    path factors each chunk's decay around a per-channel reference when every
+ *    channel decays by at most 128 nats over the chunk, and runs a chunk with a
+ *    wider decay range token by token (neelmishra.github.io, "What makes the
+ *    architecture more than a recurrence": chunk sizes and intermediate
+ *    numerical ranges).
  */
 #ifndef GDN2_H
 #define GDN2_H
@@ -82,8 +85,7 @@ enum gdn2_flags {
                               mixer's activations (neelmishra.github.io, "What makes the architecture
                               more than a recurrence" and "Read the limiting cases"):
                               q <- q / sqrt(|q|^2 + 1e-6), k likewise (over d_k);
-                              log_a <- log sigmoid(log_a); b <- sigmoid(b); w <- sigmoid(w).
-                              The range precondition on log_a applies to the activated values. */
+                              log_a <- log sigmoid(log_a); b <- sigmoid(b); w <- sigmoid(w). */
 };
 
 /*
@@ -360,6 +362,28 @@ int gdn2_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
  * gdn2_chunk_fwd_noalloc clears the word, so read it before that call.
  */
 int gdn2_chunk_fwd_noalloc_status(gdn2_stream_t stream);
+
+/*
+ * gdn2_debug_timeout_once -- test hook for the failure detection of the bounded
+ * device-side waits; not for production use.  It arms a one-shot fault for the
+ * next launch of the kernel named by `site`:
+ *   GDN2_DEBUG_CHUNK   the tensor-core chunk kernel (gdn2_chunk_fwd and the calls
+ *                      built on it),
+ *   GDN2_DEBUG_DECODE  the streaming decode kernel (d_k = d_v = 128).
+ * In that launch every bounded wait uses the limit `wait_ns` instead of 1 s, and
+ * the first CTA announces the bytes of its first load group to its mbarrier but
+ * issues none of the copies, so its wait runs out: the kernel records
+ * GDN2_ERR_TIMEOUT in its status word (read by gdn2_check_status /
+ * gdn2_decode_status), lets the copies and MMAs it did issue finish (each wait
+ * bounded by the same limit), frees its tensor memory and returns.  No copy is
+ * left in flight, no address is faulted, and the outputs of that launch are
+ * undefined.  The hook is per process and consumed by the first matching
+ * launch; the pages have no counterpart (failure detection is this library's).
+ * Errors: GDN2_ERR_INVALID_ARG for an unknown site or wait_ns outside
+ * [1000, 10^10].
+ */
+enum gdn2_debug_site { GDN2_DEBUG_CHUNK = 1, GDN2_DEBUG_DECODE = 2 };
+int gdn2_debug_timeout_once(int32_t site, uint64_t wait_ns);
 
 /* Thread-local description of the last non-zero status on this thread ("" if none). */
 const char *gdn2_last_error(void);

@@ -295,7 +295,7 @@ def test_tc_degenerate_cases(dev, case):
         inp["w"] = torch.zeros_like(inp["w"])
     elif case == "zero_key":
         inp["k"] = torch.zeros_like(inp["k"])
-    elif case == "strong_decay":      # -2.4 per step: half a chunk sums to -76.8 (precondition >= -80)
+    elif case == "strong_decay":      # -2.4 per step: a 151-nat range per chunk, run token by token
         inp["log_a"] = torch.full_like(inp["log_a"], -2.4)
     elif case == "no_decay_no_gates":  # alpha = 1, b = w = 0: the state holds
         inp["log_a"] = torch.zeros_like(inp["log_a"])
