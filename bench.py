@@ -564,13 +564,55 @@ def main():
             raise RuntimeError("decode kernel reported a timed-out wait")
         step_bytes = 2 * Nd * Hd * d * d * 4 + 6 * Nd * Hd * d * 2 + Nd * Hd * d * 4
         gbs = step_bytes * steps / (dms / 1e3) / 1e9
+
+        def decode_variant(fn, reps, vec_bytes):
+            """Plain launch loop of `reps` steps of fn(t); returns (us per step, HBM fraction)."""
+            for t in range(3):
+                fn(t)
+            barrier()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for t in range(reps):
+                fn(t)
+            a1.record(stream)
+            barrier()
+            ms = rmax(a0.elapsed_time(a1))
+            vb = 2 * Nd * Hd * d * d * 4 + vec_bytes + Nd * Hd * d * 4
+            return 1e3 * ms / reps, vb * reps / (ms / 1e3) / 1e9 / hbm_peak
+
+        # continuous batching: the same 256 x 16 rows read and update slots of a pool of 512
+        # sequences' states through a shuffled slot index
+        reps_v = min(steps, 256)
+        pool = torch.zeros(2 * Nd, Hd, d, d, dtype=torch.float32, device=dev)
+        gperm = torch.Generator(device="cpu")
+        gperm.manual_seed(700 + rank)
+        slots = torch.randperm(2 * Nd, generator=gperm)[:Nd].to(torch.int32).to(dev)
+        pool[slots.long()] = S
+        idx_us, idx_frac = decode_variant(
+            lambda t: gdn2.decode_step_indexed(*(di[n][t] for n in names), pool, slots, o=od), reps_v,
+            6 * Nd * Hd * d * 2)
+        del pool
+        # the scalar-gate Gated DeltaNet decode (one alpha and one beta per row, b = w = beta)
+        sc_la = di["log_a"][:, :, :, 0].contiguous()
+        sc_b = di["b"][:, :, :, 0].contiguous()
+        sc_us, sc_frac = decode_variant(
+            lambda t: gdn2.decode_step(di["q"][t], di["k"][t], di["v"][t], sc_la[t], sc_b[t], None, S, o=od,
+                                       scalar_decay=True, scalar_gates=True, tied_gates=True), reps_v,
+            3 * Nd * Hd * d * 2 + 2 * Nd * Hd * 2)
+        del sc_la, sc_b
         decode = {"value": Nd * world * steps / (dms / 1e3), "unit": "tokens/s", "steps": steps,
                   "us_per_step": 1e3 * dms / steps, "bytes_per_step": step_bytes, "hbm_gbs": gbs,
                   "hbm_frac": gbs / hbm_peak, "peak_source": peak_src, "sequences": Nd, "heads": Hd,
                   "state_bytes": Nd * Hd * d * d * 4, "clocks": dclocks, "kernel": "decode_stream_kernel",
                   "launch": "CUDA graph of all steps, replayed once",
                   "plain_loop_us_per_step": 1e3 * plain_ms / steps,
-                  "gpu_launches": steps}
+                  "gpu_launches": steps,
+                  "indexed": {"us_per_step": idx_us, "hbm_frac": idx_frac, "steps": reps_v,
+                              "rows": f"{Nd} x {Hd} rows into a pool of {2 * Nd} x {Hd} states, shuffled slots",
+                              "kernel": "decode_stream_kernel", "launch": "plain loop"},
+                  "scalar_gates": {"us_per_step": sc_us, "hbm_frac": sc_frac, "steps": reps_v,
+                                   "gates": "scalar alpha and tied scalar beta per row",
+                                   "kernel": "decode_stream_kernel", "launch": "plain loop"}}
         del di, S
 
     # ---------------- backward (gradients of the prefill step)

@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <vector>
 
 #include "internal.h"
 
@@ -125,7 +126,7 @@ size_t gdn2_chunk_fwd_workspace_size(const gdn2_dims *dims) {
 static int chunk_fwd_impl(const void *q, const void *k, const void *v, const void *log_a, const void *b,
                           const void *w, const float *S0, const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
                           void *o, float *S_T, const gdn2_dims *dims, void *workspace, size_t workspace_bytes,
-                          gdn2_stream_t stream, bool reset_status);
+                          gdn2_stream_t stream, bool reset_status, const int32_t *seg_bounds = nullptr);
 
 int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *log_a, const void *b, const void *w,
                    const float *S0, const int32_t *cu_seqlens, const int32_t *cu_seqlens_host, void *o, float *S_T,
@@ -134,10 +135,12 @@ int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *log_
                         workspace_bytes, stream, true);
 }
 
+// seg_bounds (internal): [2 * dims->n_seqs] device (first, end) token of every unit sequence,
+// which may leave gaps; dims->seq_len is then the packed token count the tensors span.
 static int chunk_fwd_impl(const void *q, const void *k, const void *v, const void *log_a, const void *b,
                           const void *w, const float *S0, const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
                           void *o, float *S_T, const gdn2_dims *dims, void *workspace, size_t workspace_bytes,
-                          gdn2_stream_t stream, bool reset_status) {
+                          gdn2_stream_t stream, bool reset_status, const int32_t *seg_bounds) {
   g_err[0] = '\0';
   int rc = check_dims(dims);
   if (rc) return rc;
@@ -152,7 +155,8 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const voi
   if (workspace_bytes < need)
     return fail(GDN2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
 
-  const int64_t t_total = cu_seqlens ? (int64_t)dims->seq_len : (int64_t)dims->n_seqs * dims->seq_len;
+  const int64_t t_total =
+      (cu_seqlens || seg_bounds) ? (int64_t)dims->seq_len : (int64_t)dims->n_seqs * dims->seq_len;
   if (cu_seqlens_host) {
     if (!cu_seqlens) return fail(GDN2_ERR_INVALID_ARG, "cu_seqlens_host given without cu_seqlens");
     if (cu_seqlens_host[0] != 0 || cu_seqlens_host[dims->n_seqs] != t_total)
@@ -172,11 +176,13 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const voi
   p.t_total = t_total;
   p.status = static_cast<int32_t *>(workspace);
   p.schedule = nullptr;
+  p.seg_bounds = seg_bounds;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool tc = dims->d_k == 128 && dims->d_v == 128 && dims->chunk == 64 && dims->dtype_in == GDN2_BF16;
   const bool simt = dims->d_k <= 64 && dims->d_v <= 64 &&
                     (dims->chunk == 16 || dims->chunk == 32 || dims->chunk == 64);
+  if (seg_bounds && !tc) return fail(GDN2_ERR_UNSUPPORTED, "segment bounds need the tensor-core path");
   if (!tc && !simt)
     return fail(GDN2_ERR_UNSUPPORTED,
                 "no kernel for d_k=%d d_v=%d chunk=%d dtype_in=%d (supported: 128/128/64 bf16, or d<=64 with chunk "
@@ -357,13 +363,196 @@ int gdn2_chunk_fwd_split(const void *q, const void *k, const void *v, const void
   return GDN2_OK;
 }
 
+static size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+// ---------------------------------------------------------------- packed varlen split
+// Plan of gdn2_chunk_fwd_split_varlen from the host copy of cu_seqlens.  tau = the balanced
+// share of 64-token chunks per SM; a sequence of more than 3 tau chunks is cut into segments of
+// about tau chunks (whole chunks), raised until all segment units fit in the SMs when that is
+// possible.  Passes (one chunk-kernel launch each): 2 = segments of split sequences from the
+// identity (their E = F + G); 1 = every segment from 0 (unsplit sequences from S0): G and the
+// provisional o; combine; 3 = split segments that start from a non-zero state, re-run from it:
+// the final o.
+struct VarlenPlan {
+  int N = 0, H = 0, NS = 0, N2 = 0, N3 = 0;
+  bool any_split = false;
+  std::vector<int32_t> ints;  // cu1 [NS + 1] | src1 [NS] | src2 [N2] | b2 [2 N2] | b3 [2 N3] | info [4 N]
+  size_t i_cu1 = 0, i_src1 = 0, i_src2 = 0, i_b2 = 0, i_b3 = 0, i_info = 0;
+  size_t off_ints = 0, off_G = 0, off_E = 0, off_S3 = 0, total = 0, inner = 0;
+};
+
+static VarlenPlan varlen_plan(const gdn2_dims *d, const int32_t *cu, int n_sm, bool has_S0) {
+  VarlenPlan P;
+  const int N = d->n_seqs, H = d->n_heads;
+  P.N = N;
+  P.H = H;
+  std::vector<int64_t> chunks(N);
+  int64_t total = 0, cmax = 0;
+  for (int n = 0; n < N; ++n) {
+    chunks[n] = ((int64_t)cu[n + 1] - cu[n] + 63) / 64;
+    total += chunks[n];
+    cmax = chunks[n] > cmax ? chunks[n] : cmax;
+  }
+  int64_t tau = (total * H + n_sm - 1) / (n_sm > 0 ? n_sm : 1);
+  if (tau < 1) tau = 1;
+  std::vector<int> m(N, 1);
+  for (int iter = 0; iter < 16; ++iter) {
+    int64_t units = 0;
+    for (int n = 0; n < N; ++n) {
+      m[n] = chunks[n] > 3 * tau ? (int)((chunks[n] + tau - 1) / tau) : 1;
+      units += (int64_t)m[n] * H;
+    }
+    if (units <= n_sm || 3 * tau >= cmax) break;
+    tau = (tau * units + n_sm - 1) / n_sm;  // fewer, longer segments
+  }
+  std::vector<int32_t> cu1{0}, src1, src2, b2, b3, info;
+  for (int n = 0; n < N; ++n) {
+    const int32_t bos = cu[n], eos = cu[n + 1];
+    const int first1 = (int)src1.size(), first2 = (int)src2.size(), first3 = (int)b3.size() / 2;
+    int segs = 1;
+    if (m[n] > 1) {
+      const int64_t per = (chunks[n] + m[n] - 1) / m[n];  // chunks per segment
+      segs = 0;
+      for (int64_t a = bos; a < eos; a += per * 64) {
+        const int32_t e = (int32_t)(a + per * 64 < eos ? a + per * 64 : eos);
+        cu1.push_back(e);
+        src1.push_back(-1);  // from 0
+        src2.push_back(-2);  // from the identity
+        b2.push_back((int32_t)a);
+        b2.push_back(e);
+        if (segs > 0 || has_S0) {
+          b3.push_back((int32_t)a);
+          b3.push_back(e);
+        }
+        ++segs;
+      }
+      P.any_split = true;
+    } else {
+      cu1.push_back(eos);
+      src1.push_back(has_S0 ? n : -1);
+    }
+    info.push_back(segs);
+    info.push_back(first1);
+    info.push_back(first2);
+    info.push_back(first3);
+  }
+  P.NS = (int)src1.size();
+  P.N2 = (int)src2.size();
+  P.N3 = (int)b3.size() / 2;
+  auto put = [&](const std::vector<int32_t> &v) {
+    const size_t at = P.ints.size();
+    P.ints.insert(P.ints.end(), v.begin(), v.end());
+    return at;
+  };
+  P.i_cu1 = put(cu1);
+  P.i_src1 = put(src1);
+  P.i_src2 = put(src2);
+  P.i_b2 = put(b2);
+  P.i_b3 = put(b3);
+  P.i_info = put(info);
+  // workspace: the passes' own workspace (sized for the largest pass) | plan | G | E | starts3
+  gdn2_dims inner = *d;
+  inner.n_seqs = P.NS > 0 ? P.NS : 1;
+  const size_t state = (size_t)H * 128 * 128 * sizeof(float);
+  P.inner = up256(gdn2_chunk_fwd_workspace_size(&inner));
+  P.off_ints = P.inner;
+  P.off_G = P.off_ints + up256(P.ints.size() * sizeof(int32_t));
+  P.off_E = P.off_G + up256((size_t)P.NS * state);
+  P.off_S3 = P.off_E + up256((size_t)P.N2 * state);
+  P.total = P.off_S3 + up256((size_t)P.N3 * state);
+  return P;
+}
+
+static int sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 148;
+  return sms;
+}
+
+static int check_varlen_cu(const gdn2_dims *dims, const int32_t *cu_host) {
+  if (!cu_host) return fail(GDN2_ERR_INVALID_ARG, "cu_seqlens_host is required (the plan is made on the host)");
+  if (cu_host[0] != 0 || cu_host[dims->n_seqs] != dims->seq_len)
+    return fail(GDN2_ERR_INVALID_ARG, "cu_seqlens_host must start at 0 and end at seq_len (= T_tot)");
+  for (int n = 0; n < dims->n_seqs; ++n)
+    if (cu_host[n + 1] < cu_host[n]) return fail(GDN2_ERR_INVALID_ARG, "cu_seqlens_host is not non-decreasing at %d", n);
+  return GDN2_OK;
+}
+
+size_t gdn2_chunk_fwd_split_varlen_workspace_size(const gdn2_dims *dims, const int32_t *cu_seqlens_host) {
+  if (!dims || dims->n_seqs < 1 || dims->n_heads < 1 || dims->seq_len < 0 || !cu_seqlens_host) return 0;
+  if (cu_seqlens_host[0] != 0 || cu_seqlens_host[dims->n_seqs] != dims->seq_len) return 0;
+  for (int n = 0; n < dims->n_seqs; ++n)
+    if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return 0;
+  return varlen_plan(dims, cu_seqlens_host, sm_count(), true).total;  // S0 present: the larger plan
+}
+
+int gdn2_chunk_fwd_split_varlen(const void *q, const void *k, const void *v, const void *log_a, const void *b,
+                                const void *w, const float *S0, const int32_t *cu_seqlens,
+                                const int32_t *cu_seqlens_host, void *o, float *S_T, const gdn2_dims *dims,
+                                void *workspace, size_t workspace_bytes, gdn2_stream_t stream) {
+  g_err[0] = '\0';
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->d_k != 128 || dims->d_v != 128 || dims->chunk != 64 || dims->dtype_in != GDN2_BF16)
+    return fail(GDN2_ERR_UNSUPPORTED, "gdn2_chunk_fwd_split_varlen needs d_k = d_v = 128, chunk 64 and bf16 inputs");
+  if (!cu_seqlens) return fail(GDN2_ERR_INVALID_ARG, "cu_seqlens must be non-NULL");
+  rc = check_varlen_cu(dims, cu_seqlens_host);
+  if (rc) return rc;
+  rc = check_inputs(q, k, v, log_a, b, w, dims->flags, dims->dtype_in);
+  if (rc) return rc;
+  if (!o || !aligned16(o)) return fail(GDN2_ERR_INVALID_ARG, "o must be non-NULL and 16-byte aligned");
+  if ((S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)))
+    return fail(GDN2_ERR_INVALID_ARG, "S0 / S_T must be 16-byte aligned");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(GDN2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  const size_t need = gdn2_chunk_fwd_split_varlen_workspace_size(dims, cu_seqlens_host);
+  if (workspace_bytes < need)
+    return fail(GDN2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+  const VarlenPlan P = varlen_plan(dims, cu_seqlens_host, sm_count(), S0 != nullptr);
+  if (!P.any_split)  // nothing is long enough to split: the plain forward
+    return chunk_fwd_impl(q, k, v, log_a, b, w, S0, cu_seqlens, cu_seqlens_host, o, S_T, dims, workspace,
+                          P.inner, stream, true);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char *ws = static_cast<char *>(workspace);
+  int32_t *pi = reinterpret_cast<int32_t *>(ws + P.off_ints);
+  float *G = reinterpret_cast<float *>(ws + P.off_G);
+  float *E = reinterpret_cast<float *>(ws + P.off_E);
+  float *S3 = reinterpret_cast<float *>(ws + P.off_S3);
+  const int H = dims->n_heads;
+  cudaError_t e = gdn2::write_ints(pi, P.ints.data(), P.ints.size(), s);
+  if (e == cudaSuccess) e = gdn2::launch_fill_starts(E, pi + P.i_src2, nullptr, P.N2, H, s);
+  if (e == cudaSuccess) e = gdn2::launch_fill_starts(G, pi + P.i_src1, S0, P.NS, H, s);
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "varlen split setup: %s", cudaGetErrorString(e));
+  // pass 2: split segments from the identity (their o rows are rewritten by passes 1 and 3)
+  gdn2_dims d2 = *dims;
+  d2.n_seqs = P.N2;
+  rc = chunk_fwd_impl(q, k, v, log_a, b, w, E, nullptr, nullptr, o, E, &d2, ws, P.inner, stream, true,
+                      pi + P.i_b2);
+  if (rc) return rc;
+  // pass 1: every segment (split ones from 0, unsplit sequences from S0)
+  gdn2_dims d1 = *dims;
+  d1.n_seqs = P.NS;
+  std::vector<int32_t> cu1_host(P.ints.begin() + P.i_cu1, P.ints.begin() + P.i_cu1 + P.NS + 1);
+  rc = chunk_fwd_impl(q, k, v, log_a, b, w, G, pi + P.i_cu1, cu1_host.data(), o, G, &d1, ws, P.inner, stream,
+                      false);
+  if (rc) return rc;
+  e = gdn2::launch_combine_varlen(pi + P.i_info, E, G, S3, S0, S_T, dims->n_seqs, H, s);
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "varlen split combine: %s", cudaGetErrorString(e));
+  // pass 3: the split segments that start from a non-zero state, from that state: the final o
+  if (P.N3 == 0) return GDN2_OK;
+  gdn2_dims d3 = *dims;
+  d3.n_seqs = P.N3;
+  return chunk_fwd_impl(q, k, v, log_a, b, w, S3, nullptr, nullptr, o, nullptr, &d3, ws, P.inner, stream, false,
+                        pi + P.i_b3);
+}
+
 // ---------------------------------------------------------------- one segment per rank
 // Workspace of gdn2_segment_maps / gdn2_segment_correct: the inner forward's workspace, a zero
 // v, scratch outputs and (maps only) the identity start states.
 struct SegLayout {
   size_t off_zero_v, off_o2, off_ident, total;
 };
-static size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 static SegLayout seg_layout(const gdn2_dims *d, bool maps) {
   SegLayout L;
   const size_t tok = (size_t)d->n_seqs * (size_t)d->seq_len * (size_t)d->n_heads;

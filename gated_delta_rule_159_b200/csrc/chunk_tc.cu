@@ -92,6 +92,7 @@ constexpr uint32_t MISC_BAR = 10240;   // 12 mbarriers
 constexpr uint32_t MISC_TMEM = 10336;
 constexpr uint32_t MISC_ABORT = 10340;
 constexpr uint32_t MISC_UNIT = 10344;
+constexpr uint32_t MISC_WIDE = 10348;  // int: some channel of the chunk being prepared has a wide decay range
 constexpr uint32_t MISC_ISS = 10352;   // uint32[4]   phases armed per TMA barrier (A, L, W, X)
 constexpr uint32_t MISC_L0 = 10368;    // float[128]  L_0 (the chunk's first row)
 constexpr uint32_t MISC_BYTES = 10880;
@@ -403,6 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   float *part = reinterpret_cast<float *>(gb + OFF_MISC + MISC_PART);
   float *sRef = reinterpret_cast<float *>(gb + OFF_MISC + MISC_REF);
   float *sL0 = reinterpret_cast<float *>(gb + OFF_MISC + MISC_L0);
+  volatile int *sWide = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_WIDE);
   constexpr int kIssuer = 32;      // issues a unit's first TMA loads, the log_a and b loads and the o stores
   constexpr int kIssueWarp = 15;   // issues the T-independent MMAs during the solve
   constexpr int kSolveThreads = 480;  // warps 0-14
@@ -526,8 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     }
     *reinterpret_cast<float4 *>(part + warp * 128 + 4 * lane) = acc;
     if (warp == 0) *reinterpret_cast<float4 *>(sL0 + 4 * lane) = L[0];  // L_0 = log_a of row 0
+    if (tid == 0) *sWide = 0;
     __syncthreads();
-    int wide = 0;
     if (tid < D) {  // per channel: exclusive prefix over the 16 row groups, L_C = L_63, the reference
       float run = 0.f;
 #pragma unroll
@@ -538,12 +540,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       }
       const float l0 = sL0[tid];
       const float refv = 0.5f * (l0 + run);
-      wide = !(l0 - run <= kFastSpan);
+      if (!(l0 - run <= kFastSpan)) *sWide = 1;  // any writer sets it; nobody clears it before the barrier
       sRef[tid] = refv;
       sDLb(pn)[tid] = ptx::ex2((run - refv) * kLog2eF);
       sSM[tid] = ptx::ex2(refv * kLog2eF);
     }
-    return __syncthreads_or(wide);
+    __syncthreads();
+    return *sWide;
   };
   // pass 2 (needs the k, q, v tiles and the w tile): k_r, q_r and p_r in place; rows past the
   // chunk end are zeroed (v too).  ke2 keeps k e^{L_ref - L} for pass 3.
@@ -646,7 +649,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     const int unit = p.schedule ? p.schedule[u] : u;
     const int n = unit / H, h = unit % H;
     int64_t bos, len;
-    if (p.cu_seqlens) {
+    if (p.seg_bounds) {
+      bos = p.seg_bounds[2 * n];
+      len = (int64_t)p.seg_bounds[2 * n + 1] - bos;
+    } else if (p.cu_seqlens) {
       bos = p.cu_seqlens[n];
       len = (int64_t)p.cu_seqlens[n + 1] - bos;
     } else {

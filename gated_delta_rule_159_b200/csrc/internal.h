@@ -24,6 +24,10 @@ struct ChunkProblem {
   // Device workspace: status word + optional unit schedule.
   int32_t *status;          // one int32, zeroed by the launcher before the kernel runs
   const int32_t *schedule;  // [n_units] unit ids, longest first, or null (identity order)
+  // Optional [2 * n_seqs] device array of (first token, end token) per sequence; when set it
+  // replaces cu_seqlens for the unit bounds, so the sequences may leave gaps between them
+  // (the split forward's passes over a subset of segments).  Tensor-core path only.
+  const int32_t *seg_bounds;
 };
 
 struct DecodeProblem {
@@ -89,6 +93,15 @@ cudaError_t launch_split_helpers(int what, const SplitArgs &a, cudaStream_t stre
 // Helpers of the per-rank segment calls: `units` 128 x 128 identities; o += o2 (n elements);
 // the start state of segment `upto` and the end state after n_segs segments (see prefix_kernel).
 cudaError_t launch_identities(float *dst, int units, cudaStream_t stream);
+// Packed varlen split helpers: host-planned int32 values to the device (kernel parameters,
+// no stream synchronisation); start states (src[u] = -2 identity, -1 zero, n >= 0 S0[n]);
+// the serial combine per (sequence, head) from seq_info[4 n] = {m, pass-1, pass-2, pass-3
+// index of its first segment}.
+cudaError_t write_ints(int32_t *dst, const int32_t *vals, size_t n, cudaStream_t stream);
+cudaError_t launch_fill_starts(float *dst, const int32_t *src, const float *S0, int units, int H,
+                               cudaStream_t stream);
+cudaError_t launch_combine_varlen(const int32_t *seq_info, const float *E, const float *G, float *starts3,
+                                  const float *S0, float *S_T, int N, int H, cudaStream_t stream);
 cudaError_t launch_add(void *o, const void *o2, size_t n, int dtype_out, cudaStream_t stream);
 cudaError_t launch_prefix(const float *F, const float *G, size_t seg_stride, size_t seq_stride, float *start,
                           float *S_T, int upto, int n_segs, int N, int H, cudaStream_t stream);

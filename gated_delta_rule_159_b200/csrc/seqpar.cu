@@ -23,6 +23,7 @@ namespace gdn2 {
 namespace {
 
 constexpr int kComb = 512;  // threads of the combine kernel: 4 per row, 32 columns each
+constexpr int kIntBlock = 960;  // int32 values per plan-upload launch (a 3.8 KB parameter block)
 
 // Segment boundaries of N sequences of T tokens cut every L tokens.
 __global__ void seg_bounds_kernel(int32_t *cu, int N, int T, int L, int ns) {
@@ -129,6 +130,78 @@ __global__ void __launch_bounds__(kComb) prefix_kernel(const float *F, const flo
   }
 }
 
+// ---- packed varlen split (gdn2_chunk_fwd_split_varlen)
+
+// A block of host-planned int32 values written to device memory by a launch parameter (no
+// host-side copy, no stream synchronisation).
+struct IntBlock {
+  int32_t n;
+  int32_t v[kIntBlock];
+};
+__global__ void write_ints_kernel(int32_t *dst, const __grid_constant__ IntBlock b) {
+  for (int i = threadIdx.x; i < b.n; i += blockDim.x) dst[i] = b.v[i];
+}
+
+// Start states, one CTA per (unit, head): src[unit] = -2 identity, -1 zeros, n >= 0 S0[n, h].
+__global__ void fill_starts_kernel(float *dst, const int32_t *src, const float *S0, int H) {
+  const int uh = blockIdx.x, u = uh / H, h = uh % H;
+  const int s = src[u];
+  float *d = dst + (size_t)uh * 128 * 128;
+  const float *from = (s >= 0 && S0) ? S0 + ((size_t)s * H + h) * 128 * 128 : nullptr;
+  for (int e = threadIdx.x; e < 128 * 128; e += blockDim.x)
+    d[e] = s == -2 ? ((e / 128 == e % 128) ? 1.f : 0.f) : (from ? from[e] : 0.f);
+}
+
+// Per (sequence, head), serial over its m segments (seq_info[n] = {m, first segment in the
+// pass-1 list, first in the pass-2 list, first in the pass-3 list}).  m == 1: the pass-1 end
+// state is S_T.  m > 1: with G_j the segment's end state from 0 (pass 1) and E_j from the
+// identity (pass 2), F_j = E_j - G_j; S <- F_j S + G_j from S = S0 (or 0), recording the start
+// of every segment that pass 3 re-runs (all of them with S0, else j >= 1).
+__global__ void __launch_bounds__(kComb) combine_varlen_kernel(const int32_t *seq_info, const float *E,
+                                                               const float *G, float *starts3, const float *S0,
+                                                               float *S_T, int H) {
+  extern __shared__ float Ss[];  // [128][128] current state
+  const int unit = blockIdx.x, n = unit / H, h = unit % H;
+  const int t = threadIdx.x, r = t >> 2, c0 = (t & 3) * 32;
+  const int m = seq_info[4 * n], g0 = seq_info[4 * n + 1], e0 = seq_info[4 * n + 2], c3 = seq_info[4 * n + 3];
+  auto mat = [&](const float *base, int idx) { return base + ((size_t)idx * H + h) * 128 * 128; };
+  auto mat_w = [&](float *base, int idx) { return base + ((size_t)idx * H + h) * 128 * 128; };
+  if (m == 1) {
+    if (S_T) {
+      float *d = S_T + (size_t)unit * 128 * 128;
+      for (int e = t; e < 128 * 128; e += kComb) d[e] = mat(G, g0)[e];
+    }
+    return;
+  }
+  const float *s0 = S0 ? S0 + (size_t)unit * 128 * 128 : nullptr;
+  for (int e = t; e < 128 * 128; e += kComb) Ss[e] = s0 ? s0[e] : 0.f;
+  __syncthreads();
+  int k3 = c3;
+  for (int j = 0; j < m; ++j) {
+    if (j > 0 || S0) {
+      float *d = mat_w(starts3, k3++);
+      for (int e = t; e < 128 * 128; e += kComb) d[e] = Ss[e];
+    }
+    const float *Er = mat(E, e0 + j) + (size_t)r * 128, *Gr = mat(G, g0 + j) + (size_t)r * 128;
+    float acc[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) acc[c] = Gr[c0 + c];
+    for (int kk = 0; kk < 128; ++kk) {
+      const float f = Er[kk] - Gr[kk];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) acc[c] += f * Ss[kk * 128 + c0 + c];
+    }
+    __syncthreads();  // everyone has read the old state
+#pragma unroll
+    for (int c = 0; c < 32; ++c) Ss[r * 128 + c0 + c] = acc[c];
+    __syncthreads();
+  }
+  if (S_T) {
+    float *d = S_T + (size_t)unit * 128 * 128;
+    for (int e = t; e < 128 * 128; e += kComb) d[e] = Ss[e];
+  }
+}
+
 template <typename T>
 __global__ void add_kernel(T *o, const T *d, size_t n) {
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
@@ -160,6 +233,34 @@ SplitPlan split_plan(int N, int T, int H, int n_split, int dtype_in, int dtype_o
   s.off_o2 = s.off_zero_v + up256(tok * in_e);
   s.total = s.off_o2 + up256(tok * out_e);
   return s;
+}
+
+cudaError_t write_ints(int32_t *dst, const int32_t *vals, size_t n, cudaStream_t stream) {
+  for (size_t i = 0; i < n; i += kIntBlock) {
+    IntBlock b;
+    b.n = (int32_t)(n - i < (size_t)kIntBlock ? n - i : (size_t)kIntBlock);
+    for (int j = 0; j < b.n; ++j) b.v[j] = vals[i + j];
+    write_ints_kernel<<<1, 256, 0, stream>>>(dst + i, b);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_fill_starts(float *dst, const int32_t *src, const float *S0, int units, int H,
+                               cudaStream_t stream) {
+  if (units == 0) return cudaSuccess;
+  fill_starts_kernel<<<units * H, 256, 0, stream>>>(dst, src, S0, H);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_varlen(const int32_t *seq_info, const float *E, const float *G, float *starts3,
+                                  const float *S0, float *S_T, int N, int H, cudaStream_t stream) {
+  const int smem = 128 * 128 * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(combine_varlen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  combine_varlen_kernel<<<N * H, kComb, smem, stream>>>(seq_info, E, G, starts3, S0, S_T, H);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_identities(float *dst, int units, cudaStream_t stream) {

@@ -36,6 +36,7 @@ EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_workspace_size", "gdn2_check_statu
             "gdn2_bwd_workspace_size", "gdn2_chunk_fwd_split", "gdn2_chunk_fwd_split_workspace_size",
             "gdn2_segment_maps", "gdn2_segment_maps_workspace_size", "gdn2_affine_prefix",
             "gdn2_segment_correct", "gdn2_segment_correct_workspace_size",
+            "gdn2_chunk_fwd_split_varlen", "gdn2_chunk_fwd_split_varlen_workspace_size",
             "gdn2_chunk_fwd_noalloc", "gdn2_chunk_fwd_noalloc_status", "gdn2_debug_timeout_once",
             "gdn2_last_error", "gdn2_version")
 DEBUG_CHUNK = 1
@@ -87,6 +88,10 @@ def _load():
     lib.gdn2_segment_correct_workspace_size.argtypes = [ctypes.POINTER(Dims)]
     lib.gdn2_decode_status.restype = ctypes.c_int
     lib.gdn2_decode_status.argtypes = [vp]
+    lib.gdn2_chunk_fwd_split_varlen.restype = ctypes.c_int
+    lib.gdn2_chunk_fwd_split_varlen.argtypes = [vp] * 11 + [ctypes.POINTER(Dims), vp, sz, vp]
+    lib.gdn2_chunk_fwd_split_varlen_workspace_size.restype = sz
+    lib.gdn2_chunk_fwd_split_varlen_workspace_size.argtypes = [ctypes.POINTER(Dims), vp]
     lib.gdn2_debug_timeout_once.restype = ctypes.c_int
     lib.gdn2_debug_timeout_once.argtypes = [ctypes.c_int32, ctypes.c_uint64]
     lib.gdn2_bwd.restype = ctypes.c_int
@@ -253,6 +258,44 @@ def chunk_fwd_split(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: to
                                   _ptr(S_T), ctypes.byref(dims), int(n_split), _ptr(workspace), workspace.numel(),
                                   _stream(dev))
     _check(rc)
+    return o, S_T
+
+
+def split_varlen_workspace_size(dims: Dims, cu_seqlens_host: Sequence[int]) -> int:
+    """Workspace bytes of ``gdn2_chunk_fwd_split_varlen`` for these lengths (0 if invalid)."""
+    host_cu = (ctypes.c_int32 * len(cu_seqlens_host))(*[int(x) for x in cu_seqlens_host])
+    return int(lib.gdn2_chunk_fwd_split_varlen_workspace_size(ctypes.byref(dims), host_cu))
+
+
+def chunk_fwd_split_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor,
+                           b: torch.Tensor, w: Optional[torch.Tensor], S0: Optional[torch.Tensor],
+                           cu_seqlens: torch.Tensor, cu_seqlens_host: Sequence[int], *,
+                           scalar_decay: bool = False, scalar_gates: bool = False, tied_gates: bool = False,
+                           gate_form_p3: bool = False, fused_prologue: bool = False,
+                           out_dtype: Optional[torch.dtype] = None, o: Optional[torch.Tensor] = None,
+                           S_T: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
+    """Packed varlen forward through ``gdn2_chunk_fwd_split_varlen``: sequences far longer
+    than the balanced per-SM share are cut into segments that run side by side.
+    q, k: [T_tot, H, d_k]; v: [T_tot, H, d_v]; cu_seqlens int32 [N + 1] on the device and its
+    host copy.  Returns (o [T_tot, H, d_v], S_T fp32 [N, H, d_k, d_v])."""
+    T_tot, H, dk = q.shape
+    N = cu_seqlens.numel() - 1
+    dv = v.shape[-1]
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    flags = flags_of(scalar_decay, scalar_gates, tied_gates, gate_form_p3, fused_prologue)
+    dims = make_dims(N, T_tot, H, dk, dv, 64, _dtype_code(q.dtype), _dtype_code(out_dtype), flags)
+    dev = q.device
+    if o is None:
+        o = torch.empty(T_tot, H, dv, dtype=out_dtype, device=dev)
+    if S_T is None:
+        S_T = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(split_varlen_workspace_size(dims, cu_seqlens_host), 256), dtype=torch.uint8,
+                                device=dev)
+    host_cu = (ctypes.c_int32 * len(cu_seqlens_host))(*[int(x) for x in cu_seqlens_host])
+    _check(lib.gdn2_chunk_fwd_split_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(b), _ptr(w), _ptr(S0),
+                                           _ptr(cu_seqlens), host_cu, _ptr(o), _ptr(S_T), ctypes.byref(dims),
+                                           _ptr(workspace), workspace.numel(), _stream(dev)))
     return o, S_T
 
 

@@ -206,6 +206,37 @@ int gdn2_chunk_fwd_split(const void *q, const void *k, const void *v,
 size_t gdn2_chunk_fwd_split_workspace_size(const gdn2_dims *dims, int32_t n_split);
 
 /*
+ * gdn2_chunk_fwd_split_varlen -- gdn2_chunk_fwd over a packed varlen batch in which some
+ * sequences are much longer than the balanced share of work per SM: those sequences are
+ * cut into whole-chunk segments that run side by side (the affine-composition view of
+ * neelmishra.github.io, "What makes the architecture more than a recurrence", as in
+ * gdn2_chunk_fwd_split), the others run whole.  The plan is made on the host from
+ * cu_seqlens_host: with tau the balanced number of 64-token chunks per SM, a sequence of
+ * more than 3 tau chunks is cut into segments of about tau chunks.  Four device steps:
+ * the split sequences' segments from the identity state (E = F + G per segment); every
+ * segment from the zero state (unsplit sequences from S0): G and provisional outputs; a
+ * serial combine per (sequence, head) (F = E - G, S <- F S + G, giving S_T and every
+ * segment's true start); the split segments with a non-zero start re-run from it, which
+ * writes their final outputs.  The split sequences cost about three times their work;
+ * when no sequence qualifies the call is the plain gdn2_chunk_fwd.  Same o and S_T as
+ * gdn2_chunk_fwd up to rounding.
+ * Arguments as gdn2_chunk_fwd with cu_seqlens; cu_seqlens_host is required here.
+ * Supported: d_k = d_v = 128, chunk 64, bf16 inputs.  workspace: at least
+ * gdn2_chunk_fwd_split_varlen_workspace_size(dims, cu_seqlens_host) bytes (the plan, and so
+ * the size, depends on the lengths and on the current device's SM count), 256-byte aligned;
+ * gdn2_check_status(workspace) reports a timed-out wait of any pass.
+ * Errors: GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_WORKSPACE, GDN2_ERR_CUDA.
+ */
+int gdn2_chunk_fwd_split_varlen(const void *q, const void *k, const void *v,
+                                const void *log_a, const void *b, const void *w,
+                                const float *S0, const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                                void *o, float *S_T, const gdn2_dims *dims,
+                                void *workspace, size_t workspace_bytes, gdn2_stream_t stream);
+
+/* Bytes of workspace gdn2_chunk_fwd_split_varlen needs (0 if the arguments are invalid). */
+size_t gdn2_chunk_fwd_split_varlen_workspace_size(const gdn2_dims *dims, const int32_t *cu_seqlens_host);
+
+/*
  * Sequence parallelism across ranks (one process per GPU): rank r of R holds tokens
  * [r L, (r + 1) L) of each of N equal sequences (all heads) and runs, on its own GPU,
  *

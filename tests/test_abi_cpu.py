@@ -231,3 +231,24 @@ def test_debug_timeout_hook_rejects_bad_arguments(g):
     assert g.lib.gdn2_debug_timeout_once(g.DEBUG_CHUNK, 10) == g.ERR_INVALID_ARG
     assert g.lib.gdn2_debug_timeout_once(g.DEBUG_DECODE, 20_000_000_000) == g.ERR_INVALID_ARG
     assert "wait_ns" in g.lib.gdn2_last_error().decode()
+
+
+def test_split_varlen_rejects_bad_arguments(g):
+    import ctypes as C
+    dims = _dims(g, n_seqs=3, seq_len=300)
+    cu_ok = (C.c_int32 * 4)(0, 100, 100, 300)
+    cu_bad = (C.c_int32 * 4)(0, 200, 100, 300)
+    assert g.lib.gdn2_chunk_fwd_split_varlen_workspace_size(C.byref(dims), cu_ok) > 0
+    assert g.lib.gdn2_chunk_fwd_split_varlen_workspace_size(C.byref(dims), cu_bad) == 0
+    assert g.lib.gdn2_chunk_fwd_split_varlen_workspace_size(C.byref(dims), None) == 0
+    fn = g.lib.gdn2_chunk_fwd_split_varlen
+
+    def call(cu_dev=P, cu_host=cu_ok, ws=WS, ws_bytes=1 << 30, d=dims):
+        return fn(P, P, P, P, P, P, None, cu_dev, cu_host, P, None, C.byref(d), ws, ws_bytes, None)
+
+    assert call(cu_host=None) == g.ERR_INVALID_ARG
+    assert "cu_seqlens_host" in g.lib.gdn2_last_error().decode()
+    assert call(cu_host=cu_bad) == g.ERR_INVALID_ARG
+    assert call(cu_dev=None) == g.ERR_INVALID_ARG
+    assert call(ws_bytes=16) == g.ERR_WORKSPACE
+    assert call(d=_dims(g, n_seqs=3, seq_len=300, d_k=64)) == g.ERR_UNSUPPORTED
