@@ -7,7 +7,6 @@ unsharded result exactly: the path shards with no data-path collective.  The
 max-over-ranks timing reduction bench.py uses is checked the same way.
 """
 import os
-import socket
 
 import numpy as np
 import pytest
@@ -19,11 +18,13 @@ from gated_delta_rule_159_b200 import shard
 
 
 def _free_port():
-    s = socket.socket()
-    s.bind(("127.0.0.1", 0))
-    port = s.getsockname()[1]
-    s.close()
-    return port
+    """A rendezvous for the ranks: a fresh file (no TCP port, so parallel test workers cannot
+    collide)."""
+    import tempfile
+    fd, path = tempfile.mkstemp(prefix="gdn2_rdzv_")
+    os.close(fd)
+    os.unlink(path)
+    return path
 
 
 def _problem(seed=0):
@@ -42,8 +43,7 @@ def _problem(seed=0):
 def _worker(rank, world, port, mode, out_q):
     import oracle
     os.environ["MASTER_ADDR"] = "127.0.0.1"
-    os.environ["MASTER_PORT"] = str(port)
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+    dist.init_process_group("gloo", init_method=f"file://{port}", rank=rank, world_size=world)
     try:
         cu, xs, S0 = _problem()
         if mode == "sequences":
@@ -161,8 +161,7 @@ def _seq_problem(N=2, T=48, H=2, d=4, seed=3):
 def _seq_worker(rank, world, port, out_q):
     from gated_delta_rule_159_b200 import gdn2
     os.environ["MASTER_ADDR"] = "127.0.0.1"
-    os.environ["MASTER_PORT"] = str(port)
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+    dist.init_process_group("gloo", init_method=f"file://{port}", rank=rank, world_size=world)
     try:
         xs, S0 = _seq_problem()
         T = xs[0].shape[1]
