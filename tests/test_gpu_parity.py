@@ -435,28 +435,43 @@ def test_decode_gate_form_p3(dev, dk, dv, scalar):
             assert rel_err(to_f64(S[n, h]), S_r[0, h]) <= TOL_DECODE
 
 
-def test_decode_indexed_matches_gathered_states(dev):
+@pytest.mark.parametrize("variant", ["channel", "scalar", "p3"])
+def test_decode_indexed_matches_gathered_states(dev, variant):
     """Continuous batching: row n updates pool slot state_idx[n]; padding rows (index
-    outside the pool) give zero output; slots no row names stay bit-identical."""
+    outside the pool) give zero output; slots no row names stay bit-identical.  With
+    channel-wise gates, one alpha and one tied beta per row, and the gist.science form."""
     from gated_delta_rule_159_b200 import gdn2, inputs
     P, N, H, d, steps = 7, 5, 3, 128, 3
     idx = torch.tensor([3, 0, -1, 6, 9], dtype=torch.int32, device=dev)
     live = [0, 1, 3]
-    di = inputs.make_decode_inputs(N, H, d, steps, dev, seed=13)
+    di = inputs.make_decode_inputs(N, H, d, steps, dev, seed=13, gate_form_p3=(variant == "p3"))
+    kw = {}
+    flags = 0
+    if variant == "scalar":
+        for n in ("log_a", "b"):
+            di[n] = di[n][..., 0].contiguous()
+        di["w"] = None
+        kw = dict(scalar_decay=True, scalar_gates=True, tied_gates=True)
+        flags = oracle.SCALAR_DECAY | oracle.SCALAR_GATES | oracle.TIED_GATES
+    elif variant == "p3":
+        kw = dict(gate_form_p3=True)
+        flags = oracle.GATE_FORM_P3
     g = torch.Generator(device=dev)
     g.manual_seed(17)
     pool = torch.randn(P, H, d, d, generator=g, device=dev) * 0.1
     pool_start = pool.clone()
     names = ("q", "k", "v", "log_a", "b", "w")
-    outs = [gdn2.decode_step_indexed(*(di[n][t] for n in names), pool, idx).clone() for t in range(steps)]
+    outs = [gdn2.decode_step_indexed(*(None if di[n] is None else di[n][t] for n in names), pool, idx, **kw).clone()
+            for t in range(steps)]
+    assert gdn2.decode_status() == gdn2.OK
     o_gpu = to_f64(torch.stack(outs))
     assert np.all(o_gpu[:, [2, 4]] == 0.0)
     for s in (1, 2, 4, 5):
         torch.testing.assert_close(pool[s], pool_start[s], rtol=0, atol=0)
     for n in live:
         slot = int(idx[n])
-        sl = lambda t: to_f64(t[:, n])  # noqa: E731
-        o_r, S_r = oracle.gdn2_fwd(*(sl(di[m]) for m in names), S0=to_f64(pool_start[slot])[None])
+        sl = lambda t: None if t is None else to_f64(t[:, n])  # noqa: E731
+        o_r, S_r = oracle.gdn2_fwd(*(sl(di[m]) for m in names), S0=to_f64(pool_start[slot])[None], flags=flags)
         for h in range(H):
             assert rel_err(o_gpu[:, n, h], o_r[:, h]) <= TOL_DECODE
             assert rel_err(to_f64(pool[slot, h]), S_r[0, h]) <= TOL_DECODE

@@ -79,3 +79,16 @@ def test_workspace_status_clean(dev):
     gdn2.chunk_fwd_split_varlen(*(inp[n] for n in names), inp["S0"], inp["cu_seqlens"], inp["cu_host"],
                                 out_dtype=torch.float32, workspace=ws)
     assert gdn2.check_status(ws) == gdn2.OK
+
+
+@pytest.mark.parametrize("variant", ["prologue", "p3_prologue"])
+def test_skewed_batch_fused_prologue(dev, variant):
+    """The varlen split with pre-activations (GDN2_FUSED_PROLOGUE) in both gate forms."""
+    inp = _inputs(dev, [9000, 70, 0, 1, 200], gate_form_p3=(variant == "p3_prologue"), fused_prologue=True)
+    from gated_delta_rule_159_b200 import gdn2
+    names = ("q", "k", "v", "log_a", "b", "w")
+    o, S_T = gdn2.chunk_fwd_split_varlen(*(inp[n] for n in names), inp["S0"], inp["cu_seqlens"], inp["cu_host"],
+                                         gate_form_p3=inp["gate_form_p3"], fused_prologue=True,
+                                         out_dtype=torch.float32)
+    eo, es = compare_units(inp, o, S_T, all_units(inp))
+    assert eo <= TOL_CHUNK_BF16 and es <= TOL_CHUNK_BF16, (eo, es)
