@@ -19,8 +19,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libgdn2.so")
 
-SOURCES = ["api.cu", "decode.cu", "chunk_simt.cu", "chunk_tc.cu", "noalloc.cu", "bwd.cu", "seqpar.cu"]
-HEADERS = ["common.cuh", "internal.h", "sm100_ptx.cuh"]
+SOURCES = ["api.cu", "decode.cu", "chunk_simt.cu", "chunk_tc.cu", "noalloc.cu", "bwd.cu", "bwd_tc.cu", "seqpar.cu"]
+HEADERS = ["common.cuh", "internal.h", "sm100_ptx.cuh", "tc_util.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",

@@ -212,6 +212,115 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const voi
   return GDN2_OK;
 }
 
+// gdn2_chunk_bwd workspace: [0, 256) header ([0] status, [1] forward unit counter, [2] backward
+// unit counter), the unit schedule, the per-sequence checkpoint offsets, the checkpoints.
+struct ChunkBwdLayout {
+  size_t off_sched, off_ckoff, off_ckpt, total;
+};
+static ChunkBwdLayout chunk_bwd_layout(const gdn2_dims *dims, bool packed) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  const int64_t t_total = packed ? (int64_t)dims->seq_len : (int64_t)dims->n_seqs * dims->seq_len;
+  const size_t units = (size_t)dims->n_seqs * dims->n_heads;
+  ChunkBwdLayout L;
+  L.off_sched = kWsHeader;
+  L.off_ckoff = L.off_sched + up(units * sizeof(int32_t));
+  L.off_ckpt = L.off_ckoff + up(((size_t)dims->n_seqs + 1) * sizeof(int64_t));
+  const size_t slots = gdn2::bwd_tc_ckpt_slots(dims->n_seqs, t_total, dims->n_heads, packed, dims->seq_len);
+  L.total = L.off_ckpt + slots * 128 * 128 * sizeof(float);
+  return L;
+}
+
+static const char *chunk_bwd_unsupported(const gdn2_dims *d) {
+  if (d->d_k != 128 || d->d_v != 128) return "gdn2_chunk_bwd needs d_k = d_v = 128";
+  if (d->dtype_in != GDN2_BF16) return "gdn2_chunk_bwd needs bf16 inputs";
+  if (d->flags & (GDN2_SCALAR_DECAY | GDN2_SCALAR_GATES | GDN2_GATE_FORM_P3 | GDN2_FUSED_PROLOGUE))
+    return "gdn2_chunk_bwd takes per-channel decay and gates in the default placement (GDN2_TIED_GATES "
+           "allowed); gdn2_bwd covers the other flags";
+  return nullptr;
+}
+
+size_t gdn2_chunk_bwd_workspace_size(const gdn2_dims *dims, int32_t packed) {
+  if (!dims || dims->n_seqs < 1 || dims->n_heads < 1 || dims->seq_len < 0) return 0;
+  if (chunk_bwd_unsupported(dims)) return 0;
+  return chunk_bwd_layout(dims, packed != 0).total;
+}
+
+int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_a, const void *b, const void *w,
+                   const float *S0, const int32_t *cu_seqlens, const void *dO, const float *dS_T, void *dq, void *dk,
+                   void *dv, void *dlog_a, void *db, void *dw, float *dS0, const gdn2_dims *dims, void *workspace,
+                   size_t workspace_bytes, gdn2_stream_t stream) {
+  g_err[0] = '\0';
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  rc = check_inputs(q, k, v, log_a, b, w, dims->flags, dims->dtype_in);
+  if (rc) return rc;
+  if (const char *why = chunk_bwd_unsupported(dims)) return fail(GDN2_ERR_UNSUPPORTED, "%s", why);
+  const bool tied = (dims->flags & GDN2_TIED_GATES) != 0;
+  if (!dO || !dq || !dk || !dv || !dlog_a || !db || (!dw && !tied))
+    return fail(GDN2_ERR_INVALID_ARG, "dO, dq, dk, dv, dlog_a, db (and dw without GDN2_TIED_GATES) must be non-NULL");
+  if ((S0 && !aligned16(S0)) || (dS_T && !aligned16(dS_T)) || (dS0 && !aligned16(dS0)))
+    return fail(GDN2_ERR_INVALID_ARG, "S0, dS_T and dS0 must be 16-byte aligned");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(GDN2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  const bool packed = cu_seqlens != nullptr;
+  const ChunkBwdLayout lay = chunk_bwd_layout(dims, packed);
+  if (workspace_bytes < lay.total)
+    return fail(GDN2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, lay.total);
+  const int64_t t_total = packed ? (int64_t)dims->seq_len : (int64_t)dims->n_seqs * dims->seq_len;
+  if (t_total >= (int64_t)1 << 31) return fail(GDN2_ERR_UNSUPPORTED, "gdn2_chunk_bwd needs T_tot < 2^31");
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char *ws = static_cast<char *>(workspace);
+  int32_t *status = reinterpret_cast<int32_t *>(ws);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kWsHeader, s);
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "cudaMemsetAsync(workspace): %s", cudaGetErrorString(e));
+  const int32_t *sched = nullptr;
+  int64_t *ckoff = nullptr;
+  if (packed) {
+    if (dims->n_seqs <= kMaxSortedSeqs) {
+      int32_t *sp = reinterpret_cast<int32_t *>(ws + lay.off_sched);
+      schedule_kernel<<<1, 1024, 0, s>>>(cu_seqlens, dims->n_seqs, dims->n_heads, sp);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "schedule launch: %s", cudaGetErrorString(e));
+      sched = sp;
+    }
+    ckoff = reinterpret_cast<int64_t *>(ws + lay.off_ckoff);
+    e = gdn2::launch_ckpt_offsets(cu_seqlens, dims->n_seqs, ckoff, s);
+    if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "checkpoint offsets launch: %s", cudaGetErrorString(e));
+  }
+  float *ckpt = reinterpret_cast<float *>(ws + lay.off_ckpt);
+
+  // the forward, writing the state before every chunk (and the final state) instead of o
+  gdn2::ChunkProblem f;
+  memset(&f, 0, sizeof(f));
+  f.q = q; f.k = k; f.v = v; f.log_a = log_a; f.b = b; f.w = w;
+  f.S0 = S0; f.cu_seqlens = cu_seqlens; f.o = nullptr; f.S_T = nullptr;
+  f.n_seqs = dims->n_seqs; f.seq_len = dims->seq_len; f.n_heads = dims->n_heads;
+  f.d_k = 128; f.d_v = 128; f.chunk = 64;
+  f.dtype_in = GDN2_BF16; f.dtype_out = dims->dtype_out; f.flags = dims->flags;
+  f.t_total = t_total;
+  f.status = status;
+  f.schedule = sched;
+  f.ckpt = ckpt;
+  f.ckpt_off = ckoff;
+  const char *why = "";
+  e = gdn2::launch_chunk_tc(f, s, &why);
+  if (e == cudaErrorNotSupported) return fail(GDN2_ERR_UNSUPPORTED, "%s", why);
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "chunk_tc launch: %s (%s)", cudaGetErrorString(e), why);
+
+  gdn2::BwdProblem p;
+  memset(&p, 0, sizeof(p));
+  p.q = q; p.k = k; p.v = v; p.log_a = log_a; p.b = b; p.w = tied ? nullptr : w;
+  p.S0 = S0; p.cu_seqlens = cu_seqlens; p.dO = dO; p.dS_T = dS_T;
+  p.dq = dq; p.dk = dk; p.dv = dv; p.dlog_a = dlog_a; p.db = db; p.dw = tied ? nullptr : dw; p.dS0 = dS0;
+  p.n_seqs = dims->n_seqs; p.seq_len = dims->seq_len; p.n_heads = dims->n_heads;
+  p.d_k = 128; p.d_v = 128; p.t_total = t_total;
+  p.dtype_in = GDN2_BF16; p.dtype_out = dims->dtype_out; p.flags = dims->flags;
+  e = gdn2::launch_bwd_tc(p, ckpt, ckoff, sched, status, status + 2, s);
+  if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "bwd_tc launch: %s", cudaGetErrorString(e));
+  return GDN2_OK;
+}
+
 size_t gdn2_bwd_workspace_size(const gdn2_dims *dims, int32_t packed) {
   if (!dims || dims->n_seqs < 1 || dims->n_heads < 1 || dims->seq_len < 0 || dims->d_k < 1 || dims->d_v < 1)
     return 0;
@@ -673,6 +782,8 @@ int gdn2_check_status(const void *workspace, gdn2_stream_t stream) {
   e = cudaMemcpy(&st, workspace, sizeof(st), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "reading the status word: %s", cudaGetErrorString(e));
   if (st == gdn2::kStatusTimeout) return fail(GDN2_ERR_TIMEOUT, "a bounded device wait timed out");
+  if (st == gdn2::kStatusRange)
+    return fail(GDN2_ERR_RANGE, "a chunk's decay range exceeds what gdn2_chunk_bwd handles; use gdn2_bwd");
   if (st != 0) return fail(GDN2_ERR_CUDA, "unknown device status %d", st);
   return GDN2_OK;
 }

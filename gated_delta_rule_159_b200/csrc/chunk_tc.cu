@@ -52,6 +52,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "sm100_ptx.cuh"
+#include "tc_util.cuh"
 
 namespace gdn2 {
 namespace {
@@ -120,91 +121,10 @@ struct TcParams {
   int dbg_skip;      // timeout test hook: CTA 0 arms its first k/q/v load group but issues none of its copies
 };
 
-__device__ __forceinline__ void named_bar(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-__device__ __forceinline__ uint2 lds_v2(uint32_t a) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ void sts_v2(uint32_t a, uint2 v) {
-  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(v.x), "r"(v.y) : "memory");
-}
-__device__ __forceinline__ void sts_u16(uint32_t a, uint16_t v) {
-  asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(v) : "memory");
-}
-__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
-  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint16_t bf16_bits(float v) {
-  const __nv_bfloat16 h = __float2bfloat16_rn(v);
-  return *reinterpret_cast<const uint16_t *>(&h);
-}
-__device__ __forceinline__ void sts_f32(uint32_t a, float v) {
-  asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
-}
-__device__ __forceinline__ void sts_v4(uint32_t a, uint4 v) {
-  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
-}
-__device__ __forceinline__ uint4 lds_v4(uint32_t a) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
-  return v;
-}
+using namespace tc;
 
 // fp32 64x64 scratch, rows padded to 68 floats (272 B): conflict-free float4 row writes.
 __device__ __forceinline__ int fidx(int i, int j) { return i * 68 + j; }
-
-// Byte offset of (row r, 16-byte chunk `chunk`) in a 128B-swizzled tile.
-__device__ __forceinline__ uint32_t swz(int r, uint32_t chunk) {
-  return (uint32_t)r * 128u + (((chunk ^ (uint32_t)(r & 7))) << 4);
-}
-
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                         int32_t *status, uint64_t limit_ns) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
-  if (*abort_flag) return false;
-  const uint64_t t0 = global_timer_ns();
-  uint32_t it = 0;
-  while (!ptx::mbar_try_wait(bar, parity)) {
-    if ((++it & 255u) == 0) {
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > limit_ns) {
-        *abort_flag = 1;
-        if (status) atomicExch(status, kStatusTimeout);
-        return false;
-      }
-    }
-  }
-  return true;
-}
-
-// Bounded wait that ignores the abort flag: the wind-down after a timed-out wait uses it to let
-// the copies and MMAs this CTA issued land before it frees its memory.
-__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-  const uint64_t t0 = global_timer_ns();
-  uint32_t it = 0;
-  while (!ptx::mbar_try_wait(bar, parity))
-    if ((++it & 255u) == 0 && global_timer_ns() - t0 > limit_ns) return;
-}
-
-__device__ __forceinline__ uint4 pack8(const float *f, float s) {
-  uint4 v;
-  v.x = pack_bf16x2(f[0] * s, f[1] * s);
-  v.y = pack_bf16x2(f[2] * s, f[3] * s);
-  v.z = pack_bf16x2(f[4] * s, f[5] * s);
-  v.w = pack_bf16x2(f[6] * s, f[7] * s);
-  return v;
-}
-__device__ __forceinline__ float4 unpack4(uint2 u) {
-  const float2 a = unpack_bf16x2(u.x), b = unpack_bf16x2(u.y);
-  return make_float4(a.x, a.y, b.x, b.y);
-}
-__device__ __forceinline__ uint2 pack4(float a, float b, float c, float d) {
-  return make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
-}
 
 // A chunk whose decay range is beyond the factored form, token by token (CUDA cores, fp32):
 // per token, Sbar = Diag(a) S; r = Sbar^T y; u = Sbar^T q; o = u - (q.x) r + (q.p) z;
@@ -345,7 +265,7 @@ __device__ __noinline__ void serial_chunk(const ChunkProblem &p, uint8_t *gb, ui
         u += pr.y;
       }
       const float zr = fs[SER_Z + tl * 128 + row];
-      if (cg == 0) {
+      if (cg == 0 && p.o) {
         const float ov = u - fs[SER_QX + tl] * r + fs[SER_QP + tl] * zr;
         Tout *go = static_cast<Tout *>(p.o) + ((size_t)(t0 + half * 32 + tl) * H + h) * D + row;
         *go = from_f32<Tout>(ov);
@@ -660,6 +580,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       len = p.seq_len;
     }
     const int nchunks = (int)((len + C - 1) / C);
+    // chunk-boundary states for the backward (gdn2_chunk_bwd): slot ci holds the state before
+    // chunk ci (as S = tau Sacc when the chunk starts), slot nchunks the final state
+    float *ck_unit = p.ckpt ? p.ckpt + ckpt_first_slot(p.ckpt_off, n, h, H, nchunks) * (D * D) : nullptr;
     if (tid == kIssuer && nchunks > 0 && !*sAbort) {
       issue_tma_l(h, (int)bos);
       issue_tma_a(h, (int)bos);
@@ -743,6 +666,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           issue_tma_w(h, t0 + C);
           issue_tma_a(h, t0 + C);
         }
+        if (ck_unit) {  // the state before this chunk
+          uint32_t r[32];
+          ptx::tmem_ld32(tmS + lane_base + cg * 32, r);
+          ptx::tmem_wait_ld();
+          const float *tp = sDLb(par ^ 1u) + cg * 32;
+          float *dst = ck_unit + ((size_t)ci * D + cg * 32) * D + row;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) dst[(size_t)j * D] = (ci > 0 ? tp[j] : 1.f) * __uint_as_float(r[j]);
+        }
         serial_chunk<kScalarDecay, kScalarGates, kP3, kProlog, Tout>(p, gb, tmS + lane_base + cg * 32,
                                                                    ci > 0 ? sDLb(par ^ 1u) + cg * 32 : nullptr,
                                                                    t0, nvalid, h);
@@ -797,14 +729,20 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         }
         ptx::tmem_ld32(tmS + lane_base + cg * 32, r);
         ptx::tmem_wait_ld();
+        float *ck = ck_unit ? ck_unit + ((size_t)ci * D + cg * 32) * D + row : nullptr;
 #pragma unroll
         for (int j4 = 0; j4 < 8; ++j4) {
           const float4 t4 = ci > 0 ? *reinterpret_cast<const float4 *>(tp + 4 * j4) : make_float4(1.f, 1.f, 1.f, 1.f);
           const float4 s4 = *reinterpret_cast<const float4 *>(smv + 4 * j4);
-          const float f0 = (__uint_as_float(r[4 * j4]) * t4.x) * s4.x;
-          const float f1 = (__uint_as_float(r[4 * j4 + 1]) * t4.y) * s4.y;
-          const float f2 = (__uint_as_float(r[4 * j4 + 2]) * t4.z) * s4.z;
-          const float f3 = (__uint_as_float(r[4 * j4 + 3]) * t4.w) * s4.w;
+          const float g0 = __uint_as_float(r[4 * j4]) * t4.x, g1 = __uint_as_float(r[4 * j4 + 1]) * t4.y;
+          const float g2 = __uint_as_float(r[4 * j4 + 2]) * t4.z, g3 = __uint_as_float(r[4 * j4 + 3]) * t4.w;
+          if (ck) {  // the state before this chunk
+            ck[(size_t)(4 * j4) * D] = g0;
+            ck[(size_t)(4 * j4 + 1) * D] = g1;
+            ck[(size_t)(4 * j4 + 2) * D] = g2;
+            ck[(size_t)(4 * j4 + 3) * D] = g3;
+          }
+          const float f0 = g0 * s4.x, f1 = g1 * s4.y, f2 = g2 * s4.z, f3 = g3 * s4.w;
           r[4 * j4] = __float_as_uint(f0);
           r[4 * j4 + 1] = __float_as_uint(f1);
           r[4 * j4 + 2] = __float_as_uint(f2);
@@ -1140,7 +1078,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncthreads();
-      if (nvalid == C) {
+      if (!p.o) {
+        // no output requested (the checkpointing forward of the backward)
+      } else if (nvalid == C) {
         // full chunk: asynchronous TMA store; the next chunk's epilogue rewrites the staging
         // area only after the issuing thread has seen these reads done (bulk_wait_group_read0)
         if (tid == kIssuer) {
@@ -1171,14 +1111,19 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       waitb(bar(BAR_G5), (it & 1u) ^ 1u);
       ptx::tc_fence_after();
     }
-    if (p.S_T && !*sAbort) {
-      float *dst = p.S_T + ((size_t)unit * D + cg * 32) * D + row;
+    if ((p.S_T || ck_unit) && !*sAbort) {
+      float *dst = p.S_T ? p.S_T + ((size_t)unit * D + cg * 32) * D + row : nullptr;
+      float *ck = ck_unit ? ck_unit + ((size_t)nchunks * D + cg * 32) * D + row : nullptr;
       const float *tp = sDLb((it & 1u) ^ 1u) + cg * 32;  // the last chunk's e^{L_C - L_ref}
       uint32_t r[32];
       ptx::tmem_ld32(tmS + lane_base + cg * 32, r);
       ptx::tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) dst[(size_t)j * D] = (nchunks > 0 ? tp[j] : 1.f) * __uint_as_float(r[j]);
+      for (int j = 0; j < 32; ++j) {
+        const float sv = (nchunks > 0 ? tp[j] : 1.f) * __uint_as_float(r[j]);
+        if (dst) dst[(size_t)j * D] = sv;
+        if (ck) ck[(size_t)j * D] = sv;
+      }
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -1308,7 +1253,7 @@ cudaError_t launch_chunk_tc(const ChunkProblem &p, cudaStream_t stream, const ch
   const void *g_first = p3 ? p.b : (tied ? p.b : p.w);
   const void *g_second = p3 ? (tied ? p.b : p.w) : p.b;
   if (ok && !sg) ok = make_map(&P.tm_b, g_second, T, p.n_heads) && make_map(&P.tm_w, g_first, T, p.n_heads);
-  if (ok) ok = make_map_o(&P.tm_o, p.o, T, p.n_heads, p.dtype_out == GDN2_BF16);
+  if (ok && p.o) ok = make_map_o(&P.tm_o, p.o, T, p.n_heads, p.dtype_out == GDN2_BF16);
   if (!ok) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad tensor geometry)";
     return cudaErrorInvalidValue;

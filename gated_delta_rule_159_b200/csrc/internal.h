@@ -28,6 +28,12 @@ struct ChunkProblem {
   // replaces cu_seqlens for the unit bounds, so the sequences may leave gaps between them
   // (the split forward's passes over a subset of segments).  Tensor-core path only.
   const int32_t *seg_bounds;
+  // Optional chunk-boundary state buffer for the backward (tensor-core path only): fp32
+  // [slots][d_k][d_v], the slots of a unit laid out as tc::ckpt_first_slot states; ckpt_off
+  // [n_seqs + 1] (int64) is the first slot of each sequence divided by n_heads, or NULL for
+  // equal lengths.  With ckpt set, o may be NULL (no output written).
+  float *ckpt;
+  const int64_t *ckpt_off;
 };
 
 struct DecodeProblem {
@@ -62,6 +68,8 @@ struct BwdProblem {
 
 // Status word values written by kernels (0 = fine).
 constexpr int32_t kStatusTimeout = 1;
+// A chunk of the tensor-core backward has a decay range beyond its factored form.
+constexpr int32_t kStatusRange = 2;
 
 // Activated fp32 copies of the inputs written by the backward's prologue pass.
 struct PrologueCopies {
@@ -71,6 +79,15 @@ struct PrologueCopies {
 size_t bwd_workspace_bytes(int64_t n_seqs, int64_t t_total, int n_heads, int d_k, int d_v, uint32_t flags);
 void bwd_carve(BwdProblem &p, void *workspace);
 cudaError_t launch_bwd(const BwdProblem &p, cudaStream_t stream);
+
+// Chunked tensor-core backward (bwd_tc.cu; d_k = d_v = 128, bf16 inputs, per-channel gates in
+// the default placement, tied or not).  Checkpoint slots a call needs (an upper bound for
+// packed batches), the per-sequence slot offsets for packed batches, and the reverse kernel
+// over the states a checkpointing forward wrote (ChunkProblem::ckpt).
+size_t bwd_tc_ckpt_slots(int64_t n_seqs, int64_t t_total, int n_heads, bool packed, int seq_len);
+cudaError_t launch_ckpt_offsets(const int32_t *cu_seqlens, int n_seqs, int64_t *off, cudaStream_t stream);
+cudaError_t launch_bwd_tc(const BwdProblem &p, const float *ckpt, const int64_t *ckpt_off, const int32_t *schedule,
+                          int32_t *status, int32_t *counter, cudaStream_t stream);
 
 // Sequence-parallel forward (seqpar.cu): segments of seg_len tokens, workspace offsets.
 struct SplitPlan {

@@ -23,6 +23,7 @@ ERR_UNSUPPORTED = -2
 ERR_CUDA = -3
 ERR_TIMEOUT = -4
 ERR_WORKSPACE = -5
+ERR_RANGE = -6
 BF16 = 0
 F32 = 1
 SCALAR_DECAY = 1
@@ -33,7 +34,7 @@ FUSED_PROLOGUE = 16
 
 EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_workspace_size", "gdn2_check_status",
             "gdn2_decode_step", "gdn2_decode_step_indexed", "gdn2_decode_status", "gdn2_bwd",
-            "gdn2_bwd_workspace_size", "gdn2_chunk_fwd_split", "gdn2_chunk_fwd_split_workspace_size",
+            "gdn2_bwd_workspace_size", "gdn2_chunk_bwd", "gdn2_chunk_bwd_workspace_size", "gdn2_chunk_fwd_split", "gdn2_chunk_fwd_split_workspace_size",
             "gdn2_segment_maps", "gdn2_segment_maps_workspace_size", "gdn2_affine_prefix",
             "gdn2_segment_correct", "gdn2_segment_correct_workspace_size",
             "gdn2_chunk_fwd_split_varlen", "gdn2_chunk_fwd_split_varlen_workspace_size",
@@ -98,6 +99,10 @@ def _load():
     lib.gdn2_bwd.argtypes = [vp] * 17 + [ctypes.POINTER(Dims), vp, sz, vp]
     lib.gdn2_bwd_workspace_size.restype = sz
     lib.gdn2_bwd_workspace_size.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32]
+    lib.gdn2_chunk_bwd.restype = ctypes.c_int
+    lib.gdn2_chunk_bwd.argtypes = [vp] * 17 + [ctypes.POINTER(Dims), vp, sz, vp]
+    lib.gdn2_chunk_bwd_workspace_size.restype = sz
+    lib.gdn2_chunk_bwd_workspace_size.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32]
     lib.gdn2_last_error.restype = ctypes.c_char_p
     lib.gdn2_last_error.argtypes = []
     lib.gdn2_version.restype = ctypes.c_int
@@ -451,6 +456,29 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, 
     same inputs (layouts as ``chunk_fwd``).  Gradients take dO's dtype.  Returns a dict with
     dq, dk, dv, dlog_a, db, dw (None with ``tied_gates``: its gradient is added into db) and
     dS0 (fp32, None unless ``need_dS0``)."""
+    return _bwd_call(lib.gdn2_bwd, lib.gdn2_bwd_workspace_size, q, k, v, log_a, b, w, dO, S0, dS_T, cu_seqlens,
+                     scalar_decay, scalar_gates, tied_gates, gate_form_p3, fused_prologue, need_dS0, workspace)
+
+
+def chunk_bwd_workspace_size(dims: Dims, packed: bool = False) -> int:
+    """Workspace bytes of ``gdn2_chunk_bwd`` (0: dims unsupported)."""
+    return int(lib.gdn2_chunk_bwd_workspace_size(ctypes.byref(dims), 1 if packed else 0))
+
+
+def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, b: torch.Tensor,
+              w: Optional[torch.Tensor], dO: torch.Tensor, S0: Optional[torch.Tensor] = None,
+              dS_T: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None, *,
+              tied_gates: bool = False, need_dS0: bool = True, workspace: Optional[torch.Tensor] = None) -> dict:
+    """The gradients of ``bwd`` through ``gdn2_chunk_bwd``: the chunked tensor-core backward
+    (d_k = d_v = 128, bf16 inputs, per-channel decay and gates in the default placement).
+    Same arguments and result as ``bwd``; ``gdn2_check_status(workspace)`` reports a chunk
+    whose decay range is beyond the factored form (ERR_RANGE)."""
+    return _bwd_call(lib.gdn2_chunk_bwd, lib.gdn2_chunk_bwd_workspace_size, q, k, v, log_a, b, w, dO, S0, dS_T,
+                     cu_seqlens, False, False, tied_gates, False, False, need_dS0, workspace)
+
+
+def _bwd_call(fn, ws_fn, q, k, v, log_a, b, w, dO, S0, dS_T, cu_seqlens, scalar_decay, scalar_gates, tied_gates,
+              gate_form_p3, fused_prologue, need_dS0, workspace) -> dict:
     if q.dim() == 4:
         N, T, H, dk = q.shape
         seq_len = T
@@ -470,12 +498,14 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Tensor, 
              dw=None if tied_gates else torch.empty_like(w, dtype=dO.dtype),
              dS0=torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev) if need_dS0 else None)
     if workspace is None:
-        workspace = torch.empty(bwd_workspace_size(dims, cu_seqlens is not None), dtype=torch.uint8, device=dev)
-    rc = lib.gdn2_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(b), _ptr(w), _ptr(S0), _ptr(cu_seqlens),
-                      _ptr(dO), _ptr(dS_T), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_a"]),
-                      _ptr(g["db"]), _ptr(g["dw"]), _ptr(g["dS0"]), ctypes.byref(dims), _ptr(workspace),
-                      workspace.numel(), _stream(dev))
+        nbytes = int(ws_fn(ctypes.byref(dims), 1 if cu_seqlens is not None else 0))
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(b), _ptr(w), _ptr(S0), _ptr(cu_seqlens),
+            _ptr(dO), _ptr(dS_T), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_a"]),
+            _ptr(g["db"]), _ptr(g["dw"]), _ptr(g["dS0"]), ctypes.byref(dims), _ptr(workspace),
+            workspace.numel(), _stream(dev))
     _check(rc)
+    g["workspace"] = workspace
     return g
 
 

@@ -68,7 +68,9 @@ enum gdn2_status {
   GDN2_ERR_UNSUPPORTED = -2,  /* valid request the library has no kernel for */
   GDN2_ERR_CUDA = -3,         /* a CUDA runtime call or kernel launch failed */
   GDN2_ERR_TIMEOUT = -4,      /* a bounded device-side wait gave up (reported by gdn2_check_status) */
-  GDN2_ERR_WORKSPACE = -5     /* workspace pointer NULL or smaller than the queried size */
+  GDN2_ERR_WORKSPACE = -5,    /* workspace pointer NULL or smaller than the queried size */
+  GDN2_ERR_RANGE = -6         /* gdn2_chunk_bwd met a chunk whose decay range is beyond its
+                                 factored form (reported by gdn2_check_status) */
 };
 
 /* Element types of the per-token inputs (dtype_in) and of o (dtype_out). */
@@ -155,7 +157,8 @@ size_t gdn2_chunk_fwd_workspace_size(const gdn2_dims *dims);
 /*
  * gdn2_check_status -- synchronises `stream`, then reads the device status word
  * that gdn2_chunk_fwd left in `workspace` (bounded waits inside the kernel
- * record a timeout there instead of hanging).  Returns GDN2_OK, GDN2_ERR_TIMEOUT
+ * record a timeout there instead of hanging; gdn2_chunk_bwd also records a chunk
+ * beyond its decay range there).  Returns GDN2_OK, GDN2_ERR_TIMEOUT, GDN2_ERR_RANGE
  * or GDN2_ERR_CUDA.  Optional: a caller that never checks loses nothing but the
  * diagnosis.
  */
@@ -353,6 +356,45 @@ int gdn2_bwd(const void *q, const void *k, const void *v,
  * packed != 0: the call passes cu_seqlens, so dims.seq_len is T_tot; packed == 0:
  * N equal sequences of dims.seq_len tokens. */
 size_t gdn2_bwd_workspace_size(const gdn2_dims *dims, int32_t packed);
+
+/*
+ * gdn2_chunk_bwd -- the gradients gdn2_bwd returns, computed in the chunked form on the
+ * tensor cores.  The method trains through its chunked form with a gate-aware backward
+ * (gist.science Methodologie 3, "Poortbewuste terugwaartse pass"); the pages print no
+ * formula for it, and this call differentiates the chunk algebra of gdn2_chunk_fwd:
+ *   1. a pass of the chunked forward writes the state before every 64-token chunk, and
+ *      the final state, to the workspace (fp32; o is not written);
+ *   2. one reverse pass per (sequence, head), last chunk first, recomputes each chunk's
+ *      auxiliaries from its start state and forms every gradient of the chunk with
+ *      bf16 tensor-core products accumulated in fp32, carrying dLoss/dS (fp32) from chunk
+ *      to chunk; the chain rule through the decay and the gates runs in the same pass.
+ * It returns the gradients of  sum_t <dO_t, o_t> + sum_n <dS_T[n], S_T[n]>  with the
+ * precision of the bf16-input chunked forward (the products take bf16 operands), not the
+ * fp32 precision of gdn2_bwd.
+ * Arguments, layouts and ownership: as gdn2_bwd.  dims.chunk is ignored.
+ * Supported: d_k = d_v = 128, bf16 inputs, dtype_out (dO and the gradients) bf16 or fp32,
+ * per-channel decay and gates in the default placement, GDN2_TIED_GATES allowed; other
+ * flags give GDN2_ERR_UNSUPPORTED (gdn2_bwd covers them), as does T_tot >= 2^31.
+ * Range: every chunk must keep each channel's in-chunk decay L_0 - L_63 within 128 nats
+ * (the forward's factored form).  A chunk beyond it is not computed: the call records
+ * GDN2_ERR_RANGE for gdn2_check_status(workspace) and that (sequence, head)'s gradients are
+ * undefined; gdn2_bwd handles any range.
+ * workspace  >= gdn2_chunk_bwd_workspace_size(dims, packed) bytes, 256-byte aligned; one
+ *            call at a time per workspace.  It holds the checkpoints: 64 KB per chunk and
+ *            (sequence, head), plus one final state each.
+ * Errors: GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_WORKSPACE, GDN2_ERR_CUDA;
+ * gdn2_check_status reports GDN2_ERR_TIMEOUT (a bounded device wait) or GDN2_ERR_RANGE.
+ */
+int gdn2_chunk_bwd(const void *q, const void *k, const void *v,
+                   const void *log_a, const void *b, const void *w,
+                   const float *S0, const int32_t *cu_seqlens,
+                   const void *dO, const float *dS_T,
+                   void *dq, void *dk, void *dv, void *dlog_a, void *db, void *dw, float *dS0,
+                   const gdn2_dims *dims, void *workspace, size_t workspace_bytes, gdn2_stream_t stream);
+
+/* Bytes of device workspace gdn2_chunk_bwd needs (0 if dims are unsupported); packed as
+ * for gdn2_bwd_workspace_size (for packed batches an upper bound from T_tot and N). */
+size_t gdn2_chunk_bwd_workspace_size(const gdn2_dims *dims, int32_t packed);
 
 /*
  * gdn2_chunk_fwd_noalloc -- gdn2_chunk_fwd for callers that cannot allocate
