@@ -1,0 +1,968 @@
+// bwd_tc.cu -- gradients of the chunked Gated DeltaNet-2 forward on the sm_100a tensor cores
+// (d_k = d_v = 128, chunk C = 64, bf16 inputs, fp32 accumulation), chunk by chunk in reverse.
+//
+// The method trains through its chunked form with a gate-aware backward (gist.science
+// Methodologie 3, "Poortbewuste terugwaartse pass"; alanhou.org "Core Mechanism"); the pages
+// give no formula for it.  This file differentiates the chunk algebra of chunk_tc.cu.  For one
+// chunk (rows t, s in [0, 64); the operands scaled to the per-channel reference
+// rho = (L_0 + L_63) / 2 exactly as the forward scales them):
+//
+//   k_r = k e^{L - rho}, q_r = q e^{L - rho}, x_r = b.k e^{rho - L}, p_r = w.k e^{rho - L},
+//   S_r = Diag(e^{rho}) S_c (S_c: the state before the chunk), gamma = e^{L_63 - rho},
+//   A = (k_r x_r^T)|strict, B = (k_r p_r^T)|strict, QX = (q_r x_r^T)|lower, QP = (q_r p_r^T)|lower,
+//   R = B V + k_r S_r,  M = T R with T = (I + A)^-1  (row t of M: the erase read of token t),
+//   O = q_r S_r + QP V - QX M,    S_{c+1} = Diag(gamma) (S_r + p_r^T V - x_r^T M).
+//
+// With Lam = dLoss/dS_{c+1} and Lam_g = Diag(gamma) Lam, reverse mode gives
+//
+//   dM = -(QX^T dO + x_r Lam_g),  dR = T^T dM,
+//   [dA dB; dQX dQP] = ([dR; dO] [-M; V]^T) masked like [A B; QX QP],
+//   dV   = QP^T dO + B^T dR + p_r Lam_g,
+//   dk_r = dA x_r + dB p_r + dR S_r^T,    dq_r = dQX x_r + dQP p_r + dO S_r^T,
+//   dx_r = dA^T k_r + dQX^T q_r - M Lam_g^T,   dp_r = dB^T k_r + dQP^T q_r + V Lam_g^T,
+//   dLoss/dS_c = Diag(e^{rho}) (Lam_g + q_r^T dO + k_r^T dR),
+//   dL_t = dq_r.q_r + dk_r.k_r - dx_r.x_r - dp_r.p_r (per channel), plus at t = 63 the decay
+//   term sum_j Lam_ij (S_{c+1})_ij; d log_a_s = sum_{t >= s} dL_t (inside the chunk).
+//
+// rho only moves factors between operands (the chunk's function does not depend on it), so
+// it takes no gradient.  Every product runs as a tcgen05.mma (kind::f16, bf16 operands, fp32
+// TMEM accumulators) with M = 128 rows: the 64-row matrices are stacked in pairs
+// ([k_r; q_r], [x_r; p_r], [dR; dO], [-M; V]) so that one instruction covers two of them, and
+// the transposed operand forms are MN-major shared-memory descriptors of the same tiles.  The
+// carried adjoint lives in TMEM (lane = d_k channel) for the whole sequence, so the thread of a
+// d_k channel scales and stores its row with one factor and 16-byte vectors.
+//
+// The S_r tiles come from a forward pass of chunk_tc_kernel that writes each chunk's bf16 S_r
+// (the operand it builds anyway, with the same rho) as a swizzled tile image to the workspace;
+// one bulk copy per chunk brings it to shared memory.  One CTA (512 threads) per SM takes (sequence, head) units
+// from an atomic counter and walks their chunks last to first; per chunk its phases are:
+//   1  (the raw k, q, v, log_a, b, w, dO tiles (TMA) and S_r (bulk copy) were requested while
+//      the previous chunk finished) cumulative decay, the scaled operands in place, Lam_g;
+//   2  G1 [A B; QX QP] = [k_r; q_r][x_r; p_r]^T  and  dM^T <- Lam_g^T x_r^T;  masks;
+//   3  the (I + A)^-1 solve (fp32, warps 0-14) while warp 15 issues R^T and dM^T += dO^T QX;
+//   4  R^T, -dM^T to bf16 TMEM operands; M^T = R^T T^T, dR^T = dM^T T;
+//   5  -M and dR to shared memory;
+//   6  [dA dB; dQX dQP], the adjoint update, dV^T and the S_r terms of [dk_r^T | dq_r^T];
+//   7  the decay term of the previous chunk (row sums of adjoint x state), dV out, the masks
+//      of the gradient tile;
+//   8  [dx_r^T | dp_r^T] and the rest of [dk_r^T | dq_r^T];
+//   9  the chain rule through the scaling and the gates, the reverse cumulative sum of dL,
+//      gradient stores.
+// Chunks whose decay range exceeds kFastSpan nats on some channel are outside the factored
+// form: the kernel records kStatusRange and leaves the rest of that unit (gdn2_bwd, the
+// token-serial reverse mode, covers any range).  Every mbarrier wait is bounded.
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100_ptx.cuh"
+#include "tc_util.cuh"
+
+namespace gdn2 {
+namespace {
+
+using namespace tc;
+
+constexpr int C = 64;
+constexpr int D = 128;
+constexpr int kThreads = 512;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s
+constexpr float kLog2eF = 1.4426950408889634f;
+constexpr float kFastSpan = 128.f;  // as in the forward: factors stay within e^{+-64}
+
+// Shared-memory map (byte offsets from a 1024-byte-aligned base).  The 128-row operand tiles
+// are two column blocks of 64 (16 KB apart), each a stack of 8-row x 128-byte swizzle atoms.
+constexpr uint32_t OFF_KQ = 0;          // [k_r rows 0-63 | q_r rows 64-127] per block
+constexpr uint32_t OFF_XP = 32768;      // [x_r | p_r]
+constexpr uint32_t OFF_MV = 65536;      // [-M | V]
+constexpr uint32_t OFF_RO = 98304;      // [dR | dO]
+constexpr uint32_t OFF_SR = 131072;     // S_r [d_k rows][d_v]; from phase 7 the gradient tile dG
+constexpr uint32_t OFF_LG = 163840;     // Lam_g [d_k rows][d_v]
+constexpr uint32_t OFF_BQP = 196608;    // [B rows 0-63 | QP rows 64-127], one 64-column block
+constexpr uint32_t OFF_XS = 212992;     // fp32 solve scratch, 4 KB
+constexpr uint32_t OFF_MISC = 217088;
+// Tiles that live in the rows of another tile until that tile is written:
+constexpr uint32_t OFF_T = OFF_MV;             // T bf16 [64 x 64] (the -M rows of block 0)
+constexpr uint32_t OFF_QX = OFF_MV + 16384;    // QX bf16 [64 x 64] (the -M rows of block 1)
+constexpr uint32_t OFF_AT0 = OFF_RO;           // fp32 A, then T, rows 0-31 [32][64] (dR rows, block 0)
+constexpr uint32_t OFF_AT1 = OFF_RO + 16384;   // rows 32-63 (dR rows, block 1)
+constexpr uint32_t OFF_DG = OFF_SR;            // [dA dB; dQX dQP] as [column block][128 rows][64]
+constexpr uint32_t OFF_GRAW = OFF_LG;          // raw log_a tile [2 blocks][64 rows] until Lam_g is built
+constexpr uint32_t MISC_BAR = 0;       // mbarriers
+constexpr uint32_t MISC_TMEM = 64;
+constexpr uint32_t MISC_ABORT = 68;
+constexpr uint32_t MISC_UNIT = 72;
+constexpr uint32_t MISC_WIDE = 76;
+constexpr uint32_t MISC_ISS = 80;      // uint32: load phases armed on BAR_LD
+constexpr uint32_t MISC_RHO = 128;     // float[128]     rho of the current chunk
+constexpr uint32_t MISC_ESR = 640;     // float[2][128]  e^{rho} per chunk parity
+constexpr uint32_t MISC_DLC = 1664;    // float[2][128]  decay term of L_63 per chunk parity
+constexpr uint32_t MISC_L0 = 2688;     // float[128]     L_0
+constexpr uint32_t MISC_PART = 3200;   // float[4][128]  per-row-group sums (cumulative decay, dL)
+constexpr uint32_t MISC_LPRE = 5248;   // float[4][128]  exclusive row-group prefixes of L
+constexpr uint32_t MISC_RS = 7296;     // float[4][128]  row sums per lane quadrant
+constexpr uint32_t MISC_BYTES = 9344;
+constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES + 1024;  // + base alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 limit per CTA");
+enum { BAR_LD = 0, BAR_G1, BAR_GA, BAR_GB, BAR_G5, BAR_G7, BAR_DRAIN, kNumBars };
+static_assert(MISC_BAR + 8 * kNumBars <= MISC_TMEM, "mbarriers overlap the TMEM address slot");
+
+struct BwdTcParams {
+  // raw tiles of a chunk by TMA, (channel, head, token) boxes of 64 x 1 x 64, 128-byte swizzle:
+  // k, q over the k_r, q_r rows, v over the V rows, b, w over the x_r, p_r rows, log_a into
+  // the Lam_g tile's space
+  CUtensorMap tm_q, tm_k, tm_v, tm_g, tm_b, tm_w, tm_do;  // tm_do: bf16 dO only
+  const __nv_bfloat16 *q, *k, *v, *log_a, *b, *w;  // forward inputs [T_tot][H][128]
+  const void *dO;                                  // [T_tot][H][128] Tout
+  const float *dS_T;                               // [N][H][128][128] or NULL
+  void *dq, *dk, *dv, *dlog_a, *db, *dw;           // Tout, like the inputs (dw NULL when tied)
+  float *dS0;                                      // [N][H][128][128] or NULL
+  const uint8_t *ckpt;                             // per chunk the bf16 S_r tile image (32 KB)
+  const float *S_fin;                              // [N][H][128][128] final states (fp32)
+  const int64_t *ckpt_off;                         // NULL for equal lengths
+  const int32_t *cu_seqlens;                       // NULL for equal lengths
+  const int32_t *schedule;                         // unit order (longest first) or NULL
+  int32_t *status, *counter;
+  int n_units, n_heads, seq_len;
+  uint64_t wait_ns;
+};
+
+// Sums v[c] over the 32 lanes of the warp for every column c; lane l returns the sum of
+// column l.  Each step halves the columns a lane keeps and adds its partner's half.
+__device__ __forceinline__ float warp_colsum32(float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int j = 0; j < off; ++j) {
+      const float send = up ? v[j] : v[j + off];
+      const float keep = up ? v[j + off] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0];
+}
+
+__device__ __forceinline__ float bf(const __nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Descriptors of the 128-column operand tiles (two 64-column blocks 16 KB apart), K step kk
+// of 16: K-major walks the columns (32 bytes per step), MN-major walks the rows (16 rows,
+// 2 KB per step).
+__device__ __forceinline__ uint64_t kmaj(uint32_t base, int kk) {
+  return ptx::sdesc_sw128(base + (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u, 16, 1024);
+}
+__device__ __forceinline__ uint64_t mnmaj(uint32_t base, int kk) {
+  return ptx::sdesc_sw128(base + (uint32_t)kk * 2048u, 16384, 1024);
+}
+
+template <typename Tout, bool kTied>
+__global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_constant__ BwdTcParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = ptx::smem_u32(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t *gb = smem_raw + (sb - raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, cg = warp >> 2;  // TMEM lane quadrant, column group (row group)
+  const int row = qd * 32 + lane;           // TMEM lane; the channel of the elementwise phases
+  const int H = P.n_heads;
+  constexpr int kIssuer = 480;              // warp 15 lane 0 issues every MMA, in order
+  constexpr int kSolveThreads = 480;        // warps 0-14
+  constexpr int NB_SOLVE = 1;
+
+  float *sRho = reinterpret_cast<float *>(gb + OFF_MISC + MISC_RHO);
+  float *sEsr = reinterpret_cast<float *>(gb + OFF_MISC + MISC_ESR);
+  float *sDlc = reinterpret_cast<float *>(gb + OFF_MISC + MISC_DLC);
+  float *sL0 = reinterpret_cast<float *>(gb + OFF_MISC + MISC_L0);
+  float *part = reinterpret_cast<float *>(gb + OFF_MISC + MISC_PART);
+  float *lpre = reinterpret_cast<float *>(gb + OFF_MISC + MISC_LPRE);
+  float *rs = reinterpret_cast<float *>(gb + OFF_MISC + MISC_RS);
+  volatile int *sAbort = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_ABORT);
+  volatile int *sUnit = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_UNIT);
+  volatile int *sWide = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_WIDE);
+  volatile uint32_t *sIss = reinterpret_cast<volatile uint32_t *>(gb + OFF_MISC + MISC_ISS);
+  auto bar = [&](int i) { return sb + OFF_MISC + MISC_BAR + 8u * (uint32_t)i; };
+  auto waitb = [&](uint32_t b, uint32_t parity) { return wait_bar(b, parity, sAbort, P.status, P.wait_ns); };
+  // fp32 A / T of the solve: rows 0-31 and 32-63 in two 8 KB halves, 64 floats per row; the
+  // column index is XORed with 4 (row mod 8) so that the 8 rows of an mma fragment load fall
+  // in different banks (groups of four columns stay contiguous)
+  auto at = [&](int i, int j) -> float * {
+    return reinterpret_cast<float *>(gb + (i < 32 ? OFF_AT0 : OFF_AT1) +
+                                     (uint32_t)(((i & 31) * 64 + (j ^ ((i & 7) << 2))) * 4));
+  };
+  // L_ref of channel i from the row-group sums (the same expression in every thread)
+  auto rho_of = [&](int i, float &tot) {
+    tot = ((part[i] + part[128 + i]) + part[256 + i]) + part[384 + i];
+    return 0.5f * (sL0[i] + tot);
+  };
+
+  if (tid == 0) {
+    for (int i = 0; i < kNumBars; ++i) ptx::mbar_init(bar(i), 1);
+    ptx::fence_mbar_init();
+    *sAbort = 0;
+    *sIss = 0u;
+    ptx::tma_prefetch_desc(&P.tm_q);
+    ptx::tma_prefetch_desc(&P.tm_k);
+    ptx::tma_prefetch_desc(&P.tm_v);
+    ptx::tma_prefetch_desc(&P.tm_g);
+    ptx::tma_prefetch_desc(&P.tm_b);
+    if (!kTied) ptx::tma_prefetch_desc(&P.tm_w);
+  }
+  if (warp == 0) {
+    ptx::tmem_alloc(sb + OFF_MISC + MISC_TMEM, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(gb + OFF_MISC + MISC_TMEM);
+  // TMEM columns: the adjoint Acc (lane = d_k channel i, column = d_v channel j), and three
+  // 128-column work areas:
+  //   X: G1 -> bf16 R^T (cols 0-31) and -dM^T (32-63) -> [dA dB; dQX dQP] -> [dx_r^T | dp_r^T]
+  //   Y: R^T (0-63), M^T (64-127) -> dV^T (0-63)
+  //   Z: dM^T (0-63), dR^T (64-127) -> [dk_r^T | dq_r^T]
+  const uint32_t tmAcc = tmem, tmX = tmem + 128, tmY = tmem + 256, tmZ = tmem + 384;
+  const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+  uint32_t it = 0;     // chunks processed by this CTA: the parity of the MMA barriers
+  uint32_t ld_it = 0;  // load phases consumed (a chunk outside the range consumes one, no MMA phase)
+
+  const Tout *g_do = static_cast<const Tout *>(P.dO);
+  const __nv_bfloat16 *g_w = kTied ? P.b : P.w;
+  Tout *g_dq = static_cast<Tout *>(P.dq), *g_dk = static_cast<Tout *>(P.dk), *g_dv = static_cast<Tout *>(P.dv);
+  Tout *g_dla = static_cast<Tout *>(P.dlog_a), *g_db = static_cast<Tout *>(P.db), *g_dw = static_cast<Tout *>(P.dw);
+
+  // the raw k, q, v, log_a, b (, w, dO) tiles of the chunk at token t0 of head h, and its S_r
+  // tile image (thread kIssuer)
+  constexpr bool kDoTma = sizeof(Tout) == 2;  // bf16 dO lands in its tile as it is
+  auto issue_loads = [&](int h, int t0, const uint8_t *sr_img) {
+    ptx::mbar_arrive_expect_tx(bar(BAR_LD), ((kTied ? 5u : 6u) + (kDoTma ? 1u : 0u)) * 16384u + 32768u);
+    *sIss = *sIss + 1u;
+    ptx::bulk_load(sb + OFF_SR, sr_img, 32768u, bar(BAR_LD));
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) {
+      const uint32_t o = (uint32_t)kb * 16384u;
+      ptx::tma_load_3d(sb + OFF_KQ + o, &P.tm_k, kb * 64, h, t0, bar(BAR_LD));
+      ptx::tma_load_3d(sb + OFF_KQ + o + 8192u, &P.tm_q, kb * 64, h, t0, bar(BAR_LD));
+      ptx::tma_load_3d(sb + OFF_MV + o + 8192u, &P.tm_v, kb * 64, h, t0, bar(BAR_LD));
+      ptx::tma_load_3d(sb + OFF_GRAW + (uint32_t)kb * 8192u, &P.tm_g, kb * 64, h, t0, bar(BAR_LD));
+      ptx::tma_load_3d(sb + OFF_XP + o, &P.tm_b, kb * 64, h, t0, bar(BAR_LD));
+      if (!kTied) ptx::tma_load_3d(sb + OFF_XP + o + 8192u, &P.tm_w, kb * 64, h, t0, bar(BAR_LD));
+      if (kDoTma) ptx::tma_load_3d(sb + OFF_RO + o + 8192u, &P.tm_do, kb * 64, h, t0, bar(BAR_LD));
+    }
+  };
+
+  for (;;) {
+    if (tid == 0) *sUnit = atomicAdd(P.counter, 1);
+    __syncthreads();
+    const int u = *sUnit;
+    if (u >= P.n_units || *sAbort) break;
+    const int unit = P.schedule ? P.schedule[u] : u;
+    const int n = unit / H, h = unit % H;
+    int64_t bos, len;
+    if (P.cu_seqlens) {
+      bos = P.cu_seqlens[n];
+      len = (int64_t)P.cu_seqlens[n + 1] - bos;
+    } else {
+      bos = (int64_t)n * P.seq_len;
+      len = P.seq_len;
+    }
+    const int nchunks = (int)((len + C - 1) / C);
+    const uint8_t *ck_unit = P.ckpt + ckpt_first_slot(P.ckpt_off, n, h, H, nchunks) * (size_t)(D * D * 2);
+
+    // ---- the final state's adjoint dS_T into TMEM (thread: d_k channel `row`, d_v channels
+    //      [32 cg, 32 cg + 32)), and the decay term of the last chunk, sum_j dS_T S_T per d_k
+    //      channel (S_T: the forward's final state)
+    {
+      uint32_t r[32];
+      float acc = 0.f;
+      const size_t o = ((size_t)unit * D + row) * D + cg * 32;
+#pragma unroll
+      for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 a = P.dS_T ? *reinterpret_cast<const float4 *>(P.dS_T + o + 4 * j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 st = *reinterpret_cast<const float4 *>(P.S_fin + o + 4 * j4);
+        r[4 * j4] = __float_as_uint(a.x);
+        r[4 * j4 + 1] = __float_as_uint(a.y);
+        r[4 * j4 + 2] = __float_as_uint(a.z);
+        r[4 * j4 + 3] = __float_as_uint(a.w);
+        acc += a.x * st.x + a.y * st.y + a.z * st.z + a.w * st.w;
+      }
+      ptx::tmem_st32(tmAcc + lane_base + cg * 32, r);
+      ptx::tmem_wait_st();
+      rs[cg * 128 + row] = acc;
+      if (tid < 128) sEsr[((it & 1u) ^ 1u) * 128 + tid] = 1.f;  // the last chunk reads dS_T unscaled
+      // the last chunk's tiles (every tile is free: the previous unit's MMAs are done)
+      if (tid == kIssuer && nchunks > 0 && !*sAbort)
+        issue_loads(h, (int)(bos + (int64_t)(nchunks - 1) * C), ck_unit + (size_t)(nchunks - 1) * (D * D * 2));
+    }
+    __syncthreads();
+    if (tid < 128)
+      sDlc[(it & 1u) * 128 + tid] = ((rs[tid] + rs[128 + tid]) + rs[256 + tid]) + rs[384 + tid];
+
+    bool unit_ok = true;
+    int lastpar = -1;  // parity of the last chunk processed (chunk 0): its e^{rho} gives dS0
+    for (int ci = nchunks - 1; ci >= 0; --ci) {
+      const uint32_t par = it & 1u;
+      const int t0 = (int)(bos + (int64_t)ci * C);
+      const int nvalid = (int)((len - (int64_t)ci * C) < C ? (len - (int64_t)ci * C) : C);
+
+      // ================= phase 1: loads, cumulative decay, operand tiles
+      if (ci > 0) {  // the next chunk's rows and state to L2 while this chunk runs
+        if (tid < 448) {
+          const int tsel = tid >> 6, r = tid & 63;
+          const size_t gi = ((size_t)(t0 - C + r) * H + h) * D;
+          const void *src = tsel == 0 ? (const void *)(P.q + gi) : tsel == 1 ? (const void *)(P.k + gi)
+                          : tsel == 2 ? (const void *)(P.v + gi) : tsel == 3 ? (const void *)(P.log_a + gi)
+                          : tsel == 4 ? (const void *)(P.b + gi) : tsel == 5 ? (const void *)(g_w + gi)
+                                      : (const void *)(g_do + gi);
+          if (tsel != 5 || !kTied) ptx::bulk_prefetch_l2(src, tsel == 6 ? D * (uint32_t)sizeof(Tout) : D * 2u);
+        } else if (tid < 450) {
+          ptx::bulk_prefetch_l2(ck_unit + (size_t)(ci - 1) * (D * D * 2) + (size_t)(tid - 448) * 16384, 16384u);
+        }
+      }
+      // fp32 dO: the rows of channel `row` into the bf16 tile (rows past the chunk end re-read
+      // its last row and are zeroed); the dO rows of the tile are free since the previous
+      // chunk's products.  bf16 dO arrives with the other tiles.
+      if (!kDoTma) {
+        Tout dov[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const int r = 16 * cg + t, rc = r < nvalid ? r : nvalid - 1;
+          dov[t] = g_do[((size_t)(t0 + rc) * H + h) * D + row];
+        }
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const int r = 16 * cg + t;
+          sts_u16(sb + OFF_RO + 8192u + swz_elem(r, row, 16384u), bf16_bits(r < nvalid ? to_f32<Tout>(dov[t]) : 0.f));
+        }
+      }
+      waitb(bar(BAR_LD), ld_it & 1u);
+      ++ld_it;
+      // cumulative log-decay of channel `row` over rows [16 cg, 16 cg + 16) (rows past the chunk
+      // end decay by nothing; their V rows are zeroed); the dO rows go to their tile
+      float Lloc[16];
+      {
+        float acc = 0.f;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const int r = 16 * cg + t;
+          const uint32_t o = swz_elem(r, row, 16384u);
+          const float la = r < nvalid ? bf16_value(lds_u16(sb + OFF_GRAW + swz_elem(r, row, 8192u))) : 0.f;
+          acc += la;
+          Lloc[t] = acc;
+          if (r >= nvalid) {
+            sts_u16(sb + OFF_MV + 8192u + o, 0);
+            if (kDoTma) sts_u16(sb + OFF_RO + 8192u + o, 0);
+          }
+        }
+        part[cg * 128 + row] = acc;
+        if (cg == 0) sL0[row] = Lloc[0];
+      }
+      if (tid == 0) *sWide = 0;
+      __syncthreads();
+      float pre, rho;
+      {
+        float tot;
+        rho = rho_of(row, tot);
+        pre = cg == 0 ? 0.f : part[row];
+        if (cg > 1) pre += part[128 + row];
+        if (cg > 2) pre += part[256 + row];
+        if (cg == 0) {
+          if (!(sL0[row] - tot <= kFastSpan)) *sWide = 1;
+          sRho[row] = rho;
+          sEsr[par * 128 + row] = ptx::ex2(rho * kLog2eF);
+        }
+        lpre[cg * 128 + row] = pre;
+      }
+      // k_r, q_r, x_r, p_r over the raw k, q, b, w rows (rows past the chunk end are zeroed)
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        const int r = 16 * cg + t;
+        const uint32_t o0 = swz_elem(r, row, 16384u), o1 = swz_elem(64 + r, row, 16384u);
+        float kk = 0.f, qq = 0.f, bb = 0.f, ww = 0.f;
+        if (r < nvalid) {
+          kk = bf16_value(lds_u16(sb + OFF_KQ + o0));
+          qq = bf16_value(lds_u16(sb + OFF_KQ + o1));
+          bb = bf16_value(lds_u16(sb + OFF_XP + o0));
+          ww = kTied ? bb : bf16_value(lds_u16(sb + OFF_XP + o1));
+        }
+        const float L = pre + Lloc[t];
+        const float e = ptx::ex2((L - rho) * kLog2eF), f = ptx::ex2((rho - L) * kLog2eF);
+        sts_u16(sb + OFF_KQ + o0, bf16_bits(kk * e));
+        sts_u16(sb + OFF_KQ + o1, bf16_bits(qq * e));
+        sts_u16(sb + OFF_XP + o0, bf16_bits(bb * kk * f));
+        sts_u16(sb + OFF_XP + o1, bf16_bits(ww * kk * f));
+      }
+      // Lam_g = Diag(gamma e^{rho_next}) Acc, the bf16 tile [d_k rows][d_v] and the fp32 base of
+      // this chunk's adjoint update (thread: d_k channel `row`, d_v channels [32 cg, 32 cg + 32))
+      {
+        float tot;
+        const float ri = rho_of(row, tot);
+        const float gam = ptx::ex2((tot - ri) * kLog2eF);
+        const float efac = sEsr[(par ^ 1u) * 128 + row];
+        uint32_t r[32];
+        float lg[32];
+        ptx::tmem_ld32(tmAcc + lane_base + cg * 32, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          lg[j] = (__uint_as_float(r[j]) * efac) * gam;  // e^{rho_next} first: the adjoint, O(1)
+          r[j] = __float_as_uint(lg[j]);
+        }
+        ptx::tmem_st32(tmAcc + lane_base + cg * 32, r);
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8)
+          sts_v4(sb + OFF_LG + (uint32_t)(cg >> 1) * 16384u + swz(row, (uint32_t)((cg & 1) * 4 + q8)), pack8(lg + 8 * q8, 1.f));
+        ptx::tmem_wait_st();
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      __syncthreads();
+      if (*sWide) {  // outside the factored form: recorded, the rest of the unit is left
+        if (tid == 0) atomicExch(P.status, kStatusRange);
+        unit_ok = false;
+        break;
+      }
+
+      // ================= phase 2: G1 and dM^T <- Lam_g^T x_r^T; masks
+      if (tid == kIssuer && !*sAbort) {
+        ptx::tc_fence_after();
+        constexpr uint32_t idG1 = ptx::idesc_bf16(128, 128, false, false);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmX, kmaj(sb + OFF_KQ, kk), kmaj(sb + OFF_XP, kk), idG1, kk > 0);
+        ptx::umma_commit(bar(BAR_G1));
+        constexpr uint32_t idM = ptx::idesc_bf16(128, 64, true, false);  // A = Lam_g^T (MN-major), B = x_r
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmZ, mnmaj(sb + OFF_LG, kk), kmaj(sb + OFF_XP, kk), idM, kk > 0);
+      }
+      // the bf16 T tile (over the -M rows, free until phase 5) starts as zeros: the solve writes
+      // only the blocks on and below the diagonal
+      sts_v4(sb + OFF_T + 16u * (uint32_t)tid, make_uint4(0u, 0u, 0u, 0u));
+      waitb(bar(BAR_G1), par);
+      ptx::tc_fence_after();
+      {
+        // warp (qd, cg) reads G1 row `row`, columns [32 cg, 32 cg + 32): A | B for rows 0-63,
+        // QX | QP for rows 64-127; A, B strictly lower, QX, QP lower with the diagonal
+        uint32_t r[32];
+        ptx::tmem_ld32(tmX + lane_base + cg * 32, r);
+        ptx::tmem_wait_ld();
+        const int i = row & 63, jb = (cg & 1) * 32;
+        const bool strict = row < 64;
+        float f[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) f[j] = (strict ? jb + j < i : jb + j <= i) ? __uint_as_float(r[j]) : 0.f;
+        if (strict && cg < 2) {  // A in fp32 for the solve
+#pragma unroll
+          for (int j4 = 0; j4 < 8; ++j4)
+            *reinterpret_cast<float4 *>(at(i, jb + 4 * j4)) =
+                make_float4(f[4 * j4], f[4 * j4 + 1], f[4 * j4 + 2], f[4 * j4 + 3]);
+        } else {
+          // B into rows 0-63 of [B; QP]; QX into its own tile; QP into rows 64-127 of [B; QP]
+          const uint32_t dst = strict ? sb + OFF_BQP : (cg < 2 ? sb + OFF_QX : sb + OFF_BQP + 8192u);
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) sts_v4(dst + swz(i, (uint32_t)((cg & 1) * 4 + q8)), pack8(f + 8 * q8, 1.f));
+        }
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      __syncthreads();
+
+      // ================= phase 3: T = (I + A)^-1 (warps 0-14) || R^T, dM^T += dO^T QX (warp 15)
+      if (warp == 15) {
+        if (lane == 0 && !*sAbort) {
+          ptx::tc_fence_after();
+          // R^T = V^T B^T + S_r^T k_r^T
+          constexpr uint32_t idV = ptx::idesc_bf16(128, 64, true, false);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::umma_bf16(tmY, ptx::sdesc_sw128(sb + OFF_MV + 8192u + (uint32_t)kk * 2048u, 16384, 1024),
+                           ptx::sdesc_sw128(sb + OFF_BQP + (uint32_t)kk * 32u, 16, 1024), idV, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmY, mnmaj(sb + OFF_SR, kk), kmaj(sb + OFF_KQ, kk), idV, 1);
+          // dM^T += dO^T QX (QX as [s][t]: MN-major B)
+          constexpr uint32_t idQ = ptx::idesc_bf16(128, 64, true, true);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::umma_bf16(tmZ, ptx::sdesc_sw128(sb + OFF_RO + 8192u + (uint32_t)kk * 2048u, 16384, 1024),
+                           ptx::sdesc_sw128(sb + OFF_QX + (uint32_t)kk * 2048u, 8192, 1024), idQ, 1);
+          ptx::umma_commit(bar(BAR_GA));
+        }
+        __syncwarp();
+      } else {
+        // 8x8 diagonal blocks by forward substitution (one thread per block column), then
+        // merges of block pairs of size s = 8, 16, 32: T_LU = -T_LL (A_LU T_UU).  A and T
+        // share one fp32 array: a block of T overwrites the block of A it came from once no
+        // thread reads that block any more.  Every final block also goes to the bf16 tile.
+        float a[28];
+        const int blk = tid >> 3, m = tid & 7, r0 = 8 * blk;
+        if (tid < 64) {
+          int nn = 0;
+#pragma unroll
+          for (int ii = 1; ii < 8; ++ii)
+#pragma unroll
+            for (int jj = 0; jj < ii; ++jj) a[nn++] = *at(r0 + ii, r0 + jj);
+        }
+        named_bar(NB_SOLVE, kSolveThreads);
+        if (tid < 64) {
+          float t[8];
+          int nn = 0;
+#pragma unroll
+          for (int ii = 0; ii < 8; ++ii) {
+            float acc = (ii == m) ? 1.f : 0.f;
+#pragma unroll
+            for (int jj = 0; jj < ii; ++jj) acc -= a[nn++] * t[jj];
+            t[ii] = acc;
+          }
+#pragma unroll
+          for (int ii = 0; ii < 8; ++ii) {
+            *at(r0 + ii, r0 + m) = t[ii];
+            sts_u16(sb + OFF_T + swz(r0 + ii, (uint32_t)blk) + (uint32_t)m * 2u, bf16_bits(t[ii]));
+          }
+        }
+        named_bar(NB_SOLVE, kSolveThreads);
+        float *Xs = reinterpret_cast<float *>(gb + OFF_XS);
+        // s = 8: 4 pairs x 64 outputs on CUDA cores
+        if (tid < 256) {
+          const int pr = tid >> 6, r = (tid >> 3) & 7, c = tid & 7, u0 = 16 * pr, l0 = u0 + 8;
+          float acc = 0.f;
+#pragma unroll
+          for (int k2 = 0; k2 < 8; ++k2) acc += (k2 >= c ? *at(l0 + r, u0 + k2) * *at(u0 + k2, u0 + c) : 0.f);
+          Xs[tid] = acc;
+        }
+        named_bar(NB_SOLVE, kSolveThreads);
+        if (tid < 256) {
+          const int pr = tid >> 6, r = (tid >> 3) & 7, c = tid & 7, u0 = 16 * pr, l0 = u0 + 8;
+          float acc = 0.f;
+#pragma unroll
+          for (int k2 = 0; k2 < 8; ++k2) acc -= (k2 <= r ? *at(l0 + r, l0 + k2) * Xs[pr * 64 + k2 * 8 + c] : 0.f);
+          *at(l0 + r, u0 + c) = acc;
+          sts_u16(sb + OFF_T + swz(l0 + r, (uint32_t)(u0 >> 3)) + (uint32_t)c * 2u, bf16_bits(acc));
+        }
+        named_bar(NB_SOLVE, kSolveThreads);
+        // s = 16 (2 pairs) and s = 32 (1 pair) on tf32 mma.sync, one warp per 16x8 output tile;
+        // each K step's fragments are loaded right before its MMA (few registers live)
+        const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+        for (int lev = 1; lev < 3; ++lev) {
+          const int sz = 8 << lev;                   // 16, 32
+          const int nk = sz / 8;                     // 8-wide K steps: 2, 4
+          const int tpp = (sz / 16) * (sz / 8);      // 16x8 tiles per pair: 2, 8
+          const int ntiles = (64 / (2 * sz)) * tpp;  // 4, 8
+          const int pr = warp / tpp, ti = warp % tpp, mt = ti / (sz / 8), nt = ti % (sz / 8);
+          const int u0 = pr * 2 * sz, l0 = u0 + sz, rr = 16 * mt, cc = 8 * nt;
+          // X = A_LU T_UU (T_UU is lower triangular: K steps before the tile's first column vanish)
+          if (warp < ntiles) {
+            float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              if (kk < nk && kk >= nt) {
+                const int kc = u0 + 8 * kk + t4;
+                const uint32_t av[4] = {ptx::to_tf32(*at(l0 + rr + g, kc)), ptx::to_tf32(*at(l0 + rr + g + 8, kc)),
+                                        ptx::to_tf32(*at(l0 + rr + g, kc + 4)), ptx::to_tf32(*at(l0 + rr + g + 8, kc + 4))};
+                const uint32_t bv[2] = {ptx::to_tf32(*at(kc, u0 + cc + g)), ptx::to_tf32(*at(kc + 4, u0 + cc + g))};
+                ptx::mma_tf32_16x8x8(x, av, bv);
+              }
+            }
+            float *xs = Xs + pr * sz * sz;
+            xs[(rr + g) * sz + cc + 2 * t4] = x[0];
+            xs[(rr + g) * sz + cc + 2 * t4 + 1] = x[1];
+            xs[(rr + g + 8) * sz + cc + 2 * t4] = x[2];
+            xs[(rr + g + 8) * sz + cc + 2 * t4 + 1] = x[3];
+          }
+          named_bar(NB_SOLVE, kSolveThreads);
+          // T_LU = -T_LL X (K steps past the tile's last row vanish), over A_LU
+          if (warp < ntiles) {
+            const float *xs = Xs + pr * sz * sz;
+            float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              if (kk < nk && kk <= (rr + 15) / 8) {
+                // T_LL is lower triangular (its blocks above the diagonal hold zeros of A)
+                const int kc = l0 + 8 * kk + t4;
+                const uint32_t av[4] = {ptx::to_tf32(*at(l0 + rr + g, kc)), ptx::to_tf32(*at(l0 + rr + g + 8, kc)),
+                                        ptx::to_tf32(*at(l0 + rr + g, kc + 4)), ptx::to_tf32(*at(l0 + rr + g + 8, kc + 4))};
+                const uint32_t bv[2] = {ptx::to_tf32(xs[(8 * kk + t4) * sz + cc + g]),
+                                        ptx::to_tf32(xs[(8 * kk + t4 + 4) * sz + cc + g])};
+                ptx::mma_tf32_16x8x8(y, av, bv);
+              }
+            }
+            const int ri = l0 + rr + g, cj = u0 + cc + 2 * t4;
+            if (lev == 1) {  // the last level's T_LU is read by no later level: bf16 only
+              *at(ri, cj) = -y[0];
+              *at(ri, cj + 1) = -y[1];
+              *at(ri + 8, cj) = -y[2];
+              *at(ri + 8, cj + 1) = -y[3];
+            }
+            sts_u32(sb + OFF_T + swz(ri, (uint32_t)(cj >> 3)) + (uint32_t)(cj & 7) * 2u, pack_bf16x2(-y[0], -y[1]));
+            sts_u32(sb + OFF_T + swz(ri + 8, (uint32_t)(cj >> 3)) + (uint32_t)(cj & 7) * 2u, pack_bf16x2(-y[2], -y[3]));
+          }
+          if (lev == 1) named_bar(NB_SOLVE, kSolveThreads);
+        }
+        ptx::fence_proxy_async_smem();  // the bf16 T tile is read by the tensor core
+      }
+      ptx::tc_fence_before();
+      __syncthreads();
+
+      // ================= phase 4: R^T and -dM^T as bf16 TMEM operands; M^T, dR^T
+      waitb(bar(BAR_GA), par);
+      ptx::tc_fence_after();
+      {
+        uint32_t r[16], hb[8];
+        ptx::tmem_ld16(tmY + lane_base + cg * 16, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) hb[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+        ptx::tmem_st8(tmX + lane_base + cg * 8, hb);
+        ptx::tmem_ld16(tmZ + lane_base + cg * 16, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) hb[j] = pack_bf16x2(-__uint_as_float(r[2 * j]), -__uint_as_float(r[2 * j + 1]));
+        ptx::tmem_st8(tmX + 32 + lane_base + cg * 8, hb);
+        ptx::tmem_wait_st();
+      }
+      ptx::tc_fence_before();
+      __syncthreads();
+      if (tid == kIssuer && !*sAbort) {
+        ptx::tc_fence_after();
+        // M^T = R^T T^T (B = T as [t][s], K-major); dR^T = dM^T T (B = T as [s][t], MN-major)
+        constexpr uint32_t idK = ptx::idesc_bf16(128, 64, false, false);
+        constexpr uint32_t idN = ptx::idesc_bf16(128, 64, false, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::umma_bf16_ts(tmY + 64, tmX + (uint32_t)kk * 8u, ptx::sdesc_sw128(sb + OFF_T + (uint32_t)kk * 32u, 16, 1024),
+                            idK, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::umma_bf16_ts(tmZ + 64, tmX + 32u + (uint32_t)kk * 8u,
+                            ptx::sdesc_sw128(sb + OFF_T + (uint32_t)kk * 2048u, 8192, 1024), idN, kk > 0);
+        ptx::umma_commit(bar(BAR_GB));
+      }
+
+      // ================= phase 5: -M and dR to their tiles ([t][j], over T, QX and the solve array)
+      waitb(bar(BAR_GB), par);
+      ptx::tc_fence_after();
+      {
+        uint32_t r[16];
+        ptx::tmem_ld16(tmY + 64 + lane_base + cg * 16, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          sts_u16(sb + OFF_MV + swz_elem(cg * 16 + j, row, 16384u), bf16_bits(-__uint_as_float(r[j])));
+        ptx::tmem_ld16(tmZ + 64 + lane_base + cg * 16, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          sts_u16(sb + OFF_RO + swz_elem(cg * 16 + j, row, 16384u), bf16_bits(__uint_as_float(r[j])));
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      __syncthreads();
+
+      // ================= phase 6: [dA dB; dQX dQP] = [dR; dO][-M; V]^T, the adjoint update
+      //      Acc += [k_r; q_r]^T [dR; dO], dV^T = [dR; dO]^T [B; QP] + Lam_g^T p_r^T and the
+      //      S_r terms [dk_r^T | dq_r^T] = S_r [dR; dO]^T
+      if (tid == kIssuer && !*sAbort) {
+        ptx::tc_fence_after();
+        constexpr uint32_t idKK = ptx::idesc_bf16(128, 128, false, false);
+        constexpr uint32_t idNN = ptx::idesc_bf16(128, 128, true, true);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmX, kmaj(sb + OFF_RO, kk), kmaj(sb + OFF_MV, kk), idKK, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmAcc, mnmaj(sb + OFF_KQ, kk), mnmaj(sb + OFF_RO, kk), idNN, 1);
+        constexpr uint32_t idV1 = ptx::idesc_bf16(128, 64, true, true);
+        constexpr uint32_t idV2 = ptx::idesc_bf16(128, 64, true, false);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          ptx::umma_bf16(tmY, mnmaj(sb + OFF_RO, kk), ptx::sdesc_sw128(sb + OFF_BQP + (uint32_t)kk * 2048u, 8192, 1024),
+                         idV1, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmY, mnmaj(sb + OFF_LG, kk), kmaj(sb + OFF_XP + 8192u, kk), idV2, 1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmZ, kmaj(sb + OFF_SR, kk), kmaj(sb + OFF_RO, kk), idKK, kk > 0);
+        ptx::umma_commit(bar(BAR_G5));
+      }
+
+      // ================= phase 7: the previous chunk's decay term, dV, the gradient-tile masks
+      waitb(bar(BAR_G5), par);
+      ptx::tc_fence_after();
+      if (ci > 0) {
+        // sum_j Lam_{c-1}[i][j] S_c[i][j] = sum_j Acc[i][j] S_r[i][j] (Lam_{c-1} = e^{rho} Acc):
+        // thread (d_k channel `row`, d_v channels [32 cg, 32 cg + 32)), summed over the four
+        // column groups by the chunk before
+        uint32_t r[32];
+        ptx::tmem_ld32(tmAcc + lane_base + cg * 32, r);
+        ptx::tmem_wait_ld();
+        float acc = 0.f;
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          const uint4 sv = lds_v4(sb + OFF_SR + (uint32_t)(cg >> 1) * 16384u + swz(row, (uint32_t)((cg & 1) * 4 + q8)));
+          const uint32_t w4[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float2 f = unpack_bf16x2(w4[e2]);
+            acc = fmaf(__uint_as_float(r[8 * q8 + 2 * e2]), f.x, acc);
+            acc = fmaf(__uint_as_float(r[8 * q8 + 2 * e2 + 1]), f.y, acc);
+          }
+        }
+        rs[cg * 128 + row] = acc;
+      }
+      {  // dV (= dZ: the values enter unscaled); thread: d_v channel `row`, tokens [16 cg, 16 cg + 16)
+        uint32_t r[16];
+        ptx::tmem_ld16(tmY + lane_base + cg * 16, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int t = cg * 16 + j;
+          if (t < nvalid) g_dv[((size_t)(t0 + t) * H + h) * D + row] = from_f32<Tout>(__uint_as_float(r[j]));
+        }
+      }
+      __syncthreads();  // S_r is read; its space takes the gradient tile
+      if (ci > 0 && tid < 128)
+        sDlc[(par ^ 1u) * 128 + tid] = ((rs[tid] + rs[128 + tid]) + rs[256 + tid]) + rs[384 + tid];
+      {
+        // row `row` of [dA dB; dQX dQP], columns [32 cg, 32 cg + 32): strictly lower for the dR
+        // rows, lower with the diagonal for the dO rows; stored as [column block][row][64]
+        uint32_t r[32];
+        ptx::tmem_ld32(tmX + lane_base + cg * 32, r);
+        ptx::tmem_wait_ld();
+        const int i = row & 63, jb = (cg & 1) * 32;
+        const bool strict = row < 64;
+        float f[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) f[j] = (strict ? jb + j < i : jb + j <= i) ? __uint_as_float(r[j]) : 0.f;
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8)
+          sts_v4(sb + OFF_DG + (uint32_t)(cg >> 1) * 16384u + swz(row, (uint32_t)((cg & 1) * 4 + q8)), pack8(f + 8 * q8, 1.f));
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      __syncthreads();
+
+      // ================= phase 8: [dx_r^T | dp_r^T] = [k_r; q_r]^T dG + Lam_g [-M; V]^T,
+      //      [dk_r^T | dq_r^T] += [x_r; p_r]^T dG^T
+      if (tid == kIssuer && !*sAbort) {
+        ptx::tc_fence_after();
+        constexpr uint32_t idNN = ptx::idesc_bf16(128, 128, true, true);
+        constexpr uint32_t idKK = ptx::idesc_bf16(128, 128, false, false);
+        constexpr uint32_t idNK = ptx::idesc_bf16(128, 128, true, false);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmX, mnmaj(sb + OFF_KQ, kk), mnmaj(sb + OFF_DG, kk), idNN, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmX, kmaj(sb + OFF_LG, kk), kmaj(sb + OFF_MV, kk), idKK, 1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmZ, mnmaj(sb + OFF_XP, kk), kmaj(sb + OFF_DG, kk), idNK, 1);
+        ptx::umma_commit(bar(BAR_G7));
+      }
+      waitb(bar(BAR_G7), par);
+      ptx::tc_fence_after();
+      // every tile is free (the epilogue reads TMEM and global memory only): the next chunk's
+      // raw tiles land while this chunk's gradients are formed and stored
+      if (tid == kIssuer && ci > 0 && !*sAbort) issue_loads(h, t0 - C, ck_unit + (size_t)(ci - 1) * (D * D * 2));
+
+      // ================= phase 9: chain rule and stores.  Thread: d_k channel i = `row`, tokens
+      //      [16 cg, 16 cg + 16).  The cumulative decay is recomputed as phase 1 computed it.
+      {
+        const int i = row;
+        const float pre = lpre[cg * 128 + i], rho = sRho[i], dlc = sDlc[par * 128 + i];
+        float dL[16];
+        float loc = 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int c0 = cg * 16 + half * 8;
+          asm volatile("" ::: "memory");
+          uint32_t vx[8], vp[8], vk[8], vq[8];
+          ptx::tmem_ld8(tmX + lane_base + (uint32_t)c0, vx);
+          ptx::tmem_ld8(tmX + lane_base + 64u + (uint32_t)c0, vp);
+          ptx::tmem_ld8(tmZ + lane_base + (uint32_t)c0, vk);
+          ptx::tmem_ld8(tmZ + lane_base + 64u + (uint32_t)c0, vq);
+          // the raw inputs of the 8 rows, all requested before any is used (rows past the
+          // chunk end re-read its last row and are ignored)
+          __nv_bfloat16 rla[8], rk[8], rq[8], rb[8], rw[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int t = c0 + j, tc = t < nvalid ? t : nvalid - 1;
+            const size_t gi = ((size_t)(t0 + tc) * H + h) * D + i;
+            rla[j] = P.log_a[gi];
+            rk[j] = P.k[gi];
+            rq[j] = P.q[gi];
+            rb[j] = P.b[gi];
+            rw[j] = kTied ? rb[j] : g_w[gi];
+          }
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int t = c0 + j;
+            const bool valid = t < nvalid;
+            const float la = valid ? bf(rla[j]) : 0.f, kk = valid ? bf(rk[j]) : 0.f, qq = valid ? bf(rq[j]) : 0.f;
+            const float bb = valid ? bf(rb[j]) : 0.f, ww = valid ? bf(rw[j]) : 0.f;
+            loc += la;
+            const float L = pre + loc;
+            const float e = ptx::ex2((L - rho) * kLog2eF), f = ptx::ex2((rho - L) * kLog2eF);
+            const float dxr = __uint_as_float(vx[j]), dpr = __uint_as_float(vp[j]);
+            const float dkr = __uint_as_float(vk[j]), dqr = __uint_as_float(vq[j]);
+            const float dx = dxr * f, dp = dpr * f;
+            float dLt = e * (dqr * qq + dkr * kk) - f * kk * (dxr * bb + dpr * ww);
+            if (t == C - 1) dLt += dlc;
+            dL[half * 8 + j] = dLt;
+            if (valid) {
+              const size_t gi = ((size_t)(t0 + t) * H + h) * D + i;
+              g_dq[gi] = from_f32<Tout>(dqr * e);
+              g_dk[gi] = from_f32<Tout>(dkr * e + bb * dx + ww * dp);
+              if (kTied) {
+                g_db[gi] = from_f32<Tout>(kk * (dx + dp));
+              } else {
+                g_db[gi] = from_f32<Tout>(kk * dx);
+                g_dw[gi] = from_f32<Tout>(kk * dp);
+              }
+            }
+          }
+        }
+        // d log_a_s = sum_{t >= s} dL_t: suffix sums inside the thread's 16 rows, then the
+        // totals of the later row groups
+        float suf = 0.f;
+#pragma unroll
+        for (int j = 15; j >= 0; --j) {
+          suf += dL[j];
+          dL[j] = suf;
+        }
+        part[cg * 128 + i] = suf;
+        __syncthreads();
+        float above = 0.f;
+        for (int g = 3; g > cg; --g) above += part[g * 128 + i];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int t = cg * 16 + j;
+          if (t < nvalid) g_dla[((size_t)(t0 + t) * H + h) * D + i] = from_f32<Tout>(dL[j] + above);
+        }
+      }
+      ptx::tc_fence_before();
+      __syncthreads();  // part and the TMEM work areas are reused by the next chunk
+      lastpar = (int)par;
+      ++it;
+      if (*sAbort) break;
+    }
+
+    // ---- dS0 = Diag(e^{rho_0}) Acc (the first chunk's adjoint update has landed)
+    if (unit_ok && !*sAbort && P.dS0) {
+      uint32_t r[32];
+      ptx::tmem_ld32(tmAcc + lane_base + cg * 32, r);
+      ptx::tmem_wait_ld();
+      float4 *dst = reinterpret_cast<float4 *>(P.dS0 + ((size_t)unit * D + row) * D + cg * 32);
+      const float es = lastpar >= 0 ? sEsr[lastpar * 128 + row] : 1.f;
+#pragma unroll
+      for (int j4 = 0; j4 < 8; ++j4)
+        dst[j4] = make_float4(__uint_as_float(r[4 * j4]) * es, __uint_as_float(r[4 * j4 + 1]) * es,
+                              __uint_as_float(r[4 * j4 + 2]) * es, __uint_as_float(r[4 * j4 + 3]) * es);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+  }
+
+  if (*sAbort) {
+    // wind-down after a timed-out wait: let the MMAs the issuing thread queued finish (bounded)
+    // before the tensor memory is freed
+    if (tid == kIssuer) {
+      ptx::umma_commit(bar(BAR_DRAIN));
+      drain_bar(bar(BAR_DRAIN), 0u, P.wait_ns);
+      if (*sIss > 0u) drain_bar(bar(BAR_LD), (*sIss - 1u) & 1u, P.wait_ns);  // the last armed load phase
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 0) ptx::tmem_dealloc(tmem, kTmemCols);
+}
+
+// off[n] = sum over m < n of ceil(len_m / 64), off[N] the total: the first checkpoint
+// slot of each sequence divided by the head count.  One block; each thread owns a contiguous
+// range of sequences.
+__global__ void ckpt_offsets_kernel(const int32_t *cu, int N, int64_t *off) {
+  __shared__ int64_t sums[1024];
+  const int per = (N + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int a = (int)threadIdx.x * per, e = a + per < N ? a + per : N;
+  int64_t s = 0;
+  for (int n = a; n < e; ++n) s += (cu[n + 1] - cu[n] + C - 1) / C;
+  sums[threadIdx.x] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int64_t run = 0;
+    for (int i = 0; i < (int)blockDim.x; ++i) {
+      const int64_t v = sums[i];
+      sums[i] = run;
+      run += v;
+    }
+    off[N] = run;
+  }
+  __syncthreads();
+  int64_t run = sums[threadIdx.x];
+  for (int n = a; n < e; ++n) {
+    off[n] = run;
+    run += (cu[n + 1] - cu[n] + C - 1) / C;
+  }
+}
+
+template <typename Tout, bool kTied>
+cudaError_t launch_t(const BwdTcParams &P, int grid, cudaStream_t stream) {
+  auto kern = bwd_tc_kernel<Tout, kTied>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, kSmemBytes, stream>>>(P);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t bwd_tc_ckpt_slots(int64_t n_seqs, int64_t t_total, int n_heads, bool packed, int seq_len) {
+  if (packed) return (size_t)n_heads * (size_t)(t_total / C + n_seqs);  // sum of ceil(len / 64) <= T/64 + N
+  return (size_t)n_heads * (size_t)n_seqs * (size_t)((seq_len + C - 1) / C);
+}
+
+cudaError_t launch_ckpt_offsets(const int32_t *cu_seqlens, int n_seqs, int64_t *off, cudaStream_t stream) {
+  ckpt_offsets_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, n_seqs, off);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_tc(const BwdProblem &p, const void *ckpt, const float *S_fin, const int64_t *ckpt_off,
+                          const int32_t *schedule, int32_t *status, int32_t *counter, cudaStream_t stream) {
+  BwdTcParams P;
+  memset(&P, 0, sizeof(P));
+  P.q = static_cast<const __nv_bfloat16 *>(p.q);
+  P.k = static_cast<const __nv_bfloat16 *>(p.k);
+  P.v = static_cast<const __nv_bfloat16 *>(p.v);
+  P.log_a = static_cast<const __nv_bfloat16 *>(p.log_a);
+  P.b = static_cast<const __nv_bfloat16 *>(p.b);
+  P.w = static_cast<const __nv_bfloat16 *>(p.w);
+  P.dO = p.dO;
+  P.dS_T = p.dS_T;
+  P.dq = p.dq; P.dk = p.dk; P.dv = p.dv; P.dlog_a = p.dlog_a; P.db = p.db; P.dw = p.dw;
+  P.dS0 = p.dS0;
+  P.ckpt = static_cast<const uint8_t *>(ckpt);
+  P.S_fin = S_fin;
+  P.ckpt_off = ckpt_off;
+  P.cu_seqlens = p.cu_seqlens;
+  P.schedule = schedule;
+  P.status = status;
+  P.counter = counter;
+  P.n_units = p.n_seqs * p.n_heads;
+  P.n_heads = p.n_heads;
+  P.seq_len = p.seq_len;
+  P.wait_ns = kWaitTimeoutNs;
+  if (P.n_units == 0) return cudaSuccess;
+  const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
+  const int64_t T = p.t_total > 0 ? p.t_total : 1;
+  bool ok = make_row_tile_map(&P.tm_q, p.q, T, p.n_heads) && make_row_tile_map(&P.tm_k, p.k, T, p.n_heads) &&
+            make_row_tile_map(&P.tm_v, p.v, T, p.n_heads) && make_row_tile_map(&P.tm_g, p.log_a, T, p.n_heads) &&
+            make_row_tile_map(&P.tm_b, p.b, T, p.n_heads);
+  if (ok && !tied) ok = make_row_tile_map(&P.tm_w, p.w, T, p.n_heads);
+  if (ok && p.dtype_out == GDN2_BF16) ok = make_row_tile_map(&P.tm_do, p.dO, T, p.n_heads);
+  if (!ok) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = P.n_units < sms ? P.n_units : sms;
+  if (p.dtype_out == GDN2_BF16)
+    return tied ? launch_t<__nv_bfloat16, true>(P, grid, stream) : launch_t<__nv_bfloat16, false>(P, grid, stream);
+  return tied ? launch_t<float, true>(P, grid, stream) : launch_t<float, false>(P, grid, stream);
+}
+
+}  // namespace gdn2

@@ -213,9 +213,10 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const voi
 }
 
 // gdn2_chunk_bwd workspace: [0, 256) header ([0] status, [1] forward unit counter, [2] backward
-// unit counter), the unit schedule, the per-sequence checkpoint offsets, the checkpoints.
+// unit counter), the unit schedule, the per-sequence checkpoint offsets, the final states
+// (fp32), the checkpoints (one 32 KB bf16 S_r tile image per chunk and (sequence, head)).
 struct ChunkBwdLayout {
-  size_t off_sched, off_ckoff, off_ckpt, total;
+  size_t off_sched, off_ckoff, off_fin, off_ckpt, total;
 };
 static ChunkBwdLayout chunk_bwd_layout(const gdn2_dims *dims, bool packed) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
@@ -224,9 +225,10 @@ static ChunkBwdLayout chunk_bwd_layout(const gdn2_dims *dims, bool packed) {
   ChunkBwdLayout L;
   L.off_sched = kWsHeader;
   L.off_ckoff = L.off_sched + up(units * sizeof(int32_t));
-  L.off_ckpt = L.off_ckoff + up(((size_t)dims->n_seqs + 1) * sizeof(int64_t));
+  L.off_fin = L.off_ckoff + up(((size_t)dims->n_seqs + 1) * sizeof(int64_t));
+  L.off_ckpt = L.off_fin + units * 128 * 128 * sizeof(float);
   const size_t slots = gdn2::bwd_tc_ckpt_slots(dims->n_seqs, t_total, dims->n_heads, packed, dims->seq_len);
-  L.total = L.off_ckpt + slots * 128 * 128 * sizeof(float);
+  L.total = L.off_ckpt + slots * 128 * 128 * 2;
   return L;
 }
 
@@ -288,13 +290,14 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_
     e = gdn2::launch_ckpt_offsets(cu_seqlens, dims->n_seqs, ckoff, s);
     if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "checkpoint offsets launch: %s", cudaGetErrorString(e));
   }
-  float *ckpt = reinterpret_cast<float *>(ws + lay.off_ckpt);
+  void *ckpt = ws + lay.off_ckpt;
+  float *S_fin = reinterpret_cast<float *>(ws + lay.off_fin);
 
-  // the forward, writing the state before every chunk (and the final state) instead of o
+  // the forward, writing every chunk's S_r tile and the final states instead of o
   gdn2::ChunkProblem f;
   memset(&f, 0, sizeof(f));
   f.q = q; f.k = k; f.v = v; f.log_a = log_a; f.b = b; f.w = w;
-  f.S0 = S0; f.cu_seqlens = cu_seqlens; f.o = nullptr; f.S_T = nullptr;
+  f.S0 = S0; f.cu_seqlens = cu_seqlens; f.o = nullptr; f.S_T = S_fin;
   f.n_seqs = dims->n_seqs; f.seq_len = dims->seq_len; f.n_heads = dims->n_heads;
   f.d_k = 128; f.d_v = 128; f.chunk = 64;
   f.dtype_in = GDN2_BF16; f.dtype_out = dims->dtype_out; f.flags = dims->flags;
@@ -316,7 +319,7 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_
   p.n_seqs = dims->n_seqs; p.seq_len = dims->seq_len; p.n_heads = dims->n_heads;
   p.d_k = 128; p.d_v = 128; p.t_total = t_total;
   p.dtype_in = GDN2_BF16; p.dtype_out = dims->dtype_out; p.flags = dims->flags;
-  e = gdn2::launch_bwd_tc(p, ckpt, ckoff, sched, status, status + 2, s);
+  e = gdn2::launch_bwd_tc(p, ckpt, S_fin, ckoff, sched, status, status + 2, s);
   if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "bwd_tc launch: %s", cudaGetErrorString(e));
   return GDN2_OK;
 }

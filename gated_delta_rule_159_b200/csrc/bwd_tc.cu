@@ -29,13 +29,15 @@
 // TMEM accumulators) with M = 128 rows: the 64-row matrices are stacked in pairs
 // ([k_r; q_r], [x_r; p_r], [dR; dO], [-M; V]) so that one instruction covers two of them, and
 // the transposed operand forms are MN-major shared-memory descriptors of the same tiles.  The
-// carried adjoint lives in TMEM, transposed (lane = d_v channel), for the whole sequence.
+// carried adjoint lives in TMEM (lane = d_k channel) for the whole sequence, so the thread of a
+// d_k channel scales and stores its row with one factor and 16-byte vectors.
 //
-// The states S_c come from a forward pass of chunk_tc_kernel that writes every chunk's start
-// state (fp32) to the workspace.  One CTA (512 threads) per SM takes (sequence, head) units
+// The S_r tiles come from a forward pass of chunk_tc_kernel that writes each chunk's bf16 S_r
+// (the operand it builds anyway, with the same rho) as a swizzled tile image to the workspace;
+// one bulk copy per chunk brings it to shared memory.  One CTA (512 threads) per SM takes (sequence, head) units
 // from an atomic counter and walks their chunks last to first; per chunk its phases are:
-//   1  loads (plain coalesced loads; the next chunk's rows are prefetched to L2), cumulative
-//      decay, the scaled operand tiles, S_r, Lam_g (from the TMEM adjoint), dO and V tiles;
+//   1  (the raw k, q, v, log_a, b, w, dO tiles (TMA) and S_r (bulk copy) were requested while
+//      the previous chunk finished) cumulative decay, the scaled operands in place, Lam_g;
 //   2  G1 [A B; QX QP] = [k_r; q_r][x_r; p_r]^T  and  dM^T <- Lam_g^T x_r^T;  masks;
 //   3  the (I + A)^-1 solve (fp32, warps 0-14) while warp 15 issues R^T and dM^T += dO^T QX;
 //   4  R^T, -dM^T to bf16 TMEM operands; M^T = R^T T^T, dR^T = dM^T T;
@@ -86,11 +88,13 @@ constexpr uint32_t OFF_QX = OFF_MV + 16384;    // QX bf16 [64 x 64] (the -M rows
 constexpr uint32_t OFF_AT0 = OFF_RO;           // fp32 A, then T, rows 0-31 [32][64] (dR rows, block 0)
 constexpr uint32_t OFF_AT1 = OFF_RO + 16384;   // rows 32-63 (dR rows, block 1)
 constexpr uint32_t OFF_DG = OFF_SR;            // [dA dB; dQX dQP] as [column block][128 rows][64]
+constexpr uint32_t OFF_GRAW = OFF_LG;          // raw log_a tile [2 blocks][64 rows] until Lam_g is built
 constexpr uint32_t MISC_BAR = 0;       // mbarriers
 constexpr uint32_t MISC_TMEM = 64;
 constexpr uint32_t MISC_ABORT = 68;
 constexpr uint32_t MISC_UNIT = 72;
 constexpr uint32_t MISC_WIDE = 76;
+constexpr uint32_t MISC_ISS = 80;      // uint32: load phases armed on BAR_LD
 constexpr uint32_t MISC_RHO = 128;     // float[128]     rho of the current chunk
 constexpr uint32_t MISC_ESR = 640;     // float[2][128]  e^{rho} per chunk parity
 constexpr uint32_t MISC_DLC = 1664;    // float[2][128]  decay term of L_63 per chunk parity
@@ -101,16 +105,21 @@ constexpr uint32_t MISC_RS = 7296;     // float[4][128]  row sums per lane quadr
 constexpr uint32_t MISC_BYTES = 9344;
 constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES + 1024;  // + base alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 limit per CTA");
-enum { BAR_G1 = 0, BAR_GA, BAR_GB, BAR_G5, BAR_G7, BAR_DRAIN, kNumBars };
+enum { BAR_LD = 0, BAR_G1, BAR_GA, BAR_GB, BAR_G5, BAR_G7, BAR_DRAIN, kNumBars };
 static_assert(MISC_BAR + 8 * kNumBars <= MISC_TMEM, "mbarriers overlap the TMEM address slot");
 
 struct BwdTcParams {
+  // raw tiles of a chunk by TMA, (channel, head, token) boxes of 64 x 1 x 64, 128-byte swizzle:
+  // k, q over the k_r, q_r rows, v over the V rows, b, w over the x_r, p_r rows, log_a into
+  // the Lam_g tile's space
+  CUtensorMap tm_q, tm_k, tm_v, tm_g, tm_b, tm_w, tm_do;  // tm_do: bf16 dO only
   const __nv_bfloat16 *q, *k, *v, *log_a, *b, *w;  // forward inputs [T_tot][H][128]
   const void *dO;                                  // [T_tot][H][128] Tout
   const float *dS_T;                               // [N][H][128][128] or NULL
   void *dq, *dk, *dv, *dlog_a, *db, *dw;           // Tout, like the inputs (dw NULL when tied)
   float *dS0;                                      // [N][H][128][128] or NULL
-  const float *ckpt;                               // chunk-boundary states (tc::ckpt_first_slot)
+  const uint8_t *ckpt;                             // per chunk the bf16 S_r tile image (32 KB)
+  const float *S_fin;                              // [N][H][128][128] final states (fp32)
   const int64_t *ckpt_off;                         // NULL for equal lengths
   const int32_t *cu_seqlens;                       // NULL for equal lengths
   const int32_t *schedule;                         // unit order (longest first) or NULL
@@ -172,11 +181,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
   volatile int *sAbort = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_ABORT);
   volatile int *sUnit = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_UNIT);
   volatile int *sWide = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_WIDE);
+  volatile uint32_t *sIss = reinterpret_cast<volatile uint32_t *>(gb + OFF_MISC + MISC_ISS);
   auto bar = [&](int i) { return sb + OFF_MISC + MISC_BAR + 8u * (uint32_t)i; };
   auto waitb = [&](uint32_t b, uint32_t parity) { return wait_bar(b, parity, sAbort, P.status, P.wait_ns); };
-  // fp32 A / T of the solve: rows 0-31 and 32-63 in two 8 KB halves, 64 floats per row
+  // fp32 A / T of the solve: rows 0-31 and 32-63 in two 8 KB halves, 64 floats per row; the
+  // column index is XORed with 4 (row mod 8) so that the 8 rows of an mma fragment load fall
+  // in different banks (groups of four columns stay contiguous)
   auto at = [&](int i, int j) -> float * {
-    return reinterpret_cast<float *>(gb + (i < 32 ? OFF_AT0 : OFF_AT1) + (uint32_t)(((i & 31) * 64 + j) * 4));
+    return reinterpret_cast<float *>(gb + (i < 32 ? OFF_AT0 : OFF_AT1) +
+                                     (uint32_t)(((i & 31) * 64 + (j ^ ((i & 7) << 2))) * 4));
   };
   // L_ref of channel i from the row-group sums (the same expression in every thread)
   auto rho_of = [&](int i, float &tot) {
@@ -188,6 +201,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
     for (int i = 0; i < kNumBars; ++i) ptx::mbar_init(bar(i), 1);
     ptx::fence_mbar_init();
     *sAbort = 0;
+    *sIss = 0u;
+    ptx::tma_prefetch_desc(&P.tm_q);
+    ptx::tma_prefetch_desc(&P.tm_k);
+    ptx::tma_prefetch_desc(&P.tm_v);
+    ptx::tma_prefetch_desc(&P.tm_g);
+    ptx::tma_prefetch_desc(&P.tm_b);
+    if (!kTied) ptx::tma_prefetch_desc(&P.tm_w);
   }
   if (warp == 0) {
     ptx::tmem_alloc(sb + OFF_MISC + MISC_TMEM, kTmemCols);
@@ -197,19 +217,40 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(gb + OFF_MISC + MISC_TMEM);
-  // TMEM columns: the adjoint Acc^T (lane = d_v channel j, column = d_k channel i), and three
+  // TMEM columns: the adjoint Acc (lane = d_k channel i, column = d_v channel j), and three
   // 128-column work areas:
   //   X: G1 -> bf16 R^T (cols 0-31) and -dM^T (32-63) -> [dA dB; dQX dQP] -> [dx_r^T | dp_r^T]
   //   Y: R^T (0-63), M^T (64-127) -> dV^T (0-63)
   //   Z: dM^T (0-63), dR^T (64-127) -> [dk_r^T | dq_r^T]
   const uint32_t tmAcc = tmem, tmX = tmem + 128, tmY = tmem + 256, tmZ = tmem + 384;
   const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
-  uint32_t it = 0;  // chunks processed by this CTA: the parity of every mbarrier
+  uint32_t it = 0;     // chunks processed by this CTA: the parity of the MMA barriers
+  uint32_t ld_it = 0;  // load phases consumed (a chunk outside the range consumes one, no MMA phase)
 
   const Tout *g_do = static_cast<const Tout *>(P.dO);
   const __nv_bfloat16 *g_w = kTied ? P.b : P.w;
   Tout *g_dq = static_cast<Tout *>(P.dq), *g_dk = static_cast<Tout *>(P.dk), *g_dv = static_cast<Tout *>(P.dv);
   Tout *g_dla = static_cast<Tout *>(P.dlog_a), *g_db = static_cast<Tout *>(P.db), *g_dw = static_cast<Tout *>(P.dw);
+
+  // the raw k, q, v, log_a, b (, w, dO) tiles of the chunk at token t0 of head h, and its S_r
+  // tile image (thread kIssuer)
+  constexpr bool kDoTma = sizeof(Tout) == 2;  // bf16 dO lands in its tile as it is
+  auto issue_loads = [&](int h, int t0, const uint8_t *sr_img) {
+    ptx::mbar_arrive_expect_tx(bar(BAR_LD), ((kTied ? 5u : 6u) + (kDoTma ? 1u : 0u)) * 16384u + 32768u);
+    *sIss = *sIss + 1u;
+    ptx::bulk_load(sb + OFF_SR, sr_img, 32768u, bar(BAR_LD));
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) {
+      const uint32_t o = (uint32_t)kb * 16384u;
+      ptx::tma_load_3d(sb + OFF_KQ + o, &P.tm_k, kb * 64, h, t0, bar(BAR_LD));
+      ptx::tma_load_3d(sb + OFF_KQ + o + 8192u, &P.tm_q, kb * 64, h, t0, bar(BAR_LD));
+      ptx::tma_load_3d(sb + OFF_MV + o + 8192u, &P.tm_v, kb * 64, h, t0, bar(BAR_LD));
+      ptx::tma_load_3d(sb + OFF_GRAW + (uint32_t)kb * 8192u, &P.tm_g, kb * 64, h, t0, bar(BAR_LD));
+      ptx::tma_load_3d(sb + OFF_XP + o, &P.tm_b, kb * 64, h, t0, bar(BAR_LD));
+      if (!kTied) ptx::tma_load_3d(sb + OFF_XP + o + 8192u, &P.tm_w, kb * 64, h, t0, bar(BAR_LD));
+      if (kDoTma) ptx::tma_load_3d(sb + OFF_RO + o + 8192u, &P.tm_do, kb * 64, h, t0, bar(BAR_LD));
+    }
+  };
 
   for (;;) {
     if (tid == 0) *sUnit = atomicAdd(P.counter, 1);
@@ -227,26 +268,32 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       len = P.seq_len;
     }
     const int nchunks = (int)((len + C - 1) / C);
-    const float *ck_unit = P.ckpt + ckpt_first_slot(P.ckpt_off, n, h, H, nchunks) * (D * D);
+    const uint8_t *ck_unit = P.ckpt + ckpt_first_slot(P.ckpt_off, n, h, H, nchunks) * (size_t)(D * D * 2);
 
-    // ---- the final state's adjoint dS_T into TMEM (thread: d_v channel `row`, d_k channels
+    // ---- the final state's adjoint dS_T into TMEM (thread: d_k channel `row`, d_v channels
     //      [32 cg, 32 cg + 32)), and the decay term of the last chunk, sum_j dS_T S_T per d_k
-    //      channel (S_T is the last checkpoint slot)
+    //      channel (S_T: the forward's final state)
     {
       uint32_t r[32];
-      float prod[32];
-      const float *st = ck_unit + ((size_t)nchunks * D + cg * 32) * D + row;
-      const float *dst = P.dS_T ? P.dS_T + ((size_t)unit * D + cg * 32) * D + row : nullptr;
+      float acc = 0.f;
+      const size_t o = ((size_t)unit * D + row) * D + cg * 32;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float a = dst ? dst[(size_t)j * D] : 0.f;
-        r[j] = __float_as_uint(a);
-        prod[j] = a * st[(size_t)j * D];
+      for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 a = P.dS_T ? *reinterpret_cast<const float4 *>(P.dS_T + o + 4 * j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 st = *reinterpret_cast<const float4 *>(P.S_fin + o + 4 * j4);
+        r[4 * j4] = __float_as_uint(a.x);
+        r[4 * j4 + 1] = __float_as_uint(a.y);
+        r[4 * j4 + 2] = __float_as_uint(a.z);
+        r[4 * j4 + 3] = __float_as_uint(a.w);
+        acc += a.x * st.x + a.y * st.y + a.z * st.z + a.w * st.w;
       }
       ptx::tmem_st32(tmAcc + lane_base + cg * 32, r);
       ptx::tmem_wait_st();
-      rs[qd * 128 + cg * 32 + lane] = warp_colsum32(prod);
+      rs[cg * 128 + row] = acc;
       if (tid < 128) sEsr[((it & 1u) ^ 1u) * 128 + tid] = 1.f;  // the last chunk reads dS_T unscaled
+      // the last chunk's tiles (every tile is free: the previous unit's MMAs are done)
+      if (tid == kIssuer && nchunks > 0 && !*sAbort)
+        issue_loads(h, (int)(bos + (int64_t)(nchunks - 1) * C), ck_unit + (size_t)(nchunks - 1) * (D * D * 2));
     }
     __syncthreads();
     if (tid < 128)
@@ -260,12 +307,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       const int nvalid = (int)((len - (int64_t)ci * C) < C ? (len - (int64_t)ci * C) : C);
 
       // ================= phase 1: loads, cumulative decay, operand tiles
-      float sc[32];  // S_c (thread: d_v channel `row`, d_k rows [32 cg, 32 cg + 32)), loaded first
-      {
-        const float *src = ck_unit + ((size_t)ci * D + cg * 32) * D + row;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) sc[j] = src[(size_t)j * D];
-      }
       if (ci > 0) {  // the next chunk's rows and state to L2 while this chunk runs
         if (tid < 448) {
           const int tsel = tid >> 6, r = tid & 63;
@@ -275,29 +316,44 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
                           : tsel == 4 ? (const void *)(P.b + gi) : tsel == 5 ? (const void *)(g_w + gi)
                                       : (const void *)(g_do + gi);
           if (tsel != 5 || !kTied) ptx::bulk_prefetch_l2(src, tsel == 6 ? D * (uint32_t)sizeof(Tout) : D * 2u);
-        } else if (tid < 452) {
-          ptx::bulk_prefetch_l2(ck_unit + (size_t)(ci - 1) * D * D + (size_t)(tid - 448) * 4096, 16384u);
+        } else if (tid < 450) {
+          ptx::bulk_prefetch_l2(ck_unit + (size_t)(ci - 1) * (D * D * 2) + (size_t)(tid - 448) * 16384, 16384u);
         }
       }
-      // cumulative log-decay of channel `row` over rows [16 cg, 16 cg + 16) (rows past the
-      // chunk end decay by nothing); the V and dO rows go to their tiles as they are
+      // fp32 dO: the rows of channel `row` into the bf16 tile (rows past the chunk end re-read
+      // its last row and are zeroed); the dO rows of the tile are free since the previous
+      // chunk's products.  bf16 dO arrives with the other tiles.
+      if (!kDoTma) {
+        Tout dov[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const int r = 16 * cg + t, rc = r < nvalid ? r : nvalid - 1;
+          dov[t] = g_do[((size_t)(t0 + rc) * H + h) * D + row];
+        }
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const int r = 16 * cg + t;
+          sts_u16(sb + OFF_RO + 8192u + swz_elem(r, row, 16384u), bf16_bits(r < nvalid ? to_f32<Tout>(dov[t]) : 0.f));
+        }
+      }
+      waitb(bar(BAR_LD), ld_it & 1u);
+      ++ld_it;
+      // cumulative log-decay of channel `row` over rows [16 cg, 16 cg + 16) (rows past the chunk
+      // end decay by nothing; their V rows are zeroed); the dO rows go to their tile
       float Lloc[16];
       {
         float acc = 0.f;
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
           const int r = 16 * cg + t;
-          float la = 0.f, vv = 0.f, dd = 0.f;
-          if (r < nvalid) {
-            const size_t gi = ((size_t)(t0 + r) * H + h) * D + row;
-            la = bf(P.log_a[gi]);
-            vv = bf(P.v[gi]);
-            dd = to_f32<Tout>(g_do[gi]);
-          }
+          const uint32_t o = swz_elem(r, row, 16384u);
+          const float la = r < nvalid ? bf16_value(lds_u16(sb + OFF_GRAW + swz_elem(r, row, 8192u))) : 0.f;
           acc += la;
           Lloc[t] = acc;
-          sts_u16(sb + OFF_MV + 8192u + swz_elem(r, row, 16384u), bf16_bits(vv));
-          sts_u16(sb + OFF_RO + 8192u + swz_elem(r, row, 16384u), bf16_bits(dd));
+          if (r >= nvalid) {
+            sts_u16(sb + OFF_MV + 8192u + o, 0);
+            if (kDoTma) sts_u16(sb + OFF_RO + 8192u + o, 0);
+          }
         }
         part[cg * 128 + row] = acc;
         if (cg == 0) sL0[row] = Lloc[0];
@@ -318,46 +374,45 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         }
         lpre[cg * 128 + row] = pre;
       }
-      // k_r, q_r, x_r, p_r (rows past the chunk end are zero)
+      // k_r, q_r, x_r, p_r over the raw k, q, b, w rows (rows past the chunk end are zeroed)
 #pragma unroll
       for (int t = 0; t < 16; ++t) {
         const int r = 16 * cg + t;
+        const uint32_t o0 = swz_elem(r, row, 16384u), o1 = swz_elem(64 + r, row, 16384u);
         float kk = 0.f, qq = 0.f, bb = 0.f, ww = 0.f;
         if (r < nvalid) {
-          const size_t gi = ((size_t)(t0 + r) * H + h) * D + row;
-          kk = bf(P.k[gi]);
-          qq = bf(P.q[gi]);
-          bb = bf(P.b[gi]);
-          ww = kTied ? bb : bf(g_w[gi]);
+          kk = bf16_value(lds_u16(sb + OFF_KQ + o0));
+          qq = bf16_value(lds_u16(sb + OFF_KQ + o1));
+          bb = bf16_value(lds_u16(sb + OFF_XP + o0));
+          ww = kTied ? bb : bf16_value(lds_u16(sb + OFF_XP + o1));
         }
         const float L = pre + Lloc[t];
         const float e = ptx::ex2((L - rho) * kLog2eF), f = ptx::ex2((rho - L) * kLog2eF);
-        const uint32_t o0 = swz_elem(r, row, 16384u), o1 = swz_elem(64 + r, row, 16384u);
         sts_u16(sb + OFF_KQ + o0, bf16_bits(kk * e));
         sts_u16(sb + OFF_KQ + o1, bf16_bits(qq * e));
         sts_u16(sb + OFF_XP + o0, bf16_bits(bb * kk * f));
         sts_u16(sb + OFF_XP + o1, bf16_bits(ww * kk * f));
       }
-      // S_r = Diag(e^{rho}) S_c and Lam_g = Diag(gamma e^{rho_next}) Acc (bf16 tiles [d_k][d_v]);
-      // Lam_g also replaces Acc in TMEM: the adjoint update accumulates onto it
+      // Lam_g = Diag(gamma e^{rho_next}) Acc, the bf16 tile [d_k rows][d_v] and the fp32 base of
+      // this chunk's adjoint update (thread: d_k channel `row`, d_v channels [32 cg, 32 cg + 32))
       {
+        float tot;
+        const float ri = rho_of(row, tot);
+        const float gam = ptx::ex2((tot - ri) * kLog2eF);
+        const float efac = sEsr[(par ^ 1u) * 128 + row];
         uint32_t r[32];
+        float lg[32];
         ptx::tmem_ld32(tmAcc + lane_base + cg * 32, r);
         ptx::tmem_wait_ld();
-        const float *efac = sEsr + (par ^ 1u) * 128 + cg * 32;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const int i = cg * 32 + j;
-          float tot;
-          const float ri = rho_of(i, tot);
-          const float gam = ptx::ex2((tot - ri) * kLog2eF);
-          const float lg = (__uint_as_float(r[j]) * efac[j]) * gam;  // e^{rho_next} first: the adjoint, O(1)
-          r[j] = __float_as_uint(lg);
-          const uint32_t o = swz_elem(i, row, 16384u);
-          sts_u16(sb + OFF_SR + o, bf16_bits(sc[j] * ptx::ex2(ri * kLog2eF)));
-          sts_u16(sb + OFF_LG + o, bf16_bits(lg));
+          lg[j] = (__uint_as_float(r[j]) * efac) * gam;  // e^{rho_next} first: the adjoint, O(1)
+          r[j] = __float_as_uint(lg[j]);
         }
         ptx::tmem_st32(tmAcc + lane_base + cg * 32, r);
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8)
+          sts_v4(sb + OFF_LG + (uint32_t)(cg >> 1) * 16384u + swz(row, (uint32_t)((cg & 1) * 4 + q8)), pack8(lg + 8 * q8, 1.f));
         ptx::tmem_wait_st();
       }
       ptx::fence_proxy_async_smem();
@@ -397,10 +452,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
 #pragma unroll
         for (int j = 0; j < 32; ++j) f[j] = (strict ? jb + j < i : jb + j <= i) ? __uint_as_float(r[j]) : 0.f;
         if (strict && cg < 2) {  // A in fp32 for the solve
-          float *dst = at(i, jb);
 #pragma unroll
           for (int j4 = 0; j4 < 8; ++j4)
-            *reinterpret_cast<float4 *>(dst + 4 * j4) = make_float4(f[4 * j4], f[4 * j4 + 1], f[4 * j4 + 2], f[4 * j4 + 3]);
+            *reinterpret_cast<float4 *>(at(i, jb + 4 * j4)) =
+                make_float4(f[4 * j4], f[4 * j4 + 1], f[4 * j4 + 2], f[4 * j4 + 3]);
         } else {
           // B into rows 0-63 of [B; QP]; QX into its own tile; QP into rows 64-127 of [B; QP]
           const uint32_t dst = strict ? sb + OFF_BQP : (cg < 2 ? sb + OFF_QX : sb + OFF_BQP + 8192u);
@@ -466,28 +521,82 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         }
         named_bar(NB_SOLVE, kSolveThreads);
         float *Xs = reinterpret_cast<float *>(gb + OFF_XS);
-#pragma unroll 1
-        for (int s = 8; s <= 32; s *= 2) {
-          const int tot = 32 * s;  // (64 / 2s) pairs x s^2 outputs
-          for (int idx = tid; idx < tot; idx += kSolveThreads) {
-            const int pr = idx / (s * s), rem = idx % (s * s), r = rem / s, c = rem % s;
-            const int u0 = 2 * s * pr, l0 = u0 + s;
-            float acc = 0.f;
-            for (int k2 = c; k2 < s; ++k2) acc += *at(l0 + r, u0 + k2) * *at(u0 + k2, u0 + c);
-            Xs[idx] = acc;
+        // s = 8: 4 pairs x 64 outputs on CUDA cores
+        if (tid < 256) {
+          const int pr = tid >> 6, r = (tid >> 3) & 7, c = tid & 7, u0 = 16 * pr, l0 = u0 + 8;
+          float acc = 0.f;
+#pragma unroll
+          for (int k2 = 0; k2 < 8; ++k2) acc += (k2 >= c ? *at(l0 + r, u0 + k2) * *at(u0 + k2, u0 + c) : 0.f);
+          Xs[tid] = acc;
+        }
+        named_bar(NB_SOLVE, kSolveThreads);
+        if (tid < 256) {
+          const int pr = tid >> 6, r = (tid >> 3) & 7, c = tid & 7, u0 = 16 * pr, l0 = u0 + 8;
+          float acc = 0.f;
+#pragma unroll
+          for (int k2 = 0; k2 < 8; ++k2) acc -= (k2 <= r ? *at(l0 + r, l0 + k2) * Xs[pr * 64 + k2 * 8 + c] : 0.f);
+          *at(l0 + r, u0 + c) = acc;
+          sts_u16(sb + OFF_T + swz(l0 + r, (uint32_t)(u0 >> 3)) + (uint32_t)c * 2u, bf16_bits(acc));
+        }
+        named_bar(NB_SOLVE, kSolveThreads);
+        // s = 16 (2 pairs) and s = 32 (1 pair) on tf32 mma.sync, one warp per 16x8 output tile;
+        // each K step's fragments are loaded right before its MMA (few registers live)
+        const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+        for (int lev = 1; lev < 3; ++lev) {
+          const int sz = 8 << lev;                   // 16, 32
+          const int nk = sz / 8;                     // 8-wide K steps: 2, 4
+          const int tpp = (sz / 16) * (sz / 8);      // 16x8 tiles per pair: 2, 8
+          const int ntiles = (64 / (2 * sz)) * tpp;  // 4, 8
+          const int pr = warp / tpp, ti = warp % tpp, mt = ti / (sz / 8), nt = ti % (sz / 8);
+          const int u0 = pr * 2 * sz, l0 = u0 + sz, rr = 16 * mt, cc = 8 * nt;
+          // X = A_LU T_UU (T_UU is lower triangular: K steps before the tile's first column vanish)
+          if (warp < ntiles) {
+            float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              if (kk < nk && kk >= nt) {
+                const int kc = u0 + 8 * kk + t4;
+                const uint32_t av[4] = {ptx::to_tf32(*at(l0 + rr + g, kc)), ptx::to_tf32(*at(l0 + rr + g + 8, kc)),
+                                        ptx::to_tf32(*at(l0 + rr + g, kc + 4)), ptx::to_tf32(*at(l0 + rr + g + 8, kc + 4))};
+                const uint32_t bv[2] = {ptx::to_tf32(*at(kc, u0 + cc + g)), ptx::to_tf32(*at(kc + 4, u0 + cc + g))};
+                ptx::mma_tf32_16x8x8(x, av, bv);
+              }
+            }
+            float *xs = Xs + pr * sz * sz;
+            xs[(rr + g) * sz + cc + 2 * t4] = x[0];
+            xs[(rr + g) * sz + cc + 2 * t4 + 1] = x[1];
+            xs[(rr + g + 8) * sz + cc + 2 * t4] = x[2];
+            xs[(rr + g + 8) * sz + cc + 2 * t4 + 1] = x[3];
           }
           named_bar(NB_SOLVE, kSolveThreads);
-          for (int idx = tid; idx < tot; idx += kSolveThreads) {
-            const int pr = idx / (s * s), rem = idx % (s * s), r = rem / s, c = rem % s;
-            const int u0 = 2 * s * pr, l0 = u0 + s;
-            const float *xs = Xs + pr * s * s;
-            float acc = 0.f;
-            for (int k2 = 0; k2 <= r; ++k2) acc += *at(l0 + r, l0 + k2) * xs[k2 * s + c];
-            *at(l0 + r, u0 + c) = -acc;
-            const int cc = u0 + c;
-            sts_u16(sb + OFF_T + swz(l0 + r, (uint32_t)(cc >> 3)) + (uint32_t)(cc & 7) * 2u, bf16_bits(-acc));
+          // T_LU = -T_LL X (K steps past the tile's last row vanish), over A_LU
+          if (warp < ntiles) {
+            const float *xs = Xs + pr * sz * sz;
+            float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              if (kk < nk && kk <= (rr + 15) / 8) {
+                // T_LL is lower triangular (its blocks above the diagonal hold zeros of A)
+                const int kc = l0 + 8 * kk + t4;
+                const uint32_t av[4] = {ptx::to_tf32(*at(l0 + rr + g, kc)), ptx::to_tf32(*at(l0 + rr + g + 8, kc)),
+                                        ptx::to_tf32(*at(l0 + rr + g, kc + 4)), ptx::to_tf32(*at(l0 + rr + g + 8, kc + 4))};
+                const uint32_t bv[2] = {ptx::to_tf32(xs[(8 * kk + t4) * sz + cc + g]),
+                                        ptx::to_tf32(xs[(8 * kk + t4 + 4) * sz + cc + g])};
+                ptx::mma_tf32_16x8x8(y, av, bv);
+              }
+            }
+            const int ri = l0 + rr + g, cj = u0 + cc + 2 * t4;
+            if (lev == 1) {  // the last level's T_LU is read by no later level: bf16 only
+              *at(ri, cj) = -y[0];
+              *at(ri, cj + 1) = -y[1];
+              *at(ri + 8, cj) = -y[2];
+              *at(ri + 8, cj + 1) = -y[3];
+            }
+            sts_u32(sb + OFF_T + swz(ri, (uint32_t)(cj >> 3)) + (uint32_t)(cj & 7) * 2u, pack_bf16x2(-y[0], -y[1]));
+            sts_u32(sb + OFF_T + swz(ri + 8, (uint32_t)(cj >> 3)) + (uint32_t)(cj & 7) * 2u, pack_bf16x2(-y[2], -y[3]));
           }
-          named_bar(NB_SOLVE, kSolveThreads);
+          if (lev == 1) named_bar(NB_SOLVE, kSolveThreads);
         }
         ptx::fence_proxy_async_smem();  // the bf16 T tile is read by the tensor core
       }
@@ -550,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       __syncthreads();
 
       // ================= phase 6: [dA dB; dQX dQP] = [dR; dO][-M; V]^T, the adjoint update
-      //      Acc^T += [dR; dO]^T [k_r; q_r], dV^T = [dR; dO]^T [B; QP] + Lam_g^T p_r^T and the
+      //      Acc += [k_r; q_r]^T [dR; dO], dV^T = [dR; dO]^T [B; QP] + Lam_g^T p_r^T and the
       //      S_r terms [dk_r^T | dq_r^T] = S_r [dR; dO]^T
       if (tid == kIssuer && !*sAbort) {
         ptx::tc_fence_after();
@@ -559,7 +668,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmX, kmaj(sb + OFF_RO, kk), kmaj(sb + OFF_MV, kk), idKK, kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmAcc, mnmaj(sb + OFF_RO, kk), mnmaj(sb + OFF_KQ, kk), idNN, 1);
+        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmAcc, mnmaj(sb + OFF_KQ, kk), mnmaj(sb + OFF_RO, kk), idNN, 1);
         constexpr uint32_t idV1 = ptx::idesc_bf16(128, 64, true, true);
         constexpr uint32_t idV2 = ptx::idesc_bf16(128, 64, true, false);
 #pragma unroll
@@ -578,16 +687,24 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       ptx::tc_fence_after();
       if (ci > 0) {
         // sum_j Lam_{c-1}[i][j] S_c[i][j] = sum_j Acc[i][j] S_r[i][j] (Lam_{c-1} = e^{rho} Acc):
-        // thread (d_v channel `row`, d_k channels [32 cg, 32 cg + 32)), summed over the warp's
-        // 32 d_v channels here and over the four lane quadrants by the chunk before
+        // thread (d_k channel `row`, d_v channels [32 cg, 32 cg + 32)), summed over the four
+        // column groups by the chunk before
         uint32_t r[32];
-        float prod[32];
         ptx::tmem_ld32(tmAcc + lane_base + cg * 32, r);
         ptx::tmem_wait_ld();
+        float acc = 0.f;
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          prod[j] = __uint_as_float(r[j]) * bf16_value(lds_u16(sb + OFF_SR + swz_elem(cg * 32 + j, row, 16384u)));
-        rs[qd * 128 + cg * 32 + lane] = warp_colsum32(prod);
+        for (int q8 = 0; q8 < 4; ++q8) {
+          const uint4 sv = lds_v4(sb + OFF_SR + (uint32_t)(cg >> 1) * 16384u + swz(row, (uint32_t)((cg & 1) * 4 + q8)));
+          const uint32_t w4[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float2 f = unpack_bf16x2(w4[e2]);
+            acc = fmaf(__uint_as_float(r[8 * q8 + 2 * e2]), f.x, acc);
+            acc = fmaf(__uint_as_float(r[8 * q8 + 2 * e2 + 1]), f.y, acc);
+          }
+        }
+        rs[cg * 128 + row] = acc;
       }
       {  // dV (= dZ: the values enter unscaled); thread: d_v channel `row`, tokens [16 cg, 16 cg + 16)
         uint32_t r[16];
@@ -638,6 +755,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       }
       waitb(bar(BAR_G7), par);
       ptx::tc_fence_after();
+      // every tile is free (the epilogue reads TMEM and global memory only): the next chunk's
+      // raw tiles land while this chunk's gradients are formed and stored
+      if (tid == kIssuer && ci > 0 && !*sAbort) issue_loads(h, t0 - C, ck_unit + (size_t)(ci - 1) * (D * D * 2));
 
       // ================= phase 9: chain rule and stores.  Thread: d_k channel i = `row`, tokens
       //      [16 cg, 16 cg + 16).  The cumulative decay is recomputed as phase 1 computed it.
@@ -654,19 +774,26 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           ptx::tmem_ld8(tmX + lane_base + 64u + (uint32_t)c0, vp);
           ptx::tmem_ld8(tmZ + lane_base + (uint32_t)c0, vk);
           ptx::tmem_ld8(tmZ + lane_base + 64u + (uint32_t)c0, vq);
+          // the raw inputs of the 8 rows, all requested before any is used (rows past the
+          // chunk end re-read its last row and are ignored)
+          __nv_bfloat16 rla[8], rk[8], rq[8], rb[8], rw[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int t = c0 + j, tc = t < nvalid ? t : nvalid - 1;
+            const size_t gi = ((size_t)(t0 + tc) * H + h) * D + i;
+            rla[j] = P.log_a[gi];
+            rk[j] = P.k[gi];
+            rq[j] = P.q[gi];
+            rb[j] = P.b[gi];
+            rw[j] = kTied ? rb[j] : g_w[gi];
+          }
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int t = c0 + j;
-            float la = 0.f, kk = 0.f, qq = 0.f, bb = 0.f, ww = 0.f;
-            const size_t gi = ((size_t)(t0 + t) * H + h) * D + i;
-            if (t < nvalid) {
-              la = bf(P.log_a[gi]);
-              kk = bf(P.k[gi]);
-              qq = bf(P.q[gi]);
-              bb = bf(P.b[gi]);
-              ww = kTied ? bb : bf(g_w[gi]);
-            }
+            const bool valid = t < nvalid;
+            const float la = valid ? bf(rla[j]) : 0.f, kk = valid ? bf(rk[j]) : 0.f, qq = valid ? bf(rq[j]) : 0.f;
+            const float bb = valid ? bf(rb[j]) : 0.f, ww = valid ? bf(rw[j]) : 0.f;
             loc += la;
             const float L = pre + loc;
             const float e = ptx::ex2((L - rho) * kLog2eF), f = ptx::ex2((rho - L) * kLog2eF);
@@ -676,7 +803,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
             float dLt = e * (dqr * qq + dkr * kk) - f * kk * (dxr * bb + dpr * ww);
             if (t == C - 1) dLt += dlc;
             dL[half * 8 + j] = dLt;
-            if (t < nvalid) {
+            if (valid) {
+              const size_t gi = ((size_t)(t0 + t) * H + h) * D + i;
               g_dq[gi] = from_f32<Tout>(dqr * e);
               g_dk[gi] = from_f32<Tout>(dkr * e + bb * dx + ww * dp);
               if (kTied) {
@@ -718,10 +846,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       uint32_t r[32];
       ptx::tmem_ld32(tmAcc + lane_base + cg * 32, r);
       ptx::tmem_wait_ld();
-      float *dst = P.dS0 + ((size_t)unit * D + cg * 32) * D + row;
-      const float *es = lastpar >= 0 ? sEsr + lastpar * 128 + cg * 32 : nullptr;
+      float4 *dst = reinterpret_cast<float4 *>(P.dS0 + ((size_t)unit * D + row) * D + cg * 32);
+      const float es = lastpar >= 0 ? sEsr[lastpar * 128 + row] : 1.f;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) dst[(size_t)j * D] = __uint_as_float(r[j]) * (es ? es[j] : 1.f);
+      for (int j4 = 0; j4 < 8; ++j4)
+        dst[j4] = make_float4(__uint_as_float(r[4 * j4]) * es, __uint_as_float(r[4 * j4 + 1]) * es,
+                              __uint_as_float(r[4 * j4 + 2]) * es, __uint_as_float(r[4 * j4 + 3]) * es);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -733,6 +863,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
     if (tid == kIssuer) {
       ptx::umma_commit(bar(BAR_DRAIN));
       drain_bar(bar(BAR_DRAIN), 0u, P.wait_ns);
+      if (*sIss > 0u) drain_bar(bar(BAR_LD), (*sIss - 1u) & 1u, P.wait_ns);  // the last armed load phase
     }
   }
   ptx::tc_fence_before();
@@ -741,7 +872,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
   if (warp == 0) ptx::tmem_dealloc(tmem, kTmemCols);
 }
 
-// off[n] = sum over m < n of (ceil(len_m / 64) + 1), off[N] the total: the first checkpoint
+// off[n] = sum over m < n of ceil(len_m / 64), off[N] the total: the first checkpoint
 // slot of each sequence divided by the head count.  One block; each thread owns a contiguous
 // range of sequences.
 __global__ void ckpt_offsets_kernel(const int32_t *cu, int N, int64_t *off) {
@@ -749,7 +880,7 @@ __global__ void ckpt_offsets_kernel(const int32_t *cu, int N, int64_t *off) {
   const int per = (N + (int)blockDim.x - 1) / (int)blockDim.x;
   const int a = (int)threadIdx.x * per, e = a + per < N ? a + per : N;
   int64_t s = 0;
-  for (int n = a; n < e; ++n) s += (cu[n + 1] - cu[n] + C - 1) / C + 1;
+  for (int n = a; n < e; ++n) s += (cu[n + 1] - cu[n] + C - 1) / C;
   sums[threadIdx.x] = s;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -765,7 +896,7 @@ __global__ void ckpt_offsets_kernel(const int32_t *cu, int N, int64_t *off) {
   int64_t run = sums[threadIdx.x];
   for (int n = a; n < e; ++n) {
     off[n] = run;
-    run += (cu[n + 1] - cu[n] + C - 1) / C + 1;
+    run += (cu[n + 1] - cu[n] + C - 1) / C;
   }
 }
 
@@ -781,8 +912,8 @@ cudaError_t launch_t(const BwdTcParams &P, int grid, cudaStream_t stream) {
 }  // namespace
 
 size_t bwd_tc_ckpt_slots(int64_t n_seqs, int64_t t_total, int n_heads, bool packed, int seq_len) {
-  if (packed) return (size_t)n_heads * (size_t)(t_total / C + 2 * n_seqs);
-  return (size_t)n_heads * (size_t)n_seqs * (size_t)((seq_len + C - 1) / C + 1);
+  if (packed) return (size_t)n_heads * (size_t)(t_total / C + n_seqs);  // sum of ceil(len / 64) <= T/64 + N
+  return (size_t)n_heads * (size_t)n_seqs * (size_t)((seq_len + C - 1) / C);
 }
 
 cudaError_t launch_ckpt_offsets(const int32_t *cu_seqlens, int n_seqs, int64_t *off, cudaStream_t stream) {
@@ -790,8 +921,8 @@ cudaError_t launch_ckpt_offsets(const int32_t *cu_seqlens, int n_seqs, int64_t *
   return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_tc(const BwdProblem &p, const float *ckpt, const int64_t *ckpt_off, const int32_t *schedule,
-                          int32_t *status, int32_t *counter, cudaStream_t stream) {
+cudaError_t launch_bwd_tc(const BwdProblem &p, const void *ckpt, const float *S_fin, const int64_t *ckpt_off,
+                          const int32_t *schedule, int32_t *status, int32_t *counter, cudaStream_t stream) {
   BwdTcParams P;
   memset(&P, 0, sizeof(P));
   P.q = static_cast<const __nv_bfloat16 *>(p.q);
@@ -804,7 +935,8 @@ cudaError_t launch_bwd_tc(const BwdProblem &p, const float *ckpt, const int64_t 
   P.dS_T = p.dS_T;
   P.dq = p.dq; P.dk = p.dk; P.dv = p.dv; P.dlog_a = p.dlog_a; P.db = p.db; P.dw = p.dw;
   P.dS0 = p.dS0;
-  P.ckpt = ckpt;
+  P.ckpt = static_cast<const uint8_t *>(ckpt);
+  P.S_fin = S_fin;
   P.ckpt_off = ckpt_off;
   P.cu_seqlens = p.cu_seqlens;
   P.schedule = schedule;
@@ -815,11 +947,18 @@ cudaError_t launch_bwd_tc(const BwdProblem &p, const float *ckpt, const int64_t 
   P.seq_len = p.seq_len;
   P.wait_ns = kWaitTimeoutNs;
   if (P.n_units == 0) return cudaSuccess;
+  const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
+  const int64_t T = p.t_total > 0 ? p.t_total : 1;
+  bool ok = make_row_tile_map(&P.tm_q, p.q, T, p.n_heads) && make_row_tile_map(&P.tm_k, p.k, T, p.n_heads) &&
+            make_row_tile_map(&P.tm_v, p.v, T, p.n_heads) && make_row_tile_map(&P.tm_g, p.log_a, T, p.n_heads) &&
+            make_row_tile_map(&P.tm_b, p.b, T, p.n_heads);
+  if (ok && !tied) ok = make_row_tile_map(&P.tm_w, p.w, T, p.n_heads);
+  if (ok && p.dtype_out == GDN2_BF16) ok = make_row_tile_map(&P.tm_do, p.dO, T, p.n_heads);
+  if (!ok) return cudaErrorInvalidValue;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = P.n_units < sms ? P.n_units : sms;
-  const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
   if (p.dtype_out == GDN2_BF16)
     return tied ? launch_t<__nv_bfloat16, true>(P, grid, stream) : launch_t<__nv_bfloat16, false>(P, grid, stream);
   return tied ? launch_t<float, true>(P, grid, stream) : launch_t<float, false>(P, grid, stream);

@@ -68,6 +68,7 @@ constexpr float kLog2eF = 1.4426950408889634f;
 // a state term that underflows in S_r = e^{L_ref} S can only have been worth e^{64 - 87.3}
 // of the state's size in any output.
 constexpr float kFastSpan = 128.f;
+constexpr size_t kCkptBytes = (size_t)D * D * 2;  // one bf16 S_r tile image
 
 // Shared-memory map, byte offsets from a 1024-byte-aligned base.  Every operand
 // tile is a stack of 8-row x 128-byte swizzle atoms.
@@ -580,9 +581,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       len = p.seq_len;
     }
     const int nchunks = (int)((len + C - 1) / C);
-    // chunk-boundary states for the backward (gdn2_chunk_bwd): slot ci holds the state before
-    // chunk ci (as S = tau Sacc when the chunk starts), slot nchunks the final state
-    float *ck_unit = p.ckpt ? p.ckpt + ckpt_first_slot(p.ckpt_off, n, h, H, nchunks) * (D * D) : nullptr;
+    // chunk-start states for the backward (gdn2_chunk_bwd): slot ci receives the bf16 S_r of
+    // chunk ci as this chunk builds it, in the swizzled [d_k rows][d_v] tile image the backward
+    // copies to shared memory as it is (chunks of the token-serial form write nothing)
+    uint8_t *ck_unit = p.ckpt ? static_cast<uint8_t *>(p.ckpt) + ckpt_first_slot(p.ckpt_off, n, h, H, nchunks) * kCkptBytes
+                              : nullptr;
     if (tid == kIssuer && nchunks > 0 && !*sAbort) {
       issue_tma_l(h, (int)bos);
       issue_tma_a(h, (int)bos);
@@ -666,15 +669,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           issue_tma_w(h, t0 + C);
           issue_tma_a(h, t0 + C);
         }
-        if (ck_unit) {  // the state before this chunk
-          uint32_t r[32];
-          ptx::tmem_ld32(tmS + lane_base + cg * 32, r);
-          ptx::tmem_wait_ld();
-          const float *tp = sDLb(par ^ 1u) + cg * 32;
-          float *dst = ck_unit + ((size_t)ci * D + cg * 32) * D + row;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) dst[(size_t)j * D] = (ci > 0 ? tp[j] : 1.f) * __uint_as_float(r[j]);
-        }
         serial_chunk<kScalarDecay, kScalarGates, kP3, kProlog, Tout>(p, gb, tmS + lane_base + cg * 32,
                                                                    ci > 0 ? sDLb(par ^ 1u) + cg * 32 : nullptr,
                                                                    t0, nvalid, h);
@@ -729,20 +723,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         }
         ptx::tmem_ld32(tmS + lane_base + cg * 32, r);
         ptx::tmem_wait_ld();
-        float *ck = ck_unit ? ck_unit + ((size_t)ci * D + cg * 32) * D + row : nullptr;
 #pragma unroll
         for (int j4 = 0; j4 < 8; ++j4) {
           const float4 t4 = ci > 0 ? *reinterpret_cast<const float4 *>(tp + 4 * j4) : make_float4(1.f, 1.f, 1.f, 1.f);
           const float4 s4 = *reinterpret_cast<const float4 *>(smv + 4 * j4);
-          const float g0 = __uint_as_float(r[4 * j4]) * t4.x, g1 = __uint_as_float(r[4 * j4 + 1]) * t4.y;
-          const float g2 = __uint_as_float(r[4 * j4 + 2]) * t4.z, g3 = __uint_as_float(r[4 * j4 + 3]) * t4.w;
-          if (ck) {  // the state before this chunk
-            ck[(size_t)(4 * j4) * D] = g0;
-            ck[(size_t)(4 * j4 + 1) * D] = g1;
-            ck[(size_t)(4 * j4 + 2) * D] = g2;
-            ck[(size_t)(4 * j4 + 3) * D] = g3;
-          }
-          const float f0 = g0 * s4.x, f1 = g1 * s4.y, f2 = g2 * s4.z, f3 = g3 * s4.w;
+          const float f0 = (__uint_as_float(r[4 * j4]) * t4.x) * s4.x;
+          const float f1 = (__uint_as_float(r[4 * j4 + 1]) * t4.y) * s4.y;
+          const float f2 = (__uint_as_float(r[4 * j4 + 2]) * t4.z) * s4.z;
+          const float f3 = (__uint_as_float(r[4 * j4 + 3]) * t4.w) * s4.w;
           r[4 * j4] = __float_as_uint(f0);
           r[4 * j4 + 1] = __float_as_uint(f1);
           r[4 * j4 + 2] = __float_as_uint(f2);
@@ -752,6 +740,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         }
         ptx::tmem_st32(tmS + lane_base + cg * 32, r);
         ptx::tmem_st16(tmSR + lane_base + cg * 16, hb);
+        if (ck_unit) {  // S_r[i][j] of this chunk, i = 32 cg + jj, j = `row`
+          uint8_t *img = ck_unit + (size_t)ci * kCkptBytes;
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) {
+            const uint32_t pair = hb[jj >> 1];
+            *reinterpret_cast<uint16_t *>(img + swz_elem(cg * 32 + jj, row, 16384u)) =
+                (uint16_t)((jj & 1) ? (pair >> 16) : (pair & 0xffffu));
+          }
+        }
         ptx::tmem_wait_st();
       }
       ptx::tc_fence_before();
@@ -1111,19 +1108,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       waitb(bar(BAR_G5), (it & 1u) ^ 1u);
       ptx::tc_fence_after();
     }
-    if ((p.S_T || ck_unit) && !*sAbort) {
-      float *dst = p.S_T ? p.S_T + ((size_t)unit * D + cg * 32) * D + row : nullptr;
-      float *ck = ck_unit ? ck_unit + ((size_t)nchunks * D + cg * 32) * D + row : nullptr;
+    if (p.S_T && !*sAbort) {
+      float *dst = p.S_T + ((size_t)unit * D + cg * 32) * D + row;
       const float *tp = sDLb((it & 1u) ^ 1u) + cg * 32;  // the last chunk's e^{L_C - L_ref}
       uint32_t r[32];
       ptx::tmem_ld32(tmS + lane_base + cg * 32, r);
       ptx::tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float sv = (nchunks > 0 ? tp[j] : 1.f) * __uint_as_float(r[j]);
-        if (dst) dst[(size_t)j * D] = sv;
-        if (ck) ck[(size_t)j * D] = sv;
-      }
+      for (int j = 0; j < 32; ++j) dst[(size_t)j * D] = (nchunks > 0 ? tp[j] : 1.f) * __uint_as_float(r[j]);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -1223,6 +1215,10 @@ cudaError_t launch_gates(const TcParams &P, int grid, cudaStream_t stream, bool 
 }
 
 }  // namespace
+
+bool make_row_tile_map(CUtensorMap *m, const void *base, int64_t t_total, int H) {
+  return make_map(m, base, t_total, H);
+}
 
 cudaError_t launch_chunk_tc(const ChunkProblem &p, cudaStream_t stream, const char **why) {
   if (p.d_k != D || p.d_v != D || p.chunk != C || p.dtype_in != GDN2_BF16) {

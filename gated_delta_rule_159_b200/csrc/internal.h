@@ -2,6 +2,7 @@
 // and the kernel translation units.  Not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -28,11 +29,12 @@ struct ChunkProblem {
   // replaces cu_seqlens for the unit bounds, so the sequences may leave gaps between them
   // (the split forward's passes over a subset of segments).  Tensor-core path only.
   const int32_t *seg_bounds;
-  // Optional chunk-boundary state buffer for the backward (tensor-core path only): fp32
-  // [slots][d_k][d_v], the slots of a unit laid out as tc::ckpt_first_slot states; ckpt_off
-  // [n_seqs + 1] (int64) is the first slot of each sequence divided by n_heads, or NULL for
-  // equal lengths.  With ckpt set, o may be NULL (no output written).
-  float *ckpt;
+  // Optional chunk-start state buffer for the backward (tensor-core path only): per chunk the
+  // bf16 S_r = Diag(e^{L_ref}) S tile image (32 KB, the chunk kernel's swizzled [d_k][d_v]
+  // layout), the slots of a unit laid out as tc::ckpt_first_slot says; ckpt_off [n_seqs + 1]
+  // (int64) is the first slot of each sequence divided by n_heads, or NULL for equal lengths.
+  // With ckpt set, o may be NULL (no output written).
+  void *ckpt;
   const int64_t *ckpt_off;
 };
 
@@ -83,11 +85,11 @@ cudaError_t launch_bwd(const BwdProblem &p, cudaStream_t stream);
 // Chunked tensor-core backward (bwd_tc.cu; d_k = d_v = 128, bf16 inputs, per-channel gates in
 // the default placement, tied or not).  Checkpoint slots a call needs (an upper bound for
 // packed batches), the per-sequence slot offsets for packed batches, and the reverse kernel
-// over the states a checkpointing forward wrote (ChunkProblem::ckpt).
+// over the S_r tiles a checkpointing forward wrote (ChunkProblem::ckpt) and its final states.
 size_t bwd_tc_ckpt_slots(int64_t n_seqs, int64_t t_total, int n_heads, bool packed, int seq_len);
 cudaError_t launch_ckpt_offsets(const int32_t *cu_seqlens, int n_seqs, int64_t *off, cudaStream_t stream);
-cudaError_t launch_bwd_tc(const BwdProblem &p, const float *ckpt, const int64_t *ckpt_off, const int32_t *schedule,
-                          int32_t *status, int32_t *counter, cudaStream_t stream);
+cudaError_t launch_bwd_tc(const BwdProblem &p, const void *ckpt, const float *S_fin, const int64_t *ckpt_off,
+                          const int32_t *schedule, int32_t *status, int32_t *counter, cudaStream_t stream);
 
 // Sequence-parallel forward (seqpar.cu): segments of seg_len tokens, workspace offsets.
 struct SplitPlan {
@@ -138,5 +140,9 @@ cudaError_t launch_chunk_simt(const ChunkProblem &p, cudaStream_t stream);
 // Tensor-core path (d_k = d_v = 128, C = 64, bf16 in).  Returns cudaErrorNotSupported
 // when the problem is outside what it handles.
 cudaError_t launch_chunk_tc(const ChunkProblem &p, cudaStream_t stream, const char **why);
+// Tensor map of a [t_total][H][128] bf16 tensor viewed as (channel, head, token): boxes of 64
+// channels x 1 head x 64 tokens with the 128-byte swizzle (the tile layout of the tensor-core
+// kernels).  False when the driver entry point is missing or the geometry is rejected.
+bool make_row_tile_map(CUtensorMap *m, const void *base, int64_t t_total, int H);
 
 }  // namespace gdn2

@@ -109,13 +109,13 @@ __device__ __forceinline__ uint2 pack4(float a, float b, float c, float d) {
   return make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
 }
 
-// First checkpoint slot of unit (n, h) in the chunk-boundary state buffer: sequence n owns
-// (nchunks_n + 1) * H consecutive slots from ckpt_off[n] * H (n * (nchunks + 1) * H for equal
-// lengths, ckpt_off == NULL), head h the (nchunks_n + 1) of them from h * (nchunks_n + 1);
-// slot c holds the state before chunk c, slot nchunks_n the final state.
+// First checkpoint slot of unit (n, h) in the chunk-start state buffer: sequence n owns
+// nchunks_n * H consecutive slots from ckpt_off[n] * H (n * nchunks * H for equal lengths,
+// ckpt_off == NULL), head h the nchunks_n of them from h * nchunks_n; slot c holds chunk c's
+// start state.
 __device__ __forceinline__ int64_t ckpt_first_slot(const int64_t *ckpt_off, int n, int h, int H, int nchunks) {
-  const int64_t base = ckpt_off ? ckpt_off[n] : (int64_t)n * (nchunks + 1);
-  return base * H + (int64_t)h * (nchunks + 1);
+  const int64_t base = ckpt_off ? ckpt_off[n] : (int64_t)n * nchunks;
+  return base * H + (int64_t)h * nchunks;
 }
 
 }  // namespace tc

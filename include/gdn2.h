@@ -362,8 +362,9 @@ size_t gdn2_bwd_workspace_size(const gdn2_dims *dims, int32_t packed);
  * tensor cores.  The method trains through its chunked form with a gate-aware backward
  * (gist.science Methodologie 3, "Poortbewuste terugwaartse pass"); the pages print no
  * formula for it, and this call differentiates the chunk algebra of gdn2_chunk_fwd:
- *   1. a pass of the chunked forward writes the state before every 64-token chunk, and
- *      the final state, to the workspace (fp32; o is not written);
+ *   1. a pass of the chunked forward writes each 64-token chunk's start state (as the
+ *      bf16 operand tile the chunk uses) and the final state (fp32) to the workspace;
+ *      o is not written;
  *   2. one reverse pass per (sequence, head), last chunk first, recomputes each chunk's
  *      auxiliaries from its start state and forms every gradient of the chunk with
  *      bf16 tensor-core products accumulated in fp32, carrying dLoss/dS (fp32) from chunk
@@ -380,8 +381,8 @@ size_t gdn2_bwd_workspace_size(const gdn2_dims *dims, int32_t packed);
  * GDN2_ERR_RANGE for gdn2_check_status(workspace) and that (sequence, head)'s gradients are
  * undefined; gdn2_bwd handles any range.
  * workspace  >= gdn2_chunk_bwd_workspace_size(dims, packed) bytes, 256-byte aligned; one
- *            call at a time per workspace.  It holds the checkpoints: 64 KB per chunk and
- *            (sequence, head), plus one final state each.
+ *            call at a time per workspace.  It holds the checkpoints: 32 KB per chunk and
+ *            (sequence, head), plus one fp32 final state each.
  * Errors: GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_WORKSPACE, GDN2_ERR_CUDA;
  * gdn2_check_status reports GDN2_ERR_TIMEOUT (a bounded device wait) or GDN2_ERR_RANGE.
  */
