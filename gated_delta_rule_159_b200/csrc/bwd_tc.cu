@@ -99,10 +99,11 @@ constexpr uint32_t MISC_RHO = 128;     // float[128]     rho of the current chun
 constexpr uint32_t MISC_ESR = 640;     // float[2][128]  e^{rho} per chunk parity
 constexpr uint32_t MISC_DLC = 1664;    // float[2][128]  decay term of L_63 per chunk parity
 constexpr uint32_t MISC_L0 = 2688;     // float[128]     L_0
-constexpr uint32_t MISC_PART = 3200;   // float[4][128]  per-row-group sums (cumulative decay, dL)
+constexpr uint32_t MISC_PART = 3200;   // float[4][128]  per-row-group sums of dL
 constexpr uint32_t MISC_LPRE = 5248;   // float[4][128]  exclusive row-group prefixes of L
 constexpr uint32_t MISC_RS = 7296;     // float[4][128]  row sums per lane quadrant
-constexpr uint32_t MISC_BYTES = 9344;
+constexpr uint32_t MISC_GAM = 9344;    // float[128]     gamma = e^{L_63 - rho} of the current chunk
+constexpr uint32_t MISC_BYTES = 9856;
 constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES + 1024;  // + base alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 limit per CTA");
 enum { BAR_LD = 0, BAR_G1, BAR_GA, BAR_GB, BAR_G5, BAR_G7, BAR_DRAIN, kNumBars };
@@ -178,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
   float *part = reinterpret_cast<float *>(gb + OFF_MISC + MISC_PART);
   float *lpre = reinterpret_cast<float *>(gb + OFF_MISC + MISC_LPRE);
   float *rs = reinterpret_cast<float *>(gb + OFF_MISC + MISC_RS);
+  float *sGam = reinterpret_cast<float *>(gb + OFF_MISC + MISC_GAM);
   volatile int *sAbort = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_ABORT);
   volatile int *sUnit = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_UNIT);
   volatile int *sWide = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_WIDE);
@@ -191,12 +193,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
     return reinterpret_cast<float *>(gb + (i < 32 ? OFF_AT0 : OFF_AT1) +
                                      (uint32_t)(((i & 31) * 64 + (j ^ ((i & 7) << 2))) * 4));
   };
-  // L_ref of channel i from the row-group sums (the same expression in every thread)
-  auto rho_of = [&](int i, float &tot) {
-    tot = ((part[i] + part[128 + i]) + part[256 + i]) + part[384 + i];
-    return 0.5f * (sL0[i] + tot);
-  };
-
   if (tid == 0) {
     for (int i = 0; i < kNumBars; ++i) ptx::mbar_init(bar(i), 1);
     ptx::fence_mbar_init();
@@ -338,67 +334,84 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       }
       waitb(bar(BAR_LD), ld_it & 1u);
       ++ld_it;
-      // cumulative log-decay of channel `row` over rows [16 cg, 16 cg + 16) (rows past the chunk
-      // end decay by nothing; their V rows are zeroed); the dO rows go to their tile
-      float Lloc[16];
+      // cumulative log-decay, thread: channels 4 lane .. 4 lane + 3, rows 4 warp .. 4 warp + 3
+      // (8-byte accesses); rows past the chunk end decay by nothing and their V and dO rows
+      // are zeroed.  Row-group sums go to a [16][128] scratch in the [B; QP] tile (free until
+      // the masks).
+      float *part16 = reinterpret_cast<float *>(gb + OFF_BQP);
+      const int e_kb = lane >> 4;
+      const uint32_t e_ch16 = (uint32_t)((lane & 15) >> 1), e_cofs = (uint32_t)(lane & 1) * 8u;
+      float4 L4[4];
       {
-        float acc = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          const int r = 16 * cg + t;
-          const uint32_t o = swz_elem(r, row, 16384u);
-          const float la = r < nvalid ? bf16_value(lds_u16(sb + OFF_GRAW + swz_elem(r, row, 8192u))) : 0.f;
-          acc += la;
-          Lloc[t] = acc;
-          if (r >= nvalid) {
-            sts_u16(sb + OFF_MV + 8192u + o, 0);
-            if (kDoTma) sts_u16(sb + OFF_RO + 8192u + o, 0);
+        for (int rr = 0; rr < 4; ++rr) {
+          const int r = warp * 4 + rr;
+          float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (r < nvalid) {
+            g4 = unpack4(lds_v2(sb + OFF_GRAW + (uint32_t)e_kb * 8192u + swz(r, e_ch16) + e_cofs));
+          } else {
+            const uint32_t o = (uint32_t)e_kb * 16384u + 8192u + swz(r, e_ch16) + e_cofs;
+            sts_v2(sb + OFF_MV + o, make_uint2(0u, 0u));
+            if (kDoTma) sts_v2(sb + OFF_RO + o, make_uint2(0u, 0u));
           }
+          acc.x += g4.x; acc.y += g4.y; acc.z += g4.z; acc.w += g4.w;
+          L4[rr] = acc;
         }
-        part[cg * 128 + row] = acc;
-        if (cg == 0) sL0[row] = Lloc[0];
+        *reinterpret_cast<float4 *>(part16 + warp * 128 + 4 * lane) = acc;
+        if (warp == 0) *reinterpret_cast<float4 *>(sL0 + 4 * lane) = L4[0];
       }
       if (tid == 0) *sWide = 0;
       __syncthreads();
-      float pre, rho;
-      {
-        float tot;
-        rho = rho_of(row, tot);
-        pre = cg == 0 ? 0.f : part[row];
-        if (cg > 1) pre += part[128 + row];
-        if (cg > 2) pre += part[256 + row];
-        if (cg == 0) {
-          if (!(sL0[row] - tot <= kFastSpan)) *sWide = 1;
-          sRho[row] = rho;
-          sEsr[par * 128 + row] = ptx::ex2(rho * kLog2eF);
-        }
-        lpre[cg * 128 + row] = pre;
-      }
-      // k_r, q_r, x_r, p_r over the raw k, q, b, w rows (rows past the chunk end are zeroed)
+      if (tid < D) {  // per channel: exclusive prefixes over the 16 row groups, L_ref, the range check
+        float run = 0.f;
 #pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        const int r = 16 * cg + t;
-        const uint32_t o0 = swz_elem(r, row, 16384u), o1 = swz_elem(64 + r, row, 16384u);
-        float kk = 0.f, qq = 0.f, bb = 0.f, ww = 0.f;
-        if (r < nvalid) {
-          kk = bf16_value(lds_u16(sb + OFF_KQ + o0));
-          qq = bf16_value(lds_u16(sb + OFF_KQ + o1));
-          bb = bf16_value(lds_u16(sb + OFF_XP + o0));
-          ww = kTied ? bb : bf16_value(lds_u16(sb + OFF_XP + o1));
+        for (int j = 0; j < 16; ++j) {
+          const float pj = part16[j * 128 + tid];
+          part16[j * 128 + tid] = run;
+          if ((j & 3) == 0) lpre[(j >> 2) * 128 + tid] = run;  // the epilogue's 16-row groups
+          run += pj;
         }
-        const float L = pre + Lloc[t];
-        const float e = ptx::ex2((L - rho) * kLog2eF), f = ptx::ex2((rho - L) * kLog2eF);
-        sts_u16(sb + OFF_KQ + o0, bf16_bits(kk * e));
-        sts_u16(sb + OFF_KQ + o1, bf16_bits(qq * e));
-        sts_u16(sb + OFF_XP + o0, bf16_bits(bb * kk * f));
-        sts_u16(sb + OFF_XP + o1, bf16_bits(ww * kk * f));
+        const float l0 = sL0[tid];
+        const float rho = 0.5f * (l0 + run);
+        if (!(l0 - run <= kFastSpan)) *sWide = 1;
+        sRho[tid] = rho;
+        sGam[tid] = ptx::ex2((run - rho) * kLog2eF);
+        sEsr[par * 128 + tid] = ptx::ex2(rho * kLog2eF);
+      }
+      __syncthreads();
+      // k_r, q_r, x_r, p_r over the raw k, q, b, w rows (zero past the chunk end)
+      {
+        const float4 off = *reinterpret_cast<const float4 *>(part16 + warp * 128 + 4 * lane);
+        const float4 ref = *reinterpret_cast<const float4 *>(sRho + 4 * lane);
+        const float4 base = make_float4((off.x - ref.x) * kLog2eF, (off.y - ref.y) * kLog2eF,
+                                        (off.z - ref.z) * kLog2eF, (off.w - ref.w) * kLog2eF);
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          const int r = warp * 4 + rr;
+          const uint32_t o0 = (uint32_t)e_kb * 16384u + swz(r, e_ch16) + e_cofs, o1 = o0 + 8192u;
+          const float l0 = fmaf(L4[rr].x, kLog2eF, base.x), l1 = fmaf(L4[rr].y, kLog2eF, base.y);
+          const float l2 = fmaf(L4[rr].z, kLog2eF, base.z), l3 = fmaf(L4[rr].w, kLog2eF, base.w);
+          const float4 e = make_float4(ptx::ex2(l0), ptx::ex2(l1), ptx::ex2(l2), ptx::ex2(l3));
+          const float4 f = make_float4(ptx::ex2(-l0), ptx::ex2(-l1), ptx::ex2(-l2), ptx::ex2(-l3));
+          float4 kk = make_float4(0.f, 0.f, 0.f, 0.f), qq = kk, bb = kk, ww = kk;
+          if (r < nvalid) {
+            kk = unpack4(lds_v2(sb + OFF_KQ + o0));
+            qq = unpack4(lds_v2(sb + OFF_KQ + o1));
+            bb = unpack4(lds_v2(sb + OFF_XP + o0));
+            ww = kTied ? bb : unpack4(lds_v2(sb + OFF_XP + o1));
+          }
+          const float4 kf = make_float4(kk.x * f.x, kk.y * f.y, kk.z * f.z, kk.w * f.w);
+          sts_v2(sb + OFF_KQ + o0, pack4(kk.x * e.x, kk.y * e.y, kk.z * e.z, kk.w * e.w));
+          sts_v2(sb + OFF_KQ + o1, pack4(qq.x * e.x, qq.y * e.y, qq.z * e.z, qq.w * e.w));
+          sts_v2(sb + OFF_XP + o0, pack4(bb.x * kf.x, bb.y * kf.y, bb.z * kf.z, bb.w * kf.w));
+          sts_v2(sb + OFF_XP + o1, pack4(ww.x * kf.x, ww.y * kf.y, ww.z * kf.z, ww.w * kf.w));
+        }
       }
       // Lam_g = Diag(gamma e^{rho_next}) Acc, the bf16 tile [d_k rows][d_v] and the fp32 base of
       // this chunk's adjoint update (thread: d_k channel `row`, d_v channels [32 cg, 32 cg + 32))
       {
-        float tot;
-        const float ri = rho_of(row, tot);
-        const float gam = ptx::ex2((tot - ri) * kLog2eF);
+        const float gam = sGam[row];
         const float efac = sEsr[(par ^ 1u) * 128 + row];
         uint32_t r[32];
         float lg[32];
@@ -753,6 +766,22 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmZ, mnmaj(sb + OFF_XP, kk), kmaj(sb + OFF_DG, kk), idNK, 1);
         ptx::umma_commit(bar(BAR_G7));
       }
+      // the raw inputs of the epilogue's rows [16 cg, 16 cg + 8) (channel `row`), requested while
+      // the last products run; rows past the chunk end re-read its last row and are ignored
+      __nv_bfloat16 rla[8], rk[8], rq[8], rb[8], rw[8];
+      auto load_raw = [&](int c0) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int t = c0 + j, tc = t < nvalid ? t : nvalid - 1;
+          const size_t gi = ((size_t)(t0 + tc) * H + h) * D + row;
+          rla[j] = P.log_a[gi];
+          rk[j] = P.k[gi];
+          rq[j] = P.q[gi];
+          rb[j] = P.b[gi];
+          rw[j] = kTied ? rb[j] : g_w[gi];
+        }
+      };
+      load_raw(cg * 16);
       waitb(bar(BAR_G7), par);
       ptx::tc_fence_after();
       // every tile is free (the epilogue reads TMEM and global memory only): the next chunk's
@@ -774,19 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           ptx::tmem_ld8(tmX + lane_base + 64u + (uint32_t)c0, vp);
           ptx::tmem_ld8(tmZ + lane_base + (uint32_t)c0, vk);
           ptx::tmem_ld8(tmZ + lane_base + 64u + (uint32_t)c0, vq);
-          // the raw inputs of the 8 rows, all requested before any is used (rows past the
-          // chunk end re-read its last row and are ignored)
-          __nv_bfloat16 rla[8], rk[8], rq[8], rb[8], rw[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int t = c0 + j, tc = t < nvalid ? t : nvalid - 1;
-            const size_t gi = ((size_t)(t0 + tc) * H + h) * D + i;
-            rla[j] = P.log_a[gi];
-            rk[j] = P.k[gi];
-            rq[j] = P.q[gi];
-            rb[j] = P.b[gi];
-            rw[j] = kTied ? rb[j] : g_w[gi];
-          }
+          if (half == 1) load_raw(c0);  // the first half's were requested before the wait
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
