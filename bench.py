@@ -27,8 +27,10 @@ prefill (tokens/s and fraction of HBM bandwidth), the roofline of the chunk
 kernel, the end-to-end number through host buffers, the float64 CPU oracle as
 `cpu_baseline`, and the SM clocks sampled while timing.
 
-`bwd` times gdn2_bwd (all gradients of the forward, fp32 reverse mode) on the
-prefill workload with random dO and dS_T.
+`bwd` times gdn2_chunk_bwd (all gradients of the forward: a checkpointing
+chunked forward, then the chunked reverse pass on the tensor cores) on the
+prefill workload with random bf16 dO and dS_T; `bwd.token_serial` times the
+fp32 token-serial gdn2_bwd on the same inputs once, for comparison.
 
 `--impl reference` times the float64 CPU oracle on a bounded sample of the
 same workload instead (rank 0 only).
@@ -62,10 +64,22 @@ FLOP_PER_TOKHEAD_TIED = FLOP_PER_TOKHEAD - 4 * 64 * 128
 BYTES_PER_TOKHEAD = 6 * 128 * 2 + 128 * 2                      # six bf16 inputs + bf16 o
 BYTES_PER_TOKHEAD_SCALAR = 3 * 128 * 2 + 2 * 2 + 128 * 2       # q, k, v + scalar alpha, beta + o
 STATE_BYTES = 128 * 128 * 4                                    # one fp32 state
-# fp32 operations of the backward per token-head (d_k = d_v = 128): per state
-# element, the forward sweep and the block recompute take 7 each (decay, erase
+# fp32 operations of the token-serial backward per token-head (d_k = d_v = 128): per
+# state element, the forward sweep and the block recompute take 7 each (decay, erase
 # read, erase and write updates) and the reverse step 26.
 BWD_FLOP_PER_TOKHEAD = (7 + 7 + 26) * 128 * 128
+# tcgen05 products of the chunked backward per chunk-head (C = 64, d = 128): G1 128x128x128,
+# dM 128x64x(128 + 64), R 128x64x192, M and dR 128x64x64 each, [dA dB; dQX dQP], the adjoint
+# update and the S_r terms of dk_r, dq_r 128x128x128 each, dV 128x64x256, [dx_r | dp_r]
+# 128x128x256, the rest of dk_r, dq_r 128x128x128; per token-head, plus the checkpointing
+# forward's products.
+CBWD_FLOP_PER_TOKHEAD = 2 * (128 * 128 * 128 * 5 + 128 * 64 * (192 + 192 + 64 + 64 + 256)
+                             + 128 * 128 * 256) // 64 + FLOP_PER_TOKHEAD
+# DRAM bytes of one gdn2_chunk_bwd per token-head: the forward reads the six bf16 inputs and
+# writes the bf16 S_r checkpoint (32 KB per 64 tokens); the reverse pass reads the six inputs,
+# dO and the checkpoint and writes six bf16 gradients (final states and dS_T, dS0 per sequence
+# are not counted)
+CBWD_BYTES_PER_TOKHEAD = 6 * 256 + 512 + (7 * 256 + 512) + 6 * 256
 
 
 def fp32_peak_tflops(sm_max_mhz: float) -> float:
@@ -84,7 +98,7 @@ def peaks():
 
 def kernel_sha() -> str:
     h = hashlib.sha256()
-    for f in ("chunk_tc.cu", "sm100_ptx.cuh", "common.cuh"):
+    for f in ("chunk_tc.cu", "sm100_ptx.cuh", "common.cuh", "tc_util.cuh"):
         with open(os.path.join(ROOT, "gated_delta_rule_159_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -296,6 +310,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--bwd-steps", type=int, default=3)
     ap.add_argument("--no-bwd", action="store_true")
+    ap.add_argument("--no-token-serial-bwd", action="store_true",
+                    help="skip the one timed step of the token-serial gdn2_bwd")
     ap.add_argument("--no-long", action="store_true")
     ap.add_argument("--split", type=int, default=0,
                     help="segments per sequence of the long-context split forward (0: as many as keep "
@@ -626,12 +642,13 @@ def main():
         dS_T = torch.randn(Nb, 16, 128, 128, generator=gen, device=dev) * 0.1
         bargs = [bi[n].view(Nb, Tb, *bi[n].shape[1:]) for n in names]
         bdims = gdn2.make_dims(Nb, Tb, 16, 128, 128, 64, gdn2.BF16, gdn2.BF16, 0)
-        bws = torch.empty(gdn2.bwd_workspace_size(bdims), dtype=torch.uint8, device=dev)
+        cws = torch.empty(gdn2.chunk_bwd_workspace_size(bdims), dtype=torch.uint8, device=dev)
 
-        def bstep():
-            return gdn2.bwd(*bargs, dO, S0=bi["S0"], dS_T=dS_T, workspace=bws)
+        def cstep():
+            return gdn2.chunk_bwd(*bargs, dO, S0=bi["S0"], dS_T=dS_T, workspace=cws)
 
-        bstep()
+        for _ in range(3):
+            cstep()
         torch.cuda.synchronize()
         barrier()
         bs = ClockSampler(dev.index if dev.index is not None else 0)
@@ -639,23 +656,53 @@ def main():
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.bwd_steps):
-            bstep()
+            cstep()
         e1.record(stream)
         barrier()
         bclocks = bs.stop()
-        bms = rmax(e0.elapsed_time(e1)) / args.bwd_steps
+        cms = rmax(e0.elapsed_time(e1)) / args.bwd_steps
+        st = gdn2.lib.gdn2_check_status(gdn2._ptr(cws), gdn2._stream(dev))
         tokheads = Nb * Tb * 16
-        tflops = BWD_FLOP_PER_TOKHEAD * tokheads / (bms / 1e3) / 1e12
-        peak32 = fp32_peak_tflops(bclocks.get("sm_max_mhz") or 1965.0)
-        bwd = {"value": Nb * Tb * world / (bms / 1e3), "unit": "tokens/s", "ms_per_step": bms,
-               "steps": args.bwd_steps, "dtype": "f32 arithmetic, bf16 inputs and gradients",
-               "roofline": {"bound": "alu", "achieved": tflops, "peak": peak32, "unit": "TFLOP/s",
-                            "frac": tflops / peak32, "traffic": None,
-                            "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x sm_max_mhz",
-                            "alg_flops_per_tokhead": BWD_FLOP_PER_TOKHEAD},
-               "kernels": ["bwd_kernel", "finish_kernel"], "gpu_launches": 2 * args.bwd_steps,
-               "workspace_bytes": bws.numel(), "clocks": bclocks}
-        del bi, dO, dS_T, bargs, bws
+        gbs = CBWD_BYTES_PER_TOKHEAD * tokheads / (cms / 1e3) / 1e9
+        ctf = CBWD_FLOP_PER_TOKHEAD * tokheads / (cms / 1e3) / 1e12
+        bwd = {"value": Nb * Tb * world / (cms / 1e3), "unit": "tokens/s", "ms_per_step": cms,
+               "steps": args.bwd_steps, "status": st,
+               "dtype": "bf16 operands, fp32 accumulation (tcgen05), bf16 gradients",
+               "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                            "traffic": None, "peak_source": peak_src,
+                            "alg_bytes_per_tokhead": CBWD_BYTES_PER_TOKHEAD,
+                            "scope": "whole gdn2_chunk_bwd call (checkpointing forward + reverse pass)"},
+               "tensor": {"achieved": ctf, "peak": tc_peak, "unit": "TFLOP/s", "frac": ctf / tc_peak,
+                          "alg_flops_per_tokhead": CBWD_FLOP_PER_TOKHEAD},
+               "kernels": ["chunk_tc_kernel (checkpointing forward)", "bwd_tc_kernel"],
+               "gpu_launches": 2 * args.bwd_steps, "workspace_bytes": cws.numel(), "clocks": bclocks}
+        del cws
+        if not args.no_token_serial_bwd:
+            bws = torch.empty(gdn2.bwd_workspace_size(bdims), dtype=torch.uint8, device=dev)
+
+            def bstep():
+                return gdn2.bwd(*bargs, dO, S0=bi["S0"], dS_T=dS_T, workspace=bws)
+
+            bstep()
+            torch.cuda.synchronize()
+            barrier()
+            e0.record(stream)
+            bstep()
+            e1.record(stream)
+            barrier()
+            bms = rmax(e0.elapsed_time(e1))
+            tflops = BWD_FLOP_PER_TOKHEAD * tokheads / (bms / 1e3) / 1e12
+            peak32 = fp32_peak_tflops(bclocks.get("sm_max_mhz") or 1965.0)
+            bwd["token_serial"] = {
+                "value": Nb * Tb * world / (bms / 1e3), "unit": "tokens/s", "ms_per_step": bms, "steps": 1,
+                "dtype": "f32 arithmetic, bf16 inputs and gradients",
+                "roofline": {"bound": "alu", "achieved": tflops, "peak": peak32, "unit": "TFLOP/s",
+                             "frac": tflops / peak32, "traffic": None,
+                             "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x sm_max_mhz",
+                             "alg_flops_per_tokhead": BWD_FLOP_PER_TOKHEAD},
+                "kernels": ["bwd_kernel", "finish_kernel"], "workspace_bytes": bws.numel()}
+            del bws
+        del bi, dO, dS_T, bargs
 
     # ---------------- long context: one sequence of 65,536 tokens, 16 heads (16 units on 148
     # SMs), plain chunked forward against the sequence-parallel split forward
