@@ -70,6 +70,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s
 constexpr float kLog2eF = 1.4426950408889634f;
 constexpr float kFastSpan = 128.f;  // as in the forward: factors stay within e^{+-64}
+constexpr size_t kSlotBytes = kBwdCkptSlotBytes;  // per chunk: bf16 S_r tile image, then bf16 T
 
 // Shared-memory map (byte offsets from a 1024-byte-aligned base).  The 128-row operand tiles
 // are two column blocks of 64 (16 KB apart), each a stack of 8-row x 128-byte swizzle atoms.
@@ -80,13 +81,10 @@ constexpr uint32_t OFF_RO = 98304;      // [dR | dO]
 constexpr uint32_t OFF_SR = 131072;     // S_r [d_k rows][d_v]; from phase 7 the gradient tile dG
 constexpr uint32_t OFF_LG = 163840;     // Lam_g [d_k rows][d_v]
 constexpr uint32_t OFF_BQP = 196608;    // [B rows 0-63 | QP rows 64-127], one 64-column block
-constexpr uint32_t OFF_XS = 212992;     // fp32 solve scratch, 4 KB
-constexpr uint32_t OFF_MISC = 217088;
+constexpr uint32_t OFF_MISC = 212992;
 // Tiles that live in the rows of another tile until that tile is written:
 constexpr uint32_t OFF_T = OFF_MV;             // T bf16 [64 x 64] (the -M rows of block 0)
 constexpr uint32_t OFF_QX = OFF_MV + 16384;    // QX bf16 [64 x 64] (the -M rows of block 1)
-constexpr uint32_t OFF_AT0 = OFF_RO;           // fp32 A, then T, rows 0-31 [32][64] (dR rows, block 0)
-constexpr uint32_t OFF_AT1 = OFF_RO + 16384;   // rows 32-63 (dR rows, block 1)
 constexpr uint32_t OFF_DG = OFF_SR;            // [dA dB; dQX dQP] as [column block][128 rows][64]
 constexpr uint32_t OFF_GRAW = OFF_LG;          // raw log_a tile [2 blocks][64 rows] until Lam_g is built
 constexpr uint32_t MISC_BAR = 0;       // mbarriers
@@ -106,7 +104,7 @@ constexpr uint32_t MISC_GAM = 9344;    // float[128]     gamma = e^{L_63 - rho} 
 constexpr uint32_t MISC_BYTES = 9856;
 constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES + 1024;  // + base alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 limit per CTA");
-enum { BAR_LD = 0, BAR_G1, BAR_GA, BAR_GB, BAR_G5, BAR_G7, BAR_DRAIN, kNumBars };
+enum { BAR_LD = 0, BAR_G1, BAR_GA, BAR_GB, BAR_G5, BAR_GZ, BAR_G7, BAR_DRAIN, kNumBars };
 static_assert(MISC_BAR + 8 * kNumBars <= MISC_TMEM, "mbarriers overlap the TMEM address slot");
 
 struct BwdTcParams {
@@ -169,8 +167,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
   const int row = qd * 32 + lane;           // TMEM lane; the channel of the elementwise phases
   const int H = P.n_heads;
   constexpr int kIssuer = 480;              // warp 15 lane 0 issues every MMA, in order
-  constexpr int kSolveThreads = 480;        // warps 0-14
-  constexpr int NB_SOLVE = 1;
 
   float *sRho = reinterpret_cast<float *>(gb + OFF_MISC + MISC_RHO);
   float *sEsr = reinterpret_cast<float *>(gb + OFF_MISC + MISC_ESR);
@@ -186,13 +182,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
   volatile uint32_t *sIss = reinterpret_cast<volatile uint32_t *>(gb + OFF_MISC + MISC_ISS);
   auto bar = [&](int i) { return sb + OFF_MISC + MISC_BAR + 8u * (uint32_t)i; };
   auto waitb = [&](uint32_t b, uint32_t parity) { return wait_bar(b, parity, sAbort, P.status, P.wait_ns); };
-  // fp32 A / T of the solve: rows 0-31 and 32-63 in two 8 KB halves, 64 floats per row; the
-  // column index is XORed with 4 (row mod 8) so that the 8 rows of an mma fragment load fall
-  // in different banks (groups of four columns stay contiguous)
-  auto at = [&](int i, int j) -> float * {
-    return reinterpret_cast<float *>(gb + (i < 32 ? OFF_AT0 : OFF_AT1) +
-                                     (uint32_t)(((i & 31) * 64 + (j ^ ((i & 7) << 2))) * 4));
-  };
   if (tid == 0) {
     for (int i = 0; i < kNumBars; ++i) ptx::mbar_init(bar(i), 1);
     ptx::fence_mbar_init();
@@ -232,9 +221,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
   // tile image (thread kIssuer)
   constexpr bool kDoTma = sizeof(Tout) == 2;  // bf16 dO lands in its tile as it is
   auto issue_loads = [&](int h, int t0, const uint8_t *sr_img) {
-    ptx::mbar_arrive_expect_tx(bar(BAR_LD), ((kTied ? 5u : 6u) + (kDoTma ? 1u : 0u)) * 16384u + 32768u);
+    ptx::mbar_arrive_expect_tx(bar(BAR_LD), ((kTied ? 5u : 6u) + (kDoTma ? 1u : 0u)) * 16384u + (uint32_t)kSlotBytes);
     *sIss = *sIss + 1u;
     ptx::bulk_load(sb + OFF_SR, sr_img, 32768u, bar(BAR_LD));
+    ptx::bulk_load(sb + OFF_T, sr_img + 32768, 8192u, bar(BAR_LD));
 #pragma unroll
     for (int kb = 0; kb < 2; ++kb) {
       const uint32_t o = (uint32_t)kb * 16384u;
@@ -264,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       len = P.seq_len;
     }
     const int nchunks = (int)((len + C - 1) / C);
-    const uint8_t *ck_unit = P.ckpt + ckpt_first_slot(P.ckpt_off, n, h, H, nchunks) * (size_t)(D * D * 2);
+    const uint8_t *ck_unit = P.ckpt + ckpt_first_slot(P.ckpt_off, n, h, H, nchunks) * kSlotBytes;
 
     // ---- the final state's adjoint dS_T into TMEM (thread: d_k channel `row`, d_v channels
     //      [32 cg, 32 cg + 32)), and the decay term of the last chunk, sum_j dS_T S_T per d_k
@@ -289,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       if (tid < 128) sEsr[((it & 1u) ^ 1u) * 128 + tid] = 1.f;  // the last chunk reads dS_T unscaled
       // the last chunk's tiles (every tile is free: the previous unit's MMAs are done)
       if (tid == kIssuer && nchunks > 0 && !*sAbort)
-        issue_loads(h, (int)(bos + (int64_t)(nchunks - 1) * C), ck_unit + (size_t)(nchunks - 1) * (D * D * 2));
+        issue_loads(h, (int)(bos + (int64_t)(nchunks - 1) * C), ck_unit + (size_t)(nchunks - 1) * kSlotBytes);
     }
     __syncthreads();
     if (tid < 128)
@@ -312,8 +302,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
                           : tsel == 4 ? (const void *)(P.b + gi) : tsel == 5 ? (const void *)(g_w + gi)
                                       : (const void *)(g_do + gi);
           if (tsel != 5 || !kTied) ptx::bulk_prefetch_l2(src, tsel == 6 ? D * (uint32_t)sizeof(Tout) : D * 2u);
-        } else if (tid < 450) {
-          ptx::bulk_prefetch_l2(ck_unit + (size_t)(ci - 1) * (D * D * 2) + (size_t)(tid - 448) * 16384, 16384u);
+        } else if (tid < 451) {  // the 40 KB checkpoint slot: 16 + 16 + 8 KB
+          ptx::bulk_prefetch_l2(ck_unit + (size_t)(ci - 1) * kSlotBytes + (size_t)(tid - 448) * 16384,
+                                tid < 450 ? 16384u : 8192u);
         }
       }
       // fp32 dO: the rows of channel `row` into the bf16 tile (rows past the chunk end re-read
@@ -437,25 +428,26 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         break;
       }
 
-      // ================= phase 2: G1 and dM^T <- Lam_g^T x_r^T; masks
+      // ================= phase 2: G1, and the products that need no mask: dM^T = Lam_g^T x_r^T
+      //      and the S_r part of R^T = S_r^T k_r^T; the masks of G1
       if (tid == kIssuer && !*sAbort) {
         ptx::tc_fence_after();
         constexpr uint32_t idG1 = ptx::idesc_bf16(128, 128, false, false);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmX, kmaj(sb + OFF_KQ, kk), kmaj(sb + OFF_XP, kk), idG1, kk > 0);
         ptx::umma_commit(bar(BAR_G1));
-        constexpr uint32_t idM = ptx::idesc_bf16(128, 64, true, false);  // A = Lam_g^T (MN-major), B = x_r
+        constexpr uint32_t idM = ptx::idesc_bf16(128, 64, true, false);  // A MN-major (Lam_g^T, S_r^T)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmZ, mnmaj(sb + OFF_LG, kk), kmaj(sb + OFF_XP, kk), idM, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmY, mnmaj(sb + OFF_SR, kk), kmaj(sb + OFF_KQ, kk), idM, kk > 0);
       }
-      // the bf16 T tile (over the -M rows, free until phase 5) starts as zeros: the solve writes
-      // only the blocks on and below the diagonal
-      sts_v4(sb + OFF_T + 16u * (uint32_t)tid, make_uint4(0u, 0u, 0u, 0u));
       waitb(bar(BAR_G1), par);
       ptx::tc_fence_after();
-      {
-        // warp (qd, cg) reads G1 row `row`, columns [32 cg, 32 cg + 32): A | B for rows 0-63,
-        // QX | QP for rows 64-127; A, B strictly lower, QX, QP lower with the diagonal
+      if (!(row < 64 && cg < 2)) {
+        // warp (qd, cg) reads G1 row `row`, columns [32 cg, 32 cg + 32): B for rows 0-63 (strictly
+        // lower), QX | QP for rows 64-127 (lower with the diagonal); A is not needed (T came
+        // from the forward)
         uint32_t r[32];
         ptx::tmem_ld32(tmX + lane_base + cg * 32, r);
         ptx::tmem_wait_ld();
@@ -464,157 +456,31 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         float f[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) f[j] = (strict ? jb + j < i : jb + j <= i) ? __uint_as_float(r[j]) : 0.f;
-        if (strict && cg < 2) {  // A in fp32 for the solve
+        // B into rows 0-63 of [B; QP]; QX into its own tile; QP into rows 64-127 of [B; QP]
+        const uint32_t dst = strict ? sb + OFF_BQP : (cg < 2 ? sb + OFF_QX : sb + OFF_BQP + 8192u);
 #pragma unroll
-          for (int j4 = 0; j4 < 8; ++j4)
-            *reinterpret_cast<float4 *>(at(i, jb + 4 * j4)) =
-                make_float4(f[4 * j4], f[4 * j4 + 1], f[4 * j4 + 2], f[4 * j4 + 3]);
-        } else {
-          // B into rows 0-63 of [B; QP]; QX into its own tile; QP into rows 64-127 of [B; QP]
-          const uint32_t dst = strict ? sb + OFF_BQP : (cg < 2 ? sb + OFF_QX : sb + OFF_BQP + 8192u);
-#pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) sts_v4(dst + swz(i, (uint32_t)((cg & 1) * 4 + q8)), pack8(f + 8 * q8, 1.f));
-        }
+        for (int q8 = 0; q8 < 4; ++q8) sts_v4(dst + swz(i, (uint32_t)((cg & 1) * 4 + q8)), pack8(f + 8 * q8, 1.f));
+        ptx::fence_proxy_async_smem();
       }
-      ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncthreads();
 
-      // ================= phase 3: T = (I + A)^-1 (warps 0-14) || R^T, dM^T += dO^T QX (warp 15)
-      if (warp == 15) {
-        if (lane == 0 && !*sAbort) {
-          ptx::tc_fence_after();
-          // R^T = V^T B^T + S_r^T k_r^T
-          constexpr uint32_t idV = ptx::idesc_bf16(128, 64, true, false);
+      // ================= phase 3: the masked products: R^T += V^T B^T, dM^T += dO^T QX
+      if (tid == kIssuer && !*sAbort) {
+        ptx::tc_fence_after();
+        constexpr uint32_t idV = ptx::idesc_bf16(128, 64, true, false);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            ptx::umma_bf16(tmY, ptx::sdesc_sw128(sb + OFF_MV + 8192u + (uint32_t)kk * 2048u, 16384, 1024),
-                           ptx::sdesc_sw128(sb + OFF_BQP + (uint32_t)kk * 32u, 16, 1024), idV, kk > 0);
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::umma_bf16(tmY, ptx::sdesc_sw128(sb + OFF_MV + 8192u + (uint32_t)kk * 2048u, 16384, 1024),
+                         ptx::sdesc_sw128(sb + OFF_BQP + (uint32_t)kk * 32u, 16, 1024), idV, 1);
+        // QX as [s][t]: MN-major B
+        constexpr uint32_t idQ = ptx::idesc_bf16(128, 64, true, true);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmY, mnmaj(sb + OFF_SR, kk), kmaj(sb + OFF_KQ, kk), idV, 1);
-          // dM^T += dO^T QX (QX as [s][t]: MN-major B)
-          constexpr uint32_t idQ = ptx::idesc_bf16(128, 64, true, true);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            ptx::umma_bf16(tmZ, ptx::sdesc_sw128(sb + OFF_RO + 8192u + (uint32_t)kk * 2048u, 16384, 1024),
-                           ptx::sdesc_sw128(sb + OFF_QX + (uint32_t)kk * 2048u, 8192, 1024), idQ, 1);
-          ptx::umma_commit(bar(BAR_GA));
-        }
-        __syncwarp();
-      } else {
-        // 8x8 diagonal blocks by forward substitution (one thread per block column), then
-        // merges of block pairs of size s = 8, 16, 32: T_LU = -T_LL (A_LU T_UU).  A and T
-        // share one fp32 array: a block of T overwrites the block of A it came from once no
-        // thread reads that block any more.  Every final block also goes to the bf16 tile.
-        float a[28];
-        const int blk = tid >> 3, m = tid & 7, r0 = 8 * blk;
-        if (tid < 64) {
-          int nn = 0;
-#pragma unroll
-          for (int ii = 1; ii < 8; ++ii)
-#pragma unroll
-            for (int jj = 0; jj < ii; ++jj) a[nn++] = *at(r0 + ii, r0 + jj);
-        }
-        named_bar(NB_SOLVE, kSolveThreads);
-        if (tid < 64) {
-          float t[8];
-          int nn = 0;
-#pragma unroll
-          for (int ii = 0; ii < 8; ++ii) {
-            float acc = (ii == m) ? 1.f : 0.f;
-#pragma unroll
-            for (int jj = 0; jj < ii; ++jj) acc -= a[nn++] * t[jj];
-            t[ii] = acc;
-          }
-#pragma unroll
-          for (int ii = 0; ii < 8; ++ii) {
-            *at(r0 + ii, r0 + m) = t[ii];
-            sts_u16(sb + OFF_T + swz(r0 + ii, (uint32_t)blk) + (uint32_t)m * 2u, bf16_bits(t[ii]));
-          }
-        }
-        named_bar(NB_SOLVE, kSolveThreads);
-        float *Xs = reinterpret_cast<float *>(gb + OFF_XS);
-        // s = 8: 4 pairs x 64 outputs on CUDA cores
-        if (tid < 256) {
-          const int pr = tid >> 6, r = (tid >> 3) & 7, c = tid & 7, u0 = 16 * pr, l0 = u0 + 8;
-          float acc = 0.f;
-#pragma unroll
-          for (int k2 = 0; k2 < 8; ++k2) acc += (k2 >= c ? *at(l0 + r, u0 + k2) * *at(u0 + k2, u0 + c) : 0.f);
-          Xs[tid] = acc;
-        }
-        named_bar(NB_SOLVE, kSolveThreads);
-        if (tid < 256) {
-          const int pr = tid >> 6, r = (tid >> 3) & 7, c = tid & 7, u0 = 16 * pr, l0 = u0 + 8;
-          float acc = 0.f;
-#pragma unroll
-          for (int k2 = 0; k2 < 8; ++k2) acc -= (k2 <= r ? *at(l0 + r, l0 + k2) * Xs[pr * 64 + k2 * 8 + c] : 0.f);
-          *at(l0 + r, u0 + c) = acc;
-          sts_u16(sb + OFF_T + swz(l0 + r, (uint32_t)(u0 >> 3)) + (uint32_t)c * 2u, bf16_bits(acc));
-        }
-        named_bar(NB_SOLVE, kSolveThreads);
-        // s = 16 (2 pairs) and s = 32 (1 pair) on tf32 mma.sync, one warp per 16x8 output tile;
-        // each K step's fragments are loaded right before its MMA (few registers live)
-        const int g = lane >> 2, t4 = lane & 3;
-#pragma unroll
-        for (int lev = 1; lev < 3; ++lev) {
-          const int sz = 8 << lev;                   // 16, 32
-          const int nk = sz / 8;                     // 8-wide K steps: 2, 4
-          const int tpp = (sz / 16) * (sz / 8);      // 16x8 tiles per pair: 2, 8
-          const int ntiles = (64 / (2 * sz)) * tpp;  // 4, 8
-          const int pr = warp / tpp, ti = warp % tpp, mt = ti / (sz / 8), nt = ti % (sz / 8);
-          const int u0 = pr * 2 * sz, l0 = u0 + sz, rr = 16 * mt, cc = 8 * nt;
-          // X = A_LU T_UU (T_UU is lower triangular: K steps before the tile's first column vanish)
-          if (warp < ntiles) {
-            float x[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              if (kk < nk && kk >= nt) {
-                const int kc = u0 + 8 * kk + t4;
-                const uint32_t av[4] = {ptx::to_tf32(*at(l0 + rr + g, kc)), ptx::to_tf32(*at(l0 + rr + g + 8, kc)),
-                                        ptx::to_tf32(*at(l0 + rr + g, kc + 4)), ptx::to_tf32(*at(l0 + rr + g + 8, kc + 4))};
-                const uint32_t bv[2] = {ptx::to_tf32(*at(kc, u0 + cc + g)), ptx::to_tf32(*at(kc + 4, u0 + cc + g))};
-                ptx::mma_tf32_16x8x8(x, av, bv);
-              }
-            }
-            float *xs = Xs + pr * sz * sz;
-            xs[(rr + g) * sz + cc + 2 * t4] = x[0];
-            xs[(rr + g) * sz + cc + 2 * t4 + 1] = x[1];
-            xs[(rr + g + 8) * sz + cc + 2 * t4] = x[2];
-            xs[(rr + g + 8) * sz + cc + 2 * t4 + 1] = x[3];
-          }
-          named_bar(NB_SOLVE, kSolveThreads);
-          // T_LU = -T_LL X (K steps past the tile's last row vanish), over A_LU
-          if (warp < ntiles) {
-            const float *xs = Xs + pr * sz * sz;
-            float y[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              if (kk < nk && kk <= (rr + 15) / 8) {
-                // T_LL is lower triangular (its blocks above the diagonal hold zeros of A)
-                const int kc = l0 + 8 * kk + t4;
-                const uint32_t av[4] = {ptx::to_tf32(*at(l0 + rr + g, kc)), ptx::to_tf32(*at(l0 + rr + g + 8, kc)),
-                                        ptx::to_tf32(*at(l0 + rr + g, kc + 4)), ptx::to_tf32(*at(l0 + rr + g + 8, kc + 4))};
-                const uint32_t bv[2] = {ptx::to_tf32(xs[(8 * kk + t4) * sz + cc + g]),
-                                        ptx::to_tf32(xs[(8 * kk + t4 + 4) * sz + cc + g])};
-                ptx::mma_tf32_16x8x8(y, av, bv);
-              }
-            }
-            const int ri = l0 + rr + g, cj = u0 + cc + 2 * t4;
-            if (lev == 1) {  // the last level's T_LU is read by no later level: bf16 only
-              *at(ri, cj) = -y[0];
-              *at(ri, cj + 1) = -y[1];
-              *at(ri + 8, cj) = -y[2];
-              *at(ri + 8, cj + 1) = -y[3];
-            }
-            sts_u32(sb + OFF_T + swz(ri, (uint32_t)(cj >> 3)) + (uint32_t)(cj & 7) * 2u, pack_bf16x2(-y[0], -y[1]));
-            sts_u32(sb + OFF_T + swz(ri + 8, (uint32_t)(cj >> 3)) + (uint32_t)(cj & 7) * 2u, pack_bf16x2(-y[2], -y[3]));
-          }
-          if (lev == 1) named_bar(NB_SOLVE, kSolveThreads);
-        }
-        ptx::fence_proxy_async_smem();  // the bf16 T tile is read by the tensor core
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::umma_bf16(tmZ, ptx::sdesc_sw128(sb + OFF_RO + 8192u + (uint32_t)kk * 2048u, 16384, 1024),
+                         ptx::sdesc_sw128(sb + OFF_QX + (uint32_t)kk * 2048u, 8192, 1024), idQ, 1);
+        ptx::umma_commit(bar(BAR_GA));
       }
-      ptx::tc_fence_before();
-      __syncthreads();
 
       // ================= phase 4: R^T and -dM^T as bf16 TMEM operands; M^T, dR^T
       waitb(bar(BAR_GA), par);
@@ -671,17 +537,21 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       ptx::tc_fence_before();
       __syncthreads();
 
-      // ================= phase 6: [dA dB; dQX dQP] = [dR; dO][-M; V]^T, the adjoint update
-      //      Acc += [k_r; q_r]^T [dR; dO], dV^T = [dR; dO]^T [B; QP] + Lam_g^T p_r^T and the
-      //      S_r terms [dk_r^T | dq_r^T] = S_r [dR; dO]^T
+      // ================= phase 6: the adjoint update Acc += [k_r; q_r]^T [dR; dO], the S_r terms
+      //      [dk_r^T | dq_r^T] = S_r [dR; dO]^T and [dA dB; dQX dQP] = [dR; dO][-M; V]^T (commit
+      //      G5: the masks and the decay term need these), then dV^T = [dR; dO]^T [B; QP] +
+      //      Lam_g^T p_r^T, which runs under the masks (the epilogue reads it)
       if (tid == kIssuer && !*sAbort) {
         ptx::tc_fence_after();
         constexpr uint32_t idKK = ptx::idesc_bf16(128, 128, false, false);
         constexpr uint32_t idNN = ptx::idesc_bf16(128, 128, true, true);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmX, kmaj(sb + OFF_RO, kk), kmaj(sb + OFF_MV, kk), idKK, kk > 0);
-#pragma unroll
         for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmAcc, mnmaj(sb + OFF_KQ, kk), mnmaj(sb + OFF_RO, kk), idNN, 1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmZ, kmaj(sb + OFF_SR, kk), kmaj(sb + OFF_RO, kk), idKK, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmX, kmaj(sb + OFF_RO, kk), kmaj(sb + OFF_MV, kk), idKK, kk > 0);
+        ptx::umma_commit(bar(BAR_G5));
         constexpr uint32_t idV1 = ptx::idesc_bf16(128, 64, true, true);
         constexpr uint32_t idV2 = ptx::idesc_bf16(128, 64, true, false);
 #pragma unroll
@@ -690,12 +560,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
                          idV1, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmY, mnmaj(sb + OFF_LG, kk), kmaj(sb + OFF_XP + 8192u, kk), idV2, 1);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmZ, kmaj(sb + OFF_SR, kk), kmaj(sb + OFF_RO, kk), idKK, kk > 0);
-        ptx::umma_commit(bar(BAR_G5));
+        ptx::umma_commit(bar(BAR_GZ));
       }
 
-      // ================= phase 7: the previous chunk's decay term, dV, the gradient-tile masks
+      // ================= phase 7: the previous chunk's decay term, the gradient-tile masks
       waitb(bar(BAR_G5), par);
       ptx::tc_fence_after();
       if (ci > 0) {
@@ -718,16 +586,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           }
         }
         rs[cg * 128 + row] = acc;
-      }
-      {  // dV (= dZ: the values enter unscaled); thread: d_v channel `row`, tokens [16 cg, 16 cg + 16)
-        uint32_t r[16];
-        ptx::tmem_ld16(tmY + lane_base + cg * 16, r);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int t = cg * 16 + j;
-          if (t < nvalid) g_dv[((size_t)(t0 + t) * H + h) * D + row] = from_f32<Tout>(__uint_as_float(r[j]));
-        }
       }
       __syncthreads();  // S_r is read; its space takes the gradient tile
       if (ci > 0 && tid < 128)
@@ -782,11 +640,23 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         }
       };
       load_raw(cg * 16);
+      waitb(bar(BAR_GZ), par);  // dV^T is done: it goes out while the last products run
+      ptx::tc_fence_after();
+      {  // dV (= dZ: the values enter unscaled); thread: d_v channel `row`, tokens [16 cg, 16 cg + 16)
+        uint32_t r[16];
+        ptx::tmem_ld16(tmY + lane_base + cg * 16, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int t = cg * 16 + j;
+          if (t < nvalid) g_dv[((size_t)(t0 + t) * H + h) * D + row] = from_f32<Tout>(__uint_as_float(r[j]));
+        }
+      }
       waitb(bar(BAR_G7), par);
       ptx::tc_fence_after();
       // every tile is free (the epilogue reads TMEM and global memory only): the next chunk's
       // raw tiles land while this chunk's gradients are formed and stored
-      if (tid == kIssuer && ci > 0 && !*sAbort) issue_loads(h, t0 - C, ck_unit + (size_t)(ci - 1) * (D * D * 2));
+      if (tid == kIssuer && ci > 0 && !*sAbort) issue_loads(h, t0 - C, ck_unit + (size_t)(ci - 1) * kSlotBytes);
 
       // ================= phase 9: chain rule and stores.  Thread: d_k channel i = `row`, tokens
       //      [16 cg, 16 cg + 16).  The cumulative decay is recomputed as phase 1 computed it.

@@ -214,7 +214,7 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const voi
 
 // gdn2_chunk_bwd workspace: [0, 256) header ([0] status, [1] forward unit counter, [2] backward
 // unit counter), the unit schedule, the per-sequence checkpoint offsets, the final states
-// (fp32), the checkpoints (one 32 KB bf16 S_r tile image per chunk and (sequence, head)).
+// (fp32), the checkpoints (per chunk and (sequence, head) the bf16 S_r and T tile images).
 struct ChunkBwdLayout {
   size_t off_sched, off_ckoff, off_fin, off_ckpt, total;
 };
@@ -228,7 +228,7 @@ static ChunkBwdLayout chunk_bwd_layout(const gdn2_dims *dims, bool packed) {
   L.off_fin = L.off_ckoff + up(((size_t)dims->n_seqs + 1) * sizeof(int64_t));
   L.off_ckpt = L.off_fin + units * 128 * 128 * sizeof(float);
   const size_t slots = gdn2::bwd_tc_ckpt_slots(dims->n_seqs, t_total, dims->n_heads, packed, dims->seq_len);
-  L.total = L.off_ckpt + slots * 128 * 128 * 2;
+  L.total = L.off_ckpt + slots * gdn2::kBwdCkptSlotBytes;
   return L;
 }
 

@@ -68,7 +68,11 @@ constexpr float kLog2eF = 1.4426950408889634f;
 // a state term that underflows in S_r = e^{L_ref} S can only have been worth e^{64 - 87.3}
 // of the state's size in any output.
 constexpr float kFastSpan = 128.f;
-constexpr size_t kCkptBytes = (size_t)D * D * 2;  // one bf16 S_r tile image
+// One backward checkpoint slot per chunk: the bf16 S_r tile image (32 KB), then the bf16 T tile
+// image (8 KB), both in the swizzled layout of this kernel's shared-memory tiles.
+constexpr size_t kCkptT = (size_t)D * D * 2;
+constexpr size_t kCkptBytes = kBwdCkptSlotBytes;
+static_assert(kCkptBytes == kCkptT + (size_t)C * C * 2, "checkpoint slot layout");
 
 // Shared-memory map, byte offsets from a 1024-byte-aligned base.  Every operand
 // tile is a stack of 8-row x 128-byte swizzle atoms.
@@ -581,9 +585,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       len = p.seq_len;
     }
     const int nchunks = (int)((len + C - 1) / C);
-    // chunk-start states for the backward (gdn2_chunk_bwd): slot ci receives the bf16 S_r of
-    // chunk ci as this chunk builds it, in the swizzled [d_k rows][d_v] tile image the backward
-    // copies to shared memory as it is (chunks of the token-serial form write nothing)
+    // checkpoints for the backward (gdn2_chunk_bwd): slot ci receives the bf16 S_r of chunk ci
+    // as this chunk builds it (the swizzled [d_k rows][d_v] tile image the backward copies to
+    // shared memory as it is) and the chunk's bf16 T tile; chunks of the token-serial form
+    // write nothing
     uint8_t *ck_unit = p.ckpt ? static_cast<uint8_t *>(p.ckpt) + ckpt_first_slot(p.ckpt_off, n, h, H, nchunks) * kCkptBytes
                               : nullptr;
     if (tid == kIssuer && nchunks > 0 && !*sAbort) {
@@ -740,19 +745,25 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         }
         ptx::tmem_st32(tmS + lane_base + cg * 32, r);
         ptx::tmem_st16(tmSR + lane_base + cg * 16, hb);
-        if (ck_unit) {  // S_r[i][j] of this chunk, i = 32 cg + jj, j = `row`
-          uint8_t *img = ck_unit + (size_t)ci * kCkptBytes;
+        if (ck_unit) {
+          // S_r[i][j] of this chunk (i = 32 cg + jj, j = `row`) into the o staging area, which a
+          // checkpointing forward (no o) leaves free; one bulk copy takes the image to the slot.
+          // The previous chunk's copies have read the area (bulk_wait_group_read0 after GB).
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) {
             const uint32_t pair = hb[jj >> 1];
-            *reinterpret_cast<uint16_t *>(img + swz_elem(cg * 32 + jj, row, 16384u)) =
-                (uint16_t)((jj & 1) ? (pair >> 16) : (pair & 0xffffu));
+            sts_u16(sb + OFF_OS + swz_elem(cg * 32 + jj, row, 16384u), (uint16_t)((jj & 1) ? (pair >> 16) : (pair & 0xffffu)));
           }
+          ptx::fence_proxy_async_smem();
         }
         ptx::tmem_wait_st();
       }
       ptx::tc_fence_before();
       __syncthreads();
+      if (ck_unit && tid == kIssuer && !*sAbort) {
+        ptx::bulk_store(ck_unit + (size_t)ci * kCkptBytes, sb + OFF_OS, 32768u);
+        ptx::bulk_commit_group();
+      }
 
 
       waitb(bar(BAR_G1), par);
@@ -972,6 +983,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       if (warp < 8) ptx::fence_proxy_async_smem();  // warps 0-7 wrote the bf16 T tile
       ptx::tc_fence_before();
       __syncthreads();
+      // the backward's checkpoint also keeps this chunk's bf16 T (the tile image after S_r); the
+      // issuing thread waits for this copy's reads before the next chunk's solve rewrites it
+      // (bulk_wait_group_read0 before the epilogue below)
+      if (ck_unit && tid == kIssuer && !*sAbort) {
+        ptx::bulk_store(ck_unit + (size_t)ci * kCkptBytes + kCkptT, sb + OFF_T, 8192u);
+        ptx::bulk_commit_group();
+      }
 
       // ---- R^T (fp32, D1 cols 0-63) -> bf16 TMEM A operand
       waitb(bar(BAR_GA), par);
@@ -1045,7 +1063,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       ptx::tc_fence_after();
 
       // ---- a8: outputs (the state was updated by the increment GEMMs)
-      {
+      if (p.o) {
         // o^T: lane = dv channel `row`, columns = tokens [16 cg, 16 cg + 16)
         uint32_t r[16];
         ptx::tmem_ld16(tmO + lane_base + cg * 16, r);

@@ -29,9 +29,10 @@ struct ChunkProblem {
   // replaces cu_seqlens for the unit bounds, so the sequences may leave gaps between them
   // (the split forward's passes over a subset of segments).  Tensor-core path only.
   const int32_t *seg_bounds;
-  // Optional chunk-start state buffer for the backward (tensor-core path only): per chunk the
-  // bf16 S_r = Diag(e^{L_ref}) S tile image (32 KB, the chunk kernel's swizzled [d_k][d_v]
-  // layout), the slots of a unit laid out as tc::ckpt_first_slot says; ckpt_off [n_seqs + 1]
+  // Optional checkpoint buffer for the backward (tensor-core path only): per chunk a slot of
+  // kBwdCkptSlotBytes with the bf16 S_r = Diag(e^{L_ref}) S tile image (the chunk kernel's
+  // swizzled [d_k][d_v] layout) and the bf16 T tile, the slots of a unit laid out as
+  // tc::ckpt_first_slot says; ckpt_off [n_seqs + 1]
   // (int64) is the first slot of each sequence divided by n_heads, or NULL for equal lengths.
   // With ckpt set, o may be NULL (no output written).
   void *ckpt;
@@ -67,6 +68,10 @@ struct BwdProblem {
   int dtype_in, dtype_out;
   uint32_t flags;
 };
+
+// Bytes of one backward checkpoint slot (per chunk and (sequence, head)): the bf16 S_r tile
+// image (32 KB) and the bf16 T = (I + A)^-1 tile image (8 KB) the checkpointing forward writes.
+constexpr size_t kBwdCkptSlotBytes = 128 * 128 * 2 + 64 * 64 * 2;
 
 // Status word values written by kernels (0 = fine).
 constexpr int32_t kStatusTimeout = 1;
