@@ -104,6 +104,27 @@ def kernel_sha() -> str:
     return h.hexdigest()[:16]
 
 
+def bwd_kernel_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("chunk_tc.cu", "bwd_tc.cu", "sm100_ptx.cuh", "common.cuh", "tc_util.cuh"):
+        with open(os.path.join(ROOT, "gated_delta_rule_159_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def bwd_traffic_per_call():
+    """DRAM bytes of one gdn2_chunk_bwd call on the bench workload (both kernels) from the
+    committed ncu summary, if it was taken on the current kernel sources (else None)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "chunk_bwd_traffic.json")) as f:
+            t = json.load(f)
+        if t.get("kernel_sha") == bwd_kernel_sha():
+            return t["bytes_per_call_full_workload"]
+    except Exception:
+        pass
+    return None
+
+
 def traffic_per_launch():
     """DRAM bytes per chunk-kernel launch from the committed ncu summary, if it
     was taken on the current kernel source (else None)."""
@@ -669,7 +690,7 @@ def main():
                "steps": args.bwd_steps, "status": st,
                "dtype": "bf16 operands, fp32 accumulation (tcgen05), bf16 gradients",
                "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
-                            "traffic": None, "peak_source": peak_src,
+                            "traffic": bwd_traffic_per_call() if Nb == 8 else None, "peak_source": peak_src,
                             "alg_bytes_per_tokhead": CBWD_BYTES_PER_TOKHEAD,
                             "scope": "whole gdn2_chunk_bwd call (checkpointing forward + reverse pass)"},
                "tensor": {"achieved": ctf, "peak": tc_peak, "unit": "TFLOP/s", "frac": ctf / tc_peak,
