@@ -106,7 +106,7 @@ int gdn2_version(void) { return 100; }
 
 int gdn2_debug_timeout_once(int32_t site, uint64_t wait_ns) {
   g_err[0] = '\0';
-  if (site != GDN2_DEBUG_CHUNK && site != GDN2_DEBUG_DECODE)
+  if (site != GDN2_DEBUG_CHUNK && site != GDN2_DEBUG_DECODE && site != GDN2_DEBUG_BWD)
     return fail(GDN2_ERR_INVALID_ARG, "unknown debug site %d", site);
   if (wait_ns < 1000ull || wait_ns > 10000000000ull)
     return fail(GDN2_ERR_INVALID_ARG, "wait_ns must lie in [1000, 1e10] (got %llu)", (unsigned long long)wait_ns);

@@ -124,7 +124,8 @@ struct BwdTcParams {
   const int32_t *schedule;                         // unit order (longest first) or NULL
   int32_t *status, *counter;
   int n_units, n_heads, seq_len;
-  uint64_t wait_ns;
+  uint64_t wait_ns;  // limit of every mbarrier wait (kWaitTimeoutNs unless the timeout test hook is armed)
+  int dbg_skip;      // timeout test hook: CTA 0 arms its first load group but issues none of its copies
 };
 
 // Sums v[c] over the 32 lanes of the warp for every column c; lane l returns the sum of
@@ -220,9 +221,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
   // the raw k, q, v, log_a, b (, w, dO) tiles of the chunk at token t0 of head h, and its S_r
   // tile image (thread kIssuer)
   constexpr bool kDoTma = sizeof(Tout) == 2;  // bf16 dO lands in its tile as it is
+  bool dbg_armed = P.dbg_skip != 0 && blockIdx.x == 0;  // the timeout test hook (thread kIssuer)
   auto issue_loads = [&](int h, int t0, const uint8_t *sr_img) {
     ptx::mbar_arrive_expect_tx(bar(BAR_LD), ((kTied ? 5u : 6u) + (kDoTma ? 1u : 0u)) * 16384u + (uint32_t)kSlotBytes);
     *sIss = *sIss + 1u;
+    if (dbg_armed) {  // bytes announced, no copy issued: the wait for this group runs out
+      dbg_armed = false;
+      return;
+    }
     ptx::bulk_load(sb + OFF_SR, sr_img, 32768u, bar(BAR_LD));
     ptx::bulk_load(sb + OFF_T, sr_img + 32768, 8192u, bar(BAR_LD));
 #pragma unroll
@@ -422,8 +428,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncthreads();
-      if (*sWide) {  // outside the factored form: recorded, the rest of the unit is left
-        if (tid == 0) atomicExch(P.status, kStatusRange);
+      if (*sWide || *sAbort) {
+        // outside the factored form (recorded unless an earlier error was), or a timed-out
+        // wait: the rest of the unit is left
+        if (tid == 0 && !*sAbort) atomicCAS(P.status, 0, kStatusRange);
         unit_ok = false;
         break;
       }
@@ -834,6 +842,11 @@ cudaError_t launch_bwd_tc(const BwdProblem &p, const void *ckpt, const float *S_
   P.seq_len = p.seq_len;
   P.wait_ns = kWaitTimeoutNs;
   if (P.n_units == 0) return cudaSuccess;
+  uint64_t hook_ns = 0;
+  if (take_debug_timeout(GDN2_DEBUG_BWD, &hook_ns)) {  // the timeout test hook, armed for this launch
+    P.dbg_skip = 1;
+    P.wait_ns = hook_ns;
+  }
   const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
   const int64_t T = p.t_total > 0 ? p.t_total : 1;
   bool ok = make_row_tile_map(&P.tm_q, p.q, T, p.n_heads) && make_row_tile_map(&P.tm_k, p.k, T, p.n_heads) &&

@@ -42,6 +42,7 @@ EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_workspace_size", "gdn2_check_statu
             "gdn2_last_error", "gdn2_version")
 DEBUG_CHUNK = 1
 DEBUG_DECODE = 2
+DEBUG_BWD = 3
 
 
 class Dims(ctypes.Structure):

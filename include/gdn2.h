@@ -443,7 +443,9 @@ int gdn2_chunk_fwd_noalloc_status(gdn2_stream_t stream);
  * next launch of the kernel named by `site`:
  *   GDN2_DEBUG_CHUNK   the tensor-core chunk kernel (gdn2_chunk_fwd and the calls
  *                      built on it),
- *   GDN2_DEBUG_DECODE  the streaming decode kernel (d_k = d_v = 128).
+ *   GDN2_DEBUG_DECODE  the streaming decode kernel (d_k = d_v = 128),
+ *   GDN2_DEBUG_BWD     the reverse kernel of gdn2_chunk_bwd (its checkpointing
+ *                      forward runs normally).
  * In that launch every bounded wait uses the limit `wait_ns` instead of 1 s, and
  * the first CTA announces the bytes of its first load group to its mbarrier but
  * issues none of the copies, so its wait runs out: the kernel records
@@ -456,7 +458,7 @@ int gdn2_chunk_fwd_noalloc_status(gdn2_stream_t stream);
  * Errors: GDN2_ERR_INVALID_ARG for an unknown site or wait_ns outside
  * [1000, 10^10].
  */
-enum gdn2_debug_site { GDN2_DEBUG_CHUNK = 1, GDN2_DEBUG_DECODE = 2 };
+enum gdn2_debug_site { GDN2_DEBUG_CHUNK = 1, GDN2_DEBUG_DECODE = 2, GDN2_DEBUG_BWD = 3 };
 int gdn2_debug_timeout_once(int32_t site, uint64_t wait_ns);
 
 /* Thread-local description of the last non-zero status on this thread ("" if none). */

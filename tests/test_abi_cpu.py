@@ -227,8 +227,9 @@ def test_debug_timeout_hook_rejects_bad_arguments(g):
     """The timeout test hook validates its site and wait limit on the host (invalid calls arm nothing)."""
     assert g.lib.gdn2_debug_timeout_once(0, 1_000_000) == g.ERR_INVALID_ARG
     assert "site" in g.lib.gdn2_last_error().decode()
-    assert g.lib.gdn2_debug_timeout_once(3, 1_000_000) == g.ERR_INVALID_ARG
+    assert g.lib.gdn2_debug_timeout_once(4, 1_000_000) == g.ERR_INVALID_ARG
     assert g.lib.gdn2_debug_timeout_once(g.DEBUG_CHUNK, 10) == g.ERR_INVALID_ARG
+    assert g.lib.gdn2_debug_timeout_once(g.DEBUG_BWD, 500) == g.ERR_INVALID_ARG
     assert g.lib.gdn2_debug_timeout_once(g.DEBUG_DECODE, 20_000_000_000) == g.ERR_INVALID_ARG
     assert "wait_ns" in g.lib.gdn2_last_error().decode()
 

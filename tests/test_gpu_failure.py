@@ -65,6 +65,28 @@ def test_chunk_hook_is_one_shot(dev):
     assert gdn2.check_status(ws) == gdn2.OK
 
 
+def test_bwd_wait_times_out_then_recovers(dev):
+    """The chunked backward's reverse kernel: its first load group never lands."""
+    from gated_delta_rule_159_b200 import gdn2
+    from parity_utils import compare_bwd_units
+    inp = _small(dev, n_seqs=2, seq_len=200, n_heads=2)
+    names = ("q", "k", "v", "log_a", "b", "w")
+    args = [inp[n].view(2, 200, *inp[n].shape[1:]) for n in names]
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    dO = torch.randn(400, 2, 128, generator=g, device=dev)
+    gdn2.debug_timeout_once(gdn2.DEBUG_BWD, WAIT_NS)
+    res = gdn2.chunk_bwd(*args, dO.view(2, 200, 2, 128), S0=inp["S0"])
+    ws = res["workspace"]
+    assert gdn2.check_status(ws) == gdn2.ERR_TIMEOUT
+    res = gdn2.chunk_bwd(*args, dO.view(2, 200, 2, 128), S0=inp["S0"], workspace=ws)
+    assert gdn2.check_status(ws) == gdn2.OK
+    grads = {k: (v.reshape(400, *v.shape[2:]) if k not in ("dS0", "workspace") and v is not None else v)
+             for k, v in res.items()}
+    errs = compare_bwd_units(inp, grads, dO, None, all_units(inp))
+    assert max(errs.values()) <= TOL_CHUNK_BF16, errs
+
+
 def test_decode_wait_times_out_then_recovers(dev):
     from gated_delta_rule_159_b200 import gdn2, inputs
     import oracle
