@@ -235,9 +235,9 @@ static ChunkBwdLayout chunk_bwd_layout(const gdn2_dims *dims, bool packed) {
 static const char *chunk_bwd_unsupported(const gdn2_dims *d) {
   if (d->d_k != 128 || d->d_v != 128) return "gdn2_chunk_bwd needs d_k = d_v = 128";
   if (d->dtype_in != GDN2_BF16) return "gdn2_chunk_bwd needs bf16 inputs";
-  if (d->flags & (GDN2_SCALAR_DECAY | GDN2_SCALAR_GATES | GDN2_GATE_FORM_P3 | GDN2_FUSED_PROLOGUE))
-    return "gdn2_chunk_bwd takes per-channel decay and gates in the default placement (GDN2_TIED_GATES "
-           "allowed); gdn2_bwd covers the other flags";
+  if (d->flags & GDN2_FUSED_PROLOGUE) return "gdn2_chunk_bwd does not take GDN2_FUSED_PROLOGUE; gdn2_bwd does";
+  if (((d->flags & GDN2_SCALAR_DECAY) != 0) != ((d->flags & GDN2_SCALAR_GATES) != 0))
+    return "gdn2_chunk_bwd takes scalar decay and scalar gates together or neither; gdn2_bwd covers the other mixes";
   return nullptr;
 }
 

@@ -101,7 +101,9 @@ constexpr uint32_t MISC_PART = 3200;   // float[4][128]  per-row-group sums of d
 constexpr uint32_t MISC_LPRE = 5248;   // float[4][128]  exclusive row-group prefixes of L
 constexpr uint32_t MISC_RS = 7296;     // float[4][128]  row sums per lane quadrant
 constexpr uint32_t MISC_GAM = 9344;    // float[128]     gamma = e^{L_63 - rho} of the current chunk
-constexpr uint32_t MISC_BYTES = 9856;
+constexpr uint32_t MISC_SCAL = 9856;   // float[3][64]   scalar log_a, b, w per token of the current chunk
+constexpr uint32_t MISC_RED = 10624;   // float[4][3][64] channel sums per lane quadrant (scalar gradients)
+constexpr uint32_t MISC_BYTES = 13696;
 constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES + 1024;  // + base alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 limit per CTA");
 enum { BAR_LD = 0, BAR_G1, BAR_GA, BAR_GB, BAR_G5, BAR_GZ, BAR_G7, BAR_DRAIN, kNumBars };
@@ -157,7 +159,10 @@ __device__ __forceinline__ uint64_t mnmaj(uint32_t base, int kk) {
   return ptx::sdesc_sw128(base + (uint32_t)kk * 2048u, 16384, 1024);
 }
 
-template <typename Tout, bool kTied>
+// kP3: the gist.science gate placement (erase read y = b.k, erase and write outer factors
+// x = p = k, values z = w.v); kScalar: log_a, b, w are [T_tot, H] (one value per token and head,
+// broadcast over the channels; their gradients are channel sums).
+template <typename Tout, bool kTied, bool kP3, bool kScalar>
 __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_constant__ BwdTcParams P) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_u32(smem_raw);
@@ -177,6 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
   float *lpre = reinterpret_cast<float *>(gb + OFF_MISC + MISC_LPRE);
   float *rs = reinterpret_cast<float *>(gb + OFF_MISC + MISC_RS);
   float *sGam = reinterpret_cast<float *>(gb + OFF_MISC + MISC_GAM);
+  float *sScal = reinterpret_cast<float *>(gb + OFF_MISC + MISC_SCAL);
+  float *red = reinterpret_cast<float *>(gb + OFF_MISC + MISC_RED);
   volatile int *sAbort = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_ABORT);
   volatile int *sUnit = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_UNIT);
   volatile int *sWide = reinterpret_cast<volatile int *>(gb + OFF_MISC + MISC_WIDE);
@@ -223,7 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
   constexpr bool kDoTma = sizeof(Tout) == 2;  // bf16 dO lands in its tile as it is
   bool dbg_armed = P.dbg_skip != 0 && blockIdx.x == 0;  // the timeout test hook (thread kIssuer)
   auto issue_loads = [&](int h, int t0, const uint8_t *sr_img) {
-    ptx::mbar_arrive_expect_tx(bar(BAR_LD), ((kTied ? 5u : 6u) + (kDoTma ? 1u : 0u)) * 16384u + (uint32_t)kSlotBytes);
+    constexpr uint32_t kTiles = 3u + (kDoTma ? 1u : 0u) + (kScalar ? 0u : (kTied ? 2u : 3u));
+    ptx::mbar_arrive_expect_tx(bar(BAR_LD), kTiles * 16384u + (uint32_t)kSlotBytes);
     *sIss = *sIss + 1u;
     if (dbg_armed) {  // bytes announced, no copy issued: the wait for this group runs out
       dbg_armed = false;
@@ -237,9 +245,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       ptx::tma_load_3d(sb + OFF_KQ + o, &P.tm_k, kb * 64, h, t0, bar(BAR_LD));
       ptx::tma_load_3d(sb + OFF_KQ + o + 8192u, &P.tm_q, kb * 64, h, t0, bar(BAR_LD));
       ptx::tma_load_3d(sb + OFF_MV + o + 8192u, &P.tm_v, kb * 64, h, t0, bar(BAR_LD));
-      ptx::tma_load_3d(sb + OFF_GRAW + (uint32_t)kb * 8192u, &P.tm_g, kb * 64, h, t0, bar(BAR_LD));
-      ptx::tma_load_3d(sb + OFF_XP + o, &P.tm_b, kb * 64, h, t0, bar(BAR_LD));
-      if (!kTied) ptx::tma_load_3d(sb + OFF_XP + o + 8192u, &P.tm_w, kb * 64, h, t0, bar(BAR_LD));
+      if (!kScalar) {
+        ptx::tma_load_3d(sb + OFF_GRAW + (uint32_t)kb * 8192u, &P.tm_g, kb * 64, h, t0, bar(BAR_LD));
+        ptx::tma_load_3d(sb + OFF_XP + o, &P.tm_b, kb * 64, h, t0, bar(BAR_LD));
+        if (!kTied) ptx::tma_load_3d(sb + OFF_XP + o + 8192u, &P.tm_w, kb * 64, h, t0, bar(BAR_LD));
+      }
       if (kDoTma) ptx::tma_load_3d(sb + OFF_RO + o + 8192u, &P.tm_do, kb * 64, h, t0, bar(BAR_LD));
     }
   };
@@ -307,11 +317,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
                           : tsel == 2 ? (const void *)(P.v + gi) : tsel == 3 ? (const void *)(P.log_a + gi)
                           : tsel == 4 ? (const void *)(P.b + gi) : tsel == 5 ? (const void *)(g_w + gi)
                                       : (const void *)(g_do + gi);
-          if (tsel != 5 || !kTied) ptx::bulk_prefetch_l2(src, tsel == 6 ? D * (uint32_t)sizeof(Tout) : D * 2u);
+          const bool scalar_t = kScalar && (tsel == 3 || tsel == 4 || tsel == 5);  // [T, H]: no 256-byte rows
+          if (!scalar_t && (tsel != 5 || !kTied)) ptx::bulk_prefetch_l2(src, tsel == 6 ? D * (uint32_t)sizeof(Tout) : D * 2u);
         } else if (tid < 451) {  // the 40 KB checkpoint slot: 16 + 16 + 8 KB
           ptx::bulk_prefetch_l2(ck_unit + (size_t)(ci - 1) * kSlotBytes + (size_t)(tid - 448) * 16384,
                                 tid < 450 ? 16384u : 8192u);
         }
+      }
+      if (kScalar) {  // the chunk's scalar log_a, b, w (zero past the chunk end)
+        if (tid < 192) {
+          const int which = tid >> 6, r = tid & 63;
+          const __nv_bfloat16 *src = which == 0 ? P.log_a : (which == 1 || kTied) ? P.b : g_w;
+          sScal[tid] = r < nvalid ? bf(src[(size_t)(t0 + r) * H + h]) : 0.f;
+        }
+        __syncthreads();
       }
       // fp32 dO: the rows of channel `row` into the bf16 tile (rows past the chunk end re-read
       // its last row and are zeroed); the dO rows of the tile are free since the previous
@@ -346,7 +365,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           const int r = warp * 4 + rr;
           float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f);
           if (r < nvalid) {
-            g4 = unpack4(lds_v2(sb + OFF_GRAW + (uint32_t)e_kb * 8192u + swz(r, e_ch16) + e_cofs));
+            if (kScalar) {
+              const float sv = sScal[r];
+              g4 = make_float4(sv, sv, sv, sv);
+            } else {
+              g4 = unpack4(lds_v2(sb + OFF_GRAW + (uint32_t)e_kb * 8192u + swz(r, e_ch16) + e_cofs));
+            }
           } else {
             const uint32_t o = (uint32_t)e_kb * 16384u + 8192u + swz(r, e_ch16) + e_cofs;
             sts_v2(sb + OFF_MV + o, make_uint2(0u, 0u));
@@ -395,14 +419,29 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           if (r < nvalid) {
             kk = unpack4(lds_v2(sb + OFF_KQ + o0));
             qq = unpack4(lds_v2(sb + OFF_KQ + o1));
-            bb = unpack4(lds_v2(sb + OFF_XP + o0));
-            ww = kTied ? bb : unpack4(lds_v2(sb + OFF_XP + o1));
+            if (kScalar) {
+              const float sbv = sScal[64 + r], swv = sScal[128 + r];
+              bb = make_float4(sbv, sbv, sbv, sbv);
+              ww = make_float4(swv, swv, swv, swv);
+            } else {
+              bb = unpack4(lds_v2(sb + OFF_XP + o0));
+              ww = kTied ? bb : unpack4(lds_v2(sb + OFF_XP + o1));
+            }
           }
           const float4 kf = make_float4(kk.x * f.x, kk.y * f.y, kk.z * f.z, kk.w * f.w);
-          sts_v2(sb + OFF_KQ + o0, pack4(kk.x * e.x, kk.y * e.y, kk.z * e.z, kk.w * e.w));
           sts_v2(sb + OFF_KQ + o1, pack4(qq.x * e.x, qq.y * e.y, qq.z * e.z, qq.w * e.w));
-          sts_v2(sb + OFF_XP + o0, pack4(bb.x * kf.x, bb.y * kf.y, bb.z * kf.z, bb.w * kf.w));
-          sts_v2(sb + OFF_XP + o1, pack4(ww.x * kf.x, ww.y * kf.y, ww.z * kf.z, ww.w * kf.w));
+          if (kP3) {  // k_r = (b.k) e, x_r = p_r = k f, V = w.v (d_v channels, the same 4 columns)
+            sts_v2(sb + OFF_KQ + o0, pack4(bb.x * kk.x * e.x, bb.y * kk.y * e.y, bb.z * kk.z * e.z, bb.w * kk.w * e.w));
+            const uint2 kfp = pack4(kf.x, kf.y, kf.z, kf.w);
+            sts_v2(sb + OFF_XP + o0, kfp);
+            sts_v2(sb + OFF_XP + o1, kfp);
+            const float4 vv = unpack4(lds_v2(sb + OFF_MV + o0 + 8192u));
+            sts_v2(sb + OFF_MV + o0 + 8192u, pack4(vv.x * ww.x, vv.y * ww.y, vv.z * ww.z, vv.w * ww.w));
+          } else {
+            sts_v2(sb + OFF_KQ + o0, pack4(kk.x * e.x, kk.y * e.y, kk.z * e.z, kk.w * e.w));
+            sts_v2(sb + OFF_XP + o0, pack4(bb.x * kf.x, bb.y * kf.y, bb.z * kf.z, bb.w * kf.w));
+            sts_v2(sb + OFF_XP + o1, pack4(ww.x * kf.x, ww.y * kf.y, ww.z * kf.z, ww.w * kf.w));
+          }
         }
       }
       // Lam_g = Diag(gamma e^{rho_next}) Acc, the bf16 tile [d_k rows][d_v] and the fp32 base of
@@ -633,31 +672,59 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         ptx::umma_commit(bar(BAR_G7));
       }
       // the raw inputs of the epilogue's rows [16 cg, 16 cg + 8) (channel `row`), requested while
-      // the last products run; rows past the chunk end re-read its last row and are ignored
+      // the last products run; rows past the chunk end re-read its last row and are ignored.
+      // Scalar log_a, b, w come from shared memory; the gist.science placement needs no w here.
       __nv_bfloat16 rla[8], rk[8], rq[8], rb[8], rw[8];
       auto load_raw = [&](int c0) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int t = c0 + j, tc = t < nvalid ? t : nvalid - 1;
           const size_t gi = ((size_t)(t0 + tc) * H + h) * D + row;
-          rla[j] = P.log_a[gi];
           rk[j] = P.k[gi];
           rq[j] = P.q[gi];
-          rb[j] = P.b[gi];
-          rw[j] = kTied ? rb[j] : g_w[gi];
+          if (!kScalar) {
+            rla[j] = P.log_a[gi];
+            rb[j] = P.b[gi];
+            if (!kP3) rw[j] = kTied ? rb[j] : g_w[gi];
+          }
         }
       };
       load_raw(cg * 16);
       waitb(bar(BAR_GZ), par);  // dV^T is done: it goes out while the last products run
       ptx::tc_fence_after();
-      {  // dV (= dZ: the values enter unscaled); thread: d_v channel `row`, tokens [16 cg, 16 cg + 16)
+      // dV: thread d_v channel `row`, tokens [16 cg, 16 cg + 16).  dZ is the gradient of the
+      // values as they enter (v, or w.v in the gist.science placement: dv = w dZ, and v dZ goes
+      // to the value gate: out as dw, or kept for db (tied) or the channel sums (scalar))
+      float vdz[16];
+      {
         uint32_t r[16];
         ptx::tmem_ld16(tmY + lane_base + cg * 16, r);
+        float vr[16], wr[16];
+        if (kP3) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int t = cg * 16 + j, tc = t < nvalid ? t : nvalid - 1;
+            const size_t gi = ((size_t)(t0 + tc) * H + h) * D + row;
+            vr[j] = bf(P.v[gi]);
+            wr[j] = kScalar ? sScal[128 + t] : bf((kTied ? P.b : g_w)[gi]);
+          }
+        }
         ptx::tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int t = cg * 16 + j;
-          if (t < nvalid) g_dv[((size_t)(t0 + t) * H + h) * D + row] = from_f32<Tout>(__uint_as_float(r[j]));
+          const float dz = __uint_as_float(r[j]);
+          vdz[j] = 0.f;
+          if (t < nvalid) {
+            const size_t gi = ((size_t)(t0 + t) * H + h) * D + row;
+            if (kP3) {
+              g_dv[gi] = from_f32<Tout>(wr[j] * dz);
+              vdz[j] = vr[j] * dz;
+              if (!kTied && !kScalar) g_dw[gi] = from_f32<Tout>(vdz[j]);
+            } else {
+              g_dv[gi] = from_f32<Tout>(dz);
+            }
+          }
         }
       }
       waitb(bar(BAR_G7), par);
@@ -668,10 +735,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
 
       // ================= phase 9: chain rule and stores.  Thread: d_k channel i = `row`, tokens
       //      [16 cg, 16 cg + 16).  The cumulative decay is recomputed as phase 1 computed it.
+      //      Per channel: dx = dx_r e^{L_ref - L}, dp = dp_r e^{L_ref - L}, and
+      //        default placement:     dk = dk_r e^{L - L_ref} + b dx + w dp,  db = k dx,  dw = k dp;
+      //        gist.science placement: dy = dk_r e^{L - L_ref} (y = b.k), dk = b dy + dx + dp,
+      //                                db = k dy (+ v dZ of the same channel when tied);
+      //      scalar gates and decay take the channel sums of db, dw, d log_a.
       {
         const int i = row;
         const float pre = lpre[cg * 128 + i], rho = sRho[i], dlc = sDlc[par * 128 + i];
-        float dL[16];
+        float dL[16], gbv[16], gwv[16];
         float loc = 0.f;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -685,31 +757,52 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const int t = c0 + j;
+            const int t = c0 + j, jj = half * 8 + j;
             const bool valid = t < nvalid;
-            const float la = valid ? bf(rla[j]) : 0.f, kk = valid ? bf(rk[j]) : 0.f, qq = valid ? bf(rq[j]) : 0.f;
-            const float bb = valid ? bf(rb[j]) : 0.f, ww = valid ? bf(rw[j]) : 0.f;
+            const float kk = valid ? bf(rk[j]) : 0.f, qq = valid ? bf(rq[j]) : 0.f;
+            const float la = kScalar ? sScal[t] : (valid ? bf(rla[j]) : 0.f);
+            const float bb = kScalar ? sScal[64 + t] : (valid ? bf(rb[j]) : 0.f);
+            const float ww = kP3 ? 0.f : kScalar ? sScal[128 + t] : (valid ? bf(rw[j]) : 0.f);
             loc += la;
             const float L = pre + loc;
             const float e = ptx::ex2((L - rho) * kLog2eF), f = ptx::ex2((rho - L) * kLog2eF);
             const float dxr = __uint_as_float(vx[j]), dpr = __uint_as_float(vp[j]);
             const float dkr = __uint_as_float(vk[j]), dqr = __uint_as_float(vq[j]);
             const float dx = dxr * f, dp = dpr * f;
-            float dLt = e * (dqr * qq + dkr * kk) - f * kk * (dxr * bb + dpr * ww);
+            float dLt, dkv;
+            if (kP3) {
+              const float dy = dkr * e;
+              dLt = e * (dqr * qq + dkr * bb * kk) - f * kk * (dxr + dpr);
+              dkv = bb * dy + dx + dp;
+              gbv[jj] = kk * dy + (kTied ? vdz[jj] : 0.f);
+              gwv[jj] = vdz[jj];
+            } else {
+              dLt = e * (dqr * qq + dkr * kk) - f * kk * (dxr * bb + dpr * ww);
+              dkv = dkr * e + bb * dx + ww * dp;
+              gbv[jj] = kTied ? kk * (dx + dp) : kk * dx;
+              gwv[jj] = kk * dp;
+            }
             if (t == C - 1) dLt += dlc;
-            dL[half * 8 + j] = dLt;
+            dL[jj] = dLt;
             if (valid) {
               const size_t gi = ((size_t)(t0 + t) * H + h) * D + i;
               g_dq[gi] = from_f32<Tout>(dqr * e);
-              g_dk[gi] = from_f32<Tout>(dkr * e + bb * dx + ww * dp);
-              if (kTied) {
-                g_db[gi] = from_f32<Tout>(kk * (dx + dp));
-              } else {
-                g_db[gi] = from_f32<Tout>(kk * dx);
-                g_dw[gi] = from_f32<Tout>(kk * dp);
+              g_dk[gi] = from_f32<Tout>(dkv);
+              if (!kScalar) {
+                g_db[gi] = from_f32<Tout>(gbv[jj]);
+                if (!kTied && !kP3) g_dw[gi] = from_f32<Tout>(gwv[jj]);
               }
             }
           }
+        }
+        if (kScalar) {  // db, dw channel sums: over the warp's 32 channels, then the lane quadrants
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            v[j] = gbv[j];
+            v[16 + j] = gwv[j];
+          }
+          red[(qd * 3 + (lane >> 4)) * 64 + cg * 16 + (lane & 15)] = warp_colsum32(v);
         }
         // d log_a_s = sum_{t >= s} dL_t: suffix sums inside the thread's 16 rows, then the
         // totals of the later row groups
@@ -723,10 +816,30 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         __syncthreads();
         float above = 0.f;
         for (int g = 3; g > cg; --g) above += part[g * 128 + i];
+        if (kScalar) {
+          float v[32];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int t = cg * 16 + j;
-          if (t < nvalid) g_dla[((size_t)(t0 + t) * H + h) * D + i] = from_f32<Tout>(dL[j] + above);
+          for (int j = 0; j < 16; ++j) {
+            v[j] = dL[j] + above;
+            v[16 + j] = 0.f;
+          }
+          const float sum = warp_colsum32(v);
+          if (lane < 16) red[(qd * 3 + 2) * 64 + cg * 16 + lane] = sum;
+          __syncthreads();
+          if (tid < 192) {  // one thread per (quantity, token): db, dw, d log_a
+            const int q = tid >> 6, t = tid & 63;
+            const float tot = ((red[q * 64 + t] + red[(3 + q) * 64 + t]) + red[(6 + q) * 64 + t]) + red[(9 + q) * 64 + t];
+            if (t < nvalid && !(q == 1 && kTied)) {
+              Tout *dst = q == 0 ? g_db : q == 1 ? g_dw : g_dla;
+              dst[(size_t)(t0 + t) * H + h] = from_f32<Tout>(tot);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int t = cg * 16 + j;
+            if (t < nvalid) g_dla[((size_t)(t0 + t) * H + h) * D + i] = from_f32<Tout>(dL[j] + above);
+          }
         }
       }
       ptx::tc_fence_before();
@@ -795,13 +908,23 @@ __global__ void ckpt_offsets_kernel(const int32_t *cu, int N, int64_t *off) {
   }
 }
 
-template <typename Tout, bool kTied>
+template <typename Tout, bool kTied, bool kP3, bool kScalar>
 cudaError_t launch_t(const BwdTcParams &P, int grid, cudaStream_t stream) {
-  auto kern = bwd_tc_kernel<Tout, kTied>;
+  auto kern = bwd_tc_kernel<Tout, kTied, kP3, kScalar>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, kSmemBytes, stream>>>(P);
   return cudaGetLastError();
+}
+
+template <typename Tout>
+cudaError_t launch_flags(const BwdTcParams &P, int grid, cudaStream_t stream, bool tied, bool p3, bool scalar) {
+  if (p3) {
+    if (scalar) return tied ? launch_t<Tout, true, true, true>(P, grid, stream) : launch_t<Tout, false, true, true>(P, grid, stream);
+    return tied ? launch_t<Tout, true, true, false>(P, grid, stream) : launch_t<Tout, false, true, false>(P, grid, stream);
+  }
+  if (scalar) return tied ? launch_t<Tout, true, false, true>(P, grid, stream) : launch_t<Tout, false, false, true>(P, grid, stream);
+  return tied ? launch_t<Tout, true, false, false>(P, grid, stream) : launch_t<Tout, false, false, false>(P, grid, stream);
 }
 
 }  // namespace
@@ -849,19 +972,22 @@ cudaError_t launch_bwd_tc(const BwdProblem &p, const void *ckpt, const float *S_
   }
   const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
   const int64_t T = p.t_total > 0 ? p.t_total : 1;
+  const bool scalar_g = (p.flags & GDN2_SCALAR_DECAY) != 0;
   bool ok = make_row_tile_map(&P.tm_q, p.q, T, p.n_heads) && make_row_tile_map(&P.tm_k, p.k, T, p.n_heads) &&
-            make_row_tile_map(&P.tm_v, p.v, T, p.n_heads) && make_row_tile_map(&P.tm_g, p.log_a, T, p.n_heads) &&
-            make_row_tile_map(&P.tm_b, p.b, T, p.n_heads);
-  if (ok && !tied) ok = make_row_tile_map(&P.tm_w, p.w, T, p.n_heads);
+            make_row_tile_map(&P.tm_v, p.v, T, p.n_heads);
+  if (ok && !scalar_g)
+    ok = make_row_tile_map(&P.tm_g, p.log_a, T, p.n_heads) && make_row_tile_map(&P.tm_b, p.b, T, p.n_heads);
+  if (ok && !scalar_g && !tied) ok = make_row_tile_map(&P.tm_w, p.w, T, p.n_heads);
   if (ok && p.dtype_out == GDN2_BF16) ok = make_row_tile_map(&P.tm_do, p.dO, T, p.n_heads);
   if (!ok) return cudaErrorInvalidValue;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = P.n_units < sms ? P.n_units : sms;
-  if (p.dtype_out == GDN2_BF16)
-    return tied ? launch_t<__nv_bfloat16, true>(P, grid, stream) : launch_t<__nv_bfloat16, false>(P, grid, stream);
-  return tied ? launch_t<float, true>(P, grid, stream) : launch_t<float, false>(P, grid, stream);
+  const bool p3 = (p.flags & GDN2_GATE_FORM_P3) != 0;
+  const bool scalar = (p.flags & GDN2_SCALAR_DECAY) != 0;  // the caller checks that the gates are scalar too
+  if (p.dtype_out == GDN2_BF16) return launch_flags<__nv_bfloat16>(P, grid, stream, tied, p3, scalar);
+  return launch_flags<float>(P, grid, stream, tied, p3, scalar);
 }
 
 }  // namespace gdn2

@@ -23,19 +23,26 @@ def dev():
     return torch.device("cuda:0")
 
 
-def _case(dev, lengths, tied=False, n_heads=2, seed=0, do_dtype=torch.float32, with_S0=True, with_dST=True,
-          batch=None):
+def _case(dev, lengths, tied=None, n_heads=2, seed=0, do_dtype=torch.float32, with_S0=True, with_dST=True,
+          batch=None, scalar=False, p3=False):
+    """Inputs of the bwd tests.  scalar: one alpha and one beta per token and head (and, unless
+    tied is False, b = w); p3: the gist.science placement (w gates the d_v value channels)."""
     from gated_delta_rule_159_b200 import inputs
     if batch is None:
-        w = inputs.Workload("cbwd", len(lengths), 0, n_heads, 128, 128, 64, torch.bfloat16, 0.05, False, 0.05)
-        inp = inputs.make_inputs(w, dev, seed=seed, lengths=lengths)
+        w = inputs.Workload("cbwd", len(lengths), 0, n_heads, 128, 128, 64, torch.bfloat16, 0.05, scalar, 0.05)
+        inp = inputs.make_inputs(w, dev, seed=seed, lengths=lengths, gate_form_p3=p3)
     else:
         n, T = batch
-        w = inputs.Workload("cbwd", n, T, n_heads, 128, 128, 64, torch.bfloat16, 0.05, False, 0.05)
-        inp = inputs.make_inputs(w, dev, seed=seed)
-    if tied:
-        inp["tied_gates"] = True
-        inp["w"] = None
+        w = inputs.Workload("cbwd", n, T, n_heads, 128, 128, 64, torch.bfloat16, 0.05, scalar, 0.05)
+        inp = inputs.make_inputs(w, dev, seed=seed, gate_form_p3=p3)
+    if tied is not None:
+        inp["tied_gates"] = tied
+        if tied:
+            inp["w"] = None
+        elif inp["w"] is None:  # scalar but untied: an independent w per token and head
+            g = torch.Generator(device=dev)
+            g.manual_seed(seed + 77)
+            inp["w"] = torch.sigmoid(torch.randn(inp["b"].shape, generator=g, device=dev)).to(inp["b"].dtype)
     if not with_S0:
         inp["S0"] = None
     g = torch.Generator(device=dev)
@@ -50,13 +57,15 @@ def _run(inp, dO, dS_T, batch=None):
     """gdn2.chunk_bwd on a workload dict; ``batch`` = (B, T) passes [B, T, H, d] tensors (no
     cu_seqlens).  Returns the gradients with token-major [T_tot, H, ...] shapes."""
     from gated_delta_rule_159_b200 import gdn2
+    flags = dict(tied_gates=inp["tied_gates"], scalar_decay=inp["scalar_decay"], scalar_gates=inp["scalar_gates"],
+                 gate_form_p3=inp.get("gate_form_p3", False))
     if batch is None:
         return gdn2.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["log_a"], inp["b"], inp["w"], dO, S0=inp["S0"],
-                              dS_T=dS_T, cu_seqlens=inp["cu_seqlens"], tied_gates=inp["tied_gates"])
+                              dS_T=dS_T, cu_seqlens=inp["cu_seqlens"], **flags)
     B, T = batch
     r4 = lambda t: None if t is None else t.reshape(B, T, *t.shape[1:])  # noqa: E731
     g = gdn2.chunk_bwd(r4(inp["q"]), r4(inp["k"]), r4(inp["v"]), r4(inp["log_a"]), r4(inp["b"]), r4(inp["w"]),
-                       r4(dO), S0=inp["S0"], dS_T=dS_T, tied_gates=inp["tied_gates"])
+                       r4(dO), S0=inp["S0"], dS_T=dS_T, **flags)
     for name in ("dq", "dk", "dv", "dlog_a", "db", "dw"):
         if g[name] is not None:
             g[name] = g[name].reshape(B * T, *g[name].shape[2:])
@@ -71,10 +80,13 @@ def _status(grads):
 LENS = [1, 7, 64, 0, 65, 130, 200]
 
 
-@pytest.mark.parametrize("variant", ["default", "tied", "bf16_grads", "no_state"])
+@pytest.mark.parametrize("variant", ["default", "tied", "bf16_grads", "no_state", "scalar_tied", "scalar_untied",
+                                     "p3", "p3_tied", "p3_scalar", "p3_scalar_tied"])
 def test_chunk_bwd_varlen(dev, variant):
     kw = dict(default={}, tied=dict(tied=True), bf16_grads=dict(do_dtype=torch.bfloat16),
-              no_state=dict(with_S0=False, with_dST=False))[variant]
+              no_state=dict(with_S0=False, with_dST=False), scalar_tied=dict(scalar=True),
+              scalar_untied=dict(scalar=True, tied=False), p3=dict(p3=True), p3_tied=dict(p3=True, tied=True),
+              p3_scalar=dict(p3=True, scalar=True, tied=False), p3_scalar_tied=dict(p3=True, scalar=True))[variant]
     inp, dO, dS_T = _case(dev, LENS, **kw)
     grads = _run(inp, dO, dS_T)
     assert _status(grads) == 0
