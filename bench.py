@@ -76,10 +76,12 @@ BWD_FLOP_PER_TOKHEAD = (7 + 7 + 26) * 128 * 128
 CBWD_FLOP_PER_TOKHEAD = 2 * (128 * 128 * 128 * 5 + 128 * 64 * (192 + 192 + 64 + 64 + 256)
                              + 128 * 128 * 256) // 64 + FLOP_PER_TOKHEAD
 # DRAM bytes of one gdn2_chunk_bwd per token-head: the forward reads the six bf16 inputs and
-# writes the bf16 S_r checkpoint (32 KB per 64 tokens); the reverse pass reads the six inputs,
-# dO and the checkpoint and writes six bf16 gradients (final states and dS_T, dS0 per sequence
-# are not counted)
-CBWD_BYTES_PER_TOKHEAD = 6 * 256 + 512 + (7 * 256 + 512) + 6 * 256
+# writes the checkpoint (bf16 S_r and T tiles, 40 KB per 64 tokens); the reverse pass reads the
+# six inputs, dO and the checkpoint and writes six bf16 gradients (final states and dS_T, dS0
+# per sequence are not counted)
+CBWD_BYTES_PER_TOKHEAD = 6 * 256 + 640 + (7 * 256 + 640) + 6 * 256
+# the tied scalar-gate batch: q, k, v (and dO, dq, dk, dv) per channel, log_a and b per token
+CBWD_BYTES_PER_TOKHEAD_SCALAR = (3 * 256 + 4) + 640 + (4 * 256 + 4 + 640) + (3 * 256 + 4)
 
 
 def fp32_peak_tflops(sm_max_mhz: float) -> float:
@@ -698,6 +700,40 @@ def main():
                "kernels": ["chunk_tc_kernel (checkpointing forward)", "bwd_tc_kernel"],
                "gpu_launches": 2 * args.bwd_steps, "workspace_bytes": cws.numel(), "clocks": bclocks}
         del cws
+        # the tied scalar-gate Gated DeltaNet batch (4 x 4096 x 16) through the same backward
+        si = inputs.make_inputs("gdn_scalar_b4_t4k", dev, seed=310 + rank)
+        Ns, Ts = si["n_seqs"], si["T_tot"] // si["n_seqs"]
+        sdO = torch.randn(Ns, Ts, 16, 128, generator=gen, device=dev).to(torch.bfloat16)
+        sdS = torch.randn(Ns, 16, 128, 128, generator=gen, device=dev) * 0.1
+        sargs = [None if si[n] is None else si[n].view(Ns, Ts, *si[n].shape[1:]) for n in names]
+        sdims = gdn2.make_dims(Ns, Ts, 16, 128, 128, 64, gdn2.BF16, gdn2.BF16,
+                               gdn2.SCALAR_DECAY | gdn2.SCALAR_GATES | gdn2.TIED_GATES)
+        sws = torch.empty(gdn2.chunk_bwd_workspace_size(sdims), dtype=torch.uint8, device=dev)
+
+        def sstep():
+            return gdn2.chunk_bwd(*sargs, sdO, S0=si["S0"], dS_T=sdS, scalar_decay=True, scalar_gates=True,
+                                  tied_gates=True, workspace=sws)
+
+        for _ in range(3):
+            sstep()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(args.bwd_steps):
+            sstep()
+        e1.record(stream)
+        barrier()
+        sms = rmax(e0.elapsed_time(e1)) / args.bwd_steps
+        sst = gdn2.lib.gdn2_check_status(gdn2._ptr(sws), gdn2._stream(dev))
+        sgbs = CBWD_BYTES_PER_TOKHEAD_SCALAR * Ns * Ts * 16 / (sms / 1e3) / 1e9
+        bwd["gdn_scalar_b4_t4k"] = {
+            "value": Ns * Ts * world / (sms / 1e3), "unit": "tokens/s", "ms_per_step": sms, "status": sst,
+            "gates": "scalar alpha, tied scalar beta (Gated DeltaNet)",
+            "roofline": {"bound": "hbm", "achieved": sgbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": sgbs / hbm_peak, "traffic": None, "peak_source": peak_src,
+                         "alg_bytes_per_tokhead": CBWD_BYTES_PER_TOKHEAD_SCALAR},
+            "units": Ns * 16, "workspace_bytes": sws.numel()}
+        del si, sdO, sdS, sargs, sws
         if not args.no_token_serial_bwd:
             bws = torch.empty(gdn2.bwd_workspace_size(bdims), dtype=torch.uint8, device=dev)
 
