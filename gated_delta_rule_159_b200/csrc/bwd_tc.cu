@@ -32,22 +32,25 @@
 // carried adjoint lives in TMEM (lane = d_k channel) for the whole sequence, so the thread of a
 // d_k channel scales and stores its row with one factor and 16-byte vectors.
 //
-// The S_r tiles come from a forward pass of chunk_tc_kernel that writes each chunk's bf16 S_r
-// (the operand it builds anyway, with the same rho) as a swizzled tile image to the workspace;
-// one bulk copy per chunk brings it to shared memory.  One CTA (512 threads) per SM takes (sequence, head) units
+// The S_r and T tiles come from a forward pass of chunk_tc_kernel that writes each chunk's bf16
+// S_r (the operand it builds anyway, with the same rho) and bf16 T = (I + A)^-1 as swizzled tile
+// images to the workspace; bulk copies bring them to shared memory, so this pass neither
+// recomputes the state nor solves.  One CTA (512 threads) per SM takes (sequence, head) units
 // from an atomic counter and walks their chunks last to first; per chunk its phases are:
-//   1  (the raw k, q, v, log_a, b, w, dO tiles (TMA) and S_r (bulk copy) were requested while
-//      the previous chunk finished) cumulative decay, the scaled operands in place, Lam_g;
-//   2  G1 [A B; QX QP] = [k_r; q_r][x_r; p_r]^T  and  dM^T <- Lam_g^T x_r^T;  masks;
-//   3  the (I + A)^-1 solve (fp32, warps 0-14) while warp 15 issues R^T and dM^T += dO^T QX;
+//   1  (the raw k, q, v, log_a, b, w, dO tiles (TMA) and the S_r, T images (bulk copies) were
+//      requested right after the previous chunk's last products) cumulative decay, the scaled
+//      operands in place, Lam_g from the TMEM adjoint;
+//   2  G1 [A B; QX QP] = [k_r; q_r][x_r; p_r]^T, then dM^T = Lam_g^T x_r^T and R^T = S_r^T k_r^T
+//      while the masks write B, QX, QP;
+//   3  R^T += V^T B^T, dM^T += dO^T QX;
 //   4  R^T, -dM^T to bf16 TMEM operands; M^T = R^T T^T, dR^T = dM^T T;
-//   5  -M and dR to shared memory;
-//   6  [dA dB; dQX dQP], the adjoint update, dV^T and the S_r terms of [dk_r^T | dq_r^T];
-//   7  the decay term of the previous chunk (row sums of adjoint x state), dV out, the masks
-//      of the gradient tile;
-//   8  [dx_r^T | dp_r^T] and the rest of [dk_r^T | dq_r^T];
-//   9  the chain rule through the scaling and the gates, the reverse cumulative sum of dL,
-//      gradient stores.
+//   5  -M and dR to their shared-memory tiles;
+//   6  the adjoint update, the S_r terms of [dk_r^T | dq_r^T], [dA dB; dQX dQP] (one commit),
+//      then dV^T;
+//   7  the decay term of the next chunk (row sums of adjoint x S_r), the masks of the gradient
+//      tile (over S_r's space);
+//   8  [dx_r^T | dp_r^T] and the rest of [dk_r^T | dq_r^T]; dV out while they run;
+//   9  the chain rule through the scaling and the gates, the suffix sums of dL, the stores.
 // Chunks whose decay range exceeds kFastSpan nats on some channel are outside the factored
 // form: the kernel records kStatusRange and leaves the rest of that unit (gdn2_bwd, the
 // token-serial reverse mode, covers any range).  Every mbarrier wait is bounded.
@@ -92,7 +95,7 @@ constexpr uint32_t MISC_TMEM = 64;
 constexpr uint32_t MISC_ABORT = 68;
 constexpr uint32_t MISC_UNIT = 72;
 constexpr uint32_t MISC_WIDE = 76;
-constexpr uint32_t MISC_ISS = 80;      // uint32: load phases armed on BAR_LD
+constexpr uint32_t MISC_ISS = 80;      // uint32: load phases armed on BAR_LD (for the wind-down)
 constexpr uint32_t MISC_RHO = 128;     // float[128]     rho of the current chunk
 constexpr uint32_t MISC_ESR = 640;     // float[2][128]  e^{rho} per chunk parity
 constexpr uint32_t MISC_DLC = 1664;    // float[2][128]  decay term of L_63 per chunk parity
@@ -610,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         ptx::umma_commit(bar(BAR_GZ));
       }
 
-      // ================= phase 7: the previous chunk's decay term, the gradient-tile masks
+      // ================= phase 7: the decay term of chunk ci - 1 (processed next), the gradient-tile masks
       waitb(bar(BAR_G5), par);
       ptx::tc_fence_after();
       if (ci > 0) {
