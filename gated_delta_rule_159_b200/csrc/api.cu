@@ -216,7 +216,7 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const voi
 // unit counter), the unit schedule, the per-sequence checkpoint offsets, the final states
 // (fp32), the checkpoints (per chunk and (sequence, head) the bf16 S_r and T tile images).
 struct ChunkBwdLayout {
-  size_t off_sched, off_ckoff, off_fin, off_ckpt, total;
+  size_t off_sched, off_ckoff, off_fin, off_ckpt, off_pro, total;
 };
 static ChunkBwdLayout chunk_bwd_layout(const gdn2_dims *dims, bool packed) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
@@ -229,13 +229,20 @@ static ChunkBwdLayout chunk_bwd_layout(const gdn2_dims *dims, bool packed) {
   L.off_ckpt = L.off_fin + units * 128 * 128 * sizeof(float);
   const size_t slots = gdn2::bwd_tc_ckpt_slots(dims->n_seqs, t_total, dims->n_heads, packed, dims->seq_len);
   L.total = L.off_ckpt + slots * gdn2::kBwdCkptSlotBytes;
+  // with the fused prologue: activated bf16 copies of q, k (and of log_a, b, w: per channel or
+  // per token) and the fp32 inverse norms of q and k per (token, head)
+  L.off_pro = up(L.total);
+  if (dims->flags & GDN2_FUSED_PROLOGUE) {
+    const size_t rows = (size_t)t_total * dims->n_heads;
+    const size_t g = (dims->flags & GDN2_SCALAR_DECAY) ? 1 : 128;
+    L.total = L.off_pro + up(rows * 128 * 2) * 2 + up(rows * g * 2) * 3 + up(rows * 2 * sizeof(float));
+  }
   return L;
 }
 
 static const char *chunk_bwd_unsupported(const gdn2_dims *d) {
   if (d->d_k != 128 || d->d_v != 128) return "gdn2_chunk_bwd needs d_k = d_v = 128";
   if (d->dtype_in != GDN2_BF16) return "gdn2_chunk_bwd needs bf16 inputs";
-  if (d->flags & GDN2_FUSED_PROLOGUE) return "gdn2_chunk_bwd does not take GDN2_FUSED_PROLOGUE; gdn2_bwd does";
   if (((d->flags & GDN2_SCALAR_DECAY) != 0) != ((d->flags & GDN2_SCALAR_GATES) != 0))
     return "gdn2_chunk_bwd takes scalar decay and scalar gates together or neither; gdn2_bwd covers the other mixes";
   return nullptr;
@@ -264,6 +271,9 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_
     return fail(GDN2_ERR_INVALID_ARG, "S0, dS_T and dS0 must be 16-byte aligned");
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return fail(GDN2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  if ((dims->flags & GDN2_FUSED_PROLOGUE) &&
+      (!aligned16(dq) || !aligned16(dk) || !aligned16(dlog_a) || !aligned16(db) || (dw && !aligned16(dw))))
+    return fail(GDN2_ERR_INVALID_ARG, "with GDN2_FUSED_PROLOGUE the gradients must be 16-byte aligned");
   const bool packed = cu_seqlens != nullptr;
   const ChunkBwdLayout lay = chunk_bwd_layout(dims, packed);
   if (workspace_bytes < lay.total)
@@ -292,15 +302,40 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_
   }
   void *ckpt = ws + lay.off_ckpt;
   float *S_fin = reinterpret_cast<float *>(ws + lay.off_fin);
+  // raw inputs as given; with the fused prologue the passes below run on activated copies
+  const void *aq = q, *ak = k, *ala = log_a, *ab = b, *aw = w;
+  uint32_t aflags = dims->flags;
+  gdn2::PrologueCopiesBf16 pc{};
+  gdn2::BwdProblem raw;
+  memset(&raw, 0, sizeof(raw));
+  raw.q = q; raw.k = k; raw.log_a = log_a; raw.b = b; raw.w = tied ? nullptr : w;
+  raw.dq = dq; raw.dk = dk; raw.dlog_a = dlog_a; raw.db = db; raw.dw = tied ? nullptr : dw;
+  raw.n_heads = dims->n_heads; raw.t_total = t_total; raw.dtype_out = dims->dtype_out; raw.flags = dims->flags;
+  if (dims->flags & GDN2_FUSED_PROLOGUE) {
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t rows = (size_t)t_total * dims->n_heads;
+    const size_t g = (dims->flags & GDN2_SCALAR_DECAY) ? 1 : 128;
+    char *base = ws + lay.off_pro;
+    pc.q = reinterpret_cast<__nv_bfloat16 *>(base);
+    pc.k = reinterpret_cast<__nv_bfloat16 *>(base + up(rows * 256));
+    pc.log_a = reinterpret_cast<__nv_bfloat16 *>(base + 2 * up(rows * 256));
+    pc.b = reinterpret_cast<__nv_bfloat16 *>(base + 2 * up(rows * 256) + up(rows * g * 2));
+    pc.w = reinterpret_cast<__nv_bfloat16 *>(base + 2 * up(rows * 256) + 2 * up(rows * g * 2));
+    pc.inv_norm = reinterpret_cast<float *>(base + 2 * up(rows * 256) + 3 * up(rows * g * 2));
+    e = gdn2::launch_prolog_act(raw, pc, s);
+    if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "prologue launch: %s", cudaGetErrorString(e));
+    aq = pc.q; ak = pc.k; ala = pc.log_a; ab = pc.b; aw = tied ? nullptr : pc.w;
+    aflags &= ~(uint32_t)GDN2_FUSED_PROLOGUE;
+  }
 
   // the forward, writing every chunk's S_r tile and the final states instead of o
   gdn2::ChunkProblem f;
   memset(&f, 0, sizeof(f));
-  f.q = q; f.k = k; f.v = v; f.log_a = log_a; f.b = b; f.w = w;
+  f.q = aq; f.k = ak; f.v = v; f.log_a = ala; f.b = ab; f.w = aw;
   f.S0 = S0; f.cu_seqlens = cu_seqlens; f.o = nullptr; f.S_T = S_fin;
   f.n_seqs = dims->n_seqs; f.seq_len = dims->seq_len; f.n_heads = dims->n_heads;
   f.d_k = 128; f.d_v = 128; f.chunk = 64;
-  f.dtype_in = GDN2_BF16; f.dtype_out = dims->dtype_out; f.flags = dims->flags;
+  f.dtype_in = GDN2_BF16; f.dtype_out = dims->dtype_out; f.flags = aflags;
   f.t_total = t_total;
   f.status = status;
   f.schedule = sched;
@@ -313,14 +348,18 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_
 
   gdn2::BwdProblem p;
   memset(&p, 0, sizeof(p));
-  p.q = q; p.k = k; p.v = v; p.log_a = log_a; p.b = b; p.w = tied ? nullptr : w;
+  p.q = aq; p.k = ak; p.v = v; p.log_a = ala; p.b = ab; p.w = tied ? nullptr : aw;
   p.S0 = S0; p.cu_seqlens = cu_seqlens; p.dO = dO; p.dS_T = dS_T;
   p.dq = dq; p.dk = dk; p.dv = dv; p.dlog_a = dlog_a; p.db = db; p.dw = tied ? nullptr : dw; p.dS0 = dS0;
   p.n_seqs = dims->n_seqs; p.seq_len = dims->seq_len; p.n_heads = dims->n_heads;
   p.d_k = 128; p.d_v = 128; p.t_total = t_total;
-  p.dtype_in = GDN2_BF16; p.dtype_out = dims->dtype_out; p.flags = dims->flags;
+  p.dtype_in = GDN2_BF16; p.dtype_out = dims->dtype_out; p.flags = aflags;
   e = gdn2::launch_bwd_tc(p, ckpt, S_fin, ckoff, sched, status, status + 2, s);
   if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "bwd_tc launch: %s", cudaGetErrorString(e));
+  if (dims->flags & GDN2_FUSED_PROLOGUE) {  // gradients of the raw inputs
+    e = gdn2::launch_prolog_chain(raw, pc.inv_norm, s);
+    if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "prologue chain-rule launch: %s", cudaGetErrorString(e));
+  }
   return GDN2_OK;
 }
 

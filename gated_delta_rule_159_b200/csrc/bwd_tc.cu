@@ -993,4 +993,157 @@ cudaError_t launch_bwd_tc(const BwdProblem &p, const void *ckpt, const float *S_
   return launch_flags<float>(P, grid, stream, tied, p3, scalar);
 }
 
+// ---------------------------------------------------------------- fused prologue (GDN2_FUSED_PROLOGUE)
+// gdn2_chunk_bwd with the prologue flag runs the chunked backward on activated copies of the
+// inputs and applies the activations' chain rule to its gradients afterwards; both passes are
+// elementwise over (token, head) rows, one warp per row, lane l holding channels 4 l .. 4 l + 3.
+namespace {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int sh = 16; sh >= 1; sh >>= 1) v += __shfl_xor_sync(0xffffffffu, v, sh);
+  return v;
+}
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p) {
+  return tc::unpack4(*reinterpret_cast<const uint2 *>(p));
+}
+__device__ __forceinline__ void st4(__nv_bfloat16 *p, float4 v) {
+  *reinterpret_cast<uint2 *>(p) = tc::pack4(v.x, v.y, v.z, v.w);
+}
+template <typename T>
+__device__ __forceinline__ float4 ld4t(const T *p);
+template <>
+__device__ __forceinline__ float4 ld4t<float>(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+template <>
+__device__ __forceinline__ float4 ld4t<__nv_bfloat16>(const __nv_bfloat16 *p) { return ld4(p); }
+template <typename T>
+__device__ __forceinline__ void st4t(T *p, float4 v);
+template <>
+__device__ __forceinline__ void st4t<float>(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+template <>
+__device__ __forceinline__ void st4t<__nv_bfloat16>(__nv_bfloat16 *p, float4 v) { st4(p, v); }
+
+// Activated bf16 copies: q / |q|, k / |k| (|x| = sqrt(sum x^2 + kNormEps)), log sigmoid(log_a),
+// sigmoid(b), sigmoid(w); inv[2 row] = 1/|q|, inv[2 row + 1] = 1/|k|.
+__global__ void prolog_act_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *la,
+                                  const __nv_bfloat16 *b, const __nv_bfloat16 *w, int64_t rows, bool scalar,
+                                  __nv_bfloat16 *qa, __nv_bfloat16 *ka, __nv_bfloat16 *laa, __nv_bfloat16 *ba,
+                                  __nv_bfloat16 *wa, float *inv) {
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const size_t o = (size_t)row * 128 + 4 * lane;
+  const float4 qq = ld4(q + o), kk = ld4(k + o);
+  const float iq = rsqrtf(warp_sum(qq.x * qq.x + qq.y * qq.y + qq.z * qq.z + qq.w * qq.w) + kNormEps);
+  const float ik = rsqrtf(warp_sum(kk.x * kk.x + kk.y * kk.y + kk.z * kk.z + kk.w * kk.w) + kNormEps);
+  st4(qa + o, make_float4(qq.x * iq, qq.y * iq, qq.z * iq, qq.w * iq));
+  st4(ka + o, make_float4(kk.x * ik, kk.y * ik, kk.z * ik, kk.w * ik));
+  if (lane == 0) {
+    inv[2 * row] = iq;
+    inv[2 * row + 1] = ik;
+  }
+  if (scalar) {
+    if (lane == 0) {
+      laa[row] = __float2bfloat16_rn(log_sigmoid_f(__bfloat162float(la[row])));
+      ba[row] = __float2bfloat16_rn(sigmoid_f(__bfloat162float(b[row])));
+      if (w) wa[row] = __float2bfloat16_rn(sigmoid_f(__bfloat162float(w[row])));
+    }
+  } else {
+    const float4 g = ld4(la + o), bb = ld4(b + o);
+    st4(laa + o, make_float4(log_sigmoid_f(g.x), log_sigmoid_f(g.y), log_sigmoid_f(g.z), log_sigmoid_f(g.w)));
+    st4(ba + o, make_float4(sigmoid_f(bb.x), sigmoid_f(bb.y), sigmoid_f(bb.z), sigmoid_f(bb.w)));
+    if (w) {
+      const float4 ww = ld4(w + o);
+      st4(wa + o, make_float4(sigmoid_f(ww.x), sigmoid_f(ww.y), sigmoid_f(ww.z), sigmoid_f(ww.w)));
+    }
+  }
+}
+
+// The activations' chain rule, in place on the gradients with respect to the activated inputs:
+// dq = (dq^ - q^ (q^ . dq^)) / |q| (k alike), d log_a *= 1 - sigmoid(log_a), db *= s (1 - s) with
+// s = sigmoid(b) (w alike; dw absent with tied gates).
+template <typename Tout>
+__global__ void prolog_chain_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *la,
+                                    const __nv_bfloat16 *b, const __nv_bfloat16 *w, const float *inv, int64_t rows,
+                                    bool scalar, Tout *dq, Tout *dk, Tout *dla, Tout *db, Tout *dw) {
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const size_t o = (size_t)row * 128 + 4 * lane;
+  const float iq = inv[2 * row], ik = inv[2 * row + 1];
+  {
+    const float4 qq = ld4(q + o), g = ld4t<Tout>(dq + o);
+    const float4 qh = make_float4(qq.x * iq, qq.y * iq, qq.z * iq, qq.w * iq);
+    const float s = warp_sum(qh.x * g.x + qh.y * g.y + qh.z * g.z + qh.w * g.w);
+    st4t<Tout>(dq + o, make_float4((g.x - qh.x * s) * iq, (g.y - qh.y * s) * iq, (g.z - qh.z * s) * iq,
+                                   (g.w - qh.w * s) * iq));
+  }
+  {
+    const float4 kk = ld4(k + o), g = ld4t<Tout>(dk + o);
+    const float4 kh = make_float4(kk.x * ik, kk.y * ik, kk.z * ik, kk.w * ik);
+    const float s = warp_sum(kh.x * g.x + kh.y * g.y + kh.z * g.z + kh.w * g.w);
+    st4t<Tout>(dk + o, make_float4((g.x - kh.x * s) * ik, (g.y - kh.y * s) * ik, (g.z - kh.z * s) * ik,
+                                   (g.w - kh.w * s) * ik));
+  }
+  auto dsig = [](float x) {
+    const float s = sigmoid_f(x);
+    return s * (1.f - s);
+  };
+  if (scalar) {
+    if (lane == 0) {
+      dla[row] = from_f32<Tout>(to_f32<Tout>(dla[row]) * (1.f - sigmoid_f(__bfloat162float(la[row]))));
+      db[row] = from_f32<Tout>(to_f32<Tout>(db[row]) * dsig(__bfloat162float(b[row])));
+      if (dw) dw[row] = from_f32<Tout>(to_f32<Tout>(dw[row]) * dsig(__bfloat162float(w[row])));
+    }
+  } else {
+    const float4 g = ld4(la + o), gd = ld4t<Tout>(dla + o);
+    st4t<Tout>(dla + o, make_float4(gd.x * (1.f - sigmoid_f(g.x)), gd.y * (1.f - sigmoid_f(g.y)),
+                                    gd.z * (1.f - sigmoid_f(g.z)), gd.w * (1.f - sigmoid_f(g.w))));
+    const float4 bb = ld4(b + o), gb = ld4t<Tout>(db + o);
+    st4t<Tout>(db + o, make_float4(gb.x * dsig(bb.x), gb.y * dsig(bb.y), gb.z * dsig(bb.z), gb.w * dsig(bb.w)));
+    if (dw) {
+      const float4 ww = ld4(w + o), gw = ld4t<Tout>(dw + o);
+      st4t<Tout>(dw + o, make_float4(gw.x * dsig(ww.x), gw.y * dsig(ww.y), gw.z * dsig(ww.z), gw.w * dsig(ww.w)));
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prolog_act(const BwdProblem &p, const PrologueCopiesBf16 &c, cudaStream_t stream) {
+  const int64_t rows = p.t_total * p.n_heads;
+  if (rows == 0) return cudaSuccess;
+  const bool scalar = (p.flags & GDN2_SCALAR_DECAY) != 0;
+  const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
+  prolog_act_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16 *>(p.q), static_cast<const __nv_bfloat16 *>(p.k),
+      static_cast<const __nv_bfloat16 *>(p.log_a), static_cast<const __nv_bfloat16 *>(p.b),
+      tied ? nullptr : static_cast<const __nv_bfloat16 *>(p.w), rows, scalar, c.q, c.k, c.log_a, c.b,
+      tied ? nullptr : c.w, c.inv_norm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prolog_chain(const BwdProblem &p, const float *inv_norm, cudaStream_t stream) {
+  const int64_t rows = p.t_total * p.n_heads;
+  if (rows == 0) return cudaSuccess;
+  const bool scalar = (p.flags & GDN2_SCALAR_DECAY) != 0;
+  const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
+  const auto *q = static_cast<const __nv_bfloat16 *>(p.q), *k = static_cast<const __nv_bfloat16 *>(p.k);
+  const auto *la = static_cast<const __nv_bfloat16 *>(p.log_a), *b = static_cast<const __nv_bfloat16 *>(p.b);
+  const auto *w = tied ? nullptr : static_cast<const __nv_bfloat16 *>(p.w);
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  if (p.dtype_out == GDN2_BF16) {
+    using T = __nv_bfloat16;
+    prolog_chain_kernel<T><<<grid, 256, 0, stream>>>(q, k, la, b, w, inv_norm, rows, scalar, static_cast<T *>(p.dq),
+                                                     static_cast<T *>(p.dk), static_cast<T *>(p.dlog_a),
+                                                     static_cast<T *>(p.db), tied ? nullptr : static_cast<T *>(p.dw));
+  } else {
+    prolog_chain_kernel<float><<<grid, 256, 0, stream>>>(q, k, la, b, w, inv_norm, rows, scalar,
+                                                         static_cast<float *>(p.dq), static_cast<float *>(p.dk),
+                                                         static_cast<float *>(p.dlog_a), static_cast<float *>(p.db),
+                                                         tied ? nullptr : static_cast<float *>(p.dw));
+  }
+  return cudaGetLastError();
+}
+
 }  // namespace gdn2

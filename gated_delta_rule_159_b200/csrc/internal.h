@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -95,6 +96,15 @@ size_t bwd_tc_ckpt_slots(int64_t n_seqs, int64_t t_total, int n_heads, bool pack
 cudaError_t launch_ckpt_offsets(const int32_t *cu_seqlens, int n_seqs, int64_t *off, cudaStream_t stream);
 cudaError_t launch_bwd_tc(const BwdProblem &p, const void *ckpt, const float *S_fin, const int64_t *ckpt_off,
                           const int32_t *schedule, int32_t *status, int32_t *counter, cudaStream_t stream);
+// The fused prologue of gdn2_chunk_bwd: activated bf16 copies of q, k, log_a, b, w (w NULL with
+// tied gates) and the inverse norms 1/|q|, 1/|k| per (token, head); afterwards the activations'
+// chain rule in place on the gradients (p's inputs are the raw ones).
+struct PrologueCopiesBf16 {
+  __nv_bfloat16 *q, *k, *log_a, *b, *w;
+  float *inv_norm;
+};
+cudaError_t launch_prolog_act(const BwdProblem &p, const PrologueCopiesBf16 &c, cudaStream_t stream);
+cudaError_t launch_prolog_chain(const BwdProblem &p, const float *inv_norm, cudaStream_t stream);
 
 // Sequence-parallel forward (seqpar.cu): segments of seg_len tokens, workspace offsets.
 struct SplitPlan {

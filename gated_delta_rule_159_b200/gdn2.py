@@ -470,15 +470,16 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Te
               w: Optional[torch.Tensor], dO: torch.Tensor, S0: Optional[torch.Tensor] = None,
               dS_T: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None, *,
               scalar_decay: bool = False, scalar_gates: bool = False, tied_gates: bool = False,
-              gate_form_p3: bool = False, need_dS0: bool = True,
+              gate_form_p3: bool = False, fused_prologue: bool = False, need_dS0: bool = True,
               workspace: Optional[torch.Tensor] = None) -> dict:
     """The gradients of ``bwd`` through ``gdn2_chunk_bwd``: the chunked tensor-core backward
     (d_k = d_v = 128, bf16 inputs; scalar decay and gates together or neither; either gate
-    placement; no fused prologue).  Same arguments and result as ``bwd``;
+    placement; with or without the fused prologue).  Same arguments and result as ``bwd``;
     ``gdn2_check_status(workspace)`` reports a chunk whose decay range is beyond the
     factored form (ERR_RANGE)."""
     return _bwd_call(lib.gdn2_chunk_bwd, lib.gdn2_chunk_bwd_workspace_size, q, k, v, log_a, b, w, dO, S0, dS_T,
-                     cu_seqlens, scalar_decay, scalar_gates, tied_gates, gate_form_p3, False, need_dS0, workspace)
+                     cu_seqlens, scalar_decay, scalar_gates, tied_gates, gate_form_p3, fused_prologue, need_dS0,
+                     workspace)
 
 
 def _bwd_call(fn, ws_fn, q, k, v, log_a, b, w, dO, S0, dS_T, cu_seqlens, scalar_decay, scalar_gates, tied_gates,

@@ -373,16 +373,21 @@ size_t gdn2_bwd_workspace_size(const gdn2_dims *dims, int32_t packed);
  * precision of the bf16-input chunked forward (the products take bf16 operands), not the
  * fp32 precision of gdn2_bwd.
  * Arguments, layouts and ownership: as gdn2_bwd.  dims.chunk is ignored.
- * Supported: d_k = d_v = 128, bf16 inputs, dtype_out (dO and the gradients) bf16 or fp32,
- * per-channel decay and gates in the default placement, GDN2_TIED_GATES allowed; other
- * flags give GDN2_ERR_UNSUPPORTED (gdn2_bwd covers them), as does T_tot >= 2^31.
+ * Supported: d_k = d_v = 128, bf16 inputs, dtype_out (dO and the gradients) bf16 or fp32;
+ * either gate placement (GDN2_GATE_FORM_P3), GDN2_TIED_GATES, scalar decay and gates
+ * (GDN2_SCALAR_DECAY and GDN2_SCALAR_GATES together), and GDN2_FUSED_PROLOGUE (the passes
+ * then run on activated bf16 copies of q, k, log_a, b, w kept in the workspace, and the
+ * activations' chain rule is applied to the gradients at the end).  Scalar decay without
+ * scalar gates (or the reverse) gives GDN2_ERR_UNSUPPORTED (gdn2_bwd covers it), as does
+ * T_tot >= 2^31.
  * Range: every chunk must keep each channel's in-chunk decay L_0 - L_63 within 128 nats
  * (the forward's factored form).  A chunk beyond it is not computed: the call records
  * GDN2_ERR_RANGE for gdn2_check_status(workspace) and that (sequence, head)'s gradients are
  * undefined; gdn2_bwd handles any range.
  * workspace  >= gdn2_chunk_bwd_workspace_size(dims, packed) bytes, 256-byte aligned; one
- *            call at a time per workspace.  It holds the checkpoints: 32 KB per chunk and
- *            (sequence, head), plus one fp32 final state each.
+ *            call at a time per workspace.  It holds the checkpoints: 40 KB per chunk and
+ *            (sequence, head) (the bf16 S_r and T tiles), plus one fp32 final state each, and
+ *            with the fused prologue the activated copies.
  * Errors: GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_WORKSPACE, GDN2_ERR_CUDA;
  * gdn2_check_status reports GDN2_ERR_TIMEOUT (a bounded device wait) or GDN2_ERR_RANGE.
  */

@@ -24,13 +24,13 @@ def dev():
 
 
 def _case(dev, lengths, tied=None, n_heads=2, seed=0, do_dtype=torch.float32, with_S0=True, with_dST=True,
-          batch=None, scalar=False, p3=False):
+          batch=None, scalar=False, p3=False, prolog=False):
     """Inputs of the bwd tests.  scalar: one alpha and one beta per token and head (and, unless
     tied is False, b = w); p3: the gist.science placement (w gates the d_v value channels)."""
     from gated_delta_rule_159_b200 import inputs
     if batch is None:
         w = inputs.Workload("cbwd", len(lengths), 0, n_heads, 128, 128, 64, torch.bfloat16, 0.05, scalar, 0.05)
-        inp = inputs.make_inputs(w, dev, seed=seed, lengths=lengths, gate_form_p3=p3)
+        inp = inputs.make_inputs(w, dev, seed=seed, lengths=lengths, gate_form_p3=p3, fused_prologue=prolog)
     else:
         n, T = batch
         w = inputs.Workload("cbwd", n, T, n_heads, 128, 128, 64, torch.bfloat16, 0.05, scalar, 0.05)
@@ -58,7 +58,7 @@ def _run(inp, dO, dS_T, batch=None):
     cu_seqlens).  Returns the gradients with token-major [T_tot, H, ...] shapes."""
     from gated_delta_rule_159_b200 import gdn2
     flags = dict(tied_gates=inp["tied_gates"], scalar_decay=inp["scalar_decay"], scalar_gates=inp["scalar_gates"],
-                 gate_form_p3=inp.get("gate_form_p3", False))
+                 gate_form_p3=inp.get("gate_form_p3", False), fused_prologue=inp.get("fused_prologue", False))
     if batch is None:
         return gdn2.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["log_a"], inp["b"], inp["w"], dO, S0=inp["S0"],
                               dS_T=dS_T, cu_seqlens=inp["cu_seqlens"], **flags)
@@ -81,12 +81,15 @@ LENS = [1, 7, 64, 0, 65, 130, 200]
 
 
 @pytest.mark.parametrize("variant", ["default", "tied", "bf16_grads", "no_state", "scalar_tied", "scalar_untied",
-                                     "p3", "p3_tied", "p3_scalar", "p3_scalar_tied"])
+                                     "p3", "p3_tied", "p3_scalar", "p3_scalar_tied", "prolog", "prolog_scalar_tied",
+                                     "prolog_p3"])
 def test_chunk_bwd_varlen(dev, variant):
     kw = dict(default={}, tied=dict(tied=True), bf16_grads=dict(do_dtype=torch.bfloat16),
               no_state=dict(with_S0=False, with_dST=False), scalar_tied=dict(scalar=True),
               scalar_untied=dict(scalar=True, tied=False), p3=dict(p3=True), p3_tied=dict(p3=True, tied=True),
-              p3_scalar=dict(p3=True, scalar=True, tied=False), p3_scalar_tied=dict(p3=True, scalar=True))[variant]
+              p3_scalar=dict(p3=True, scalar=True, tied=False), p3_scalar_tied=dict(p3=True, scalar=True),
+              prolog=dict(prolog=True), prolog_scalar_tied=dict(prolog=True, scalar=True),
+              prolog_p3=dict(prolog=True, p3=True))[variant]
     inp, dO, dS_T = _case(dev, LENS, **kw)
     grads = _run(inp, dO, dS_T)
     assert _status(grads) == 0
