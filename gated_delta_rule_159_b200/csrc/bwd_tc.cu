@@ -91,11 +91,11 @@ constexpr uint32_t OFF_QX = OFF_MV + 16384;    // QX bf16 [64 x 64] (the -M rows
 constexpr uint32_t OFF_DG = OFF_SR;            // [dA dB; dQX dQP] as [column block][128 rows][64]
 constexpr uint32_t OFF_GRAW = OFF_LG;          // raw log_a tile [2 blocks][64 rows] until Lam_g is built
 constexpr uint32_t MISC_BAR = 0;       // mbarriers
-constexpr uint32_t MISC_TMEM = 64;
-constexpr uint32_t MISC_ABORT = 68;
-constexpr uint32_t MISC_UNIT = 72;
-constexpr uint32_t MISC_WIDE = 76;
-constexpr uint32_t MISC_ISS = 80;      // uint32: load phases armed on BAR_LD (for the wind-down)
+constexpr uint32_t MISC_TMEM = 80;
+constexpr uint32_t MISC_ABORT = 84;
+constexpr uint32_t MISC_UNIT = 88;
+constexpr uint32_t MISC_WIDE = 92;
+constexpr uint32_t MISC_ISS = 96;      // uint32: load phases armed on BAR_LD (for the wind-down)
 constexpr uint32_t MISC_RHO = 128;     // float[128]     rho of the current chunk
 constexpr uint32_t MISC_ESR = 640;     // float[2][128]  e^{rho} per chunk parity
 constexpr uint32_t MISC_DLC = 1664;    // float[2][128]  decay term of L_63 per chunk parity
@@ -109,7 +109,7 @@ constexpr uint32_t MISC_RED = 10624;   // float[4][3][64] channel sums per lane 
 constexpr uint32_t MISC_BYTES = 13696;
 constexpr uint32_t kSmemBytes = OFF_MISC + MISC_BYTES + 1024;  // + base alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 limit per CTA");
-enum { BAR_LD = 0, BAR_G1, BAR_GA, BAR_GB, BAR_G5, BAR_GZ, BAR_G7, BAR_DRAIN, kNumBars };
+enum { BAR_LD = 0, BAR_G1, BAR_GA, BAR_GB, BAR_G5, BAR_GL, BAR_GZ, BAR_G7, BAR_DRAIN, kNumBars };
 static_assert(MISC_BAR + 8 * kNumBars <= MISC_TMEM, "mbarriers overlap the TMEM address slot");
 
 struct BwdTcParams {
@@ -387,21 +387,36 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       }
       if (tid == 0) *sWide = 0;
       __syncthreads();
-      if (tid < D) {  // per channel: exclusive prefixes over the 16 row groups, L_ref, the range check
-        float run = 0.f;
+      {
+        // per channel c: exclusive prefixes over the 16 row groups (thread: groups 4 g4 .. 4 g4 + 3
+        // of channel c; the four threads of a channel are adjacent lanes and scan their totals
+        // with shuffles), L_ref, the range check
+        const int c = tid >> 2, g4 = tid & 3;
+        float v[4];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float pj = part16[j * 128 + tid];
-          part16[j * 128 + tid] = run;
-          if ((j & 3) == 0) lpre[(j >> 2) * 128 + tid] = run;  // the epilogue's 16-row groups
-          run += pj;
+        for (int j = 0; j < 4; ++j) v[j] = part16[(4 * g4 + j) * 128 + c];
+        const float tl = ((v[0] + v[1]) + v[2]) + v[3];
+        float incl = tl;
+        const float u1 = __shfl_up_sync(0xffffffffu, incl, 1, 4);
+        if (g4 >= 1) incl += u1;
+        const float u2 = __shfl_up_sync(0xffffffffu, incl, 2, 4);
+        if (g4 >= 2) incl += u2;
+        const float run = __shfl_sync(0xffffffffu, incl, 3, 4);  // the channel's total L_63
+        float pre4 = incl - tl;
+        lpre[g4 * 128 + c] = pre4;  // the epilogue's 16-row groups
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          part16[(4 * g4 + j) * 128 + c] = pre4;
+          pre4 += v[j];
         }
-        const float l0 = sL0[tid];
-        const float rho = 0.5f * (l0 + run);
-        if (!(l0 - run <= kFastSpan)) *sWide = 1;
-        sRho[tid] = rho;
-        sGam[tid] = ptx::ex2((run - rho) * kLog2eF);
-        sEsr[par * 128 + tid] = ptx::ex2(rho * kLog2eF);
+        if (g4 == 3) {
+          const float l0 = sL0[c];
+          const float rho = 0.5f * (l0 + run);
+          if (!(l0 - run <= kFastSpan)) *sWide = 1;
+          sRho[c] = rho;
+          sGam[c] = ptx::ex2((run - rho) * kLog2eF);
+          sEsr[par * 128 + c] = ptx::ex2(rho * kLog2eF);
+        }
       }
       __syncthreads();
       // k_r, q_r, x_r, p_r over the raw k, q, b, w rows (zero past the chunk end)
@@ -583,25 +598,33 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         for (int j = 0; j < 16; ++j)
           sts_u16(sb + OFF_RO + swz_elem(cg * 16 + j, row, 16384u), bf16_bits(__uint_as_float(r[j])));
       }
+      // this thread's S_r values (d_k channel `row`, d_v channels [32 cg, 32 cg + 32)) for the
+      // decay term, taken before the barrier after which the gradient tile may overwrite them
+      uint4 srv[4];
+#pragma unroll
+      for (int q8 = 0; q8 < 4; ++q8)
+        srv[q8] = lds_v4(sb + OFF_SR + (uint32_t)(cg >> 1) * 16384u + swz(row, (uint32_t)((cg & 1) * 4 + q8)));
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncthreads();
 
-      // ================= phase 6: the adjoint update Acc += [k_r; q_r]^T [dR; dO], the S_r terms
-      //      [dk_r^T | dq_r^T] = S_r [dR; dO]^T and [dA dB; dQX dQP] = [dR; dO][-M; V]^T (commit
-      //      G5: the masks and the decay term need these), then dV^T = [dR; dO]^T [B; QP] +
-      //      Lam_g^T p_r^T, which runs under the masks (the epilogue reads it)
+      // ================= phase 6: the S_r terms [dk_r^T | dq_r^T] = S_r [dR; dO]^T and
+      //      [dA dB; dQX dQP] = [dR; dO][-M; V]^T (commit G5: the masks need these, and then S_r's
+      //      space is free); the adjoint update Acc += [k_r; q_r]^T [dR; dO] (commit GL: the decay
+      //      term and the next chunk need it); dV^T = [dR; dO]^T [B; QP] + Lam_g^T p_r^T (commit
+      //      GZ).  The last two run under the masks.
       if (tid == kIssuer && !*sAbort) {
         ptx::tc_fence_after();
         constexpr uint32_t idKK = ptx::idesc_bf16(128, 128, false, false);
         constexpr uint32_t idNN = ptx::idesc_bf16(128, 128, true, true);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmAcc, mnmaj(sb + OFF_KQ, kk), mnmaj(sb + OFF_RO, kk), idNN, 1);
-#pragma unroll
         for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmZ, kmaj(sb + OFF_SR, kk), kmaj(sb + OFF_RO, kk), idKK, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmX, kmaj(sb + OFF_RO, kk), kmaj(sb + OFF_MV, kk), idKK, kk > 0);
         ptx::umma_commit(bar(BAR_G5));
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmAcc, mnmaj(sb + OFF_KQ, kk), mnmaj(sb + OFF_RO, kk), idNN, 1);
+        ptx::umma_commit(bar(BAR_GL));
         constexpr uint32_t idV1 = ptx::idesc_bf16(128, 64, true, true);
         constexpr uint32_t idV2 = ptx::idesc_bf16(128, 64, true, false);
 #pragma unroll
@@ -613,33 +636,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         ptx::umma_commit(bar(BAR_GZ));
       }
 
-      // ================= phase 7: the decay term of chunk ci - 1 (processed next), the gradient-tile masks
+      // ================= phase 7: the gradient-tile masks (over S_r's space: every thread took
+      //      its S_r values for the decay term before the barrier that ended phase 5)
       waitb(bar(BAR_G5), par);
       ptx::tc_fence_after();
-      if (ci > 0) {
-        // sum_j Lam_{c-1}[i][j] S_c[i][j] = sum_j Acc[i][j] S_r[i][j] (Lam_{c-1} = e^{rho} Acc):
-        // thread (d_k channel `row`, d_v channels [32 cg, 32 cg + 32)), summed over the four
-        // column groups by the chunk before
-        uint32_t r[32];
-        ptx::tmem_ld32(tmAcc + lane_base + cg * 32, r);
-        ptx::tmem_wait_ld();
-        float acc = 0.f;
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          const uint4 sv = lds_v4(sb + OFF_SR + (uint32_t)(cg >> 1) * 16384u + swz(row, (uint32_t)((cg & 1) * 4 + q8)));
-          const uint32_t w4[4] = {sv.x, sv.y, sv.z, sv.w};
-#pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            const float2 f = unpack_bf16x2(w4[e2]);
-            acc = fmaf(__uint_as_float(r[8 * q8 + 2 * e2]), f.x, acc);
-            acc = fmaf(__uint_as_float(r[8 * q8 + 2 * e2 + 1]), f.y, acc);
-          }
-        }
-        rs[cg * 128 + row] = acc;
-      }
-      __syncthreads();  // S_r is read; its space takes the gradient tile
-      if (ci > 0 && tid < 128)
-        sDlc[(par ^ 1u) * 128 + tid] = ((rs[tid] + rs[128 + tid]) + rs[256 + tid]) + rs[384 + tid];
       {
         // row `row` of [dA dB; dQX dQP], columns [32 cg, 32 cg + 32): strictly lower for the dR
         // rows, lower with the diagonal for the dO rows; stored as [column block][row][64]
@@ -693,6 +693,28 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         }
       };
       load_raw(cg * 16);
+      waitb(bar(BAR_GL), par);  // the adjoint is final for this chunk
+      ptx::tc_fence_after();
+      if (ci > 0) {
+        // the decay term of chunk ci - 1 (processed next): sum_j Lam_{c-1}[i][j] S_c[i][j] =
+        // sum_j Acc[i][j] S_r[i][j] (Lam_{c-1} = e^{rho} Acc); thread (d_k channel `row`, d_v
+        // channels [32 cg, 32 cg + 32)), summed over the four column groups after the next barrier
+        uint32_t r[32];
+        ptx::tmem_ld32(tmAcc + lane_base + cg * 32, r);
+        ptx::tmem_wait_ld();
+        float acc = 0.f;
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          const uint32_t w4[4] = {srv[q8].x, srv[q8].y, srv[q8].z, srv[q8].w};
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float2 f = unpack_bf16x2(w4[e2]);
+            acc = fmaf(__uint_as_float(r[8 * q8 + 2 * e2]), f.x, acc);
+            acc = fmaf(__uint_as_float(r[8 * q8 + 2 * e2 + 1]), f.y, acc);
+          }
+        }
+        rs[cg * 128 + row] = acc;
+      }
       waitb(bar(BAR_GZ), par);  // dV^T is done: it goes out while the last products run
       ptx::tc_fence_after();
       // dV: thread d_v channel `row`, tokens [16 cg, 16 cg + 16).  dZ is the gradient of the
@@ -817,6 +839,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         }
         part[cg * 128 + i] = suf;
         __syncthreads();
+        if (ci > 0 && tid < 128)  // the decay term of chunk ci - 1 (rs is complete)
+          sDlc[(par ^ 1u) * 128 + tid] = ((rs[tid] + rs[128 + tid]) + rs[256 + tid]) + rs[384 + tid];
         float above = 0.f;
         for (int g = 3; g > cg; --g) above += part[g * 128 + i];
         if (kScalar) {
