@@ -312,21 +312,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       const int nvalid = (int)((len - (int64_t)ci * C) < C ? (len - (int64_t)ci * C) : C);
 
       // ================= phase 1: loads, cumulative decay, operand tiles
-      if (ci > 0) {  // the next chunk's rows and state to L2 while this chunk runs
-        if (tid < 448) {
-          const int tsel = tid >> 6, r = tid & 63;
-          const size_t gi = ((size_t)(t0 - C + r) * H + h) * D;
-          const void *src = tsel == 0 ? (const void *)(P.q + gi) : tsel == 1 ? (const void *)(P.k + gi)
-                          : tsel == 2 ? (const void *)(P.v + gi) : tsel == 3 ? (const void *)(P.log_a + gi)
-                          : tsel == 4 ? (const void *)(P.b + gi) : tsel == 5 ? (const void *)(g_w + gi)
-                                      : (const void *)(g_do + gi);
-          const bool scalar_t = kScalar && (tsel == 3 || tsel == 4 || tsel == 5);  // [T, H]: no 256-byte rows
-          if (!scalar_t && (tsel != 5 || !kTied)) ptx::bulk_prefetch_l2(src, tsel == 6 ? D * (uint32_t)sizeof(Tout) : D * 2u);
-        } else if (tid < 451) {  // the 40 KB checkpoint slot: 16 + 16 + 8 KB
-          ptx::bulk_prefetch_l2(ck_unit + (size_t)(ci - 1) * kSlotBytes + (size_t)(tid - 448) * 16384,
-                                tid < 450 ? 16384u : 8192u);
-        }
-      }
       if (kScalar) {  // the chunk's scalar log_a, b, w (zero past the chunk end)
         if (tid < 192) {
           const int which = tid >> 6, r = tid & 63;
