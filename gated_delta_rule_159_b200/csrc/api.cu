@@ -234,8 +234,8 @@ static ChunkBwdLayout chunk_bwd_layout(const gdn2_dims *dims, bool packed) {
   L.off_pro = up(L.total);
   if (dims->flags & GDN2_FUSED_PROLOGUE) {
     const size_t rows = (size_t)t_total * dims->n_heads;
-    const size_t g = (dims->flags & GDN2_SCALAR_DECAY) ? 1 : 128;
-    L.total = L.off_pro + up(rows * 128 * 2) * 2 + up(rows * g * 2) * 3 + up(rows * 2 * sizeof(float));
+    const size_t gd = (dims->flags & GDN2_SCALAR_DECAY) ? 1 : 128, gg = (dims->flags & GDN2_SCALAR_GATES) ? 1 : 128;
+    L.total = L.off_pro + up(rows * 128 * 2) * 2 + up(rows * gd * 2) + up(rows * gg * 2) * 2 + up(rows * 2 * sizeof(float));
   }
   return L;
 }
@@ -243,8 +243,6 @@ static ChunkBwdLayout chunk_bwd_layout(const gdn2_dims *dims, bool packed) {
 static const char *chunk_bwd_unsupported(const gdn2_dims *d) {
   if (d->d_k != 128 || d->d_v != 128) return "gdn2_chunk_bwd needs d_k = d_v = 128";
   if (d->dtype_in != GDN2_BF16) return "gdn2_chunk_bwd needs bf16 inputs";
-  if (((d->flags & GDN2_SCALAR_DECAY) != 0) != ((d->flags & GDN2_SCALAR_GATES) != 0))
-    return "gdn2_chunk_bwd takes scalar decay and scalar gates together or neither; gdn2_bwd covers the other mixes";
   return nullptr;
 }
 
@@ -314,14 +312,19 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_
   if (dims->flags & GDN2_FUSED_PROLOGUE) {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
     const size_t rows = (size_t)t_total * dims->n_heads;
-    const size_t g = (dims->flags & GDN2_SCALAR_DECAY) ? 1 : 128;
+    const size_t gd = (dims->flags & GDN2_SCALAR_DECAY) ? 1 : 128, gg = (dims->flags & GDN2_SCALAR_GATES) ? 1 : 128;
     char *base = ws + lay.off_pro;
     pc.q = reinterpret_cast<__nv_bfloat16 *>(base);
-    pc.k = reinterpret_cast<__nv_bfloat16 *>(base + up(rows * 256));
-    pc.log_a = reinterpret_cast<__nv_bfloat16 *>(base + 2 * up(rows * 256));
-    pc.b = reinterpret_cast<__nv_bfloat16 *>(base + 2 * up(rows * 256) + up(rows * g * 2));
-    pc.w = reinterpret_cast<__nv_bfloat16 *>(base + 2 * up(rows * 256) + 2 * up(rows * g * 2));
-    pc.inv_norm = reinterpret_cast<float *>(base + 2 * up(rows * 256) + 3 * up(rows * g * 2));
+    base += up(rows * 256);
+    pc.k = reinterpret_cast<__nv_bfloat16 *>(base);
+    base += up(rows * 256);
+    pc.log_a = reinterpret_cast<__nv_bfloat16 *>(base);
+    base += up(rows * gd * 2);
+    pc.b = reinterpret_cast<__nv_bfloat16 *>(base);
+    base += up(rows * gg * 2);
+    pc.w = reinterpret_cast<__nv_bfloat16 *>(base);
+    base += up(rows * gg * 2);
+    pc.inv_norm = reinterpret_cast<float *>(base);
     e = gdn2::launch_prolog_act(raw, pc, s);
     if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "prologue launch: %s", cudaGetErrorString(e));
     aq = pc.q; ak = pc.k; ala = pc.log_a; ab = pc.b; aw = tied ? nullptr : pc.w;

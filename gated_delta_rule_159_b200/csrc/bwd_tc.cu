@@ -163,9 +163,9 @@ __device__ __forceinline__ uint64_t mnmaj(uint32_t base, int kk) {
 }
 
 // kP3: the gist.science gate placement (erase read y = b.k, erase and write outer factors
-// x = p = k, values z = w.v); kScalar: log_a, b, w are [T_tot, H] (one value per token and head,
-// broadcast over the channels; their gradients are channel sums).
-template <typename Tout, bool kTied, bool kP3, bool kScalar>
+// x = p = k, values z = w.v); kSD: log_a is [T_tot, H], kSG: b and w are [T_tot, H] (one value
+// per token and head, broadcast over the channels; their gradients are channel sums).
+template <typename Tout, bool kTied, bool kP3, bool kSD, bool kSG>
 __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_constant__ BwdTcParams P) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_u32(smem_raw);
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
   constexpr bool kDoTma = sizeof(Tout) == 2;  // bf16 dO lands in its tile as it is
   bool dbg_armed = P.dbg_skip != 0 && blockIdx.x == 0;  // the timeout test hook (thread kIssuer)
   auto issue_loads = [&](int h, int t0, const uint8_t *sr_img) {
-    constexpr uint32_t kTiles = 3u + (kDoTma ? 1u : 0u) + (kScalar ? 0u : (kTied ? 2u : 3u));
+    constexpr uint32_t kTiles = 3u + (kDoTma ? 1u : 0u) + (kSD ? 0u : 1u) + (kSG ? 0u : (kTied ? 1u : 2u));
     ptx::mbar_arrive_expect_tx(bar(BAR_LD), kTiles * 16384u + (uint32_t)kSlotBytes);
     *sIss = *sIss + 1u;
     if (dbg_armed) {  // bytes announced, no copy issued: the wait for this group runs out
@@ -248,8 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       ptx::tma_load_3d(sb + OFF_KQ + o, &P.tm_k, kb * 64, h, t0, bar(BAR_LD));
       ptx::tma_load_3d(sb + OFF_KQ + o + 8192u, &P.tm_q, kb * 64, h, t0, bar(BAR_LD));
       ptx::tma_load_3d(sb + OFF_MV + o + 8192u, &P.tm_v, kb * 64, h, t0, bar(BAR_LD));
-      if (!kScalar) {
-        ptx::tma_load_3d(sb + OFF_GRAW + (uint32_t)kb * 8192u, &P.tm_g, kb * 64, h, t0, bar(BAR_LD));
+      if (!kSD) ptx::tma_load_3d(sb + OFF_GRAW + (uint32_t)kb * 8192u, &P.tm_g, kb * 64, h, t0, bar(BAR_LD));
+      if (!kSG) {
         ptx::tma_load_3d(sb + OFF_XP + o, &P.tm_b, kb * 64, h, t0, bar(BAR_LD));
         if (!kTied) ptx::tma_load_3d(sb + OFF_XP + o + 8192u, &P.tm_w, kb * 64, h, t0, bar(BAR_LD));
       }
@@ -312,11 +312,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       const int nvalid = (int)((len - (int64_t)ci * C) < C ? (len - (int64_t)ci * C) : C);
 
       // ================= phase 1: loads, cumulative decay, operand tiles
-      if (kScalar) {  // the chunk's scalar log_a, b, w (zero past the chunk end)
+      if (kSD || kSG) {  // the chunk's scalar log_a and / or b, w (zero past the chunk end)
         if (tid < 192) {
           const int which = tid >> 6, r = tid & 63;
-          const __nv_bfloat16 *src = which == 0 ? P.log_a : (which == 1 || kTied) ? P.b : g_w;
-          sScal[tid] = r < nvalid ? bf(src[(size_t)(t0 + r) * H + h]) : 0.f;
+          if (which == 0 ? kSD : kSG) {
+            const __nv_bfloat16 *src = which == 0 ? P.log_a : (which == 1 || kTied) ? P.b : g_w;
+            sScal[tid] = r < nvalid ? bf(src[(size_t)(t0 + r) * H + h]) : 0.f;
+          }
         }
         __syncthreads();
       }
@@ -353,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           const int r = warp * 4 + rr;
           float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f);
           if (r < nvalid) {
-            if (kScalar) {
+            if (kSD) {
               const float sv = sScal[r];
               g4 = make_float4(sv, sv, sv, sv);
             } else {
@@ -422,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           if (r < nvalid) {
             kk = unpack4(lds_v2(sb + OFF_KQ + o0));
             qq = unpack4(lds_v2(sb + OFF_KQ + o1));
-            if (kScalar) {
+            if (kSG) {
               const float sbv = sScal[64 + r], swv = sScal[128 + r];
               bb = make_float4(sbv, sbv, sbv, sbv);
               ww = make_float4(swv, swv, swv, swv);
@@ -670,8 +672,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           const size_t gi = ((size_t)(t0 + tc) * H + h) * D + row;
           rk[j] = P.k[gi];
           rq[j] = P.q[gi];
-          if (!kScalar) {
-            rla[j] = P.log_a[gi];
+          if (!kSD) rla[j] = P.log_a[gi];
+          if (!kSG) {
             rb[j] = P.b[gi];
             if (!kP3) rw[j] = kTied ? rb[j] : g_w[gi];
           }
@@ -716,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
             const int t = cg * 16 + j, tc = t < nvalid ? t : nvalid - 1;
             const size_t gi = ((size_t)(t0 + tc) * H + h) * D + row;
             vr[j] = bf(P.v[gi]);
-            wr[j] = kScalar ? sScal[128 + t] : bf((kTied ? P.b : g_w)[gi]);
+            wr[j] = kSG ? sScal[128 + t] : bf((kTied ? P.b : g_w)[gi]);
           }
         }
         ptx::tmem_wait_ld();
@@ -730,7 +732,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
             if (kP3) {
               g_dv[gi] = from_f32<Tout>(wr[j] * dz);
               vdz[j] = vr[j] * dz;
-              if (!kTied && !kScalar) g_dw[gi] = from_f32<Tout>(vdz[j]);
+              if (!kTied && !kSG) g_dw[gi] = from_f32<Tout>(vdz[j]);
             } else {
               g_dv[gi] = from_f32<Tout>(dz);
             }
@@ -770,9 +772,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
             const int t = c0 + j, jj = half * 8 + j;
             const bool valid = t < nvalid;
             const float kk = valid ? bf(rk[j]) : 0.f, qq = valid ? bf(rq[j]) : 0.f;
-            const float la = kScalar ? sScal[t] : (valid ? bf(rla[j]) : 0.f);
-            const float bb = kScalar ? sScal[64 + t] : (valid ? bf(rb[j]) : 0.f);
-            const float ww = kP3 ? 0.f : kScalar ? sScal[128 + t] : (valid ? bf(rw[j]) : 0.f);
+            const float la = kSD ? sScal[t] : (valid ? bf(rla[j]) : 0.f);
+            const float bb = kSG ? sScal[64 + t] : (valid ? bf(rb[j]) : 0.f);
+            const float ww = kP3 ? 0.f : kSG ? sScal[128 + t] : (valid ? bf(rw[j]) : 0.f);
             loc += la;
             const float L = pre + loc;
             const float e = ptx::ex2((L - rho) * kLog2eF), f = ptx::ex2((rho - L) * kLog2eF);
@@ -798,14 +800,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
               const size_t gi = ((size_t)(t0 + t) * H + h) * D + i;
               g_dq[gi] = from_f32<Tout>(dqr * e);
               g_dk[gi] = from_f32<Tout>(dkv);
-              if (!kScalar) {
+              if (!kSG) {
                 g_db[gi] = from_f32<Tout>(gbv[jj]);
                 if (!kTied && !kP3) g_dw[gi] = from_f32<Tout>(gwv[jj]);
               }
             }
           }
         }
-        if (kScalar) {  // db, dw channel sums: over the warp's 32 channels, then the lane quadrants
+        if (kSG) {  // db, dw channel sums: over the warp's 32 channels, then the lane quadrants
           float v[32];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -828,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           sDlc[(par ^ 1u) * 128 + tid] = ((rs[tid] + rs[128 + tid]) + rs[256 + tid]) + rs[384 + tid];
         float above = 0.f;
         for (int g = 3; g > cg; --g) above += part[g * 128 + i];
-        if (kScalar) {
+        if (kSD) {  // d log_a: channel sums as for db, dw
           float v[32];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -837,20 +839,23 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           }
           const float sum = warp_colsum32(v);
           if (lane < 16) red[(qd * 3 + 2) * 64 + cg * 16 + lane] = sum;
-          __syncthreads();
-          if (tid < 192) {  // one thread per (quantity, token): db, dw, d log_a
-            const int q = tid >> 6, t = tid & 63;
-            const float tot = ((red[q * 64 + t] + red[(3 + q) * 64 + t]) + red[(6 + q) * 64 + t]) + red[(9 + q) * 64 + t];
-            if (t < nvalid && !(q == 1 && kTied)) {
-              Tout *dst = q == 0 ? g_db : q == 1 ? g_dw : g_dla;
-              dst[(size_t)(t0 + t) * H + h] = from_f32<Tout>(tot);
-            }
-          }
         } else {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int t = cg * 16 + j;
             if (t < nvalid) g_dla[((size_t)(t0 + t) * H + h) * D + i] = from_f32<Tout>(dL[j] + above);
+          }
+        }
+        if (kSD || kSG) {
+          __syncthreads();
+          if (tid < 192) {  // one thread per (quantity, token): db, dw (scalar gates), d log_a (scalar decay)
+            const int q = tid >> 6, t = tid & 63;
+            const bool want = q == 2 ? kSD : (kSG && !(q == 1 && kTied));
+            if (want && t < nvalid) {
+              const float tot = ((red[q * 64 + t] + red[(3 + q) * 64 + t]) + red[(6 + q) * 64 + t]) + red[(9 + q) * 64 + t];
+              Tout *dst = q == 0 ? g_db : q == 1 ? g_dw : g_dla;
+              dst[(size_t)(t0 + t) * H + h] = from_f32<Tout>(tot);
+            }
           }
         }
       }
@@ -920,23 +925,27 @@ __global__ void ckpt_offsets_kernel(const int32_t *cu, int N, int64_t *off) {
   }
 }
 
-template <typename Tout, bool kTied, bool kP3, bool kScalar>
+template <typename Tout, bool kTied, bool kP3, bool kSD, bool kSG>
 cudaError_t launch_t(const BwdTcParams &P, int grid, cudaStream_t stream) {
-  auto kern = bwd_tc_kernel<Tout, kTied, kP3, kScalar>;
+  auto kern = bwd_tc_kernel<Tout, kTied, kP3, kSD, kSG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, kSmemBytes, stream>>>(P);
   return cudaGetLastError();
 }
 
+template <typename Tout, bool kP3, bool kSD, bool kSG>
+cudaError_t launch_tied(const BwdTcParams &P, int grid, cudaStream_t stream, bool tied) {
+  return tied ? launch_t<Tout, true, kP3, kSD, kSG>(P, grid, stream) : launch_t<Tout, false, kP3, kSD, kSG>(P, grid, stream);
+}
+template <typename Tout, bool kP3>
+cudaError_t launch_scalars(const BwdTcParams &P, int grid, cudaStream_t stream, bool tied, bool sd, bool sg) {
+  if (sd) return sg ? launch_tied<Tout, kP3, true, true>(P, grid, stream, tied) : launch_tied<Tout, kP3, true, false>(P, grid, stream, tied);
+  return sg ? launch_tied<Tout, kP3, false, true>(P, grid, stream, tied) : launch_tied<Tout, kP3, false, false>(P, grid, stream, tied);
+}
 template <typename Tout>
-cudaError_t launch_flags(const BwdTcParams &P, int grid, cudaStream_t stream, bool tied, bool p3, bool scalar) {
-  if (p3) {
-    if (scalar) return tied ? launch_t<Tout, true, true, true>(P, grid, stream) : launch_t<Tout, false, true, true>(P, grid, stream);
-    return tied ? launch_t<Tout, true, true, false>(P, grid, stream) : launch_t<Tout, false, true, false>(P, grid, stream);
-  }
-  if (scalar) return tied ? launch_t<Tout, true, false, true>(P, grid, stream) : launch_t<Tout, false, false, true>(P, grid, stream);
-  return tied ? launch_t<Tout, true, false, false>(P, grid, stream) : launch_t<Tout, false, false, false>(P, grid, stream);
+cudaError_t launch_flags(const BwdTcParams &P, int grid, cudaStream_t stream, bool tied, bool p3, bool sd, bool sg) {
+  return p3 ? launch_scalars<Tout, true>(P, grid, stream, tied, sd, sg) : launch_scalars<Tout, false>(P, grid, stream, tied, sd, sg);
 }
 
 }  // namespace
@@ -984,12 +993,12 @@ cudaError_t launch_bwd_tc(const BwdProblem &p, const void *ckpt, const float *S_
   }
   const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
   const int64_t T = p.t_total > 0 ? p.t_total : 1;
-  const bool scalar_g = (p.flags & GDN2_SCALAR_DECAY) != 0;
+  const bool sd_m = (p.flags & GDN2_SCALAR_DECAY) != 0, sg_m = (p.flags & GDN2_SCALAR_GATES) != 0;
   bool ok = make_row_tile_map(&P.tm_q, p.q, T, p.n_heads) && make_row_tile_map(&P.tm_k, p.k, T, p.n_heads) &&
             make_row_tile_map(&P.tm_v, p.v, T, p.n_heads);
-  if (ok && !scalar_g)
-    ok = make_row_tile_map(&P.tm_g, p.log_a, T, p.n_heads) && make_row_tile_map(&P.tm_b, p.b, T, p.n_heads);
-  if (ok && !scalar_g && !tied) ok = make_row_tile_map(&P.tm_w, p.w, T, p.n_heads);
+  if (ok && !sd_m) ok = make_row_tile_map(&P.tm_g, p.log_a, T, p.n_heads);
+  if (ok && !sg_m) ok = make_row_tile_map(&P.tm_b, p.b, T, p.n_heads);
+  if (ok && !sg_m && !tied) ok = make_row_tile_map(&P.tm_w, p.w, T, p.n_heads);
   if (ok && p.dtype_out == GDN2_BF16) ok = make_row_tile_map(&P.tm_do, p.dO, T, p.n_heads);
   if (!ok) return cudaErrorInvalidValue;
   int dev = 0, sms = 148;
@@ -997,9 +1006,9 @@ cudaError_t launch_bwd_tc(const BwdProblem &p, const void *ckpt, const float *S_
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = P.n_units < sms ? P.n_units : sms;
   const bool p3 = (p.flags & GDN2_GATE_FORM_P3) != 0;
-  const bool scalar = (p.flags & GDN2_SCALAR_DECAY) != 0;  // the caller checks that the gates are scalar too
-  if (p.dtype_out == GDN2_BF16) return launch_flags<__nv_bfloat16>(P, grid, stream, tied, p3, scalar);
-  return launch_flags<float>(P, grid, stream, tied, p3, scalar);
+  const bool sd = (p.flags & GDN2_SCALAR_DECAY) != 0, sg = (p.flags & GDN2_SCALAR_GATES) != 0;
+  if (p.dtype_out == GDN2_BF16) return launch_flags<__nv_bfloat16>(P, grid, stream, tied, p3, sd, sg);
+  return launch_flags<float>(P, grid, stream, tied, p3, sd, sg);
 }
 
 // ---------------------------------------------------------------- fused prologue (GDN2_FUSED_PROLOGUE)
@@ -1035,7 +1044,7 @@ __device__ __forceinline__ void st4t<__nv_bfloat16>(__nv_bfloat16 *p, float4 v) 
 // Activated bf16 copies: q / |q|, k / |k| (|x| = sqrt(sum x^2 + kNormEps)), log sigmoid(log_a),
 // sigmoid(b), sigmoid(w); inv[2 row] = 1/|q|, inv[2 row + 1] = 1/|k|.
 __global__ void prolog_act_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *la,
-                                  const __nv_bfloat16 *b, const __nv_bfloat16 *w, int64_t rows, bool scalar,
+                                  const __nv_bfloat16 *b, const __nv_bfloat16 *w, int64_t rows, bool sd, bool sg,
                                   __nv_bfloat16 *qa, __nv_bfloat16 *ka, __nv_bfloat16 *laa, __nv_bfloat16 *ba,
                                   __nv_bfloat16 *wa, float *inv) {
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -1051,15 +1060,19 @@ __global__ void prolog_act_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 *k
     inv[2 * row] = iq;
     inv[2 * row + 1] = ik;
   }
-  if (scalar) {
+  if (sd) {
+    if (lane == 0) laa[row] = __float2bfloat16_rn(log_sigmoid_f(__bfloat162float(la[row])));
+  } else {
+    const float4 g = ld4(la + o);
+    st4(laa + o, make_float4(log_sigmoid_f(g.x), log_sigmoid_f(g.y), log_sigmoid_f(g.z), log_sigmoid_f(g.w)));
+  }
+  if (sg) {
     if (lane == 0) {
-      laa[row] = __float2bfloat16_rn(log_sigmoid_f(__bfloat162float(la[row])));
       ba[row] = __float2bfloat16_rn(sigmoid_f(__bfloat162float(b[row])));
       if (w) wa[row] = __float2bfloat16_rn(sigmoid_f(__bfloat162float(w[row])));
     }
   } else {
-    const float4 g = ld4(la + o), bb = ld4(b + o);
-    st4(laa + o, make_float4(log_sigmoid_f(g.x), log_sigmoid_f(g.y), log_sigmoid_f(g.z), log_sigmoid_f(g.w)));
+    const float4 bb = ld4(b + o);
     st4(ba + o, make_float4(sigmoid_f(bb.x), sigmoid_f(bb.y), sigmoid_f(bb.z), sigmoid_f(bb.w)));
     if (w) {
       const float4 ww = ld4(w + o);
@@ -1074,7 +1087,7 @@ __global__ void prolog_act_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 *k
 template <typename Tout>
 __global__ void prolog_chain_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *la,
                                     const __nv_bfloat16 *b, const __nv_bfloat16 *w, const float *inv, int64_t rows,
-                                    bool scalar, Tout *dq, Tout *dk, Tout *dla, Tout *db, Tout *dw) {
+                                    bool sd, bool sg, Tout *dq, Tout *dk, Tout *dla, Tout *db, Tout *dw) {
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -1098,16 +1111,19 @@ __global__ void prolog_chain_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 
     const float s = sigmoid_f(x);
     return s * (1.f - s);
   };
-  if (scalar) {
-    if (lane == 0) {
-      dla[row] = from_f32<Tout>(to_f32<Tout>(dla[row]) * (1.f - sigmoid_f(__bfloat162float(la[row]))));
-      db[row] = from_f32<Tout>(to_f32<Tout>(db[row]) * dsig(__bfloat162float(b[row])));
-      if (dw) dw[row] = from_f32<Tout>(to_f32<Tout>(dw[row]) * dsig(__bfloat162float(w[row])));
-    }
+  if (sd) {
+    if (lane == 0) dla[row] = from_f32<Tout>(to_f32<Tout>(dla[row]) * (1.f - sigmoid_f(__bfloat162float(la[row]))));
   } else {
     const float4 g = ld4(la + o), gd = ld4t<Tout>(dla + o);
     st4t<Tout>(dla + o, make_float4(gd.x * (1.f - sigmoid_f(g.x)), gd.y * (1.f - sigmoid_f(g.y)),
                                     gd.z * (1.f - sigmoid_f(g.z)), gd.w * (1.f - sigmoid_f(g.w))));
+  }
+  if (sg) {
+    if (lane == 0) {
+      db[row] = from_f32<Tout>(to_f32<Tout>(db[row]) * dsig(__bfloat162float(b[row])));
+      if (dw) dw[row] = from_f32<Tout>(to_f32<Tout>(dw[row]) * dsig(__bfloat162float(w[row])));
+    }
+  } else {
     const float4 bb = ld4(b + o), gb = ld4t<Tout>(db + o);
     st4t<Tout>(db + o, make_float4(gb.x * dsig(bb.x), gb.y * dsig(bb.y), gb.z * dsig(bb.z), gb.w * dsig(bb.w)));
     if (dw) {
@@ -1122,12 +1138,12 @@ __global__ void prolog_chain_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 
 cudaError_t launch_prolog_act(const BwdProblem &p, const PrologueCopiesBf16 &c, cudaStream_t stream) {
   const int64_t rows = p.t_total * p.n_heads;
   if (rows == 0) return cudaSuccess;
-  const bool scalar = (p.flags & GDN2_SCALAR_DECAY) != 0;
+  const bool sd = (p.flags & GDN2_SCALAR_DECAY) != 0, sg = (p.flags & GDN2_SCALAR_GATES) != 0;
   const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
   prolog_act_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16 *>(p.q), static_cast<const __nv_bfloat16 *>(p.k),
       static_cast<const __nv_bfloat16 *>(p.log_a), static_cast<const __nv_bfloat16 *>(p.b),
-      tied ? nullptr : static_cast<const __nv_bfloat16 *>(p.w), rows, scalar, c.q, c.k, c.log_a, c.b,
+      tied ? nullptr : static_cast<const __nv_bfloat16 *>(p.w), rows, sd, sg, c.q, c.k, c.log_a, c.b,
       tied ? nullptr : c.w, c.inv_norm);
   return cudaGetLastError();
 }
@@ -1135,7 +1151,7 @@ cudaError_t launch_prolog_act(const BwdProblem &p, const PrologueCopiesBf16 &c, 
 cudaError_t launch_prolog_chain(const BwdProblem &p, const float *inv_norm, cudaStream_t stream) {
   const int64_t rows = p.t_total * p.n_heads;
   if (rows == 0) return cudaSuccess;
-  const bool scalar = (p.flags & GDN2_SCALAR_DECAY) != 0;
+  const bool sd = (p.flags & GDN2_SCALAR_DECAY) != 0, sg = (p.flags & GDN2_SCALAR_GATES) != 0;
   const bool tied = (p.flags & GDN2_TIED_GATES) != 0;
   const auto *q = static_cast<const __nv_bfloat16 *>(p.q), *k = static_cast<const __nv_bfloat16 *>(p.k);
   const auto *la = static_cast<const __nv_bfloat16 *>(p.log_a), *b = static_cast<const __nv_bfloat16 *>(p.b);
@@ -1143,11 +1159,11 @@ cudaError_t launch_prolog_chain(const BwdProblem &p, const float *inv_norm, cuda
   const unsigned grid = (unsigned)((rows + 7) / 8);
   if (p.dtype_out == GDN2_BF16) {
     using T = __nv_bfloat16;
-    prolog_chain_kernel<T><<<grid, 256, 0, stream>>>(q, k, la, b, w, inv_norm, rows, scalar, static_cast<T *>(p.dq),
+    prolog_chain_kernel<T><<<grid, 256, 0, stream>>>(q, k, la, b, w, inv_norm, rows, sd, sg, static_cast<T *>(p.dq),
                                                      static_cast<T *>(p.dk), static_cast<T *>(p.dlog_a),
                                                      static_cast<T *>(p.db), tied ? nullptr : static_cast<T *>(p.dw));
   } else {
-    prolog_chain_kernel<float><<<grid, 256, 0, stream>>>(q, k, la, b, w, inv_norm, rows, scalar,
+    prolog_chain_kernel<float><<<grid, 256, 0, stream>>>(q, k, la, b, w, inv_norm, rows, sd, sg,
                                                          static_cast<float *>(p.dq), static_cast<float *>(p.dk),
                                                          static_cast<float *>(p.dlog_a), static_cast<float *>(p.db),
                                                          tied ? nullptr : static_cast<float *>(p.dw));

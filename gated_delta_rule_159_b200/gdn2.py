@@ -473,8 +473,8 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a: torch.Te
               gate_form_p3: bool = False, fused_prologue: bool = False, need_dS0: bool = True,
               workspace: Optional[torch.Tensor] = None) -> dict:
     """The gradients of ``bwd`` through ``gdn2_chunk_bwd``: the chunked tensor-core backward
-    (d_k = d_v = 128, bf16 inputs; scalar decay and gates together or neither; either gate
-    placement; with or without the fused prologue).  Same arguments and result as ``bwd``;
+    (d_k = d_v = 128, bf16 inputs; any mix of the scalar flags; either gate placement; with
+    or without the fused prologue).  Same arguments and result as ``bwd``;
     ``gdn2_check_status(workspace)`` reports a chunk whose decay range is beyond the
     factored form (ERR_RANGE)."""
     return _bwd_call(lib.gdn2_chunk_bwd, lib.gdn2_chunk_bwd_workspace_size, q, k, v, log_a, b, w, dO, S0, dS_T,

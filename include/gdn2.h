@@ -374,12 +374,11 @@ size_t gdn2_bwd_workspace_size(const gdn2_dims *dims, int32_t packed);
  * fp32 precision of gdn2_bwd.
  * Arguments, layouts and ownership: as gdn2_bwd.  dims.chunk is ignored.
  * Supported: d_k = d_v = 128, bf16 inputs, dtype_out (dO and the gradients) bf16 or fp32;
- * either gate placement (GDN2_GATE_FORM_P3), GDN2_TIED_GATES, scalar decay and gates
- * (GDN2_SCALAR_DECAY and GDN2_SCALAR_GATES together), and GDN2_FUSED_PROLOGUE (the passes
- * then run on activated bf16 copies of q, k, log_a, b, w kept in the workspace, and the
- * activations' chain rule is applied to the gradients at the end).  Scalar decay without
- * scalar gates (or the reverse) gives GDN2_ERR_UNSUPPORTED (gdn2_bwd covers it), as does
- * T_tot >= 2^31.
+ * either gate placement (GDN2_GATE_FORM_P3), GDN2_TIED_GATES, GDN2_SCALAR_DECAY and
+ * GDN2_SCALAR_GATES (each alone or both), and GDN2_FUSED_PROLOGUE (the passes then run on
+ * activated bf16 copies of q, k, log_a, b, w kept in the workspace, and the activations'
+ * chain rule is applied to the gradients at the end).  T_tot >= 2^31 gives
+ * GDN2_ERR_UNSUPPORTED (gdn2_bwd covers it).
  * Range: every chunk must keep each channel's in-chunk decay L_0 - L_63 within 128 nats
  * (the forward's factored form).  A chunk beyond it is not computed: the call records
  * GDN2_ERR_RANGE for gdn2_check_status(workspace) and that (sequence, head)'s gradients are

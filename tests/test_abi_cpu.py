@@ -256,19 +256,23 @@ def test_split_varlen_rejects_bad_arguments(g):
 
 
 def test_chunk_bwd_workspace_size_covers_its_flags(g):
-    """gdn2_chunk_bwd takes either placement, tied gates, scalar decay with scalar gates and the
-    fused prologue; mixed scalar flags, other head sizes and fp32 inputs are gdn2_bwd's (size 0)."""
+    """gdn2_chunk_bwd takes either placement, tied gates, scalar decay and scalar gates (each alone
+    or both) and the fused prologue; other head sizes and fp32 inputs are gdn2_bwd's (size 0)."""
     def size(flags=0, dk=128, dtype_in=None):
         dims = g.make_dims(2, 300, 4, dk, 128, 64, g.BF16 if dtype_in is None else dtype_in, g.BF16, flags)
         return g.chunk_bwd_workspace_size(dims)
     for flags in (0, g.TIED_GATES, g.GATE_FORM_P3, g.GATE_FORM_P3 | g.TIED_GATES,
                   g.SCALAR_DECAY | g.SCALAR_GATES | g.TIED_GATES, g.SCALAR_DECAY | g.SCALAR_GATES | g.GATE_FORM_P3,
-                  g.FUSED_PROLOGUE, g.FUSED_PROLOGUE | g.SCALAR_DECAY | g.SCALAR_GATES | g.TIED_GATES):
+                  g.SCALAR_DECAY, g.SCALAR_GATES, g.SCALAR_GATES | g.TIED_GATES | g.GATE_FORM_P3,
+                  g.FUSED_PROLOGUE, g.FUSED_PROLOGUE | g.SCALAR_DECAY | g.SCALAR_GATES | g.TIED_GATES,
+                  g.FUSED_PROLOGUE | g.SCALAR_DECAY, g.FUSED_PROLOGUE | g.SCALAR_GATES):
         assert size(flags) > 0, flags
-    for flags in (g.SCALAR_DECAY, g.SCALAR_GATES):
-        assert size(flags) == 0, flags
     # the prologue's activated copies: q, k and three per-channel gate tensors (bf16) + inverse norms
     assert size(g.FUSED_PROLOGUE) - size() >= 2 * 300 * 4 * (5 * 128 * 2 + 8)
+    # scalar decay keeps one log_a copy per row instead of d_k, scalar gates one b and one w
+    rows = 2 * 300 * 4
+    assert size(g.FUSED_PROLOGUE) - size(g.FUSED_PROLOGUE | g.SCALAR_DECAY) >= rows * 127 * 2 - 512
+    assert size(g.FUSED_PROLOGUE) - size(g.FUSED_PROLOGUE | g.SCALAR_GATES) >= 2 * (rows * 127 * 2 - 512)
     assert size(dk=64) == 0 and size(dtype_in=g.F32) == 0
     # 2 sequences x 5 chunks x 4 heads slots of 40 KB, plus the fp32 final states and the header
     assert size() >= 2 * 5 * 4 * 40960 + 2 * 4 * 128 * 128 * 4

@@ -24,9 +24,11 @@ def dev():
 
 
 def _case(dev, lengths, tied=None, n_heads=2, seed=0, do_dtype=torch.float32, with_S0=True, with_dST=True,
-          batch=None, scalar=False, p3=False, prolog=False):
+          batch=None, scalar=False, p3=False, prolog=False, mix=None):
     """Inputs of the bwd tests.  scalar: one alpha and one beta per token and head (and, unless
-    tied is False, b = w); p3: the gist.science placement (w gates the d_v value channels)."""
+    tied is False, b = w); p3: the gist.science placement (w gates the d_v value channels);
+    mix "decay" / "gates": only log_a, or only b and w, one value per token and head (the
+    first channel of the per-channel draw)."""
     from gated_delta_rule_159_b200 import inputs
     if batch is None:
         w = inputs.Workload("cbwd", len(lengths), 0, n_heads, 128, 128, 64, torch.bfloat16, 0.05, scalar, 0.05)
@@ -35,6 +37,13 @@ def _case(dev, lengths, tied=None, n_heads=2, seed=0, do_dtype=torch.float32, wi
         n, T = batch
         w = inputs.Workload("cbwd", n, T, n_heads, 128, 128, 64, torch.bfloat16, 0.05, scalar, 0.05)
         inp = inputs.make_inputs(w, dev, seed=seed, gate_form_p3=p3)
+    if mix == "decay":
+        inp["log_a"] = inp["log_a"][..., 0].contiguous()
+        inp["scalar_decay"] = True
+    elif mix == "gates":
+        inp["b"] = inp["b"][..., 0].contiguous()
+        inp["w"] = inp["w"][..., 0].contiguous()
+        inp["scalar_gates"] = True
     if tied is not None:
         inp["tied_gates"] = tied
         if tied:
@@ -82,14 +91,18 @@ LENS = [1, 7, 64, 0, 65, 130, 200]
 
 @pytest.mark.parametrize("variant", ["default", "tied", "bf16_grads", "no_state", "scalar_tied", "scalar_untied",
                                      "p3", "p3_tied", "p3_scalar", "p3_scalar_tied", "prolog", "prolog_scalar_tied",
-                                     "prolog_p3"])
+                                     "prolog_p3", "scalar_decay_only", "scalar_gates_only", "scalar_gates_only_tied",
+                                     "p3_scalar_gates_only", "prolog_scalar_decay_only", "prolog_scalar_gates_only"])
 def test_chunk_bwd_varlen(dev, variant):
     kw = dict(default={}, tied=dict(tied=True), bf16_grads=dict(do_dtype=torch.bfloat16),
               no_state=dict(with_S0=False, with_dST=False), scalar_tied=dict(scalar=True),
               scalar_untied=dict(scalar=True, tied=False), p3=dict(p3=True), p3_tied=dict(p3=True, tied=True),
               p3_scalar=dict(p3=True, scalar=True, tied=False), p3_scalar_tied=dict(p3=True, scalar=True),
               prolog=dict(prolog=True), prolog_scalar_tied=dict(prolog=True, scalar=True),
-              prolog_p3=dict(prolog=True, p3=True))[variant]
+              prolog_p3=dict(prolog=True, p3=True), scalar_decay_only=dict(mix="decay"),
+              scalar_gates_only=dict(mix="gates"), scalar_gates_only_tied=dict(mix="gates", tied=True),
+              p3_scalar_gates_only=dict(mix="gates", p3=True), prolog_scalar_decay_only=dict(mix="decay", prolog=True),
+              prolog_scalar_gates_only=dict(mix="gates", prolog=True))[variant]
     inp, dO, dS_T = _case(dev, LENS, **kw)
     grads = _run(inp, dO, dS_T)
     assert _status(grads) == 0
