@@ -308,7 +308,10 @@ __device__ __noinline__ void serial_chunk(const ChunkProblem &p, uint8_t *gb, ui
 // kXP: x_r == p_r (the gist.science form always; the default form with tied gates),
 // so B = A and QP = QX: G1 runs with N = 64 and the masks write B and read QP from the
 // A and QX values.
-template <bool kScalarDecay, bool kScalarGates, bool kP3, bool kProlog, bool kXP, typename Tout>
+// kCk: the checkpointing forward of gdn2_chunk_bwd (p.ckpt set, no o): each chunk's bf16 S_r
+// and T tile images go to the chunk's checkpoint slot.  A separate instantiation keeps that
+// work out of the plain forward's code.
+template <bool kScalarDecay, bool kScalarGates, bool kP3, bool kProlog, bool kXP, typename Tout, bool kCk>
 __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_constant__ TcParams P) {
   extern __shared__ uint8_t smem_raw[];
   const ChunkProblem &p = P.p;
@@ -589,8 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     // as this chunk builds it (the swizzled [d_k rows][d_v] tile image the backward copies to
     // shared memory as it is) and the chunk's bf16 T tile; chunks of the token-serial form
     // write nothing
-    uint8_t *ck_unit = p.ckpt ? static_cast<uint8_t *>(p.ckpt) + ckpt_first_slot(p.ckpt_off, n, h, H, nchunks) * kCkptBytes
-                              : nullptr;
+    uint8_t *ck_unit = kCk ? static_cast<uint8_t *>(p.ckpt) + ckpt_first_slot(p.ckpt_off, n, h, H, nchunks) * kCkptBytes
+                           : nullptr;
     if (tid == kIssuer && nchunks > 0 && !*sAbort) {
       issue_tma_l(h, (int)bos);
       issue_tma_a(h, (int)bos);
@@ -1208,9 +1211,9 @@ bool make_map_o(CUtensorMap *m, void *base, int64_t t_total, int H, bool bf16) {
   return r == CUDA_SUCCESS;
 }
 
-template <bool SD, bool SG, bool P3, bool PR, bool XP, typename Tout>
+template <bool SD, bool SG, bool P3, bool PR, bool XP, typename Tout, bool CK = false>
 cudaError_t launch_t(const TcParams &P, int grid, cudaStream_t stream) {
-  auto kern = chunk_tc_kernel<SD, SG, P3, PR, XP, Tout>;
+  auto kern = chunk_tc_kernel<SD, SG, P3, PR, XP, Tout, CK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, kSmemBytes, stream>>>(P);
@@ -1230,6 +1233,16 @@ cudaError_t launch_gates(const TcParams &P, int grid, cudaStream_t stream, bool 
                : launch_t<false, true, P3, PR, XP, float>(P, grid, stream);
   return obf ? launch_t<false, false, P3, PR, XP, __nv_bfloat16>(P, grid, stream)
              : launch_t<false, false, P3, PR, XP, float>(P, grid, stream);
+}
+
+// the checkpointing forward: activated inputs (no prologue) and no o, so one output type
+template <bool P3, bool XP>
+cudaError_t launch_gates_ck(const TcParams &P, int grid, cudaStream_t stream, bool sd, bool sg) {
+  using B = __nv_bfloat16;
+  if (sd) return sg ? launch_t<true, true, P3, false, XP, B, true>(P, grid, stream)
+                    : launch_t<true, false, P3, false, XP, B, true>(P, grid, stream);
+  return sg ? launch_t<false, true, P3, false, XP, B, true>(P, grid, stream)
+            : launch_t<false, false, P3, false, XP, B, true>(P, grid, stream);
 }
 
 }  // namespace
@@ -1282,6 +1295,15 @@ cudaError_t launch_chunk_tc(const ChunkProblem &p, cudaStream_t stream, const ch
   if (take_debug_timeout(GDN2_DEBUG_CHUNK, &hook_ns)) {  // the timeout test hook, armed for this launch
     P.dbg_skip = 1;
     P.wait_ns = hook_ns;
+  }
+  if (p.ckpt) {
+    if (pr || p.o) {
+      *why = "the checkpointing forward takes activated inputs and writes no o";
+      return cudaErrorNotSupported;
+    }
+    if (p3) return launch_gates_ck<true, true>(P, grid, stream, sd, sg);
+    return tied ? launch_gates_ck<false, true>(P, grid, stream, sd, sg)
+                : launch_gates_ck<false, false>(P, grid, stream, sd, sg);
   }
   // x_r == p_r in the gist.science form, and in the default form when w is b
   if (p3)
