@@ -152,6 +152,55 @@ __device__ __forceinline__ float warp_colsum32(float (&v)[32]) {
 
 __device__ __forceinline__ float bf(const __nv_bfloat16 x) { return __bfloat162float(x); }
 
+// 8 x 8 transpose of bf16 values inside each 8-lane group of a warp.  On entry lane m of a
+// group holds row m as four packed pairs (w[q] = elements 2q, 2q + 1); on exit it holds
+// column m packed the same way (w[q] = rows 2q, 2q + 1).  Exchanges at lane distances 4, 2
+// and 1: at each, a lane keeps the half of its elements whose index bit matches its own
+// lane bit and trades the other half with its partner.  Every lane of the warp takes part.
+__device__ __forceinline__ void transpose8x8_bf16(uint32_t (&w)[4], int lane) {
+  const unsigned full = 0xffffffffu;
+  {  // distance 4: elements 0-3 (words 0, 1) against 4-7 (words 2, 3)
+    const bool up = (lane & 4) != 0;
+    const uint32_t r0 = __shfl_xor_sync(full, up ? w[0] : w[2], 4);
+    const uint32_t r1 = __shfl_xor_sync(full, up ? w[1] : w[3], 4);
+    if (up) {
+      w[0] = r0;
+      w[1] = r1;
+    } else {
+      w[2] = r0;
+      w[3] = r1;
+    }
+  }
+  {  // distance 2: words 0, 2 against words 1, 3
+    const bool up = (lane & 2) != 0;
+    const uint32_t r0 = __shfl_xor_sync(full, up ? w[0] : w[1], 2);
+    const uint32_t r1 = __shfl_xor_sync(full, up ? w[2] : w[3], 2);
+    if (up) {
+      w[0] = r0;
+      w[2] = r1;
+    } else {
+      w[1] = r0;
+      w[3] = r1;
+    }
+  }
+  {  // distance 1: low halves against high halves, two words' halves per exchange
+    const bool up = (lane & 1) != 0;
+    const uint32_t r0 = __shfl_xor_sync(full, __byte_perm(w[0], w[1], up ? 0x5410 : 0x7632), 1);
+    const uint32_t r1 = __shfl_xor_sync(full, __byte_perm(w[2], w[3], up ? 0x5410 : 0x7632), 1);
+    if (up) {  // keeps the high halves; the partner's high halves become the low halves
+      w[0] = __byte_perm(r0, w[0], 0x7610);
+      w[1] = __byte_perm(r0, w[1], 0x7632);
+      w[2] = __byte_perm(r1, w[2], 0x7610);
+      w[3] = __byte_perm(r1, w[3], 0x7632);
+    } else {   // keeps the low halves; the partner's low halves become the high halves
+      w[0] = __byte_perm(w[0], r0, 0x5410);
+      w[1] = __byte_perm(w[1], r0, 0x7610);
+      w[2] = __byte_perm(w[2], r1, 0x5410);
+      w[3] = __byte_perm(w[3], r1, 0x7610);
+    }
+  }
+}
+
 // Descriptors of the 128-column operand tiles (two 64-column blocks 16 KB apart), K step kk
 // of 16: K-major walks the columns (32 bytes per step), MN-major walks the rows (16 rows,
 // 2 KB per step).
@@ -664,6 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       // the raw inputs of the epilogue's rows [16 cg, 16 cg + 8) (channel `row`), requested while
       // the last products run; rows past the chunk end re-read its last row and are ignored.
       // Scalar log_a, b, w come from shared memory; the gist.science placement needs no w here.
+      // (2-byte loads: 16-byte loads of 8 channels with a transpose after them were slower.)
       __nv_bfloat16 rla[8], rk[8], rq[8], rb[8], rw[8];
       auto load_raw = [&](int c0) {
 #pragma unroll
@@ -677,6 +727,25 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
             rb[j] = P.b[gi];
             if (!kP3) rw[j] = kTied ? rb[j] : g_w[gi];
           }
+        }
+      };
+      // Gradient rows out: the thread holds one channel (`row`) of 8 consecutive tokens
+      // [c0, c0 + 8).  bf16: after an 8 x 8 transpose inside each 8-lane group, lane m writes
+      // token c0 + m for the group's 8 channels with one 16-byte store; fp32: one store per
+      // element.  Tokens past the chunk end are not written.
+      auto store8 = [&](Tout *g, const float (&v)[8], int c0) {
+        if constexpr (sizeof(Tout) == 2) {
+          uint32_t w[4] = {pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                           pack_bf16x2(v[6], v[7])};
+          transpose8x8_bf16(w, lane);
+          const int t = c0 + (lane & 7);
+          if (t < nvalid)
+            *reinterpret_cast<uint4 *>(g + ((size_t)(t0 + t) * H + h) * D + (row - (lane & 7))) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (c0 + j < nvalid) g[((size_t)(t0 + c0 + j) * H + h) * D + row] = from_f32<Tout>(v[j]);
         }
       };
       load_raw(cg * 16);
@@ -723,20 +792,19 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         }
         ptx::tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int t = cg * 16 + j;
-          const float dz = __uint_as_float(r[j]);
-          vdz[j] = 0.f;
-          if (t < nvalid) {
-            const size_t gi = ((size_t)(t0 + t) * H + h) * D + row;
-            if (kP3) {
-              g_dv[gi] = from_f32<Tout>(wr[j] * dz);
-              vdz[j] = vr[j] * dz;
-              if (!kTied && !kSG) g_dw[gi] = from_f32<Tout>(vdz[j]);
-            } else {
-              g_dv[gi] = from_f32<Tout>(dz);
-            }
+        for (int hf = 0; hf < 2; ++hf) {
+          float dv8[8], dw8[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int jj = hf * 8 + j;
+            const bool valid = cg * 16 + jj < nvalid;
+            const float dz = __uint_as_float(r[jj]);
+            vdz[jj] = (kP3 && valid) ? vr[jj] * dz : 0.f;
+            dv8[j] = kP3 ? wr[jj] * dz : dz;
+            dw8[j] = vdz[jj];
           }
+          store8(g_dv, dv8, cg * 16 + hf * 8);
+          if (kP3 && !kTied && !kSG) store8(g_dw, dw8, cg * 16 + hf * 8);
         }
       }
       waitb(bar(BAR_G7), par);
@@ -767,6 +835,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           ptx::tmem_ld8(tmZ + lane_base + 64u + (uint32_t)c0, vq);
           if (half == 1) load_raw(c0);  // the first half's were requested before the wait
           ptx::tmem_wait_ld();
+          float dq8[8], dk8[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int t = c0 + j, jj = half * 8 + j;
@@ -796,15 +865,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
             }
             if (t == C - 1) dLt += dlc;
             dL[jj] = dLt;
-            if (valid) {
-              const size_t gi = ((size_t)(t0 + t) * H + h) * D + i;
-              g_dq[gi] = from_f32<Tout>(dqr * e);
-              g_dk[gi] = from_f32<Tout>(dkv);
-              if (!kSG) {
-                g_db[gi] = from_f32<Tout>(gbv[jj]);
-                if (!kTied && !kP3) g_dw[gi] = from_f32<Tout>(gwv[jj]);
-              }
+            dq8[j] = dqr * e;
+            dk8[j] = dkv;
+          }
+          store8(g_dq, dq8, c0);
+          store8(g_dk, dk8, c0);
+          if (!kSG) {
+            float b8[8], w8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              b8[j] = gbv[half * 8 + j];
+              w8[j] = gwv[half * 8 + j];
             }
+            store8(g_db, b8, c0);
+            if (!kTied && !kP3) store8(g_dw, w8, c0);
           }
         }
         if (kSG) {  // db, dw channel sums: over the warp's 32 channels, then the lane quadrants
@@ -841,9 +915,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           if (lane < 16) red[(qd * 3 + 2) * 64 + cg * 16 + lane] = sum;
         } else {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int t = cg * 16 + j;
-            if (t < nvalid) g_dla[((size_t)(t0 + t) * H + h) * D + i] = from_f32<Tout>(dL[j] + above);
+          for (int hf = 0; hf < 2; ++hf) {
+            float l8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) l8[j] = dL[hf * 8 + j] + above;
+            store8(g_dla, l8, cg * 16 + hf * 8);
           }
         }
         if (kSD || kSG) {
