@@ -38,6 +38,7 @@ same workload instead (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import atexit
 import datetime
 import hashlib
 import json
@@ -142,16 +143,21 @@ def traffic_per_launch():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while timing."""
+    """nvidia-smi clocks and throttle reasons every 200 ms for the whole run.  It starts
+    before the first timed region, so its own start-up (process launch, NVML
+    initialisation) runs beside untimed work; each timed region then takes the samples
+    around it (``stats``)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.gpu_index = gpu_index
         self.proc = None
         self.file = None
+        self.samples = []  # (host time, SM MHz, max SM MHz, active reasons)
 
     def start(self):
         try:
@@ -159,12 +165,17 @@ class ClockSampler:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                                           "-i", str(self.gpu_index), "-lms", "200"], stdout=self.file,
                                          stderr=subprocess.DEVNULL)
+            atexit.register(self.kill)  # an exception between start and stop must not leave it running
         except Exception:
             self.proc = None
 
+    def kill(self):
+        if self.proc is not None and self.proc.poll() is None:
+            self.proc.kill()
+
     def stop(self):
         if self.proc is None:
-            return None
+            return
         time.sleep(0.25)
         self.proc.terminate()
         try:
@@ -175,21 +186,31 @@ class ClockSampler:
         self.file.seek(0)
         rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
         os.unlink(self.file.name)
-        mhz, mx, reasons = [], 0.0, set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        self.proc = None
         for r in rows:
             try:
-                mhz.append(float(r[1]))
-                mx = max(mx, float(r[2]))
-                for nm, val in zip(names, r[5:9]):
-                    if val.strip().lower() == "active":
-                        reasons.add(nm)
+                mhz, mx = float(r[2]), float(r[3])
+                reasons = {nm for nm, val in zip(self.REASONS, r[6:10]) if val.strip().lower() == "active"}
             except (ValueError, IndexError):
                 continue
-        if not mhz:
+            try:
+                t = datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                t = None  # an unreadable timestamp: the sample counts for every region
+            self.samples.append((t, mhz, mx, reasons))
+
+    def stats(self, t0: float, t1: float, margin: float = 0.25):
+        """Median SM clock, max clock and the active reasons of the samples taken from
+        ``margin`` seconds before host time ``t0`` to ``margin`` after ``t1`` (the two
+        samples nearest the region if none falls inside)."""
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(mhz)}
+        sel = [x for x in self.samples if x[0] is None or t0 - margin <= x[0] <= t1 + margin]
+        if not sel:
+            mid = 0.5 * (t0 + t1)
+            sel = sorted(self.samples, key=lambda x: abs(x[0] - mid))[:2]
+        return {"sm_mhz": statistics.median(x[1] for x in sel), "sm_max_mhz": max(x[2] for x in sel),
+                "reasons": sorted(set().union(*(x[3] for x in sel))), "samples": len(sel)}
 
 
 # ----------------------------------------------------------------------------- ranks
@@ -331,7 +352,7 @@ def main():
     ap.add_argument("--reference-step-seconds", type=float, default=6.0)
     ap.add_argument("--batch", type=int, default=0, help="override the batch size (small profiling cases)")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--bwd-steps", type=int, default=3)
+    ap.add_argument("--bwd-steps", type=int, default=10)
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-token-serial-bwd", action="store_true",
                     help="skip the one timed step of the token-serial gdn2_bwd")
@@ -374,6 +395,8 @@ def main():
         return max_over_ranks(x, world, dev)
 
     hbm_peak, tc_peak, peak_src = peaks()
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    sampler.start()
 
     # ---------------- prefill (the step)
     inp = inputs.make_inputs(WORKLOAD, dev, seed=rank, n_seqs=args.batch or None)
@@ -392,17 +415,16 @@ def main():
     for _ in range(args.warmup):
         step()
     barrier()
-    sampler = ClockSampler(dev.index if dev.index is not None else 0)
-    sampler.start()
     stream = torch.cuda.current_stream(dev)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier()
+    w_prefill = time.time()
     for i in range(args.steps):
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
     barrier()
-    clocks = sampler.stop()
+    w_prefill = (w_prefill, time.time())
     total_ms = ev[0][0].elapsed_time(ev[-1][1])
     launch_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = rmax(total_ms)
@@ -573,10 +595,9 @@ def main():
         for t in range(3):
             gdn2.decode_step(*(di[n][t] for n in names), S, o=od)
         barrier()
-        sd = ClockSampler(dev.index if dev.index is not None else 0)
-        sd.start()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
+        w_decode = time.time()
         e0.record(stream)
         for t in range(steps):
             gdn2.decode_step(*(di[n][t] for n in names), S, o=od)
@@ -596,7 +617,7 @@ def main():
         graph.replay()
         e1.record(stream)
         barrier()
-        dclocks = sd.stop()
+        w_decode = (w_decode, time.time())
         dms = rmax(e0.elapsed_time(e1))
         del graph
         if gdn2.decode_status() != gdn2.OK:
@@ -642,7 +663,7 @@ def main():
         decode = {"value": Nd * world * steps / (dms / 1e3), "unit": "tokens/s", "steps": steps,
                   "us_per_step": 1e3 * dms / steps, "bytes_per_step": step_bytes, "hbm_gbs": gbs,
                   "hbm_frac": gbs / hbm_peak, "peak_source": peak_src, "sequences": Nd, "heads": Hd,
-                  "state_bytes": Nd * Hd * d * d * 4, "clocks": dclocks, "kernel": "decode_stream_kernel",
+                  "state_bytes": Nd * Hd * d * d * 4, "clocks": w_decode, "kernel": "decode_stream_kernel",
                   "launch": "CUDA graph of all steps, replayed once",
                   "plain_loop_us_per_step": 1e3 * plain_ms / steps,
                   "gpu_launches": steps,
@@ -674,15 +695,14 @@ def main():
             cstep()
         torch.cuda.synchronize()
         barrier()
-        bs = ClockSampler(dev.index if dev.index is not None else 0)
-        bs.start()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        w_bwd = time.time()
         e0.record(stream)
         for _ in range(args.bwd_steps):
             cstep()
         e1.record(stream)
         barrier()
-        bclocks = bs.stop()
+        w_bwd = (w_bwd, time.time())
         cms = rmax(e0.elapsed_time(e1)) / args.bwd_steps
         st = gdn2.lib.gdn2_check_status(gdn2._ptr(cws), gdn2._stream(dev))
         tokheads = Nb * Tb * 16
@@ -698,7 +718,7 @@ def main():
                "tensor": {"achieved": ctf, "peak": tc_peak, "unit": "TFLOP/s", "frac": ctf / tc_peak,
                           "alg_flops_per_tokhead": CBWD_FLOP_PER_TOKHEAD},
                "kernels": ["chunk_tc_kernel (checkpointing forward)", "bwd_tc_kernel"],
-               "gpu_launches": 2 * args.bwd_steps, "workspace_bytes": cws.numel(), "clocks": bclocks}
+               "gpu_launches": 2 * args.bwd_steps, "workspace_bytes": cws.numel(), "clocks": w_bwd}
         del cws
         # the tied scalar-gate Gated DeltaNet batch (4 x 4096 x 16) through the same backward
         si = inputs.make_inputs("gdn_scalar_b4_t4k", dev, seed=310 + rank)
@@ -749,12 +769,11 @@ def main():
             barrier()
             bms = rmax(e0.elapsed_time(e1))
             tflops = BWD_FLOP_PER_TOKHEAD * tokheads / (bms / 1e3) / 1e12
-            peak32 = fp32_peak_tflops(bclocks.get("sm_max_mhz") or 1965.0)
             bwd["token_serial"] = {
                 "value": Nb * Tb * world / (bms / 1e3), "unit": "tokens/s", "ms_per_step": bms, "steps": 1,
                 "dtype": "f32 arithmetic, bf16 inputs and gradients",
-                "roofline": {"bound": "alu", "achieved": tflops, "peak": peak32, "unit": "TFLOP/s",
-                             "frac": tflops / peak32, "traffic": None,
+                "roofline": {"bound": "alu", "achieved": tflops, "peak": None, "unit": "TFLOP/s",
+                             "frac": None, "traffic": None,
                              "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x sm_max_mhz",
                              "alg_flops_per_tokhead": BWD_FLOP_PER_TOKHEAD},
                 "kernels": ["bwd_kernel", "finish_kernel"], "workspace_bytes": bws.numel()}
@@ -806,6 +825,18 @@ def main():
                                            "gdn2_affine_prefix, gdn2_segment_correct"})
         del li, largs, lws, pws
 
+    # clocks of each timed region, from the samples taken around it
+    sampler.stop()
+    clocks = sampler.stats(*w_prefill)
+    if decode is not None:
+        decode["clocks"] = sampler.stats(*decode["clocks"])
+    if bwd is not None:
+        bwd["clocks"] = sampler.stats(*bwd["clocks"])
+        ts = bwd.get("token_serial")
+        if ts is not None:
+            peak32 = fp32_peak_tflops((bwd["clocks"] or {}).get("sm_max_mhz") or 1965.0)
+            ts["roofline"]["peak"] = peak32
+            ts["roofline"]["frac"] = ts["roofline"]["achieved"] / peak32
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes and distributions of the "
