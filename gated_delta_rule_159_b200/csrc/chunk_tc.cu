@@ -101,7 +101,8 @@ constexpr uint32_t MISC_UNIT = 10344;
 constexpr uint32_t MISC_WIDE = 10348;  // int: some channel of the chunk being prepared has a wide decay range
 constexpr uint32_t MISC_ISS = 10352;   // uint32[4]   phases armed per TMA barrier (A, L, W, X)
 constexpr uint32_t MISC_L0 = 10368;    // float[128]  L_0 (the chunk's first row)
-constexpr uint32_t MISC_BYTES = 10880;
+constexpr uint32_t MISC_SCN = 10880;   // float[3][64] the next chunk's raw scalar log_a and gates
+constexpr uint32_t MISC_BYTES = 11648;
 // Token-serial chunks stage their per-token vectors in [OFF_OS, OFF_MISC) (fp32):
 // a, q, y, x, p as [32 tokens][128], z as [32][128], q.x and q.p [32], and the
 // cross-warp exchange of the column sums [2][4][128] float2.
@@ -329,6 +330,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   static_assert(MISC_DL == MISC_DL0 + 512, "the two e^{L_C - L_ref} buffers are adjacent");
   auto sDLb = [&](uint32_t parity) { return reinterpret_cast<float *>(gb + OFF_MISC + MISC_DL0 + 512u * parity); };
   float *sSM = reinterpret_cast<float *>(gb + OFF_MISC + MISC_SM);
+  // scalar flags: the raw per-token log_a [0, 64), the gate of pass 2 [64, 128) and the gate of
+  // pass 3 [128, 192) of the chunk being prepared, fetched from global memory a chunk early
+  float *sScN = reinterpret_cast<float *>(gb + OFF_MISC + MISC_SCN);
   float *part = reinterpret_cast<float *>(gb + OFF_MISC + MISC_PART);
   float *sRef = reinterpret_cast<float *>(gb + OFF_MISC + MISC_REF);
   float *sL0 = reinterpret_cast<float *>(gb + OFF_MISC + MISC_L0);
@@ -435,6 +439,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
   // into the parity-pn buffer and e^{L_ref}.  Ends with a CTA barrier, after which the log_a
   // slot is free; returns non-zero (in every thread) when some channel's decay range
   // L_0 - L_63 exceeds kFastSpan, i.e. the chunk must run token by token.
+  // scalar flags: thread tid < 192 fetches value (tid & 63) of array (tid >> 6) for the chunk
+  // starting at t0n (0 past its end); the caller stores it to sScN[tid] once it has landed
+  auto scal_load = [&](int t0n, int nvn, int h) -> float {
+    const int which = tid >> 6, r = tid & 63;
+    if (tid >= 192 || r >= nvn) return 0.f;
+    const __nv_bfloat16 *src = which == 0 ? (kScalarDecay ? g_la : nullptr)
+                               : which == 1 ? (kScalarGates ? (kP3 ? g_b : g_w) : nullptr)
+                                            : (kScalarGates ? (kP3 ? g_w : g_b) : nullptr);
+    return src ? __bfloat162float(src[(size_t)(t0n + r) * H + h]) : 0.f;
+  };
   auto elem_cumsum = [&](uint32_t pn, int t0n, int nvn, int h, float4 (&L)[4]) -> int {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -443,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       float4 g = make_float4(0.f, 0.f, 0.f, 0.f);
       if (r < nvn) {
         if (kScalarDecay) {
-          float sv = __bfloat162float(g_la[(size_t)(t0n + r) * H + h]);
+          float sv = sScN[r];
           if (kProlog) sv = log_sigmoid_f(sv);
           g = make_float4(sv, sv, sv, sv);
         } else {
@@ -497,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       if (kScalarGates) {
         ww = make_float4(0.f, 0.f, 0.f, 0.f);
         if (r < nvn) {
-          float swv = __bfloat162float((kP3 ? g_b : g_w)[(size_t)(t0n + r) * H + h]);
+          float swv = sScN[64 + r];
           if (kProlog) swv = sigmoid_f(swv);
           ww = make_float4(swv, swv, swv, swv);
         }
@@ -547,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       if (kScalarGates) {
         bb = make_float4(0.f, 0.f, 0.f, 0.f);
         if (r < nvn) {
-          float sbv = __bfloat162float((kP3 ? g_w : g_b)[(size_t)(t0n + r) * H + h]);
+          float sbv = sScN[128 + r];
           if (kProlog) sbv = sigmoid_f(sbv);
           bb = make_float4(sbv, sbv, sbv, sbv);
         }
@@ -627,6 +641,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     if (nchunks > 0) {
       const int nv0 = (int)(len < C ? len : C);
       const uint32_t par0 = it & 1u;
+      if (kScalarDecay || kScalarGates) {
+        const float sv = scal_load((int)bos, nv0, h);
+        if (tid < 192) sScN[tid] = sv;
+        __syncthreads();
+      }
       if (!kScalarDecay) waitb(bar(BAR_TMA_L), par0);
       wide_next = elem_cumsum(par0, (int)bos, nv0, h, L);
       if (tid == kIssuer && !*sAbort) issue_tma_x(h, (int)bos);
@@ -650,6 +669,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       // the log_a slot is free (the b tile it last held was consumed by this chunk's x_r):
       // the next chunk's log_a can land
       if (tid == kIssuer && has_next && !*sAbort) issue_tma_l(h, t0 + C);
+      // scalar flags: the next chunk's values, requested now and stored before the barrier
+      // that ends the masks (this chunk's were read while the previous chunk built its operands)
+      float scal_next = 0.f;
+      if ((kScalarDecay || kScalarGates) && has_next) scal_next = scal_load(t0 + C, nvalid_next, h);
 
       if (wide_next) {
         // ---- a decay range beyond the factored form: the recurrence token by token.  The
@@ -659,6 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
           ptx::tc_fence_after();
         }
         if (tid == kIssuer) ptx::bulk_wait_group_read0();  // the previous o store has read the staging area
+        if ((kScalarDecay || kScalarGates) && tid < 192) sScN[tid] = scal_next;
         __syncthreads();
         // One arrival per chunk on every MMA barrier keeps their phases in step with the chunk
         // count (plain arrivals: this chunk issues no MMA, and the previous chunk's are done).
@@ -813,6 +837,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       // a proxy fence costs each thread that runs it far more than a barrier: only the warps
       // whose stores an MMA reads (B, QX, QP) run it; the fp32 A is read by the solve's threads
       if (kXP ? (cg < 2) : !(qd < 2 && cg < 2)) ptx::fence_proxy_async_smem();
+      if ((kScalarDecay || kScalarGates) && tid < 192) sScN[tid] = scal_next;
       ptx::tc_fence_before();
       __syncthreads();
 
