@@ -355,6 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
 
     bool unit_ok = true;
     int lastpar = -1;  // parity of the last chunk processed (chunk 0): its e^{rho} gives dS0
+    float scal_pre = 0.f;  // scalar flags: this thread's value of the chunk processed next
     for (int ci = nchunks - 1; ci >= 0; --ci) {
       const uint32_t par = it & 1u;
       const int t0 = (int)(bos + (int64_t)ci * C);
@@ -362,14 +363,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
 
       // ================= phase 1: loads, cumulative decay, operand tiles
       if (kSD || kSG) {  // the chunk's scalar log_a and / or b, w (zero past the chunk end)
-        if (tid < 192) {
-          const int which = tid >> 6, r = tid & 63;
-          if (which == 0 ? kSD : kSG) {
-            const __nv_bfloat16 *src = which == 0 ? P.log_a : (which == 1 || kTied) ? P.b : g_w;
-            sScal[tid] = r < nvalid ? bf(src[(size_t)(t0 + r) * H + h]) : 0.f;
-          }
+        const int which = tid >> 6, r = tid & 63;
+        const bool mine = tid < 192 && (which == 0 ? kSD : kSG);
+        const __nv_bfloat16 *src = which == 0 ? P.log_a : (which == 1 || kTied) ? P.b : g_w;
+        if (mine) {  // the unit's first chunk fetches its own; later ones were requested a chunk ago
+          sScal[tid] = ci == nchunks - 1 ? (r < nvalid ? bf(src[(size_t)(t0 + r) * H + h]) : 0.f) : scal_pre;
         }
         __syncthreads();
+        // the next chunk to process (ci - 1, a full chunk): requested now, stored at its start
+        if (mine && ci > 0) scal_pre = bf(src[(size_t)(t0 - C + r) * H + h]);
       }
       // fp32 dO: the rows of channel `row` into the bf16 tile (rows past the chunk end re-read
       // its last row and are zeroed); the dO rows of the tile are free since the previous
@@ -833,7 +835,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
           ptx::tmem_ld8(tmX + lane_base + 64u + (uint32_t)c0, vp);
           ptx::tmem_ld8(tmZ + lane_base + (uint32_t)c0, vk);
           ptx::tmem_ld8(tmZ + lane_base + 64u + (uint32_t)c0, vq);
-          if (half == 1) load_raw(c0);  // the first half's were requested before the wait
           ptx::tmem_wait_ld();
           float dq8[8], dk8[8];
 #pragma unroll
@@ -868,6 +869,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
             dq8[j] = dqr * e;
             dk8[j] = dkv;
           }
+          // the second half's raw rows, requested while this half's gradients go out (the
+          // first half's were requested before the adjoint wait)
+          if (half == 0) load_raw(c0 + 8);
           store8(g_dq, dq8, c0);
           store8(g_dk, dk8, c0);
           if (!kSG) {
