@@ -426,34 +426,55 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
       if (tid == 0) *sWide = 0;
       __syncthreads();
       {
-        // per channel c: exclusive prefixes over the 16 row groups (thread: groups 4 g4 .. 4 g4 + 3
-        // of channel c; the four threads of a channel are adjacent lanes and scan their totals
-        // with shuffles), L_ref, the range check
-        const int c = tid >> 2, g4 = tid & 3;
-        float v[4];
+        // per channel c: exclusive prefixes over the 16 row groups, L_ref, the range check.
+        // Channel-wise decay: four adjacent lanes per channel take 4 groups each and scan their
+        // totals with shuffles; scalar decay: one thread per channel walks the 16 groups (each
+        // form measured the faster one for its case).
+        if (kSD) {
+          if (tid < D) {
+            const int c = tid;
+            float run = 0.f;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] = part16[(4 * g4 + j) * 128 + c];
-        const float tl = ((v[0] + v[1]) + v[2]) + v[3];
-        float incl = tl;
-        const float u1 = __shfl_up_sync(0xffffffffu, incl, 1, 4);
-        if (g4 >= 1) incl += u1;
-        const float u2 = __shfl_up_sync(0xffffffffu, incl, 2, 4);
-        if (g4 >= 2) incl += u2;
-        const float run = __shfl_sync(0xffffffffu, incl, 3, 4);  // the channel's total L_63
-        float pre4 = incl - tl;
-        lpre[g4 * 128 + c] = pre4;  // the epilogue's 16-row groups
+            for (int j = 0; j < 16; ++j) {
+              const float pj = part16[j * 128 + c];
+              part16[j * 128 + c] = run;
+              if ((j & 3) == 0) lpre[(j >> 2) * 128 + c] = run;
+              run += pj;
+            }
+            const float l0 = sL0[c];
+            const float rho = 0.5f * (l0 + run);
+            if (!(l0 - run <= kFastSpan)) *sWide = 1;
+            sRho[c] = rho;
+            sGam[c] = ptx::ex2((run - rho) * kLog2eF);
+            sEsr[par * 128 + c] = ptx::ex2(rho * kLog2eF);
+          }
+        } else {
+          const int c = tid >> 2, g4 = tid & 3;
+          float v[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          part16[(4 * g4 + j) * 128 + c] = pre4;
-          pre4 += v[j];
-        }
-        if (g4 == 3) {
-          const float l0 = sL0[c];
-          const float rho = 0.5f * (l0 + run);
-          if (!(l0 - run <= kFastSpan)) *sWide = 1;
-          sRho[c] = rho;
-          sGam[c] = ptx::ex2((run - rho) * kLog2eF);
-          sEsr[par * 128 + c] = ptx::ex2(rho * kLog2eF);
+          for (int j = 0; j < 4; ++j) v[j] = part16[(4 * g4 + j) * 128 + c];
+          const float tl = ((v[0] + v[1]) + v[2]) + v[3];
+          float incl = tl;
+          const float u1 = __shfl_up_sync(0xffffffffu, incl, 1, 4);
+          if (g4 >= 1) incl += u1;
+          const float u2 = __shfl_up_sync(0xffffffffu, incl, 2, 4);
+          if (g4 >= 2) incl += u2;
+          const float run = __shfl_sync(0xffffffffu, incl, 3, 4);  // the channel's total L_63
+          float pre4 = incl - tl;
+          lpre[g4 * 128 + c] = pre4;  // the epilogue's 16-row groups
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            part16[(4 * g4 + j) * 128 + c] = pre4;
+            pre4 += v[j];
+          }
+          if (g4 == 3) {
+            const float l0 = sL0[c];
+            const float rho = 0.5f * (l0 + run);
+            if (!(l0 - run <= kFastSpan)) *sWide = 1;
+            sRho[c] = rho;
+            sGam[c] = ptx::ex2((run - rho) * kLog2eF);
+            sEsr[par * 128 + c] = ptx::ex2(rho * kLog2eF);
+          }
         }
       }
       __syncthreads();
