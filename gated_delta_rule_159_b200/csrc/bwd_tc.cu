@@ -733,9 +733,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(const __grid_consta
         for (int kk = 0; kk < 8; ++kk) ptx::umma_bf16(tmZ, mnmaj(sb + OFF_XP, kk), kmaj(sb + OFF_DG, kk), idNK, 1);
         ptx::umma_commit(bar(BAR_G7));
       }
-      // the raw inputs of the epilogue's rows [16 cg, 16 cg + 8) (channel `row`), requested while
-      // the last products run; rows past the chunk end re-read its last row and are ignored.
-      // Scalar log_a, b, w come from shared memory; the gist.science placement needs no w here.
+      // the raw inputs of the epilogue's rows [c0, c0 + 8) (channel `row`): the first half's are
+      // requested while the last products run, the second half's once the first half's chain
+      // rule is done; rows past the chunk end re-read its last row and are ignored.  Scalar
+      // log_a, b, w come from shared memory; the gist.science placement needs no w here.
       // (2-byte loads: 16-byte loads of 8 channels with a transpose after them were slower.)
       __nv_bfloat16 rla[8], rk[8], rq[8], rb[8], rw[8];
       auto load_raw = [&](int c0) {
