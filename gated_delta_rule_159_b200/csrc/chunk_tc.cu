@@ -506,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
       const float e10 = ptx::ex2(l0), e11 = ptx::ex2(l1), e12 = ptx::ex2(l2), e13 = ptx::ex2(l3);
       const float4 e2 = make_float4(ptx::ex2(-l0), ptx::ex2(-l1), ptx::ex2(-l2), ptx::ex2(-l3));
       float4 kk = unpack4(lds_v2(sb + OFF_KQ + o));
-      float4 qq = unpack4(lds_v2(sb + OFF_KQ + o + 8192));
+      float4 qq = kCk ? make_float4(0.f, 0.f, 0.f, 0.f) : unpack4(lds_v2(sb + OFF_KQ + o + 8192));
       float4 ww;  // the write gate w (the erase gate b in the gist.science form)
       if (kScalarGates) {
         ww = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -546,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         sts_v2(sb + OFF_KQ + o, pack4(kk.x * e10, kk.y * e11, kk.z * e12, kk.w * e13));
         sts_v2(sb + OFF_XP + o + 8192, pack4(ww.x * ke.x, ww.y * ke.y, ww.z * ke.z, ww.w * ke.w));
       }
-      sts_v2(sb + OFF_KQ + o + 8192, pack4(qq.x * e10, qq.y * e11, qq.z * e12, qq.w * e13));
+      if (!kCk) sts_v2(sb + OFF_KQ + o + 8192, pack4(qq.x * e10, qq.y * e11, qq.z * e12, qq.w * e13));
     }
   };
   // pass 3 (needs the b tile, which lands in the log_a slot, and a free x_r slot): x_r = b.k
@@ -798,7 +798,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
 
       // masks: A, B strictly lower (fp32 A for the solve, bf16 B); QX, QP lower incl. diagonal.
       // warp (qd, cg) reads D1 columns [32 cg, 32 cg + 32); with kXP only columns 0-63 exist.
-      if (!kXP || cg < 2) {
+      // The checkpointing forward writes no o: QX and QP (rows 64-127) are not needed.
+      if ((!kXP || cg < 2) && !(kCk && qd >= 2)) {
         float *Af = reinterpret_cast<float *>(gb + OFF_AF);
         uint32_t r[32];
         ptx::tmem_ld32(tmD1 + lane_base + cg * 32, r);
@@ -858,8 +859,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             ptx::umma_bf16(tmS, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
                            ptx::sdesc_sw128(sb + OFF_XP + 8192 + kk * 2048, 16384, 1024), idS, 1);
           ptx::umma_commit(bar(BAR_E1));
-          constexpr uint32_t idV = ptx::idesc_bf16(128, 128, true, false);   // A = V^T (MN-major)
-          constexpr uint32_t idT = ptx::idesc_bf16(128, 128, false, false);  // A from TMEM
+          // the checkpointing forward writes no o: R^T alone (N = 64, the B and k_r rows)
+          constexpr uint32_t idV = ptx::idesc_bf16(128, kCk ? 64 : 128, true, false);   // A = V^T (MN-major)
+          constexpr uint32_t idT = ptx::idesc_bf16(128, kCk ? 64 : 128, false, false);  // A from TMEM
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             ptx::umma_bf16(tmD1, ptx::sdesc_sw128(sb + OFF_V + kk * 2048, 8192, 1024),
@@ -1071,7 +1073,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         constexpr uint32_t idO = ptx::idesc_bf16(128, 64, false, false);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_bf16_ts(tmO, tmMb + kk * 8, ptx::sdesc_sw128(sb + (kXP ? OFF_QP : OFF_QX) + kk * 32, 16, 1024), idO, 1);
+          if (!kCk)
+            ptx::umma_bf16_ts(tmO, tmMb + kk * 8, ptx::sdesc_sw128(sb + (kXP ? OFF_QP : OFF_QX) + kk * 32, 16, 1024), idO, 1);
         ptx::umma_commit(bar(BAR_G4));  // O^T is complete: the epilogue need not wait for dS
         // dS^T += (-M^T) x_r: B = x_r as [tokens][dk] (MN-major, N = 128)
         constexpr uint32_t idS = ptx::idesc_bf16(128, 128, false, true);
