@@ -151,3 +151,14 @@ def test_chunk_bwd_full_size_sampled(dev):
     assert _status(grads) == 0
     errs = compare_bwd_units(inp, grads, dO, dS_T, [(0, 0), (7, 15)])
     assert max(errs.values()) <= TOL_CHUNK_BF16, errs
+
+
+def test_chunk_bwd_full_size_scalar_sampled(dev):
+    """The tied scalar-gate shape of the bench (4 x 4096 tokens, 16 heads, bf16 gradients):
+    sampled units; every chunk after a unit's first takes its scalar gates from the values
+    requested a chunk ahead."""
+    inp, dO, dS_T = _case(dev, None, batch=(4, 4096), n_heads=16, seed=6, do_dtype=torch.bfloat16, scalar=True)
+    grads = _run(inp, dO, dS_T, batch=(4, 4096))
+    assert _status(grads) == 0
+    errs = compare_bwd_units(inp, grads, dO, dS_T, [(0, 0), (3, 15)])
+    assert max(errs.values()) <= TOL_CHUNK_BF16, errs
