@@ -171,7 +171,9 @@ def _seq_worker(rank, world, port, out_q):
         gathered = [None] * world
         dist.all_gather_object(gathered, (lo, hi, o, S_T))
         if rank == 0:
-            out_q.put(gathered)
+            # numpy arrays travel by value; a tensor's storage would be shared through a file
+            # descriptor that the receiver can only fetch while this process still lives
+            out_q.put([(a, z, oo.numpy(), ss.numpy()) for a, z, oo, ss in gathered])
     finally:
         dist.destroy_process_group()
 
@@ -194,6 +196,7 @@ def test_sequence_ranks_equal_unsplit(world):
     o_ref, S_ref = _OracleSegmentOps._run(*xs, S0)
     o = torch.zeros_like(o_ref)
     for lo, hi, o_r, S_r in gathered:
+        o_r, S_r = torch.from_numpy(o_r), torch.from_numpy(S_r)
         o[:, lo:hi] = o_r
         assert torch.allclose(S_r, S_ref, rtol=1e-10, atol=1e-12)
     assert torch.allclose(o, o_ref, rtol=1e-10, atol=1e-12)
